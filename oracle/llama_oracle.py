@@ -1,0 +1,358 @@
+"""fp64 CPU oracle of the Llama-2 decoder forward pass with a KV cache, plus
+greedy and top-p sampling.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+benchmark's CPU-baseline leg may import this module.  The product path (the
+CUDA library and its Python binding) never calls it and shares no code with
+it.
+
+It is the plain definition, written out: numpy float64 arithmetic, library
+matmul/exp/sort as single steps, no blocking, fusion or reordering.  Every
+function names the passage it follows.  Citations are to the two guides for
+the meta-llama/llama repository ("Llama 2 Reference Implementation —
+Administrator & Developer Guide", called *Admin Guide* below, and the
+companion *User Guide*) and to the pyshine.com source tour ("meta-llama/llama
+source tour").
+
+Readings taken where the pages leave a step open (each one is listed again
+in the design notes):
+  * RoPE frequencies are the standard theta^(-2j/head_dim); pairs are the
+    adjacent reals (2j, 2j+1) viewed as one complex number.  The pages fix
+    only theta and the complex-pair view.  Parity of the frequency schedule
+    is pinned by the textbook definition only ("parity unpinned" against the
+    pages for the schedule itself).
+  * repeat_kv maps query head h to KV head floor(h / n_rep).
+  * Argmax ties go to the lowest token id.
+  * top-p orders tokens by probability descending, equal probabilities by id
+    ascending; a token is kept iff the mass strictly before it is <= top_p;
+    the draw is the inverse CDF of the renormalised kept mass at the given
+    uniform u (the multinomial draw made deterministic).
+
+Weights are passed as a mapping:
+  w["tok_embeddings"] [V, dim], w["norm"] [dim], w["output"] [V, dim],
+  w["layers"][l][name] for name in attention_norm [dim], wq [nh*hd, dim],
+  wk [nkv*hd, dim], wv [nkv*hd, dim], wo [dim, nh*hd], ffn_norm [dim],
+  w1 [H, dim], w2 [dim, H], w3 [H, dim]   (nn.Linear layout: y = x W^T).
+Any array-like works; each one is upcast to float64 at the point of use.
+"""
+from __future__ import annotations
+
+import math
+from typing import List, Optional, Sequence
+
+import numpy as np
+
+
+def _f64(a) -> np.ndarray:
+    return np.asarray(a, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Sizes
+# ---------------------------------------------------------------------------
+
+def ffn_hidden_dim(dim: int, multiple_of: int, ffn_dim_multiplier: Optional[float] = None) -> int:
+    """SwiGLU hidden width.
+
+    Admin Guide §8.4 (FeedForward): start from 4*dim, take int(2*hidden/3),
+    optionally multiply by ffn_dim_multiplier (truncating), then round up to
+    the next multiple of multiple_of.
+    """
+    hidden = 4 * dim
+    hidden = int(2 * hidden / 3)
+    if ffn_dim_multiplier is not None and ffn_dim_multiplier > 0:
+        hidden = int(ffn_dim_multiplier * hidden)
+    return multiple_of * ((hidden + multiple_of - 1) // multiple_of)
+
+
+def kv_cache_bytes_per_tensor(max_batch_size: int, max_seq_len: int, n_kv_heads: int,
+                              head_dim: int, bytes_per_elem: int) -> int:
+    """Bytes of one cache tensor (cache_k or cache_v) of one layer.
+
+    Admin Guide §6.2: shape (max_batch_size, max_seq_len, n_local_kv_heads, head_dim).
+    """
+    return max_batch_size * max_seq_len * n_kv_heads * head_dim * bytes_per_elem
+
+
+def parameter_count(dim: int, n_layers: int, n_heads: int, n_kv_heads: int, vocab_size: int,
+                    hidden: int) -> int:
+    """Number of learned parameters (Admin Guide §8.4: Transformer, Attention,
+    FeedForward, two RMSNorms per block, a final RMSNorm; embedding and output
+    are separate modules; no biases anywhere — source tour, "One model.py")."""
+    hd = dim // n_heads
+    per_layer = (dim * n_heads * hd + 2 * dim * n_kv_heads * hd + n_heads * hd * dim  # wq wk wv wo
+                 + 3 * dim * hidden                                               # w1 w2 w3
+                 + 2 * dim)                                                       # two norms
+    return vocab_size * dim * 2 + n_layers * per_layer + dim
+
+
+# ---------------------------------------------------------------------------
+# Building blocks
+# ---------------------------------------------------------------------------
+
+def rms_norm(x, weight, eps: float) -> np.ndarray:
+    """RMSNorm over the last axis: x * 1/sqrt(mean(x^2) + eps), times weight.
+
+    Admin Guide §8.4 (RMSNorm): no mean subtraction, no bias.  The reference
+    computes the normalisation in fp32 and casts back before the weight; the
+    oracle computes all of it in fp64.
+    """
+    x = _f64(x)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * _f64(weight)
+
+
+def rope_frequencies(head_dim: int, theta: float) -> np.ndarray:
+    """freq_j = theta^(-2j/head_dim), j = 0 .. head_dim/2 - 1.
+
+    Admin Guide §8.4 (RoPE, precompute_freqs_cis): a table of e^{i t freq}
+    of shape (end, head_dim/2) with theta = 10000; the schedule itself is the
+    standard rotary one (a reading; the pages print no formula).
+    """
+    j = np.arange(head_dim // 2, dtype=np.float64)
+    return np.float64(theta) ** (-2.0 * j / head_dim)
+
+
+def apply_rope(v, positions, theta: float) -> np.ndarray:
+    """Rotate each adjacent pair (v[2j], v[2j+1]) by the angle pos*freq_j.
+
+    v: [T, n_heads, head_dim]; positions: [T].  The pair is read as the
+    complex number v[2j] + i v[2j+1] and multiplied by e^{i pos freq_j}
+    (Admin Guide §8.4, apply_rotary_emb; source tour, "One model.py").
+    """
+    v = _f64(v)
+    T, nh, hd = v.shape
+    ang = _f64(positions)[:, None] * rope_frequencies(hd, theta)[None, :]   # [T, hd/2]
+    c = np.cos(ang)[:, None, :]
+    s = np.sin(ang)[:, None, :]
+    re = v[..., 0::2]
+    im = v[..., 1::2]
+    out = np.empty_like(v)
+    out[..., 0::2] = re * c - im * s
+    out[..., 1::2] = re * s + im * c
+    return out
+
+
+def softmax(s, axis: int = -1) -> np.ndarray:
+    """exp(s - max) / sum(exp(s - max)); -inf entries get probability 0."""
+    s = _f64(s)
+    m = np.max(s, axis=axis, keepdims=True)
+    e = np.exp(s - m)
+    return e / np.sum(e, axis=axis, keepdims=True)
+
+
+def causal_mask(seqlen: int, start_pos: int) -> np.ndarray:
+    """(seqlen, start_pos+seqlen) mask: 0 where key j <= start_pos + t, -inf above.
+
+    Admin Guide §8.4 (the NOTE on mask construction in Transformer.forward):
+    the cached prefix is fully visible; the new-token block is causal.
+    """
+    t = np.arange(seqlen)[:, None]
+    j = np.arange(start_pos + seqlen)[None, :]
+    m = np.zeros((seqlen, start_pos + seqlen), dtype=np.float64)
+    m[j > start_pos + t] = -np.inf
+    return m
+
+
+def attention(q, keys, values, start_pos: int, n_rep: int) -> np.ndarray:
+    """softmax(Q K^T / sqrt(head_dim) + mask) V for each query head.
+
+    q: [T, n_heads, hd] (already rotated); keys/values: [start_pos+T, n_kv_heads, hd]
+    (the whole cache prefix, already holding this call's keys).  Query head h
+    reads KV head h // n_rep (repeat_kv; source tour, "One model.py").
+    Admin Guide §8.4, Attention forward steps 5-7.
+    """
+    q, keys, values = _f64(q), _f64(keys), _f64(values)
+    T, nh, hd = q.shape
+    mask = causal_mask(T, start_pos)
+    out = np.empty((T, nh, hd), dtype=np.float64)
+    for h in range(nh):
+        g = h // n_rep
+        scores = q[:, h, :] @ keys[:, g, :].T / math.sqrt(hd) + mask
+        out[:, h, :] = softmax(scores, axis=-1) @ values[:, g, :]
+    return out
+
+
+def silu(z) -> np.ndarray:
+    """silu(z) = z * sigmoid(z) = z / (1 + e^{-z})."""
+    z = _f64(z)
+    return z / (1.0 + np.exp(-z))
+
+
+def feed_forward(x, w1, w2, w3) -> np.ndarray:
+    """SwiGLU: w2(silu(w1 x) * w3 x)  (Admin Guide §8.4, FeedForward)."""
+    x = _f64(x)
+    return (silu(x @ _f64(w1).T) * (x @ _f64(w3).T)) @ _f64(w2).T
+
+
+# ---------------------------------------------------------------------------
+# Model with a KV cache (one batch row at a time: rows never interact)
+# ---------------------------------------------------------------------------
+
+class KVCache:
+    """cache_k / cache_v of one batch row: per layer [max_seq_len, n_kv_heads, head_dim],
+    zero-initialised (Admin Guide §6.2 and §8.4, Attention)."""
+
+    def __init__(self, n_layers: int, max_seq_len: int, n_kv_heads: int, head_dim: int):
+        self.k = [np.zeros((max_seq_len, n_kv_heads, head_dim)) for _ in range(n_layers)]
+        self.v = [np.zeros((max_seq_len, n_kv_heads, head_dim)) for _ in range(n_layers)]
+
+
+class Args:
+    """The structural fields of ModelArgs (Admin Guide §3.3)."""
+
+    def __init__(self, dim, n_layers, n_heads, n_kv_heads=None, vocab_size=-1, multiple_of=256,
+                 ffn_dim_multiplier=None, norm_eps=1e-5, rope_theta=10000.0, max_seq_len=2048):
+        self.dim = dim
+        self.n_layers = n_layers
+        self.n_heads = n_heads
+        self.n_kv_heads = n_heads if not n_kv_heads else n_kv_heads
+        assert n_heads % self.n_kv_heads == 0 and dim % n_heads == 0
+        self.vocab_size = vocab_size
+        self.multiple_of = multiple_of
+        self.ffn_dim_multiplier = ffn_dim_multiplier
+        self.norm_eps = norm_eps
+        self.rope_theta = rope_theta
+        self.max_seq_len = max_seq_len
+        self.head_dim = dim // n_heads
+        self.n_rep = n_heads // self.n_kv_heads
+        self.hidden = ffn_hidden_dim(dim, multiple_of, ffn_dim_multiplier)
+
+
+def new_cache(args: Args) -> KVCache:
+    return KVCache(args.n_layers, args.max_seq_len, args.n_kv_heads, args.head_dim)
+
+
+def layer_forward(args: Args, lw, x, cache: KVCache, layer: int, start_pos: int) -> np.ndarray:
+    """One pre-norm TransformerBlock on the T new tokens of one row.
+
+    h = x + attention(attention_norm(x)); out = h + feed_forward(ffn_norm(h))
+    (Admin Guide §8.4, TransformerBlock).  The attention writes this call's
+    keys and values into cache rows start_pos .. start_pos+T-1 and reads rows
+    0 .. start_pos+T-1 (Admin Guide §8.4, Attention forward steps 1-8).
+    """
+    x = _f64(x)
+    T = x.shape[0]
+    nh, nkv, hd = args.n_heads, args.n_kv_heads, args.head_dim
+    pos = start_pos + np.arange(T)
+    y = rms_norm(x, lw["attention_norm"], args.norm_eps)
+    q = (y @ _f64(lw["wq"]).T).reshape(T, nh, hd)
+    k = (y @ _f64(lw["wk"]).T).reshape(T, nkv, hd)
+    v = (y @ _f64(lw["wv"]).T).reshape(T, nkv, hd)
+    q = apply_rope(q, pos, args.rope_theta)
+    k = apply_rope(k, pos, args.rope_theta)
+    cache.k[layer][start_pos:start_pos + T] = k
+    cache.v[layer][start_pos:start_pos + T] = v
+    keys = cache.k[layer][:start_pos + T]
+    values = cache.v[layer][:start_pos + T]
+    o = attention(q, keys, values, start_pos, args.n_rep).reshape(T, nh * hd)
+    h = x + o @ _f64(lw["wo"]).T
+    f = rms_norm(h, lw["ffn_norm"], args.norm_eps)
+    return h + feed_forward(f, lw["w1"], lw["w2"], lw["w3"])
+
+
+def forward(args: Args, w, tokens: Sequence[int], start_pos: int, cache: KVCache,
+            n_layers: Optional[int] = None, logits_positions: Optional[Sequence[int]] = None
+            ) -> np.ndarray:
+    """Transformer.forward(tokens, start_pos) for one batch row.
+
+    Embedding lookup, the blocks, the final RMSNorm, the output projection;
+    returns fp64 logits [T, V] for every new position (or only for the
+    positions listed in `logits_positions`, indices into this call's tokens).
+    Admin Guide §8.4 ("The forward pass", steps 1-6).
+    """
+    toks = np.asarray(tokens, dtype=np.int64)
+    x = _f64(w["tok_embeddings"][toks])
+    layers = w["layers"]
+    L = args.n_layers if n_layers is None else n_layers
+    for l in range(L):
+        x = layer_forward(args, layers[l], x, cache, l, start_pos)
+    if logits_positions is not None:
+        x = x[np.asarray(logits_positions, dtype=np.int64)]
+    h = rms_norm(x, w["norm"], args.norm_eps)
+    return h @ _f64(w["output"]).T
+
+
+# ---------------------------------------------------------------------------
+# Sampling
+# ---------------------------------------------------------------------------
+
+def greedy(logits) -> int:
+    """argmax over the vocabulary, lowest id on ties (Admin Guide §8.5)."""
+    return int(np.argmax(_f64(logits)))  # numpy returns the first maximum
+
+
+def sampling_order(logits) -> np.ndarray:
+    """Token ids by probability descending, equal probabilities by id ascending.
+
+    softmax(l/T) is strictly increasing in the logit, so the exact order of
+    the probabilities is the order of the logits.
+    """
+    l = _f64(logits)
+    return np.lexsort((np.arange(l.shape[0]), -l))
+
+
+def top_p_probs(logits, temperature: float) -> np.ndarray:
+    """softmax(logits / temperature) in fp64 (Admin Guide §8.5)."""
+    l = _f64(logits)
+    return softmax((l - l.max()) / np.float64(temperature))
+
+
+def sample_top_p(logits, temperature: float, top_p: float, u: float) -> int:
+    """Nucleus sampling with the draw made deterministic by a given uniform u in [0,1).
+
+    Follows sample_top_p as the source tour ("Sampling, Stopping, and the
+    Chat Template") and the Admin Guide §6.3 / §8.5 describe it: sort the
+    probabilities descending, zero every token whose preceding cumulative
+    mass already exceeds top_p, renormalise, draw.  The draw is the inverse
+    CDF: the first kept token whose inclusive cumulative mass exceeds u*Z,
+    Z the kept mass (or the last kept token if rounding leaves none).
+    temperature == 0 is the greedy argmax.
+    """
+    if temperature == 0:
+        return greedy(logits)
+    p = top_p_probs(logits, temperature)
+    order = sampling_order(logits)
+    ps = p[order]
+    inclusive = np.cumsum(ps)
+    exclusive = inclusive - ps
+    kept = int(np.count_nonzero(exclusive <= np.float64(top_p)))
+    kept = max(kept, 1)
+    z = inclusive[kept - 1]
+    target = np.float64(u) * z
+    idx = int(np.searchsorted(inclusive[:kept], target, side="right"))
+    if idx >= kept:
+        idx = kept - 1
+    return int(order[idx])
+
+
+def top_p_kept(logits, temperature: float, top_p: float) -> List[int]:
+    """The kept set of sample_top_p, in sampling order (for tests)."""
+    p = top_p_probs(logits, temperature)
+    order = sampling_order(logits)
+    ps = p[order]
+    exclusive = np.cumsum(ps) - ps
+    kept = max(int(np.count_nonzero(exclusive <= np.float64(top_p))), 1)
+    return [int(i) for i in order[:kept]]
+
+
+def sample_margins(logits, temperature: float, top_p: float, u: float) -> float:
+    """Distance (relative to the kept mass) of this draw from a decision
+    boundary of sample_top_p: the draw target from the cumulative masses, the
+    nucleus edge from top_p, and neighbouring probabilities from each other.
+    A float-rounding difference can change an index only when this is tiny.
+    """
+    if temperature == 0:
+        l = np.sort(_f64(logits))[::-1]
+        return float(l[0] - l[1]) if l.shape[0] > 1 else math.inf
+    p = top_p_probs(logits, temperature)
+    order = sampling_order(logits)
+    ps = p[order]
+    inclusive = np.cumsum(ps)
+    exclusive = inclusive - ps
+    kept = max(int(np.count_nonzero(exclusive <= np.float64(top_p))), 1)
+    z = inclusive[kept - 1]
+    target = np.float64(u) * z
+    m = float(np.min(np.abs(inclusive[:kept] - target)) / z)
+    m = min(m, float(np.min(np.abs(exclusive - top_p))))
+    return m
