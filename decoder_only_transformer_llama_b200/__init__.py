@@ -1,0 +1,257 @@
+"""Python binding of libllama_b200.so (argument marshalling only).
+
+Every step of the forward pass and of sampling runs in the library's CUDA
+kernels; this module only turns torch tensors into device pointers and
+streams, and raises on non-zero status codes.  PyTorch provides device memory
+(the model arena) and streams.  There is no CPU path: if the shared library
+has not been built, importing this package raises ImportError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libllama_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python -m decoder_only_transformer_llama_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+LLAMA_OK = 0
+LLAMA_ERR_INVALID_ARG = 1
+LLAMA_ERR_CAPACITY = 2
+LLAMA_ERR_CUDA = 3
+LLAMA_ERR_DEVICE_TIMEOUT = 4
+LLAMA_ERR_TOKEN_RANGE = 5
+LLAMA_F32 = 0
+LLAMA_BF16 = 1
+LLAMA_DECODE_ADVANCE = 1
+
+WEIGHT_IDS = {"tok_embeddings": 0, "norm": 1, "output": 2, "attention_norm": 3, "wq": 4, "wk": 5,
+              "wv": 6, "wo": 7, "ffn_norm": 8, "w1": 9, "w2": 10, "w3": 11}
+
+EXPORTED = ("llama_model_bytes", "llama_model_create", "llama_set_weight", "llama_get_kv",
+            "llama_prefill", "llama_decode_step", "llama_sample", "llama_model_status",
+            "llama_model_destroy", "llama_last_error", "llama_launch_count",
+            "llama_op_rmsnorm", "llama_op_linear")
+
+
+class LlamaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"[{code}] {msg}")
+        self.code = code
+
+
+class ModelArgs(ctypes.Structure):
+    _fields_ = [("dim", ctypes.c_int32), ("n_layers", ctypes.c_int32), ("n_heads", ctypes.c_int32),
+                ("n_kv_heads", ctypes.c_int32), ("vocab_size", ctypes.c_int32),
+                ("multiple_of", ctypes.c_int32), ("ffn_dim_multiplier", ctypes.c_float),
+                ("norm_eps", ctypes.c_float), ("rope_theta", ctypes.c_float),
+                ("max_seq_len", ctypes.c_int32), ("max_batch_size", ctypes.c_int32),
+                ("max_tokens", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+class Sampling(ctypes.Structure):
+    _fields_ = [("temperature", ctypes.c_float), ("top_p", ctypes.c_float)]
+
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+_sz = ctypes.c_size_t
+
+
+def _sig(name, restype, argtypes):
+    fn = getattr(_lib, name)
+    fn.restype = restype
+    fn.argtypes = argtypes
+    return fn
+
+
+_sig("llama_model_bytes", _i, [ctypes.POINTER(ModelArgs), ctypes.POINTER(_sz), ctypes.POINTER(_sz),
+                                ctypes.POINTER(_sz), ctypes.POINTER(_sz), ctypes.POINTER(ctypes.c_int32)])
+_sig("llama_model_create", _i, [ctypes.POINTER(ModelArgs), _vp, _sz, _vp, ctypes.POINTER(_vp)])
+_sig("llama_set_weight", _i, [_vp, _i, _i, _vp, _vp])
+_sig("llama_get_kv", _i, [_vp, _i, ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(ctypes.c_int64)])
+_sig("llama_prefill", _i, [_vp, _vp, ctypes.POINTER(ctypes.c_int32), _i, _i, _i, _vp, _i, _vp])
+_sig("llama_decode_step", _i, [_vp, _vp, _vp, _i, ctypes.POINTER(Sampling), _vp, _vp, _vp, _i, _vp])
+_sig("llama_sample", _i, [_vp, _i, _i, _f, _f, _vp, _vp, _vp])
+_sig("llama_model_status", _i, [_vp, ctypes.POINTER(ctypes.c_int)])
+_sig("llama_model_destroy", _i, [_vp])
+_sig("llama_last_error", ctypes.c_char_p, [])
+_sig("llama_launch_count", ctypes.c_uint64, [])
+_sig("llama_op_rmsnorm", _i, [_vp, _vp, _i, _i, _f, _vp, _i, _vp])
+_sig("llama_op_linear", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp])
+
+
+def lib():
+    return _lib
+
+
+def last_error() -> str:
+    return (_lib.llama_last_error() or b"").decode()
+
+
+def launch_count() -> int:
+    return int(_lib.llama_launch_count())
+
+
+def _check(rc: int):
+    if rc != LLAMA_OK:
+        raise LlamaError(rc, last_error())
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def make_args(dim, n_layers, n_heads, n_kv_heads, vocab_size, multiple_of=256, ffn_dim_multiplier=None,
+              norm_eps=1e-5, rope_theta=10000.0, max_seq_len=2048, max_batch_size=32, max_tokens=0,
+              dtype="bf16") -> ModelArgs:
+    return ModelArgs(dim, n_layers, n_heads, n_kv_heads or 0, vocab_size, multiple_of,
+                     float(ffn_dim_multiplier or 0.0), norm_eps, rope_theta, max_seq_len,
+                     max_batch_size, max_tokens, LLAMA_BF16 if dtype == "bf16" else LLAMA_F32)
+
+
+def args_from_shape(s) -> ModelArgs:
+    """ModelArgs from any object with the ModelArgs field names (e.g. workloads.ModelShape)."""
+    return make_args(s.dim, s.n_layers, s.n_heads, s.n_kv_heads, s.vocab_size, s.multiple_of,
+                     s.ffn_dim_multiplier, s.norm_eps, s.rope_theta, s.max_seq_len, s.max_batch_size,
+                     s.max_tokens, s.dtype)
+
+
+def model_bytes(args: ModelArgs) -> dict:
+    w, kv, ws, tot = _sz(), _sz(), _sz(), _sz()
+    h = ctypes.c_int32()
+    _check(_lib.llama_model_bytes(ctypes.byref(args), ctypes.byref(w), ctypes.byref(kv), ctypes.byref(ws),
+                                  ctypes.byref(tot), ctypes.byref(h)))
+    return {"weights": w.value, "kv": kv.value, "workspace": ws.value, "total": tot.value, "hidden": h.value}
+
+
+class Model:
+    """A model laid out in one torch-allocated device arena."""
+
+    def __init__(self, args: ModelArgs, device="cuda", stream=None):
+        import torch
+        self.args = args
+        self.sizes = model_bytes(args)
+        self.arena = torch.empty(self.sizes["total"], dtype=torch.uint8, device=device)
+        h = _vp()
+        _check(_lib.llama_model_create(ctypes.byref(args), self.arena.data_ptr(), self.sizes["total"],
+                                       _stream(stream), ctypes.byref(h)))
+        self.handle = h
+
+    def close(self):
+        if self.handle:
+            _lib.llama_model_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def set_weight(self, layer: int, name: str, tensor, stream=None):
+        t = tensor.contiguous()
+        _check(_lib.llama_set_weight(self.handle, layer, WEIGHT_IDS[name], t.data_ptr(), _stream(stream)))
+        return t  # keep alive until the stream passes the copy
+
+    def load(self, weights: dict, stream=None):
+        """Upload a weight dict in the workloads layout (torch tensors on the device)."""
+        import torch
+        keep = [self.set_weight(-1, "tok_embeddings", weights["tok_embeddings"], stream),
+                self.set_weight(-1, "norm", weights["norm"], stream),
+                self.set_weight(-1, "output", weights["output"], stream)]
+        for l, layer in enumerate(weights["layers"]):
+            for name, t in layer.items():
+                keep.append(self.set_weight(l, name, t, stream))
+        torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+        del keep
+
+    def kv(self, layer: int):
+        """(k, v, strides) of one layer: device addresses and element strides of
+        the logical [batch_row][position][kv_head][d] index."""
+        k, v = _vp(), _vp()
+        st = (ctypes.c_int64 * 4)()
+        _check(_lib.llama_get_kv(self.handle, layer, ctypes.byref(k), ctypes.byref(v), st))
+        return k.value, v.value, tuple(st)
+
+    def kv_tensors(self, layer: int):
+        """Torch views of one layer's K and V caches, logical shape
+        [max_batch_size, max_seq_len, n_kv_heads, head_dim] (strided)."""
+        import torch
+        k, v, st = self.kv(layer)
+        a = self.args
+        nkv = a.n_kv_heads or a.n_heads
+        hd = a.dim // a.n_heads
+        dt = torch.bfloat16 if a.dtype == LLAMA_BF16 else torch.float32
+        esz = 2 if a.dtype == LLAMA_BF16 else 4
+        n = a.max_batch_size * a.max_seq_len * nkv * hd
+        base = self.arena.data_ptr()
+        out = []
+        for addr in (k, v):
+            flat = self.arena[addr - base: addr - base + n * esz].view(dt)
+            out.append(torch.as_strided(flat, (a.max_batch_size, a.max_seq_len, nkv, hd), st))
+        return out[0], out[1]
+
+    def prefill(self, tokens, lens: Optional[Sequence[int]] = None, start_pos: int = 0, logits=None,
+                all_logits: bool = False, stream=None):
+        B, T = tokens.shape
+        lens_arr = None
+        if lens is not None:
+            lens_arr = (ctypes.c_int32 * B)(*[int(v) for v in lens])
+        _check(_lib.llama_prefill(self.handle, tokens.data_ptr(), lens_arr, B, T, start_pos, _ptr(logits),
+                                  1 if all_logits else 0, _stream(stream)))
+        return logits
+
+    def decode_step(self, tokens, pos, temperature: Optional[float] = None, top_p: float = 0.9,
+                    uniforms=None, next_tokens=None, logits=None, advance: bool = False, stream=None):
+        B = tokens.shape[0]
+        samp = None
+        if temperature is not None:
+            samp = Sampling(float(temperature), float(top_p))
+        _check(_lib.llama_decode_step(self.handle, tokens.data_ptr(), pos.data_ptr(), B,
+                                      ctypes.byref(samp) if samp is not None else None, _ptr(uniforms),
+                                      _ptr(next_tokens), _ptr(logits),
+                                      LLAMA_DECODE_ADVANCE if advance else 0, _stream(stream)))
+        return next_tokens
+
+    def status(self) -> int:
+        s = ctypes.c_int()
+        _check(_lib.llama_model_status(self.handle, ctypes.byref(s)))
+        return s.value
+
+
+def sample(logits, temperature: float, top_p: float, uniforms, out, stream=None):
+    B, V = logits.shape
+    _check(_lib.llama_sample(logits.data_ptr(), B, V, float(temperature), float(top_p), _ptr(uniforms),
+                             out.data_ptr(), _stream(stream)))
+    return out
+
+
+def op_rmsnorm(x, w, eps: float, out, stream=None):
+    M, dim = x.shape
+    dt = LLAMA_BF16 if out.dtype.__str__() == "torch.bfloat16" else LLAMA_F32
+    _check(_lib.llama_op_rmsnorm(x.data_ptr(), w.data_ptr(), M, dim, float(eps), out.data_ptr(), dt,
+                                 _stream(stream)))
+    return out
+
+
+def op_linear(A, W, out, stream=None):
+    M, K = A.shape
+    N = W.shape[0]
+    dt = LLAMA_BF16 if A.dtype.__str__() == "torch.bfloat16" else LLAMA_F32
+    _check(_lib.llama_op_linear(A.data_ptr(), W.data_ptr(), M, N, K, dt, out.data_ptr(), _stream(stream)))
+    return out

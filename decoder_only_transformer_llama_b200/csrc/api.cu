@@ -1,0 +1,485 @@
+// C ABI of libllama_b200.so: argument validation, the arena layout, and the
+// order of kernels in prefill and decode (Admin Guide §8.4, "The forward
+// pass"; §8.5 for the sampling step).  All arithmetic happens in the kernels.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "common.cuh"
+#include "model.h"
+#include "../../include/llama_b200_ops.h"
+
+namespace llb {
+
+static thread_local char g_err[512] = "";
+static std::atomic<uint64_t> g_launches{0};
+
+void set_error(const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+}
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+int cuda_fail(cudaError_t e, const char* what) {
+    set_error("%s: %s", what, cudaGetErrorString(e));
+    return LLAMA_ERR_CUDA;
+}
+
+#define LLB_TRY(x)                       \
+    do {                                 \
+        const int _rc = (x);             \
+        if (_rc != LLAMA_OK) return _rc; \
+    } while (0)
+
+static int hidden_dim(int dim, int multiple_of, float mult) {
+    long long h = 4LL * dim;
+    h = static_cast<long long>(2 * h / 3);
+    if (mult > 0.f) h = static_cast<long long>(static_cast<double>(mult) * static_cast<double>(h));
+    return static_cast<int>(multiple_of * ((h + multiple_of - 1) / multiple_of));
+}
+
+static size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+// Sizes and offsets of everything in the arena.
+struct Layout {
+    int dim, L, nh, nkv, hd, n_rep, H, V, S, Bmax, Mmax, Mrows, Brows, dtype, esz, nq, nkvc, nqkv, n_splits;
+    size_t off_tok_emb, off_norm, off_output, layer_bytes;
+    size_t l_attn_norm, l_wqkv, l_wo, l_ffn_norm, l_w13, l_w2;
+    size_t off_layers, weight_bytes;
+    size_t off_kc, off_vc, kv_bytes;
+    size_t off_x, off_y, off_q, off_attn, off_g, off_ylast, off_tok_ids, off_tok_row, off_tok_pos, off_last,
+        off_logits, off_part_o, off_part_ml, off_status, off_rope, ws_end;
+};
+
+static int make_layout(const llama_model_args* a, Layout* o) {
+    if (!a) { set_error("args is NULL"); return LLAMA_ERR_INVALID_ARG; }
+    if (a->dim <= 0 || a->n_layers <= 0 || a->n_heads <= 0 || a->vocab_size <= 0 || a->multiple_of <= 0 ||
+        a->max_seq_len <= 0 || a->max_batch_size <= 0 || a->n_kv_heads < 0 || a->max_tokens < 0) {
+        set_error("non-positive size in llama_model_args");
+        return LLAMA_ERR_INVALID_ARG;
+    }
+    if (a->dtype != LLAMA_F32 && a->dtype != LLAMA_BF16) { set_error("dtype must be LLAMA_F32 or LLAMA_BF16"); return LLAMA_ERR_INVALID_ARG; }
+    if (!(a->norm_eps >= 0.f) || !(a->rope_theta > 0.f)) { set_error("norm_eps must be >= 0 and rope_theta > 0"); return LLAMA_ERR_INVALID_ARG; }
+    const int nkv = a->n_kv_heads ? a->n_kv_heads : a->n_heads;
+    if (a->n_heads % nkv) { set_error("n_heads %% n_kv_heads != 0"); return LLAMA_ERR_INVALID_ARG; }
+    const int n_rep = a->n_heads / nkv;
+    if (n_rep != 1 && n_rep != 2 && n_rep != 4 && n_rep != 8) { set_error("n_heads / n_kv_heads must be 1, 2, 4 or 8"); return LLAMA_ERR_INVALID_ARG; }
+    if (a->dim % a->n_heads) { set_error("dim %% n_heads != 0"); return LLAMA_ERR_INVALID_ARG; }
+    const int hd = a->dim / a->n_heads;
+    if (hd != 32 && hd != 64 && hd != 128) { set_error("head_dim %d unsupported (32, 64, 128)", hd); return LLAMA_ERR_INVALID_ARG; }
+    if (a->dim % 64) { set_error("dim must be a multiple of 64"); return LLAMA_ERR_INVALID_ARG; }
+    if (a->max_batch_size > kMaxRows) { set_error("max_batch_size > %d", kMaxRows); return LLAMA_ERR_INVALID_ARG; }
+    const int H = hidden_dim(a->dim, a->multiple_of, a->ffn_dim_multiplier);
+    if (H % 64) { set_error("FFN hidden %d must be a multiple of 64", H); return LLAMA_ERR_INVALID_ARG; }
+    if (a->dtype == LLAMA_BF16 && (a->dim < 256 || a->vocab_size < 256)) {
+        set_error("bf16 models need dim >= 256 and vocab_size >= 256");
+        return LLAMA_ERR_INVALID_ARG;
+    }
+    Layout& l = *o;
+    l.dim = a->dim; l.L = a->n_layers; l.nh = a->n_heads; l.nkv = nkv; l.hd = hd; l.n_rep = n_rep; l.H = H;
+    l.V = a->vocab_size; l.S = a->max_seq_len; l.Bmax = a->max_batch_size; l.dtype = a->dtype;
+    l.esz = a->dtype == LLAMA_BF16 ? 2 : 4;
+    const long long mt = a->max_tokens ? a->max_tokens : 1LL * a->max_batch_size * a->max_seq_len;
+    if (mt > (1LL << 30)) { set_error("max_tokens too large"); return LLAMA_ERR_INVALID_ARG; }
+    l.Mmax = static_cast<int>(mt > l.Bmax ? mt : l.Bmax);
+    l.Mrows = l.Mmax < 128 ? 128 : l.Mmax;    // activation buffers hold whole 128-row tiles
+    l.Brows = l.Bmax < 128 ? 128 : l.Bmax;
+    l.nq = l.nh * hd; l.nkvc = nkv * hd; l.nqkv = l.nq + 2 * l.nkvc;
+    l.n_splits = (l.S + kKvChunk - 1) / kKvChunk;
+    const size_t e = l.esz, D = l.dim;
+    size_t off = 0;
+    l.off_tok_emb = off; off = align256(off + static_cast<size_t>(l.V) * D * e);
+    l.off_norm = off; off = align256(off + D * 4);
+    l.off_output = off; off = align256(off + static_cast<size_t>(l.V) * D * e);
+    l.off_layers = off;
+    size_t lo = 0;
+    l.l_attn_norm = lo; lo = align256(lo + D * 4);
+    l.l_wqkv = lo; lo = align256(lo + static_cast<size_t>(l.nqkv) * D * e);
+    l.l_wo = lo; lo = align256(lo + D * l.nq * e);
+    l.l_ffn_norm = lo; lo = align256(lo + D * 4);
+    l.l_w13 = lo; lo = align256(lo + 2ull * H * D * e);
+    l.l_w2 = lo; lo = align256(lo + D * H * e);
+    l.layer_bytes = lo;
+    off += lo * l.L;
+    l.weight_bytes = off;
+    const size_t kv_one = static_cast<size_t>(l.L) * l.Bmax * nkv * l.S * hd * e;
+    l.off_kc = off; off = align256(off + kv_one);
+    l.off_vc = off; off = align256(off + kv_one);
+    l.kv_bytes = off - l.weight_bytes;
+    const size_t M = l.Mrows, Bn = l.Brows;
+    l.off_x = off; off = align256(off + M * D * 4);
+    l.off_y = off; off = align256(off + M * D * e);
+    l.off_q = off; off = align256(off + M * l.nq * e);
+    l.off_attn = off; off = align256(off + M * l.nq * e);
+    l.off_g = off; off = align256(off + M * H * e);
+    l.off_ylast = off; off = align256(off + Bn * D * e);
+    l.off_tok_ids = off; off = align256(off + M * 4);
+    l.off_tok_row = off; off = align256(off + M * 4);
+    l.off_tok_pos = off; off = align256(off + M * 4);
+    l.off_last = off; off = align256(off + Bn * 4);
+    l.off_logits = off; off = align256(off + static_cast<size_t>(l.Bmax) * l.V * 4);
+    const size_t slots = static_cast<size_t>(l.Bmax) * l.nh * l.n_splits;
+    l.off_part_o = off; off = align256(off + slots * hd * 4);
+    l.off_part_ml = off; off = align256(off + slots * 2 * 4);
+    l.off_status = off; off = align256(off + 16);
+    l.off_rope = off; off = align256(off + static_cast<size_t>(l.S) * (hd / 2) * 8);
+    l.ws_end = off;
+    return LLAMA_OK;
+}
+
+static int make_maps(TmaMaps* t, const void* base, int rows, int cols, int b_box) {
+    LLB_TRY(encode_kmajor_bf16(&t->a128, base, rows, cols, 128));
+    LLB_TRY(encode_kmajor_bf16(&t->b, base, rows, cols, b_box));
+    return LLAMA_OK;
+}
+
+int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, const void* W,
+               const TmaMaps* mapW, int M, int N, int K, const Epi& ep, cudaStream_t st) {
+    if (dtype == LLAMA_F32)
+        return linear_f32(static_cast<const float*>(A), static_cast<const float*>(W), M, N, K, ep, st);
+    (void)m;
+    return linear_bf16_tc(mapA, mapW, M, N, K, ep, st);
+}
+
+static Epi base_epi(const Model* m) {
+    Epi ep;
+    memset(&ep, 0, sizeof(ep));
+    ep.status = m->status;
+    ep.nq = m->nq;
+    ep.nkvc = m->nkvc;
+    ep.hd = m->hd;
+    ep.max_seq = m->S;
+    ep.kv_row_stride = m->kv_row_elems;
+    ep.rope = m->rope;
+    ep.H = m->H;
+    return ep;
+}
+
+static char* at(void* base, size_t off) { return static_cast<char*>(base) + off; }
+
+// One transformer block on M token rows held in m->x (Admin Guide §8.4,
+// TransformerBlock: h = x + attn(norm(x)); out = h + ffn(norm(h))).
+template <typename AttnFn>
+static int block_forward(Model* m, int l, int M, const int* tok_row, const int* tok_pos, AttnFn attn,
+                         cudaStream_t st) {
+    LayerPtrs& Lp = m->layers[l];
+    const size_t esz = m->esz;
+    LLB_TRY(launch_rmsnorm(m->x, nullptr, Lp.attn_norm, M, m->dim, m->a.norm_eps, m->y, m->dtype, st));
+    Epi ep = base_epi(m);
+    ep.mode = EPI_QKV;
+    ep.q = m->q;
+    ep.kc = static_cast<char*>(m->kc) + l * m->kv_layer_elems * esz;
+    ep.vc = static_cast<char*>(m->vc) + l * m->kv_layer_elems * esz;
+    ep.tok_row = tok_row;
+    ep.tok_pos = tok_pos;
+    LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.wqkv, &Lp.m_wqkv, M, m->nqkv, m->dim, ep, st));
+    LLB_TRY(attn());
+    Epi er = base_epi(m);
+    er.mode = EPI_RESID_F32;
+    er.out = m->x;
+    er.ldo = m->dim;
+    LLB_TRY(run_linear(m, m->dtype, m->attn, &m->m_attn, Lp.wo, &Lp.m_wo, M, m->dim, m->nq, er, st));
+    LLB_TRY(launch_rmsnorm(m->x, nullptr, Lp.ffn_norm, M, m->dim, m->a.norm_eps, m->y, m->dtype, st));
+    Epi es = base_epi(m);
+    es.mode = EPI_SWIGLU;
+    es.g = m->g;
+    LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.w13, &Lp.m_w13, M, 2 * m->H, m->dim, es, st));
+    LLB_TRY(run_linear(m, m->dtype, m->g, &m->m_g, Lp.w2, &Lp.m_w2, M, m->dim, m->H, er, st));
+    return LLAMA_OK;
+}
+
+}  // namespace llb
+
+using namespace llb;
+
+struct llama_model : public llb::Model {};
+
+extern "C" {
+
+const char* llama_last_error(void) { return g_err; }
+uint64_t llama_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int llama_model_bytes(const llama_model_args* args, size_t* weight_bytes, size_t* kv_bytes,
+                      size_t* workspace_bytes, size_t* total_bytes, int32_t* hidden) {
+    Layout l;
+    LLB_TRY(make_layout(args, &l));
+    if (weight_bytes) *weight_bytes = l.weight_bytes;
+    if (kv_bytes) *kv_bytes = l.kv_bytes;
+    if (workspace_bytes) *workspace_bytes = l.ws_end - l.weight_bytes - l.kv_bytes;
+    if (total_bytes) *total_bytes = l.ws_end;
+    if (hidden) *hidden = l.H;
+    return LLAMA_OK;
+}
+
+int llama_model_create(const llama_model_args* args, void* dev_arena, size_t arena_bytes, void* stream,
+                       llama_model** out) {
+    if (!out) { set_error("out is NULL"); return LLAMA_ERR_INVALID_ARG; }
+    *out = nullptr;
+    Layout l;
+    LLB_TRY(make_layout(args, &l));
+    if (!dev_arena) { set_error("arena is NULL"); return LLAMA_ERR_INVALID_ARG; }
+    if (reinterpret_cast<uintptr_t>(dev_arena) & 255) { set_error("arena must be 256-byte aligned"); return LLAMA_ERR_INVALID_ARG; }
+    if (arena_bytes < l.ws_end) {
+        set_error("arena too small: %zu < %zu bytes", arena_bytes, l.ws_end);
+        return LLAMA_ERR_CAPACITY;
+    }
+    llama_model* m = new (std::nothrow) llama_model();
+    if (!m) { set_error("host allocation failed"); return LLAMA_ERR_CAPACITY; }
+    m->a = *args;
+    m->dim = l.dim; m->L = l.L; m->nh = l.nh; m->nkv = l.nkv; m->hd = l.hd; m->n_rep = l.n_rep; m->H = l.H;
+    m->V = l.V; m->S = l.S; m->Bmax = l.Bmax; m->Mmax = l.Mmax; m->dtype = l.dtype; m->esz = l.esz;
+    m->nq = l.nq; m->nkvc = l.nkvc; m->nqkv = l.nqkv; m->n_splits = l.n_splits;
+    void* A = dev_arena;
+    m->tok_emb = at(A, l.off_tok_emb);
+    m->norm = reinterpret_cast<float*>(at(A, l.off_norm));
+    m->output = at(A, l.off_output);
+    m->layers.resize(l.L);
+    for (int i = 0; i < l.L; ++i) {
+        char* base = at(A, l.off_layers + i * l.layer_bytes);
+        LayerPtrs& p = m->layers[i];
+        p.attn_norm = reinterpret_cast<float*>(base + l.l_attn_norm);
+        p.wqkv = base + l.l_wqkv;
+        p.wo = base + l.l_wo;
+        p.ffn_norm = reinterpret_cast<float*>(base + l.l_ffn_norm);
+        p.w13 = base + l.l_w13;
+        p.w2 = base + l.l_w2;
+    }
+    m->kc = at(A, l.off_kc);
+    m->vc = at(A, l.off_vc);
+    m->kv_head_elems = static_cast<long long>(l.S) * l.hd;
+    m->kv_row_elems = m->kv_head_elems * l.nkv;
+    m->kv_layer_elems = m->kv_row_elems * l.Bmax;
+    m->x = reinterpret_cast<float*>(at(A, l.off_x));
+    m->y = at(A, l.off_y);
+    m->q = at(A, l.off_q);
+    m->attn = at(A, l.off_attn);
+    m->g = at(A, l.off_g);
+    m->ylast = at(A, l.off_ylast);
+    m->tok_ids = reinterpret_cast<int*>(at(A, l.off_tok_ids));
+    m->tok_row = reinterpret_cast<int*>(at(A, l.off_tok_row));
+    m->tok_pos = reinterpret_cast<int*>(at(A, l.off_tok_pos));
+    m->last_idx = reinterpret_cast<int*>(at(A, l.off_last));
+    m->logits_ws = reinterpret_cast<float*>(at(A, l.off_logits));
+    m->part_o = reinterpret_cast<float*>(at(A, l.off_part_o));
+    m->part_ml = reinterpret_cast<float*>(at(A, l.off_part_ml));
+    m->status = reinterpret_cast<int*>(at(A, l.off_status));
+    m->rope = reinterpret_cast<float2*>(at(A, l.off_rope));
+    m->last_stream = static_cast<cudaStream_t>(stream);
+
+    int rc = LLAMA_OK;
+    if (l.dtype == LLAMA_BF16) {
+        for (int i = 0; i < l.L && rc == LLAMA_OK; ++i) {
+            LayerPtrs& p = m->layers[i];
+            if (rc == LLAMA_OK) rc = make_maps(&p.m_wqkv, p.wqkv, l.nqkv, l.dim, 256);
+            if (rc == LLAMA_OK) rc = make_maps(&p.m_wo, p.wo, l.dim, l.nq, 256);
+            if (rc == LLAMA_OK) rc = make_maps(&p.m_w13, p.w13, 2 * l.H, l.dim, 256);
+            if (rc == LLAMA_OK) rc = make_maps(&p.m_w2, p.w2, l.dim, l.H, 256);
+        }
+        if (rc == LLAMA_OK) rc = make_maps(&m->m_output, m->output, l.V, l.dim, 256);
+        if (rc == LLAMA_OK) rc = make_maps(&m->m_y, m->y, l.Mrows, l.dim, 16);
+        if (rc == LLAMA_OK) rc = make_maps(&m->m_attn, m->attn, l.Mrows, l.nq, 16);
+        if (rc == LLAMA_OK) rc = make_maps(&m->m_g, m->g, l.Mrows, l.H, 16);
+        if (rc == LLAMA_OK) rc = make_maps(&m->m_ylast, m->ylast, l.Brows, l.dim, 16);
+    }
+    cudaStream_t st = m->last_stream;
+    if (rc == LLAMA_OK) {
+        cudaError_t e = cudaMemsetAsync(m->kc, 0, l.kv_bytes, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(m->status, 0, 16, st);
+        if (e != cudaSuccess) rc = cuda_fail(e, "cudaMemsetAsync");
+    }
+    if (rc == LLAMA_OK) rc = launch_rope_table(m->rope, l.S, l.hd, args->rope_theta, st);
+    if (rc != LLAMA_OK) {
+        delete m;
+        return rc;
+    }
+    *out = m;
+    return LLAMA_OK;
+}
+
+int llama_set_weight(llama_model* m, int layer, int which, const void* src, void* stream) {
+    if (!m || !src) { set_error("model or src is NULL"); return LLAMA_ERR_INVALID_ARG; }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    m->last_stream = st;
+    const size_t e = m->esz, D = m->dim;
+    const bool global = which == LLAMA_W_TOK_EMBEDDINGS || which == LLAMA_W_NORM || which == LLAMA_W_OUTPUT;
+    if (which < 0 || which > LLAMA_W_W3) { set_error("unknown weight id %d", which); return LLAMA_ERR_INVALID_ARG; }
+    if (global ? layer != -1 : (layer < 0 || layer >= m->L)) {
+        set_error("layer %d invalid for weight %d", layer, which);
+        return LLAMA_ERR_INVALID_ARG;
+    }
+    void* dst = nullptr;
+    size_t bytes = 0;
+    LayerPtrs* p = global ? nullptr : &m->layers[layer];
+    switch (which) {
+        case LLAMA_W_TOK_EMBEDDINGS: dst = m->tok_emb; bytes = static_cast<size_t>(m->V) * D * e; break;
+        case LLAMA_W_NORM: dst = m->norm; bytes = D * 4; break;
+        case LLAMA_W_OUTPUT: dst = m->output; bytes = static_cast<size_t>(m->V) * D * e; break;
+        case LLAMA_W_ATTENTION_NORM: dst = p->attn_norm; bytes = D * 4; break;
+        case LLAMA_W_WQ: dst = p->wqkv; bytes = static_cast<size_t>(m->nq) * D * e; break;
+        case LLAMA_W_WK: dst = static_cast<char*>(p->wqkv) + static_cast<size_t>(m->nq) * D * e;
+                         bytes = static_cast<size_t>(m->nkvc) * D * e; break;
+        case LLAMA_W_WV: dst = static_cast<char*>(p->wqkv) + static_cast<size_t>(m->nq + m->nkvc) * D * e;
+                         bytes = static_cast<size_t>(m->nkvc) * D * e; break;
+        case LLAMA_W_WO: dst = p->wo; bytes = D * m->nq * e; break;
+        case LLAMA_W_FFN_NORM: dst = p->ffn_norm; bytes = D * 4; break;
+        case LLAMA_W_W2: dst = p->w2; bytes = D * m->H * e; break;
+        case LLAMA_W_W1:
+        case LLAMA_W_W3:
+            if ((reinterpret_cast<uintptr_t>(src) & 15) != 0) { set_error("w1/w3 source must be 16-byte aligned"); return LLAMA_ERR_INVALID_ARG; }
+            return launch_copy_interleave_w13(src, p->w13, m->H, m->dim, which == LLAMA_W_W3 ? 1 : 0,
+                                              m->esz, st);
+    }
+    cudaError_t ce = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st);
+    if (ce != cudaSuccess) return cuda_fail(ce, "cudaMemcpyAsync(weight)");
+    return LLAMA_OK;
+}
+
+int llama_get_kv(llama_model* m, int layer, void** k, void** v, int64_t strides[4]) {
+    if (!m || layer < 0 || layer >= m->L) { set_error("bad model or layer"); return LLAMA_ERR_INVALID_ARG; }
+    const size_t off = static_cast<size_t>(layer) * m->kv_layer_elems * m->esz;
+    if (k) *k = static_cast<char*>(m->kc) + off;
+    if (v) *v = static_cast<char*>(m->vc) + off;
+    if (strides) {
+        strides[0] = m->kv_row_elems;   // batch row
+        strides[1] = m->hd;             // position
+        strides[2] = m->kv_head_elems;  // kv head
+        strides[3] = 1;                 // head dim
+    }
+    return LLAMA_OK;
+}
+
+int llama_prefill(llama_model* m, const int32_t* tokens, const int32_t* lens, int B, int T, int start_pos,
+                  float* logits, int logits_mode, void* stream) {
+    if (!m || !tokens) { set_error("model or tokens is NULL"); return LLAMA_ERR_INVALID_ARG; }
+    if (B <= 0 || T <= 0 || start_pos < 0) { set_error("B and T must be positive, start_pos >= 0"); return LLAMA_ERR_INVALID_ARG; }
+    if (logits_mode != 0 && logits_mode != 1) { set_error("logits_mode must be 0 or 1"); return LLAMA_ERR_INVALID_ARG; }
+    if (logits_mode == 1 && !logits) { set_error("logits_mode 1 needs a logits buffer"); return LLAMA_ERR_INVALID_ARG; }
+    if (B > m->Bmax) { set_error("B=%d > max_batch_size=%d", B, m->Bmax); return LLAMA_ERR_CAPACITY; }
+    if (static_cast<long long>(start_pos) + T > m->S) {
+        set_error("start_pos + T = %lld > max_seq_len=%d", static_cast<long long>(start_pos) + T, m->S);
+        return LLAMA_ERR_CAPACITY;
+    }
+    RowTable rt;
+    rt.B = B; rt.T = T; rt.start_pos = start_pos;
+    rt.cu[0] = 0;
+    for (int b = 0; b < B; ++b) {
+        const int len = lens ? lens[b] : T;
+        if (len < 1 || len > T) { set_error("lens[%d]=%d outside [1, T=%d]", b, len, T); return LLAMA_ERR_INVALID_ARG; }
+        rt.cu[b + 1] = rt.cu[b] + len;
+    }
+    const int M = rt.cu[B];
+    if (M > m->Mmax) { set_error("sum(lens)=%d > max_tokens=%d", M, m->Mmax); return LLAMA_ERR_CAPACITY; }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    m->last_stream = st;
+
+    LLB_TRY(launch_token_map(rt, tokens, m->tok_ids, m->tok_row, m->tok_pos, m->last_idx, st));
+    LLB_TRY(launch_embed(m->tok_ids, m->tok_emb, m->dtype, M, m->dim, m->V, m->x, m->status, st));
+    for (int l = 0; l < m->L; ++l) {
+        auto attn = [&]() { return launch_attention_prefill(m, l, rt, st); };
+        LLB_TRY(block_forward(m, l, M, m->tok_row, m->tok_pos, attn, st));
+    }
+    if (!logits) return LLAMA_OK;
+    Epi eo = base_epi(m);
+    eo.mode = EPI_STORE_F32;
+    eo.out = logits;
+    eo.ldo = m->V;
+    if (logits_mode == 0) {
+        LLB_TRY(launch_rmsnorm(m->x, m->last_idx, m->norm, B, m->dim, m->a.norm_eps, m->ylast, m->dtype, st));
+        return run_linear(m, m->dtype, m->ylast, &m->m_ylast, m->output, &m->m_output, B, m->V, m->dim, eo, st);
+    }
+    LLB_TRY(launch_rmsnorm(m->x, nullptr, m->norm, M, m->dim, m->a.norm_eps, m->y, m->dtype, st));
+    return run_linear(m, m->dtype, m->y, &m->m_y, m->output, &m->m_output, M, m->V, m->dim, eo, st);
+}
+
+int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B, const llama_sampling* sampling,
+                      const float* uniforms, int32_t* next_tokens, float* logits, int flags, void* stream) {
+    if (!m || !tokens || !pos) { set_error("model, tokens or pos is NULL"); return LLAMA_ERR_INVALID_ARG; }
+    if (B <= 0) { set_error("B must be positive"); return LLAMA_ERR_INVALID_ARG; }
+    if (B > m->Bmax) { set_error("B=%d > max_batch_size=%d", B, m->Bmax); return LLAMA_ERR_CAPACITY; }
+    if (sampling && !next_tokens) { set_error("sampling needs next_tokens"); return LLAMA_ERR_INVALID_ARG; }
+    if (sampling && sampling->temperature < 0.f) { set_error("temperature must be >= 0"); return LLAMA_ERR_INVALID_ARG; }
+    if (sampling && sampling->temperature > 0.f && !uniforms) { set_error("top-p sampling needs uniforms"); return LLAMA_ERR_INVALID_ARG; }
+    if ((flags & LLAMA_DECODE_ADVANCE) && !sampling) { set_error("LLAMA_DECODE_ADVANCE needs sampling"); return LLAMA_ERR_INVALID_ARG; }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    m->last_stream = st;
+
+    LLB_TRY(launch_embed(tokens, m->tok_emb, m->dtype, B, m->dim, m->V, m->x, m->status, st));
+    for (int l = 0; l < m->L; ++l) {
+        auto attn = [&]() { return launch_attention_decode(m, l, pos, B, st); };
+        LLB_TRY(block_forward(m, l, B, nullptr, pos, attn, st));
+    }
+    LLB_TRY(launch_rmsnorm(m->x, nullptr, m->norm, B, m->dim, m->a.norm_eps, m->ylast, m->dtype, st));
+    float* lg = logits ? logits : m->logits_ws;
+    Epi eo = base_epi(m);
+    eo.mode = EPI_STORE_F32;
+    eo.out = lg;
+    eo.ldo = m->V;
+    LLB_TRY(run_linear(m, m->dtype, m->ylast, &m->m_ylast, m->output, &m->m_output, B, m->V, m->dim, eo, st));
+    if (!sampling) return LLAMA_OK;
+    const bool adv = (flags & LLAMA_DECODE_ADVANCE) != 0;
+    int32_t* tok_adv = adv ? const_cast<int32_t*>(tokens) : nullptr;
+    int32_t* pos_adv = adv ? pos : nullptr;
+    if (sampling->temperature == 0.f) return launch_argmax(lg, B, m->V, next_tokens, tok_adv, pos_adv, st);
+    return launch_top_p(lg, B, m->V, sampling->temperature, sampling->top_p, uniforms, next_tokens, tok_adv,
+                        pos_adv, st);
+}
+
+int llama_sample(const float* logits, int B, int V, float temperature, float top_p, const float* uniforms,
+                 int32_t* out, void* stream) {
+    if (!logits || !out) { set_error("logits or out is NULL"); return LLAMA_ERR_INVALID_ARG; }
+    if (B <= 0 || V <= 0 || V > 262144) { set_error("B must be positive and 0 < V <= 262144"); return LLAMA_ERR_INVALID_ARG; }
+    if (!(temperature >= 0.f)) { set_error("temperature must be >= 0"); return LLAMA_ERR_INVALID_ARG; }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (temperature == 0.f) return launch_argmax(logits, B, V, out, nullptr, nullptr, st);
+    if (!uniforms) { set_error("top-p sampling needs uniforms"); return LLAMA_ERR_INVALID_ARG; }
+    if (!(top_p >= 0.f)) { set_error("top_p must be >= 0"); return LLAMA_ERR_INVALID_ARG; }
+    return launch_top_p(logits, B, V, temperature, top_p, uniforms, out, nullptr, nullptr, st);
+}
+
+int llama_model_status(llama_model* m, int* device_status) {
+    if (!m || !device_status) { set_error("model or device_status is NULL"); return LLAMA_ERR_INVALID_ARG; }
+    cudaError_t e = cudaStreamSynchronize(m->last_stream);
+    if (e == cudaSuccess) e = cudaMemcpy(device_status, m->status, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemset(m->status, 0, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "llama_model_status");
+    return LLAMA_OK;
+}
+
+int llama_model_destroy(llama_model* m) {
+    delete m;
+    return LLAMA_OK;
+}
+
+// ---------------------------------------------------------------- single-kernel ops
+int llama_op_rmsnorm(const float* x, const float* w, int M, int dim, float eps, void* out, int out_dtype,
+                     void* stream) {
+    if (!x || !w || !out || M < 0 || dim <= 0 || dim % 4) { set_error("bad rmsnorm arguments"); return LLAMA_ERR_INVALID_ARG; }
+    if (out_dtype != LLAMA_F32 && out_dtype != LLAMA_BF16) { set_error("bad out_dtype"); return LLAMA_ERR_INVALID_ARG; }
+    return launch_rmsnorm(x, nullptr, w, M, dim, eps, out, out_dtype, static_cast<cudaStream_t>(stream));
+}
+
+int llama_op_linear(const void* A, const void* W, int M, int N, int K, int dtype, float* out, void* stream) {
+    if (!A || !W || !out || M < 0 || N <= 0 || K <= 0) { set_error("bad linear arguments"); return LLAMA_ERR_INVALID_ARG; }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Epi ep;
+    memset(&ep, 0, sizeof(ep));
+    ep.mode = EPI_STORE_F32;
+    ep.out = out;
+    ep.ldo = N;
+    if (dtype == LLAMA_F32)
+        return linear_f32(static_cast<const float*>(A), static_cast<const float*>(W), M, N, K, ep, st);
+    if (dtype != LLAMA_BF16) { set_error("bad dtype"); return LLAMA_ERR_INVALID_ARG; }
+    if (K % 8) { set_error("bf16 linear needs K %% 8 == 0"); return LLAMA_ERR_INVALID_ARG; }
+    if (M == 0) return LLAMA_OK;
+    TmaMaps ma, mw;
+    LLB_TRY(encode_kmajor_bf16(&ma.a128, A, M, K, 128));
+    LLB_TRY(encode_kmajor_bf16(&ma.b, A, M, K, 16));
+    LLB_TRY(encode_kmajor_bf16(&mw.a128, W, N, K, 128));
+    LLB_TRY(encode_kmajor_bf16(&mw.b, W, N, K, 256));
+    return linear_bf16_tc(&ma, &mw, M, N, K, ep, st);
+}
+
+}  // extern "C"

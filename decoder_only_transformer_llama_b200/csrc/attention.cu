@@ -1,0 +1,352 @@
+// Causal grouped-query attention over the KV cache (Admin Guide §8.4,
+// Attention steps 5-7 and the mask NOTE; repeat_kv from the source tour):
+//   o_h = softmax_j( q_h . K[j][h / n_rep] / sqrt(hd) ) V[j][h / n_rep],
+//   keys j = 0 .. position of the query (the cached prefix plus the causal part
+//   of this call's tokens).  The -inf mask is realised as a key-range bound.
+//
+// Decode (one query per row): split-KV.  CTA (split s, kv head g, row b)
+// streams keys [s*chunk, (s+1)*chunk) of head g ONCE for all n_rep query heads
+// of the group, keeps an online softmax per head, and writes an unnormalised
+// partial (o, max, sum); a combine kernel merges the splits per (b, h).
+//
+// Prefill: one CTA per (64-query tile, head, row), online softmax over 64-key
+// tiles staged in shared memory (fp32 CUDA-core arithmetic).
+#include "common.cuh"
+#include "model.h"
+
+namespace llb {
+
+// ---------------------------------------------------------------- vector loads
+template <typename T, int N> struct Vec;
+template <> struct Vec<float, 1> { static __device__ __forceinline__ void load(const float* p, float* o) { o[0] = p[0]; } };
+template <> struct Vec<float, 2> {
+    static __device__ __forceinline__ void load(const float* p, float* o) {
+        const float2 v = *reinterpret_cast<const float2*>(p); o[0] = v.x; o[1] = v.y;
+    }
+};
+template <> struct Vec<float, 4> {
+    static __device__ __forceinline__ void load(const float* p, float* o) {
+        const float4 v = *reinterpret_cast<const float4*>(p); o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+    }
+};
+template <> struct Vec<bf16, 1> { static __device__ __forceinline__ void load(const bf16* p, float* o) { o[0] = __bfloat162float(p[0]); } };
+template <> struct Vec<bf16, 2> {
+    static __device__ __forceinline__ void load(const bf16* p, float* o) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p)); o[0] = f.x; o[1] = f.y;
+    }
+};
+template <> struct Vec<bf16, 4> {
+    static __device__ __forceinline__ void load(const bf16* p, float* o) {
+        const uint2 u = *reinterpret_cast<const uint2*>(p);
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+        o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
+    }
+};
+
+// ---------------------------------------------------------------- decode
+template <typename T, int HD, int NREP, int UNROLL>
+__global__ void __launch_bounds__(128)
+attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
+                   const int32_t* __restrict__ pos, int nq, int S, long long row_stride, int chunk,
+                   int n_splits, float* __restrict__ part_o, float* __restrict__ part_ml, int* status) {
+    constexpr int EPL = HD / 32;   // head dims per lane
+    const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int p = pos[b];
+    if (p < 0 || p >= S) {
+        if (s == 0 && g == 0 && threadIdx.x == 0) report_status(status, LLAMA_ERR_CAPACITY);
+        return;
+    }
+    const int ctx = p + 1;
+    const int j0 = s * chunk;
+    if (j0 >= ctx) return;
+    const int j1 = min(ctx, j0 + chunk);
+
+    const float scale = rsqrtf(static_cast<float>(HD));
+    float qv[NREP][EPL];
+#pragma unroll
+    for (int r = 0; r < NREP; ++r) {
+        Vec<T, EPL>::load(q + static_cast<long long>(b) * nq + (g * NREP + r) * HD + lane * EPL, qv[r]);
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) qv[r][e] *= scale;
+    }
+    const T* kb = kc + static_cast<long long>(b) * row_stride + static_cast<long long>(g) * S * HD + lane * EPL;
+    const T* vb = vc + static_cast<long long>(b) * row_stride + static_cast<long long>(g) * S * HD + lane * EPL;
+
+    float mx[NREP], sm[NREP], o[NREP][EPL];
+#pragma unroll
+    for (int r = 0; r < NREP; ++r) {
+        mx[r] = -INFINITY;
+        sm[r] = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) o[r][e] = 0.f;
+    }
+
+    // warp w takes keys j0 + w*UNROLL + 4*UNROLL*i + u
+    for (int jb = j0 + warp * UNROLL; jb < j1; jb += 4 * UNROLL) {
+        float kv[UNROLL][EPL], vv[UNROLL][EPL];
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+            const int j = min(jb + u, j1 - 1);
+            Vec<T, EPL>::load(kb + static_cast<long long>(j) * HD, kv[u]);
+            Vec<T, EPL>::load(vb + static_cast<long long>(j) * HD, vv[u]);
+        }
+#pragma unroll
+        for (int r = 0; r < NREP; ++r) {
+            float sc[UNROLL];
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                float d = 0.f;
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) d = fmaf(qv[r][e], kv[u][e], d);
+                sc[u] = warp_sum(d);
+                if (jb + u >= j1) sc[u] = -INFINITY;
+            }
+            float mnew = mx[r];
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) mnew = fmaxf(mnew, sc[u]);
+            const float corr = __expf(mx[r] - mnew);
+            sm[r] *= corr;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) o[r][e] *= corr;
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                const float pj = __expf(sc[u] - mnew);
+                sm[r] += pj;
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) o[r][e] = fmaf(pj, vv[u][e], o[r][e]);
+            }
+            mx[r] = mnew;
+        }
+    }
+
+    // merge the 4 warps
+    __shared__ float s_m[4][NREP], s_l[4][NREP];
+    __shared__ float s_o[4][NREP][HD];
+    if (lane == 0) {
+#pragma unroll
+        for (int r = 0; r < NREP; ++r) { s_m[warp][r] = mx[r]; s_l[warp][r] = sm[r]; }
+    }
+#pragma unroll
+    for (int r = 0; r < NREP; ++r)
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) s_o[warp][r][lane * EPL + e] = o[r][e];
+    __syncthreads();
+    const int nh = nq / HD;
+    for (int idx = threadIdx.x; idx < NREP * HD; idx += blockDim.x) {
+        const int r = idx / HD, d = idx % HD;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, s_m[w][r]);
+        float L = 0.f, acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const float f = (s_m[w][r] == -INFINITY) ? 0.f : __expf(s_m[w][r] - M);
+            L += s_l[w][r] * f;
+            acc += s_o[w][r][d] * f;
+        }
+        const long long slot = (static_cast<long long>(b) * nh + g * NREP + r) * n_splits + s;
+        part_o[slot * HD + d] = acc;
+        if (d == 0) {
+            part_ml[slot * 2] = M;
+            part_ml[slot * 2 + 1] = L;
+        }
+    }
+}
+
+template <typename T, int HD>
+__global__ void attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
+                                    const int32_t* __restrict__ pos, int nh, int S, int chunk, int n_splits,
+                                    T* __restrict__ out) {
+    const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+    const int p = pos[b];
+    if (p < 0 || p >= S) return;
+    const int nvalid = (p + 1 + chunk - 1) / chunk;
+    const long long base = (static_cast<long long>(b) * nh + h) * n_splits;
+    float M = -INFINITY;
+    for (int s = 0; s < nvalid; ++s) M = fmaxf(M, part_ml[(base + s) * 2]);
+    float L = 0.f, acc = 0.f;
+    for (int s = 0; s < nvalid; ++s) {
+        const float f = __expf(part_ml[(base + s) * 2] - M);
+        L += part_ml[(base + s) * 2 + 1] * f;
+        acc += part_o[(base + s) * HD + d] * f;
+    }
+    out[static_cast<long long>(b) * nh * HD + h * HD + d] = from_f32<T>(acc / L);
+}
+
+template <typename T, int HD, int NREP>
+static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st) {
+    const T* kc = static_cast<const T*>(m->kc) + layer * m->kv_layer_elems;
+    const T* vc = static_cast<const T*>(m->vc) + layer * m->kv_layer_elems;
+    dim3 grid(m->n_splits, m->nkv, B);
+    attn_decode_kernel<T, HD, NREP, 4><<<grid, 128, 0, st>>>(
+        static_cast<const T*>(m->q), kc, vc, pos, m->nq, m->S, m->kv_row_elems, kKvChunk, m->n_splits,
+        m->part_o, m->part_ml, m->status);
+    LLB_CHECK_LAUNCH("attn_decode_kernel");
+    attn_combine_kernel<T, HD><<<dim3(m->nh, B), HD, 0, st>>>(m->part_o, m->part_ml, pos, m->nh, m->S,
+                                                              kKvChunk, m->n_splits, static_cast<T*>(m->attn));
+    LLB_CHECK_LAUNCH("attn_combine_kernel");
+    return LLAMA_OK;
+}
+
+template <typename T, int HD>
+static int decode_rep(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st) {
+    switch (m->n_rep) {
+        case 1: return decode_go<T, HD, 1>(m, layer, pos, B, st);
+        case 2: return decode_go<T, HD, 2>(m, layer, pos, B, st);
+        case 4: return decode_go<T, HD, 4>(m, layer, pos, B, st);
+        case 8: return decode_go<T, HD, 8>(m, layer, pos, B, st);
+    }
+    set_error("n_heads / n_kv_heads = %d unsupported (1, 2, 4, 8)", m->n_rep);
+    return LLAMA_ERR_INVALID_ARG;
+}
+
+template <typename T>
+static int decode_hd(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st) {
+    switch (m->hd) {
+        case 32: return decode_rep<T, 32>(m, layer, pos, B, st);
+        case 64: return decode_rep<T, 64>(m, layer, pos, B, st);
+        case 128: return decode_rep<T, 128>(m, layer, pos, B, st);
+    }
+    set_error("head_dim %d unsupported", m->hd);
+    return LLAMA_ERR_INVALID_ARG;
+}
+
+int launch_attention_decode(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st) {
+    if (m->dtype == LLAMA_BF16) return decode_hd<bf16>(m, layer, pos, B, st);
+    return decode_hd<float>(m, layer, pos, B, st);
+}
+
+// ---------------------------------------------------------------- prefill
+namespace {
+constexpr int PQ = 64;    // queries per CTA
+constexpr int PK = 64;    // keys per tile
+}
+
+template <typename T, int HD>
+__global__ void __launch_bounds__(256)
+attn_prefill_kernel(RowTable rt, const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
+                    int nq, int n_rep, int S, long long row_stride, T* __restrict__ out) {
+    extern __shared__ float sm[];
+    float* Qs = sm;                        // [PQ][HD+1]
+    float* Ks = Qs + PQ * (HD + 1);        // [PK][HD+1]
+    float* Vs = Ks + PK * (HD + 1);        // [PK][HD]
+    float* Ps = Vs + PK * HD;              // [PQ][PK+1]
+    const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int len = rt.cu[b + 1] - rt.cu[b];
+    const int t0 = qt * PQ;
+    if (t0 >= len) return;
+    const int nqt = min(PQ, len - t0);
+    const int g = h / n_rep;
+    const long long tok0 = rt.cu[b] + t0;
+    const int tid = threadIdx.x, qi = tid >> 2, sub = tid & 3;
+    constexpr int DPT = HD / 4;            // output dims per thread: sub, sub+4, sub+8, ...
+    const float scale = rsqrtf(static_cast<float>(HD));
+
+    for (int i = tid; i < PQ * HD; i += 256) {
+        const int r = i / HD, d = i % HD;
+        Qs[r * (HD + 1) + d] = r < nqt ? to_f32(q[(tok0 + r) * nq + h * HD + d]) * scale : 0.f;
+    }
+    const T* kb = kc + static_cast<long long>(b) * row_stride + static_cast<long long>(g) * S * HD;
+    const T* vb = vc + static_cast<long long>(b) * row_stride + static_cast<long long>(g) * S * HD;
+    const int my_pos = rt.start_pos + t0 + qi;       // absolute position of this thread's query
+    const int kend = rt.start_pos + t0 + nqt;        // keys [0, kend) are needed by the tile
+
+    float m_run = -INFINITY, l_run = 0.f;
+    float o[DPT];
+#pragma unroll
+    for (int e = 0; e < DPT; ++e) o[e] = 0.f;
+
+    for (int k0 = 0; k0 < kend; k0 += PK) {
+        __syncthreads();
+        const int nk = min(PK, kend - k0);
+        for (int i = tid; i < PK * HD; i += 256) {
+            const int r = i / HD, d = i % HD;
+            const bool in = r < nk;
+            Ks[r * (HD + 1) + d] = in ? to_f32(kb[static_cast<long long>(k0 + r) * HD + d]) : 0.f;
+            Vs[r * HD + d] = in ? to_f32(vb[static_cast<long long>(k0 + r) * HD + d]) : 0.f;
+        }
+        __syncthreads();
+        float sc[PK / 4];
+        float tmax = -INFINITY;
+#pragma unroll
+        for (int jj = 0; jj < PK / 4; ++jj) {
+            const int j = sub + 4 * jj;
+            float d = 0.f;
+#pragma unroll 8
+            for (int e = 0; e < HD; ++e) d = fmaf(Qs[qi * (HD + 1) + e], Ks[j * (HD + 1) + e], d);
+            const bool vis = (j < nk) && (k0 + j <= my_pos) && (qi < nqt);
+            sc[jj] = vis ? d : -INFINITY;
+            tmax = fmaxf(tmax, sc[jj]);
+        }
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+        const float mnew = fmaxf(m_run, tmax);
+        const float corr = (m_run == -INFINITY) ? 0.f : __expf(m_run - mnew);
+        float psum = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < PK / 4; ++jj) {
+            const float pj = (sc[jj] == -INFINITY) ? 0.f : __expf(sc[jj] - mnew);
+            Ps[qi * (PK + 1) + sub + 4 * jj] = pj;
+            psum += pj;
+        }
+        psum += __shfl_xor_sync(0xffffffffu, psum, 1);
+        psum += __shfl_xor_sync(0xffffffffu, psum, 2);
+        l_run = l_run * corr + psum;
+        m_run = mnew;
+        __syncwarp();
+#pragma unroll
+        for (int e = 0; e < DPT; ++e) o[e] *= corr;
+        for (int j = 0; j < nk; ++j) {
+            const float pj = Ps[qi * (PK + 1) + j];
+#pragma unroll
+            for (int e = 0; e < DPT; ++e) o[e] = fmaf(pj, Vs[j * HD + sub + 4 * e], o[e]);
+        }
+    }
+    if (qi < nqt) {
+        const float inv = 1.f / l_run;
+        T* dst = out + (tok0 + qi) * nq + h * HD + sub;
+#pragma unroll
+        for (int e = 0; e < DPT; ++e) dst[4 * e] = from_f32<T>(o[e] * inv);
+    }
+}
+
+template <typename T, int HD>
+static int prefill_go(const Model* m, int layer, const RowTable& rt, cudaStream_t st) {
+    const int smem = (PQ * (HD + 1) + PK * (HD + 1) + PK * HD + PQ * (PK + 1)) * 4;
+    auto kern = attn_prefill_kernel<T, HD>;
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_prefill_kernel)");
+        attr = true;
+    }
+    int maxlen = 0;
+    for (int b = 0; b < rt.B; ++b) maxlen = max(maxlen, rt.cu[b + 1] - rt.cu[b]);
+    dim3 grid((maxlen + PQ - 1) / PQ, m->nh, rt.B);
+    const T* kc = static_cast<const T*>(m->kc) + layer * m->kv_layer_elems;
+    const T* vc = static_cast<const T*>(m->vc) + layer * m->kv_layer_elems;
+    kern<<<grid, 256, smem, st>>>(rt, static_cast<const T*>(m->q), kc, vc, m->nq, m->n_rep, m->S,
+                                  m->kv_row_elems, static_cast<T*>(m->attn));
+    LLB_CHECK_LAUNCH("attn_prefill_kernel");
+    return LLAMA_OK;
+}
+
+template <typename T>
+static int prefill_hd(const Model* m, int layer, const RowTable& rt, cudaStream_t st) {
+    switch (m->hd) {
+        case 32: return prefill_go<T, 32>(m, layer, rt, st);
+        case 64: return prefill_go<T, 64>(m, layer, rt, st);
+        case 128: return prefill_go<T, 128>(m, layer, rt, st);
+    }
+    set_error("head_dim %d unsupported", m->hd);
+    return LLAMA_ERR_INVALID_ARG;
+}
+
+int launch_attention_prefill(const Model* m, int layer, const RowTable& rt, cudaStream_t st) {
+    if (m->dtype == LLAMA_BF16) return prefill_hd<bf16>(m, layer, rt, st);
+    return prefill_hd<float>(m, layer, rt, st);
+}
+
+}  // namespace llb

@@ -1,0 +1,130 @@
+// Host-side model description and the internal launchers shared by the
+// C-ABI implementation (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <vector>
+
+#include "../../include/llama_b200.h"
+
+namespace llb {
+
+constexpr int kMaxRows = 256;         // max_batch_size limit (by-value row tables)
+constexpr int kKvChunk = 256;         // keys per split in decode attention
+
+// Token -> (batch row, position) map of one prefill call, passed by value.
+struct RowTable {
+    int B, T, start_pos;
+    int cu[kMaxRows + 1];    // packed token offsets of each row
+};
+
+// Epilogue of a projection: what happens to acc[m, n] = sum_k A[m,k] W[n,k].
+enum EpiMode { EPI_STORE_F32 = 0, EPI_RESID_F32 = 1, EPI_QKV = 2, EPI_SWIGLU = 3 };
+
+struct Epi {
+    int mode;
+    // STORE_F32: out[m*ldo + n] = acc.  RESID_F32: out[m*ldo + n] += acc.
+    float* out;
+    int ldo;
+    // QKV: columns [0, nq) -> q[m*nq + n] (RoPE), [nq, nq+nkvc) -> K cache (RoPE),
+    // [nq+nkvc, nq+2*nkvc) -> V cache; token m sits in batch row tok_row[m]
+    // (identity when NULL) at position tok_pos[m].
+    void* q;
+    void* kc;
+    void* vc;
+    const int* tok_row;
+    const int* tok_pos;
+    int nq, nkvc, hd, max_seq;
+    long long kv_row_stride;   // elements between batch rows of one layer's cache
+    const float2* rope;        // [max_seq][hd/2] (cos, sin)
+    // SWIGLU: interleaved columns (64 w1 rows, then the same 64 w3 rows, ...)
+    // -> g[m*H + h] = silu(w1) * w3.
+    void* g;
+    int H;
+    int* status;
+};
+
+struct TmaMaps {               // tensor maps of one K-major bf16 matrix
+    CUtensorMap a128;          // box 64 x 128 rows (the MMA's A operand)
+    CUtensorMap b;             // box 64 x 256 rows (weights as B) or 64 x 16 (activations as B)
+};
+
+struct LayerPtrs {
+    float* attn_norm;
+    void* wqkv;
+    void* wo;
+    float* ffn_norm;
+    void* w13;   // interleaved in blocks of 64 rows: w1[0:64], w3[0:64], w1[64:128], ...
+    void* w2;
+    TmaMaps m_wqkv, m_wo, m_w13, m_w2;
+};
+
+struct Model {
+    llama_model_args a;
+    int dim, L, nh, nkv, hd, n_rep, H, V, S, Bmax, Mmax, dtype, esz;
+    int nq, nkvc, nqkv;
+    int n_splits;
+    // weights
+    void* tok_emb;
+    float* norm;
+    void* output;
+    TmaMaps m_output;
+    std::vector<LayerPtrs> layers;
+    // KV cache: [L][Bmax][nkv][S][hd]
+    void* kc;
+    void* vc;
+    long long kv_layer_elems, kv_row_elems, kv_head_elems;
+    float2* rope;
+    // workspace
+    float* x;        // [Mmax, dim] fp32 residual stream
+    void* y;         // [Mmax, dim] normed activations (model dtype)
+    void* q;         // [Mmax, nq]
+    void* attn;      // [Mmax, nq]
+    void* g;         // [Mmax, H]
+    void* ylast;     // [Bmax, dim] final-norm rows that get logits
+    int* tok_ids;    // [Mmax]
+    int* tok_row;    // [Mmax]
+    int* tok_pos;    // [Mmax]
+    int* last_idx;   // [Bmax]
+    float* logits_ws;   // [Bmax, V]
+    float* part_o;      // [Bmax*nh*n_splits, hd]
+    float* part_ml;     // [Bmax*nh*n_splits, 2]
+    int* status;
+    TmaMaps m_y, m_attn, m_g, m_ylast;   // activation maps (A box 128 rows, B box 16 rows)
+    cudaStream_t last_stream;
+};
+
+// ---------------------------------------------------------------- launchers (return LLAMA_* codes)
+int launch_rope_table(float2* rope, int S, int hd, float theta, cudaStream_t st);
+int launch_token_map(const RowTable& rt, const int32_t* tokens, int* tok_ids, int* tok_row,
+                     int* tok_pos, int* last_idx, cudaStream_t st);
+int launch_embed(const int* tok_ids, const void* emb, int dtype, int M, int dim, int V, float* x,
+                 int* status, cudaStream_t st);
+int launch_rmsnorm(const float* x, const int* row_idx, const float* w, int M, int dim, float eps,
+                   void* out, int out_dtype, cudaStream_t st);
+int launch_copy_interleave_w13(const void* src, void* w13, int H, int dim, int which, int esz,
+                               cudaStream_t st);
+
+// out = A W^T with epilogue `ep`.  A rows: M (tokens), W rows: N, K.
+// bf16 uses tcgen05 with the given maps (A-side/W-side), fp32 the SIMT kernel.
+int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, const void* W,
+               const TmaMaps* mapW, int M, int N, int K, const Epi& ep, cudaStream_t st);
+int linear_f32(const float* A, const float* W, int M, int N, int K, const Epi& ep, cudaStream_t st);
+int linear_bf16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep,
+                   cudaStream_t st);
+
+int launch_attention_prefill(const Model* m, int layer, const RowTable& rt, cudaStream_t st);
+int launch_attention_decode(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st);
+
+int launch_argmax(const float* logits, int B, int V, int32_t* out, int32_t* tokens_adv,
+                  int32_t* pos_adv, cudaStream_t st);
+int launch_top_p(const float* logits, int B, int V, float temperature, float top_p,
+                 const float* uniforms, int32_t* out, int32_t* tokens_adv, int32_t* pos_adv,
+                 cudaStream_t st);
+
+// TMA descriptor encoding (driver entry point resolved at run time).
+int encode_kmajor_bf16(CUtensorMap* map, const void* base, int rows, int cols, int box_rows);
+
+}  // namespace llb

@@ -1,0 +1,43 @@
+/*
+ * llama_b200_ops.h — single-kernel entry points of libllama_b200.so.
+ *
+ * Each call runs one of the kernels the model path uses, on caller device
+ * buffers, so that a kernel can be checked against the CPU oracle on its own
+ * and timed in isolation.  Conventions (device pointers, void* stream,
+ * LLAMA_OK / LLAMA_ERR_* return codes, llama_last_error) are those of
+ * llama_b200.h.
+ */
+#ifndef LLAMA_B200_OPS_H
+#define LLAMA_B200_OPS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "llama_b200.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* RMSNorm of M rows: out[m,:] = x[m,:] / sqrt(mean(x[m,:]^2) + eps) * w
+ * (Admin Guide §8.4, RMSNorm), fp32 arithmetic.
+ *   x fp32 [M, dim]; w fp32 [dim]; out [M, dim] in out_dtype (LLAMA_F32 or
+ *   LLAMA_BF16, rounded once).  dim % 4 == 0. */
+LLAMA_API int llama_op_rmsnorm(const float* x, const float* w, int M, int dim, float eps,
+                     void* out, int out_dtype, void* stream);
+
+/* Dense projection out[m,n] = sum_k A[m,k] * W[n,k]  (nn.Linear, y = x W^T).
+ *   A [M, K] and W [N, K] in `dtype` (LLAMA_F32: SIMT fp32 FMA, no TF32;
+ *   LLAMA_BF16: tcgen05 tensor cores with fp32 accumulation in TMEM);
+ *   out fp32 [M, N] (row-major, overwritten).  K % 8 == 0 for bf16.
+ * The bf16 kernel is the one the model path uses: for M <= 64 it runs with
+ * the weight as the 128-row MMA operand (decode shape), else with the
+ * activations as that operand (prefill shape). */
+LLAMA_API int llama_op_linear(const void* A, const void* W, int M, int N, int K, int dtype,
+                    float* out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLAMA_B200_OPS_H */

@@ -337,10 +337,15 @@ def top_p_kept(logits, temperature: float, top_p: float) -> List[int]:
 
 
 def sample_margins(logits, temperature: float, top_p: float, u: float) -> float:
-    """Distance (relative to the kept mass) of this draw from a decision
-    boundary of sample_top_p: the draw target from the cumulative masses, the
-    nucleus edge from top_p, and neighbouring probabilities from each other.
-    A float-rounding difference can change an index only when this is tiny.
+    """How far (relative to the kept mass) this draw sits from a decision
+    boundary of sample_top_p.  A float-rounding difference can change the
+    returned index only when this is tiny or negative.
+
+    Two boundaries matter: the cumulative masses the draw target u*Z is
+    compared with, and the nucleus edge.  A token whose preceding mass lies
+    within 1e-9 of top_p may be kept or dropped by rounding; that moves Z, and
+    so the draw target, by at most that token's own mass, which is subtracted
+    from the draw margin.  For temperature 0 it is the top-2 logit gap.
     """
     if temperature == 0:
         l = np.sort(_f64(logits))[::-1]
@@ -354,5 +359,8 @@ def sample_margins(logits, temperature: float, top_p: float, u: float) -> float:
     z = inclusive[kept - 1]
     target = np.float64(u) * z
     m = float(np.min(np.abs(inclusive[:kept] - target)) / z)
-    m = min(m, float(np.min(np.abs(exclusive - top_p))))
+    near = np.abs(exclusive - np.float64(top_p)) < 1e-9
+    near[0] = False   # the first token is always kept
+    if near.any():
+        m -= float(ps[near].sum() / z)
     return m

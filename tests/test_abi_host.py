@@ -1,0 +1,109 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every symbol the headers declare, sizes the arena as the Admin Guide's KV
+footprint fixes, and rejects bad arguments before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+llb = pytest.importorskip("decoder_only_transformer_llama_b200",
+                          reason="library not built (run decoder_only_transformer_llama_b200.build)")
+from oracle import llama_oracle as O  # noqa: E402
+from workloads import WORKLOADS  # noqa: E402
+
+
+def _declared_symbols():
+    names = set()
+    for h in ("llama_b200.h", "llama_b200_ops.h"):
+        with open(os.path.join(ROOT, "include", h)) as f:
+            names |= set(re.findall(r"LLAMA_API\s+[\w\s\*]+?\b(llama_\w+)\s*\(", f.read()))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared_symbols()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(llb.lib(), n), n
+    assert set(llb.EXPORTED) == names
+
+
+def test_struct_layout_matches_header():
+    # 13 four-byte fields, no padding
+    assert ctypes.sizeof(llb.ModelArgs) == 13 * 4
+    assert ctypes.sizeof(llb.Sampling) == 8
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_model_bytes_for_every_workload(name):
+    s = WORKLOADS[name]["shape"]
+    sz = llb.model_bytes(llb.args_from_shape(s))
+    assert sz["hidden"] == s.hidden == O.ffn_hidden_dim(s.dim, s.multiple_of, s.ffn_dim_multiplier)
+    esz = 2 if s.dtype == "bf16" else 4
+    per_tensor = O.kv_cache_bytes_per_tensor(s.max_batch_size, s.max_seq_len, s.n_kv_heads, s.head_dim, esz)
+    # the cache is two tensors per layer; each region is padded to 256 bytes at most once
+    assert 2 * s.n_layers * per_tensor <= sz["kv"] <= 2 * s.n_layers * per_tensor + 512
+    n_params = O.parameter_count(s.dim, s.n_layers, s.n_heads, s.n_kv_heads, s.vocab_size, s.hidden)
+    n_norm = (2 * s.n_layers + 1) * s.dim
+    expect = (n_params - n_norm) * esz + n_norm * 4
+    assert expect <= sz["weights"] <= expect + 256 * (8 * s.n_layers + 4)
+    assert sz["total"] == sz["weights"] + sz["kv"] + sz["workspace"]
+
+
+def test_kv_bytes_match_admin_guide_figure():
+    """7B, max_batch_size 4, max_seq_len 2048, 16-bit cache: 64 MiB per tensor per layer."""
+    a = llb.make_args(4096, 32, 32, 32, 32000, max_seq_len=2048, max_batch_size=4, max_tokens=16)
+    assert llb.model_bytes(a)["kv"] == 2 * 32 * 64 * 1024 * 1024
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dim=0), llb.LLAMA_ERR_INVALID_ARG),
+    (dict(n_heads=3), llb.LLAMA_ERR_INVALID_ARG),              # dim % n_heads
+    (dict(n_kv_heads=3), llb.LLAMA_ERR_INVALID_ARG),           # n_heads % n_kv_heads
+    (dict(dim=512, n_heads=2), llb.LLAMA_ERR_INVALID_ARG),     # head_dim 256 unsupported
+    (dict(max_batch_size=1000), llb.LLAMA_ERR_INVALID_ARG),
+    (dict(max_seq_len=0), llb.LLAMA_ERR_INVALID_ARG),
+    (dict(dtype="fp8"), None),
+])
+def test_model_bytes_rejects_bad_args(kw, code):
+    base = dict(dim=256, n_layers=2, n_heads=8, n_kv_heads=2, vocab_size=512, max_seq_len=128, max_batch_size=2,
+                dtype="f32")
+    base.update(kw)
+    a = llb.make_args(**base)
+    if kw.get("dtype") == "fp8":
+        a.dtype = 7
+        code = llb.LLAMA_ERR_INVALID_ARG
+    with pytest.raises(llb.LlamaError) as ei:
+        llb.model_bytes(a)
+    assert ei.value.code == code
+    assert llb.last_error()
+
+
+def test_create_rejects_null_and_small_arena_without_gpu():
+    a = llb.make_args(256, 2, 8, 2, 512, max_seq_len=128, max_batch_size=2, dtype="f32")
+    lib = llb.lib()
+    h = ctypes.c_void_p()
+    assert lib.llama_model_create(ctypes.byref(a), None, 1 << 30, None, ctypes.byref(h)) == llb.LLAMA_ERR_INVALID_ARG
+    # misaligned arena pointer is refused before any device access
+    assert lib.llama_model_create(ctypes.byref(a), 0x1001, 1 << 30, None, ctypes.byref(h)) == llb.LLAMA_ERR_INVALID_ARG
+    total = llb.model_bytes(a)["total"]
+    assert lib.llama_model_create(ctypes.byref(a), 0x100000, total - 1, None, ctypes.byref(h)) == llb.LLAMA_ERR_CAPACITY
+    assert h.value is None
+
+
+def test_calls_reject_null_model_and_bad_sizes():
+    lib = llb.lib()
+    assert lib.llama_prefill(None, 0x1000, None, 1, 1, 0, None, 0, None) == llb.LLAMA_ERR_INVALID_ARG
+    assert lib.llama_decode_step(None, 0x1000, 0x1000, 1, None, None, None, None, 0, None) == llb.LLAMA_ERR_INVALID_ARG
+    assert lib.llama_sample(None, 1, 10, 0.0, 0.9, None, 0x1000, None) == llb.LLAMA_ERR_INVALID_ARG
+    assert lib.llama_sample(0x1000, 0, 10, 0.0, 0.9, None, 0x1000, None) == llb.LLAMA_ERR_INVALID_ARG
+    assert lib.llama_sample(0x1000, 1, 10, 0.7, 0.9, None, 0x1000, None) == llb.LLAMA_ERR_INVALID_ARG  # no uniforms
+    assert lib.llama_sample(0x1000, 1, 10, -1.0, 0.9, 0x1000, 0x1000, None) == llb.LLAMA_ERR_INVALID_ARG
+    assert lib.llama_model_status(None, None) == llb.LLAMA_ERR_INVALID_ARG
+    assert lib.llama_op_linear(None, 0x1000, 1, 1, 8, 1, 0x1000, None) == llb.LLAMA_ERR_INVALID_ARG
+    assert lib.llama_op_linear(0x1000, 0x1000, 1, 1, 7, 1, 0x1000, None) == llb.LLAMA_ERR_INVALID_ARG  # K % 8
+    assert lib.llama_op_rmsnorm(0x1000, 0x1000, 1, 6, 1e-5, 0x1000, 0, None) == llb.LLAMA_ERR_INVALID_ARG
+    assert lib.llama_get_kv(None, 0, None, None, None) == llb.LLAMA_ERR_INVALID_ARG

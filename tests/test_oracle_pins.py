@@ -444,3 +444,17 @@ def test_top_p_random_draws_chi_square():
     stat = float(np.sum((counts[kept] - exp) ** 2 / exp))
     assert stat < chi2.ppf(0.999, len(kept) - 1)
     assert counts.sum() == counts[kept].sum()
+
+
+def test_sample_margins_flags_boundary_draws_only():
+    """A draw right at a cumulative boundary has margin ~0; a draw in the
+    middle of a bin has a margin of about half the bin's share."""
+    p = [0.5, 0.3, 0.15, 0.05]
+    l = np.log(np.array(p, dtype=np.float32))
+    assert O.sample_margins(l, 1.0, 1.0, 0.5) < 1e-6          # target 0.5 = C_0
+    assert abs(O.sample_margins(l, 1.0, 1.0, 0.25) - 0.25) < 1e-6
+    # tail tokens of negligible mass near top_p = 1 do not make a mid-bin draw ambiguous
+    l2 = np.concatenate([l, np.full(5, -60.0, dtype=np.float32)])
+    assert O.sample_margins(l2, 1.0, 1.0, 0.25) > 0.2
+    # but a draw that lands on such a token is flagged
+    assert O.sample_margins(l2, 1.0, 1.0, 0.9999999999999) < 1e-9
