@@ -1,0 +1,411 @@
+"""Benchmark of the Llama-2 7B-shaped forward pass on B200: prefill + greedy decode.
+
+One step = the whole hot path over one batch: prefill of 4 x 512 random token
+ids (all 32 layers, final norm, vocabulary projection, greedy pick of the
+first token), then 256 greedy decode steps (contexts 513 .. 768), all through
+the C ABI of libllama_b200.so.  Weights are random (seeded), bf16, with fp32
+norm weights; data is synthetic.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  `value` is decode tokens/s of the whole job;
+prefill tokens/s and both rooflines are extra keys.  With N > 1 (torchrun)
+every rank runs an independent replica of the workload (batch rows never
+interact, so there is nothing to exchange) and the job time is the max over
+ranks.  `--impl reference` times the CPU oracle on a bounded sample of the
+same workload on the host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from workloads import L7B, WORKLOADS, make_tokens, make_weights, token_seed, weight_seed  # noqa: E402
+
+WL = WORKLOADS["7b"]
+METRIC = "decode tok/s (% HBM peak) + prefill tok/s (% TC peak), 7B shape, 1 B200"
+UNIT = "tok/s"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int, path: str):
+        self.index, self.path, self.proc = index, path, None
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- roofline bookkeeping
+
+def launch_bytes(M, N, K, kind):
+    """Algorithmic bytes of one projection launch: the bf16 weight matrix once,
+    the bf16 input rows once, and the epilogue's output traffic."""
+    out = {0: 4 * M * N, 1: 8 * M * N, 2: 2 * M * N, 3: M * N}[kind]
+    return 2 * N * K + 2 * M * K + out
+
+
+def launch_flops(M, N, K, kind):
+    return 2 * M * N * K
+
+
+def decode_step_bytes(s, B, ctx):
+    """Algorithmic bytes of one decode step of B rows at context ctx: every
+    weight matrix once (bf16), the norm weights (fp32), B embedding rows, the
+    K and V cache read over ctx positions and written at one, and the fp32
+    logits."""
+    hd, nkv, L = s.head_dim, s.n_kv_heads, s.n_layers
+    mats = L * (s.dim * (s.n_heads + 2 * nkv) * hd + s.dim * s.n_heads * hd + 3 * s.dim * s.hidden)
+    mats += s.vocab_size * s.dim
+    return (2 * mats + 4 * s.dim * (2 * L + 1) + 2 * B * s.dim
+            + L * 2 * nkv * hd * 2 * ctx * B + L * 2 * nkv * hd * 2 * B + 4 * B * s.vocab_size)
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(a, rank, world, local_rank):
+    import decoder_only_transformer_llama_b200 as llb
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    hbm, tc_burst, tc_sust, peak_src = _peaks()
+    s = L7B
+    B, T, steps_dec = WL["batch"], WL["prompt_len"], WL["decode_steps"]
+    w = make_weights(s, weight_seed(WL["index"]), device=dev)
+    model = llb.Model(llb.args_from_shape(s), device=dev)
+    model.load(w)
+    del w
+    torch.cuda.empty_cache()
+
+    stream = torch.cuda.current_stream()
+    prompt = make_tokens(s.vocab_size, (B, T), token_seed(WL["index"])).to(dev)
+    prompt_host = prompt.cpu().pin_memory()
+    prompt_dev = torch.empty_like(prompt)
+    logits = torch.empty(B, s.vocab_size, device=dev)
+    tok = torch.empty(B, dtype=torch.int32, device=dev)
+    pos = torch.empty(B, dtype=torch.int32, device=dev)
+    pos_init = torch.full((B,), T, dtype=torch.int32, device=dev)
+    tok_host = torch.empty(B, dtype=torch.int32).pin_memory()
+
+    def one_step():
+        model.prefill(prompt, logits=logits)
+        llb.sample(logits, 0.0, 0.9, None, tok)
+        pos.copy_(pos_init)
+        for _ in range(steps_dec):
+            model.decode_step(tok, pos, temperature=0.0, next_tokens=tok, advance=True)
+
+    def one_step_timed(ev):
+        ev[0].record(stream)
+        model.prefill(prompt, logits=logits)
+        llb.sample(logits, 0.0, 0.9, None, tok)
+        pos.copy_(pos_init)
+        ev[1].record(stream)
+        for _ in range(steps_dec):
+            model.decode_step(tok, pos, temperature=0.0, next_tokens=tok, advance=True)
+        ev[2].record(stream)
+
+    for _ in range(a.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    assert model.status() == 0
+
+    # launches per step (exact count of this library's kernels)
+    c0 = llb.launch_count()
+    one_step()
+    torch.cuda.synchronize()
+    launches_per_step = llb.launch_count() - c0
+
+    # ---------------- timed region
+    per_step_proj = (5 * s.n_layers + 1) * (steps_dec + 1)
+    model.profile_start(per_step_proj * a.steps + 16)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(a.steps)]
+    import tempfile
+    clocks = ClockSampler(local_rank, os.path.join(tempfile.gettempdir(), f"llama_b200_clocks_rank{rank}.csv"))
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    c0 = llb.launch_count()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(a.steps):
+        one_step_timed(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    launches = llb.launch_count() - c0
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    prefill_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    decode_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    recs = model.profile_stop(per_step_proj * a.steps + 16)
+    assert model.status() == 0
+
+    # ---------------- end to end through host buffers
+    e2e_ev0 = torch.cuda.Event(enable_timing=True)
+    e2e_ev1 = torch.cuda.Event(enable_timing=True)
+    e2e_dec_ms = 0.0
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_e2e0 = time.perf_counter()
+    for i in range(a.steps):
+        prompt_dev.copy_(prompt_host, non_blocking=True)
+        model.prefill(prompt_dev, logits=logits)
+        llb.sample(logits, 0.0, 0.9, None, tok)
+        tok_host.copy_(tok, non_blocking=True)
+        pos.copy_(pos_init)
+        e2e_ev0.record(stream)
+        stream.synchronize()
+        for _ in range(steps_dec):
+            model.decode_step(tok, pos, temperature=0.0, next_tokens=tok, advance=True)
+            tok_host.copy_(tok, non_blocking=True)
+            stream.synchronize()     # the host reads every generated token, like a serving loop
+        e2e_ev1.record(stream)
+        torch.cuda.synchronize()
+        e2e_dec_ms += e2e_ev0.elapsed_time(e2e_ev1)
+    t_e2e = time.perf_counter() - t_e2e0
+
+    # ---------------- max over ranks
+    vals = torch.tensor([total_ms, prefill_ms, decode_ms, e2e_dec_ms, t_e2e * 1e3], device=dev, dtype=torch.float64)
+    if world > 1:
+        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
+    total_ms, prefill_ms, decode_ms, e2e_dec_ms, e2e_wall_ms = vals.tolist()
+
+    dec_tokens = world * a.steps * B * steps_dec
+    pre_tokens = world * a.steps * B * T
+    value = dec_tokens / (decode_ms / 1e3)
+    prefill_tps = pre_tokens / (prefill_ms / 1e3)
+    e2e_value = dec_tokens / (e2e_dec_ms / 1e3)
+
+    dec = [r for r in recs if r[1] > 0 and r[0] > 0 and r[1] <= 64]
+    pre = [r for r in recs if r[0] > 0 and r[1] > 64]
+    dec_bytes = sum(launch_bytes(M, N, K, k) for _, M, N, K, k in dec)
+    dec_ms = sum(r[0] for r in dec)
+    pre_flops = sum(launch_flops(M, N, K, k) for _, M, N, K, k in pre)
+    pre_ms_k = sum(r[0] for r in pre)
+    dec_gbs = dec_bytes / (dec_ms / 1e3) / 1e9 if dec_ms else 0.0
+    pre_tfs = pre_flops / (pre_ms_k / 1e3) / 1e12 if pre_ms_k else 0.0
+
+    step_bytes = sum(decode_step_bytes(s, B, T + 1 + i) for i in range(steps_dec))
+    decode_gbs_path = step_bytes * world * a.steps / (decode_ms / 1e3) / 1e9
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": a.steps,
+        "warmup": a.warmup,
+        "ms_per_step": round(total_ms / a.steps, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded random token ids, random-init bf16 weights, fp32 norm weights)",
+        "config": {"workload": "7b: Llama-2-7B shape, 32 layers, dim 4096, 32 heads (MHA), hidden 11008, "
+                               "vocab 32000, max_seq_len 4096; prefill 4x512 then 256 greedy decode steps",
+                   "global_batch": B * world, "seq_len": T, "decode_steps": steps_dec,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2: each decode step streams 13.5 GB of weights (L2 126 MB)"},
+        "prefill_tok_s": round(prefill_tps, 1),
+        "decode_ms_per_token_step": round(decode_ms / (a.steps * steps_dec), 4),
+        "prefill_ms": round(prefill_ms / a.steps, 3),
+        "roofline": {"bound": "hbm", "kernel": "linear_tc_kernel (decode orientation: wqkv/wo/w13/w2/output)",
+                     "achieved": round(dec_gbs, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(dec_gbs / hbm, 4), "peak_source": f"{peak_src} hbm_gbs",
+                     "traffic": None, "launches": len(dec)},
+        "roofline_prefill": {"bound": "tensor", "kernel": "linear_tc_kernel (prefill orientation)",
+                             "achieved": round(pre_tfs, 1), "peak": tc_burst, "unit": "TFLOP/s",
+                             "frac": round(pre_tfs / tc_burst, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
+                             "traffic": None, "launches": len(pre)},
+        "decode_path_hbm": {"achieved": round(decode_gbs_path, 1), "unit": "GB/s",
+                            "frac": round(decode_gbs_path / hbm, 4),
+                            "what": "all algorithmic bytes of a decode step (weights, KV read+write, logits) / decode time"},
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": B * T * 4,
+                "d2h_bytes_per_step": B * 4 * (steps_dec + 1),
+                "what": "prompt copied from pinned host memory each step; every generated token read back to the "
+                        "host and synchronised on, as a serving loop does"},
+        "gpu_launches": int(launches),
+        "launches_per_step": int(launches_per_step),
+        "clocks": clk,
+        "impl": "ours",
+    }
+    return line
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) sample
+
+def oracle_sample(seconds: float = 12.0):
+    """Times the oracle on a bounded sample of the 7B workload: decode of one
+    token of one row at context 640 through `nl` layers (as many as fit the
+    time budget, at least 1) plus the final norm, vocabulary projection and
+    sampling, extrapolated to the 32-layer model.  Returns (tok_s, sample, cores)."""
+    import numpy as np
+    from oracle import llama_oracle as O
+    from workloads import LazyF64Weights, make_normal
+
+    try:
+        from threadpoolctl import threadpool_info
+    except Exception:  # pragma: no cover
+        threadpool_info = lambda: []  # noqa: E731
+    s = L7B
+    nl = 2
+    w = make_weights(s.replace(n_layers=nl), 4242, device="cpu")
+    args = O.Args(dim=s.dim, n_layers=nl, n_heads=s.n_heads, n_kv_heads=s.n_kv_heads, vocab_size=s.vocab_size,
+                  max_seq_len=1024)
+    lw = LazyF64Weights(w)
+    ctx = 640
+    cache = O.new_cache(args)
+    for l in range(nl):
+        cache.k[l][:ctx] = make_normal((ctx, s.n_kv_heads, s.head_dim), 7 + l, dtype=torch.float32).double().numpy()
+        cache.v[l][:ctx] = make_normal((ctx, s.n_kv_heads, s.head_dim), 9 + l, dtype=torch.float32).double().numpy()
+    x = np.asarray(lw["tok_embeddings"][np.array([123])], dtype=np.float64)
+    t0 = time.perf_counter()
+    layers_done = 0
+    while True:
+        for l in range(nl):
+            x = O.layer_forward(args, lw["layers"][l], x, cache, l, ctx)
+            layers_done += 1
+        if time.perf_counter() - t0 > seconds / 2 or layers_done >= 8:
+            break
+    t_layer = (time.perf_counter() - t0) / layers_done
+    t1 = time.perf_counter()
+    h = O.rms_norm(x, lw["norm"], args.norm_eps)
+    logits = h @ np.asarray(lw["output"], dtype=np.float64).T
+    O.greedy(logits[0])
+    t_head = time.perf_counter() - t1
+    t_tok = t_layer * s.n_layers + t_head
+    cores = 0
+    for info in threadpool_info():
+        cores = max(cores, int(info.get("num_threads", 0)))
+    cores = cores or (len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count())
+    sample = (f"oracle (numpy fp64) decode of 1 token of 1 row at context {ctx}: {layers_done} 7B-shaped layer "
+              f"passes timed ({t_layer * 1e3:.0f} ms each) plus final norm + 32000x4096 vocabulary projection + "
+              f"argmax ({t_head * 1e3:.0f} ms), extrapolated to 32 layers")
+    return 1.0 / t_tok, sample, cores
+
+
+def run_reference(a, rank, world):
+    if rank != 0:
+        return None
+    vals = []
+    sample = cores = None
+    for i in range(a.warmup + a.steps):
+        v, sample, cores = oracle_sample(seconds=6.0)
+        if i >= a.warmup:
+            vals.append(v)
+    value = statistics.mean(vals)
+    return {"metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": round(1e3 / value, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "7b: Llama-2-7B shape; oracle sample (see cpu_baseline.sample)",
+                       "global_batch": 1, "seq_len": 640, "parallelism": "host cores"},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+    if a.warmup < 3:
+        a.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if a.impl == "reference":
+        line = run_reference(a, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        line = run_ours(a, rank, world, local_rank)
+        if rank == 0 and world == 1 and not a.no_cpu_baseline:
+            v, sample, cores = oracle_sample()
+            line["cpu_baseline"] = {"value": round(v, 5), "unit": UNIT, "cores": cores, "kind": "oracle",
+                                    "sample": sample}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

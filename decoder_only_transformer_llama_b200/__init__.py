@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libllama_b200.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
-                      "`python -m decoder_only_transformer_llama_b200.build`")
+                      "`python decoder_only_transformer_llama_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -37,7 +37,7 @@ WEIGHT_IDS = {"tok_embeddings": 0, "norm": 1, "output": 2, "attention_norm": 3, 
 EXPORTED = ("llama_model_bytes", "llama_model_create", "llama_set_weight", "llama_get_kv",
             "llama_prefill", "llama_decode_step", "llama_sample", "llama_model_status",
             "llama_model_destroy", "llama_last_error", "llama_launch_count",
-            "llama_op_rmsnorm", "llama_op_linear")
+            "llama_op_rmsnorm", "llama_op_linear", "llama_profile_start", "llama_profile_stop")
 
 
 class LlamaError(RuntimeError):
@@ -86,6 +86,9 @@ _sig("llama_last_error", ctypes.c_char_p, [])
 _sig("llama_launch_count", ctypes.c_uint64, [])
 _sig("llama_op_rmsnorm", _i, [_vp, _vp, _i, _i, _f, _vp, _i, _vp])
 _sig("llama_op_linear", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp])
+_sig("llama_profile_start", _i, [_vp, _i])
+_sig("llama_profile_stop", _i, [_vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32), _i,
+                                ctypes.POINTER(ctypes.c_int)])
 
 
 def lib():
@@ -227,6 +230,17 @@ class Model:
                                       _ptr(next_tokens), _ptr(logits),
                                       LLAMA_DECODE_ADVANCE if advance else 0, _stream(stream)))
         return next_tokens
+
+    def profile_start(self, capacity: int):
+        _check(_lib.llama_profile_start(self.handle, capacity))
+
+    def profile_stop(self, max_records: int):
+        """[(ms, M, N, K, kind)] of the projection launches timed since profile_start."""
+        ms = (ctypes.c_float * max_records)()
+        sh = (ctypes.c_int32 * (4 * max_records))()
+        n = ctypes.c_int()
+        _check(_lib.llama_profile_stop(self.handle, ms, sh, max_records, ctypes.byref(n)))
+        return [(ms[i], sh[4 * i], sh[4 * i + 1], sh[4 * i + 2], sh[4 * i + 3]) for i in range(n.value)]
 
     def status(self) -> int:
         s = ctypes.c_int()

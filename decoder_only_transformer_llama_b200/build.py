@@ -1,6 +1,6 @@
 """Builds libllama_b200.so in place (sm_100a only) with nvcc.
 
-    python -m decoder_only_transformer_llama_b200.build [--force] [-j N]
+    python decoder_only_transformer_llama_b200/build.py [--force] [-j N] [--ptxas-v]
 
 Each csrc/*.cu file compiles to an object under _build/, then one nvcc link
 produces the shared library next to this file.  A file is recompiled only

@@ -138,10 +138,34 @@ static int make_maps(TmaMaps* t, const void* base, int rows, int cols, int b_box
 
 int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, const void* W,
                const TmaMaps* mapW, int M, int N, int K, const Epi& ep, cudaStream_t st) {
+    Profile* pr = const_cast<Profile*>(&m->prof);
+    const bool timed = pr->n < pr->capacity;
+    if (timed) {
+        cudaError_t e = cudaEventRecord(pr->ev[2 * pr->n], st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord(profile)");
+    }
+    int rc;
     if (dtype == LLAMA_F32)
-        return linear_f32(static_cast<const float*>(A), static_cast<const float*>(W), M, N, K, ep, st);
-    (void)m;
-    return linear_bf16_tc(mapA, mapW, M, N, K, ep, st);
+        rc = linear_f32(static_cast<const float*>(A), static_cast<const float*>(W), M, N, K, ep, st);
+    else
+        rc = linear_bf16_tc(mapA, mapW, M, N, K, ep, st);
+    if (timed && rc == LLAMA_OK) {
+        cudaError_t e = cudaEventRecord(pr->ev[2 * pr->n + 1], st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord(profile)");
+        const int kind = ep.mode == EPI_STORE_F32 ? 0 : ep.mode == EPI_RESID_F32 ? 1 : ep.mode == EPI_QKV ? 2 : 3;
+        int32_t* sh = &pr->shapes[4 * pr->n];
+        sh[0] = M; sh[1] = N; sh[2] = K; sh[3] = kind;
+        pr->n++;
+    }
+    return rc;
+}
+
+static void profile_release(Profile& p) {
+    for (cudaEvent_t e : p.ev) cudaEventDestroy(e);
+    p.ev.clear();
+    p.shapes.clear();
+    p.capacity = 0;
+    p.n = 0;
 }
 
 static Epi base_epi(const Model* m) {
@@ -449,8 +473,44 @@ int llama_model_status(llama_model* m, int* device_status) {
 }
 
 int llama_model_destroy(llama_model* m) {
+    if (m) profile_release(m->prof);
     delete m;
     return LLAMA_OK;
+}
+
+int llama_profile_start(llama_model* m, int capacity) {
+    if (!m || capacity <= 0) { set_error("bad profile arguments"); return LLAMA_ERR_INVALID_ARG; }
+    profile_release(m->prof);
+    m->prof.ev.resize(2 * static_cast<size_t>(capacity), nullptr);
+    for (auto& e : m->prof.ev) {
+        cudaError_t ce = cudaEventCreate(&e);
+        if (ce != cudaSuccess) {
+            profile_release(m->prof);
+            return cuda_fail(ce, "cudaEventCreate(profile)");
+        }
+    }
+    m->prof.shapes.assign(4 * static_cast<size_t>(capacity), 0);
+    m->prof.capacity = capacity;
+    m->prof.n = 0;
+    return LLAMA_OK;
+}
+
+int llama_profile_stop(llama_model* m, float* ms, int32_t* shapes, int max, int* n) {
+    if (!m) { set_error("model is NULL"); return LLAMA_ERR_INVALID_ARG; }
+    Profile& p = m->prof;
+    const int cnt = p.n < max ? p.n : max;
+    int rc = LLAMA_OK;
+    for (int i = 0; i < cnt && rc == LLAMA_OK; ++i) {
+        cudaError_t e = cudaEventSynchronize(p.ev[2 * i + 1]);
+        float t = 0.f;
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&t, p.ev[2 * i], p.ev[2 * i + 1]);
+        if (e != cudaSuccess) rc = cuda_fail(e, "profile events");
+        if (ms) ms[i] = t;
+        if (shapes) for (int k = 0; k < 4; ++k) shapes[4 * i + k] = p.shapes[4 * i + k];
+    }
+    if (n) *n = cnt;
+    profile_release(p);
+    return rc;
 }
 
 // ---------------------------------------------------------------- single-kernel ops

@@ -61,6 +61,13 @@ struct LayerPtrs {
     TmaMaps m_wqkv, m_wo, m_w13, m_w2;
 };
 
+struct Profile {
+    int capacity = 0;
+    int n = 0;
+    std::vector<cudaEvent_t> ev;     // 2 per launch
+    std::vector<int32_t> shapes;     // 4 per launch
+};
+
 struct Model {
     llama_model_args a;
     int dim, L, nh, nkv, hd, n_rep, H, V, S, Bmax, Mmax, dtype, esz;
@@ -94,6 +101,7 @@ struct Model {
     int* status;
     TmaMaps m_y, m_attn, m_g, m_ylast;   // activation maps (A box 128 rows, B box 16 rows)
     cudaStream_t last_stream;
+    Profile prof;
 };
 
 // ---------------------------------------------------------------- launchers (return LLAMA_* codes)

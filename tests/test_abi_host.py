@@ -10,7 +10,7 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 llb = pytest.importorskip("decoder_only_transformer_llama_b200",
-                          reason="library not built (run decoder_only_transformer_llama_b200.build)")
+                          reason="library not built (run decoder_only_transformer_llama_b200/build.py)")
 from oracle import llama_oracle as O  # noqa: E402
 from workloads import WORKLOADS  # noqa: E402
 
