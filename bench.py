@@ -176,8 +176,12 @@ def run_ours(a, rank, world, local_rank):
     launches_per_step = llb.launch_count() - c0
 
     # ---------------- timed region
-    per_step_proj = (5 * s.n_layers + 1) * (steps_dec + 1)
-    model.profile_start(per_step_proj * a.steps + 16)
+    # Projection launches are bracketed by timing events only in the first
+    # bench step's prefill and first PROF_DECODE decode steps: events between
+    # every launch would slow the whole region down.
+    PROF_DECODE = 16
+    prof_cap = (5 * s.n_layers + 1) * (1 + PROF_DECODE)
+    model.profile_start(prof_cap)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(a.steps)]
     import tempfile
     clocks = ClockSampler(local_rank, os.path.join(tempfile.gettempdir(), f"llama_b200_clocks_rank{rank}.csv"))
@@ -198,7 +202,7 @@ def run_ours(a, rank, world, local_rank):
     total_ms = t_start.elapsed_time(t_end)
     prefill_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
     decode_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
-    recs = model.profile_stop(per_step_proj * a.steps + 16)
+    recs = model.profile_stop(prof_cap)
     assert model.status() == 0
 
     # ---------------- end to end through host buffers

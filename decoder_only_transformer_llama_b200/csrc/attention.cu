@@ -9,8 +9,9 @@
 // of the group, keeps an online softmax per head, and writes an unnormalised
 // partial (o, max, sum); a combine kernel merges the splits per (b, h).
 //
-// Prefill: one CTA per (64-query tile, head, row), online softmax over 64-key
-// tiles staged in shared memory (fp32 CUDA-core arithmetic).
+// Prefill of fp32 models: one CTA per (64-query tile, head, row), online
+// softmax over 64-key tiles staged in shared memory (fp32 CUDA-core
+// arithmetic).  bf16 models use the tensor-core kernel of attention_prefill_tc.cu.
 #include "common.cuh"
 #include "model.h"
 
@@ -345,7 +346,8 @@ static int prefill_hd(const Model* m, int layer, const RowTable& rt, cudaStream_
 }
 
 int launch_attention_prefill(const Model* m, int layer, const RowTable& rt, cudaStream_t st) {
-    if (m->dtype == LLAMA_BF16) return prefill_hd<bf16>(m, layer, rt, st);
+    // bf16 models run the tensor-core kernel; fp32 models the CUDA-core one (no TF32)
+    if (m->dtype == LLAMA_BF16) return launch_attention_prefill_tc(m, layer, rt, st);
     return prefill_hd<float>(m, layer, rt, st);
 }
 

@@ -124,6 +124,7 @@ int linear_bf16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K
                    cudaStream_t st);
 
 int launch_attention_prefill(const Model* m, int layer, const RowTable& rt, cudaStream_t st);
+int launch_attention_prefill_tc(const Model* m, int layer, const RowTable& rt, cudaStream_t st);
 int launch_attention_decode(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st);
 
 int launch_argmax(const float* logits, int B, int V, int32_t* out, int32_t* tokens_adv,
