@@ -147,31 +147,61 @@ def run_ours(a, rank, world, local_rank):
     pos_init = torch.full((B,), T, dtype=torch.int32, device=dev)
     tok_host = torch.empty(B, dtype=torch.int32).pin_memory()
 
+    graph = None
+
+    def decode_once():
+        if graph is not None:
+            graph.replay()
+        else:
+            model.decode_step(tok, pos, temperature=0.0, next_tokens=tok, advance=True)
+
     def one_step():
         model.prefill(prompt, logits=logits)
         llb.sample(logits, 0.0, 0.9, None, tok)
         pos.copy_(pos_init)
         for _ in range(steps_dec):
-            model.decode_step(tok, pos, temperature=0.0, next_tokens=tok, advance=True)
+            decode_once()
 
-    def one_step_timed(ev):
+    def one_step_timed(ev, prof_steps=0):
         ev[0].record(stream)
         model.prefill(prompt, logits=logits)
         llb.sample(logits, 0.0, 0.9, None, tok)
         pos.copy_(pos_init)
         ev[1].record(stream)
-        for _ in range(steps_dec):
-            model.decode_step(tok, pos, temperature=0.0, next_tokens=tok, advance=True)
+        for i in range(steps_dec):
+            if i < prof_steps:   # launched directly so that the timing events see every projection
+                model.decode_step(tok, pos, temperature=0.0, next_tokens=tok, advance=True)
+            else:
+                decode_once()
         ev[2].record(stream)
 
     for _ in range(a.warmup):
         one_step()
     torch.cuda.synchronize()
     assert model.status() == 0
+    if not a.no_graph:
+        # one decode step (tokens and positions advance on the device) as a CUDA graph
+        s_cap = torch.cuda.Stream(device=dev)
+        s_cap.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s_cap):
+            with torch.cuda.graph(graph, stream=s_cap):
+                model.decode_step(tok, pos, temperature=0.0, next_tokens=tok, advance=True)
+        stream.wait_stream(s_cap)
+        torch.cuda.synchronize()
+        for _ in range(2):
+            one_step()
+        torch.cuda.synchronize()
+        assert model.status() == 0
 
-    # launches per step (exact count of this library's kernels)
+    # launches per bench step (exact count of this library's kernels, counted
+    # on a step launched without the graph)
     c0 = llb.launch_count()
-    one_step()
+    model.prefill(prompt, logits=logits)
+    llb.sample(logits, 0.0, 0.9, None, tok)
+    pos.copy_(pos_init)
+    for _ in range(steps_dec):
+        model.decode_step(tok, pos, temperature=0.0, next_tokens=tok, advance=True)
     torch.cuda.synchronize()
     launches_per_step = llb.launch_count() - c0
 
@@ -189,15 +219,14 @@ def run_ours(a, rank, world, local_rank):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     clocks.start()
-    c0 = llb.launch_count()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for i in range(a.steps):
-        one_step_timed(evs[i])
+        one_step_timed(evs[i], PROF_DECODE if i == 0 else 0)
     t_end.record(stream)
     torch.cuda.synchronize()
-    launches = llb.launch_count() - c0
+    launches = launches_per_step * a.steps
     clk = clocks.stop()
     total_ms = t_start.elapsed_time(t_end)
     prefill_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
@@ -292,6 +321,7 @@ def run_ours(a, rank, world, local_rank):
                         "host and synchronised on, as a serving loop does"},
         "gpu_launches": int(launches),
         "launches_per_step": int(launches_per_step),
+        "decode_graph": graph is not None,
         "clocks": clk,
         "impl": "ours",
     }
@@ -371,6 +401,41 @@ def run_reference(a, rank, world):
             "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# ----------------------------------------------------------------------------- single projection
+
+def run_op_linear(a):
+    """Times one bf16 projection (llama_op_linear) back to back: M token rows
+    against an N x K weight, rotating over enough weight copies that the
+    working set exceeds L2.  Prints a JSON line with GB/s and TFLOP/s."""
+    import decoder_only_transformer_llama_b200 as llb
+    M, N, K = (int(v) for v in a.op_linear.split(","))
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    hbm, tc_burst, _, peak_src = _peaks()
+    wbytes = 2 * N * K
+    copies = max(1, -(-3 * 126 * 2 ** 20 // wbytes))
+    g = torch.Generator(device=dev).manual_seed(1)
+    Ws = [(torch.randn(N, K, generator=g, device=dev) * 0.02).to(torch.bfloat16) for _ in range(copies)]
+    A = torch.randn(M, K, generator=g, device=dev).to(torch.bfloat16)
+    out = torch.empty(M, N, device=dev)
+    for i in range(3):
+        llb.op_linear(A, Ws[i % copies], out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(a.iters):
+        llb.op_linear(A, Ws[i % copies], out)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / a.iters
+    byts = wbytes + 2 * M * K + 4 * M * N
+    print(json.dumps({"op": "linear_bf16", "M": M, "N": N, "K": K, "us": round(ms * 1e3, 2),
+                      "GB_s": round(byts / ms / 1e6, 1), "hbm_frac": round(byts / ms / 1e6 / hbm, 4),
+                      "TFLOP_s": round(2 * M * N * K / ms / 1e9, 1),
+                      "tc_frac": round(2 * M * N * K / ms / 1e9 / tc_burst, 4), "weight_copies": copies,
+                      "peak_source": peak_src}), flush=True)
+
+
 # ----------------------------------------------------------------------------- main
 
 def main():
@@ -380,7 +445,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op-linear", default=None, metavar="M,N,K",
+                    help="time one bf16 projection instead of the model (kernel microbenchmark)")
+    ap.add_argument("--iters", type=int, default=50)
+    ap.add_argument("--no-graph", action="store_true", help="launch decode steps directly instead of a CUDA graph")
     a = ap.parse_args()
+    if a.op_linear:
+        run_op_linear(a)
+        return
     if a.warmup < 3:
         a.warmup = 3
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -1,6 +1,7 @@
 // C ABI of libllama_b200.so: argument validation, the arena layout, and the
 // order of kernels in prefill and decode (Admin Guide §8.4, "The forward
 // pass"; §8.5 for the sampling step).  All arithmetic happens in the kernels.
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -51,7 +52,8 @@ struct Layout {
     size_t off_layers, weight_bytes;
     size_t off_kc, off_vc, kv_bytes;
     size_t off_x, off_y, off_q, off_attn, off_g, off_ylast, off_tok_ids, off_tok_row, off_tok_pos, off_last,
-        off_logits, off_part_o, off_part_ml, off_status, off_rope, ws_end;
+        off_logits, off_part_o, off_part_ml, off_attn_cnt, off_status, off_rope, off_gemm_part, off_gemm_cnt,
+        off_ssq, ws_end;
 };
 
 static int make_layout(const llama_model_args* a, Layout* o) {
@@ -74,8 +76,13 @@ static int make_layout(const llama_model_args* a, Layout* o) {
     if (a->max_batch_size > kMaxRows) { set_error("max_batch_size > %d", kMaxRows); return LLAMA_ERR_INVALID_ARG; }
     const int H = hidden_dim(a->dim, a->multiple_of, a->ffn_dim_multiplier);
     if (H % 64) { set_error("FFN hidden %d must be a multiple of 64", H); return LLAMA_ERR_INVALID_ARG; }
-    if (a->dtype == LLAMA_BF16 && (a->dim < 256 || a->vocab_size < 256)) {
-        set_error("bf16 models need dim >= 256 and vocab_size >= 256");
+    {
+        const long long widest = std::max(std::max(static_cast<long long>(a->vocab_size), 2LL * H),
+                                          static_cast<long long>(a->dim) + 2LL * nkv * (a->dim / a->n_heads) + a->dim);
+        if ((widest + 127) / 128 > kMaxTiles) { set_error("a projection is wider than %d x 128 rows", kMaxTiles); return LLAMA_ERR_INVALID_ARG; }
+    }
+    if (a->dtype == LLAMA_BF16 && (a->dim < 256 || a->vocab_size < 256 || a->dim % 128)) {
+        set_error("bf16 models need dim >= 256 (a multiple of 128) and vocab_size >= 256");
         return LLAMA_ERR_INVALID_ARG;
     }
     Layout& l = *o;
@@ -88,7 +95,7 @@ static int make_layout(const llama_model_args* a, Layout* o) {
     l.Mrows = l.Mmax < 128 ? 128 : l.Mmax;    // activation buffers hold whole 128-row tiles
     l.Brows = l.Bmax < 128 ? 128 : l.Bmax;
     l.nq = l.nh * hd; l.nkvc = nkv * hd; l.nqkv = l.nq + 2 * l.nkvc;
-    l.n_splits = (l.S + kKvChunk - 1) / kKvChunk;
+    l.n_splits = (l.S + kChunk - 1) / kChunk;
     const size_t e = l.esz, D = l.dim;
     size_t off = 0;
     l.off_tok_emb = off; off = align256(off + static_cast<size_t>(l.V) * D * e);
@@ -124,8 +131,12 @@ static int make_layout(const llama_model_args* a, Layout* o) {
     const size_t slots = static_cast<size_t>(l.Bmax) * l.nh * l.n_splits;
     l.off_part_o = off; off = align256(off + slots * hd * 4);
     l.off_part_ml = off; off = align256(off + slots * 2 * 4);
+    l.off_attn_cnt = off; off = align256(off + static_cast<size_t>(l.Bmax) * nkv * 4);
     l.off_status = off; off = align256(off + 16);
     l.off_rope = off; off = align256(off + static_cast<size_t>(l.S) * (hd / 2) * 8);
+    l.off_gemm_part = off; off = align256(off + (a->dtype == LLAMA_BF16 ? kDecodePartBytes : 0));
+    l.off_gemm_cnt = off; off = align256(off + kMaxTiles * sizeof(int));
+    l.off_ssq = off; off = align256(off + static_cast<size_t>(l.Bmax) * (l.dim / 128 + 1) * 4);
     l.ws_end = off;
     return LLAMA_OK;
 }
@@ -137,7 +148,8 @@ static int make_maps(TmaMaps* t, const void* base, int rows, int cols, int b_box
 }
 
 int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, const void* W,
-               const TmaMaps* mapW, int M, int N, int K, const Epi& ep, cudaStream_t st) {
+               const TmaMaps* mapW, int M, int N, int K, const Epi& ep, cudaStream_t st, bool pdl,
+               const NormIO* nio) {
     Profile* pr = const_cast<Profile*>(&m->prof);
     const bool timed = pr->n < pr->capacity;
     if (timed) {
@@ -148,7 +160,7 @@ int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, co
     if (dtype == LLAMA_F32)
         rc = linear_f32(static_cast<const float*>(A), static_cast<const float*>(W), M, N, K, ep, st);
     else
-        rc = linear_bf16_tc(mapA, mapW, M, N, K, ep, st);
+        rc = linear_bf16(mapA, mapW, M, N, K, ep, m->gemm_part, m->gemm_cnt, st, pdl && !timed, nio);
     if (timed && rc == LLAMA_OK) {
         cudaError_t e = cudaEventRecord(pr->ev[2 * pr->n + 1], st);
         if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord(profile)");
@@ -188,10 +200,10 @@ static char* at(void* base, size_t off) { return static_cast<char*>(base) + off;
 // TransformerBlock: h = x + attn(norm(x)); out = h + ffn(norm(h))).
 template <typename AttnFn>
 static int block_forward(Model* m, int l, int M, const int* tok_row, const int* tok_pos, AttnFn attn,
-                         cudaStream_t st) {
+                         cudaStream_t st, bool pdl) {
     LayerPtrs& Lp = m->layers[l];
     const size_t esz = m->esz;
-    LLB_TRY(launch_rmsnorm(m->x, nullptr, Lp.attn_norm, M, m->dim, m->a.norm_eps, m->y, m->dtype, st));
+    LLB_TRY(launch_rmsnorm(m->x, nullptr, Lp.attn_norm, M, m->dim, m->a.norm_eps, m->y, m->dtype, st, pdl));
     Epi ep = base_epi(m);
     ep.mode = EPI_QKV;
     ep.q = m->q;
@@ -199,19 +211,19 @@ static int block_forward(Model* m, int l, int M, const int* tok_row, const int* 
     ep.vc = static_cast<char*>(m->vc) + l * m->kv_layer_elems * esz;
     ep.tok_row = tok_row;
     ep.tok_pos = tok_pos;
-    LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.wqkv, &Lp.m_wqkv, M, m->nqkv, m->dim, ep, st));
+    LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.wqkv, &Lp.m_wqkv, M, m->nqkv, m->dim, ep, st, pdl));
     LLB_TRY(attn());
     Epi er = base_epi(m);
     er.mode = EPI_RESID_F32;
     er.out = m->x;
     er.ldo = m->dim;
-    LLB_TRY(run_linear(m, m->dtype, m->attn, &m->m_attn, Lp.wo, &Lp.m_wo, M, m->dim, m->nq, er, st));
-    LLB_TRY(launch_rmsnorm(m->x, nullptr, Lp.ffn_norm, M, m->dim, m->a.norm_eps, m->y, m->dtype, st));
+    LLB_TRY(run_linear(m, m->dtype, m->attn, &m->m_attn, Lp.wo, &Lp.m_wo, M, m->dim, m->nq, er, st, pdl));
+    LLB_TRY(launch_rmsnorm(m->x, nullptr, Lp.ffn_norm, M, m->dim, m->a.norm_eps, m->y, m->dtype, st, pdl));
     Epi es = base_epi(m);
     es.mode = EPI_SWIGLU;
     es.g = m->g;
-    LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.w13, &Lp.m_w13, M, 2 * m->H, m->dim, es, st));
-    LLB_TRY(run_linear(m, m->dtype, m->g, &m->m_g, Lp.w2, &Lp.m_w2, M, m->dim, m->H, er, st));
+    LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.w13, &Lp.m_w13, M, 2 * m->H, m->dim, es, st, pdl));
+    LLB_TRY(run_linear(m, m->dtype, m->g, &m->m_g, Lp.w2, &Lp.m_w2, M, m->dim, m->H, er, st, pdl));
     return LLAMA_OK;
 }
 
@@ -289,8 +301,12 @@ int llama_model_create(const llama_model_args* args, void* dev_arena, size_t are
     m->logits_ws = reinterpret_cast<float*>(at(A, l.off_logits));
     m->part_o = reinterpret_cast<float*>(at(A, l.off_part_o));
     m->part_ml = reinterpret_cast<float*>(at(A, l.off_part_ml));
+    m->attn_cnt = reinterpret_cast<int*>(at(A, l.off_attn_cnt));
     m->status = reinterpret_cast<int*>(at(A, l.off_status));
     m->rope = reinterpret_cast<float2*>(at(A, l.off_rope));
+    m->gemm_part = reinterpret_cast<float*>(at(A, l.off_gemm_part));
+    m->gemm_cnt = reinterpret_cast<int*>(at(A, l.off_gemm_cnt));
+    m->ssq = reinterpret_cast<float*>(at(A, l.off_ssq));
     m->last_stream = static_cast<cudaStream_t>(stream);
 
     int rc = LLAMA_OK;
@@ -312,6 +328,8 @@ int llama_model_create(const llama_model_args* args, void* dev_arena, size_t are
     if (rc == LLAMA_OK) {
         cudaError_t e = cudaMemsetAsync(m->kc, 0, l.kv_bytes, st);
         if (e == cudaSuccess) e = cudaMemsetAsync(m->status, 0, 16, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(m->gemm_cnt, 0, kMaxTiles * sizeof(int), st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(m->attn_cnt, 0, static_cast<size_t>(l.Bmax) * l.nkv * 4, st);
         if (e != cudaSuccess) rc = cuda_fail(e, "cudaMemsetAsync");
     }
     if (rc == LLAMA_OK) rc = launch_rope_table(m->rope, l.S, l.hd, args->rope_theta, st);
@@ -403,7 +421,7 @@ int llama_prefill(llama_model* m, const int32_t* tokens, const int32_t* lens, in
     LLB_TRY(launch_embed(m->tok_ids, m->tok_emb, m->dtype, M, m->dim, m->V, m->x, m->status, st));
     for (int l = 0; l < m->L; ++l) {
         auto attn = [&]() { return launch_attention_prefill(m, l, rt, st); };
-        LLB_TRY(block_forward(m, l, M, m->tok_row, m->tok_pos, attn, st));
+        LLB_TRY(block_forward(m, l, M, m->tok_row, m->tok_pos, attn, st, false));
     }
     if (!logits) return LLAMA_OK;
     Epi eo = base_epi(m);
@@ -430,25 +448,70 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     m->last_stream = st;
 
-    LLB_TRY(launch_embed(tokens, m->tok_emb, m->dtype, B, m->dim, m->V, m->x, m->status, st));
-    for (int l = 0; l < m->L; ++l) {
-        auto attn = [&]() { return launch_attention_decode(m, l, pos, B, st); };
-        LLB_TRY(block_forward(m, l, B, nullptr, pos, attn, st));
-    }
-    LLB_TRY(launch_rmsnorm(m->x, nullptr, m->norm, B, m->dim, m->a.norm_eps, m->ylast, m->dtype, st));
     float* lg = logits ? logits : m->logits_ws;
     Epi eo = base_epi(m);
     eo.mode = EPI_STORE_F32;
     eo.out = lg;
     eo.ldo = m->V;
-    LLB_TRY(run_linear(m, m->dtype, m->ylast, &m->m_ylast, m->output, &m->m_output, B, m->V, m->dim, eo, st));
+    if (m->dtype == LLAMA_BF16) {
+        // The decode chain: five kernels per layer.  Every kernel may launch
+        // before its predecessor ends (programmatic dependent launch) and waits
+        // for it before reading its outputs.  RMSNorm runs inside the
+        // projections that consume it; the residual epilogues and the
+        // embedding leave per-block sums of squares for it in m->ssq.
+        const int nb = m->dim / 128;
+        const float eps = m->a.norm_eps;
+        LLB_TRY(launch_embed(tokens, m->tok_emb, m->dtype, B, m->dim, m->V, m->x, m->status, st, true, m->ssq, m->y,
+                             m->layers[0].attn_norm));
+        for (int l = 0; l < m->L; ++l) {
+            LayerPtrs& Lp = m->layers[l];
+            const float* next_norm = l + 1 < m->L ? m->layers[l + 1].attn_norm : m->norm;
+            Epi ep = base_epi(m);
+            ep.mode = EPI_QKV;
+            ep.q = m->q;
+            ep.kc = static_cast<char*>(m->kc) + l * m->kv_layer_elems * m->esz;
+            ep.vc = static_cast<char*>(m->vc) + l * m->kv_layer_elems * m->esz;
+            ep.tok_pos = pos;
+            const NormIO n_in = {m->ssq, nb, eps, nullptr, nullptr, nullptr};
+            LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.wqkv, &Lp.m_wqkv, B, m->nqkv, m->dim, ep, st, true,
+                               &n_in));
+            LLB_TRY(launch_attention_decode(m, l, pos, B, st, true));
+            Epi er = base_epi(m);
+            er.mode = EPI_RESID_F32;
+            er.out = m->x;
+            er.ldo = m->dim;
+            const NormIO n_to_ffn = {nullptr, 0, 0.f, m->ssq, m->y, Lp.ffn_norm};
+            LLB_TRY(run_linear(m, m->dtype, m->attn, &m->m_attn, Lp.wo, &Lp.m_wo, B, m->dim, m->nq, er, st, true,
+                               &n_to_ffn));
+            Epi es = base_epi(m);
+            es.mode = EPI_SWIGLU;
+            es.g = m->g;
+            LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.w13, &Lp.m_w13, B, 2 * m->H, m->dim, es, st, true,
+                               &n_in));
+            const NormIO n_to_next = {nullptr, 0, 0.f, m->ssq, m->y, next_norm};
+            LLB_TRY(run_linear(m, m->dtype, m->g, &m->m_g, Lp.w2, &Lp.m_w2, B, m->dim, m->H, er, st, true,
+                               &n_to_next));
+        }
+        const NormIO n_in = {m->ssq, nb, eps, nullptr, nullptr, nullptr};
+        LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, m->output, &m->m_output, B, m->V, m->dim, eo, st, true,
+                           &n_in));
+    } else {
+        LLB_TRY(launch_embed(tokens, m->tok_emb, m->dtype, B, m->dim, m->V, m->x, m->status, st));
+        for (int l = 0; l < m->L; ++l) {
+            auto attn = [&]() { return launch_attention_decode(m, l, pos, B, st); };
+            LLB_TRY(block_forward(m, l, B, nullptr, pos, attn, st, false));
+        }
+        LLB_TRY(launch_rmsnorm(m->x, nullptr, m->norm, B, m->dim, m->a.norm_eps, m->ylast, m->dtype, st));
+        LLB_TRY(run_linear(m, m->dtype, m->ylast, &m->m_ylast, m->output, &m->m_output, B, m->V, m->dim, eo, st));
+    }
     if (!sampling) return LLAMA_OK;
+    const bool pdl = m->dtype == LLAMA_BF16;
     const bool adv = (flags & LLAMA_DECODE_ADVANCE) != 0;
     int32_t* tok_adv = adv ? const_cast<int32_t*>(tokens) : nullptr;
     int32_t* pos_adv = adv ? pos : nullptr;
-    if (sampling->temperature == 0.f) return launch_argmax(lg, B, m->V, next_tokens, tok_adv, pos_adv, st);
+    if (sampling->temperature == 0.f) return launch_argmax(lg, B, m->V, next_tokens, tok_adv, pos_adv, st, pdl);
     return launch_top_p(lg, B, m->V, sampling->temperature, sampling->top_p, uniforms, next_tokens, tok_adv,
-                        pos_adv, st);
+                        pos_adv, st, pdl);
 }
 
 int llama_sample(const float* logits, int B, int V, float temperature, float top_p, const float* uniforms,
@@ -521,7 +584,10 @@ int llama_op_rmsnorm(const float* x, const float* w, int M, int dim, float eps, 
     return launch_rmsnorm(x, nullptr, w, M, dim, eps, out, out_dtype, static_cast<cudaStream_t>(stream));
 }
 
-int llama_op_linear(const void* A, const void* W, int M, int N, int K, int dtype, float* out, void* stream) {
+size_t llama_op_linear_workspace_bytes(void) { return kDecodePartBytes + kMaxTiles * sizeof(int); }
+
+int llama_op_linear(const void* A, const void* W, int M, int N, int K, int dtype, float* out, void* workspace,
+                    size_t workspace_bytes, void* stream) {
     if (!A || !W || !out || M < 0 || N <= 0 || K <= 0) { set_error("bad linear arguments"); return LLAMA_ERR_INVALID_ARG; }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Epi ep;
@@ -533,13 +599,21 @@ int llama_op_linear(const void* A, const void* W, int M, int N, int K, int dtype
         return linear_f32(static_cast<const float*>(A), static_cast<const float*>(W), M, N, K, ep, st);
     if (dtype != LLAMA_BF16) { set_error("bad dtype"); return LLAMA_ERR_INVALID_ARG; }
     if (K % 8) { set_error("bf16 linear needs K %% 8 == 0"); return LLAMA_ERR_INVALID_ARG; }
+    if ((N + 127) / 128 > kMaxTiles) { set_error("N too large"); return LLAMA_ERR_INVALID_ARG; }
+    if (M <= 64 && (!workspace || workspace_bytes < llama_op_linear_workspace_bytes() ||
+                    (reinterpret_cast<uintptr_t>(workspace) & 255))) {
+        set_error("bf16 linear with M <= 64 needs a 256-byte aligned workspace of llama_op_linear_workspace_bytes()");
+        return LLAMA_ERR_INVALID_ARG;
+    }
     if (M == 0) return LLAMA_OK;
     TmaMaps ma, mw;
     LLB_TRY(encode_kmajor_bf16(&ma.a128, A, M, K, 128));
     LLB_TRY(encode_kmajor_bf16(&ma.b, A, M, K, 16));
     LLB_TRY(encode_kmajor_bf16(&mw.a128, W, N, K, 128));
     LLB_TRY(encode_kmajor_bf16(&mw.b, W, N, K, 256));
-    return linear_bf16_tc(&ma, &mw, M, N, K, ep, st);
+    float* part = static_cast<float*>(workspace);
+    int* cnt = workspace ? reinterpret_cast<int*>(static_cast<char*>(workspace) + kDecodePartBytes) : nullptr;
+    return linear_bf16(&ma, &mw, M, N, K, ep, part, cnt, st);
 }
 
 }  // extern "C"

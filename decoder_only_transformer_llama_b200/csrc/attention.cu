@@ -4,10 +4,8 @@
 //   keys j = 0 .. position of the query (the cached prefix plus the causal part
 //   of this call's tokens).  The -inf mask is realised as a key-range bound.
 //
-// Decode (one query per row): split-KV.  CTA (split s, kv head g, row b)
-// streams keys [s*chunk, (s+1)*chunk) of head g ONCE for all n_rep query heads
-// of the group, keeps an online softmax per head, and writes an unnormalised
-// partial (o, max, sum); a combine kernel merges the splits per (b, h).
+// Decode (one query per row): split-KV.  Each KV head is read once for its
+// whole query group; split partials are merged by the last split to finish.
 //
 // Prefill of fp32 models: one CTA per (64-query tile, head, row), online
 // softmax over 64-key tiles staged in shared memory (fp32 CUDA-core
@@ -46,12 +44,31 @@ template <> struct Vec<bf16, 4> {
 };
 
 // ---------------------------------------------------------------- decode
-template <typename T, int HD, int NREP, int UNROLL>
+// CTA (split s, kv head g, row b) handles keys [s*kChunk, (s+1)*kChunk) of
+// head g for all n_rep query heads of the group.  The chunk of K and the
+// chunk of V are each one contiguous block of the cache (positions of one
+// head are adjacent), fetched by two bulk async copies into shared memory.
+// Warp w scores keys w, w+4, ...; lane l holds head dims [l*EPL, l*EPL+EPL).
+// A row whose context fits one chunk writes its output directly; otherwise
+// every split publishes an unnormalised partial (o, max, sum) and the split
+// that arrives last at the (row, kv head) counter merges them in split order.
+template <typename T, int HD, int NREP>
 __global__ void __launch_bounds__(128)
 attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
-                   const int32_t* __restrict__ pos, int nq, int S, long long row_stride, int chunk,
-                   int n_splits, float* __restrict__ part_o, float* __restrict__ part_ml, int* status) {
+                   const int32_t* __restrict__ pos, int nq, int S, long long row_stride, int n_splits,
+                   float* __restrict__ part_o, float* __restrict__ part_ml, int* __restrict__ counters,
+                   T* __restrict__ out, int* status) {
     constexpr int EPL = HD / 32;   // head dims per lane
+    constexpr int ROW = HD * static_cast<int>(sizeof(T));
+    extern __shared__ __align__(128) uint8_t dsm[];
+    T* sK = reinterpret_cast<T*>(dsm);
+    T* sV = reinterpret_cast<T*>(dsm + kChunk * ROW);
+    __shared__ uint64_t bar;
+    __shared__ float s_m[4][NREP], s_l[4][NREP];
+    __shared__ float s_o[4][NREP][HD];
+    __shared__ int s_last;
+    pdl_trigger();
+    pdl_wait();
     const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int p = pos[b];
@@ -60,10 +77,18 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
         return;
     }
     const int ctx = p + 1;
-    const int j0 = s * chunk;
+    const int j0 = s * kChunk;
     if (j0 >= ctx) return;
-    const int j1 = min(ctx, j0 + chunk);
-
+    const int n = min(kChunk, ctx - j0);
+    const int nvalid = (ctx + kChunk - 1) / kChunk;
+    const long long head_off = static_cast<long long>(b) * row_stride + static_cast<long long>(g) * S * HD;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(&bar, 2u * n * ROW);
+        bulk_load(sK, kc + head_off + static_cast<long long>(j0) * HD, n * ROW, &bar);
+        bulk_load(sV, vc + head_off + static_cast<long long>(j0) * HD, n * ROW, &bar);
+    }
     const float scale = rsqrtf(static_cast<float>(HD));
     float qv[NREP][EPL];
 #pragma unroll
@@ -72,62 +97,53 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
 #pragma unroll
         for (int e = 0; e < EPL; ++e) qv[r][e] *= scale;
     }
-    const T* kb = kc + static_cast<long long>(b) * row_stride + static_cast<long long>(g) * S * HD + lane * EPL;
-    const T* vb = vc + static_cast<long long>(b) * row_stride + static_cast<long long>(g) * S * HD + lane * EPL;
+    __syncthreads();   // barrier initialised
+    const bool ok = mbar_wait(&bar, 0);
+    if (!ok && threadIdx.x == 0) report_status(status, LLAMA_ERR_DEVICE_TIMEOUT);
 
-    float mx[NREP], sm[NREP], o[NREP][EPL];
+    float mx[NREP], sl[NREP], o[NREP][EPL];
 #pragma unroll
     for (int r = 0; r < NREP; ++r) {
         mx[r] = -INFINITY;
-        sm[r] = 0.f;
+        sl[r] = 0.f;
 #pragma unroll
         for (int e = 0; e < EPL; ++e) o[r][e] = 0.f;
     }
-
-    // warp w takes keys j0 + w*UNROLL + 4*UNROLL*i + u
-    for (int jb = j0 + warp * UNROLL; jb < j1; jb += 4 * UNROLL) {
-        float kv[UNROLL][EPL], vv[UNROLL][EPL];
+    if (ok) {
+        for (int jb = warp * 2; jb < n; jb += 8) {
+            float kv[2][EPL], vv[2][EPL];
 #pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
-            const int j = min(jb + u, j1 - 1);
-            Vec<T, EPL>::load(kb + static_cast<long long>(j) * HD, kv[u]);
-            Vec<T, EPL>::load(vb + static_cast<long long>(j) * HD, vv[u]);
-        }
-#pragma unroll
-        for (int r = 0; r < NREP; ++r) {
-            float sc[UNROLL];
-#pragma unroll
-            for (int u = 0; u < UNROLL; ++u) {
-                float d = 0.f;
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) d = fmaf(qv[r][e], kv[u][e], d);
-                sc[u] = warp_sum(d);
-                if (jb + u >= j1) sc[u] = -INFINITY;
+            for (int u = 0; u < 2; ++u) {
+                const int j = min(jb + u, n - 1);
+                Vec<T, EPL>::load(sK + j * HD + lane * EPL, kv[u]);
+                Vec<T, EPL>::load(sV + j * HD + lane * EPL, vv[u]);
             }
-            float mnew = mx[r];
 #pragma unroll
-            for (int u = 0; u < UNROLL; ++u) mnew = fmaxf(mnew, sc[u]);
-            const float corr = __expf(mx[r] - mnew);
-            sm[r] *= corr;
+            for (int r = 0; r < NREP; ++r) {
+                float sc[2];
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) o[r][e] *= corr;
+                for (int u = 0; u < 2; ++u) {
+                    float d = 0.f;
 #pragma unroll
-            for (int u = 0; u < UNROLL; ++u) {
-                const float pj = __expf(sc[u] - mnew);
-                sm[r] += pj;
+                    for (int e = 0; e < EPL; ++e) d = fmaf(qv[r][e], kv[u][e], d);
+                    sc[u] = warp_sum(d);
+                }
+                if (jb + 1 >= n) sc[1] = -INFINITY;
+                const float mnew = fmaxf(mx[r], fmaxf(sc[0], sc[1]));
+                const float corr = __expf(mx[r] - mnew);
+                const float p0 = __expf(sc[0] - mnew), p1 = __expf(sc[1] - mnew);
+                sl[r] = sl[r] * corr + p0 + p1;
 #pragma unroll
-                for (int e = 0; e < EPL; ++e) o[r][e] = fmaf(pj, vv[u][e], o[r][e]);
+                for (int e = 0; e < EPL; ++e) o[r][e] = fmaf(p1, vv[1][e], fmaf(p0, vv[0][e], o[r][e] * corr));
+                mx[r] = mnew;
             }
-            mx[r] = mnew;
         }
     }
 
-    // merge the 4 warps
-    __shared__ float s_m[4][NREP], s_l[4][NREP];
-    __shared__ float s_o[4][NREP][HD];
+    // merge the 4 warps of this split
     if (lane == 0) {
 #pragma unroll
-        for (int r = 0; r < NREP; ++r) { s_m[warp][r] = mx[r]; s_l[warp][r] = sm[r]; }
+        for (int r = 0; r < NREP; ++r) { s_m[warp][r] = mx[r]; s_l[warp][r] = sl[r]; }
     }
 #pragma unroll
     for (int r = 0; r < NREP; ++r)
@@ -147,76 +163,90 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
             L += s_l[w][r] * f;
             acc += s_o[w][r][d] * f;
         }
-        const long long slot = (static_cast<long long>(b) * nh + g * NREP + r) * n_splits + s;
-        part_o[slot * HD + d] = acc;
-        if (d == 0) {
-            part_ml[slot * 2] = M;
-            part_ml[slot * 2 + 1] = L;
+        const int h = g * NREP + r;
+        if (nvalid == 1) {
+            out[static_cast<long long>(b) * nq + h * HD + d] = from_f32<T>(acc / L);
+        } else {
+            const long long slot = (static_cast<long long>(b) * nh + h) * n_splits + s;
+            part_o[slot * HD + d] = acc;
+            if (d == 0) {
+                part_ml[slot * 2] = M;
+                part_ml[slot * 2 + 1] = L;
+            }
         }
     }
-}
-
-template <typename T, int HD>
-__global__ void attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
-                                    const int32_t* __restrict__ pos, int nh, int S, int chunk, int n_splits,
-                                    T* __restrict__ out) {
-    const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
-    const int p = pos[b];
-    if (p < 0 || p >= S) return;
-    const int nvalid = (p + 1 + chunk - 1) / chunk;
-    const long long base = (static_cast<long long>(b) * nh + h) * n_splits;
-    float M = -INFINITY;
-    for (int s = 0; s < nvalid; ++s) M = fmaxf(M, part_ml[(base + s) * 2]);
-    float L = 0.f, acc = 0.f;
-    for (int s = 0; s < nvalid; ++s) {
-        const float f = __expf(part_ml[(base + s) * 2] - M);
-        L += part_ml[(base + s) * 2 + 1] * f;
-        acc += part_o[(base + s) * HD + d] * f;
+    if (nvalid == 1) return;
+    // publish the partial; the last split of (b, g) merges all of them
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(&counters[b * gridDim.y + g], 1) == nvalid - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int idx = threadIdx.x; idx < NREP * HD; idx += blockDim.x) {
+        const int r = idx / HD, d = idx % HD;
+        const int h = g * NREP + r;
+        const long long base = (static_cast<long long>(b) * nh + h) * n_splits;
+        float M = -INFINITY;
+        for (int t = 0; t < nvalid; ++t) M = fmaxf(M, part_ml[(base + t) * 2]);
+        float L = 0.f, acc = 0.f;
+        for (int t = 0; t < nvalid; ++t) {
+            const float f = __expf(part_ml[(base + t) * 2] - M);
+            L += part_ml[(base + t) * 2 + 1] * f;
+            acc += part_o[(base + t) * HD + d] * f;
+        }
+        out[static_cast<long long>(b) * nq + h * HD + d] = from_f32<T>(acc / L);
     }
-    out[static_cast<long long>(b) * nh * HD + h * HD + d] = from_f32<T>(acc / L);
+    if (threadIdx.x == 0) counters[b * gridDim.y + g] = 0;
 }
 
 template <typename T, int HD, int NREP>
-static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st) {
+static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl) {
     const T* kc = static_cast<const T*>(m->kc) + layer * m->kv_layer_elems;
     const T* vc = static_cast<const T*>(m->vc) + layer * m->kv_layer_elems;
+    auto kern = attn_decode_kernel<T, HD, NREP>;
+    const int smem = 2 * kChunk * HD * static_cast<int>(sizeof(T));
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_decode_kernel)");
+        attr = true;
+    }
     dim3 grid(m->n_splits, m->nkv, B);
-    attn_decode_kernel<T, HD, NREP, 4><<<grid, 128, 0, st>>>(
-        static_cast<const T*>(m->q), kc, vc, pos, m->nq, m->S, m->kv_row_elems, kKvChunk, m->n_splits,
-        m->part_o, m->part_ml, m->status);
-    LLB_CHECK_LAUNCH("attn_decode_kernel");
-    attn_combine_kernel<T, HD><<<dim3(m->nh, B), HD, 0, st>>>(m->part_o, m->part_ml, pos, m->nh, m->S,
-                                                              kKvChunk, m->n_splits, static_cast<T*>(m->attn));
-    LLB_CHECK_LAUNCH("attn_combine_kernel");
+    cudaError_t e = launch_k(kern, grid, dim3(128), smem, st, pdl, static_cast<const T*>(m->q), kc, vc, pos, m->nq,
+                             m->S, m->kv_row_elems, m->n_splits, m->part_o, m->part_ml, m->attn_cnt,
+                             static_cast<T*>(m->attn), m->status);
+    count_launch();
+    if (e != cudaSuccess) return cuda_fail(e, "attn_decode_kernel");
     return LLAMA_OK;
 }
 
 template <typename T, int HD>
-static int decode_rep(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st) {
+static int decode_rep(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl) {
     switch (m->n_rep) {
-        case 1: return decode_go<T, HD, 1>(m, layer, pos, B, st);
-        case 2: return decode_go<T, HD, 2>(m, layer, pos, B, st);
-        case 4: return decode_go<T, HD, 4>(m, layer, pos, B, st);
-        case 8: return decode_go<T, HD, 8>(m, layer, pos, B, st);
+        case 1: return decode_go<T, HD, 1>(m, layer, pos, B, st, pdl);
+        case 2: return decode_go<T, HD, 2>(m, layer, pos, B, st, pdl);
+        case 4: return decode_go<T, HD, 4>(m, layer, pos, B, st, pdl);
+        case 8: return decode_go<T, HD, 8>(m, layer, pos, B, st, pdl);
     }
     set_error("n_heads / n_kv_heads = %d unsupported (1, 2, 4, 8)", m->n_rep);
     return LLAMA_ERR_INVALID_ARG;
 }
 
 template <typename T>
-static int decode_hd(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st) {
+static int decode_hd(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl) {
     switch (m->hd) {
-        case 32: return decode_rep<T, 32>(m, layer, pos, B, st);
-        case 64: return decode_rep<T, 64>(m, layer, pos, B, st);
-        case 128: return decode_rep<T, 128>(m, layer, pos, B, st);
+        case 32: return decode_rep<T, 32>(m, layer, pos, B, st, pdl);
+        case 64: return decode_rep<T, 64>(m, layer, pos, B, st, pdl);
+        case 128: return decode_rep<T, 128>(m, layer, pos, B, st, pdl);
     }
     set_error("head_dim %d unsupported", m->hd);
     return LLAMA_ERR_INVALID_ARG;
 }
 
-int launch_attention_decode(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st) {
-    if (m->dtype == LLAMA_BF16) return decode_hd<bf16>(m, layer, pos, B, st);
-    return decode_hd<float>(m, layer, pos, B, st);
+int launch_attention_decode(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl) {
+    if (m->dtype == LLAMA_BF16) return decode_hd<bf16>(m, layer, pos, B, st, pdl);
+    return decode_hd<float>(m, layer, pos, B, st, pdl);
 }
 
 // ---------------------------------------------------------------- prefill

@@ -51,27 +51,63 @@ int launch_token_map(const RowTable& rt, const int32_t* tokens, int* tok_ids, in
 // ---------------------------------------------------------------- embedding
 // x[m, :] = E[tok[m], :] as fp32 (Admin Guide §8.4, tok_embeddings).  An id
 // outside [0, V) yields a zero row and sets LLAMA_ERR_TOKEN_RANGE.
+// With `ssq`, also writes the sum of x^2 over each 128-feature block of the
+// row (ssq[m * dim/128 + block]) and y[m, :] = bf16(x * w_next): the next
+// projection's fused RMSNorm inputs.
 template <typename T>
-__global__ void embed_kernel(const int* tok, const T* emb, int dim, int V, float* x, int* status) {
+__global__ void embed_kernel(const int* tok, const T* emb, int dim, int V, float* x, int* status, float* ssq,
+                             bf16* y, const float* w_next) {
+    pdl_trigger();
+    pdl_wait();
     const int m = blockIdx.x;
     const int id = tok[m];
     float* dst = x + static_cast<long long>(m) * dim;
     if (id < 0 || id >= V) {
         if (threadIdx.x == 0) report_status(status, LLAMA_ERR_TOKEN_RANGE);
         for (int i = threadIdx.x; i < dim; i += blockDim.x) dst[i] = 0.f;
+        if (ssq)
+            for (int i = threadIdx.x; i < dim / 128; i += blockDim.x) ssq[static_cast<long long>(m) * (dim / 128) + i] = 0.f;
         return;
     }
     const T* src = emb + static_cast<long long>(id) * dim;
     if constexpr (sizeof(T) == 2) {
         // 8 bf16 per 16-byte load
+        // blockDim.x is a multiple of 16, so the 16 vectors of one 128-feature
+        // block always sit in 16 adjacent lanes of one pass
         const uint4* s4 = reinterpret_cast<const uint4*>(src);
-        for (int i = threadIdx.x; i < dim / 8; i += blockDim.x) {
-            uint4 u = s4[i];
-            const bf16* h = reinterpret_cast<const bf16*>(&u);
-            float4 lo = make_float4(to_f32(h[0]), to_f32(h[1]), to_f32(h[2]), to_f32(h[3]));
-            float4 hi = make_float4(to_f32(h[4]), to_f32(h[5]), to_f32(h[6]), to_f32(h[7]));
-            reinterpret_cast<float4*>(dst)[2 * i] = lo;
-            reinterpret_cast<float4*>(dst)[2 * i + 1] = hi;
+        for (int base = 0; base < dim / 8; base += blockDim.x) {
+            const int i = base + threadIdx.x;
+            float sq = 0.f;
+            if (i < dim / 8) {
+                uint4 u = s4[i];
+                const bf16* h = reinterpret_cast<const bf16*>(&u);
+                float4 lo = make_float4(to_f32(h[0]), to_f32(h[1]), to_f32(h[2]), to_f32(h[3]));
+                float4 hi = make_float4(to_f32(h[4]), to_f32(h[5]), to_f32(h[6]), to_f32(h[7]));
+                reinterpret_cast<float4*>(dst)[2 * i] = lo;
+                reinterpret_cast<float4*>(dst)[2 * i + 1] = hi;
+                sq = lo.x * lo.x + lo.y * lo.y + lo.z * lo.z + lo.w * lo.w + hi.x * hi.x + hi.y * hi.y +
+                     hi.z * hi.z + hi.w * hi.w;
+                if (y) {
+                    const float4 w0 = reinterpret_cast<const float4*>(w_next)[2 * i];
+                    const float4 w1 = reinterpret_cast<const float4*>(w_next)[2 * i + 1];
+                    __nv_bfloat162 p0 = __floats2bfloat162_rn(lo.x * w0.x, lo.y * w0.y);
+                    __nv_bfloat162 p1 = __floats2bfloat162_rn(lo.z * w0.z, lo.w * w0.w);
+                    __nv_bfloat162 p2 = __floats2bfloat162_rn(hi.x * w1.x, hi.y * w1.y);
+                    __nv_bfloat162 p3 = __floats2bfloat162_rn(hi.z * w1.z, hi.w * w1.w);
+                    uint4 pk;
+                    pk.x = *reinterpret_cast<uint32_t*>(&p0);
+                    pk.y = *reinterpret_cast<uint32_t*>(&p1);
+                    pk.z = *reinterpret_cast<uint32_t*>(&p2);
+                    pk.w = *reinterpret_cast<uint32_t*>(&p3);
+                    reinterpret_cast<uint4*>(y + static_cast<long long>(m) * dim)[i] = pk;
+                }
+            }
+            if (ssq) {
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                if ((threadIdx.x & 15) == 0 && i < dim / 8)
+                    ssq[static_cast<long long>(m) * (dim / 128) + i / 16] = sq;
+            }
         }
     } else {
         const float4* s4 = reinterpret_cast<const float4*>(src);
@@ -81,13 +117,18 @@ __global__ void embed_kernel(const int* tok, const T* emb, int dim, int V, float
 }
 
 int launch_embed(const int* tok_ids, const void* emb, int dtype, int M, int dim, int V, float* x,
-                 int* status, cudaStream_t st) {
+                 int* status, cudaStream_t st, bool pdl, float* ssq, void* y, const float* w_next) {
     if (M <= 0) return LLAMA_OK;
+    cudaError_t e;
     if (dtype == LLAMA_BF16)
-        embed_kernel<bf16><<<M, 128, 0, st>>>(tok_ids, static_cast<const bf16*>(emb), dim, V, x, status);
+        e = launch_k(embed_kernel<bf16>, dim3(M), dim3(128), 0, st, pdl, tok_ids, static_cast<const bf16*>(emb),
+                     dim, V, x, status, ssq, static_cast<bf16*>(y), w_next);
     else
-        embed_kernel<float><<<M, 128, 0, st>>>(tok_ids, static_cast<const float*>(emb), dim, V, x, status);
-    LLB_CHECK_LAUNCH("embed_kernel");
+        e = launch_k(embed_kernel<float>, dim3(M), dim3(128), 0, st, pdl, tok_ids, static_cast<const float*>(emb),
+                     dim, V, x, status, static_cast<float*>(nullptr), static_cast<bf16*>(nullptr),
+                     static_cast<const float*>(nullptr));
+    count_launch();
+    if (e != cudaSuccess) return cuda_fail(e, "embed_kernel");
     return LLAMA_OK;
 }
 
@@ -98,6 +139,8 @@ int launch_embed(const int* tok_ids, const void* emb, int dtype, int M, int dim,
 template <typename TO, int kVecPerThread>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* x, const int* row_idx,
                                                       const float* w, int dim, float eps, TO* out) {
+    pdl_trigger();
+    pdl_wait();
     const int m = blockIdx.x;
     const int r = row_idx ? row_idx[m] : m;
     const float4* xr = reinterpret_cast<const float4*>(x + static_cast<long long>(r) * dim);
@@ -146,35 +189,38 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* x, const int*
 
 template <typename TO>
 static int rmsnorm_dispatch(const float* x, const int* row_idx, const float* w, int M, int dim,
-                            float eps, TO* out, cudaStream_t st) {
+                            float eps, TO* out, cudaStream_t st, bool pdl) {
     const int nv = dim / 4;
     const int threads = nv >= 256 ? 256 : ((nv + 31) / 32) * 32;
     const int per = (nv + threads - 1) / threads;
-    if (per <= 1)      rmsnorm_kernel<TO, 1><<<M, threads, 0, st>>>(x, row_idx, w, dim, eps, out);
-    else if (per <= 2) rmsnorm_kernel<TO, 2><<<M, threads, 0, st>>>(x, row_idx, w, dim, eps, out);
-    else if (per <= 4) rmsnorm_kernel<TO, 4><<<M, threads, 0, st>>>(x, row_idx, w, dim, eps, out);
-    else if (per <= 8) rmsnorm_kernel<TO, 8><<<M, threads, 0, st>>>(x, row_idx, w, dim, eps, out);
-    else if (per <= 16) rmsnorm_kernel<TO, 16><<<M, threads, 0, st>>>(x, row_idx, w, dim, eps, out);
+    cudaError_t e;
+    if (per <= 1)       e = launch_k(rmsnorm_kernel<TO, 1>, dim3(M), dim3(threads), 0, st, pdl, x, row_idx, w, dim, eps, out);
+    else if (per <= 2)  e = launch_k(rmsnorm_kernel<TO, 2>, dim3(M), dim3(threads), 0, st, pdl, x, row_idx, w, dim, eps, out);
+    else if (per <= 4)  e = launch_k(rmsnorm_kernel<TO, 4>, dim3(M), dim3(threads), 0, st, pdl, x, row_idx, w, dim, eps, out);
+    else if (per <= 8)  e = launch_k(rmsnorm_kernel<TO, 8>, dim3(M), dim3(threads), 0, st, pdl, x, row_idx, w, dim, eps, out);
+    else if (per <= 16) e = launch_k(rmsnorm_kernel<TO, 16>, dim3(M), dim3(threads), 0, st, pdl, x, row_idx, w, dim, eps, out);
     else { set_error("rmsnorm: dim %d too large", dim); return LLAMA_ERR_INVALID_ARG; }
-    LLB_CHECK_LAUNCH("rmsnorm_kernel");
+    count_launch();
+    if (e != cudaSuccess) return cuda_fail(e, "rmsnorm_kernel");
     return LLAMA_OK;
 }
 
 int launch_rmsnorm(const float* x, const int* row_idx, const float* w, int M, int dim, float eps,
-                   void* out, int out_dtype, cudaStream_t st) {
+                   void* out, int out_dtype, cudaStream_t st, bool pdl) {
     if (M <= 0) return LLAMA_OK;
     if (out_dtype == LLAMA_BF16)
-        return rmsnorm_dispatch<bf16>(x, row_idx, w, M, dim, eps, static_cast<bf16*>(out), st);
-    return rmsnorm_dispatch<float>(x, row_idx, w, M, dim, eps, static_cast<float*>(out), st);
+        return rmsnorm_dispatch<bf16>(x, row_idx, w, M, dim, eps, static_cast<bf16*>(out), st, pdl);
+    return rmsnorm_dispatch<float>(x, row_idx, w, M, dim, eps, static_cast<float*>(out), st, pdl);
 }
 
 // ---------------------------------------------------------------- w1/w3 interleave
 // Copies w1 (which=0) or w3 (which=1) [H, dim] into the fused w13 matrix,
-// whose rows are blocks of 64: block 2i holds w1 rows 64i..64i+63 and block
-// 2i+1 the same w3 rows.  One CTA per source row, 16-byte copies.
+// whose rows are blocks of 16: block 2i holds w1 rows 16i..16i+15 and block
+// 2i+1 the same w3 rows, so that a w1 row and its w3 row are 16 rows apart
+// inside every 32-row group.  One CTA per source row, 16-byte copies.
 __global__ void interleave_w13_kernel(const uint4* src, uint4* dst, int row_vecs, int which) {
     const int r = blockIdx.x;
-    const int drow = (r / 64) * 128 + which * 64 + (r % 64);
+    const int drow = (r / 16) * 32 + which * 16 + (r % 16);
     const uint4* s = src + static_cast<long long>(r) * row_vecs;
     uint4* d = dst + static_cast<long long>(drow) * row_vecs;
     for (int i = threadIdx.x; i < row_vecs; i += blockDim.x) d[i] = s[i];

@@ -2,9 +2,10 @@
 // fused epilogues.  acc[m, n] = sum_k A[m, k] * W[n, k]  (nn.Linear, y = x W^T).
 //
 // Tile 32 x 128, k-step 16, 256 threads.  Thread (ty, tx) owns rows
-// 4ty..4ty+3 and columns {2tx, 2tx+1, 64+2tx, 65+2tx}: the first two form a
-// RoPE pair, and column c with c+64 form a w1/w3 pair of the interleaved
-// SwiGLU weight, so every epilogue sees its operands in one thread.
+// 4ty..4ty+3 and columns {c0, c0+1, c0+16, c0+17}, c0 = 32*(tx/8) + 2*(tx%8):
+// the first two form a RoPE pair, and column c with c+16 form a w1/w3 pair of
+// the SwiGLU weight (interleaved in blocks of 16 rows), so every epilogue
+// sees its operands in one thread.
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "model.h"
@@ -23,7 +24,8 @@ __global__ void __launch_bounds__(256) linear_f32_kernel(const float* __restrict
     const int tid = threadIdx.x, tx = tid & 31, ty = tid >> 5;
     const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
     float acc[4][4] = {};
-    const int cols[4] = {2 * tx, 2 * tx + 1, 64 + 2 * tx, 65 + 2 * tx};
+    const int c0 = 32 * (tx >> 3) + 2 * (tx & 7);
+    const int cols[4] = {c0, c0 + 1, c0 + 16, c0 + 17};
 
     for (int k0 = 0; k0 < K; k0 += BK) {
         for (int i = tid; i < BM * BK; i += 256) {
@@ -61,7 +63,7 @@ __global__ void __launch_bounds__(256) linear_f32_kernel(const float* __restrict
             for (int e = 0; e < 2; ++e) {
                 const int n = n0 + cols[e];
                 if (n >= N) continue;
-                const int h = (n0 / 128) * 64 + cols[e];
+                const int h = ((n0 + cols[e]) / 32) * 16 + (cols[e] & 15);
                 static_cast<float*>(ep.g)[static_cast<long long>(m) * ep.H + h] =
                     silu_f(acc[i][e]) * acc[i][e + 2];
             }

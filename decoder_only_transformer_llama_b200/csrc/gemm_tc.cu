@@ -3,19 +3,17 @@
 // (Admin Guide §8.4: wq/wk/wv + RoPE + KV-cache append, wo + residual,
 // w1/w3 + silu*mul, w2 + residual, output projection).
 //
-// D[i, j] = sum_k A[i, k] * B[j, k]; A and B are K-major bf16 matrices read
-// through 128-byte-swizzled TMA boxes of 64 K-elements.  One CTA computes one
-// 128 x BN tile of D over its K range:
+// This file holds the prefill-shaped kernel (many token rows); decode-shaped
+// projections (<= 64 rows) run in gemm_decode.cu.
+//
+// D[i, j] = sum_k A[i, k] * B[j, k]; A = activations [tokens, K], B = weights
+// [N, K], both K-major bf16 read through 128-byte-swizzled TMA boxes of 64
+// K-elements.  One CTA computes one 128 x 256 tile of D:
 //   warp 0 lane 0  TMA producer (STAGES-deep ring of A/B tiles)
-//   warp 1 lane 0  MMA issuer (tcgen05.mma kind::f16, M=128, N=BN, K=16)
+//   warp 1 lane 0  MMA issuer (tcgen05.mma kind::f16, M=128, N=256, K=16)
 //   warp 1         TMEM allocation / release
-//   warps 0-3      epilogue: TMEM lane i (row i of the tile) -> thread i
-// Two orientations:
-//   prefill (SWAP=false): A = activations [tokens, K], B = weights [N, K],
-//       BN = 256; thread = token row, TMEM columns = output features.
-//   decode  (SWAP=true):  A = weights [N, K], B = activations [tokens, K],
-//       BN = 16..64 (tokens padded); thread = output feature, columns = tokens.
-//       The residual epilogue may split K over gridDim.z (fp32 atomics).
+//   warps 0-3      epilogue: TMEM lane i (token row i of the tile) -> thread i,
+//                  TMEM columns = output features
 // No TMA multicast is used.
 #include "common.cuh"
 #include "epilogue.cuh"
@@ -28,7 +26,6 @@ namespace llb {
 namespace {
 
 constexpr int kA_BYTES = 128 * 128;          // 128 rows x 64 bf16
-constexpr uint32_t kTmemColsMin = 32;
 
 template <int BN>
 struct TcCfg {
@@ -36,10 +33,6 @@ struct TcCfg {
     static constexpr int STAGE_BYTES = kA_BYTES + B_BYTES;
     static constexpr uint32_t TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
 };
-
-__device__ __forceinline__ void named_barrier_sync(int id, int n) {
-    asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(n) : "memory");
-}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
@@ -62,7 +55,7 @@ __device__ __forceinline__ void store32_bf16(bf16* dst, const float* v) {
 
 }  // namespace
 
-template <int BN, int STAGES, bool SWAP, int B_BOX>
+template <int BN, int STAGES, int B_BOX>
 __global__ void __launch_bounds__(128, 1)
 linear_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                  int rowsA, int rowsB, int K, int kt_per_split, Epi ep) {
@@ -145,26 +138,33 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
     if (!ok && threadIdx.x == 0) report_status(ep.status, LLAMA_ERR_DEVICE_TIMEOUT);
     const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
 
-    if constexpr (!SWAP) {
+    {
         // thread = token row m; TMEM columns = features n
         const int m = tileA * 128 + warp * 32 + lane;
         const bool row_ok = ok && m < rowsA;
         const int nbase = tileB * BN;
         if (ep.mode == EPI_SWIGLU) {
+            // each 32-column chunk holds 16 w1 outputs then the same 16 w3 outputs
 #pragma unroll 1
-            for (int grp = 0; grp < BN / 128; ++grp) {
-#pragma unroll 1
-                for (int half = 0; half < 2; ++half) {
-                    float a[32], b[32];
-                    tmem_ld_32x32b_x32(trow + grp * 128 + half * 32, a);
-                    tmem_ld_32x32b_x32(trow + grp * 128 + 64 + half * 32, b);
-                    tc_wait_ld();
-                    const int n = nbase + grp * 128;
-                    if (row_ok && n < rowsB) {
+            for (int c = 0; c < BN / 32; ++c) {
+                float v[32];
+                tmem_ld_32x32b_x32(trow + c * 32, v);
+                tc_wait_ld();
+                const int n0 = nbase + c * 32;
+                if (row_ok && n0 < rowsB) {
+                    float g16[16];
 #pragma unroll
-                        for (int t = 0; t < 32; ++t) a[t] = silu_f(a[t]) * b[t];
-                        const int h = (n / 128) * 64 + half * 32;
-                        store32_bf16(static_cast<bf16*>(ep.g) + static_cast<long long>(m) * ep.H + h, a);
+                    for (int t = 0; t < 16; ++t) g16[t] = silu_f(v[t]) * v[16 + t];
+                    bf16* dst = static_cast<bf16*>(ep.g) + static_cast<long long>(m) * ep.H + (n0 / 32) * 16;
+                    uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        uint4 u;
+                        u.x = pack_bf16x2(g16[8 * q + 0], g16[8 * q + 1]);
+                        u.y = pack_bf16x2(g16[8 * q + 2], g16[8 * q + 3]);
+                        u.z = pack_bf16x2(g16[8 * q + 4], g16[8 * q + 5]);
+                        u.w = pack_bf16x2(g16[8 * q + 6], g16[8 * q + 7]);
+                        d4[q] = u;
                     }
                 }
             }
@@ -222,76 +222,6 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
                 }
             }
         }
-    } else {
-        // thread = output feature n; TMEM columns = tokens b
-        const int n = tileA * 128 + warp * 32 + lane;
-        float v[BN];
-#pragma unroll
-        for (int c = 0; c < BN / 16; ++c) tmem_ld_32x32b_x16(trow + c * 16, v + c * 16);
-        tc_wait_ld();
-        const int nb = min(BN, rowsB);
-        const bool feat_ok = ok && n < rowsA;
-        if (ep.mode == EPI_SWIGLU) {
-            // tile rows 0-63 are w1 rows, 64-127 the matching w3 rows
-            float* xch = reinterpret_cast<float*>(smem);   // pipeline buffers are idle now
-            if (warp >= 2) {
-#pragma unroll
-                for (int b = 0; b < BN; ++b) xch[b * 64 + (warp - 2) * 32 + lane] = v[b];
-            }
-            named_barrier_sync(1, 128);
-            if (warp < 2 && ok) {
-                const int h = tileA * 64 + warp * 32 + lane;
-                if (h < ep.H) {
-#pragma unroll
-                    for (int b = 0; b < BN; ++b)
-                        if (b < nb)
-                            static_cast<bf16*>(ep.g)[static_cast<long long>(b) * ep.H + h] =
-                                __float2bfloat16_rn(silu_f(v[b]) * xch[b * 64 + warp * 32 + lane]);
-                }
-            }
-        } else if (ep.mode == EPI_QKV) {
-            const bool even = (lane & 1) == 0;
-#pragma unroll
-            for (int b = 0; b < BN; ++b) {
-                const float partner = __shfl_xor_sync(0xffffffffu, v[b], 1);
-                if (!feat_ok || b >= nb) continue;
-                const int pos = ep.tok_pos[b];
-                if (pos < 0 || pos >= ep.max_seq) continue;
-                float re = even ? v[b] : partner, im = even ? partner : v[b];
-                if (n < ep.nq) {
-                    rope_pair(ep.rope, ep.hd, pos, (n % ep.hd) >> 1, re, im);
-                    static_cast<bf16*>(ep.q)[static_cast<long long>(b) * ep.nq + n] =
-                        __float2bfloat16_rn(even ? re : im);
-                } else {
-                    int cc = n - ep.nq;
-                    bf16* cache = static_cast<bf16*>(ep.kc);
-                    const bool is_k = cc < ep.nkvc;
-                    if (!is_k) { cc -= ep.nkvc; cache = static_cast<bf16*>(ep.vc); }
-                    const int head = cc / ep.hd, d = cc % ep.hd;
-                    float val = v[b];
-                    if (is_k) {
-                        rope_pair(ep.rope, ep.hd, pos, d >> 1, re, im);
-                        val = even ? re : im;
-                    }
-                    const int row = ep.tok_row ? ep.tok_row[b] : b;
-                    cache[static_cast<long long>(row) * ep.kv_row_stride +
-                          (static_cast<long long>(head) * ep.max_seq + pos) * ep.hd + d] = __float2bfloat16_rn(val);
-                }
-            }
-        } else if (feat_ok) {
-            const bool atomic = gridDim.z > 1;
-#pragma unroll
-            for (int b = 0; b < BN; ++b) {
-                if (b >= nb) continue;
-                float* o = ep.out + static_cast<long long>(b) * ep.ldo + n;
-                if (ep.mode == EPI_RESID_F32) {
-                    if (atomic) atomicAdd(o, v[b]);
-                    else *o += v[b];
-                } else {
-                    *o = v[b];
-                }
-            }
-        }
     }
 
     tc_fence_before();
@@ -333,12 +263,12 @@ int encode_kmajor_bf16(CUtensorMap* map, const void* base, int rows, int cols, i
     return LLAMA_OK;
 }
 
-template <int BN, int STAGES, bool SWAP, int B_BOX>
+template <int BN, int STAGES, int B_BOX>
 static int launch_tc(const CUtensorMap& a, const CUtensorMap& b, int rowsA, int rowsB, int K, int splits,
                      const Epi& ep, cudaStream_t st) {
     using C = TcCfg<BN>;
     constexpr int smem = STAGES * C::STAGE_BYTES + 1024 + (2 * STAGES + 1) * 8 + 16;
-    auto kern = linear_tc_kernel<BN, STAGES, SWAP, B_BOX>;
+    auto kern = linear_tc_kernel<BN, STAGES, B_BOX>;
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -348,41 +278,23 @@ static int launch_tc(const CUtensorMap& a, const CUtensorMap& b, int rowsA, int 
     const int KT = (K + 63) / 64;
     const int per = (KT + splits - 1) / splits;
     const int z = (KT + per - 1) / per;   // every split gets >= 1 k-tile
-    dim3 grid((rowsA + 127) / 128, SWAP ? 1 : (rowsB + BN - 1) / BN, z);
+    dim3 grid((rowsA + 127) / 128, (rowsB + BN - 1) / BN, z);
     kern<<<grid, 128, smem, st>>>(a, b, rowsA, rowsB, K, per, ep);
     LLB_CHECK_LAUNCH("linear_tc_kernel");
     return LLAMA_OK;
 }
 
-static int g_num_sms = 0;
-
 int linear_bf16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep,
                    cudaStream_t st) {
     if (M <= 0 || N <= 0) return LLAMA_OK;
-    if (g_num_sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-        if (g_num_sms <= 0) g_num_sms = 148;
-    }
-    if (M <= 64) {
-        // decode orientation: weights are the 128-row operand, tokens the N side
-        const int tiles = (N + 127) / 128;
-        int splits = 1;
-        if (ep.mode == EPI_RESID_F32) {
-            const int slots = 2 * g_num_sms;   // two CTAs fit per SM
-            splits = slots / tiles;
-            const int KT = (K + 63) / 64;
-            if (splits > KT / 4) splits = KT / 4;
-            if (splits < 1) splits = 1;
-        }
-        if (M <= 16) return launch_tc<16, 4, true, 16>(mapW->a128, mapA->b, N, M, K, splits, ep, st);
-        if (M <= 32) return launch_tc<32, 4, true, 16>(mapW->a128, mapA->b, N, M, K, splits, ep, st);
-        if (M <= 48) return launch_tc<48, 4, true, 16>(mapW->a128, mapA->b, N, M, K, splits, ep, st);
-        return launch_tc<64, 4, true, 16>(mapW->a128, mapA->b, N, M, K, splits, ep, st);
-    }
-    // prefill orientation: tokens are the 128-row operand, 256 features per tile
-    return launch_tc<256, 4, false, 256>(mapA->a128, mapW->b, M, N, K, 1, ep, st);
+    return launch_tc<256, 4, 256>(mapA->a128, mapW->b, M, N, K, 1, ep, st);
+}
+
+int linear_bf16(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
+                int* counters, cudaStream_t st, bool pdl, const NormIO* nio) {
+    if (M <= 64) return linear_bf16_decode(mapA, mapW, M, N, K, ep, part, counters, st, pdl, nio);
+    if (nio && (nio->ssq_in || nio->ssq_out)) { set_error("fused RMSNorm is a decode-shape feature"); return LLAMA_ERR_INVALID_ARG; }
+    return linear_bf16_tc(mapA, mapW, M, N, K, ep, st);
 }
 
 }  // namespace llb

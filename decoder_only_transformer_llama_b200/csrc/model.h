@@ -12,7 +12,11 @@
 namespace llb {
 
 constexpr int kMaxRows = 256;         // max_batch_size limit (by-value row tables)
-constexpr int kKvChunk = 256;         // keys per split in decode attention
+constexpr int kChunk = 128;           // keys per split in decode attention
+constexpr int kMaxDecodeCtas = 256;   // persistent CTAs of the decode projection kernel
+// fp32 partials of split tiles: two 128 x 64 blocks per persistent CTA
+constexpr size_t kDecodePartBytes = static_cast<size_t>(kMaxDecodeCtas) * 2 * 128 * 64 * 4;
+constexpr int kMaxTiles = 4096;       // tile counters: N / 128 of the widest projection
 
 // Token -> (batch row, position) map of one prefill call, passed by value.
 struct RowTable {
@@ -39,11 +43,29 @@ struct Epi {
     int nq, nkvc, hd, max_seq;
     long long kv_row_stride;   // elements between batch rows of one layer's cache
     const float2* rope;        // [max_seq][hd/2] (cos, sin)
-    // SWIGLU: interleaved columns (64 w1 rows, then the same 64 w3 rows, ...)
+    // SWIGLU: interleaved columns (16 w1 rows, then the same 16 w3 rows, ...)
     // -> g[m*H + h] = silu(w1) * w3.
     void* g;
     int H;
     int* status;
+};
+
+// RMSNorm folded into the decode projections (bf16 decode chain), using
+// norm(x) W^T = r_b * ((x * w) W^T) with r_b = 1/sqrt(mean(x_b^2) + eps):
+//   producer side (residual epilogue of wo / w2, and the embedding): besides
+//     x it writes y_out[b, n] = bf16(x[b, n] * w_next[n]) -- the operand of the
+//     next projection, w_next the weight of the norm in front of it -- and
+//     ssq_out[b * n_tiles + t] = sum of x^2 over the 128 features of tile t;
+//   consumer side (wq/wk/wv, w1/w3, output): multiplies accumulator column b
+//     by r_b = 1/sqrt(sum_t ssq_in[b * n_in + t] / K + eps) before its epilogue.
+// Null pointers switch either side off.
+struct NormIO {
+    const float* ssq_in;
+    int n_in;
+    float eps;
+    float* ssq_out;
+    void* y_out;
+    const float* w_next;
 };
 
 struct TmaMaps {               // tensor maps of one K-major bf16 matrix
@@ -56,7 +78,7 @@ struct LayerPtrs {
     void* wqkv;
     void* wo;
     float* ffn_norm;
-    void* w13;   // interleaved in blocks of 64 rows: w1[0:64], w3[0:64], w1[64:128], ...
+    void* w13;   // interleaved in blocks of 16 rows: w1[0:16], w3[0:16], w1[16:32], ...
     void* w2;
     TmaMaps m_wqkv, m_wo, m_w13, m_w2;
 };
@@ -98,6 +120,10 @@ struct Model {
     float* logits_ws;   // [Bmax, V]
     float* part_o;      // [Bmax*nh*n_splits, hd]
     float* part_ml;     // [Bmax*nh*n_splits, 2]
+    int* attn_cnt;      // [Bmax*nkv] split arrival counters (zero between launches)
+    float* gemm_part;   // split-tile partials of the decode projection kernel
+    int* gemm_cnt;      // per-tile arrival counters (zero between launches)
+    float* ssq;         // [Bmax, dim/128] per-tile sums of x^2 for the fused RMSNorm
     int* status;
     TmaMaps m_y, m_attn, m_g, m_ylast;   // activation maps (A box 128 rows, B box 16 rows)
     cudaStream_t last_stream;
@@ -108,30 +134,41 @@ struct Model {
 int launch_rope_table(float2* rope, int S, int hd, float theta, cudaStream_t st);
 int launch_token_map(const RowTable& rt, const int32_t* tokens, int* tok_ids, int* tok_row,
                      int* tok_pos, int* last_idx, cudaStream_t st);
+// `pdl`: launch as part of the decode chain (may start before its predecessor ends).
+// With `ssq`, also writes the sum of x^2 of every 128-feature block and
+// y = bf16(x * w_next) (the fused RMSNorm's producer side, see NormIO).
 int launch_embed(const int* tok_ids, const void* emb, int dtype, int M, int dim, int V, float* x,
-                 int* status, cudaStream_t st);
+                 int* status, cudaStream_t st, bool pdl = false, float* ssq = nullptr, void* y = nullptr,
+                 const float* w_next = nullptr);
 int launch_rmsnorm(const float* x, const int* row_idx, const float* w, int M, int dim, float eps,
-                   void* out, int out_dtype, cudaStream_t st);
+                   void* out, int out_dtype, cudaStream_t st, bool pdl = false);
 int launch_copy_interleave_w13(const void* src, void* w13, int H, int dim, int which, int esz,
                                cudaStream_t st);
 
 // out = A W^T with epilogue `ep`.  A rows: M (tokens), W rows: N, K.
 // bf16 uses tcgen05 with the given maps (A-side/W-side), fp32 the SIMT kernel.
 int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, const void* W,
-               const TmaMaps* mapW, int M, int N, int K, const Epi& ep, cudaStream_t st);
+               const TmaMaps* mapW, int M, int N, int K, const Epi& ep, cudaStream_t st, bool pdl = false,
+               const NormIO* nio = nullptr);
 int linear_f32(const float* A, const float* W, int M, int N, int K, const Epi& ep, cudaStream_t st);
 int linear_bf16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep,
                    cudaStream_t st);
+int linear_bf16_decode(const TmaMaps* mapX, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
+                       int* counters, cudaStream_t st, bool pdl, const NormIO* nio = nullptr);
+// bf16 projection: M <= 64 token rows -> linear_bf16_decode, else linear_bf16_tc.
+int linear_bf16(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
+                int* counters, cudaStream_t st, bool pdl = false, const NormIO* nio = nullptr);
 
 int launch_attention_prefill(const Model* m, int layer, const RowTable& rt, cudaStream_t st);
 int launch_attention_prefill_tc(const Model* m, int layer, const RowTable& rt, cudaStream_t st);
-int launch_attention_decode(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st);
+int launch_attention_decode(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st,
+                            bool pdl = false);
 
 int launch_argmax(const float* logits, int B, int V, int32_t* out, int32_t* tokens_adv,
-                  int32_t* pos_adv, cudaStream_t st);
+                  int32_t* pos_adv, cudaStream_t st, bool pdl = false);
 int launch_top_p(const float* logits, int B, int V, float temperature, float top_p,
                  const float* uniforms, int32_t* out, int32_t* tokens_adv, int32_t* pos_adv,
-                 cudaStream_t st);
+                 cudaStream_t st, bool pdl = false);
 
 // TMA descriptor encoding (driver entry point resolved at run time).
 int encode_kmajor_bf16(CUtensorMap* map, const void* base, int rows, int cols, int box_rows);

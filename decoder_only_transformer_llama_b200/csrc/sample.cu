@@ -36,6 +36,8 @@ __device__ __forceinline__ uint64_t sort_key(float l, int id) {
 // ---------------------------------------------------------------- argmax
 __global__ void __launch_bounds__(kSampleThreads)
 argmax_kernel(const float* __restrict__ logits, int V, int32_t* out, int32_t* tokens_adv, int32_t* pos_adv) {
+    pdl_trigger();
+    pdl_wait();
     const int b = blockIdx.x;
     const float* row = logits + static_cast<long long>(b) * V;
     float best = -INFINITY;
@@ -191,6 +193,8 @@ top_p_kernel(const float* __restrict__ logits, int V, float temperature, float t
              const float* __restrict__ uniforms, int32_t* out, int32_t* tokens_adv, int32_t* pos_adv) {
     extern __shared__ uint8_t smem_raw[];
     TopPShared& sh = *reinterpret_cast<TopPShared*>(smem_raw);
+    pdl_trigger();
+    pdl_wait();
     const int b = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const float* row = logits + static_cast<long long>(b) * V;
@@ -244,14 +248,16 @@ top_p_kernel(const float* __restrict__ logits, int V, float temperature, float t
 }
 
 int launch_argmax(const float* logits, int B, int V, int32_t* out, int32_t* tokens_adv, int32_t* pos_adv,
-                  cudaStream_t st) {
-    argmax_kernel<<<B, kSampleThreads, 0, st>>>(logits, V, out, tokens_adv, pos_adv);
-    LLB_CHECK_LAUNCH("argmax_kernel");
+                  cudaStream_t st, bool pdl) {
+    cudaError_t e = launch_k(argmax_kernel, dim3(B), dim3(kSampleThreads), 0, st, pdl, logits, V, out, tokens_adv,
+                             pos_adv);
+    count_launch();
+    if (e != cudaSuccess) return cuda_fail(e, "argmax_kernel");
     return LLAMA_OK;
 }
 
 int launch_top_p(const float* logits, int B, int V, float temperature, float top_p, const float* uniforms,
-                 int32_t* out, int32_t* tokens_adv, int32_t* pos_adv, cudaStream_t st) {
+                 int32_t* out, int32_t* tokens_adv, int32_t* pos_adv, cudaStream_t st, bool pdl) {
     const int smem = static_cast<int>(sizeof(TopPShared));
     static bool attr = false;
     if (!attr) {
@@ -259,9 +265,10 @@ int launch_top_p(const float* logits, int B, int V, float temperature, float top
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(top_p_kernel)");
         attr = true;
     }
-    top_p_kernel<<<B, kSampleThreads, smem, st>>>(logits, V, temperature, top_p, uniforms, out, tokens_adv,
-                                                   pos_adv);
-    LLB_CHECK_LAUNCH("top_p_kernel");
+    cudaError_t e = launch_k(top_p_kernel, dim3(B), dim3(kSampleThreads), smem, st, pdl, logits, V, temperature,
+                             top_p, uniforms, out, tokens_adv, pos_adv);
+    count_launch();
+    if (e != cudaSuccess) return cuda_fail(e, "top_p_kernel");
     return LLAMA_OK;
 }
 

@@ -30,11 +30,17 @@ LLAMA_API int llama_op_rmsnorm(const float* x, const float* w, int M, int dim, f
  *   A [M, K] and W [N, K] in `dtype` (LLAMA_F32: SIMT fp32 FMA, no TF32;
  *   LLAMA_BF16: tcgen05 tensor cores with fp32 accumulation in TMEM);
  *   out fp32 [M, N] (row-major, overwritten).  K % 8 == 0 for bf16.
- * The bf16 kernel is the one the model path uses: for M <= 64 it runs with
- * the weight as the 128-row MMA operand (decode shape), else with the
- * activations as that operand (prefill shape). */
+ * The bf16 kernels are the ones the model path uses: for M <= 64 the
+ * persistent weight-streaming kernel (the weight is the 128-row MMA operand,
+ * K split across CTAs), else the 128 x 256-tile kernel.
+ *   workspace  device scratch of llama_op_linear_workspace_bytes(), 256-byte
+ *              aligned, zero-filled before its first use (the kernel leaves
+ *              its counters at zero again); needed for bf16 with M <= 64,
+ *              otherwise may be NULL.  Calls sharing a workspace must not
+ *              overlap on the device. */
+LLAMA_API size_t llama_op_linear_workspace_bytes(void);
 LLAMA_API int llama_op_linear(const void* A, const void* W, int M, int N, int K, int dtype,
-                    float* out, void* stream);
+                    float* out, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Per-launch timing of a model's projection kernels (for benchmarks).
  * llama_profile_start: from now on every projection launch the model enqueues

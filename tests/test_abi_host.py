@@ -25,7 +25,7 @@ def _declared_symbols():
 
 def test_library_exports_every_declared_symbol():
     names = _declared_symbols()
-    assert len(names) >= 13
+    assert len(names) >= 16
     for n in names:
         assert hasattr(llb.lib(), n), n
     assert set(llb.EXPORTED) == names
@@ -103,7 +103,10 @@ def test_calls_reject_null_model_and_bad_sizes():
     assert lib.llama_sample(0x1000, 1, 10, 0.7, 0.9, None, 0x1000, None) == llb.LLAMA_ERR_INVALID_ARG  # no uniforms
     assert lib.llama_sample(0x1000, 1, 10, -1.0, 0.9, 0x1000, 0x1000, None) == llb.LLAMA_ERR_INVALID_ARG
     assert lib.llama_model_status(None, None) == llb.LLAMA_ERR_INVALID_ARG
-    assert lib.llama_op_linear(None, 0x1000, 1, 1, 8, 1, 0x1000, None) == llb.LLAMA_ERR_INVALID_ARG
-    assert lib.llama_op_linear(0x1000, 0x1000, 1, 1, 7, 1, 0x1000, None) == llb.LLAMA_ERR_INVALID_ARG  # K % 8
+    assert lib.llama_op_linear(None, 0x1000, 1, 1, 8, 1, 0x1000, None, 0, None) == llb.LLAMA_ERR_INVALID_ARG
+    assert lib.llama_op_linear(0x1000, 0x1000, 1, 1, 7, 1, 0x1000, None, 0, None) == llb.LLAMA_ERR_INVALID_ARG  # K % 8
+    # decode-shaped bf16 needs the scratch workspace
+    assert lib.llama_op_linear(0x1000, 0x1000, 4, 128, 64, 1, 0x1000, None, 0, None) == llb.LLAMA_ERR_INVALID_ARG
+    assert lib.llama_op_linear_workspace_bytes() > 0
     assert lib.llama_op_rmsnorm(0x1000, 0x1000, 1, 6, 1e-5, 0x1000, 0, None) == llb.LLAMA_ERR_INVALID_ARG
     assert lib.llama_get_kv(None, 0, None, None, None) == llb.LLAMA_ERR_INVALID_ARG
