@@ -149,7 +149,7 @@ static int make_maps(TmaMaps* t, const void* base, int rows, int cols, int b_box
 
 int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, const void* W,
                const TmaMaps* mapW, int M, int N, int K, const Epi& ep, cudaStream_t st, bool pdl,
-               const NormIO* nio) {
+               const NormIO* nio, const NextProj* next) {
     Profile* pr = const_cast<Profile*>(&m->prof);
     const bool timed = pr->n < pr->capacity;
     if (timed) {
@@ -160,7 +160,7 @@ int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, co
     if (dtype == LLAMA_F32)
         rc = linear_f32(static_cast<const float*>(A), static_cast<const float*>(W), M, N, K, ep, st);
     else
-        rc = linear_bf16(mapA, mapW, M, N, K, ep, m->gemm_part, m->gemm_cnt, st, pdl && !timed, nio);
+        rc = linear_bf16(mapA, mapW, M, N, K, ep, m->gemm_part, m->gemm_cnt, st, pdl && !timed, nio, next);
     if (timed && rc == LLAMA_OK) {
         cudaError_t e = cudaEventRecord(pr->ev[2 * pr->n + 1], st);
         if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord(profile)");
@@ -473,8 +473,14 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B
             ep.vc = static_cast<char*>(m->vc) + l * m->kv_layer_elems * m->esz;
             ep.tok_pos = pos;
             const NormIO n_in = {m->ssq, nb, eps, nullptr, nullptr, nullptr};
+            // each projection warms L2 with the first weight tiles of the next one
+            const NextProj nx_wo = {&Lp.m_wo.a128, m->dim, m->nq};
+            const NextProj nx_w13 = {&Lp.m_w13.a128, 2 * m->H, m->dim};
+            const NextProj nx_w2 = {&Lp.m_w2.a128, m->dim, m->H};
+            const NextProj nx_after = l + 1 < m->L ? NextProj{&m->layers[l + 1].m_wqkv.a128, m->nqkv, m->dim}
+                                                    : NextProj{&m->m_output.a128, m->V, m->dim};
             LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.wqkv, &Lp.m_wqkv, B, m->nqkv, m->dim, ep, st, true,
-                               &n_in));
+                               &n_in, &nx_wo));
             LLB_TRY(launch_attention_decode(m, l, pos, B, st, true));
             Epi er = base_epi(m);
             er.mode = EPI_RESID_F32;
@@ -482,15 +488,15 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B
             er.ldo = m->dim;
             const NormIO n_to_ffn = {nullptr, 0, 0.f, m->ssq, m->y, Lp.ffn_norm};
             LLB_TRY(run_linear(m, m->dtype, m->attn, &m->m_attn, Lp.wo, &Lp.m_wo, B, m->dim, m->nq, er, st, true,
-                               &n_to_ffn));
+                               &n_to_ffn, &nx_w13));
             Epi es = base_epi(m);
             es.mode = EPI_SWIGLU;
             es.g = m->g;
             LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.w13, &Lp.m_w13, B, 2 * m->H, m->dim, es, st, true,
-                               &n_in));
+                               &n_in, &nx_w2));
             const NormIO n_to_next = {nullptr, 0, 0.f, m->ssq, m->y, next_norm};
             LLB_TRY(run_linear(m, m->dtype, m->g, &m->m_g, Lp.w2, &Lp.m_w2, B, m->dim, m->H, er, st, true,
-                               &n_to_next));
+                               &n_to_next, &nx_after));
         }
         const NormIO n_in = {m->ssq, nb, eps, nullptr, nullptr, nullptr};
         LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, m->output, &m->m_output, B, m->V, m->dim, eo, st, true,

@@ -10,6 +10,8 @@
 // Prefill of fp32 models: one CTA per (64-query tile, head, row), online
 // softmax over 64-key tiles staged in shared memory (fp32 CUDA-core
 // arithmetic).  bf16 models use the tensor-core kernel of attention_prefill_tc.cu.
+#include <algorithm>
+
 #include "common.cuh"
 #include "model.h"
 
@@ -44,50 +46,58 @@ template <> struct Vec<bf16, 4> {
 };
 
 // ---------------------------------------------------------------- decode
-// CTA (split s, kv head g, row b) handles keys [s*kChunk, (s+1)*kChunk) of
-// head g for all n_rep query heads of the group.  The chunk of K and the
-// chunk of V are each one contiguous block of the cache (positions of one
-// head are adjacent), fetched by two bulk async copies into shared memory.
-// Warp w scores keys w, w+4, ...; lane l holds head dims [l*EPL, l*EPL+EPL).
-// A row whose context fits one chunk writes its output directly; otherwise
-// every split publishes an unnormalised partial (o, max, sum) and the split
-// that arrives last at the (row, kv head) counter merges them in split order.
+// Flash-decoding over the cache: CTA (z, kv head g, row b) walks the 64-key
+// chunks z, z+P, z+2P, ... of head g's positions 0 .. pos[b] for all n_rep
+// query heads of the group.  Each chunk of K and of V is one contiguous block
+// of the cache (the positions of one head are adjacent), fetched by one bulk
+// async copy into a two-deep shared-memory ring.  Warp w scores keys 2w,
+// 2w+1, 2w+8, ... of a chunk; lane l holds head dims [l*EPL, (l+1)*EPL).
+// The P CTAs of (b, g) with at least one chunk publish unnormalised partials
+// (o, max, sum); the one that arrives last at the (b, g) counter merges them in
+// CTA order.  With a single active CTA the output is written directly.
 template <typename T, int HD, int NREP>
 __global__ void __launch_bounds__(128)
 attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
-                   const int32_t* __restrict__ pos, int nq, int S, long long row_stride, int n_splits,
+                   const int32_t* __restrict__ pos, int nq, int S, long long row_stride,
                    float* __restrict__ part_o, float* __restrict__ part_ml, int* __restrict__ counters,
                    T* __restrict__ out, int* status) {
     constexpr int EPL = HD / 32;   // head dims per lane
     constexpr int ROW = HD * static_cast<int>(sizeof(T));
+    constexpr int CH_BYTES = kChunk * ROW;
     extern __shared__ __align__(128) uint8_t dsm[];
-    T* sK = reinterpret_cast<T*>(dsm);
-    T* sV = reinterpret_cast<T*>(dsm + kChunk * ROW);
-    __shared__ uint64_t bar;
+    __shared__ uint64_t bar[2];
     __shared__ float s_m[4][NREP], s_l[4][NREP];
     __shared__ float s_o[4][NREP][HD];
     __shared__ int s_last;
     pdl_trigger();
     pdl_wait();
-    const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int z = blockIdx.x, P = gridDim.x, g = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int p = pos[b];
     if (p < 0 || p >= S) {
-        if (s == 0 && g == 0 && threadIdx.x == 0) report_status(status, LLAMA_ERR_CAPACITY);
+        if (z == 0 && g == 0 && threadIdx.x == 0) report_status(status, LLAMA_ERR_CAPACITY);
         return;
     }
     const int ctx = p + 1;
-    const int j0 = s * kChunk;
-    if (j0 >= ctx) return;
-    const int n = min(kChunk, ctx - j0);
-    const int nvalid = (ctx + kChunk - 1) / kChunk;
+    const int nchunks = (ctx + kChunk - 1) / kChunk;
+    if (z >= nchunks) return;
+    const int pact = min(P, nchunks);                  // CTAs of (b, g) with work
+    const int mine = (nchunks - z + P - 1) / P;        // chunks of this CTA
     const long long head_off = static_cast<long long>(b) * row_stride + static_cast<long long>(g) * S * HD;
+    auto issue = [&](int i) {                          // i-th chunk of this CTA into ring slot i % 2
+        const int j0 = (z + i * P) * kChunk;
+        const int n = min(kChunk, ctx - j0);
+        uint8_t* slot = dsm + (i & 1) * 2 * CH_BYTES;
+        mbar_arrive_expect_tx(&bar[i & 1], 2u * n * ROW);
+        bulk_load(slot, kc + head_off + static_cast<long long>(j0) * HD, n * ROW, &bar[i & 1]);
+        bulk_load(slot + CH_BYTES, vc + head_off + static_cast<long long>(j0) * HD, n * ROW, &bar[i & 1]);
+    };
     if (threadIdx.x == 0) {
-        mbar_init(&bar, 1);
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(&bar, 2u * n * ROW);
-        bulk_load(sK, kc + head_off + static_cast<long long>(j0) * HD, n * ROW, &bar);
-        bulk_load(sV, vc + head_off + static_cast<long long>(j0) * HD, n * ROW, &bar);
+        issue(0);
+        if (mine > 1) issue(1);
     }
     const float scale = rsqrtf(static_cast<float>(HD));
     float qv[NREP][EPL];
@@ -97,10 +107,6 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
 #pragma unroll
         for (int e = 0; e < EPL; ++e) qv[r][e] *= scale;
     }
-    __syncthreads();   // barrier initialised
-    const bool ok = mbar_wait(&bar, 0);
-    if (!ok && threadIdx.x == 0) report_status(status, LLAMA_ERR_DEVICE_TIMEOUT);
-
     float mx[NREP], sl[NREP], o[NREP][EPL];
 #pragma unroll
     for (int r = 0; r < NREP; ++r) {
@@ -109,7 +115,14 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
 #pragma unroll
         for (int e = 0; e < EPL; ++e) o[r][e] = 0.f;
     }
-    if (ok) {
+    __syncthreads();   // barriers initialised
+    bool ok = true;
+    for (int i = 0; i < mine && ok; ++i) {
+        ok = mbar_wait(&bar[i & 1], (i >> 1) & 1);
+        if (!ok) break;
+        const T* sK = reinterpret_cast<const T*>(dsm + (i & 1) * 2 * CH_BYTES);
+        const T* sV = reinterpret_cast<const T*>(dsm + (i & 1) * 2 * CH_BYTES + CH_BYTES);
+        const int n = min(kChunk, ctx - (z + i * P) * kChunk);
         for (int jb = warp * 2; jb < n; jb += 8) {
             float kv[2][EPL], vv[2][EPL];
 #pragma unroll
@@ -138,9 +151,12 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
                 mx[r] = mnew;
             }
         }
+        __syncthreads();                               // ring slot i % 2 is free again
+        if (threadIdx.x == 0 && i + 2 < mine) issue(i + 2);
     }
+    if (!ok && threadIdx.x == 0) report_status(status, LLAMA_ERR_DEVICE_TIMEOUT);
 
-    // merge the 4 warps of this split
+    // merge the 4 warps of this CTA
     if (lane == 0) {
 #pragma unroll
         for (int r = 0; r < NREP; ++r) { s_m[warp][r] = mx[r]; s_l[warp][r] = sl[r]; }
@@ -164,10 +180,10 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
             acc += s_o[w][r][d] * f;
         }
         const int h = g * NREP + r;
-        if (nvalid == 1) {
+        if (pact == 1) {
             out[static_cast<long long>(b) * nq + h * HD + d] = from_f32<T>(acc / L);
         } else {
-            const long long slot = (static_cast<long long>(b) * nh + h) * n_splits + s;
+            const long long slot = (static_cast<long long>(b) * nh + h) * P + z;
             part_o[slot * HD + d] = acc;
             if (d == 0) {
                 part_ml[slot * 2] = M;
@@ -175,22 +191,21 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
             }
         }
     }
-    if (nvalid == 1) return;
-    // publish the partial; the last split of (b, g) merges all of them
+    if (pact == 1) return;
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) s_last = atomicAdd(&counters[b * gridDim.y + g], 1) == nvalid - 1;
+    if (threadIdx.x == 0) s_last = atomicAdd(&counters[b * gridDim.y + g], 1) == pact - 1;
     __syncthreads();
     if (!s_last) return;
     __threadfence();
     for (int idx = threadIdx.x; idx < NREP * HD; idx += blockDim.x) {
         const int r = idx / HD, d = idx % HD;
         const int h = g * NREP + r;
-        const long long base = (static_cast<long long>(b) * nh + h) * n_splits;
+        const long long base = (static_cast<long long>(b) * nh + h) * P;
         float M = -INFINITY;
-        for (int t = 0; t < nvalid; ++t) M = fmaxf(M, part_ml[(base + t) * 2]);
+        for (int t = 0; t < pact; ++t) M = fmaxf(M, part_ml[(base + t) * 2]);
         float L = 0.f, acc = 0.f;
-        for (int t = 0; t < nvalid; ++t) {
+        for (int t = 0; t < pact; ++t) {
             const float f = __expf(part_ml[(base + t) * 2] - M);
             L += part_ml[(base + t) * 2 + 1] * f;
             acc += part_o[(base + t) * HD + d] * f;
@@ -200,22 +215,35 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
     if (threadIdx.x == 0) counters[b * gridDim.y + g] = 0;
 }
 
+static int g_attn_sms = 0;
+
 template <typename T, int HD, int NREP>
 static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl) {
     const T* kc = static_cast<const T*>(m->kc) + layer * m->kv_layer_elems;
     const T* vc = static_cast<const T*>(m->vc) + layer * m->kv_layer_elems;
     auto kern = attn_decode_kernel<T, HD, NREP>;
-    const int smem = 2 * kChunk * HD * static_cast<int>(sizeof(T));
+    const int smem = 4 * kChunk * HD * static_cast<int>(sizeof(T));
     static bool attr = false;
     if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_decode_kernel)");
         attr = true;
     }
-    dim3 grid(m->n_splits, m->nkv, B);
+    if (g_attn_sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&g_attn_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (g_attn_sms <= 0) g_attn_sms = 148;
+    }
+    // about two CTAs per SM over all (row, kv head) pairs, never more than the chunks
+    int P = (2 * g_attn_sms + m->nkv * B - 1) / (m->nkv * B);
+    P = std::max(1, std::min(P, m->n_splits));
+    dim3 grid(P, m->nkv, B);
     cudaError_t e = launch_k(kern, grid, dim3(128), smem, st, pdl, static_cast<const T*>(m->q), kc, vc, pos, m->nq,
-                             m->S, m->kv_row_elems, m->n_splits, m->part_o, m->part_ml, m->attn_cnt,
-                             static_cast<T*>(m->attn), m->status);
+                             m->S, m->kv_row_elems, m->part_o, m->part_ml, m->attn_cnt, static_cast<T*>(m->attn),
+                             m->status);
     count_launch();
     if (e != cudaSuccess) return cuda_fail(e, "attn_decode_kernel");
     return LLAMA_OK;

@@ -127,6 +127,11 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint3
         :: "r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
+// Fetch one tensor-map box into L2 only (no shared memory, no completion).
+__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* map, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];"
+                 :: "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y) : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -218,6 +223,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 }
 
 #ifdef __CUDACC__
+// Kernels of the decode chain all ask for the largest shared-memory carveout,
+// so that consecutive kernels never wait for an SM to change its L1/shared
+// split (which would also stop them from overlapping).
+template <typename... KArgs>
+static inline cudaError_t carveout_max(void (*kern)(KArgs...)) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+}
+
 // Launch `kern` with or without the programmatic-serialisation attribute.
 template <typename... KArgs, typename... Args>
 static inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,

@@ -119,6 +119,13 @@ __global__ void embed_kernel(const int* tok, const T* emb, int dim, int V, float
 int launch_embed(const int* tok_ids, const void* emb, int dtype, int M, int dim, int V, float* x,
                  int* status, cudaStream_t st, bool pdl, float* ssq, void* y, const float* w_next) {
     if (M <= 0) return LLAMA_OK;
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t ce = carveout_max(embed_kernel<bf16>);
+        if (ce == cudaSuccess) ce = carveout_max(embed_kernel<float>);
+        if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute(embed_kernel)");
+        attr = true;
+    }
     cudaError_t e;
     if (dtype == LLAMA_BF16)
         e = launch_k(embed_kernel<bf16>, dim3(M), dim3(128), 0, st, pdl, tok_ids, static_cast<const bf16*>(emb),

@@ -21,6 +21,10 @@
 // A deep ring (about 200 KB of weight tiles in flight per SM) keeps HBM
 // busy; the next projection's CTAs launch early (programmatic dependent
 // launch) and start streaming as soon as this kernel's CTAs leave their SMs.
+// Weights never change during decode, so when a CTA's producer has issued
+// its last load it also pulls the first ring's worth of the NEXT projection's
+// weight tiles for the same CTA index into L2: the next kernel starts on L2
+// hits, and HBM stays busy during this kernel's epilogue and fixup tail.
 // Two TMEM accumulators let the MMA of the next segment overlap the epilogue
 // of the previous one.  With programmatic dependent launch, weight tiles are
 // requested before the previous kernel has finished; the activation tiles
@@ -55,22 +59,20 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 }
 
 // CTA owning flat unit u when W units are split into P contiguous runs
-__device__ __forceinline__ int owner(long long u, long long W, int P) {
-    return static_cast<int>(((u + 1) * P - 1) / W);
-}
-__device__ __forceinline__ long long run_begin(int c, long long W, int P) { return c * W / P; }
+// (W * P stays far below 2^31: W <= kMaxTiles * 256 k-tiles, P <= 256).
+__device__ __forceinline__ int owner(int u, int W, int P) { return ((u + 1) * P - 1) / W; }
+__device__ __forceinline__ int run_begin(int c, int W, int P) { return c * W / P; }
 
 struct Seg {
     int tile, ks, ke;
 };
 
 // Next segment (one tile's k-range) of a run of units; false past the end.
-__device__ __forceinline__ bool next_seg(long long& u, long long u1, int KT, Seg& s) {
+__device__ __forceinline__ bool next_seg(int& u, int u1, int KT, Seg& s) {
     if (u >= u1) return false;
-    s.tile = static_cast<int>(u / KT);
-    s.ks = static_cast<int>(u % KT);
-    const long long rem = u1 - u;
-    s.ke = static_cast<int>(min(static_cast<long long>(KT), s.ks + rem));
+    s.tile = u / KT;
+    s.ks = u - s.tile * KT;
+    s.ke = min(KT, s.ks + (u1 - u));
     u += s.ke - s.ks;
     return true;
 }
@@ -79,7 +81,8 @@ __device__ __forceinline__ bool next_seg(long long& u, long long u1, int KT, Seg
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUtensorMap mapX,
-                     int N, int M, int K, Epi ep, float* __restrict__ part, int* __restrict__ counters, NormIO nio) {
+                     int N, int M, int K, Epi ep, float* __restrict__ part, int* __restrict__ counters, NormIO nio,
+                     const __grid_constant__ CUtensorMap mapNext, int Nn, int Kn, int Pn) {
     constexpr int B_BYTES = BN * 128;
     constexpr int STAGE = kABytes + B_BYTES;
     extern __shared__ uint8_t smem_raw[];
@@ -97,8 +100,8 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = gridDim.x, c = blockIdx.x;
     const int T = (N + 127) / 128, KT = (K + 63) / 64;
-    const long long W = static_cast<long long>(T) * KT;
-    const long long u0 = run_begin(c, W, P), u1 = run_begin(c + 1, W, P);
+    const int W = T * KT;
+    const int u0 = run_begin(c, W, P), u1 = run_begin(c + 1, W, P);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -120,38 +123,50 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
         // tiles per ring slot, walking this CTA's units in order.  Weight
         // tiles of the first slots are requested before the previous kernel
         // has finished; activation tiles only after it has.
-        const int nunits = static_cast<int>(u1 - u0);
+        const int nunits = u1 - u0;
         const int npre = nunits < STAGES ? nunits : STAGES;
-        const uint32_t tx = STAGE;
+        int t0 = u0 / KT, k0 = u0 - t0 * KT;          // walk (tile, k) without divisions
+        int tt = t0, kk = k0;
         for (int i = 0; i < npre; ++i) {
-            const long long u = u0 + i;
-            mbar_arrive_expect_tx(&full[i], tx);
-            tma_load_2d(smem + i * STAGE, &mapW, static_cast<int>(u % KT) * 64, static_cast<int>(u / KT) * 128,
-                        &full[i]);
+            mbar_arrive_expect_tx(&full[i], STAGE);
+            tma_load_2d(smem + i * STAGE, &mapW, kk * 64, tt * 128, &full[i]);
+            if (++kk == KT) { kk = 0; ++tt; }
         }
         pdl_wait();
+        tt = t0;
+        kk = k0;
         for (int i = 0; i < npre; ++i) {
-            const long long u = u0 + i;
 #pragma unroll
             for (int rr = 0; rr < BN / 16; ++rr)
-                tma_load_2d(smem + i * STAGE + kABytes + rr * 2048, &mapX, static_cast<int>(u % KT) * 64,
-                            rr * 16, &full[i]);
+                tma_load_2d(smem + i * STAGE + kABytes + rr * 2048, &mapX, kk * 64, rr * 16, &full[i]);
+            if (++kk == KT) { kk = 0; ++tt; }
         }
         for (int i = npre; i < nunits; ++i) {
             const int s = i % STAGES;
             if (!mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1)) { atomicExch(&flag[0], 1); break; }
-            const long long u = u0 + i;
-            const int kx = static_cast<int>(u % KT) * 64;
             uint8_t* st = smem + s * STAGE;
-            mbar_arrive_expect_tx(&full[s], tx);
-            tma_load_2d(st, &mapW, kx, static_cast<int>(u / KT) * 128, &full[s]);
+            mbar_arrive_expect_tx(&full[s], STAGE);
+            tma_load_2d(st, &mapW, kk * 64, tt * 128, &full[s]);
 #pragma unroll
-            for (int rr = 0; rr < BN / 16; ++rr) tma_load_2d(st + kABytes + rr * 2048, &mapX, kx, rr * 16, &full[s]);
+            for (int rr = 0; rr < BN / 16; ++rr) tma_load_2d(st + kABytes + rr * 2048, &mapX, kk * 64, rr * 16, &full[s]);
+            if (++kk == KT) { kk = 0; ++tt; }
+        }
+        if (Nn > 0 && c < Pn) {
+            // warm L2 with the first units of this CTA index's run in the next projection
+            const int KTn = (Kn + 63) / 64;
+            const int Wn = ((Nn + 127) / 128) * KTn;
+            const int v0 = run_begin(c, Wn, Pn), v1 = run_begin(c + 1, Wn, Pn);
+            const int nv = min(v1 - v0, STAGES);
+            int tn = v0 / KTn, kn = v0 - tn * KTn;
+            for (int i = 0; i < nv; ++i) {
+                tma_prefetch_l2(&mapNext, kn * 64, tn * 128);
+                if (++kn == KTn) { kn = 0; ++tn; }
+            }
         }
     } else if (warp == 1 && lane == 0) {
         // ---------------- MMA issuer
         const uint32_t idesc = idesc_bf16_f32(128, BN);
-        long long u = u0;
+        int u = u0;
         Seg sg;
         int i = 0, j = 0;
         bool abort = false;
@@ -189,7 +204,7 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
             rs[epi_tid] = rsqrtf(ss / static_cast<float>(K) + nio.eps);
         }
         named_sync(1, 128);
-        long long u = u0;
+        int u = u0;
         Seg sg;
         int j = 0;
         const int nb = M < BN ? M : BN;
@@ -210,7 +225,7 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
                 break;
             }
             const int t = sg.tile;
-            const long long tb = static_cast<long long>(t) * KT;
+            const int tb = t * KT;
             const int cf = owner(tb, W, P), cl = owner(tb + KT - 1, W, P);
             if (cl > cf) {
                 // split tile: publish this CTA's partial, the last arrival reduces
@@ -228,14 +243,32 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
                 __threadfence();
 #pragma unroll
                 for (int b = 0; b < BN; ++b) v[b] = 0.f;
-                for (int cc = cf; cc <= cl; ++cc) {
-                    // slot 0 holds a CTA's first segment, slot 1 its last
-                    const int sl = run_begin(cc, W, P) >= tb ? 0 : 1;
-                    const float* pp = part + ((static_cast<long long>(cc) * 2 + sl) * 128 + r) * BN;
+                // partials in CTA order, CB contributors per batch of independent loads
+                constexpr int CB = BN <= 16 ? 4 : (BN <= 32 ? 2 : 1);
+                for (int cb = cf; cb <= cl; cb += CB) {
+                    float4 f[CB][BN / 4];
 #pragma unroll
-                    for (int b = 0; b < BN; b += 4) {
-                        const float4 f = *reinterpret_cast<const float4*>(pp + b);
-                        v[b] += f.x; v[b + 1] += f.y; v[b + 2] += f.z; v[b + 3] += f.w;
+                    for (int e = 0; e < CB; ++e) {
+                        const int cc = cb + e;
+                        if (cc <= cl) {
+                            const int sl = run_begin(cc, W, P) >= tb ? 0 : 1;   // slot 0: first segment, 1: last
+                            const float4* pp = reinterpret_cast<const float4*>(
+                                part + ((static_cast<long long>(cc) * 2 + sl) * 128 + r) * BN);
+#pragma unroll
+                            for (int qq = 0; qq < BN / 4; ++qq) f[e][qq] = pp[qq];
+                        }
+                    }
+#pragma unroll
+                    for (int e = 0; e < CB; ++e) {
+                        if (cb + e <= cl) {
+#pragma unroll
+                            for (int qq = 0; qq < BN / 4; ++qq) {
+                                v[4 * qq] += f[e][qq].x;
+                                v[4 * qq + 1] += f[e][qq].y;
+                                v[4 * qq + 2] += f[e][qq].z;
+                                v[4 * qq + 3] += f[e][qq].w;
+                            }
+                        }
                     }
                 }
                 if (epi_tid == 0) counters[t] = 0;
@@ -331,27 +364,41 @@ static int g_sms = 0;
 
 template <int BN, int STAGES>
 static int launch_decode(const CUtensorMap& w, const CUtensorMap& x, int N, int M, int K, const Epi& ep,
-                         float* part, int* counters, int max_ctas, cudaStream_t st, bool pdl, const NormIO& nio) {
+                         float* part, int* counters, int max_ctas, cudaStream_t st, bool pdl, const NormIO& nio,
+                         const NextProj* next) {
     constexpr int smem = 1024 + STAGES * (kABytes + BN * 128) + (2 * STAGES + 4) * 8 + 32 + 5 * 64 * 4;
     static_assert(smem <= 227 * 1024, "shared memory per CTA");
     auto kern = linear_decode_kernel<BN, STAGES>;
     static bool attr = false;
     if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(linear_decode_kernel)");
         attr = true;
     }
     const long long units = static_cast<long long>((N + 127) / 128) * ((K + 63) / 64);
+    if (units > (1 << 22)) { set_error("decode projection too large (%lld work units)", units); return LLAMA_ERR_INVALID_ARG; }
     int P = max_ctas;
     if (units < P) P = static_cast<int>(units);
-    cudaError_t e = launch_k(kern, dim3(P), dim3(kThreads), smem, st, pdl, w, x, N, M, K, ep, part, counters, nio);
+    int Nn = 0, Kn = 0, Pn = 0;
+    const CUtensorMap* mn = &w;
+    if (next && next->map) {
+        Nn = next->N;
+        Kn = next->K;
+        const long long un = static_cast<long long>((Nn + 127) / 128) * ((Kn + 63) / 64);
+        Pn = un < max_ctas ? static_cast<int>(un) : max_ctas;   // the grid the next launch will use
+        mn = next->map;
+    }
+    cudaError_t e = launch_k(kern, dim3(P), dim3(kThreads), smem, st, pdl, w, x, N, M, K, ep, part, counters, nio,
+                             *mn, Nn, Kn, Pn);
     count_launch();
     if (e != cudaSuccess) return cuda_fail(e, "linear_decode_kernel");
     return LLAMA_OK;
 }
 
 int linear_bf16_decode(const TmaMaps* mapX, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
-                       int* counters, cudaStream_t st, bool pdl, const NormIO* nio_in) {
+                       int* counters, cudaStream_t st, bool pdl, const NormIO* nio_in, const NextProj* next) {
     if (M <= 0 || N <= 0) return LLAMA_OK;
     NormIO nio = {};
     if (nio_in) nio = *nio_in;
@@ -367,10 +414,10 @@ int linear_bf16_decode(const TmaMaps* mapX, const TmaMaps* mapW, int M, int N, i
         if (g_sms <= 0) g_sms = 148;
         if (g_sms > kMaxDecodeCtas) g_sms = kMaxDecodeCtas;
     }
-    if (M <= 16) return launch_decode<16, 12>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio);
-    if (M <= 32) return launch_decode<32, 11>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio);
-    if (M <= 48) return launch_decode<48, 10>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio);
-    return launch_decode<64, 9>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio);
+    if (M <= 16) return launch_decode<16, 12>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio, next);
+    if (M <= 32) return launch_decode<32, 11>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio, next);
+    if (M <= 48) return launch_decode<48, 10>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio, next);
+    return launch_decode<64, 9>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio, next);
 }
 
 }  // namespace llb

@@ -291,8 +291,8 @@ int linear_bf16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K
 }
 
 int linear_bf16(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
-                int* counters, cudaStream_t st, bool pdl, const NormIO* nio) {
-    if (M <= 64) return linear_bf16_decode(mapA, mapW, M, N, K, ep, part, counters, st, pdl, nio);
+                int* counters, cudaStream_t st, bool pdl, const NormIO* nio, const NextProj* next) {
+    if (M <= 64) return linear_bf16_decode(mapA, mapW, M, N, K, ep, part, counters, st, pdl, nio, next);
     if (nio && (nio->ssq_in || nio->ssq_out)) { set_error("fused RMSNorm is a decode-shape feature"); return LLAMA_ERR_INVALID_ARG; }
     return linear_bf16_tc(mapA, mapW, M, N, K, ep, st);
 }

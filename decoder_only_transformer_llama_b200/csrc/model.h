@@ -12,7 +12,7 @@
 namespace llb {
 
 constexpr int kMaxRows = 256;         // max_batch_size limit (by-value row tables)
-constexpr int kChunk = 128;           // keys per split in decode attention
+constexpr int kChunk = 64;            // keys per chunk in decode attention
 constexpr int kMaxDecodeCtas = 256;   // persistent CTAs of the decode projection kernel
 // fp32 partials of split tiles: two 128 x 64 blocks per persistent CTA
 constexpr size_t kDecodePartBytes = static_cast<size_t>(kMaxDecodeCtas) * 2 * 128 * 64 * 4;
@@ -66,6 +66,13 @@ struct NormIO {
     float* ssq_out;
     void* y_out;
     const float* w_next;
+};
+
+// The projection launched after this one in the decode chain (its weight
+// map, N rows, K columns): used to warm L2 with its first weight tiles.
+struct NextProj {
+    const CUtensorMap* map;
+    int N, K;
 };
 
 struct TmaMaps {               // tensor maps of one K-major bf16 matrix
@@ -149,15 +156,17 @@ int launch_copy_interleave_w13(const void* src, void* w13, int H, int dim, int w
 // bf16 uses tcgen05 with the given maps (A-side/W-side), fp32 the SIMT kernel.
 int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, const void* W,
                const TmaMaps* mapW, int M, int N, int K, const Epi& ep, cudaStream_t st, bool pdl = false,
-               const NormIO* nio = nullptr);
+               const NormIO* nio = nullptr, const NextProj* next = nullptr);
 int linear_f32(const float* A, const float* W, int M, int N, int K, const Epi& ep, cudaStream_t st);
 int linear_bf16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep,
                    cudaStream_t st);
 int linear_bf16_decode(const TmaMaps* mapX, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
-                       int* counters, cudaStream_t st, bool pdl, const NormIO* nio = nullptr);
+                       int* counters, cudaStream_t st, bool pdl, const NormIO* nio = nullptr,
+                       const NextProj* next = nullptr);
 // bf16 projection: M <= 64 token rows -> linear_bf16_decode, else linear_bf16_tc.
 int linear_bf16(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
-                int* counters, cudaStream_t st, bool pdl = false, const NormIO* nio = nullptr);
+                int* counters, cudaStream_t st, bool pdl = false, const NormIO* nio = nullptr,
+                const NextProj* next = nullptr);
 
 int launch_attention_prefill(const Model* m, int layer, const RowTable& rt, cudaStream_t st);
 int launch_attention_prefill_tc(const Model* m, int layer, const RowTable& rt, cudaStream_t st);

@@ -249,6 +249,12 @@ top_p_kernel(const float* __restrict__ logits, int V, float temperature, float t
 
 int launch_argmax(const float* logits, int B, int V, int32_t* out, int32_t* tokens_adv, int32_t* pos_adv,
                   cudaStream_t st, bool pdl) {
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t ce = carveout_max(argmax_kernel);
+        if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute(argmax_kernel)");
+        attr = true;
+    }
     cudaError_t e = launch_k(argmax_kernel, dim3(B), dim3(kSampleThreads), 0, st, pdl, logits, V, out, tokens_adv,
                              pos_adv);
     count_launch();
@@ -262,6 +268,7 @@ int launch_top_p(const float* logits, int B, int V, float temperature, float top
     static bool attr = false;
     if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(top_p_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e == cudaSuccess) e = carveout_max(top_p_kernel);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(top_p_kernel)");
         attr = true;
     }
