@@ -37,8 +37,8 @@ WEIGHT_IDS = {"tok_embeddings": 0, "norm": 1, "output": 2, "attention_norm": 3, 
 EXPORTED = ("llama_model_bytes", "llama_model_create", "llama_set_weight", "llama_get_kv",
             "llama_prefill", "llama_decode_step", "llama_sample", "llama_model_status",
             "llama_model_destroy", "llama_last_error", "llama_launch_count",
-            "llama_op_rmsnorm", "llama_op_linear", "llama_op_linear_workspace_bytes", "llama_profile_start",
-            "llama_profile_stop")
+            "llama_op_rmsnorm", "llama_op_linear", "llama_op_linear_workspace_bytes", "llama_op_linear_noalloc",
+            "llama_profile_start", "llama_profile_stop")
 
 
 class LlamaError(RuntimeError):
@@ -88,6 +88,7 @@ _sig("llama_launch_count", ctypes.c_uint64, [])
 _sig("llama_op_rmsnorm", _i, [_vp, _vp, _i, _i, _f, _vp, _i, _vp])
 _sig("llama_op_linear", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp])
 _sig("llama_op_linear_workspace_bytes", _sz, [])
+_sig("llama_op_linear_noalloc", _i, [_vp, _vp, _i, _i, _i, _vp, _vp])
 _sig("llama_profile_start", _i, [_vp, _i])
 _sig("llama_profile_stop", _i, [_vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32), _i,
                                 ctypes.POINTER(ctypes.c_int)])
@@ -275,6 +276,15 @@ def op_linear_workspace(device):
     if key not in _op_ws:
         _op_ws[key] = torch.zeros(int(_lib.llama_op_linear_workspace_bytes()), dtype=torch.uint8, device=device)
     return _op_ws[key]
+
+
+def op_linear_noalloc(A, W, out, stream=None):
+    """bf16 projection out = A W^T (A: <= 16 rows) without any scratch from
+    the caller: for callers that cannot allocate device memory."""
+    M, K = A.shape
+    N = W.shape[0]
+    _check(_lib.llama_op_linear_noalloc(A.data_ptr(), W.data_ptr(), M, N, K, out.data_ptr(), _stream(stream)))
+    return out
 
 
 def op_linear(A, W, out, stream=None, workspace=None):

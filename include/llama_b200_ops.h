@@ -42,6 +42,29 @@ LLAMA_API size_t llama_op_linear_workspace_bytes(void);
 LLAMA_API int llama_op_linear(const void* A, const void* W, int M, int N, int K, int dtype,
                     float* out, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Allocation-free decode-shaped projection.  The source pages have no
+ * counterpart: it exists for callers that cannot allocate device memory --
+ * code running where cudaMalloc is not allowed (inside an allocator or memory
+ * pool owned by someone else, a locked-down process, a plug-in that must not
+ * touch the device heap) and so cannot provide the scratch workspace that
+ * llama_op_linear needs.
+ * Computes exactly what llama_op_linear computes for dtype LLAMA_BF16:
+ *   out[m,n] = sum_k A[m,k] * W[n,k], A bf16 [M, K], W bf16 [N, K], out fp32
+ *   [M, N] (device pointers owned by the caller), with the same persistent
+ *   weight-streaming kernel, but its split-tile scratch is a fixed array in
+ *   the library's device image (4 MiB + 16 KiB, held on every GPU that loads
+ *   the library until the process exits).  Nothing is allocated on any call.
+ * Limits: 1 <= M <= 16 token rows, N <= 4096 * 128, K a multiple of 8;
+ *   larger M or N returns LLAMA_ERR_CAPACITY with a message.
+ * The first call on a device, made with that device current, looks up the
+ *   array's device address (a host-side symbol lookup); make that first call
+ *   before any stream capture.  Every call clears the array's counters on
+ *   `stream` before its kernel.
+ * All calls share the one array: calls that overlap on the GPU (different
+ *   streams, or threads without ordering) race and give wrong results. */
+LLAMA_API int llama_op_linear_noalloc(const void* A, const void* W, int M, int N, int K, float* out,
+                                      void* stream);
+
 /* Per-launch timing of a model's projection kernels (for benchmarks).
  * llama_profile_start: from now on every projection launch the model enqueues
  *   (wq/wk/wv, wo, w1/w3, w2, output) is bracketed by two CUDA events recorded
