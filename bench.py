@@ -98,17 +98,6 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- roofline bookkeeping
 
-def launch_bytes(M, N, K, kind):
-    """Algorithmic bytes of one projection launch: the bf16 weight matrix once,
-    the bf16 input rows once, and the epilogue's output traffic."""
-    out = {0: 4 * M * N, 1: 8 * M * N, 2: 2 * M * N, 3: M * N}[kind]
-    return 2 * N * K + 2 * M * K + out
-
-
-def launch_flops(M, N, K, kind):
-    return 2 * M * N * K
-
-
 def decode_step_bytes(s, B, ctx):
     """Algorithmic bytes of one decode step of B rows at context ctx: every
     weight matrix once (bf16), the norm weights (fp32), B embedding rows, the
@@ -210,7 +199,7 @@ def run_ours(a, rank, world, local_rank):
     # bench step's prefill and first PROF_DECODE decode steps: events between
     # every launch would slow the whole region down.
     PROF_DECODE = 16
-    prof_cap = (5 * s.n_layers + 1) * (1 + PROF_DECODE)
+    prof_cap = (5 * s.n_layers + 1) * (1 + PROF_DECODE)   # an upper bound on projection launches
     model.profile_start(prof_cap)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(a.steps)]
     import tempfile
@@ -233,6 +222,25 @@ def run_ours(a, rank, world, local_rank):
     decode_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
     recs = model.profile_stop(prof_cap)
     assert model.status() == 0
+
+    # ---------------- second run: top-p 0.9 at temperature 0.6, seeded uniforms
+    # (one uniform per row per step; launched step by step, each with its row)
+    from workloads import make_uniforms, uniform_seed
+    uni = make_uniforms((steps_dec, B), uniform_seed(WL["index"])).to(dev)
+    tp_ev0 = torch.cuda.Event(enable_timing=True)
+    tp_ev1 = torch.cuda.Event(enable_timing=True)
+    model.prefill(prompt, logits=logits)
+    llb.sample(logits, WL["temperature"], WL["top_p"], uni[0], tok)
+    pos.copy_(pos_init)
+    torch.cuda.synchronize()
+    tp_ev0.record(stream)
+    for i in range(steps_dec):
+        model.decode_step(tok, pos, temperature=WL["temperature"], top_p=WL["top_p"], uniforms=uni[i],
+                          next_tokens=tok, advance=True)
+    tp_ev1.record(stream)
+    torch.cuda.synchronize()
+    assert model.status() == 0
+    top_p_tps = B * steps_dec / (tp_ev0.elapsed_time(tp_ev1) / 1e3)
 
     # ---------------- end to end through host buffers
     e2e_ev0 = torch.cuda.Event(enable_timing=True)
@@ -271,11 +279,11 @@ def run_ours(a, rank, world, local_rank):
     prefill_tps = pre_tokens / (prefill_ms / 1e3)
     e2e_value = dec_tokens / (e2e_dec_ms / 1e3)
 
-    dec = [r for r in recs if r[1] > 0 and r[0] > 0 and r[1] <= 64]
-    pre = [r for r in recs if r[0] > 0 and r[1] > 64]
-    dec_bytes = sum(launch_bytes(M, N, K, k) for _, M, N, K, k in dec)
+    dec = [r for r in recs if r[0] > 0 and 0 < r[3] <= 64]
+    pre = [r for r in recs if r[0] > 0 and r[3] > 64]
+    dec_bytes = sum(r[1] for r in dec)
     dec_ms = sum(r[0] for r in dec)
-    pre_flops = sum(launch_flops(M, N, K, k) for _, M, N, K, k in pre)
+    pre_flops = sum(r[2] for r in pre)
     pre_ms_k = sum(r[0] for r in pre)
     dec_gbs = dec_bytes / (dec_ms / 1e3) / 1e9 if dec_ms else 0.0
     pre_tfs = pre_flops / (pre_ms_k / 1e3) / 1e12 if pre_ms_k else 0.0
@@ -303,8 +311,10 @@ def run_ours(a, rank, world, local_rank):
                    "l2": "inputs larger than L2: each decode step streams 13.5 GB of weights (L2 126 MB)"},
         "prefill_tok_s": round(prefill_tps, 1),
         "decode_ms_per_token_step": round(decode_ms / (a.steps * steps_dec), 4),
+        "decode_top_p_tok_s": round(top_p_tps * world, 2),
+        "decode_top_p_what": "second run: temperature 0.6, top-p 0.9, seeded uniforms; steps launched one by one",
         "prefill_ms": round(prefill_ms / a.steps, 3),
-        "roofline": {"bound": "hbm", "kernel": "linear_tc_kernel (decode orientation: wqkv/wo/w13/w2/output)",
+        "roofline": {"bound": "hbm", "kernel": "linear_decode_kernel (decode projections: wq/wk/wv, wo, w1/w3, w2, output)",
                      "achieved": round(dec_gbs, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(dec_gbs / hbm, 4), "peak_source": f"{peak_src} hbm_gbs",
                      "traffic": None, "launches": len(dec)},
@@ -436,6 +446,121 @@ def run_op_linear(a):
                       "peak_source": peak_src}), flush=True)
 
 
+# ----------------------------------------------------------------------------- other workloads
+
+def _timed(fn, iters, stream):
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(iters):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / iters
+
+
+def run_workload(a):
+    """Throughput lines for the other workloads (one JSON line per measurement):
+    7b_layer_decode (one 7B layer, cache pre-filled, B x context grid),
+    13b_ragged (16 prompts of 64..1024 tokens, then 128 decode steps),
+    70b_slice (16 GQA layers, 8 x 2048 prefill, then decode), tiny_f32."""
+    import decoder_only_transformer_llama_b200 as llb
+    from workloads import make_lengths, make_normal
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    hbm, tc_burst, _, peak_src = _peaks()
+    name = a.workload
+    wl = WORKLOADS[name]
+    s = wl["shape"]
+    stream = torch.cuda.current_stream()
+    w = make_weights(s, weight_seed(wl["index"]), device=dev)
+    model = llb.Model(llb.args_from_shape(s), device=dev)
+    model.load(w)
+    del w
+    torch.cuda.empty_cache()
+    out = []
+    if name == "7b_layer_decode":
+        kv, vv = model.kv_tensors(0)
+        for L in wl["contexts"]:
+            kv[:, :L].copy_(make_normal(kv[:, :L].shape, 11, device=dev))
+            vv[:, :L].copy_(make_normal(vv[:, :L].shape, 12, device=dev))
+            for B in wl["batches"]:
+                tok = make_tokens(s.vocab_size, (B,), token_seed(wl["index"])).to(dev)
+                pos = torch.full((B,), L, dtype=torch.int32, device=dev)
+                lg = torch.empty(B, s.vocab_size, device=dev)
+                step = lambda: model.decode_step(tok, pos, logits=lg)
+                for _ in range(5):
+                    step()
+                g = torch.cuda.CUDAGraph()
+                sc = torch.cuda.Stream(device=dev)
+                sc.wait_stream(stream)
+                with torch.cuda.stream(sc):
+                    with torch.cuda.graph(g, stream=sc):
+                        step()
+                stream.wait_stream(sc)
+                torch.cuda.synchronize()
+                ms = _timed(g.replay, max(20, a.iters), stream)
+                byts = decode_step_bytes(s, B, L + 1)
+                out.append({"workload": name, "batch": B, "context": L + 1, "us_per_step": round(ms * 1e3, 2),
+                            "tok_s": round(B / (ms / 1e3), 1), "GB_s": round(byts / ms / 1e6, 1),
+                            "hbm_frac": round(byts / ms / 1e6 / hbm, 4), "peak_source": peak_src})
+                del g
+    else:
+        B = wl["batch"]
+        if name == "13b_ragged":
+            lens = make_lengths(B, wl["min_len"], wl["max_len"], token_seed(wl["index"]))
+            T = max(lens)
+            steps = wl["decode_steps"]
+        elif name == "70b_slice":
+            T = wl["prompt_len"]
+            lens = [T] * B
+            steps = a.decode_steps or (wl["decode_to"] - T)
+        else:
+            T = wl["prompt_len"]
+            lens = [T] * B
+            steps = wl["decode_steps"]
+        prompt = make_tokens(s.vocab_size, (B, T), token_seed(wl["index"])).to(dev)
+        logits = torch.empty(B, s.vocab_size, device=dev)
+        tok = torch.empty(B, dtype=torch.int32, device=dev)
+        pos0 = torch.tensor(lens, dtype=torch.int32, device=dev)
+        pos = pos0.clone()
+        for _ in range(2):
+            model.prefill(prompt, lens=lens, logits=logits)
+        torch.cuda.synchronize()
+        pre_ms = _timed(lambda: model.prefill(prompt, lens=lens, logits=logits), 3, stream)
+        llb.sample(logits, 0.0, 0.9, None, tok)
+        pos.copy_(pos0)
+        for _ in range(3):
+            model.decode_step(tok, pos, temperature=0.0, next_tokens=tok, advance=True)
+        pos.copy_(pos0)
+        torch.cuda.synchronize()
+        g = None
+        if s.dtype == "bf16":
+            g = torch.cuda.CUDAGraph()
+            sc = torch.cuda.Stream(device=dev)
+            sc.wait_stream(stream)
+            with torch.cuda.stream(sc):
+                with torch.cuda.graph(g, stream=sc):
+                    model.decode_step(tok, pos, temperature=0.0, next_tokens=tok, advance=True)
+            stream.wait_stream(sc)
+            pos.copy_(pos0)
+            torch.cuda.synchronize()
+        step = g.replay if g is not None else (lambda: model.decode_step(tok, pos, temperature=0.0,
+                                                                           next_tokens=tok, advance=True))
+        dec_ms = _timed(step, steps, stream)
+        assert model.status() == 0
+        n_tok = sum(lens)
+        mean_ctx = sum(lens) / B + steps / 2
+        byts = decode_step_bytes(s, B, int(mean_ctx)) if s.dtype == "bf16" else None
+        out.append({"workload": name, "batch": B, "prompt_tokens": n_tok, "prefill_ms": round(pre_ms, 3),
+                    "prefill_tok_s": round(n_tok / (pre_ms / 1e3), 1), "decode_steps": steps,
+                    "decode_ms_per_step": round(dec_ms, 4), "decode_tok_s": round(B / (dec_ms / 1e3), 1),
+                    "decode_hbm_frac": round(byts / dec_ms / 1e6 / hbm, 4) if byts else None,
+                    "peak_source": peak_src})
+        del g
+    for line in out:
+        print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------- main
 
 def main():
@@ -449,9 +574,15 @@ def main():
                     help="time one bf16 projection instead of the model (kernel microbenchmark)")
     ap.add_argument("--iters", type=int, default=50)
     ap.add_argument("--no-graph", action="store_true", help="launch decode steps directly instead of a CUDA graph")
+    ap.add_argument("--workload", default="7b", choices=list(WORKLOADS),
+                    help="7b is the headline line; the others print throughput lines of their own")
+    ap.add_argument("--decode-steps", type=int, default=0, help="decode steps of the 70b_slice workload")
     a = ap.parse_args()
     if a.op_linear:
         run_op_linear(a)
+        return
+    if a.workload != "7b":
+        run_workload(a)
         return
     if a.warmup < 3:
         a.warmup = 3

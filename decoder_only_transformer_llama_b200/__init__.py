@@ -90,7 +90,8 @@ _sig("llama_op_linear", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp])
 _sig("llama_op_linear_workspace_bytes", _sz, [])
 _sig("llama_op_linear_noalloc", _i, [_vp, _vp, _i, _i, _i, _vp, _vp])
 _sig("llama_profile_start", _i, [_vp, _i])
-_sig("llama_profile_stop", _i, [_vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int32), _i,
+_sig("llama_profile_stop", _i, [_vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int64),
+                                ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int32), _i,
                                 ctypes.POINTER(ctypes.c_int)])
 
 
@@ -238,12 +239,15 @@ class Model:
         _check(_lib.llama_profile_start(self.handle, capacity))
 
     def profile_stop(self, max_records: int):
-        """[(ms, M, N, K, kind)] of the projection launches timed since profile_start."""
+        """[(ms, algorithmic bytes, flops, token rows)] of the projection launches
+        timed since profile_start."""
         ms = (ctypes.c_float * max_records)()
-        sh = (ctypes.c_int32 * (4 * max_records))()
+        by = (ctypes.c_int64 * max_records)()
+        fl = (ctypes.c_int64 * max_records)()
+        rw = (ctypes.c_int32 * max_records)()
         n = ctypes.c_int()
-        _check(_lib.llama_profile_stop(self.handle, ms, sh, max_records, ctypes.byref(n)))
-        return [(ms[i], sh[4 * i], sh[4 * i + 1], sh[4 * i + 2], sh[4 * i + 3]) for i in range(n.value)]
+        _check(_lib.llama_profile_stop(self.handle, ms, by, fl, rw, max_records, ctypes.byref(n)))
+        return [(ms[i], by[i], fl[i], rw[i]) for i in range(n.value)]
 
     def status(self) -> int:
         s = ctypes.c_int()

@@ -147,6 +147,12 @@ static int make_maps(TmaMaps* t, const void* base, int rows, int cols, int b_box
     return LLAMA_OK;
 }
 
+static int64_t proj_bytes(int M, int N, int K, int mode) {
+    const int64_t mn = static_cast<int64_t>(M) * N;
+    const int64_t out = mode == EPI_STORE_F32 ? 4 * mn : mode == EPI_RESID_F32 ? 8 * mn : mode == EPI_QKV ? 2 * mn : mn;
+    return 2LL * N * K + 2LL * M * K + out;
+}
+
 int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, const void* W,
                const TmaMaps* mapW, int M, int N, int K, const Epi& ep, cudaStream_t st, bool pdl,
                const NormIO* nio, const NextProj* next) {
@@ -164,9 +170,9 @@ int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, co
     if (timed && rc == LLAMA_OK) {
         cudaError_t e = cudaEventRecord(pr->ev[2 * pr->n + 1], st);
         if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord(profile)");
-        const int kind = ep.mode == EPI_STORE_F32 ? 0 : ep.mode == EPI_RESID_F32 ? 1 : ep.mode == EPI_QKV ? 2 : 3;
-        int32_t* sh = &pr->shapes[4 * pr->n];
-        sh[0] = M; sh[1] = N; sh[2] = K; sh[3] = kind;
+        pr->bytes[pr->n] = proj_bytes(M, N, K, ep.mode);
+        pr->flops[pr->n] = 2LL * M * N * K;
+        pr->rows[pr->n] = M;
         pr->n++;
     }
     return rc;
@@ -175,7 +181,9 @@ int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, co
 static void profile_release(Profile& p) {
     for (cudaEvent_t e : p.ev) cudaEventDestroy(e);
     p.ev.clear();
-    p.shapes.clear();
+    p.bytes.clear();
+    p.flops.clear();
+    p.rows.clear();
     p.capacity = 0;
     p.n = 0;
 }
@@ -558,13 +566,15 @@ int llama_profile_start(llama_model* m, int capacity) {
             return cuda_fail(ce, "cudaEventCreate(profile)");
         }
     }
-    m->prof.shapes.assign(4 * static_cast<size_t>(capacity), 0);
+    m->prof.bytes.assign(static_cast<size_t>(capacity), 0);
+    m->prof.flops.assign(static_cast<size_t>(capacity), 0);
+    m->prof.rows.assign(static_cast<size_t>(capacity), 0);
     m->prof.capacity = capacity;
     m->prof.n = 0;
     return LLAMA_OK;
 }
 
-int llama_profile_stop(llama_model* m, float* ms, int32_t* shapes, int max, int* n) {
+int llama_profile_stop(llama_model* m, float* ms, int64_t* bytes, int64_t* flops, int32_t* rows, int max, int* n) {
     if (!m) { set_error("model is NULL"); return LLAMA_ERR_INVALID_ARG; }
     Profile& p = m->prof;
     const int cnt = p.n < max ? p.n : max;
@@ -575,7 +585,9 @@ int llama_profile_stop(llama_model* m, float* ms, int32_t* shapes, int max, int*
         if (e == cudaSuccess) e = cudaEventElapsedTime(&t, p.ev[2 * i], p.ev[2 * i + 1]);
         if (e != cudaSuccess) rc = cuda_fail(e, "profile events");
         if (ms) ms[i] = t;
-        if (shapes) for (int k = 0; k < 4; ++k) shapes[4 * i + k] = p.shapes[4 * i + k];
+        if (bytes) bytes[i] = p.bytes[i];
+        if (flops) flops[i] = p.flops[i];
+        if (rows) rows[i] = p.rows[i];
     }
     if (n) *n = cnt;
     profile_release(p);

@@ -50,8 +50,10 @@ template <> struct Vec<bf16, 4> {
 // chunks z, z+P, z+2P, ... of head g's positions 0 .. pos[b] for all n_rep
 // query heads of the group.  Each chunk of K and of V is one contiguous block
 // of the cache (the positions of one head are adjacent), fetched by one bulk
-// async copy into a two-deep shared-memory ring.  Warp w scores keys 2w,
-// 2w+1, 2w+8, ... of a chunk; lane l holds head dims [l*EPL, (l+1)*EPL).
+// async copy into a three-deep shared-memory ring.  Warp w scores keys
+// 16w .. 16w+15 of a chunk, eight at a time; lane l holds head dims
+// [l*EPL, (l+1)*EPL) and the eight partial dot products are summed across the
+// warp by a transposing butterfly (one full sum per lane, then broadcast).
 // The P CTAs of (b, g) with at least one chunk publish unnormalised partials
 // (o, max, sum); the one that arrives last at the (b, g) counter merges them in
 // CTA order.  With a single active CTA the output is written directly.
@@ -64,8 +66,9 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
     constexpr int EPL = HD / 32;   // head dims per lane
     constexpr int ROW = HD * static_cast<int>(sizeof(T));
     constexpr int CH_BYTES = kChunk * ROW;
+    constexpr int NSLOT = 3;
     extern __shared__ __align__(128) uint8_t dsm[];
-    __shared__ uint64_t bar[2];
+    __shared__ uint64_t bar[NSLOT];
     __shared__ float s_m[4][NREP], s_l[4][NREP];
     __shared__ float s_o[4][NREP][HD];
     __shared__ int s_last;
@@ -84,20 +87,18 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
     const int pact = min(P, nchunks);                  // CTAs of (b, g) with work
     const int mine = (nchunks - z + P - 1) / P;        // chunks of this CTA
     const long long head_off = static_cast<long long>(b) * row_stride + static_cast<long long>(g) * S * HD;
-    auto issue = [&](int i) {                          // i-th chunk of this CTA into ring slot i % 2
+    auto issue = [&](int i) {                          // i-th chunk of this CTA into ring slot i % NSLOT
         const int j0 = (z + i * P) * kChunk;
         const int n = min(kChunk, ctx - j0);
-        uint8_t* slot = dsm + (i & 1) * 2 * CH_BYTES;
-        mbar_arrive_expect_tx(&bar[i & 1], 2u * n * ROW);
-        bulk_load(slot, kc + head_off + static_cast<long long>(j0) * HD, n * ROW, &bar[i & 1]);
-        bulk_load(slot + CH_BYTES, vc + head_off + static_cast<long long>(j0) * HD, n * ROW, &bar[i & 1]);
+        uint8_t* slot = dsm + (i % NSLOT) * 2 * CH_BYTES;
+        mbar_arrive_expect_tx(&bar[i % NSLOT], 2u * n * ROW);
+        bulk_load(slot, kc + head_off + static_cast<long long>(j0) * HD, n * ROW, &bar[i % NSLOT]);
+        bulk_load(slot + CH_BYTES, vc + head_off + static_cast<long long>(j0) * HD, n * ROW, &bar[i % NSLOT]);
     };
     if (threadIdx.x == 0) {
-        mbar_init(&bar[0], 1);
-        mbar_init(&bar[1], 1);
+        for (int k = 0; k < NSLOT; ++k) mbar_init(&bar[k], 1);
         fence_mbar_init();
-        issue(0);
-        if (mine > 1) issue(1);
+        for (int k = 0; k < NSLOT && k < mine; ++k) issue(k);
     }
     const float scale = rsqrtf(static_cast<float>(HD));
     float qv[NREP][EPL];
@@ -118,41 +119,75 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
     __syncthreads();   // barriers initialised
     bool ok = true;
     for (int i = 0; i < mine && ok; ++i) {
-        ok = mbar_wait(&bar[i & 1], (i >> 1) & 1);
+        ok = mbar_wait(&bar[i % NSLOT], (i / NSLOT) & 1);
         if (!ok) break;
-        const T* sK = reinterpret_cast<const T*>(dsm + (i & 1) * 2 * CH_BYTES);
-        const T* sV = reinterpret_cast<const T*>(dsm + (i & 1) * 2 * CH_BYTES + CH_BYTES);
+        const T* sK = reinterpret_cast<const T*>(dsm + (i % NSLOT) * 2 * CH_BYTES);
+        const T* sV = reinterpret_cast<const T*>(dsm + (i % NSLOT) * 2 * CH_BYTES + CH_BYTES);
         const int n = min(kChunk, ctx - (z + i * P) * kChunk);
-        for (int jb = warp * 2; jb < n; jb += 8) {
-            float kv[2][EPL], vv[2][EPL];
+#pragma unroll 1
+        for (int jb = warp * 16; jb < min(n, warp * 16 + 16); jb += 8) {
+            // eight keys: this lane's partial dot products ...
+            float kv[8][EPL];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int j = min(jb + u, n - 1);
-                Vec<T, EPL>::load(sK + j * HD + lane * EPL, kv[u]);
-                Vec<T, EPL>::load(sV + j * HD + lane * EPL, vv[u]);
-            }
+            for (int u = 0; u < 8; ++u) Vec<T, EPL>::load(sK + min(jb + u, n - 1) * HD + lane * EPL, kv[u]);
 #pragma unroll
             for (int r = 0; r < NREP; ++r) {
-                float sc[2];
+                float d[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    d[u] = 0.f;
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) d[u] = fmaf(qv[r][e], kv[u][e], d[u]);
+                }
+                // ... summed by a transposing butterfly: after it, lane l holds the
+                // full dot of key 4*b4 + 2*b3 + b2 (b4, b3, b2 = bits 4, 3, 2 of l)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const bool hi = lane & 16;
+                    const float send = hi ? d[u] : d[u + 4];
+                    d[u] = (hi ? d[u + 4] : d[u]) + __shfl_xor_sync(0xffffffffu, send, 16);
+                }
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
-                    float d = 0.f;
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e) d = fmaf(qv[r][e], kv[u][e], d);
-                    sc[u] = warp_sum(d);
+                    const bool hi = lane & 8;
+                    const float send = hi ? d[u] : d[u + 2];
+                    d[u] = (hi ? d[u + 2] : d[u]) + __shfl_xor_sync(0xffffffffu, send, 8);
                 }
-                if (jb + 1 >= n) sc[1] = -INFINITY;
-                const float mnew = fmaxf(mx[r], fmaxf(sc[0], sc[1]));
-                const float corr = __expf(mx[r] - mnew);
-                const float p0 = __expf(sc[0] - mnew), p1 = __expf(sc[1] - mnew);
-                sl[r] = sl[r] * corr + p0 + p1;
+                {
+                    const bool hi = lane & 4;
+                    const float send = hi ? d[0] : d[1];
+                    d[0] = (hi ? d[1] : d[0]) + __shfl_xor_sync(0xffffffffu, send, 4);
+                }
+                d[0] += __shfl_xor_sync(0xffffffffu, d[0], 2);
+                d[0] += __shfl_xor_sync(0xffffffffu, d[0], 1);
+                float sc[8];
 #pragma unroll
-                for (int e = 0; e < EPL; ++e) o[r][e] = fmaf(p1, vv[1][e], fmaf(p0, vv[0][e], o[r][e] * corr));
+                for (int u = 0; u < 8; ++u) {
+                    sc[u] = __shfl_sync(0xffffffffu, d[0], ((u >> 2) << 4) | (((u >> 1) & 1) << 3) | ((u & 1) << 2));
+                    if (jb + u >= n) sc[u] = -INFINITY;
+                }
+                float mnew = mx[r];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) mnew = fmaxf(mnew, sc[u]);
+                const float corr = __expf(mx[r] - mnew);
+                float pj[8], ps = 0.f;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) { pj[u] = __expf(sc[u] - mnew); ps += pj[u]; }
+                sl[r] = sl[r] * corr + ps;
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) o[r][e] *= corr;
                 mx[r] = mnew;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    float vv[EPL];
+                    Vec<T, EPL>::load(sV + min(jb + u, n - 1) * HD + lane * EPL, vv);
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) o[r][e] = fmaf(pj[u], vv[e], o[r][e]);
+                }
             }
         }
-        __syncthreads();                               // ring slot i % 2 is free again
-        if (threadIdx.x == 0 && i + 2 < mine) issue(i + 2);
+        __syncthreads();                               // ring slot i % NSLOT is free again
+        if (threadIdx.x == 0 && i + NSLOT < mine) issue(i + NSLOT);
     }
     if (!ok && threadIdx.x == 0) report_status(status, LLAMA_ERR_DEVICE_TIMEOUT);
 
@@ -222,7 +257,7 @@ static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaS
     const T* kc = static_cast<const T*>(m->kc) + layer * m->kv_layer_elems;
     const T* vc = static_cast<const T*>(m->vc) + layer * m->kv_layer_elems;
     auto kern = attn_decode_kernel<T, HD, NREP>;
-    const int smem = 4 * kChunk * HD * static_cast<int>(sizeof(T));
+    const int smem = 3 * 2 * kChunk * HD * static_cast<int>(sizeof(T));   // three K+V chunks
     static bool attr = false;
     if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

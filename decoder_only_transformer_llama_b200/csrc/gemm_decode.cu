@@ -41,6 +41,7 @@ constexpr int kThreads = 192;
 constexpr int kAccStride = 64;      // TMEM columns per accumulator buffer
 constexpr int kTmemCols = 128;      // two accumulator buffers
 constexpr int kABytes = 128 * 128;  // 128 weight rows x 64 bf16
+constexpr int kL2Ahead = 16;        // units pulled into L2 beyond the ring at kernel start
 
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(n) : "memory"); }
 // OR of `v` over the `n` threads of named barrier `id` (they all block).
@@ -131,6 +132,16 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
             mbar_arrive_expect_tx(&full[i], STAGE);
             tma_load_2d(smem + i * STAGE, &mapW, kk * 64, tt * 128, &full[i]);
             if (++kk == KT) { kk = 0; ++tt; }
+        }
+        {
+            // before waiting for the previous kernel, also pull the units after the
+            // ring into L2, so that HBM keeps streaming through that kernel's tail
+            const int nl = min(nunits - npre, kL2Ahead);
+            int tl = tt, kl = kk;
+            for (int i = 0; i < nl; ++i) {
+                tma_prefetch_l2(&mapW, kl * 64, tl * 128);
+                if (++kl == KT) { kl = 0; ++tl; }
+            }
         }
         pdl_wait();
         tt = t0;
@@ -294,45 +305,63 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
                 }
             } else if (ep.mode == EPI_QKV) {
                 const bool even = (lane & 1) == 0;
+                const bool is_q = n < ep.nq;
+                int cc = n - ep.nq;
+                bf16* cache = static_cast<bf16*>(ep.kc);
+                const bool is_k = !is_q && cc < ep.nkvc;
+                if (!is_q && !is_k) { cc -= ep.nkvc; cache = static_cast<bf16*>(ep.vc); }
+                const int d = is_q ? n % ep.hd : cc % ep.hd;
+                const int head = is_q ? 0 : cc / ep.hd;
+                // per group of 16 columns: all positions and RoPE factors first
+                // (independent loads), then the rotations and stores
 #pragma unroll
-                for (int b = 0; b < BN; ++b) {
-                    const float partner = __shfl_xor_sync(0xffffffffu, v[b], 1);
-                    if (!row_ok || b >= nb) continue;
-                    const int pos = ep.tok_pos[b];
-                    if (pos < 0 || pos >= ep.max_seq) continue;
-                    float re = even ? v[b] : partner, im = even ? partner : v[b];
-                    if (n < ep.nq) {
-                        rope_pair(ep.rope, ep.hd, pos, (n % ep.hd) >> 1, re, im);
-                        static_cast<bf16*>(ep.q)[static_cast<long long>(b) * ep.nq + n] =
-                            __float2bfloat16_rn(even ? re : im);
-                    } else {
-                        int cc = n - ep.nq;
-                        bf16* cache = static_cast<bf16*>(ep.kc);
-                        const bool is_k = cc < ep.nkvc;
-                        if (!is_k) { cc -= ep.nkvc; cache = static_cast<bf16*>(ep.vc); }
-                        const int head = cc / ep.hd, d = cc % ep.hd;
-                        float val = v[b];
-                        if (is_k) {
-                            rope_pair(ep.rope, ep.hd, pos, d >> 1, re, im);
-                            val = even ? re : im;
+                for (int b0 = 0; b0 < BN; b0 += 16) {
+                    int posv[16];
+                    float2 cs[16];
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) posv[u] = (b0 + u < nb) ? ep.tok_pos[b0 + u] : -1;
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const bool okp = row_ok && posv[u] >= 0 && posv[u] < ep.max_seq && (is_q || is_k);
+                        cs[u] = okp ? ep.rope[static_cast<long long>(posv[u]) * (ep.hd / 2) + (d >> 1)]
+                                    : make_float2(1.f, 0.f);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const int b = b0 + u;
+                        const float partner = __shfl_xor_sync(0xffffffffu, v[b], 1);
+                        const int pos = posv[u];
+                        if (!row_ok || b >= nb || pos < 0 || pos >= ep.max_seq) continue;
+                        const float re = even ? v[b] : partner, im = even ? partner : v[b];
+                        const float rot = even ? re * cs[u].x - im * cs[u].y : re * cs[u].y + im * cs[u].x;
+                        if (is_q) {
+                            static_cast<bf16*>(ep.q)[static_cast<long long>(b) * ep.nq + n] = __float2bfloat16_rn(rot);
+                        } else {
+                            const int row = ep.tok_row ? ep.tok_row[b] : b;
+                            cache[static_cast<long long>(row) * ep.kv_row_stride +
+                                  (static_cast<long long>(head) * ep.max_seq + pos) * ep.hd + d] =
+                                __float2bfloat16_rn(is_k ? rot : v[b]);
                         }
-                        const int row = ep.tok_row ? ep.tok_row[b] : b;
-                        cache[static_cast<long long>(row) * ep.kv_row_stride +
-                              (static_cast<long long>(head) * ep.max_seq + pos) * ep.hd + d] = __float2bfloat16_rn(val);
                     }
                 }
             } else if (ep.mode == EPI_RESID_F32 && nio.ssq_out) {
-                // residual add, plus this tile's share of sum(x^2) for the next RMSNorm
+                // residual add, plus this tile's share of sum(x^2) for the next RMSNorm;
+                // the old x values of a 16-column group are loaded together
+                const float wn = row_ok ? nio.w_next[n] : 0.f;
+                float xo[16];
 #pragma unroll
                 for (int b = 0; b < BN; ++b) {
+                    if ((b & 15) == 0) {
+#pragma unroll
+                        for (int u = 0; u < 16; ++u)
+                            xo[u] = (row_ok && b + u < nb) ? ep.out[static_cast<long long>(b + u) * ep.ldo + n] : 0.f;
+                    }
                     float sq = 0.f;
                     if (row_ok && b < nb) {
-                        float* o = ep.out + static_cast<long long>(b) * ep.ldo + n;
-                        const float nv = *o + v[b];
-                        *o = nv;
+                        const float nv = xo[b & 15] + v[b];
+                        ep.out[static_cast<long long>(b) * ep.ldo + n] = nv;
+                        static_cast<bf16*>(nio.y_out)[static_cast<long long>(b) * ep.ldo + n] = __float2bfloat16_rn(nv * wn);
                         sq = nv * nv;
-                        static_cast<bf16*>(nio.y_out)[static_cast<long long>(b) * ep.ldo + n] =
-                            __float2bfloat16_rn(nv * nio.w_next[n]);
                     }
                     sq = warp_sum(sq);
                     if (lane == 0) red[q * 64 + b] = sq;
@@ -343,12 +372,21 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
                                                    red[192 + epi_tid];
                 named_sync(2, 128);
             } else if (row_ok) {
+                if (ep.mode == EPI_RESID_F32) {
 #pragma unroll
-                for (int b = 0; b < BN; ++b) {
-                    if (b >= nb) continue;
-                    float* o = ep.out + static_cast<long long>(b) * ep.ldo + n;
-                    if (ep.mode == EPI_RESID_F32) *o += v[b];
-                    else *o = v[b];
+                    for (int b0 = 0; b0 < BN; b0 += 16) {
+                        float xo[16];
+#pragma unroll
+                        for (int u = 0; u < 16; ++u)
+                            xo[u] = (b0 + u < nb) ? ep.out[static_cast<long long>(b0 + u) * ep.ldo + n] : 0.f;
+#pragma unroll
+                        for (int u = 0; u < 16; ++u)
+                            if (b0 + u < nb) ep.out[static_cast<long long>(b0 + u) * ep.ldo + n] = xo[u] + v[b0 + u];
+                    }
+                } else {
+#pragma unroll
+                    for (int b = 0; b < BN; ++b)
+                        if (b < nb) ep.out[static_cast<long long>(b) * ep.ldo + n] = v[b];
                 }
             }
         }

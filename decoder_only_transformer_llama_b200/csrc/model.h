@@ -94,7 +94,9 @@ struct Profile {
     int capacity = 0;
     int n = 0;
     std::vector<cudaEvent_t> ev;     // 2 per launch
-    std::vector<int32_t> shapes;     // 4 per launch
+    std::vector<int64_t> bytes;      // algorithmic bytes per launch
+    std::vector<int64_t> flops;      // flops per launch
+    std::vector<int32_t> rows;       // token rows (M) per launch
 };
 
 struct Model {

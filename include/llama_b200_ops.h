@@ -68,14 +68,17 @@ LLAMA_API int llama_op_linear_noalloc(const void* A, const void* W, int M, int N
 /* Per-launch timing of a model's projection kernels (for benchmarks).
  * llama_profile_start: from now on every projection launch the model enqueues
  *   (wq/wk/wv, wo, w1/w3, w2, output) is bracketed by two CUDA events recorded
- *   on the launch's own stream, for the first `capacity` launches.
+ *   on the launch's own stream, for the first `capacity` launches.  Timed
+ *   launches do not overlap their neighbours (no early launch).
  * llama_profile_stop: synchronises the events, writes up to `max` records
- *   (host arrays): ms[i] = duration of launch i, shapes[4*i..4*i+3] = (M, N, K,
- *   epilogue: 0 logits, 1 residual, 2 qkv+rope+cache, 3 silu*mul), sets *n to
- *   the number of timed launches and stops timing.  Events are created by
- *   start and destroyed by stop (or by llama_model_destroy). */
+ *   (host arrays, any may be NULL): ms[i] = duration of launch i, bytes[i] =
+ *   its algorithmic bytes (every weight once, the bf16 input rows once, the
+ *   epilogue's outputs), flops[i] = 2*M*N*K summed over its projections,
+ *   rows[i] = M; sets *n to the number of timed launches and stops timing.
+ *   Events are created by start and destroyed by stop or llama_model_destroy. */
 LLAMA_API int llama_profile_start(llama_model* m, int capacity);
-LLAMA_API int llama_profile_stop(llama_model* m, float* ms, int32_t* shapes, int max, int* n);
+LLAMA_API int llama_profile_stop(llama_model* m, float* ms, int64_t* bytes, int64_t* flops, int32_t* rows, int max,
+                                 int* n);
 
 #ifdef __cplusplus
 }
