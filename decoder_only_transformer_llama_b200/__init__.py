@@ -291,6 +291,18 @@ def op_linear_noalloc(A, W, out, stream=None):
     return out
 
 
+def op_linear_whole_tiles(A, W, out, stream=None):
+    """bf16 projection with M > 64 and no workspace: every tile runs whole
+    (no stream-K split of the last wave)."""
+    M, K = A.shape
+    N = W.shape[0]
+    if M <= 64:
+        raise ValueError("op_linear_whole_tiles takes M > 64 token rows")
+    _check(_lib.llama_op_linear(A.data_ptr(), W.data_ptr(), M, N, K, LLAMA_BF16, out.data_ptr(), None, 0,
+                                _stream(stream)))
+    return out
+
+
 def op_linear(A, W, out, stream=None, workspace=None):
     M, K = A.shape
     N = W.shape[0]

@@ -128,13 +128,13 @@ static int make_layout(const llama_model_args* a, Layout* o) {
     l.off_tok_pos = off; off = align256(off + M * 4);
     l.off_last = off; off = align256(off + Bn * 4);
     l.off_logits = off; off = align256(off + static_cast<size_t>(l.Bmax) * l.V * 4);
-    const size_t slots = static_cast<size_t>(l.Bmax) * l.nh * l.n_splits;
+    const size_t slots = static_cast<size_t>(2) * kMaxAttnCtas * n_rep;   // decode attention partials
     l.off_part_o = off; off = align256(off + slots * hd * 4);
     l.off_part_ml = off; off = align256(off + slots * 2 * 4);
     l.off_attn_cnt = off; off = align256(off + static_cast<size_t>(l.Bmax) * nkv * 4);
     l.off_status = off; off = align256(off + 16);
     l.off_rope = off; off = align256(off + static_cast<size_t>(l.S) * (hd / 2) * 8);
-    l.off_gemm_part = off; off = align256(off + (a->dtype == LLAMA_BF16 ? kDecodePartBytes : 0));
+    l.off_gemm_part = off; off = align256(off + (a->dtype == LLAMA_BF16 ? kGemmPartBytes : 0));
     l.off_gemm_cnt = off; off = align256(off + kMaxTiles * sizeof(int));
     l.off_ssq = off; off = align256(off + static_cast<size_t>(l.Bmax) * (l.dim / 128 + 1) * 4);
     l.ws_end = off;
@@ -155,7 +155,7 @@ static int64_t proj_bytes(int M, int N, int K, int mode) {
 
 int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, const void* W,
                const TmaMaps* mapW, int M, int N, int K, const Epi& ep, cudaStream_t st, bool pdl,
-               const NormIO* nio, const NextProj* next) {
+               const NormIO* nio) {
     Profile* pr = const_cast<Profile*>(&m->prof);
     const bool timed = pr->n < pr->capacity;
     if (timed) {
@@ -166,7 +166,7 @@ int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, co
     if (dtype == LLAMA_F32)
         rc = linear_f32(static_cast<const float*>(A), static_cast<const float*>(W), M, N, K, ep, st);
     else
-        rc = linear_bf16(mapA, mapW, M, N, K, ep, m->gemm_part, m->gemm_cnt, st, pdl && !timed, nio, next);
+        rc = linear_bf16(mapA, mapW, M, N, K, ep, m->gemm_part, kGemmPartBytes, m->gemm_cnt, st, pdl && !timed, nio);
     if (timed && rc == LLAMA_OK) {
         cudaError_t e = cudaEventRecord(pr->ev[2 * pr->n + 1], st);
         if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord(profile)");
@@ -481,14 +481,8 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B
             ep.vc = static_cast<char*>(m->vc) + l * m->kv_layer_elems * m->esz;
             ep.tok_pos = pos;
             const NormIO n_in = {m->ssq, nb, eps, nullptr, nullptr, nullptr};
-            // each projection warms L2 with the first weight tiles of the next one
-            const NextProj nx_wo = {&Lp.m_wo.a128, m->dim, m->nq};
-            const NextProj nx_w13 = {&Lp.m_w13.a128, 2 * m->H, m->dim};
-            const NextProj nx_w2 = {&Lp.m_w2.a128, m->dim, m->H};
-            const NextProj nx_after = l + 1 < m->L ? NextProj{&m->layers[l + 1].m_wqkv.a128, m->nqkv, m->dim}
-                                                    : NextProj{&m->m_output.a128, m->V, m->dim};
             LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.wqkv, &Lp.m_wqkv, B, m->nqkv, m->dim, ep, st, true,
-                               &n_in, &nx_wo));
+                               &n_in));
             LLB_TRY(launch_attention_decode(m, l, pos, B, st, true));
             Epi er = base_epi(m);
             er.mode = EPI_RESID_F32;
@@ -496,15 +490,15 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B
             er.ldo = m->dim;
             const NormIO n_to_ffn = {nullptr, 0, 0.f, m->ssq, m->y, Lp.ffn_norm};
             LLB_TRY(run_linear(m, m->dtype, m->attn, &m->m_attn, Lp.wo, &Lp.m_wo, B, m->dim, m->nq, er, st, true,
-                               &n_to_ffn, &nx_w13));
+                               &n_to_ffn));
             Epi es = base_epi(m);
             es.mode = EPI_SWIGLU;
             es.g = m->g;
             LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.w13, &Lp.m_w13, B, 2 * m->H, m->dim, es, st, true,
-                               &n_in, &nx_w2));
+                               &n_in));
             const NormIO n_to_next = {nullptr, 0, 0.f, m->ssq, m->y, next_norm};
             LLB_TRY(run_linear(m, m->dtype, m->g, &m->m_g, Lp.w2, &Lp.m_w2, B, m->dim, m->H, er, st, true,
-                               &n_to_next, &nx_after));
+                               &n_to_next));
         }
         const NormIO n_in = {m->ssq, nb, eps, nullptr, nullptr, nullptr};
         LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, m->output, &m->m_output, B, m->V, m->dim, eo, st, true,
@@ -602,7 +596,7 @@ int llama_op_rmsnorm(const float* x, const float* w, int M, int dim, float eps, 
     return launch_rmsnorm(x, nullptr, w, M, dim, eps, out, out_dtype, static_cast<cudaStream_t>(stream));
 }
 
-size_t llama_op_linear_workspace_bytes(void) { return kDecodePartBytes + kMaxTiles * sizeof(int); }
+size_t llama_op_linear_workspace_bytes(void) { return kGemmPartBytes + kMaxTiles * sizeof(int); }
 
 int llama_op_linear(const void* A, const void* W, int M, int N, int K, int dtype, float* out, void* workspace,
                     size_t workspace_bytes, void* stream) {
@@ -618,9 +612,10 @@ int llama_op_linear(const void* A, const void* W, int M, int N, int K, int dtype
     if (dtype != LLAMA_BF16) { set_error("bad dtype"); return LLAMA_ERR_INVALID_ARG; }
     if (K % 8) { set_error("bf16 linear needs K %% 8 == 0"); return LLAMA_ERR_INVALID_ARG; }
     if ((N + 127) / 128 > kMaxTiles) { set_error("N too large"); return LLAMA_ERR_INVALID_ARG; }
-    if (M <= 64 && (!workspace || workspace_bytes < llama_op_linear_workspace_bytes() ||
-                    (reinterpret_cast<uintptr_t>(workspace) & 255))) {
-        set_error("bf16 linear with M <= 64 needs a 256-byte aligned workspace of llama_op_linear_workspace_bytes()");
+    if ((M <= 64 || workspace) && (!workspace || workspace_bytes < llama_op_linear_workspace_bytes() ||
+                                   (reinterpret_cast<uintptr_t>(workspace) & 255))) {
+        set_error("bf16 linear needs a 256-byte aligned workspace of llama_op_linear_workspace_bytes() "
+                  "(optional only for M > 64)");
         return LLAMA_ERR_INVALID_ARG;
     }
     if (M == 0) return LLAMA_OK;
@@ -630,8 +625,8 @@ int llama_op_linear(const void* A, const void* W, int M, int N, int K, int dtype
     LLB_TRY(encode_kmajor_bf16(&mw.a128, W, N, K, 128));
     LLB_TRY(encode_kmajor_bf16(&mw.b, W, N, K, 256));
     float* part = static_cast<float*>(workspace);
-    int* cnt = workspace ? reinterpret_cast<int*>(static_cast<char*>(workspace) + kDecodePartBytes) : nullptr;
-    return linear_bf16(&ma, &mw, M, N, K, ep, part, cnt, st);
+    int* cnt = workspace ? reinterpret_cast<int*>(static_cast<char*>(workspace) + kGemmPartBytes) : nullptr;
+    return linear_bf16(&ma, &mw, M, N, K, ep, part, part ? kGemmPartBytes : 0, cnt, st);
 }
 
 }  // extern "C"

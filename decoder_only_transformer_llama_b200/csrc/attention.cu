@@ -46,21 +46,37 @@ template <> struct Vec<bf16, 4> {
 };
 
 // ---------------------------------------------------------------- decode
-// Flash-decoding over the cache: CTA (z, kv head g, row b) walks the 64-key
-// chunks z, z+P, z+2P, ... of head g's positions 0 .. pos[b] for all n_rep
-// query heads of the group.  Each chunk of K and of V is one contiguous block
-// of the cache (the positions of one head are adjacent), fetched by one bulk
-// async copy into a three-deep shared-memory ring.  Warp w scores keys
-// 16w .. 16w+15 of a chunk, eight at a time; lane l holds head dims
-// [l*EPL, (l+1)*EPL) and the eight partial dot products are summed across the
-// warp by a transposing butterfly (one full sum per lane, then broadcast).
-// The P CTAs of (b, g) with at least one chunk publish unnormalised partials
-// (o, max, sum); the one that arrives last at the (b, g) counter merges them in
-// CTA order.  With a single active CTA the output is written directly.
+// Flash-decoding over the cache as one persistent, balanced pass.  The work
+// is a flat list of units, one unit = 64 consecutive key positions of one
+// (row b, KV head g) pair, pairs in (b, g) order; pair (b, g) has
+// ceil((pos[b] + 1) / 64) units.  Each of the P CTAs (as many as fit on the
+// GPU at once) takes an equal contiguous run of the list, so every CTA reads
+// the same number of cache bytes whatever the mix of context lengths, and all
+// CTAs run in one wave.  A run is cut into segments at pair boundaries.
+//
+// Each unit's K and V blocks are contiguous in the cache (the positions of one
+// head are adjacent) and are fetched by bulk async copies into a three-deep
+// shared-memory ring that runs across segments.  Warp w scores keys
+// 16w .. 16w+15 of a unit, eight at a time, for all n_rep query heads of the
+// group; lane l holds head dims [l*EPL, (l+1)*EPL) and the eight partial dot
+// products are summed across the warp by a transposing butterfly (one full
+// sum per lane, then broadcast).  Online softmax state (max, sum, o) is kept
+// per warp and merged across the 4 warps at the end of a segment.
+//
+// A segment that covers its whole pair writes the output row directly.  A pair
+// split between CTAs has at most one partial segment per CTA at each end of
+// its run (slot 0 = the run's first segment, slot 1 = its last); each writes
+// its unnormalised (o, max, sum) and the CTA that arrives last at the pair's
+// counter merges them in CTA order (deterministic).  No CTA waits for another.
+__device__ __forceinline__ long long run_begin64(long long c, long long W, long long P) { return c * W / P; }
+__device__ __forceinline__ int owner64(long long u, long long W, long long P) {
+    return static_cast<int>(((u + 1) * P - 1) / W);
+}
+
 template <typename T, int HD, int NREP>
 __global__ void __launch_bounds__(128)
 attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
-                   const int32_t* __restrict__ pos, int nq, int S, long long row_stride,
+                   const int32_t* __restrict__ pos, int B, int nkv, int nq, int S, long long row_stride,
                    float* __restrict__ part_o, float* __restrict__ part_ml, int* __restrict__ counters,
                    T* __restrict__ out, int* status) {
     constexpr int EPL = HD / 32;   // head dims per lane
@@ -71,59 +87,175 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
     __shared__ uint64_t bar[NSLOT];
     __shared__ float s_m[4][NREP], s_l[4][NREP];
     __shared__ float s_o[4][NREP][HD];
+    __shared__ int s_cum[kMaxRows + 1];   // units before row b, in units of one pair's chunks
+    __shared__ int s_nch[kMaxRows];       // chunks of each pair of row b (0: row skipped)
+    __shared__ int s_pos[kMaxRows];       // position of row b's query
+    __shared__ int s_wsum[4];
     __shared__ int s_last;
     pdl_trigger();
-    pdl_wait();
-    const int z = blockIdx.x, P = gridDim.x, g = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int p = pos[b];
-    if (p < 0 || p >= S) {
-        if (z == 0 && g == 0 && threadIdx.x == 0) report_status(status, LLAMA_ERR_CAPACITY);
-        return;
+
+    // ---- chunks per row and their prefix sums (rows in order, 2 per thread)
+    int my_pos[2] = {-1, -1};
+    auto make_plan = [&]() {
+        int v[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int b = 2 * threadIdx.x + e;
+            int n = 0;
+            if (b < B) {
+                const int p = __ldcg(pos + b);   // L2: read again after the grid dependency resolves
+                my_pos[e] = p;
+                if (p >= 0 && p < S) n = (p + kChunk) / kChunk;
+                s_nch[b] = n;
+                s_pos[b] = p;
+            }
+            v[e] = n;
+        }
+        const int t = v[0] + v[1];
+        int incl = t;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) s_wsum[warp] = incl;
+        __syncthreads();
+        int before = incl - t;
+        for (int w = 0; w < warp; ++w) before += s_wsum[w];
+        const int b0 = 2 * threadIdx.x;
+        if (threadIdx.x == 0) s_cum[0] = 0;
+        if (b0 + 1 <= B) s_cum[b0 + 1] = before + v[0];
+        if (b0 + 2 <= B) s_cum[b0 + 2] = before + t;
+        __syncthreads();
+    };
+    // Before the previous kernel (which writes this step's K/V row and q) has
+    // finished: plan with the positions as they read now and pull this CTA's
+    // cache blocks into L2 (a prefetch only: nothing read here is used, and L2
+    // is coherent with the writes that follow).  After the grid dependency has
+    // resolved, the positions are read again and the plan is redone if any
+    // changed.
+    make_plan();
+    {
+        const long long W0 = static_cast<long long>(s_cum[B]) * nkv;
+        const int P0 = static_cast<int>(W0 < gridDim.x ? W0 : gridDim.x);
+        if (threadIdx.x == 0 && blockIdx.x < P0) {
+            const long long v0 = run_begin64(blockIdx.x, W0, P0), v1 = run_begin64(blockIdx.x + 1, W0, P0);
+            int lo = 0, hi = B - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (static_cast<long long>(s_cum[mid]) * nkv <= v0) lo = mid; else hi = mid - 1;
+            }
+            int b = lo;
+            long long rem = v0 - static_cast<long long>(s_cum[lo]) * nkv;
+            int g = static_cast<int>(rem / s_nch[b]);
+            int jj = static_cast<int>(rem - static_cast<long long>(g) * s_nch[b]);
+            for (long long u = v0; u < v1 && b < B; ++u) {
+                const int ctx = s_pos[b] + 1;
+                const int j0 = jj * kChunk;
+                const int n = min(kChunk, ctx - j0);
+                if (n > 0) {
+                    const long long ho = static_cast<long long>(b) * row_stride + static_cast<long long>(g) * S * HD +
+                                         static_cast<long long>(j0) * HD;
+                    bulk_prefetch_l2(kc + ho, n * ROW);
+                    bulk_prefetch_l2(vc + ho, n * ROW);
+                }
+                if (++jj >= s_nch[b]) {
+                    jj = 0;
+                    if (++g >= nkv) { g = 0; do { ++b; } while (b < B && s_nch[b] == 0); }
+                }
+            }
+        }
     }
-    const int ctx = p + 1;
-    const int nchunks = (ctx + kChunk - 1) / kChunk;
-    if (z >= nchunks) return;
-    const int pact = min(P, nchunks);                  // CTAs of (b, g) with work
-    const int mine = (nchunks - z + P - 1) / P;        // chunks of this CTA
-    const long long head_off = static_cast<long long>(b) * row_stride + static_cast<long long>(g) * S * HD;
-    auto issue = [&](int i) {                          // i-th chunk of this CTA into ring slot i % NSLOT
-        const int j0 = (z + i * P) * kChunk;
+    pdl_wait();
+    {
+        bool changed = false;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int b = 2 * threadIdx.x + e;
+            if (b < B) {
+                const int p = __ldcg(pos + b);
+                changed |= p != my_pos[e];
+                if ((p < 0 || p >= S) && blockIdx.x == 0) report_status(status, LLAMA_ERR_CAPACITY);
+            }
+        }
+        if (__syncthreads_or(changed)) make_plan();
+    }
+    const long long W = static_cast<long long>(s_cum[B]) * nkv;
+    const int P = static_cast<int>(W < gridDim.x ? W : gridDim.x), c = blockIdx.x;
+    if (c >= P) return;
+    const long long u0 = run_begin64(c, W, P), u1 = run_begin64(c + 1, W, P);
+    const int len = static_cast<int>(u1 - u0);
+
+    // cursor over (row, kv head, chunk) starting at unit u
+    struct Cur { int b, g, j; };
+    auto cur_at = [&](long long u) {
+        int lo = 0, hi = B - 1;                  // largest b with s_cum[b] * nkv <= u
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (static_cast<long long>(s_cum[mid]) * nkv <= u) lo = mid; else hi = mid - 1;
+        }
+        Cur r;
+        r.b = lo;
+        const long long rem = u - static_cast<long long>(s_cum[lo]) * nkv;
+        r.g = static_cast<int>(rem / s_nch[lo]);
+        r.j = static_cast<int>(rem - static_cast<long long>(r.g) * s_nch[lo]);
+        return r;
+    };
+    auto advance = [&](Cur& r) {
+        if (++r.j < s_nch[r.b]) return;
+        r.j = 0;
+        if (++r.g < nkv) return;
+        r.g = 0;
+        do { ++r.b; } while (r.b < B && s_nch[r.b] == 0);
+    };
+    auto head_off = [&](const Cur& r) {
+        return static_cast<long long>(r.b) * row_stride + static_cast<long long>(r.g) * S * HD;
+    };
+    Cur icur = cur_at(u0);                       // issue cursor (thread 0)
+    auto issue = [&](int i) {                    // i-th unit of this run into ring slot i % NSLOT
+        const int ctx = s_pos[icur.b] + 1;
+        const int j0 = icur.j * kChunk;
         const int n = min(kChunk, ctx - j0);
         uint8_t* slot = dsm + (i % NSLOT) * 2 * CH_BYTES;
+        const long long ho = head_off(icur);
         mbar_arrive_expect_tx(&bar[i % NSLOT], 2u * n * ROW);
-        bulk_load(slot, kc + head_off + static_cast<long long>(j0) * HD, n * ROW, &bar[i % NSLOT]);
-        bulk_load(slot + CH_BYTES, vc + head_off + static_cast<long long>(j0) * HD, n * ROW, &bar[i % NSLOT]);
+        bulk_load(slot, kc + ho + static_cast<long long>(j0) * HD, n * ROW, &bar[i % NSLOT]);
+        bulk_load(slot + CH_BYTES, vc + ho + static_cast<long long>(j0) * HD, n * ROW, &bar[i % NSLOT]);
+        advance(icur);
     };
     if (threadIdx.x == 0) {
         for (int k = 0; k < NSLOT; ++k) mbar_init(&bar[k], 1);
         fence_mbar_init();
-        for (int k = 0; k < NSLOT && k < mine; ++k) issue(k);
+        for (int k = 0; k < NSLOT && k < len; ++k) issue(k);
     }
     const float scale = rsqrtf(static_cast<float>(HD));
+    Cur cur = cur_at(u0);
     float qv[NREP][EPL];
-#pragma unroll
-    for (int r = 0; r < NREP; ++r) {
-        Vec<T, EPL>::load(q + static_cast<long long>(b) * nq + (g * NREP + r) * HD + lane * EPL, qv[r]);
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) qv[r][e] *= scale;
-    }
     float mx[NREP], sl[NREP], o[NREP][EPL];
+    auto start_pair = [&]() {
 #pragma unroll
-    for (int r = 0; r < NREP; ++r) {
-        mx[r] = -INFINITY;
-        sl[r] = 0.f;
+        for (int r = 0; r < NREP; ++r) {
+            Vec<T, EPL>::load(q + static_cast<long long>(cur.b) * nq + (cur.g * NREP + r) * HD + lane * EPL, qv[r]);
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) o[r][e] = 0.f;
-    }
+            for (int e = 0; e < EPL; ++e) qv[r][e] *= scale;
+            mx[r] = -INFINITY;
+            sl[r] = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) o[r][e] = 0.f;
+        }
+    };
+    start_pair();
     __syncthreads();   // barriers initialised
     bool ok = true;
-    for (int i = 0; i < mine && ok; ++i) {
+    int seg_j0 = cur.j, seg_i0 = 0;
+    for (int i = 0; i < len; ++i) {
         ok = mbar_wait(&bar[i % NSLOT], (i / NSLOT) & 1);
         if (!ok) break;
         const T* sK = reinterpret_cast<const T*>(dsm + (i % NSLOT) * 2 * CH_BYTES);
         const T* sV = reinterpret_cast<const T*>(dsm + (i % NSLOT) * 2 * CH_BYTES + CH_BYTES);
-        const int n = min(kChunk, ctx - (z + i * P) * kChunk);
+        const int ctx = s_pos[cur.b] + 1;
+        const int n = min(kChunk, ctx - cur.j * kChunk);
 #pragma unroll 1
         for (int jb = warp * 16; jb < min(n, warp * 16 + 16); jb += 8) {
             // eight keys: this lane's partial dot products ...
@@ -187,67 +319,85 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
             }
         }
         __syncthreads();                               // ring slot i % NSLOT is free again
-        if (threadIdx.x == 0 && i + NSLOT < mine) issue(i + NSLOT);
-    }
-    if (!ok && threadIdx.x == 0) report_status(status, LLAMA_ERR_DEVICE_TIMEOUT);
+        if (threadIdx.x == 0 && i + NSLOT < len) issue(i + NSLOT);
+        const int nch = s_nch[cur.b];
+        if (cur.j + 1 < nch && i + 1 < len) { advance(cur); continue; }
 
-    // merge the 4 warps of this CTA
-    if (lane == 0) {
+        // ---- end of a segment: merge the 4 warps, then write the row or a partial
+        const bool whole = seg_j0 == 0 && cur.j + 1 == nch;
+        if (lane == 0) {
 #pragma unroll
-        for (int r = 0; r < NREP; ++r) { s_m[warp][r] = mx[r]; s_l[warp][r] = sl[r]; }
-    }
-#pragma unroll
-    for (int r = 0; r < NREP; ++r)
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) s_o[warp][r][lane * EPL + e] = o[r][e];
-    __syncthreads();
-    const int nh = nq / HD;
-    for (int idx = threadIdx.x; idx < NREP * HD; idx += blockDim.x) {
-        const int r = idx / HD, d = idx % HD;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) M = fmaxf(M, s_m[w][r]);
-        float L = 0.f, acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            const float f = (s_m[w][r] == -INFINITY) ? 0.f : __expf(s_m[w][r] - M);
-            L += s_l[w][r] * f;
-            acc += s_o[w][r][d] * f;
+            for (int r = 0; r < NREP; ++r) { s_m[warp][r] = mx[r]; s_l[warp][r] = sl[r]; }
         }
-        const int h = g * NREP + r;
-        if (pact == 1) {
-            out[static_cast<long long>(b) * nq + h * HD + d] = from_f32<T>(acc / L);
-        } else {
-            const long long slot = (static_cast<long long>(b) * nh + h) * P + z;
-            part_o[slot * HD + d] = acc;
-            if (d == 0) {
-                part_ml[slot * 2] = M;
-                part_ml[slot * 2 + 1] = L;
+#pragma unroll
+        for (int r = 0; r < NREP; ++r)
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) s_o[warp][r][lane * EPL + e] = o[r][e];
+        __syncthreads();
+        const long long pair_u0 = static_cast<long long>(s_cum[cur.b]) * nkv + static_cast<long long>(cur.g) * nch;
+        const int slot_id = c * 2 + (seg_i0 == 0 ? 0 : 1);
+        for (int idx = threadIdx.x; idx < NREP * HD; idx += blockDim.x) {
+            const int r = idx / HD, d = idx % HD;
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) M = fmaxf(M, s_m[w][r]);
+            float L = 0.f, acc = 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float f = (s_m[w][r] == -INFINITY) ? 0.f : __expf(s_m[w][r] - M);
+                L += s_l[w][r] * f;
+                acc += s_o[w][r][d] * f;
+            }
+            const int h = cur.g * NREP + r;
+            if (whole) {
+                out[static_cast<long long>(cur.b) * nq + h * HD + d] = from_f32<T>(acc / L);
+            } else {
+                part_o[(static_cast<long long>(slot_id) * NREP + r) * HD + d] = acc;
+                if (d == 0) {
+                    part_ml[(static_cast<long long>(slot_id) * NREP + r) * 2] = M;
+                    part_ml[(static_cast<long long>(slot_id) * NREP + r) * 2 + 1] = L;
+                }
             }
         }
-    }
-    if (pact == 1) return;
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) s_last = atomicAdd(&counters[b * gridDim.y + g], 1) == pact - 1;
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    for (int idx = threadIdx.x; idx < NREP * HD; idx += blockDim.x) {
-        const int r = idx / HD, d = idx % HD;
-        const int h = g * NREP + r;
-        const long long base = (static_cast<long long>(b) * nh + h) * P;
-        float M = -INFINITY;
-        for (int t = 0; t < pact; ++t) M = fmaxf(M, part_ml[(base + t) * 2]);
-        float L = 0.f, acc = 0.f;
-        for (int t = 0; t < pact; ++t) {
-            const float f = __expf(part_ml[(base + t) * 2] - M);
-            L += part_ml[(base + t) * 2 + 1] * f;
-            acc += part_o[(base + t) * HD + d] * f;
+        if (!whole) {
+            const int cf = owner64(pair_u0, W, P), cl = owner64(pair_u0 + nch - 1, W, P);
+            const int cnt_idx = cur.b * nkv + cur.g;
+            __threadfence();
+            __syncthreads();
+            if (threadIdx.x == 0) s_last = atomicAdd(&counters[cnt_idx], 1) == cl - cf;
+            __syncthreads();
+            if (s_last) {
+                __threadfence();
+                for (int idx = threadIdx.x; idx < NREP * HD; idx += blockDim.x) {
+                    const int r = idx / HD, d = idx % HD;
+                    const int h = cur.g * NREP + r;
+                    float M = -INFINITY;
+                    for (int cc = cf; cc <= cl; ++cc) {
+                        const int sid = cc * 2 + (run_begin64(cc, W, P) >= pair_u0 ? 0 : 1);
+                        M = fmaxf(M, part_ml[(static_cast<long long>(sid) * NREP + r) * 2]);
+                    }
+                    float L = 0.f, acc = 0.f;
+                    for (int cc = cf; cc <= cl; ++cc) {
+                        const int sid = cc * 2 + (run_begin64(cc, W, P) >= pair_u0 ? 0 : 1);
+                        const float mm = part_ml[(static_cast<long long>(sid) * NREP + r) * 2];
+                        const float f = (mm == -INFINITY) ? 0.f : __expf(mm - M);
+                        L += part_ml[(static_cast<long long>(sid) * NREP + r) * 2 + 1] * f;
+                        acc += part_o[(static_cast<long long>(sid) * NREP + r) * HD + d] * f;
+                    }
+                    out[static_cast<long long>(cur.b) * nq + h * HD + d] = from_f32<T>(acc / L);
+                }
+                if (threadIdx.x == 0) counters[cnt_idx] = 0;
+            }
         }
-        out[static_cast<long long>(b) * nq + h * HD + d] = from_f32<T>(acc / L);
+        __syncthreads();   // s_m / s_o / s_last reused by the next segment
+        if (i + 1 < len) {
+            advance(cur);
+            seg_j0 = cur.j;
+            seg_i0 = i + 1;
+            start_pair();
+        }
     }
-    if (threadIdx.x == 0) counters[b * gridDim.y + g] = 0;
+    if (!ok && threadIdx.x == 0) report_status(status, LLAMA_ERR_DEVICE_TIMEOUT);
 }
 
 static int g_attn_sms = 0;
@@ -258,13 +408,14 @@ static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaS
     const T* vc = static_cast<const T*>(m->vc) + layer * m->kv_layer_elems;
     auto kern = attn_decode_kernel<T, HD, NREP>;
     const int smem = 3 * 2 * kChunk * HD * static_cast<int>(sizeof(T));   // three K+V chunks
-    static bool attr = false;
-    if (!attr) {
+    static int per_sm = 0;
+    if (per_sm == 0) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+        if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 128, smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_decode_kernel)");
-        attr = true;
+        if (per_sm < 1) per_sm = 1;
     }
     if (g_attn_sms == 0) {
         int dev = 0;
@@ -272,13 +423,15 @@ static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaS
         cudaDeviceGetAttribute(&g_attn_sms, cudaDevAttrMultiProcessorCount, dev);
         if (g_attn_sms <= 0) g_attn_sms = 148;
     }
-    // about two CTAs per SM over all (row, kv head) pairs, never more than the chunks
-    int P = (2 * g_attn_sms + m->nkv * B - 1) / (m->nkv * B);
-    P = std::max(1, std::min(P, m->n_splits));
-    dim3 grid(P, m->nkv, B);
-    cudaError_t e = launch_k(kern, grid, dim3(128), smem, st, pdl, static_cast<const T*>(m->q), kc, vc, pos, m->nq,
-                             m->S, m->kv_row_elems, m->part_o, m->part_ml, m->attn_cnt, static_cast<T*>(m->attn),
-                             m->status);
+    if (B > kMaxRows) { set_error("decode attention takes at most %d rows", kMaxRows); return LLAMA_ERR_INVALID_ARG; }
+    // one resident wave; never more CTAs than units (at least one unit per row and KV head)
+    long long P = static_cast<long long>(g_attn_sms) * per_sm;
+    P = std::min<long long>(P, kMaxAttnCtas);
+    P = std::min<long long>(P, static_cast<long long>(B) * m->nkv * m->n_splits);
+    P = std::max<long long>(P, 1);
+    cudaError_t e = launch_k(kern, dim3(static_cast<unsigned>(P)), dim3(128), smem, st, pdl, static_cast<const T*>(m->q),
+                             kc, vc, pos, B, m->nkv, m->nq, m->S, m->kv_row_elems, m->part_o, m->part_ml,
+                             m->attn_cnt, static_cast<T*>(m->attn), m->status);
     count_launch();
     if (e != cudaSuccess) return cuda_fail(e, "attn_decode_kernel");
     return LLAMA_OK;

@@ -21,11 +21,8 @@
 // A deep ring (about 200 KB of weight tiles in flight per SM) keeps HBM
 // busy; the next projection's CTAs launch early (programmatic dependent
 // launch) and start streaming as soon as this kernel's CTAs leave their SMs.
-// Weights never change during decode, so when a CTA's producer has issued
-// its last load it also pulls the first ring's worth of the NEXT projection's
-// weight tiles for the same CTA index into L2: the next kernel starts on L2
-// hits, and HBM stays busy during this kernel's epilogue and fixup tail.
-// Two TMEM accumulators let the MMA of the next segment overlap the epilogue
+// (Extra L2 prefetches of weight tiles that are bulk-loaded soon after were
+// measured to lower the streaming rate, so there are none.)  Two TMEM accumulators let the MMA of the next segment overlap the epilogue
 // of the previous one.  With programmatic dependent launch, weight tiles are
 // requested before the previous kernel has finished; the activation tiles
 // and every global read of the epilogue wait for it (griddepcontrol.wait).
@@ -41,28 +38,6 @@ constexpr int kThreads = 192;
 constexpr int kAccStride = 64;      // TMEM columns per accumulator buffer
 constexpr int kTmemCols = 128;      // two accumulator buffers
 constexpr int kABytes = 128 * 128;  // 128 weight rows x 64 bf16
-constexpr int kL2Ahead = 16;        // units pulled into L2 beyond the ring at kernel start
-
-__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(n) : "memory"); }
-// OR of `v` over the `n` threads of named barrier `id` (they all block).
-__device__ __forceinline__ bool named_any(int id, int n, bool v) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.or.pred p, %2, %3, q;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(r) : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(n) : "memory");
-    return r != 0;
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(bar)) : "memory");
-}
-
-// CTA owning flat unit u when W units are split into P contiguous runs
-// (W * P stays far below 2^31: W <= kMaxTiles * 256 k-tiles, P <= 256).
-__device__ __forceinline__ int owner(int u, int W, int P) { return ((u + 1) * P - 1) / W; }
-__device__ __forceinline__ int run_begin(int c, int W, int P) { return c * W / P; }
 
 struct Seg {
     int tile, ks, ke;
@@ -79,11 +54,124 @@ __device__ __forceinline__ bool next_seg(int& u, int u1, int KT, Seg& s) {
 }
 }  // namespace
 
+// Epilogue of one finished 128-row weight tile t: v[b] = acc[row r of the
+// tile, token column b] for the nb real token columns.  All 128 epilogue
+// threads of the CTA call it together (the residual + sum-of-squares mode
+// synchronises them on named barrier 2).
+template <int BN>
+__device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int lane, int q, int epi_tid, int nb,
+                                            int N, int T, const Epi& ep, const NormIO& nio, bool scale_in,
+                                            const float* rs, float* red) {
+    if (scale_in) {
+#pragma unroll
+        for (int b = 0; b < BN; ++b) v[b] *= (b < nb) ? rs[b] : 0.f;
+    }
+    const int n = t * 128 + r;
+    const bool row_ok = n < N;
+    if (ep.mode == EPI_SWIGLU) {
+        // rows are interleaved in blocks of 16: lanes 0-15 of a warp hold
+        // w1 rows, lanes 16-31 the matching w3 rows
+#pragma unroll
+        for (int b = 0; b < BN; ++b) {
+            const float up = __shfl_xor_sync(0xffffffffu, v[b], 16);
+            if (lane < 16 && row_ok && b < nb) {
+                const int h = (n >> 5) * 16 + (n & 15);
+                static_cast<bf16*>(ep.g)[static_cast<long long>(b) * ep.H + h] =
+                    __float2bfloat16_rn(silu_f(v[b]) * up);
+            }
+        }
+    } else if (ep.mode == EPI_QKV) {
+        const bool even = (lane & 1) == 0;
+        const bool is_q = n < ep.nq;
+        int cc = n - ep.nq;
+        bf16* cache = static_cast<bf16*>(ep.kc);
+        const bool is_k = !is_q && cc < ep.nkvc;
+        if (!is_q && !is_k) { cc -= ep.nkvc; cache = static_cast<bf16*>(ep.vc); }
+        const int d = is_q ? n % ep.hd : cc % ep.hd;
+        const int head = is_q ? 0 : cc / ep.hd;
+        // per group of 16 columns: all positions and RoPE factors first
+        // (independent loads), then the rotations and stores
+#pragma unroll
+        for (int b0 = 0; b0 < BN; b0 += 16) {
+            int posv[16];
+            float2 cs[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) posv[u] = (b0 + u < nb) ? ep.tok_pos[b0 + u] : -1;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const bool okp = row_ok && posv[u] >= 0 && posv[u] < ep.max_seq && (is_q || is_k);
+                cs[u] = okp ? ep.rope[static_cast<long long>(posv[u]) * (ep.hd / 2) + (d >> 1)]
+                            : make_float2(1.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int b = b0 + u;
+                const float partner = __shfl_xor_sync(0xffffffffu, v[b], 1);
+                const int pos = posv[u];
+                if (!row_ok || b >= nb || pos < 0 || pos >= ep.max_seq) continue;
+                const float re = even ? v[b] : partner, im = even ? partner : v[b];
+                const float rot = even ? re * cs[u].x - im * cs[u].y : re * cs[u].y + im * cs[u].x;
+                if (is_q) {
+                    static_cast<bf16*>(ep.q)[static_cast<long long>(b) * ep.nq + n] = __float2bfloat16_rn(rot);
+                } else {
+                    const int row = ep.tok_row ? ep.tok_row[b] : b;
+                    cache[static_cast<long long>(row) * ep.kv_row_stride +
+                          (static_cast<long long>(head) * ep.max_seq + pos) * ep.hd + d] =
+                        __float2bfloat16_rn(is_k ? rot : v[b]);
+                }
+            }
+        }
+    } else if (ep.mode == EPI_RESID_F32 && nio.ssq_out) {
+        // residual add, plus this tile's share of sum(x^2) for the next RMSNorm;
+        // the old x values of a 16-column group are loaded together
+        const float wn = row_ok ? nio.w_next[n] : 0.f;
+        float xo[16];
+#pragma unroll
+        for (int b = 0; b < BN; ++b) {
+            if ((b & 15) == 0) {
+#pragma unroll
+                for (int u = 0; u < 16; ++u)
+                    xo[u] = (row_ok && b + u < nb) ? ep.out[static_cast<long long>(b + u) * ep.ldo + n] : 0.f;
+            }
+            float sq = 0.f;
+            if (row_ok && b < nb) {
+                const float nv = xo[b & 15] + v[b];
+                ep.out[static_cast<long long>(b) * ep.ldo + n] = nv;
+                static_cast<bf16*>(nio.y_out)[static_cast<long long>(b) * ep.ldo + n] = __float2bfloat16_rn(nv * wn);
+                sq = nv * nv;
+            }
+            sq = warp_sum(sq);
+            if (lane == 0) red[q * 64 + b] = sq;
+        }
+        named_sync(2, 128);
+        if (epi_tid < nb)
+            nio.ssq_out[epi_tid * T + t] = ((red[epi_tid] + red[64 + epi_tid]) + red[128 + epi_tid]) +
+                                           red[192 + epi_tid];
+        named_sync(2, 128);
+    } else if (row_ok) {
+        if (ep.mode == EPI_RESID_F32) {
+#pragma unroll
+            for (int b0 = 0; b0 < BN; b0 += 16) {
+                float xo[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u)
+                    xo[u] = (b0 + u < nb) ? ep.out[static_cast<long long>(b0 + u) * ep.ldo + n] : 0.f;
+#pragma unroll
+                for (int u = 0; u < 16; ++u)
+                    if (b0 + u < nb) ep.out[static_cast<long long>(b0 + u) * ep.ldo + n] = xo[u] + v[b0 + u];
+            }
+        } else {
+#pragma unroll
+            for (int b = 0; b < BN; ++b)
+                if (b < nb) ep.out[static_cast<long long>(b) * ep.ldo + n] = v[b];
+        }
+    }
+}
+
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUtensorMap mapX,
-                     int N, int M, int K, Epi ep, float* __restrict__ part, int* __restrict__ counters, NormIO nio,
-                     const __grid_constant__ CUtensorMap mapNext, int Nn, int Kn, int Pn) {
+                     int N, int M, int K, Epi ep, float* __restrict__ part, int* __restrict__ counters, NormIO nio) {
     constexpr int B_BYTES = BN * 128;
     constexpr int STAGE = kABytes + B_BYTES;
     extern __shared__ uint8_t smem_raw[];
@@ -133,16 +221,6 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
             tma_load_2d(smem + i * STAGE, &mapW, kk * 64, tt * 128, &full[i]);
             if (++kk == KT) { kk = 0; ++tt; }
         }
-        {
-            // before waiting for the previous kernel, also pull the units after the
-            // ring into L2, so that HBM keeps streaming through that kernel's tail
-            const int nl = min(nunits - npre, kL2Ahead);
-            int tl = tt, kl = kk;
-            for (int i = 0; i < nl; ++i) {
-                tma_prefetch_l2(&mapW, kl * 64, tl * 128);
-                if (++kl == KT) { kl = 0; ++tl; }
-            }
-        }
         pdl_wait();
         tt = t0;
         kk = k0;
@@ -161,18 +239,6 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
 #pragma unroll
             for (int rr = 0; rr < BN / 16; ++rr) tma_load_2d(st + kABytes + rr * 2048, &mapX, kk * 64, rr * 16, &full[s]);
             if (++kk == KT) { kk = 0; ++tt; }
-        }
-        if (Nn > 0 && c < Pn) {
-            // warm L2 with the first units of this CTA index's run in the next projection
-            const int KTn = (Kn + 63) / 64;
-            const int Wn = ((Nn + 127) / 128) * KTn;
-            const int v0 = run_begin(c, Wn, Pn), v1 = run_begin(c + 1, Wn, Pn);
-            const int nv = min(v1 - v0, STAGES);
-            int tn = v0 / KTn, kn = v0 - tn * KTn;
-            for (int i = 0; i < nv; ++i) {
-                tma_prefetch_l2(&mapNext, kn * 64, tn * 128);
-                if (++kn == KTn) { kn = 0; ++tn; }
-            }
         }
     } else if (warp == 1 && lane == 0) {
         // ---------------- MMA issuer
@@ -284,111 +350,7 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
                 }
                 if (epi_tid == 0) counters[t] = 0;
             }
-            // ---- epilogue on the finished tile
-            if (scale_in) {
-#pragma unroll
-                for (int b = 0; b < BN; ++b) v[b] *= (b < nb) ? rs[b] : 0.f;
-            }
-            const int n = t * 128 + r;
-            const bool row_ok = n < N;
-            if (ep.mode == EPI_SWIGLU) {
-                // rows are interleaved in blocks of 16: lanes 0-15 of a warp hold
-                // w1 rows, lanes 16-31 the matching w3 rows
-#pragma unroll
-                for (int b = 0; b < BN; ++b) {
-                    const float up = __shfl_xor_sync(0xffffffffu, v[b], 16);
-                    if (lane < 16 && row_ok && b < nb) {
-                        const int h = (n >> 5) * 16 + (n & 15);
-                        static_cast<bf16*>(ep.g)[static_cast<long long>(b) * ep.H + h] =
-                            __float2bfloat16_rn(silu_f(v[b]) * up);
-                    }
-                }
-            } else if (ep.mode == EPI_QKV) {
-                const bool even = (lane & 1) == 0;
-                const bool is_q = n < ep.nq;
-                int cc = n - ep.nq;
-                bf16* cache = static_cast<bf16*>(ep.kc);
-                const bool is_k = !is_q && cc < ep.nkvc;
-                if (!is_q && !is_k) { cc -= ep.nkvc; cache = static_cast<bf16*>(ep.vc); }
-                const int d = is_q ? n % ep.hd : cc % ep.hd;
-                const int head = is_q ? 0 : cc / ep.hd;
-                // per group of 16 columns: all positions and RoPE factors first
-                // (independent loads), then the rotations and stores
-#pragma unroll
-                for (int b0 = 0; b0 < BN; b0 += 16) {
-                    int posv[16];
-                    float2 cs[16];
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) posv[u] = (b0 + u < nb) ? ep.tok_pos[b0 + u] : -1;
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const bool okp = row_ok && posv[u] >= 0 && posv[u] < ep.max_seq && (is_q || is_k);
-                        cs[u] = okp ? ep.rope[static_cast<long long>(posv[u]) * (ep.hd / 2) + (d >> 1)]
-                                    : make_float2(1.f, 0.f);
-                    }
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const int b = b0 + u;
-                        const float partner = __shfl_xor_sync(0xffffffffu, v[b], 1);
-                        const int pos = posv[u];
-                        if (!row_ok || b >= nb || pos < 0 || pos >= ep.max_seq) continue;
-                        const float re = even ? v[b] : partner, im = even ? partner : v[b];
-                        const float rot = even ? re * cs[u].x - im * cs[u].y : re * cs[u].y + im * cs[u].x;
-                        if (is_q) {
-                            static_cast<bf16*>(ep.q)[static_cast<long long>(b) * ep.nq + n] = __float2bfloat16_rn(rot);
-                        } else {
-                            const int row = ep.tok_row ? ep.tok_row[b] : b;
-                            cache[static_cast<long long>(row) * ep.kv_row_stride +
-                                  (static_cast<long long>(head) * ep.max_seq + pos) * ep.hd + d] =
-                                __float2bfloat16_rn(is_k ? rot : v[b]);
-                        }
-                    }
-                }
-            } else if (ep.mode == EPI_RESID_F32 && nio.ssq_out) {
-                // residual add, plus this tile's share of sum(x^2) for the next RMSNorm;
-                // the old x values of a 16-column group are loaded together
-                const float wn = row_ok ? nio.w_next[n] : 0.f;
-                float xo[16];
-#pragma unroll
-                for (int b = 0; b < BN; ++b) {
-                    if ((b & 15) == 0) {
-#pragma unroll
-                        for (int u = 0; u < 16; ++u)
-                            xo[u] = (row_ok && b + u < nb) ? ep.out[static_cast<long long>(b + u) * ep.ldo + n] : 0.f;
-                    }
-                    float sq = 0.f;
-                    if (row_ok && b < nb) {
-                        const float nv = xo[b & 15] + v[b];
-                        ep.out[static_cast<long long>(b) * ep.ldo + n] = nv;
-                        static_cast<bf16*>(nio.y_out)[static_cast<long long>(b) * ep.ldo + n] = __float2bfloat16_rn(nv * wn);
-                        sq = nv * nv;
-                    }
-                    sq = warp_sum(sq);
-                    if (lane == 0) red[q * 64 + b] = sq;
-                }
-                named_sync(2, 128);
-                if (epi_tid < nb)
-                    nio.ssq_out[epi_tid * T + t] = ((red[epi_tid] + red[64 + epi_tid]) + red[128 + epi_tid]) +
-                                                   red[192 + epi_tid];
-                named_sync(2, 128);
-            } else if (row_ok) {
-                if (ep.mode == EPI_RESID_F32) {
-#pragma unroll
-                    for (int b0 = 0; b0 < BN; b0 += 16) {
-                        float xo[16];
-#pragma unroll
-                        for (int u = 0; u < 16; ++u)
-                            xo[u] = (b0 + u < nb) ? ep.out[static_cast<long long>(b0 + u) * ep.ldo + n] : 0.f;
-#pragma unroll
-                        for (int u = 0; u < 16; ++u)
-                            if (b0 + u < nb) ep.out[static_cast<long long>(b0 + u) * ep.ldo + n] = xo[u] + v[b0 + u];
-                    }
-                } else {
-#pragma unroll
-                    for (int b = 0; b < BN; ++b)
-                        if (b < nb) ep.out[static_cast<long long>(b) * ep.ldo + n] = v[b];
-                }
-            }
+            finish_tile<BN>(v, t, r, lane, q, epi_tid, nb, N, T, ep, nio, scale_in, rs, red);
         }
     }
 
@@ -397,13 +359,13 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+
 // ---------------------------------------------------------------- host side
 static int g_sms = 0;
 
 template <int BN, int STAGES>
 static int launch_decode(const CUtensorMap& w, const CUtensorMap& x, int N, int M, int K, const Epi& ep,
-                         float* part, int* counters, int max_ctas, cudaStream_t st, bool pdl, const NormIO& nio,
-                         const NextProj* next) {
+                         float* part, int* counters, int max_ctas, cudaStream_t st, bool pdl, const NormIO& nio) {
     constexpr int smem = 1024 + STAGES * (kABytes + BN * 128) + (2 * STAGES + 4) * 8 + 32 + 5 * 64 * 4;
     static_assert(smem <= 227 * 1024, "shared memory per CTA");
     auto kern = linear_decode_kernel<BN, STAGES>;
@@ -419,24 +381,14 @@ static int launch_decode(const CUtensorMap& w, const CUtensorMap& x, int N, int 
     if (units > (1 << 22)) { set_error("decode projection too large (%lld work units)", units); return LLAMA_ERR_INVALID_ARG; }
     int P = max_ctas;
     if (units < P) P = static_cast<int>(units);
-    int Nn = 0, Kn = 0, Pn = 0;
-    const CUtensorMap* mn = &w;
-    if (next && next->map) {
-        Nn = next->N;
-        Kn = next->K;
-        const long long un = static_cast<long long>((Nn + 127) / 128) * ((Kn + 63) / 64);
-        Pn = un < max_ctas ? static_cast<int>(un) : max_ctas;   // the grid the next launch will use
-        mn = next->map;
-    }
-    cudaError_t e = launch_k(kern, dim3(P), dim3(kThreads), smem, st, pdl, w, x, N, M, K, ep, part, counters, nio,
-                             *mn, Nn, Kn, Pn);
+    cudaError_t e = launch_k(kern, dim3(P), dim3(kThreads), smem, st, pdl, w, x, N, M, K, ep, part, counters, nio);
     count_launch();
     if (e != cudaSuccess) return cuda_fail(e, "linear_decode_kernel");
     return LLAMA_OK;
 }
 
 int linear_bf16_decode(const TmaMaps* mapX, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
-                       int* counters, cudaStream_t st, bool pdl, const NormIO* nio_in, const NextProj* next) {
+                       size_t part_bytes, int* counters, cudaStream_t st, bool pdl, const NormIO* nio_in) {
     if (M <= 0 || N <= 0) return LLAMA_OK;
     NormIO nio = {};
     if (nio_in) nio = *nio_in;
@@ -445,6 +397,15 @@ int linear_bf16_decode(const TmaMaps* mapX, const TmaMaps* mapW, int M, int N, i
         return LLAMA_ERR_INVALID_ARG;
     }
     if (M > 64) { set_error("decode projection takes at most 64 token rows"); return LLAMA_ERR_INVALID_ARG; }
+    {
+        // split partials: two 128 x BN fp32 blocks per persistent CTA
+        const int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 48 ? 48 : 64;
+        const size_t need = static_cast<size_t>(kMaxDecodeCtas) * 2 * 128 * bn * 4;
+        if (!part || !counters || part_bytes < need) {
+            set_error("decode projection needs %zu bytes of split partials and the tile counters", need);
+            return LLAMA_ERR_CAPACITY;
+        }
+    }
     if (g_sms == 0) {
         int dev = 0;
         cudaGetDevice(&dev);
@@ -452,10 +413,10 @@ int linear_bf16_decode(const TmaMaps* mapX, const TmaMaps* mapW, int M, int N, i
         if (g_sms <= 0) g_sms = 148;
         if (g_sms > kMaxDecodeCtas) g_sms = kMaxDecodeCtas;
     }
-    if (M <= 16) return launch_decode<16, 12>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio, next);
-    if (M <= 32) return launch_decode<32, 11>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio, next);
-    if (M <= 48) return launch_decode<48, 10>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio, next);
-    return launch_decode<64, 9>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio, next);
+    if (M <= 16) return launch_decode<16, 12>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio);
+    if (M <= 32) return launch_decode<32, 11>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio);
+    if (M <= 48) return launch_decode<48, 10>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio);
+    return launch_decode<64, 9>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio);
 }
 
 }  // namespace llb

@@ -8,31 +8,45 @@
 //
 // D[i, j] = sum_k A[i, k] * B[j, k]; A = activations [tokens, K], B = weights
 // [N, K], both K-major bf16 read through 128-byte-swizzled TMA boxes of 64
-// K-elements.  One CTA computes one 128 x 256 tile of D:
-//   warp 0 lane 0  TMA producer (STAGES-deep ring of A/B tiles)
+// K-elements.  D is cut into 128 x 256 tiles, ordered in groups of 16 tiles
+// along M (all N-tiles of one group before the next group), so that the
+// tiles in flight at any time share a few hundred KB of A and B in L2.
+//
+// The kernel is persistent: one CTA per SM walks a fixed list of work items.
+// The first `dp` tiles go round-robin, one whole tile per item.  The last
+// `sk` tiles (the partial last wave plus one full wave) form one flat run of
+// sk * K/64 k-tile units cut into P equal contiguous runs (stream-K), so every
+// SM ends at the same time whatever the tile count.  A tile split between CTAs
+// is finished by the contributor that arrives last at the tile's counter: it
+// adds the fp32 partials in CTA order (deterministic) and applies the
+// epilogue; no CTA ever waits for another.
+//
+// Warp roles (192 threads):
+//   warp 0 lane 0  TMA producer (4-deep ring of 128x64 A + 256x64 B tiles)
 //   warp 1 lane 0  MMA issuer (tcgen05.mma kind::f16, M=128, N=256, K=16)
-//   warp 1         TMEM allocation / release
-//   warps 0-3      epilogue: TMEM lane i (token row i of the tile) -> thread i,
-//                  TMEM columns = output features
-// No TMA multicast is used.
+//   warp 1         TMEM owner: two 256-column accumulators, so the MMAs of
+//                  one item run while the epilogue drains the previous one
+//   warps 2-5      epilogue: warp w reads TMEM lanes 32*(w%4)..+31 = token rows
+// Every wait is bounded; no TMA multicast.
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "model.h"
 
+#include <algorithm>
 #include <cudaTypedefs.h>
 
 namespace llb {
 
 namespace {
 
+constexpr int kThreadsTc = 192;
+constexpr int kBN = 256;                     // tile width along N (weight rows)
+constexpr int kStagesTc = 4;
 constexpr int kA_BYTES = 128 * 128;          // 128 rows x 64 bf16
-
-template <int BN>
-struct TcCfg {
-    static constexpr int B_BYTES = BN * 128;
-    static constexpr int STAGE_BYTES = kA_BYTES + B_BYTES;
-    static constexpr uint32_t TMEM_COLS = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
-};
+constexpr int kB_BYTES = kBN * 128;
+constexpr int kStageBytes = kA_BYTES + kB_BYTES;
+constexpr int kGroupM = 16;                  // M-tiles per rasterisation group
+constexpr int kPartFloats = 128 * kBN;       // one fp32 partial tile
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
@@ -53,43 +67,151 @@ __device__ __forceinline__ void store32_bf16(bf16* dst, const float* v) {
     }
 }
 
+// Work list of one CTA: whole tiles c, c+P, ... below dp, then its stream-K run.
+struct TcPlan {
+    int TM, TN, KT;
+    int dp, sk;
+};
+struct Item {
+    int tile, ks, ke;
+};
+struct WorkIt {
+    int next_dp, u, u1;
+};
+
+__device__ __forceinline__ WorkIt work_begin(const TcPlan& p, int c, int P) {
+    WorkIt w;
+    w.next_dp = c;
+    const int W = p.sk * p.KT;
+    w.u = run_begin(c, W, P);
+    w.u1 = run_begin(c + 1, W, P);
+    return w;
+}
+
+__device__ __forceinline__ bool work_next(WorkIt& w, const TcPlan& p, int P, Item& it) {
+    if (w.next_dp < p.dp) {
+        it.tile = w.next_dp;
+        it.ks = 0;
+        it.ke = p.KT;
+        w.next_dp += P;
+        return true;
+    }
+    if (w.u >= w.u1) return false;
+    const int tl = w.u / p.KT;
+    it.tile = p.dp + tl;
+    it.ks = w.u - tl * p.KT;
+    it.ke = min(p.KT, it.ks + (w.u1 - w.u));
+    w.u += it.ke - it.ks;
+    return true;
+}
+
+// Tile t -> (M-tile, N-tile): groups of kGroupM M-tiles, N-major inside a group.
+__device__ __forceinline__ void tile_coords(int t, const TcPlan& p, int& tm, int& tn) {
+    const int per_group = kGroupM * p.TN;
+    const int g = t / per_group;
+    const int rem = t - g * per_group;
+    const int gm = min(kGroupM, p.TM - g * kGroupM);
+    tn = rem / gm;
+    tm = g * kGroupM + (rem - tn * gm);
+}
+
+// Epilogue of 32 consecutive output features n0..n0+31 of token row m.
+__device__ __forceinline__ void epi_chunk(const Epi& ep, int m, int n0, int rowsB, float (&v)[32]) {
+    if (n0 >= rowsB) return;
+    if (ep.mode == EPI_SWIGLU) {
+        // each 32-column chunk holds 16 w1 outputs then the same 16 w3 outputs
+        float g16[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) g16[t] = silu_f(v[t]) * v[16 + t];
+        bf16* dst = static_cast<bf16*>(ep.g) + static_cast<long long>(m) * ep.H + (n0 / 32) * 16;
+        uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            uint4 u;
+            u.x = pack_bf16x2(g16[8 * q + 0], g16[8 * q + 1]);
+            u.y = pack_bf16x2(g16[8 * q + 2], g16[8 * q + 3]);
+            u.z = pack_bf16x2(g16[8 * q + 4], g16[8 * q + 5]);
+            u.w = pack_bf16x2(g16[8 * q + 6], g16[8 * q + 7]);
+            d4[q] = u;
+        }
+    } else if (ep.mode == EPI_QKV) {
+        const int pos = ep.tok_pos[m];
+        if (pos < 0 || pos >= ep.max_seq) return;
+        bf16* dst;
+        bool rot;
+        int d0;
+        if (n0 < ep.nq) {
+            d0 = n0 % ep.hd;
+            rot = true;
+            dst = static_cast<bf16*>(ep.q) + static_cast<long long>(m) * ep.nq + n0;
+        } else {
+            int cc = n0 - ep.nq;
+            bf16* cache = static_cast<bf16*>(ep.kc);
+            rot = cc < ep.nkvc;
+            if (!rot) { cc -= ep.nkvc; cache = static_cast<bf16*>(ep.vc); }
+            const int head = cc / ep.hd;
+            d0 = cc % ep.hd;
+            const int row = ep.tok_row ? ep.tok_row[m] : m;
+            dst = cache + static_cast<long long>(row) * ep.kv_row_stride +
+                  (static_cast<long long>(head) * ep.max_seq + pos) * ep.hd + d0;
+        }
+        if (rot) {
+#pragma unroll
+            for (int t = 0; t < 32; t += 2) rope_pair(ep.rope, ep.hd, pos, (d0 + t) >> 1, v[t], v[t + 1]);
+        }
+        store32_bf16(dst, v);
+    } else {
+        float* o = ep.out + static_cast<long long>(m) * ep.ldo + n0;
+        const int lim = min(32, rowsB - n0);
+        if (lim == 32 && (ep.ldo % 4) == 0) {
+            float4* o4 = reinterpret_cast<float4*>(o);
+            if (ep.mode == EPI_RESID_F32) {
+                float4 p[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) p[q] = o4[q];
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    o4[q] = make_float4(p[q].x + v[4 * q], p[q].y + v[4 * q + 1], p[q].z + v[4 * q + 2],
+                                        p[q].w + v[4 * q + 3]);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) o4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            }
+        } else {
+#pragma unroll
+            for (int t = 0; t < 32; ++t)
+                if (t < lim) o[t] = (ep.mode == EPI_RESID_F32) ? o[t] + v[t] : v[t];
+        }
+    }
+}
+
 }  // namespace
 
-template <int BN, int STAGES, int B_BOX>
-__global__ void __launch_bounds__(128, 1)
-linear_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                 int rowsA, int rowsB, int K, int kt_per_split, Epi ep) {
-    using C = TcCfg<BN>;
+__global__ void __launch_bounds__(kThreadsTc, 1)
+linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                  int rowsA, int rowsB, TcPlan plan, Epi ep, float* __restrict__ part, int* __restrict__ counters) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
-    uint64_t* empty = full + STAGES;
-    uint64_t* accum = empty + STAGES;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
-    int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStagesTc * kStageBytes);
+    uint64_t* empty = full + kStagesTc;
+    uint64_t* tfull = empty + kStagesTc;   // [2]
+    uint64_t* tempty = tfull + 2;          // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+    int* flag = reinterpret_cast<int*>(tmem_slot + 1);   // [0] abort, [1] arrival broadcast
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tileA = blockIdx.x, tileB = blockIdx.y;
-    const int KT = (K + 63) / 64;
-    const int kt0 = blockIdx.z * kt_per_split;
-    const int kt1 = min(KT, kt0 + kt_per_split);
-    const int nk = kt1 - kt0;
+    const int P = gridDim.x, c = blockIdx.x;
+    const int KT = plan.KT;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
-        mbar_init(accum, 1);
-        *abort_flag = 0;
+        for (int s = 0; s < kStagesTc; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 128); }
+        flag[0] = 0;
         fence_mbar_init();
         tma_prefetch_desc(&mapA);
         tma_prefetch_desc(&mapB);
     }
-    if (warp == 1) {
-        tmem_alloc(tmem_slot, C::TMEM_COLS);
-        tmem_relinquish();
-    }
+    if (warp == 1) { tmem_alloc(tmem_slot, 2 * kBN); tmem_relinquish(); }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -97,136 +219,145 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
 
     if (warp == 0 && lane == 0) {
         // ---------------- TMA producer
-        for (int i = 0; i < nk; ++i) {
-            const int s = i % STAGES;
-            const uint32_t ph = (i / STAGES) & 1;
-            if (!mbar_wait(&empty[s], ph ^ 1)) { atomicExch(abort_flag, 1); break; }
-            mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-            const int kx = (kt0 + i) * 64;
-            uint8_t* st = smem + s * C::STAGE_BYTES;
-            tma_load_2d(st, &mapA, kx, tileA * 128, &full[s]);
-#pragma unroll
-            for (int j = 0; j < BN / B_BOX; ++j)
-                tma_load_2d(st + kA_BYTES + j * B_BOX * 128, &mapB, kx, tileB * BN + j * B_BOX, &full[s]);
+        WorkIt w = work_begin(plan, c, P);
+        Item it;
+        int i = 0;
+        bool abort = false;
+        while (!abort && work_next(w, plan, P, it)) {
+            int tm, tn;
+            tile_coords(it.tile, plan, tm, tn);
+            for (int k = it.ks; k < it.ke; ++k, ++i) {
+                const int s = i % kStagesTc;
+                if (!mbar_wait(&empty[s], ((i / kStagesTc) & 1) ^ 1)) { atomicExch(&flag[0], 1); abort = true; break; }
+                mbar_arrive_expect_tx(&full[s], kStageBytes);
+                uint8_t* st = smem + s * kStageBytes;
+                tma_load_2d(st, &mapA, k * 64, tm * 128, &full[s]);
+                tma_load_2d(st + kA_BYTES, &mapB, k * 64, tn * kBN, &full[s]);
+            }
         }
     } else if (warp == 1 && lane == 0) {
         // ---------------- MMA issuer
-        const uint32_t idesc = idesc_bf16_f32(128, BN);
-        for (int i = 0; i < nk; ++i) {
-            const int s = i % STAGES;
-            const uint32_t ph = (i / STAGES) & 1;
-            if (!mbar_wait(&full[s], ph)) { atomicExch(abort_flag, 1); break; }
+        const uint32_t idesc = idesc_bf16_f32(128, kBN);
+        WorkIt w = work_begin(plan, c, P);
+        Item it;
+        int i = 0, j = 0;
+        bool abort = false;
+        while (!abort && work_next(w, plan, P, it)) {
+            const int acc = j & 1;
+            if (!mbar_wait(&tempty[acc], ((j >> 1) & 1) ^ 1)) { atomicExch(&flag[0], 1); break; }
             tc_fence_after();
-            const uint32_t a0 = smem_u32(smem + s * C::STAGE_BYTES);
-            const uint32_t b0 = a0 + kA_BYTES;
+            const uint32_t d = tmem + acc * kBN;
+            for (int k = it.ks; k < it.ke; ++k, ++i) {
+                const int s = i % kStagesTc;
+                if (!mbar_wait(&full[s], (i / kStagesTc) & 1)) { atomicExch(&flag[0], 1); abort = true; break; }
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(smem + s * kStageBytes);
+                const uint32_t b0 = a0 + kA_BYTES;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                tc_mma_bf16(tmem, smem_desc_k_sw128(a0 + kk * 32), smem_desc_k_sw128(b0 + kk * 32), idesc,
-                            (i > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < 4; ++kk)
+                    tc_mma_bf16(d, smem_desc_k_sw128(a0 + kk * 32), smem_desc_k_sw128(b0 + kk * 32), idesc,
+                                (k > it.ks || kk > 0) ? 1u : 0u);
+                tc_commit(&empty[s]);
             }
-            tc_commit(&empty[s]);
+            tc_commit(&tfull[acc]);
+            ++j;
         }
-        tc_commit(accum);
-    }
-    __syncthreads();
-
-    // ---------------- epilogue
-    const bool acc_ok = mbar_wait(accum, 0);
-    tc_fence_after();
-    __syncwarp();
-    const bool ok = acc_ok && (*reinterpret_cast<volatile int*>(abort_flag) == 0) && nk > 0;
-    if (!ok && threadIdx.x == 0) report_status(ep.status, LLAMA_ERR_DEVICE_TIMEOUT);
-    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-
-    {
-        // thread = token row m; TMEM columns = features n
-        const int m = tileA * 128 + warp * 32 + lane;
-        const bool row_ok = ok && m < rowsA;
-        const int nbase = tileB * BN;
-        if (ep.mode == EPI_SWIGLU) {
-            // each 32-column chunk holds 16 w1 outputs then the same 16 w3 outputs
+    } else if (warp >= 2) {
+        // ---------------- epilogue: thread = token row of the tile, TMEM columns = features
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        const int epi_tid = threadIdx.x - 64;
+        const int Wsk = plan.sk * KT;
+        const int u0 = run_begin(c, Wsk, P);
+        WorkIt w = work_begin(plan, c, P);
+        Item it;
+        int j = 0;
+        while (work_next(w, plan, P, it)) {
+            const int acc = j & 1;
+            const bool ok_wait = mbar_wait(&tfull[acc], (j >> 1) & 1);
+            tc_fence_after();
+            if (named_any(1, 128, !ok_wait || *reinterpret_cast<volatile int*>(&flag[0]) != 0)) {
+                if (epi_tid == 0) report_status(ep.status, LLAMA_ERR_DEVICE_TIMEOUT);
+                break;
+            }
+            ++j;
+            int tm, tn;
+            tile_coords(it.tile, plan, tm, tn);
+            const int m = tm * 128 + r;
+            const bool row_ok = m < rowsA;
+            const uint32_t tb = tmem + lane_base + acc * kBN;
+            const int nbase = tn * kBN;
+            if (it.ks == 0 && it.ke == KT) {
+                // whole tile: TMEM -> epilogue, 32 features at a time
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
+                for (int cc = 0; cc < kBN / 32; ++cc) {
+                    float v[32];
+                    tmem_ld_32x32b_x32(tb + cc * 32, v);
+                    tc_wait_ld();
+                    if (row_ok) epi_chunk(ep, m, nbase + cc * 32, rowsB, v);
+                }
+                tc_fence_before();
+                mbar_arrive(&tempty[acc]);
+                continue;
+            }
+            // split tile: publish this CTA's partial (feature-major, coalesced over rows)
+            const int tl = it.tile - plan.dp;
+            const int ub = tl * KT;
+            const int cf = owner(ub, Wsk, P), cl = owner(ub + KT - 1, Wsk, P);
+            const int slot = (ub + it.ks == u0) ? 0 : 1;   // the run's first segment, or its last
+            float* my = part + (static_cast<long long>(c) * 2 + slot) * kPartFloats + r;
+#pragma unroll 1
+            for (int cc = 0; cc < kBN / 32; ++cc) {
                 float v[32];
-                tmem_ld_32x32b_x32(trow + c * 32, v);
+                tmem_ld_32x32b_x32(tb + cc * 32, v);
                 tc_wait_ld();
-                const int n0 = nbase + c * 32;
-                if (row_ok && n0 < rowsB) {
-                    float g16[16];
 #pragma unroll
-                    for (int t = 0; t < 16; ++t) g16[t] = silu_f(v[t]) * v[16 + t];
-                    bf16* dst = static_cast<bf16*>(ep.g) + static_cast<long long>(m) * ep.H + (n0 / 32) * 16;
-                    uint4* d4 = reinterpret_cast<uint4*>(dst);
+                for (int t = 0; t < 32; ++t) my[(cc * 32 + t) * 128] = v[t];
+            }
+            __threadfence();
+            named_sync(1, 128);
+            if (epi_tid == 0) flag[1] = atomicAdd(&counters[tl], 1);
+            named_sync(1, 128);
+            if (flag[1] != cl - cf) {   // not the last contributor
+                tc_fence_before();
+                mbar_arrive(&tempty[acc]);
+                continue;
+            }
+            __threadfence();
+            // last contributor: sum the partials in CTA order, then the epilogue
+#pragma unroll 1
+            for (int cc = 0; cc < kBN / 32; ++cc) {
+                float own[32], v[32];
+                tmem_ld_32x32b_x32(tb + cc * 32, own);
+                tc_wait_ld();
 #pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        uint4 u;
-                        u.x = pack_bf16x2(g16[8 * q + 0], g16[8 * q + 1]);
-                        u.y = pack_bf16x2(g16[8 * q + 2], g16[8 * q + 3]);
-                        u.z = pack_bf16x2(g16[8 * q + 4], g16[8 * q + 5]);
-                        u.w = pack_bf16x2(g16[8 * q + 6], g16[8 * q + 7]);
-                        d4[q] = u;
+                for (int t = 0; t < 32; ++t) v[t] = 0.f;
+                for (int cb = cf; cb <= cl; ++cb) {
+                    if (cb == c) {
+#pragma unroll
+                        for (int t = 0; t < 32; ++t) v[t] += own[t];
+                    } else {
+                        const int sl = run_begin(cb, Wsk, P) >= ub ? 0 : 1;
+                        const float* pp = part + (static_cast<long long>(cb) * 2 + sl) * kPartFloats + r;
+                        float f[32];
+#pragma unroll
+                        for (int t = 0; t < 32; ++t) f[t] = pp[(cc * 32 + t) * 128];
+#pragma unroll
+                        for (int t = 0; t < 32; ++t) v[t] += f[t];
                     }
                 }
+                if (row_ok) epi_chunk(ep, m, nbase + cc * 32, rowsB, v);
             }
-        } else {
-#pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                float v[32];
-                tmem_ld_32x32b_x32(trow + c * 32, v);
-                tc_wait_ld();
-                const int n0 = nbase + c * 32;
-                if (!row_ok || n0 >= rowsB) continue;
-                if (ep.mode == EPI_QKV) {
-                    const int pos = ep.tok_pos[m];
-                    if (pos < 0 || pos >= ep.max_seq) continue;
-                    bf16* dst;
-                    bool rot;
-                    int d0;
-                    if (n0 < ep.nq) {
-                        d0 = n0 % ep.hd;
-                        rot = true;
-                        dst = static_cast<bf16*>(ep.q) + static_cast<long long>(m) * ep.nq + n0;
-                    } else {
-                        int cc = n0 - ep.nq;
-                        bf16* cache = static_cast<bf16*>(ep.kc);
-                        rot = cc < ep.nkvc;
-                        if (!rot) { cc -= ep.nkvc; cache = static_cast<bf16*>(ep.vc); }
-                        const int head = cc / ep.hd;
-                        d0 = cc % ep.hd;
-                        const int row = ep.tok_row ? ep.tok_row[m] : m;
-                        dst = cache + static_cast<long long>(row) * ep.kv_row_stride +
-                              (static_cast<long long>(head) * ep.max_seq + pos) * ep.hd + d0;
-                    }
-                    if (rot) {
-#pragma unroll
-                        for (int t = 0; t < 32; t += 2) rope_pair(ep.rope, ep.hd, pos, (d0 + t) >> 1, v[t], v[t + 1]);
-                    }
-                    store32_bf16(dst, v);
-                } else {
-                    float* o = ep.out + static_cast<long long>(m) * ep.ldo + n0;
-                    const int lim = min(32, rowsB - n0);
-                    if (lim == 32 && (ep.ldo % 4) == 0) {
-                        float4* o4 = reinterpret_cast<float4*>(o);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            float4 r = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                            if (ep.mode == EPI_RESID_F32) {
-                                const float4 p = o4[q];
-                                r.x += p.x; r.y += p.y; r.z += p.z; r.w += p.w;
-                            }
-                            o4[q] = r;
-                        }
-                    } else {
-                        for (int t = 0; t < lim; ++t) o[t] = (ep.mode == EPI_RESID_F32) ? o[t] + v[t] : v[t];
-                    }
-                }
-            }
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            if (epi_tid == 0) counters[tl] = 0;
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+    if (warp == 1) tmem_dealloc(tmem, 2 * kBN);
 }
 
 // ---------------------------------------------------------------- host side
@@ -263,38 +394,73 @@ int encode_kmajor_bf16(CUtensorMap* map, const void* base, int rows, int cols, i
     return LLAMA_OK;
 }
 
-template <int BN, int STAGES, int B_BOX>
-static int launch_tc(const CUtensorMap& a, const CUtensorMap& b, int rowsA, int rowsB, int K, int splits,
-                     const Epi& ep, cudaStream_t st) {
-    using C = TcCfg<BN>;
-    constexpr int smem = STAGES * C::STAGE_BYTES + 1024 + (2 * STAGES + 1) * 8 + 16;
-    auto kern = linear_tc_kernel<BN, STAGES, B_BOX>;
+// Work split of one prefill projection over P persistent CTAs: whole tiles
+// round-robin, and a stream-K run over the tail unless the last wave is nearly
+// full (>= 85 % of the CTAs) or there is no workspace for split tiles.
+static void plan_tc(int T, int KT, int P, bool can_split, TcPlan* p, int* grid) {
+    p->dp = T;
+    p->sk = 0;
+    *grid = T < P ? T : P;
+    if (!can_split || T % P == 0 || KT < 2) return;
+    const int full = T / P, R = T % P;
+    if (full >= 1 && R * 100 >= 85 * P) return;
+    if (full >= 1) {
+        p->dp = (full - 1) * P;
+        p->sk = T - p->dp;
+        *grid = P;
+    } else {
+        // fewer tiles than SMs: split each tile at most 4 ways
+        p->dp = 0;
+        p->sk = T;
+        const long long g = std::min<long long>(std::min<long long>(P, 4LL * T), static_cast<long long>(T) * KT);
+        *grid = static_cast<int>(g);
+    }
+    if (static_cast<long long>(p->sk) * KT * (*grid) >= (1LL << 31)) {   // keep unit arithmetic in int
+        p->dp = T;
+        p->sk = 0;
+        *grid = T < P ? T : P;
+    }
+}
+
+static int g_sms_tc = 0;
+
+int linear_bf16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
+                   int* counters, cudaStream_t st) {
+    if (M <= 0 || N <= 0) return LLAMA_OK;
+    constexpr int smem = 1024 + kStagesTc * kStageBytes + (2 * kStagesTc + 4) * 8 + 16;
+    static_assert(smem <= 227 * 1024, "shared memory per CTA");
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(linear_tc_kernel)");
+        cudaError_t e = cudaFuncSetAttribute(linear_tcp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(linear_tcp_kernel)");
         attr_set = true;
     }
-    const int KT = (K + 63) / 64;
-    const int per = (KT + splits - 1) / splits;
-    const int z = (KT + per - 1) / per;   // every split gets >= 1 k-tile
-    dim3 grid((rowsA + 127) / 128, (rowsB + BN - 1) / BN, z);
-    kern<<<grid, 128, smem, st>>>(a, b, rowsA, rowsB, K, per, ep);
-    LLB_CHECK_LAUNCH("linear_tc_kernel");
+    if (g_sms_tc == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&g_sms_tc, cudaDevAttrMultiProcessorCount, dev);
+        if (g_sms_tc <= 0) g_sms_tc = 148;
+        if (g_sms_tc > kMaxDecodeCtas) g_sms_tc = kMaxDecodeCtas;
+    }
+    TcPlan plan;
+    plan.TM = (M + 127) / 128;
+    plan.TN = (N + kBN - 1) / kBN;
+    plan.KT = (K + 63) / 64;
+    const long long T = static_cast<long long>(plan.TM) * plan.TN;
+    if (T >= (1LL << 30)) { set_error("prefill projection too large (%lld tiles)", T); return LLAMA_ERR_INVALID_ARG; }
+    int grid = 0;
+    plan_tc(static_cast<int>(T), plan.KT, g_sms_tc, part != nullptr && counters != nullptr, &plan, &grid);
+    if (plan.sk > kMaxTiles) { set_error("internal: %d split tiles exceed the counters", plan.sk); return LLAMA_ERR_INVALID_ARG; }
+    linear_tcp_kernel<<<grid, kThreadsTc, smem, st>>>(mapA->a128, mapW->b, M, N, plan, ep, part, counters);
+    LLB_CHECK_LAUNCH("linear_tcp_kernel");
     return LLAMA_OK;
 }
 
-int linear_bf16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep,
-                   cudaStream_t st) {
-    if (M <= 0 || N <= 0) return LLAMA_OK;
-    return launch_tc<256, 4, 256>(mapA->a128, mapW->b, M, N, K, 1, ep, st);
-}
-
 int linear_bf16(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
-                int* counters, cudaStream_t st, bool pdl, const NormIO* nio, const NextProj* next) {
-    if (M <= 64) return linear_bf16_decode(mapA, mapW, M, N, K, ep, part, counters, st, pdl, nio, next);
+                size_t part_bytes, int* counters, cudaStream_t st, bool pdl, const NormIO* nio) {
+    if (M <= 64) return linear_bf16_decode(mapA, mapW, M, N, K, ep, part, part_bytes, counters, st, pdl, nio);
     if (nio && (nio->ssq_in || nio->ssq_out)) { set_error("fused RMSNorm is a decode-shape feature"); return LLAMA_ERR_INVALID_ARG; }
-    return linear_bf16_tc(mapA, mapW, M, N, K, ep, st);
+    return linear_bf16_tc(mapA, mapW, M, N, K, ep, part, counters, st);
 }
 
 }  // namespace llb

@@ -14,9 +14,13 @@ namespace llb {
 constexpr int kMaxRows = 256;         // max_batch_size limit (by-value row tables)
 constexpr int kChunk = 64;            // keys per chunk in decode attention
 constexpr int kMaxDecodeCtas = 256;   // persistent CTAs of the decode projection kernel
-// fp32 partials of split tiles: two 128 x 64 blocks per persistent CTA
+// fp32 partials of split tiles, two per persistent CTA: 128 x 64 blocks in the
+// decode projection, 128 x 256 tiles in the prefill projection
 constexpr size_t kDecodePartBytes = static_cast<size_t>(kMaxDecodeCtas) * 2 * 128 * 64 * 4;
+constexpr size_t kPrefillPartBytes = static_cast<size_t>(kMaxDecodeCtas) * 2 * 128 * 256 * 4;
+constexpr size_t kGemmPartBytes = kPrefillPartBytes > kDecodePartBytes ? kPrefillPartBytes : kDecodePartBytes;
 constexpr int kMaxTiles = 4096;       // tile counters: N / 128 of the widest projection
+constexpr int kMaxAttnCtas = 1024;    // persistent CTAs of the decode attention kernel
 
 // Token -> (batch row, position) map of one prefill call, passed by value.
 struct RowTable {
@@ -66,13 +70,6 @@ struct NormIO {
     float* ssq_out;
     void* y_out;
     const float* w_next;
-};
-
-// The projection launched after this one in the decode chain (its weight
-// map, N rows, K columns): used to warm L2 with its first weight tiles.
-struct NextProj {
-    const CUtensorMap* map;
-    int N, K;
 };
 
 struct TmaMaps {               // tensor maps of one K-major bf16 matrix
@@ -127,8 +124,8 @@ struct Model {
     int* tok_pos;    // [Mmax]
     int* last_idx;   // [Bmax]
     float* logits_ws;   // [Bmax, V]
-    float* part_o;      // [Bmax*nh*n_splits, hd]
-    float* part_ml;     // [Bmax*nh*n_splits, 2]
+    float* part_o;      // [2 * kMaxAttnCtas * n_rep, hd] split partials of decode attention
+    float* part_ml;     // [2 * kMaxAttnCtas * n_rep, 2]
     int* attn_cnt;      // [Bmax*nkv] split arrival counters (zero between launches)
     float* gemm_part;   // split-tile partials of the decode projection kernel
     int* gemm_cnt;      // per-tile arrival counters (zero between launches)
@@ -158,17 +155,17 @@ int launch_copy_interleave_w13(const void* src, void* w13, int H, int dim, int w
 // bf16 uses tcgen05 with the given maps (A-side/W-side), fp32 the SIMT kernel.
 int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, const void* W,
                const TmaMaps* mapW, int M, int N, int K, const Epi& ep, cudaStream_t st, bool pdl = false,
-               const NormIO* nio = nullptr, const NextProj* next = nullptr);
+               const NormIO* nio = nullptr);
 int linear_f32(const float* A, const float* W, int M, int N, int K, const Epi& ep, cudaStream_t st);
-int linear_bf16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep,
-                   cudaStream_t st);
+// Prefill-shaped projection; with part/counters (kGemmPartBytes, kMaxTiles
+// zeroed ints) the tail wave is split stream-K, without them whole tiles only.
+int linear_bf16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
+                   int* counters, cudaStream_t st);
 int linear_bf16_decode(const TmaMaps* mapX, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
-                       int* counters, cudaStream_t st, bool pdl, const NormIO* nio = nullptr,
-                       const NextProj* next = nullptr);
+                       size_t part_bytes, int* counters, cudaStream_t st, bool pdl, const NormIO* nio = nullptr);
 // bf16 projection: M <= 64 token rows -> linear_bf16_decode, else linear_bf16_tc.
 int linear_bf16(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
-                int* counters, cudaStream_t st, bool pdl = false, const NormIO* nio = nullptr,
-                const NextProj* next = nullptr);
+                size_t part_bytes, int* counters, cudaStream_t st, bool pdl = false, const NormIO* nio = nullptr);
 
 int launch_attention_prefill(const Model* m, int layer, const RowTable& rt, cudaStream_t st);
 int launch_attention_prefill_tc(const Model* m, int layer, const RowTable& rt, cudaStream_t st);

@@ -96,5 +96,5 @@ extern "C" int llama_op_linear_noalloc(const void* A, const void* W, int M, int 
     ep.mode = EPI_STORE_F32;
     ep.out = out;
     ep.ldo = N;
-    return linear_bf16_decode(&ma, &mw, M, N, K, ep, part, cnt, st, false);
+    return linear_bf16_decode(&ma, &mw, M, N, K, ep, part, kNoAllocPartBytes, cnt, st, false);
 }

@@ -32,12 +32,15 @@ LLAMA_API int llama_op_rmsnorm(const float* x, const float* w, int M, int dim, f
  *   out fp32 [M, N] (row-major, overwritten).  K % 8 == 0 for bf16.
  * The bf16 kernels are the ones the model path uses: for M <= 64 the
  * persistent weight-streaming kernel (the weight is the 128-row MMA operand,
- * K split across CTAs), else the 128 x 256-tile kernel.
+ * K split across CTAs), else the persistent 128 x 256-tile kernel.
  *   workspace  device scratch of llama_op_linear_workspace_bytes(), 256-byte
- *              aligned, zero-filled before its first use (the kernel leaves
- *              its counters at zero again); needed for bf16 with M <= 64,
- *              otherwise may be NULL.  Calls sharing a workspace must not
- *              overlap on the device. */
+ *              aligned, zero-filled before its first use (the kernels leave
+ *              their counters at zero again).  Required for bf16 with
+ *              M <= 64.  Optional for M > 64: with it the last wave of tiles
+ *              is split along K over all SMs (stream-K), with NULL every tile
+ *              runs whole.  A non-NULL workspace that is too small or
+ *              misaligned is rejected (LLAMA_ERR_INVALID_ARG).  Calls sharing
+ *              a workspace must not overlap on the device. */
 LLAMA_API size_t llama_op_linear_workspace_bytes(void);
 LLAMA_API int llama_op_linear(const void* A, const void* W, int M, int N, int K, int dtype,
                     float* out, void* workspace, size_t workspace_bytes, void* stream);

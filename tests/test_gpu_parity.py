@@ -74,6 +74,56 @@ def test_linear_bf16_tcgen05_kernel(llb, M, N, K):
     np.testing.assert_allclose(got, want, atol=1e-3 + 1e-4 * np.abs(want).max())
 
 
+@pytest.mark.gpu
+@pytest.mark.parametrize("M,N,K", [
+    (512, 9472, 256),      # 148 tiles: one full wave, whole tiles only
+    (2048, 2560, 1024),    # 160 tiles: all split along K over the SMs (stream-K)
+    (2048, 4864, 512),     # 304 tiles: one wave of whole tiles, then a stream-K run
+    (256, 35584, 256),     # 278 tiles: last wave 88 % full, whole tiles only
+    (1000, 1000, 4160),    # ragged M, N and K, 32 tiles split up to 4 ways
+])
+def test_linear_bf16_prefill_work_split(llb, M, N, K):
+    """The persistent prefill projection under each of its work splits, with
+    and without the split-tile workspace; split results are bit-identical
+    from run to run (partials added in a fixed order)."""
+    g = torch.Generator().manual_seed(11 * M + N + K)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16).cuda()
+    W = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16).cuda()
+    want = A.cpu().double().numpy() @ W.cpu().double().numpy().T
+    outs = []
+    for ws in (None, False, None):
+        out = torch.full((M, N), float("nan"), device="cuda")
+        if ws is False:
+            llb.op_linear_whole_tiles(A, W, out)
+        else:
+            llb.op_linear(A, W, out)
+        torch.cuda.synchronize()
+        got = out.cpu().double().numpy()
+        assert np.isfinite(got).all()
+        assert rel_l2(got, want) < 2e-5
+        np.testing.assert_allclose(got, want, atol=1e-3 + 1e-4 * np.abs(want).max())
+        outs.append(out.cpu())
+    assert torch.equal(outs[0], outs[2])
+
+
+@pytest.mark.gpu
+def test_linear_bf16_prefill_7b_qkv_sampled(llb):
+    """7B wq/wk/wv shape at 4 x 512 prompt tokens (2048 x 12288 x 4096),
+    checked on 64 sampled token rows against fp64."""
+    M, N, K = 2048, 12288, 4096
+    g = torch.Generator().manual_seed(77)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    W = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16)
+    out = torch.empty((M, N), device="cuda")
+    llb.op_linear(A.cuda(), W.cuda(), out)
+    torch.cuda.synchronize()
+    rows = torch.randperm(M, generator=g)[:64].sort().values
+    want = A[rows].double().numpy() @ W.double().numpy().T
+    got = out.cpu()[rows].double().numpy()
+    assert rel_l2(got, want) < 2e-5
+    np.testing.assert_allclose(got, want, atol=1e-3 + 1e-4 * np.abs(want).max())
+
+
 # ----------------------------------------------------------------------------- sampling
 
 def test_greedy_sampler_ties_and_values(llb):
