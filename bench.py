@@ -318,7 +318,7 @@ def run_ours(a, rank, world, local_rank):
                      "achieved": round(dec_gbs, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(dec_gbs / hbm, 4), "peak_source": f"{peak_src} hbm_gbs",
                      "traffic": None, "launches": len(dec)},
-        "roofline_prefill": {"bound": "tensor", "kernel": "linear_tc_kernel (prefill orientation)",
+        "roofline_prefill": {"bound": "tensor", "kernel": "linear_tcp_kernel (prefill projections: wq/wk/wv, wo, w1/w3, w2; persistent, 128x256 tiles)",
                              "achieved": round(pre_tfs, 1), "peak": tc_burst, "unit": "TFLOP/s",
                              "frac": round(pre_tfs / tc_burst, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
                              "traffic": None, "launches": len(pre)},
