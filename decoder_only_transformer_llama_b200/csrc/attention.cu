@@ -68,6 +68,8 @@ template <> struct Vec<bf16, 4> {
 // its run (slot 0 = the run's first segment, slot 1 = its last); each writes
 // its unnormalised (o, max, sum) and the CTA that arrives last at the pair's
 // counter merges them in CTA order (deterministic).  No CTA waits for another.
+constexpr int kPrefetchUnits = 4;   // cache blocks per CTA pulled into L2 ahead of the grid dependency
+
 __device__ __forceinline__ long long run_begin64(long long c, long long W, long long P) { return c * W / P; }
 __device__ __forceinline__ int owner64(long long u, long long W, long long P) {
     return static_cast<int>(((u + 1) * P - 1) / W);
@@ -130,9 +132,11 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
         __syncthreads();
     };
     // Before the previous kernel (which writes this step's K/V row and q) has
-    // finished: plan with the positions as they read now and pull this CTA's
-    // cache blocks into L2 (a prefetch only: nothing read here is used, and L2
-    // is coherent with the writes that follow).  After the grid dependency has
+    // finished: plan with the positions as they read now and pull the first
+    // kPrefetchUnits cache blocks of this CTA's run into L2 (a prefetch only:
+    // nothing read here is used, and L2 is coherent with the writes that
+    // follow; the cap keeps the total far below the L2 size, so long runs do
+    // not evict their own blocks before use).  After the grid dependency has
     // resolved, the positions are read again and the plan is redone if any
     // changed.
     make_plan();
@@ -150,7 +154,8 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
             long long rem = v0 - static_cast<long long>(s_cum[lo]) * nkv;
             int g = static_cast<int>(rem / s_nch[b]);
             int jj = static_cast<int>(rem - static_cast<long long>(g) * s_nch[b]);
-            for (long long u = v0; u < v1 && b < B; ++u) {
+            const long long v1p = v1 < v0 + kPrefetchUnits ? v1 : v0 + kPrefetchUnits;
+            for (long long u = v0; u < v1p && b < B; ++u) {
                 const int ctx = s_pos[b] + 1;
                 const int j0 = jj * kChunk;
                 const int n = min(kChunk, ctx - j0);

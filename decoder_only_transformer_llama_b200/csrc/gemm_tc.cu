@@ -13,13 +13,14 @@
 // tiles in flight at any time share a few hundred KB of A and B in L2.
 //
 // The kernel is persistent: one CTA per SM walks a fixed list of work items.
-// The first `dp` tiles go round-robin, one whole tile per item.  The last
-// `sk` tiles (the partial last wave plus one full wave) form one flat run of
-// sk * K/64 k-tile units cut into P equal contiguous runs (stream-K), so every
-// SM ends at the same time whatever the tile count.  A tile split between CTAs
-// is finished by the contributor that arrives last at the tile's counter: it
-// adds the fp32 partials in CTA order (deterministic) and applies the
-// epilogue; no CTA ever waits for another.
+// The first `dp` tiles (all full waves) go round-robin, one whole tile per
+// item: the CTAs of a wave walk K in step, so the A and B tiles in flight at
+// any moment share a few MB of L2.  The `sk` tiles of a partial last wave form
+// one flat run of sk * K/64 k-tile units cut into psk equal contiguous runs
+// (stream-K, at most 4 runs per tile), so the SMs end together.  A tile split
+// between CTAs is finished by the contributor that arrives last at the tile's
+// counter: it adds the fp32 partials in CTA order (deterministic) and applies
+// the epilogue; no CTA ever waits for another.
 //
 // Warp roles (192 threads):
 //   warp 0 lane 0  TMA producer (4-deep ring of 128x64 A + 256x64 B tiles)
@@ -67,10 +68,11 @@ __device__ __forceinline__ void store32_bf16(bf16* dst, const float* v) {
     }
 }
 
-// Work list of one CTA: whole tiles c, c+P, ... below dp, then its stream-K run.
+// Work list of one CTA: whole tiles c, c+P, ... below dp, then (c < psk) its
+// stream-K run over the last sk tiles.
 struct TcPlan {
     int TM, TN, KT;
-    int dp, sk;
+    int dp, sk, psk;
 };
 struct Item {
     int tile, ks, ke;
@@ -83,8 +85,8 @@ __device__ __forceinline__ WorkIt work_begin(const TcPlan& p, int c, int P) {
     WorkIt w;
     w.next_dp = c;
     const int W = p.sk * p.KT;
-    w.u = run_begin(c, W, P);
-    w.u1 = run_begin(c + 1, W, P);
+    w.u = c < p.psk ? run_begin(c, W, p.psk) : 0;
+    w.u1 = c < p.psk ? run_begin(c + 1, W, p.psk) : 0;
     return w;
 }
 
@@ -269,7 +271,8 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const int epi_tid = threadIdx.x - 64;
         const int Wsk = plan.sk * KT;
-        const int u0 = run_begin(c, Wsk, P);
+        const int Psk = plan.psk;
+        const int u0 = c < Psk ? run_begin(c, Wsk, Psk) : 0;
         WorkIt w = work_begin(plan, c, P);
         Item it;
         int j = 0;
@@ -304,7 +307,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
             // split tile: publish this CTA's partial (feature-major, coalesced over rows)
             const int tl = it.tile - plan.dp;
             const int ub = tl * KT;
-            const int cf = owner(ub, Wsk, P), cl = owner(ub + KT - 1, Wsk, P);
+            const int cf = owner(ub, Wsk, Psk), cl = owner(ub + KT - 1, Wsk, Psk);
             const int slot = (ub + it.ks == u0) ? 0 : 1;   // the run's first segment, or its last
             float* my = part + (static_cast<long long>(c) * 2 + slot) * kPartFloats + r;
 #pragma unroll 1
@@ -338,7 +341,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
 #pragma unroll
                         for (int t = 0; t < 32; ++t) v[t] += own[t];
                     } else {
-                        const int sl = run_begin(cb, Wsk, P) >= ub ? 0 : 1;
+                        const int sl = run_begin(cb, Wsk, Psk) >= ub ? 0 : 1;
                         const float* pp = part + (static_cast<long long>(cb) * 2 + sl) * kPartFloats + r;
                         float f[32];
 #pragma unroll
@@ -395,31 +398,28 @@ int encode_kmajor_bf16(CUtensorMap* map, const void* base, int rows, int cols, i
 }
 
 // Work split of one prefill projection over P persistent CTAs: whole tiles
-// round-robin, and a stream-K run over the tail unless the last wave is nearly
-// full (>= 85 % of the CTAs) or there is no workspace for split tiles.
+// round-robin for every full wave, and a stream-K run over a partial last
+// wave unless it is nearly full (>= 85 % of the CTAs) or there is no workspace
+// for split tiles.  A split tile is cut at most 4 ways (finishing it reads the
+// other pieces' 128 KB partials back).
 static void plan_tc(int T, int KT, int P, bool can_split, TcPlan* p, int* grid) {
     p->dp = T;
     p->sk = 0;
+    p->psk = 0;
     *grid = T < P ? T : P;
     if (!can_split || T % P == 0 || KT < 2) return;
     const int full = T / P, R = T % P;
     if (full >= 1 && R * 100 >= 85 * P) return;
-    if (full >= 1) {
-        p->dp = (full - 1) * P;
-        p->sk = T - p->dp;
-        *grid = P;
-    } else {
-        // fewer tiles than SMs: split each tile at most 4 ways
-        p->dp = 0;
-        p->sk = T;
-        const long long g = std::min<long long>(std::min<long long>(P, 4LL * T), static_cast<long long>(T) * KT);
-        *grid = static_cast<int>(g);
-    }
-    if (static_cast<long long>(p->sk) * KT * (*grid) >= (1LL << 31)) {   // keep unit arithmetic in int
+    p->dp = full * P;
+    p->sk = R;
+    long long psk = std::min<long long>(std::min<long long>(P, 4LL * R), static_cast<long long>(R) * KT);
+    if (static_cast<long long>(R) * KT * psk >= (1LL << 31)) {   // keep unit arithmetic in int
         p->dp = T;
         p->sk = 0;
-        *grid = T < P ? T : P;
+        return;
     }
+    p->psk = static_cast<int>(psk);
+    *grid = full >= 1 ? P : p->psk;
 }
 
 static int g_sms_tc = 0;
