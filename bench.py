@@ -98,6 +98,25 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- roofline bookkeeping
 
+def _traffic(kernel):
+    """DRAM bytes per launch of `kernel` in this workload from the committed
+    ncu record (profiles/dram_traffic_7b.json), or None when the kernel's
+    sources no longer match the ones the counters were taken on."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic_7b.json")) as f:
+            rec = json.load(f)[kernel]
+        m = hashlib.sha256()
+        for name in rec["source_files"]:
+            with open(os.path.join(ROOT, "decoder_only_transformer_llama_b200", "csrc", name), "rb") as f:
+                m.update(f.read())
+        if m.hexdigest() != rec["source_sha256"]:
+            return None
+        return int(rec["bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def decode_step_bytes(s, B, ctx):
     """Algorithmic bytes of one decode step of B rows at context ctx: every
     weight matrix once (bf16), the norm weights (fp32), B embedding rows, the
@@ -317,11 +336,15 @@ def run_ours(a, rank, world, local_rank):
         "roofline": {"bound": "hbm", "kernel": "linear_decode_kernel (decode projections: wq/wk/wv, wo, w1/w3, w2, output)",
                      "achieved": round(dec_gbs, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(dec_gbs / hbm, 4), "peak_source": f"{peak_src} hbm_gbs",
-                     "traffic": None, "launches": len(dec)},
+                     "traffic": _traffic("linear_decode_kernel"), "launches": len(dec),
+                     "traffic_what": "DRAM bytes per launch, mean over one decode step's 129 projection launches "
+                                     "(ncu record in profiles/dram_traffic_7b.json; null if the kernel changed since)"},
         "roofline_prefill": {"bound": "tensor", "kernel": "linear_tcp_kernel (prefill projections: wq/wk/wv, wo, w1/w3, w2; persistent, 128x256 tiles)",
                              "achieved": round(pre_tfs, 1), "peak": tc_burst, "unit": "TFLOP/s",
                              "frac": round(pre_tfs / tc_burst, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
-                             "traffic": None, "launches": len(pre)},
+                             "traffic": _traffic("linear_tcp_kernel"), "launches": len(pre),
+                             "traffic_what": "DRAM bytes per launch, mean over the 128 projection launches of one "
+                                             "prefill (ncu record in profiles/dram_traffic_7b.json; null if the kernel changed since)"},
         "decode_path_hbm": {"achieved": round(decode_gbs_path, 1), "unit": "GB/s",
                             "frac": round(decode_gbs_path / hbm, 4),
                             "what": "all algorithmic bytes of a decode step (weights, KV read+write, logits) / decode time"},
