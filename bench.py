@@ -98,6 +98,20 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- roofline bookkeeping
 
+def max_over_ranks(vals, world):
+    """Element-wise maximum of the float64 tensor `vals` over all ranks, in
+    place: a replicated job ends when its slowest rank does."""
+    if world > 1:
+        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
+    return vals
+
+
+def whole_job_rate(units_per_rank, world, ms):
+    """Units that all `world` ranks processed, per second of the slowest rank's
+    device time `ms` (every rank runs the same fixed work: weak scaling)."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 def _traffic(kernel):
     """DRAM bytes per launch of `kernel` in this workload from the committed
     ncu record (profiles/dram_traffic_7b.json), or None when the kernel's
@@ -288,15 +302,13 @@ def run_ours(a, rank, world, local_rank):
 
     # ---------------- max over ranks
     vals = torch.tensor([total_ms, prefill_ms, decode_ms, e2e_dec_ms, t_e2e * 1e3], device=dev, dtype=torch.float64)
-    if world > 1:
-        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
-    total_ms, prefill_ms, decode_ms, e2e_dec_ms, e2e_wall_ms = vals.tolist()
+    total_ms, prefill_ms, decode_ms, e2e_dec_ms, e2e_wall_ms = max_over_ranks(vals, world).tolist()
 
     dec_tokens = world * a.steps * B * steps_dec
     pre_tokens = world * a.steps * B * T
-    value = dec_tokens / (decode_ms / 1e3)
-    prefill_tps = pre_tokens / (prefill_ms / 1e3)
-    e2e_value = dec_tokens / (e2e_dec_ms / 1e3)
+    value = whole_job_rate(a.steps * B * steps_dec, world, decode_ms)
+    prefill_tps = whole_job_rate(a.steps * B * T, world, prefill_ms)
+    e2e_value = whole_job_rate(a.steps * B * steps_dec, world, e2e_dec_ms)
 
     dec = [r for r in recs if r[0] > 0 and 0 < r[3] <= 64]
     pre = [r for r in recs if r[0] > 0 and r[3] > 64]
@@ -485,7 +497,8 @@ def run_workload(a):
     """Throughput lines for the other workloads (one JSON line per measurement):
     7b_layer_decode (one 7B layer, cache pre-filled, B x context grid),
     13b_ragged (16 prompts of 64..1024 tokens, then 128 decode steps),
-    70b_slice (16 GQA layers, 8 x 2048 prefill, then decode), tiny_f32."""
+    70b_slice (16 GQA layers, 8 x 2048 prefill, then decode), tiny_f32,
+    7b_batch1 (the full 7B shape, one 512-token prompt, then 256 decode steps)."""
     import decoder_only_transformer_llama_b200 as llb
     from workloads import make_lengths, make_normal
     dev = torch.device("cuda", 0)

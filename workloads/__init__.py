@@ -80,6 +80,9 @@ WORKLOADS: Dict[str, dict] = {
                temperature=0.6, top_p=0.9),
     "13b_ragged": dict(index=3, shape=L13B, batch=16, min_len=64, max_len=1024, decode_steps=128),
     "70b_slice": dict(index=4, shape=L70B_SLICE, batch=8, prompt_len=2048, decode_to=4096),
+    # the full 7B shape at batch 1 (same weights and prompt seed as "7b"): the
+    # single-sequence decode case that a 7B roofline target is quoted on
+    "7b_batch1": dict(index=2, shape=L7B, batch=1, prompt_len=512, decode_steps=256),
 }
 
 
