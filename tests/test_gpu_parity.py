@@ -260,6 +260,57 @@ def test_small_bf16_gqa_ragged_prefill_and_decode(llb):
     _oracle_check(SMALL_BF16, w, seq, gl, lens, BF16_TOL)
 
 
+def test_small_bf16_decode_with_top_p_sampling(llb):
+    """Decode steps that sample in the step itself (temperature 0.6, top-p 0.9,
+    one seeded uniform per row and step): every sampled id equals the oracle's
+    nucleus draw on the step's own logits with the same uniform (or, for a draw
+    within rounding of a boundary, lies in the kept set), and the logits of the
+    sampled sequence match the oracle's teacher-forced forward pass."""
+    T_, P_ = 0.6, 0.9
+    w = make_weights(SMALL_BF16, 98)
+    m = build_model(SMALL_BF16, w)
+    B, T, steps = 3, 48, 8
+    lens = [48, 17, 30]
+    toks = make_tokens(SMALL_BF16.vocab_size, (B, T), token_seed(5)).cuda()
+    logits = torch.empty(B, SMALL_BF16.vocab_size, device="cuda")
+    m.prefill(toks, lens=lens, logits=logits)
+    uni = make_uniforms((steps + 1, B), 3100)
+    cur = torch.empty(B, dtype=torch.int32, device="cuda")
+    llb.sample(logits, T_, P_, uni[0].cuda(), cur)
+    seq = [toks[b, :lens[b]].cpu().tolist() for b in range(B)]
+    gl = [[logits[b].cpu().numpy().copy()] for b in range(B)]
+    pos = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    nxt = torch.empty(B, dtype=torch.int32, device="cuda")
+    ambiguous = 0
+    for i in range(steps):
+        for b in range(B):
+            seq[b].append(int(cur[b]))
+        step_logits = torch.empty(B, SMALL_BF16.vocab_size, device="cuda")
+        u = uni[i + 1]
+        m.decode_step(cur, pos, temperature=T_, top_p=P_, uniforms=u.cuda(), next_tokens=nxt, logits=step_logits)
+        torch.cuda.synchronize()
+        got = nxt.cpu().tolist()
+        for b in range(B):
+            row = step_logits[b].cpu().numpy().astype(np.float64)
+            gl[b].append(row.copy())
+            if O.sample_margins(row, T_, P_, float(u[b])) < 1e-9:
+                ambiguous += 1
+                assert got[b] in O.top_p_kept(row, T_, P_)
+            else:
+                assert got[b] == O.sample_top_p(row, T_, P_, float(u[b])), (i, b)
+        cur = nxt.clone()
+        pos += 1
+    assert ambiguous == 0
+    assert m.status() == 0
+    m.close()
+    args = oracle_args(SMALL_BF16)
+    w64 = to_numpy_f64_weights(w)
+    for b in range(B):
+        want = O.forward(args, w64, seq[b], 0, O.new_cache(args))[lens[b] - 1:]
+        got = np.stack(gl[b][:want.shape[0]])
+        assert rel_l2(got, want) <= BF16_TOL, (b, rel_l2(got, want))
+
+
 @pytest.mark.parametrize("B,L", [(1, 128), (8, 1024), (32, 4096)])
 def test_7b_layer_decode_against_oracle(llb, B, L):
     """One 7B-shaped layer (bf16, fp32 norms), KV cache filled with N(0,1) for
