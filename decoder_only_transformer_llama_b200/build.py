@@ -72,7 +72,11 @@ def build(force: bool = False, jobs: int = 0, verbose: bool = False, extra=()) -
                 msg = f.result()
                 if verbose and msg:
                     print(msg, file=sys.stderr)
-    if todo or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
+    manifest = os.path.join(BUILD, "link.txt")   # the object set of the last link
+    listed = "\n".join(os.path.basename(o) for o in objs)
+    same_set = os.path.exists(manifest) and open(manifest).read() == listed
+    if todo or not same_set or not os.path.exists(LIB) or \
+            any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
         tmp = LIB + ".tmp"
         # static cudart; the driver is reached through cudaGetDriverEntryPoint,
         # so the library loads (and its host-side checks run) without a GPU
@@ -81,6 +85,8 @@ def build(force: bool = False, jobs: int = 0, verbose: bool = False, extra=()) -
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
         os.replace(tmp, LIB)
+        with open(manifest, "w") as f:
+            f.write(listed)
     return LIB
 
 

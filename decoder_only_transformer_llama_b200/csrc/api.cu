@@ -483,12 +483,12 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B
             const NormIO n_in = {m->ssq, nb, eps, nullptr, nullptr, nullptr};
             LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.wqkv, &Lp.m_wqkv, B, m->nqkv, m->dim, ep, st, true,
                                &n_in));
-            LLB_TRY(launch_attention_decode(m, l, pos, B, st, true));
             Epi er = base_epi(m);
             er.mode = EPI_RESID_F32;
             er.out = m->x;
             er.ldo = m->dim;
             const NormIO n_to_ffn = {nullptr, 0, 0.f, m->ssq, m->y, Lp.ffn_norm};
+            LLB_TRY(launch_attention_decode(m, l, pos, B, st, true));
             LLB_TRY(run_linear(m, m->dtype, m->attn, &m->m_attn, Lp.wo, &Lp.m_wo, B, m->dim, m->nq, er, st, true,
                                &n_to_ffn));
             Epi es = base_epi(m);

@@ -27,9 +27,7 @@
 // requested before the previous kernel has finished; the activation tiles
 // and every global read of the epilogue wait for it (griddepcontrol.wait).
 // Every wait is bounded; no TMA multicast.
-#include "common.cuh"
-#include "epilogue.cuh"
-#include "model.h"
+#include "decode_tile.cuh"
 
 namespace llb {
 
@@ -37,136 +35,7 @@ namespace {
 constexpr int kThreads = 192;
 constexpr int kAccStride = 64;      // TMEM columns per accumulator buffer
 constexpr int kTmemCols = 128;      // two accumulator buffers
-constexpr int kABytes = 128 * 128;  // 128 weight rows x 64 bf16
-
-struct Seg {
-    int tile, ks, ke;
-};
-
-// Next segment (one tile's k-range) of a run of units; false past the end.
-__device__ __forceinline__ bool next_seg(int& u, int u1, int KT, Seg& s) {
-    if (u >= u1) return false;
-    s.tile = u / KT;
-    s.ks = u - s.tile * KT;
-    s.ke = min(KT, s.ks + (u1 - u));
-    u += s.ke - s.ks;
-    return true;
-}
 }  // namespace
-
-// Epilogue of one finished 128-row weight tile t: v[b] = acc[row r of the
-// tile, token column b] for the nb real token columns.  All 128 epilogue
-// threads of the CTA call it together (the residual + sum-of-squares mode
-// synchronises them on named barrier 2).
-template <int BN>
-__device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int lane, int q, int epi_tid, int nb,
-                                            int N, int T, const Epi& ep, const NormIO& nio, bool scale_in,
-                                            const float* rs, float* red) {
-    if (scale_in) {
-#pragma unroll
-        for (int b = 0; b < BN; ++b) v[b] *= (b < nb) ? rs[b] : 0.f;
-    }
-    const int n = t * 128 + r;
-    const bool row_ok = n < N;
-    if (ep.mode == EPI_SWIGLU) {
-        // rows are interleaved in blocks of 16: lanes 0-15 of a warp hold
-        // w1 rows, lanes 16-31 the matching w3 rows
-#pragma unroll
-        for (int b = 0; b < BN; ++b) {
-            const float up = __shfl_xor_sync(0xffffffffu, v[b], 16);
-            if (lane < 16 && row_ok && b < nb) {
-                const int h = (n >> 5) * 16 + (n & 15);
-                static_cast<bf16*>(ep.g)[static_cast<long long>(b) * ep.H + h] =
-                    __float2bfloat16_rn(silu_f(v[b]) * up);
-            }
-        }
-    } else if (ep.mode == EPI_QKV) {
-        const bool even = (lane & 1) == 0;
-        const bool is_q = n < ep.nq;
-        int cc = n - ep.nq;
-        bf16* cache = static_cast<bf16*>(ep.kc);
-        const bool is_k = !is_q && cc < ep.nkvc;
-        if (!is_q && !is_k) { cc -= ep.nkvc; cache = static_cast<bf16*>(ep.vc); }
-        const int d = is_q ? n % ep.hd : cc % ep.hd;
-        const int head = is_q ? 0 : cc / ep.hd;
-        // per group of 16 columns: all positions and RoPE factors first
-        // (independent loads), then the rotations and stores
-#pragma unroll
-        for (int b0 = 0; b0 < BN; b0 += 16) {
-            int posv[16];
-            float2 cs[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u) posv[u] = (b0 + u < nb) ? ep.tok_pos[b0 + u] : -1;
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const bool okp = row_ok && posv[u] >= 0 && posv[u] < ep.max_seq && (is_q || is_k);
-                cs[u] = okp ? ep.rope[static_cast<long long>(posv[u]) * (ep.hd / 2) + (d >> 1)]
-                            : make_float2(1.f, 0.f);
-            }
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int b = b0 + u;
-                const float partner = __shfl_xor_sync(0xffffffffu, v[b], 1);
-                const int pos = posv[u];
-                if (!row_ok || b >= nb || pos < 0 || pos >= ep.max_seq) continue;
-                const float re = even ? v[b] : partner, im = even ? partner : v[b];
-                const float rot = even ? re * cs[u].x - im * cs[u].y : re * cs[u].y + im * cs[u].x;
-                if (is_q) {
-                    static_cast<bf16*>(ep.q)[static_cast<long long>(b) * ep.nq + n] = __float2bfloat16_rn(rot);
-                } else {
-                    const int row = ep.tok_row ? ep.tok_row[b] : b;
-                    cache[static_cast<long long>(row) * ep.kv_row_stride +
-                          (static_cast<long long>(head) * ep.max_seq + pos) * ep.hd + d] =
-                        __float2bfloat16_rn(is_k ? rot : v[b]);
-                }
-            }
-        }
-    } else if (ep.mode == EPI_RESID_F32 && nio.ssq_out) {
-        // residual add, plus this tile's share of sum(x^2) for the next RMSNorm;
-        // the old x values of a 16-column group are loaded together
-        const float wn = row_ok ? nio.w_next[n] : 0.f;
-        float xo[16];
-#pragma unroll
-        for (int b = 0; b < BN; ++b) {
-            if ((b & 15) == 0) {
-#pragma unroll
-                for (int u = 0; u < 16; ++u)
-                    xo[u] = (row_ok && b + u < nb) ? ep.out[static_cast<long long>(b + u) * ep.ldo + n] : 0.f;
-            }
-            float sq = 0.f;
-            if (row_ok && b < nb) {
-                const float nv = xo[b & 15] + v[b];
-                ep.out[static_cast<long long>(b) * ep.ldo + n] = nv;
-                static_cast<bf16*>(nio.y_out)[static_cast<long long>(b) * ep.ldo + n] = __float2bfloat16_rn(nv * wn);
-                sq = nv * nv;
-            }
-            sq = warp_sum(sq);
-            if (lane == 0) red[q * 64 + b] = sq;
-        }
-        named_sync(2, 128);
-        if (epi_tid < nb)
-            nio.ssq_out[epi_tid * T + t] = ((red[epi_tid] + red[64 + epi_tid]) + red[128 + epi_tid]) +
-                                           red[192 + epi_tid];
-        named_sync(2, 128);
-    } else if (row_ok) {
-        if (ep.mode == EPI_RESID_F32) {
-#pragma unroll
-            for (int b0 = 0; b0 < BN; b0 += 16) {
-                float xo[16];
-#pragma unroll
-                for (int u = 0; u < 16; ++u)
-                    xo[u] = (b0 + u < nb) ? ep.out[static_cast<long long>(b0 + u) * ep.ldo + n] : 0.f;
-#pragma unroll
-                for (int u = 0; u < 16; ++u)
-                    if (b0 + u < nb) ep.out[static_cast<long long>(b0 + u) * ep.ldo + n] = xo[u] + v[b0 + u];
-            }
-        } else {
-#pragma unroll
-            for (int b = 0; b < BN; ++b)
-                if (b < nb) ep.out[static_cast<long long>(b) * ep.ldo + n] = v[b];
-        }
-    }
-}
 
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -281,77 +150,8 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
             rs[epi_tid] = rsqrtf(ss / static_cast<float>(K) + nio.eps);
         }
         named_sync(1, 128);
-        int u = u0;
-        Seg sg;
-        int j = 0;
-        const int nb = M < BN ? M : BN;
-        while (next_seg(u, u1, KT, sg)) {
-            const int acc = j & 1;
-            const bool ok_wait = mbar_wait(&tfull[acc], (j >> 1) & 1);
-            tc_fence_after();
-            float v[BN];
-#pragma unroll
-            for (int cc = 0; cc < BN / 16; ++cc)
-                tmem_ld_32x32b_x16(tmem + lane_base + acc * kAccStride + cc * 16, v + cc * 16);
-            tc_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&tempty[acc]);
-            ++j;
-            if (named_any(1, 128, !ok_wait || *reinterpret_cast<volatile int*>(&flag[0]) != 0)) {
-                if (epi_tid == 0) report_status(ep.status, LLAMA_ERR_DEVICE_TIMEOUT);
-                break;
-            }
-            const int t = sg.tile;
-            const int tb = t * KT;
-            const int cf = owner(tb, W, P), cl = owner(tb + KT - 1, W, P);
-            if (cl > cf) {
-                // split tile: publish this CTA's partial, the last arrival reduces
-                const int slot = (tb + sg.ks == u0) ? 0 : 1;   // the run's first segment, or its last
-                float* my = part + ((static_cast<long long>(c) * 2 + slot) * 128 + r) * BN;
-#pragma unroll
-                for (int b = 0; b < BN; b += 4)
-                    *reinterpret_cast<float4*>(my + b) = make_float4(v[b], v[b + 1], v[b + 2], v[b + 3]);
-                __threadfence();
-                named_sync(1, 128);
-                if (epi_tid == 0) flag[1] = atomicAdd(&counters[t], 1);
-                named_sync(1, 128);
-                const int arrived = flag[1];
-                if (arrived != cl - cf) continue;      // not the last contributor
-                __threadfence();
-#pragma unroll
-                for (int b = 0; b < BN; ++b) v[b] = 0.f;
-                // partials in CTA order, CB contributors per batch of independent loads
-                constexpr int CB = BN <= 16 ? 4 : (BN <= 32 ? 2 : 1);
-                for (int cb = cf; cb <= cl; cb += CB) {
-                    float4 f[CB][BN / 4];
-#pragma unroll
-                    for (int e = 0; e < CB; ++e) {
-                        const int cc = cb + e;
-                        if (cc <= cl) {
-                            const int sl = run_begin(cc, W, P) >= tb ? 0 : 1;   // slot 0: first segment, 1: last
-                            const float4* pp = reinterpret_cast<const float4*>(
-                                part + ((static_cast<long long>(cc) * 2 + sl) * 128 + r) * BN);
-#pragma unroll
-                            for (int qq = 0; qq < BN / 4; ++qq) f[e][qq] = pp[qq];
-                        }
-                    }
-#pragma unroll
-                    for (int e = 0; e < CB; ++e) {
-                        if (cb + e <= cl) {
-#pragma unroll
-                            for (int qq = 0; qq < BN / 4; ++qq) {
-                                v[4 * qq] += f[e][qq].x;
-                                v[4 * qq + 1] += f[e][qq].y;
-                                v[4 * qq + 2] += f[e][qq].z;
-                                v[4 * qq + 3] += f[e][qq].w;
-                            }
-                        }
-                    }
-                }
-                if (epi_tid == 0) counters[t] = 0;
-            }
-            finish_tile<BN>(v, t, r, lane, q, epi_tid, nb, N, T, ep, nio, scale_in, rs, red);
-        }
+        decode_epilogue_loop<BN>(tmem + lane_base, tfull, tempty, flag, part, counters, c, P, u0, u1, KT, N, M, ep,
+                                 nio, scale_in, rs, red, r, lane, q, epi_tid);
     }
 
     tc_fence_before();
