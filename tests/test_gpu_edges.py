@@ -1,0 +1,112 @@
+"""Edge cases of the CUDA path against the oracle: the last cache position,
+one-token prompts at full batch, and inputs that the kernels' own range checks
+turn into a device status code (a position past max_seq_len, a token id
+outside the vocabulary) while the other rows of the batch stay exact."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import llama_oracle as O
+from tests.helpers import build_model, oracle_args, rel_l2
+from workloads import ModelShape, TINY, make_tokens, make_weights, to_numpy_f64_weights, token_seed
+
+pytestmark = pytest.mark.gpu
+
+BF16_TOL = 2e-2
+SMALL = ModelShape(dim=256, n_layers=2, n_heads=2, n_kv_heads=1, vocab_size=512, max_seq_len=96,
+                   max_batch_size=4, dtype="bf16", hidden=768)
+
+
+@pytest.fixture(scope="module")
+def llb(cuda_device):
+    import decoder_only_transformer_llama_b200 as m
+    return m
+
+
+def _oracle_logits(shape, w64, seq):
+    args = oracle_args(shape)
+    return O.forward(args, w64, seq, 0, O.new_cache(args))
+
+
+@pytest.mark.parametrize("shape,tol", [(TINY, 1e-4), (SMALL, BF16_TOL)])
+def test_decode_at_the_last_cache_position(llb, shape, tol):
+    """Prefill max_seq_len - 1 tokens, then one decode step at position
+    max_seq_len - 1: the step fills the cache exactly and matches the oracle."""
+    S = shape.max_seq_len
+    w = make_weights(shape, 41)
+    m = build_model(shape, w)
+    B, T = 2, S - 1
+    toks = make_tokens(shape.vocab_size, (B, T), token_seed(7)).cuda()
+    logits = torch.empty(B, shape.vocab_size, device="cuda")
+    m.prefill(toks, logits=logits)
+    nxt_tok = make_tokens(shape.vocab_size, (B,), token_seed(8)).cuda()
+    pos = torch.full((B,), S - 1, dtype=torch.int32, device="cuda")
+    step = torch.empty(B, shape.vocab_size, device="cuda")
+    m.decode_step(nxt_tok, pos, logits=step)
+    torch.cuda.synchronize()
+    assert m.status() == 0
+    w64 = to_numpy_f64_weights(w)
+    for b in range(B):
+        seq = toks[b].cpu().tolist() + [int(nxt_tok[b])]
+        want = _oracle_logits(shape, w64, seq)[-1]
+        assert rel_l2(step[b].cpu().numpy(), want) <= tol, b
+    m.close()
+
+
+def test_one_token_prompts_at_full_batch(llb):
+    """max_batch_size rows whose prompts are 1, 2, 1 and 5 tokens long."""
+    w = make_weights(SMALL, 42)
+    m = build_model(SMALL, w)
+    B, T = SMALL.max_batch_size, 5
+    lens = [1, 2, 1, 5]
+    toks = make_tokens(SMALL.vocab_size, (B, T), token_seed(9)).cuda()
+    logits = torch.empty(B, SMALL.vocab_size, device="cuda")
+    m.prefill(toks, lens=lens, logits=logits)
+    torch.cuda.synchronize()
+    assert m.status() == 0
+    w64 = to_numpy_f64_weights(w)
+    for b in range(B):
+        want = _oracle_logits(SMALL, w64, toks[b, :lens[b]].cpu().tolist())[-1]
+        assert rel_l2(logits[b].cpu().numpy(), want) <= BF16_TOL, b
+    m.close()
+
+
+def test_position_past_the_cache_sets_capacity_status(llb):
+    """Row 1 asks for position max_seq_len: the kernels skip it and report
+    LLAMA_ERR_CAPACITY; rows 0 and 2 are computed as usual."""
+    S = SMALL.max_seq_len
+    w = make_weights(SMALL, 43)
+    m = build_model(SMALL, w)
+    B, T = 3, 10
+    toks = make_tokens(SMALL.vocab_size, (B, T), token_seed(10)).cuda()
+    logits = torch.empty(B, SMALL.vocab_size, device="cuda")
+    m.prefill(toks, logits=logits)
+    nxt_tok = make_tokens(SMALL.vocab_size, (B,), token_seed(11)).cuda()
+    pos = torch.tensor([T, S, T], dtype=torch.int32, device="cuda")
+    step = torch.empty(B, SMALL.vocab_size, device="cuda")
+    m.decode_step(nxt_tok, pos, logits=step)
+    torch.cuda.synchronize()
+    assert m.status() == llb.LLAMA_ERR_CAPACITY
+    w64 = to_numpy_f64_weights(w)
+    for b in (0, 2):
+        seq = toks[b].cpu().tolist() + [int(nxt_tok[b])]
+        want = _oracle_logits(SMALL, w64, seq)[-1]
+        assert rel_l2(step[b].cpu().numpy(), want) <= BF16_TOL, b
+    m.close()
+
+
+def test_token_outside_the_vocabulary_sets_token_range_status(llb):
+    """A prompt token id equal to vocab_size: its embedding row reads as zero
+    and the model reports LLAMA_ERR_TOKEN_RANGE; the other row is exact."""
+    w = make_weights(SMALL, 44)
+    m = build_model(SMALL, w)
+    B, T = 2, 6
+    toks = make_tokens(SMALL.vocab_size, (B, T), token_seed(12))
+    toks[1, 3] = SMALL.vocab_size
+    logits = torch.empty(B, SMALL.vocab_size, device="cuda")
+    m.prefill(toks.cuda(), logits=logits)
+    torch.cuda.synchronize()
+    assert m.status() == llb.LLAMA_ERR_TOKEN_RANGE
+    want = _oracle_logits(SMALL, to_numpy_f64_weights(w), toks[0].tolist())[-1]
+    assert rel_l2(logits[0].cpu().numpy(), want) <= BF16_TOL
+    m.close()
