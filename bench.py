@@ -98,6 +98,16 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- roofline bookkeeping
 
+def bench_config(world):
+    """The headline workload, as both arms print it (the reference arm times a
+    bounded sample of it, described in its cpu_baseline.sample)."""
+    return {"workload": "7b: Llama-2-7B shape, 32 layers, dim 4096, 32 heads (MHA), hidden 11008, "
+                        "vocab 32000, max_seq_len 4096; prefill 4x512 then 256 greedy decode steps",
+            "global_batch": WL["batch"] * world, "seq_len": WL["prompt_len"], "decode_steps": WL["decode_steps"],
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "inputs larger than L2: each decode step streams 13.5 GB of weights (L2 126 MB)"}
+
+
 def max_over_ranks(vals, world):
     """Element-wise maximum of the float64 tensor `vals` over all ranks, in
     place: a replicated job ends when its slowest rank does."""
@@ -335,11 +345,7 @@ def run_ours(a, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded random token ids, random-init bf16 weights, fp32 norm weights)",
-        "config": {"workload": "7b: Llama-2-7B shape, 32 layers, dim 4096, 32 heads (MHA), hidden 11008, "
-                               "vocab 32000, max_seq_len 4096; prefill 4x512 then 256 greedy decode steps",
-                   "global_batch": B * world, "seq_len": T, "decode_steps": steps_dec,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "inputs larger than L2: each decode step streams 13.5 GB of weights (L2 126 MB)"},
+        "config": bench_config(world),
         "prefill_tok_s": round(prefill_tps, 1),
         "decode_ms_per_token_step": round(decode_ms / (a.steps * steps_dec), 4),
         "decode_top_p_tok_s": round(top_p_tps * world, 2),
@@ -438,8 +444,7 @@ def run_reference(a, rank, world):
     return {"metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": round(1e3 / value, 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "7b: Llama-2-7B shape; oracle sample (see cpu_baseline.sample)",
-                       "global_batch": 1, "seq_len": 640, "parallelism": "host cores"},
+            "config": bench_config(world),
             "impl": "reference",
             "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": sample},
