@@ -130,9 +130,9 @@ __device__ __forceinline__ bool named_any(int id, int n, bool v) {
 // ---------------------------------------------------------------- stream-K runs
 // W work units split into P contiguous runs: run c is [run_begin(c), run_begin(c+1)).
 // The caller keeps W * P below 2^31.
-__device__ __forceinline__ int run_begin(int c, int W, int P) { return c * W / P; }
+__host__ __device__ __forceinline__ int run_begin(int c, int W, int P) { return c * W / P; }
 // Run (CTA) holding unit u.
-__device__ __forceinline__ int owner(int u, int W, int P) { return ((u + 1) * P - 1) / W; }
+__host__ __device__ __forceinline__ int owner(int u, int W, int P) { return ((u + 1) * P - 1) / W; }
 
 // ---------------------------------------------------------------- TMA (no multicast anywhere)
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int x, int y,

@@ -16,11 +16,11 @@ struct Seg {
 };
 
 // Next segment (one tile's k-range) of a run of units; false past the end.
-__device__ __forceinline__ bool next_seg(int& u, int u1, int KT, Seg& s) {
+__host__ __device__ __forceinline__ bool next_seg(int& u, int u1, int KT, Seg& s) {
     if (u >= u1) return false;
     s.tile = u / KT;
     s.ks = u - s.tile * KT;
-    s.ke = min(KT, s.ks + (u1 - u));
+    s.ke = KT < s.ks + (u1 - u) ? KT : s.ks + (u1 - u);
     u += s.ke - s.ks;
     return true;
 }

@@ -32,6 +32,7 @@
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "model.h"
+#include "work_split.cuh"
 
 #include <algorithm>
 #include <cudaTypedefs.h>
@@ -46,7 +47,6 @@ constexpr int kStagesTc = 4;
 constexpr int kA_BYTES = 128 * 128;          // 128 rows x 64 bf16
 constexpr int kB_BYTES = kBN * 128;
 constexpr int kStageBytes = kA_BYTES + kB_BYTES;
-constexpr int kGroupM = 16;                  // M-tiles per rasterisation group
 constexpr int kPartFloats = 128 * kBN;       // one fp32 partial tile
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
@@ -66,55 +66,6 @@ __device__ __forceinline__ void store32_bf16(bf16* dst, const float* v) {
         u.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
         d[q] = u;
     }
-}
-
-// Work list of one CTA: whole tiles c, c+P, ... below dp, then (c < psk) its
-// stream-K run over the last sk tiles.
-struct TcPlan {
-    int TM, TN, KT;
-    int dp, sk, psk;
-};
-struct Item {
-    int tile, ks, ke;
-};
-struct WorkIt {
-    int next_dp, u, u1;
-};
-
-__device__ __forceinline__ WorkIt work_begin(const TcPlan& p, int c, int P) {
-    WorkIt w;
-    w.next_dp = c;
-    const int W = p.sk * p.KT;
-    w.u = c < p.psk ? run_begin(c, W, p.psk) : 0;
-    w.u1 = c < p.psk ? run_begin(c + 1, W, p.psk) : 0;
-    return w;
-}
-
-__device__ __forceinline__ bool work_next(WorkIt& w, const TcPlan& p, int P, Item& it) {
-    if (w.next_dp < p.dp) {
-        it.tile = w.next_dp;
-        it.ks = 0;
-        it.ke = p.KT;
-        w.next_dp += P;
-        return true;
-    }
-    if (w.u >= w.u1) return false;
-    const int tl = w.u / p.KT;
-    it.tile = p.dp + tl;
-    it.ks = w.u - tl * p.KT;
-    it.ke = min(p.KT, it.ks + (w.u1 - w.u));
-    w.u += it.ke - it.ks;
-    return true;
-}
-
-// Tile t -> (M-tile, N-tile): groups of kGroupM M-tiles, N-major inside a group.
-__device__ __forceinline__ void tile_coords(int t, const TcPlan& p, int& tm, int& tn) {
-    const int per_group = kGroupM * p.TN;
-    const int g = t / per_group;
-    const int rem = t - g * per_group;
-    const int gm = min(kGroupM, p.TM - g * kGroupM);
-    tn = rem / gm;
-    tm = g * kGroupM + (rem - tn * gm);
 }
 
 // Epilogue of 32 consecutive output features n0..n0+31 of token row m.
@@ -395,31 +346,6 @@ int encode_kmajor_bf16(CUtensorMap* map, const void* base, int rows, int cols, i
         return LLAMA_ERR_CUDA;
     }
     return LLAMA_OK;
-}
-
-// Work split of one prefill projection over P persistent CTAs: whole tiles
-// round-robin for every full wave, and a stream-K run over a partial last
-// wave unless it is nearly full (>= 85 % of the CTAs) or there is no workspace
-// for split tiles.  A split tile is cut at most 4 ways (finishing it reads the
-// other pieces' 128 KB partials back).
-static void plan_tc(int T, int KT, int P, bool can_split, TcPlan* p, int* grid) {
-    p->dp = T;
-    p->sk = 0;
-    p->psk = 0;
-    *grid = T < P ? T : P;
-    if (!can_split || T % P == 0 || KT < 2) return;
-    const int full = T / P, R = T % P;
-    if (full >= 1 && R * 100 >= 85 * P) return;
-    p->dp = full * P;
-    p->sk = R;
-    long long psk = std::min<long long>(std::min<long long>(P, 4LL * R), static_cast<long long>(R) * KT);
-    if (static_cast<long long>(R) * KT * psk >= (1LL << 31)) {   // keep unit arithmetic in int
-        p->dp = T;
-        p->sk = 0;
-        return;
-    }
-    p->psk = static_cast<int>(psk);
-    *grid = full >= 1 ? P : p->psk;
 }
 
 static int g_sms_tc = 0;
