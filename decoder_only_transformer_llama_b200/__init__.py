@@ -38,7 +38,7 @@ EXPORTED = ("llama_model_bytes", "llama_model_create", "llama_set_weight", "llam
             "llama_prefill", "llama_decode_step", "llama_sample", "llama_model_status",
             "llama_model_destroy", "llama_last_error", "llama_launch_count",
             "llama_op_rmsnorm", "llama_op_linear", "llama_op_linear_workspace_bytes", "llama_op_linear_noalloc",
-            "llama_profile_start", "llama_profile_stop")
+            "llama_profile_start", "llama_profile_stop", "llama_token_logprobs")
 
 
 class LlamaError(RuntimeError):
@@ -88,6 +88,7 @@ _sig("llama_launch_count", ctypes.c_uint64, [])
 _sig("llama_op_rmsnorm", _i, [_vp, _vp, _i, _i, _f, _vp, _i, _vp])
 _sig("llama_op_linear", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp])
 _sig("llama_op_linear_workspace_bytes", _sz, [])
+_sig("llama_token_logprobs", _i, [_vp, _vp, _i, _i, _vp, _vp])
 _sig("llama_op_linear_noalloc", _i, [_vp, _vp, _i, _i, _i, _vp, _vp])
 _sig("llama_profile_start", _i, [_vp, _i])
 _sig("llama_profile_stop", _i, [_vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int64),
@@ -259,6 +260,13 @@ def sample(logits, temperature: float, top_p: float, uniforms, out, stream=None)
     B, V = logits.shape
     _check(_lib.llama_sample(logits.data_ptr(), B, V, float(temperature), float(top_p), _ptr(uniforms),
                              out.data_ptr(), _stream(stream)))
+    return out
+
+
+def token_logprobs(logits, tokens, out, stream=None):
+    """out[i] = log_softmax(logits[i])[tokens[i]] (fp32 logits [N, V], int32 tokens [N])."""
+    N, V = logits.shape
+    _check(_lib.llama_token_logprobs(logits.data_ptr(), tokens.data_ptr(), N, V, out.data_ptr(), _stream(stream)))
     return out
 
 

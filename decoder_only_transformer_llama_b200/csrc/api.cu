@@ -534,6 +534,13 @@ int llama_sample(const float* logits, int B, int V, float temperature, float top
     return launch_top_p(logits, B, V, temperature, top_p, uniforms, out, nullptr, nullptr, st);
 }
 
+int llama_token_logprobs(const float* logits, const int32_t* tokens, int N, int V, float* out, void* stream) {
+    if (!logits || !tokens || !out) { set_error("logits, tokens or out is NULL"); return LLAMA_ERR_INVALID_ARG; }
+    if (N < 0 || V <= 0) { set_error("N must be >= 0 and V positive"); return LLAMA_ERR_INVALID_ARG; }
+    if (N == 0) return LLAMA_OK;
+    return launch_logprobs(logits, tokens, N, V, out, static_cast<cudaStream_t>(stream));
+}
+
 int llama_model_status(llama_model* m, int* device_status) {
     if (!m || !device_status) { set_error("model or device_status is NULL"); return LLAMA_ERR_INVALID_ARG; }
     cudaError_t e = cudaStreamSynchronize(m->last_stream);

@@ -174,6 +174,7 @@ int launch_attention_decode(const Model* m, int layer, const int32_t* pos, int B
 
 int launch_argmax(const float* logits, int B, int V, int32_t* out, int32_t* tokens_adv,
                   int32_t* pos_adv, cudaStream_t st, bool pdl = false);
+int launch_logprobs(const float* logits, const int32_t* tokens, int N, int V, float* out, cudaStream_t st);
 int launch_top_p(const float* logits, int B, int V, float temperature, float top_p,
                  const float* uniforms, int32_t* out, int32_t* tokens_adv, int32_t* pos_adv,
                  cudaStream_t st, bool pdl = false);

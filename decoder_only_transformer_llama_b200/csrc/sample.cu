@@ -247,6 +247,44 @@ top_p_kernel(const float* __restrict__ logits, int V, float temperature, float t
     }
 }
 
+// ---------------------------------------------------------------- token log-probabilities
+// out[i] = log softmax(logits[i, :])[tok[i]] = l[tok] - (m + log sum_j exp(l_j - m)),
+// m = max_j l_j, the sum in fp64 (the log-probabilities that generate returns,
+// Admin Guide §8.5).  An id outside [0, V) gives NaN.
+__global__ void __launch_bounds__(kSampleThreads)
+logprob_kernel(const float* __restrict__ logits, const int32_t* __restrict__ tok, int V, float* __restrict__ out) {
+    __shared__ float s_max[kWarps];
+    __shared__ double s_sum[kWarps];
+    const int i = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float* row = logits + static_cast<long long>(i) * V;
+    float mx = -INFINITY;
+    for (int j = threadIdx.x; j < V; j += blockDim.x) mx = fmaxf(mx, row[j]);
+    mx = warp_max(mx);
+    if (lane == 0) s_max[warp] = mx;
+    __syncthreads();
+    mx = s_max[0];
+    for (int w = 1; w < kWarps; ++w) mx = fmaxf(mx, s_max[w]);
+    const double m = static_cast<double>(mx);
+    double sum = 0.0;
+    for (int j = threadIdx.x; j < V; j += blockDim.x) sum += exp(static_cast<double>(row[j]) - m);
+    sum = warp_sum_d(sum);
+    if (lane == 0) s_sum[warp] = sum;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double total = 0.0;
+        for (int w = 0; w < kWarps; ++w) total += s_sum[w];
+        const int t = tok[i];
+        out[i] = (t >= 0 && t < V) ? static_cast<float>(static_cast<double>(row[t]) - m - log(total)) : NAN;
+    }
+}
+
+int launch_logprobs(const float* logits, const int32_t* tokens, int N, int V, float* out, cudaStream_t st) {
+    logprob_kernel<<<N, kSampleThreads, 0, st>>>(logits, tokens, V, out);
+    LLB_CHECK_LAUNCH("logprob_kernel");
+    return LLAMA_OK;
+}
+
 int launch_argmax(const float* logits, int B, int V, int32_t* out, int32_t* tokens_adv, int32_t* pos_adv,
                   cudaStream_t st, bool pdl) {
     static bool attr = false;

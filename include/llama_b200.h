@@ -189,6 +189,18 @@ LLAMA_API int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* 
 LLAMA_API int llama_sample(const float* logits, int B, int V, float temperature, float top_p,
                  const float* uniforms, int32_t* out, void* stream);
 
+/* Log-probabilities of given tokens under their logits rows: the per-token
+ * logprobs that the generation loop returns (Admin Guide §8.5, generate with
+ * logprobs=True):
+ *   logits  device fp32 [N, V], row i the model's logits predicting token i;
+ *   tokens  device int32 [N];  out  device fp32 [N], written
+ *   out[i] = logits[i, t] - (m + log sum_j exp(logits[i, j] - m)),
+ *   t = tokens[i], m = max_j logits[i, j], the sum in fp64.
+ * A token outside [0, V) gives NaN.  N == 0 is a no-op.  Needs no model.
+ * LLAMA_ERR_INVALID_ARG for NULL pointers, N < 0 or V <= 0. */
+LLAMA_API int llama_token_logprobs(const float* logits, const int32_t* tokens, int N, int V, float* out,
+                                   void* stream);
+
 /* Copies the device status word to *device_status (synchronous on the model's
  * last stream) and clears it.  0 = no device-side error since the last read. */
 LLAMA_API int llama_model_status(llama_model* m, int* device_status);

@@ -364,3 +364,91 @@ def sample_margins(logits, temperature: float, top_p: float, u: float) -> float:
     if near.any():
         m -= float(ps[near].sum() / z)
     return m
+
+
+def token_logprobs(logits, tokens) -> np.ndarray:
+    """log softmax(logits[i])[tokens[i]] for each row i, in fp64: the
+    per-token log-probabilities generate returns (Admin Guide §8.5)."""
+    lg = _f64(logits)
+    m = lg.max(axis=-1, keepdims=True)
+    lse = m[:, 0] + np.log(np.exp(lg - m).sum(axis=-1))
+    return lg[np.arange(lg.shape[0]), np.asarray(tokens, dtype=np.int64)] - lse
+
+
+def generate(args: Args, w, prompts: Sequence[Sequence[int]], max_gen_len: Optional[int] = None,
+             temperature: float = 0.6, top_p: float = 0.9, uniforms=None, logprobs: bool = False,
+             echo: bool = False, eos_id: Optional[int] = None):
+    """The generation loop of the reference (Admin Guide §8.5; User Guide §1
+    and the per-call parameters of §3.4; source tour, "The decode loop in
+    generate"), one row at a time with its own KV cache.
+
+    All rows advance through the same positions: prompts are right-padded into
+    a (rows, total_len) table; the first forward runs the first min(prompt
+    lengths) tokens of every row; then, for each later position, one forward
+    over the slice not yet consumed, a greedy or nucleus choice for the next
+    position, which keeps the prompt's own token where the row's prompt still
+    covers that position; a row has finished once it produced EOS outside its
+    prompt, and the loop ends early when every row has.
+
+    Readings of what the pages leave open (the GPU driver takes the same):
+    total_len = min(max_seq_len, max_gen_len + longest prompt), max_gen_len
+    defaulting to max_seq_len - 1; the draw for position p of row b uses
+    uniforms[p][b]; the log-probability of the token at position p is the
+    log-softmax (of the raw logits, not temperature-scaled) at that token of
+    the logits that predict p, and 0 for position 0, which nothing predicts; a
+    row's result runs from position 0 (echo) or from the end of its prompt up
+    to prompt length + max_gen_len, cut before the first EOS at or after the
+    end of its prompt.  Returns (token lists, log-probability lists or None).
+    """
+    B = len(prompts)
+    S = args.max_seq_len
+    if max_gen_len is None:
+        max_gen_len = S - 1
+    lens = [len(p) for p in prompts]
+    assert B >= 1 and min(lens) >= 1 and max(lens) <= S
+    total = min(S, max_gen_len + max(lens))
+    pad = -1
+    tok = np.full((B, total), pad, dtype=np.int64)
+    for b, p in enumerate(prompts):
+        tok[b, :len(p)] = p
+    in_prompt = tok != pad
+    lp = np.zeros((B, total))
+    caches = [new_cache(args) for _ in range(B)]
+    done = np.zeros(B, dtype=bool)
+    start = min(lens)
+    if start == total:
+        # nothing to generate: only the prompts' log-probabilities
+        for b in range(B):
+            lg = forward(args, w, tok[b, :total].tolist(), 0, caches[b])
+            lp[b, 1:total] = token_logprobs(lg[:-1], tok[b, 1:total])
+    prev = 0
+    for cur in range(start, total):
+        for b in range(B):
+            lg = forward(args, w, tok[b, prev:cur].tolist(), prev, caches[b])   # rows predict prev+1 .. cur
+            if in_prompt[b, cur]:
+                nxt = int(tok[b, cur])
+            elif temperature > 0:
+                nxt = sample_top_p(lg[-1], temperature, top_p, float(uniforms[cur][b]))
+            else:
+                nxt = greedy(lg[-1])
+            tok[b, cur] = nxt
+            lp[b, prev + 1:cur + 1] = token_logprobs(lg, tok[b, prev + 1:cur + 1])
+            if eos_id is not None and not in_prompt[b, cur] and nxt == eos_id:
+                done[b] = True
+        prev = cur
+        if eos_id is not None and done.all():
+            break
+    out_tok, out_lp = [], []
+    for b in range(B):
+        first = 0 if echo else lens[b]
+        last = min(total, lens[b] + max_gen_len)
+        t = tok[b, first:last].tolist()
+        l = lp[b, first:last].tolist()
+        if eos_id is not None:
+            for i in range(max(0, lens[b] - first), len(t)):
+                if t[i] == eos_id:
+                    t, l = t[:i], l[:i]
+                    break
+        out_tok.append(t)
+        out_lp.append(l)
+    return out_tok, (out_lp if logprobs else None)
