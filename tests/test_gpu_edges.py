@@ -110,3 +110,30 @@ def test_token_outside_the_vocabulary_sets_token_range_status(llb):
     want = _oracle_logits(SMALL, to_numpy_f64_weights(w), toks[0].tolist())[-1]
     assert rel_l2(logits[0].cpu().numpy(), want) <= BF16_TOL
     m.close()
+
+
+def test_prefix_reuse_across_prefill_calls(llb):
+    """A prefix prefilled once, then two different continuations prefilled at
+    start_pos = len(prefix) one after the other (the second overwrites the
+    first's cache entries): every position's logits equal the oracle's on
+    prefix + continuation.  Continuation lengths put the projections on both
+    kernels (<= 64 token rows: the weight-streaming kernel; more: the
+    128 x 256-tile kernel) and the prefill attention on start_pos > 0."""
+    shape = SMALL.replace(max_seq_len=192)
+    w = make_weights(shape, 45)
+    m = build_model(shape, w)
+    w64 = to_numpy_f64_weights(w)
+    B, P = 2, 40
+    prefix = make_tokens(shape.vocab_size, (B, P), token_seed(13)).cuda()
+    m.prefill(prefix, logits=torch.empty(B, shape.vocab_size, device="cuda"))
+    for T, seed in ((30, 14), (100, 15)):
+        cont = make_tokens(shape.vocab_size, (B, T), token_seed(seed)).cuda()
+        lg = torch.empty(B, T, shape.vocab_size, device="cuda")
+        m.prefill(cont, start_pos=P, logits=lg, all_logits=True)
+        torch.cuda.synchronize()
+        assert m.status() == 0
+        for b in range(B):
+            seq = prefix[b].cpu().tolist() + cont[b].cpu().tolist()
+            want = _oracle_logits(shape, w64, seq)[P:]
+            assert rel_l2(lg[b].cpu().numpy(), want) <= BF16_TOL, (T, b)
+    m.close()
