@@ -575,7 +575,7 @@ def run_workload(a):
         pos.copy_(pos0)
         torch.cuda.synchronize()
         g = None
-        if s.dtype == "bf16":
+        if s.dtype != "f32":
             g = torch.cuda.CUDAGraph()
             sc = torch.cuda.Stream(device=dev)
             sc.wait_stream(stream)
@@ -591,7 +591,7 @@ def run_workload(a):
         assert model.status() == 0
         n_tok = sum(lens)
         mean_ctx = sum(lens) / B + steps / 2
-        byts = decode_step_bytes(s, B, int(mean_ctx)) if s.dtype == "bf16" else None
+        byts = decode_step_bytes(s, B, int(mean_ctx)) if s.dtype != "f32" else None
         out.append({"workload": name, "batch": B, "prompt_tokens": n_tok, "prefill_ms": round(pre_ms, 3),
                     "prefill_tok_s": round(n_tok / (pre_ms / 1e3), 1), "decode_steps": steps,
                     "decode_ms_per_step": round(dec_ms, 4), "decode_tok_s": round(B / (dec_ms / 1e3), 1),

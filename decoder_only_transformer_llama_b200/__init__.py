@@ -29,6 +29,7 @@ LLAMA_ERR_DEVICE_TIMEOUT = 4
 LLAMA_ERR_TOKEN_RANGE = 5
 LLAMA_F32 = 0
 LLAMA_BF16 = 1
+LLAMA_F16 = 2
 LLAMA_DECODE_ADVANCE = 1
 
 WEIGHT_IDS = {"tok_embeddings": 0, "norm": 1, "output": 2, "attention_norm": 3, "wq": 4, "wk": 5,
@@ -45,6 +46,9 @@ class LlamaError(RuntimeError):
     def __init__(self, code: int, msg: str):
         super().__init__(f"[{code}] {msg}")
         self.code = code
+
+
+_DTYPES = {"f32": LLAMA_F32, "bf16": LLAMA_BF16, "f16": LLAMA_F16}
 
 
 class ModelArgs(ctypes.Structure):
@@ -127,9 +131,11 @@ def _stream(stream) -> Optional[int]:
 def make_args(dim, n_layers, n_heads, n_kv_heads, vocab_size, multiple_of=256, ffn_dim_multiplier=None,
               norm_eps=1e-5, rope_theta=10000.0, max_seq_len=2048, max_batch_size=32, max_tokens=0,
               dtype="bf16") -> ModelArgs:
+    if dtype not in _DTYPES:
+        raise ValueError(f"dtype must be one of {sorted(_DTYPES)}")
     return ModelArgs(dim, n_layers, n_heads, n_kv_heads or 0, vocab_size, multiple_of,
                      float(ffn_dim_multiplier or 0.0), norm_eps, rope_theta, max_seq_len,
-                     max_batch_size, max_tokens, LLAMA_BF16 if dtype == "bf16" else LLAMA_F32)
+                     max_batch_size, max_tokens, _DTYPES[dtype])
 
 
 def args_from_shape(s) -> ModelArgs:
@@ -204,8 +210,8 @@ class Model:
         a = self.args
         nkv = a.n_kv_heads or a.n_heads
         hd = a.dim // a.n_heads
-        dt = torch.bfloat16 if a.dtype == LLAMA_BF16 else torch.float32
-        esz = 2 if a.dtype == LLAMA_BF16 else 4
+        dt = {LLAMA_BF16: torch.bfloat16, LLAMA_F16: torch.float16}.get(a.dtype, torch.float32)
+        esz = 4 if a.dtype == LLAMA_F32 else 2
         n = a.max_batch_size * a.max_seq_len * nkv * hd
         base = self.arena.data_ptr()
         out = []
@@ -272,7 +278,7 @@ def token_logprobs(logits, tokens, out, stream=None):
 
 def op_rmsnorm(x, w, eps: float, out, stream=None):
     M, dim = x.shape
-    dt = LLAMA_BF16 if out.dtype.__str__() == "torch.bfloat16" else LLAMA_F32
+    dt = {"torch.bfloat16": LLAMA_BF16, "torch.float16": LLAMA_F16}.get(out.dtype.__str__(), LLAMA_F32)
     _check(_lib.llama_op_rmsnorm(x.data_ptr(), w.data_ptr(), M, dim, float(eps), out.data_ptr(), dt,
                                  _stream(stream)))
     return out

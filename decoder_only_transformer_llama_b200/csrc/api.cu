@@ -63,7 +63,10 @@ static int make_layout(const llama_model_args* a, Layout* o) {
         set_error("non-positive size in llama_model_args");
         return LLAMA_ERR_INVALID_ARG;
     }
-    if (a->dtype != LLAMA_F32 && a->dtype != LLAMA_BF16) { set_error("dtype must be LLAMA_F32 or LLAMA_BF16"); return LLAMA_ERR_INVALID_ARG; }
+    if (a->dtype != LLAMA_F32 && a->dtype != LLAMA_BF16 && a->dtype != LLAMA_F16) {
+        set_error("dtype must be LLAMA_F32, LLAMA_BF16 or LLAMA_F16");
+        return LLAMA_ERR_INVALID_ARG;
+    }
     if (!(a->norm_eps >= 0.f) || !(a->rope_theta > 0.f)) { set_error("norm_eps must be >= 0 and rope_theta > 0"); return LLAMA_ERR_INVALID_ARG; }
     const int nkv = a->n_kv_heads ? a->n_kv_heads : a->n_heads;
     if (a->n_heads % nkv) { set_error("n_heads %% n_kv_heads != 0"); return LLAMA_ERR_INVALID_ARG; }
@@ -81,14 +84,14 @@ static int make_layout(const llama_model_args* a, Layout* o) {
                                           static_cast<long long>(a->dim) + 2LL * nkv * (a->dim / a->n_heads) + a->dim);
         if ((widest + 127) / 128 > kMaxTiles) { set_error("a projection is wider than %d x 128 rows", kMaxTiles); return LLAMA_ERR_INVALID_ARG; }
     }
-    if (a->dtype == LLAMA_BF16 && (a->dim < 256 || a->vocab_size < 256 || a->dim % 128)) {
-        set_error("bf16 models need dim >= 256 (a multiple of 128) and vocab_size >= 256");
+    if (a->dtype != LLAMA_F32 && (a->dim < 256 || a->vocab_size < 256 || a->dim % 128)) {
+        set_error("16-bit models need dim >= 256 (a multiple of 128) and vocab_size >= 256");
         return LLAMA_ERR_INVALID_ARG;
     }
     Layout& l = *o;
     l.dim = a->dim; l.L = a->n_layers; l.nh = a->n_heads; l.nkv = nkv; l.hd = hd; l.n_rep = n_rep; l.H = H;
     l.V = a->vocab_size; l.S = a->max_seq_len; l.Bmax = a->max_batch_size; l.dtype = a->dtype;
-    l.esz = a->dtype == LLAMA_BF16 ? 2 : 4;
+    l.esz = a->dtype == LLAMA_F32 ? 4 : 2;
     const long long mt = a->max_tokens ? a->max_tokens : 1LL * a->max_batch_size * a->max_seq_len;
     if (mt > (1LL << 30)) { set_error("max_tokens too large"); return LLAMA_ERR_INVALID_ARG; }
     l.Mmax = static_cast<int>(mt > l.Bmax ? mt : l.Bmax);
@@ -134,16 +137,16 @@ static int make_layout(const llama_model_args* a, Layout* o) {
     l.off_attn_cnt = off; off = align256(off + static_cast<size_t>(l.Bmax) * nkv * 4);
     l.off_status = off; off = align256(off + 16);
     l.off_rope = off; off = align256(off + static_cast<size_t>(l.S) * (hd / 2) * 8);
-    l.off_gemm_part = off; off = align256(off + (a->dtype == LLAMA_BF16 ? kGemmPartBytes : 0));
+    l.off_gemm_part = off; off = align256(off + (a->dtype != LLAMA_F32 ? kGemmPartBytes : 0));
     l.off_gemm_cnt = off; off = align256(off + kMaxTiles * sizeof(int));
     l.off_ssq = off; off = align256(off + static_cast<size_t>(l.Bmax) * (l.dim / 128 + 1) * 4);
     l.ws_end = off;
     return LLAMA_OK;
 }
 
-static int make_maps(TmaMaps* t, const void* base, int rows, int cols, int b_box) {
-    LLB_TRY(encode_kmajor_bf16(&t->a128, base, rows, cols, 128));
-    LLB_TRY(encode_kmajor_bf16(&t->b, base, rows, cols, b_box));
+static int make_maps(TmaMaps* t, const void* base, int rows, int cols, int b_box, int dtype) {
+    LLB_TRY(encode_kmajor_16(&t->a128, base, rows, cols, 128, dtype));
+    LLB_TRY(encode_kmajor_16(&t->b, base, rows, cols, b_box, dtype));
     return LLAMA_OK;
 }
 
@@ -166,7 +169,7 @@ int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, co
     if (dtype == LLAMA_F32)
         rc = linear_f32(static_cast<const float*>(A), static_cast<const float*>(W), M, N, K, ep, st);
     else
-        rc = linear_bf16(mapA, mapW, M, N, K, ep, m->gemm_part, kGemmPartBytes, m->gemm_cnt, st, pdl && !timed, nio);
+        rc = linear16(mapA, mapW, M, N, K, dtype, ep, m->gemm_part, kGemmPartBytes, m->gemm_cnt, st, pdl && !timed, nio);
     if (timed && rc == LLAMA_OK) {
         cudaError_t e = cudaEventRecord(pr->ev[2 * pr->n + 1], st);
         if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord(profile)");
@@ -318,19 +321,19 @@ int llama_model_create(const llama_model_args* args, void* dev_arena, size_t are
     m->last_stream = static_cast<cudaStream_t>(stream);
 
     int rc = LLAMA_OK;
-    if (l.dtype == LLAMA_BF16) {
+    if (l.dtype != LLAMA_F32) {
         for (int i = 0; i < l.L && rc == LLAMA_OK; ++i) {
             LayerPtrs& p = m->layers[i];
-            if (rc == LLAMA_OK) rc = make_maps(&p.m_wqkv, p.wqkv, l.nqkv, l.dim, 256);
-            if (rc == LLAMA_OK) rc = make_maps(&p.m_wo, p.wo, l.dim, l.nq, 256);
-            if (rc == LLAMA_OK) rc = make_maps(&p.m_w13, p.w13, 2 * l.H, l.dim, 256);
-            if (rc == LLAMA_OK) rc = make_maps(&p.m_w2, p.w2, l.dim, l.H, 256);
+            if (rc == LLAMA_OK) rc = make_maps(&p.m_wqkv, p.wqkv, l.nqkv, l.dim, 256, l.dtype);
+            if (rc == LLAMA_OK) rc = make_maps(&p.m_wo, p.wo, l.dim, l.nq, 256, l.dtype);
+            if (rc == LLAMA_OK) rc = make_maps(&p.m_w13, p.w13, 2 * l.H, l.dim, 256, l.dtype);
+            if (rc == LLAMA_OK) rc = make_maps(&p.m_w2, p.w2, l.dim, l.H, 256, l.dtype);
         }
-        if (rc == LLAMA_OK) rc = make_maps(&m->m_output, m->output, l.V, l.dim, 256);
-        if (rc == LLAMA_OK) rc = make_maps(&m->m_y, m->y, l.Mrows, l.dim, 16);
-        if (rc == LLAMA_OK) rc = make_maps(&m->m_attn, m->attn, l.Mrows, l.nq, 16);
-        if (rc == LLAMA_OK) rc = make_maps(&m->m_g, m->g, l.Mrows, l.H, 16);
-        if (rc == LLAMA_OK) rc = make_maps(&m->m_ylast, m->ylast, l.Brows, l.dim, 16);
+        if (rc == LLAMA_OK) rc = make_maps(&m->m_output, m->output, l.V, l.dim, 256, l.dtype);
+        if (rc == LLAMA_OK) rc = make_maps(&m->m_y, m->y, l.Mrows, l.dim, 16, l.dtype);
+        if (rc == LLAMA_OK) rc = make_maps(&m->m_attn, m->attn, l.Mrows, l.nq, 16, l.dtype);
+        if (rc == LLAMA_OK) rc = make_maps(&m->m_g, m->g, l.Mrows, l.H, 16, l.dtype);
+        if (rc == LLAMA_OK) rc = make_maps(&m->m_ylast, m->ylast, l.Brows, l.dim, 16, l.dtype);
     }
     cudaStream_t st = m->last_stream;
     if (rc == LLAMA_OK) {
@@ -461,7 +464,7 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B
     eo.mode = EPI_STORE_F32;
     eo.out = lg;
     eo.ldo = m->V;
-    if (m->dtype == LLAMA_BF16) {
+    if (m->dtype != LLAMA_F32) {
         // The decode chain: five kernels per layer.  Every kernel may launch
         // before its predecessor ends (programmatic dependent launch) and waits
         // for it before reading its outputs.  RMSNorm runs inside the
@@ -513,7 +516,7 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B
         LLB_TRY(run_linear(m, m->dtype, m->ylast, &m->m_ylast, m->output, &m->m_output, B, m->V, m->dim, eo, st));
     }
     if (!sampling) return LLAMA_OK;
-    const bool pdl = m->dtype == LLAMA_BF16;
+    const bool pdl = m->dtype != LLAMA_F32;
     const bool adv = (flags & LLAMA_DECODE_ADVANCE) != 0;
     int32_t* tok_adv = adv ? const_cast<int32_t*>(tokens) : nullptr;
     int32_t* pos_adv = adv ? pos : nullptr;
@@ -599,7 +602,7 @@ int llama_profile_stop(llama_model* m, float* ms, int64_t* bytes, int64_t* flops
 int llama_op_rmsnorm(const float* x, const float* w, int M, int dim, float eps, void* out, int out_dtype,
                      void* stream) {
     if (!x || !w || !out || M < 0 || dim <= 0 || dim % 4) { set_error("bad rmsnorm arguments"); return LLAMA_ERR_INVALID_ARG; }
-    if (out_dtype != LLAMA_F32 && out_dtype != LLAMA_BF16) { set_error("bad out_dtype"); return LLAMA_ERR_INVALID_ARG; }
+    if (out_dtype != LLAMA_F32 && out_dtype != LLAMA_BF16 && out_dtype != LLAMA_F16) { set_error("bad out_dtype"); return LLAMA_ERR_INVALID_ARG; }
     return launch_rmsnorm(x, nullptr, w, M, dim, eps, out, out_dtype, static_cast<cudaStream_t>(stream));
 }
 
@@ -627,13 +630,13 @@ int llama_op_linear(const void* A, const void* W, int M, int N, int K, int dtype
     }
     if (M == 0) return LLAMA_OK;
     TmaMaps ma, mw;
-    LLB_TRY(encode_kmajor_bf16(&ma.a128, A, M, K, 128));
-    LLB_TRY(encode_kmajor_bf16(&ma.b, A, M, K, 16));
-    LLB_TRY(encode_kmajor_bf16(&mw.a128, W, N, K, 128));
-    LLB_TRY(encode_kmajor_bf16(&mw.b, W, N, K, 256));
+    LLB_TRY(encode_kmajor_16(&ma.a128, A, M, K, 128));
+    LLB_TRY(encode_kmajor_16(&ma.b, A, M, K, 16));
+    LLB_TRY(encode_kmajor_16(&mw.a128, W, N, K, 128));
+    LLB_TRY(encode_kmajor_16(&mw.b, W, N, K, 256));
     float* part = static_cast<float*>(workspace);
     int* cnt = workspace ? reinterpret_cast<int*>(static_cast<char*>(workspace) + kGemmPartBytes) : nullptr;
-    return linear_bf16(&ma, &mw, M, N, K, ep, part, part ? kGemmPartBytes : 0, cnt, st);
+    return linear16(&ma, &mw, M, N, K, LLAMA_BF16, ep, part, part ? kGemmPartBytes : 0, cnt, st);
 }
 
 }  // extern "C"

@@ -9,7 +9,7 @@
 //
 // Prefill of fp32 models: one CTA per (64-query tile, head, row), online
 // softmax over 64-key tiles staged in shared memory (fp32 CUDA-core
-// arithmetic).  bf16 models use the tensor-core kernel of attention_prefill_tc.cu.
+// arithmetic).  16-bit models use the tensor-core kernel of attention_prefill_tc.cu.
 #include <algorithm>
 
 #include "common.cuh"
@@ -41,6 +41,20 @@ template <> struct Vec<bf16, 4> {
         const uint2 u = *reinterpret_cast<const uint2*>(p);
         const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
         const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+        o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
+    }
+};
+template <> struct Vec<f16, 1> { static __device__ __forceinline__ void load(const f16* p, float* o) { o[0] = __half2float(p[0]); } };
+template <> struct Vec<f16, 2> {
+    static __device__ __forceinline__ void load(const f16* p, float* o) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(p)); o[0] = f.x; o[1] = f.y;
+    }
+};
+template <> struct Vec<f16, 4> {
+    static __device__ __forceinline__ void load(const f16* p, float* o) {
+        const uint2 u = *reinterpret_cast<const uint2*>(p);
+        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
         o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
     }
 };
@@ -467,6 +481,7 @@ static int decode_hd(const Model* m, int layer, const int32_t* pos, int B, cudaS
 
 int launch_attention_decode(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl) {
     if (m->dtype == LLAMA_BF16) return decode_hd<bf16>(m, layer, pos, B, st, pdl);
+    if (m->dtype == LLAMA_F16) return decode_hd<f16>(m, layer, pos, B, st, pdl);
     return decode_hd<float>(m, layer, pos, B, st, pdl);
 }
 
@@ -597,8 +612,8 @@ static int prefill_hd(const Model* m, int layer, const RowTable& rt, cudaStream_
 }
 
 int launch_attention_prefill(const Model* m, int layer, const RowTable& rt, cudaStream_t st) {
-    // bf16 models run the tensor-core kernel; fp32 models the CUDA-core one (no TF32)
-    if (m->dtype == LLAMA_BF16) return launch_attention_prefill_tc(m, layer, rt, st);
+    // 16-bit models run the tensor-core kernel; fp32 models the CUDA-core one (no TF32)
+    if (m->dtype != LLAMA_F32) return launch_attention_prefill_tc(m, layer, rt, st);
     return prefill_hd<float>(m, layer, rt, st);
 }
 

@@ -1,4 +1,4 @@
-// Causal GQA prefill attention for bf16 models on the tensor cores
+// Causal GQA prefill attention for 16-bit (bf16 or fp16) models on the tensor cores
 // (Admin Guide §8.4, Attention steps 5-7 and the mask NOTE; repeat_kv from
 // the source tour): o_h = softmax(q_h K_g^T / sqrt(hd)) V_g over keys
 // 0 .. position of the query, g = h / n_rep.
@@ -6,10 +6,12 @@
 // One CTA = 64 queries of one (row, head); 4 warps x 16 queries.  Key/value
 // tiles of 64 positions stream through a double-buffered, XOR-swizzled
 // shared-memory ring (cp.async, 16-byte chunks).  S = Q K^T and O += P V are
-// m16n8k16 bf16 MMAs with fp32 accumulation; the online softmax runs on the
+// m16n8k16 16-bit MMAs with fp32 accumulation; the online softmax runs on the
 // S accumulator registers, which are re-packed as the A operand of P V
 // without leaving registers.  The causal mask is a key-range bound plus a
 // per-element test on the diagonal tile.
+#include <type_traits>
+
 #include "common.cuh"
 #include "model.h"
 
@@ -35,32 +37,38 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
 }
-__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-    __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<uint32_t*>(&p);
+// D (+)= A B, m16n8k16, 16-bit E operands (bf16 or fp16), fp32 accumulate.
+template <typename E>
+__device__ __forceinline__ void mma16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                      uint32_t b0, uint32_t b1) {
+    if constexpr (std::is_same<E, bf16>::value) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    } else {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    }
 }
 
 // byte offset of 16-byte chunk `c` of row `r` in a tile whose rows hold HD
-// bf16 (HD/8 chunks); chunks are XOR-swizzled by the row to spread banks.
+// 16-bit values (HD/8 chunks); chunks are XOR-swizzled by the row to spread banks.
 template <int HD>
 __device__ __forceinline__ uint32_t swz(int r, int c) {
     return static_cast<uint32_t>(r * (HD * 2) + ((c ^ (r & 7)) << 4));
 }
 }  // namespace
 
-template <int HD>
+template <int HD, typename E>
 __global__ void __launch_bounds__(128)
-attn_prefill_tc_kernel(RowTable rt, const bf16* __restrict__ q, const bf16* __restrict__ kc,
-                       const bf16* __restrict__ vc, int nq, int n_rep, int S, long long row_stride,
-                       bf16* __restrict__ out) {
+attn_prefill_tc_kernel(RowTable rt, const E* __restrict__ q, const E* __restrict__ kc,
+                       const E* __restrict__ vc, int nq, int n_rep, int S, long long row_stride,
+                       E* __restrict__ out) {
     constexpr int CH = HD / 8;                 // 16-byte chunks per row
     constexpr int TILE_BYTES = FK * HD * 2;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -78,8 +86,8 @@ attn_prefill_tc_kernel(RowTable rt, const bf16* __restrict__ q, const bf16* __re
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int kend = rt.start_pos + t0 + nqt;            // keys [0, kend) are needed
     const int ntiles = (kend + FK - 1) / FK;
-    const bf16* kb = kc + static_cast<long long>(b) * row_stride + static_cast<long long>(g) * S * HD;
-    const bf16* vb = vc + static_cast<long long>(b) * row_stride + static_cast<long long>(g) * S * HD;
+    const E* kb = kc + static_cast<long long>(b) * row_stride + static_cast<long long>(g) * S * HD;
+    const E* vb = vc + static_cast<long long>(b) * row_stride + static_cast<long long>(g) * S * HD;
 
     const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
     // Q tile (rows beyond the row's length are zero)
@@ -143,8 +151,8 @@ attn_prefill_tc_kernel(RowTable rt, const bf16* __restrict__ q, const bf16* __re
                 const int c = ks * 2 + ((lane >> 3) & 1);
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4(kbase + swz<HD>(r, c), b0, b1, b2, b3);
-                mma_bf16(s[2 * jp], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
-                mma_bf16(s[2 * jp + 1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b2, b3);
+                mma16<E>(s[2 * jp], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
+                mma16<E>(s[2 * jp + 1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b2, b3);
             }
         }
         // ---- mask + online softmax (rows gq and gq+8 of this warp's 16)
@@ -194,10 +202,10 @@ attn_prefill_tc_kernel(RowTable rt, const bf16* __restrict__ q, const bf16* __re
         const uint32_t vbase = sVa + buf * TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < FK / 16; ++kk) {
-            const uint32_t a0 = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
-            const uint32_t a1 = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
-            const uint32_t a2 = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-            const uint32_t a3 = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+            const uint32_t a0 = pack2<E>(s[2 * kk][0], s[2 * kk][1]);
+            const uint32_t a1 = pack2<E>(s[2 * kk][2], s[2 * kk][3]);
+            const uint32_t a2 = pack2<E>(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+            const uint32_t a3 = pack2<E>(s[2 * kk + 1][2], s[2 * kk + 1][3]);
 #pragma unroll
             for (int jd = 0; jd < HD / 16; ++jd) {
                 // matrices (transposed): (keys lo, d 16jd+0..7), (keys hi, d lo), (keys lo, d +8..15), (keys hi, d hi)
@@ -205,8 +213,8 @@ attn_prefill_tc_kernel(RowTable rt, const bf16* __restrict__ q, const bf16* __re
                 const int c = jd * 2 + (lane >> 4);
                 uint32_t b0, b1, b2, b3;
                 ldsm_x4_t(vbase + swz<HD>(r, c), b0, b1, b2, b3);
-                mma_bf16(o[2 * jd], a0, a1, a2, a3, b0, b1);
-                mma_bf16(o[2 * jd + 1], a0, a1, a2, a3, b2, b3);
+                mma16<E>(o[2 * jd], a0, a1, a2, a3, b0, b1);
+                mma16<E>(o[2 * jd + 1], a0, a1, a2, a3, b2, b3);
             }
         }
         __syncthreads();   // buffer `buf` is refilled two tiles later
@@ -218,16 +226,16 @@ attn_prefill_tc_kernel(RowTable rt, const bf16* __restrict__ q, const bf16* __re
     for (int j = 0; j < HD / 8; ++j) {
         const int d = j * 8 + 2 * tq;
         if (qrow0 < nqt)
-            *reinterpret_cast<uint32_t*>(out + (tok0 + qrow0) * nq + h * HD + d) = pack_bf16(o[j][0] * inv0, o[j][1] * inv0);
+            *reinterpret_cast<uint32_t*>(out + (tok0 + qrow0) * nq + h * HD + d) = pack2<E>(o[j][0] * inv0, o[j][1] * inv0);
         if (qrow1 < nqt)
-            *reinterpret_cast<uint32_t*>(out + (tok0 + qrow1) * nq + h * HD + d) = pack_bf16(o[j][2] * inv1, o[j][3] * inv1);
+            *reinterpret_cast<uint32_t*>(out + (tok0 + qrow1) * nq + h * HD + d) = pack2<E>(o[j][2] * inv1, o[j][3] * inv1);
     }
 }
 
-template <int HD>
+template <int HD, typename E>
 static int prefill_tc_go(const Model* m, int layer, const RowTable& rt, cudaStream_t st) {
     const int smem = (FQ * HD + 4 * FK * HD) * 2;
-    auto kern = attn_prefill_tc_kernel<HD>;
+    auto kern = attn_prefill_tc_kernel<HD, E>;
     static bool attr = false;
     if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -237,19 +245,20 @@ static int prefill_tc_go(const Model* m, int layer, const RowTable& rt, cudaStre
     int maxlen = 0;
     for (int b = 0; b < rt.B; ++b) maxlen = max(maxlen, rt.cu[b + 1] - rt.cu[b]);
     dim3 grid((maxlen + FQ - 1) / FQ, m->nh, rt.B);
-    const bf16* kc = static_cast<const bf16*>(m->kc) + layer * m->kv_layer_elems;
-    const bf16* vc = static_cast<const bf16*>(m->vc) + layer * m->kv_layer_elems;
-    kern<<<grid, 128, smem, st>>>(rt, static_cast<const bf16*>(m->q), kc, vc, m->nq, m->n_rep, m->S,
-                                  m->kv_row_elems, static_cast<bf16*>(m->attn));
+    const E* kc = static_cast<const E*>(m->kc) + layer * m->kv_layer_elems;
+    const E* vc = static_cast<const E*>(m->vc) + layer * m->kv_layer_elems;
+    kern<<<grid, 128, smem, st>>>(rt, static_cast<const E*>(m->q), kc, vc, m->nq, m->n_rep, m->S,
+                                  m->kv_row_elems, static_cast<E*>(m->attn));
     LLB_CHECK_LAUNCH("attn_prefill_tc_kernel");
     return LLAMA_OK;
 }
 
 int launch_attention_prefill_tc(const Model* m, int layer, const RowTable& rt, cudaStream_t st) {
+    const bool f16m = m->dtype == LLAMA_F16;
     switch (m->hd) {
-        case 32: return prefill_tc_go<32>(m, layer, rt, st);
-        case 64: return prefill_tc_go<64>(m, layer, rt, st);
-        case 128: return prefill_tc_go<128>(m, layer, rt, st);
+        case 32: return f16m ? prefill_tc_go<32, f16>(m, layer, rt, st) : prefill_tc_go<32, bf16>(m, layer, rt, st);
+        case 64: return f16m ? prefill_tc_go<64, f16>(m, layer, rt, st) : prefill_tc_go<64, bf16>(m, layer, rt, st);
+        case 128: return f16m ? prefill_tc_go<128, f16>(m, layer, rt, st) : prefill_tc_go<128, bf16>(m, layer, rt, st);
     }
     set_error("head_dim %d unsupported", m->hd);
     return LLAMA_ERR_INVALID_ARG;

@@ -1,9 +1,10 @@
-// Shared device helpers: bf16 conversion, warp reductions, the device status
+// Shared device helpers: 16-bit conversions, warp reductions, the device status
 // word, and thin inline-PTX wrappers for mbarrier, TMA and tcgen05 (sm_100a).
 #pragma once
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda.h>
 #include <stdint.h>
 
@@ -12,6 +13,7 @@
 namespace llb {
 
 typedef __nv_bfloat16 bf16;
+typedef __half f16;
 
 // ---------------------------------------------------------------- host side
 void set_error(const char* fmt, ...);
@@ -43,10 +45,29 @@ __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.lau
 template <typename T> __device__ __forceinline__ float to_f32(T v);
 template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f32<bf16>(bf16 v) { return __bfloat162float(v); }
+template <> __device__ __forceinline__ float to_f32<f16>(f16 v) { return __half2float(v); }
 
 template <typename T> __device__ __forceinline__ T from_f32(float v);
 template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __float2bfloat16_rn(v); }
+template <> __device__ __forceinline__ f16 from_f32<f16>(float v) { return __float2half_rn(v); }
+
+// Two floats rounded to a 16-bit type and packed low-first into 32 bits.
+template <typename T> __device__ __forceinline__ uint32_t pack2(float a, float b);
+template <> __device__ __forceinline__ uint32_t pack2<bf16>(float a, float b) {
+    __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&p);
+}
+template <> __device__ __forceinline__ uint32_t pack2<f16>(float a, float b) {
+    __half2 p = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&p);
+}
+// Four consecutive 16-bit values (8 bytes, 8-byte aligned) as floats.
+template <typename T> __device__ __forceinline__ void load4_16(const T* p, float* f) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const T* h = reinterpret_cast<const T*>(&u);
+    f[0] = to_f32<T>(h[0]); f[1] = to_f32<T>(h[1]); f[2] = to_f32<T>(h[2]); f[3] = to_f32<T>(h[3]);
+}
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -178,8 +199,9 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (bf16 in, fp32 accumulate).
-__device__ __forceinline__ void tc_mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (bf16 or fp16 in, as the
+// instruction descriptor says; fp32 accumulate).
+__device__ __forceinline__ void tc_mma_16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
                                             uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -224,7 +246,7 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, float* v) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Shared-memory matrix descriptor for a K-major bf16 tile stored as TMA
+// Shared-memory matrix descriptor for a K-major 16-bit tile stored as TMA
 // writes it with 128-byte swizzling: rows of 64 elements (128 B), groups of 8
 // rows 1024 B apart.  The tile base must be 1024-byte aligned.
 __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr) {
@@ -244,6 +266,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (1u << 10)                             // B format bf16
          | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
+}
+
+// Instruction descriptor, kind::f16: A and B both of the 16-bit type T (fp16:
+// format 0, bf16: format 1), fp32 D, both K-major.
+template <typename T> __host__ __device__ constexpr uint32_t idesc_16_f32(int M, int N);
+template <> __host__ __device__ constexpr uint32_t idesc_16_f32<bf16>(int M, int N) { return idesc_bf16_f32(M, N); }
+template <> __host__ __device__ constexpr uint32_t idesc_16_f32<f16>(int M, int N) {
+    return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 #ifdef __CUDACC__

@@ -9,7 +9,7 @@
 
 namespace llb {
 
-constexpr int kABytes = 128 * 128;  // 128 weight rows x 64 bf16: one A-operand ring stage
+constexpr int kABytes = 128 * 128;  // 128 weight rows x 64 16-bit values: one A-operand ring stage
 
 struct Seg {
     int tile, ks, ke;
@@ -29,9 +29,9 @@ __host__ __device__ __forceinline__ bool next_seg(int& u, int u1, int KT, Seg& s
 // tile, token column b] for the nb real token columns.  All 128 epilogue
 // threads of the CTA call it together (the residual + sum-of-squares mode
 // synchronises them on named barrier 2).
-template <int BN>
+template <int BN, typename T>
 __device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int lane, int q, int epi_tid, int nb,
-                                            int N, int T, const Epi& ep, const NormIO& nio, bool scale_in,
+                                            int N, int n_tiles, const Epi& ep, const NormIO& nio, bool scale_in,
                                             const float* rs, float* red) {
     if (scale_in) {
 #pragma unroll
@@ -47,17 +47,17 @@ __device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int la
             const float up = __shfl_xor_sync(0xffffffffu, v[b], 16);
             if (lane < 16 && row_ok && b < nb) {
                 const int h = (n >> 5) * 16 + (n & 15);
-                static_cast<bf16*>(ep.g)[static_cast<long long>(b) * ep.H + h] =
-                    __float2bfloat16_rn(silu_f(v[b]) * up);
+                static_cast<T*>(ep.g)[static_cast<long long>(b) * ep.H + h] =
+                    from_f32<T>(silu_f(v[b]) * up);
             }
         }
     } else if (ep.mode == EPI_QKV) {
         const bool even = (lane & 1) == 0;
         const bool is_q = n < ep.nq;
         int cc = n - ep.nq;
-        bf16* cache = static_cast<bf16*>(ep.kc);
+        T* cache = static_cast<T*>(ep.kc);
         const bool is_k = !is_q && cc < ep.nkvc;
-        if (!is_q && !is_k) { cc -= ep.nkvc; cache = static_cast<bf16*>(ep.vc); }
+        if (!is_q && !is_k) { cc -= ep.nkvc; cache = static_cast<T*>(ep.vc); }
         const int d = is_q ? n % ep.hd : cc % ep.hd;
         const int head = is_q ? 0 : cc / ep.hd;
         // per group of 16 columns: all positions and RoPE factors first
@@ -83,12 +83,12 @@ __device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int la
                 const float re = even ? v[b] : partner, im = even ? partner : v[b];
                 const float rot = even ? re * cs[u].x - im * cs[u].y : re * cs[u].y + im * cs[u].x;
                 if (is_q) {
-                    static_cast<bf16*>(ep.q)[static_cast<long long>(b) * ep.nq + n] = __float2bfloat16_rn(rot);
+                    static_cast<T*>(ep.q)[static_cast<long long>(b) * ep.nq + n] = from_f32<T>(rot);
                 } else {
                     const int row = ep.tok_row ? ep.tok_row[b] : b;
                     cache[static_cast<long long>(row) * ep.kv_row_stride +
                           (static_cast<long long>(head) * ep.max_seq + pos) * ep.hd + d] =
-                        __float2bfloat16_rn(is_k ? rot : v[b]);
+                        from_f32<T>(is_k ? rot : v[b]);
                 }
             }
         }
@@ -108,7 +108,7 @@ __device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int la
             if (row_ok && b < nb) {
                 const float nv = xo[b & 15] + v[b];
                 ep.out[static_cast<long long>(b) * ep.ldo + n] = nv;
-                static_cast<bf16*>(nio.y_out)[static_cast<long long>(b) * ep.ldo + n] = __float2bfloat16_rn(nv * wn);
+                static_cast<T*>(nio.y_out)[static_cast<long long>(b) * ep.ldo + n] = from_f32<T>(nv * wn);
                 sq = nv * nv;
             }
             sq = warp_sum(sq);
@@ -116,7 +116,7 @@ __device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int la
         }
         named_sync(2, 128);
         if (epi_tid < nb)
-            nio.ssq_out[epi_tid * T + t] = ((red[epi_tid] + red[64 + epi_tid]) + red[128 + epi_tid]) +
+            nio.ssq_out[epi_tid * n_tiles + t] = ((red[epi_tid] + red[64 + epi_tid]) + red[128 + epi_tid]) +
                                            red[192 + epi_tid];
         named_sync(2, 128);
     } else if (row_ok) {
@@ -145,15 +145,15 @@ __device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int la
 // it, hand the buffer back to the MMA warp, then either finish the tile or
 // publish this CTA's partial; the CTA that arrives last at a split tile's
 // counter adds the partials in CTA order and finishes it.  Runs are
-// run_begin(c, W, P) .. run_begin(c + 1, W, P) over W = T * KT units.
-template <int BN>
+// run_begin(c, W, P) .. run_begin(c + 1, W, P) over W = n_tiles * KT units.
+template <int BN, typename T>
 __device__ __forceinline__ void decode_epilogue_loop(uint32_t tmem_lane, uint64_t* tfull, uint64_t* tempty, int* flag,
                                                      float* part, int* counters, int c, int P, int u0, int u1,
                                                      int KT, int N, int M, const Epi& ep, const NormIO& nio,
                                                      bool scale_in, const float* rs, float* red, int r, int lane,
                                                      int q, int epi_tid) {
-    const int T = (N + 127) / 128;
-    const int W = T * KT;
+    const int n_tiles = (N + 127) / 128;
+    const int W = n_tiles * KT;
     int u = u0;
     Seg sg;
     int j = 0;
@@ -223,7 +223,7 @@ __device__ __forceinline__ void decode_epilogue_loop(uint32_t tmem_lane, uint64_
             }
             if (epi_tid == 0) counters[t] = 0;
         }
-        finish_tile<BN>(v, t, r, lane, q, epi_tid, nb, N, T, ep, nio, scale_in, rs, red);
+        finish_tile<BN, T>(v, t, r, lane, q, epi_tid, nb, N, n_tiles, ep, nio, scale_in, rs, red);
     }
 }
 

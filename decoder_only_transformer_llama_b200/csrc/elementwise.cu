@@ -52,11 +52,11 @@ int launch_token_map(const RowTable& rt, const int32_t* tokens, int* tok_ids, in
 // x[m, :] = E[tok[m], :] as fp32 (Admin Guide §8.4, tok_embeddings).  An id
 // outside [0, V) yields a zero row and sets LLAMA_ERR_TOKEN_RANGE.
 // With `ssq`, also writes the sum of x^2 over each 128-feature block of the
-// row (ssq[m * dim/128 + block]) and y[m, :] = bf16(x * w_next): the next
-// projection's fused RMSNorm inputs.
+// row (ssq[m * dim/128 + block]) and y[m, :] = x * w_next rounded to the
+// 16-bit type: the next projection's fused RMSNorm inputs.
 template <typename T>
 __global__ void embed_kernel(const int* tok, const T* emb, int dim, int V, float* x, int* status, float* ssq,
-                             bf16* y, const float* w_next) {
+                             T* y, const float* w_next) {
     pdl_trigger();
     pdl_wait();
     const int m = blockIdx.x;
@@ -71,7 +71,7 @@ __global__ void embed_kernel(const int* tok, const T* emb, int dim, int V, float
     }
     const T* src = emb + static_cast<long long>(id) * dim;
     if constexpr (sizeof(T) == 2) {
-        // 8 bf16 per 16-byte load
+        // 8 16-bit values per 16-byte load
         // blockDim.x is a multiple of 16, so the 16 vectors of one 128-feature
         // block always sit in 16 adjacent lanes of one pass
         const uint4* s4 = reinterpret_cast<const uint4*>(src);
@@ -80,7 +80,7 @@ __global__ void embed_kernel(const int* tok, const T* emb, int dim, int V, float
             float sq = 0.f;
             if (i < dim / 8) {
                 uint4 u = s4[i];
-                const bf16* h = reinterpret_cast<const bf16*>(&u);
+                const T* h = reinterpret_cast<const T*>(&u);
                 float4 lo = make_float4(to_f32(h[0]), to_f32(h[1]), to_f32(h[2]), to_f32(h[3]));
                 float4 hi = make_float4(to_f32(h[4]), to_f32(h[5]), to_f32(h[6]), to_f32(h[7]));
                 reinterpret_cast<float4*>(dst)[2 * i] = lo;
@@ -90,15 +90,11 @@ __global__ void embed_kernel(const int* tok, const T* emb, int dim, int V, float
                 if (y) {
                     const float4 w0 = reinterpret_cast<const float4*>(w_next)[2 * i];
                     const float4 w1 = reinterpret_cast<const float4*>(w_next)[2 * i + 1];
-                    __nv_bfloat162 p0 = __floats2bfloat162_rn(lo.x * w0.x, lo.y * w0.y);
-                    __nv_bfloat162 p1 = __floats2bfloat162_rn(lo.z * w0.z, lo.w * w0.w);
-                    __nv_bfloat162 p2 = __floats2bfloat162_rn(hi.x * w1.x, hi.y * w1.y);
-                    __nv_bfloat162 p3 = __floats2bfloat162_rn(hi.z * w1.z, hi.w * w1.w);
                     uint4 pk;
-                    pk.x = *reinterpret_cast<uint32_t*>(&p0);
-                    pk.y = *reinterpret_cast<uint32_t*>(&p1);
-                    pk.z = *reinterpret_cast<uint32_t*>(&p2);
-                    pk.w = *reinterpret_cast<uint32_t*>(&p3);
+                    pk.x = pack2<T>(lo.x * w0.x, lo.y * w0.y);
+                    pk.y = pack2<T>(lo.z * w0.z, lo.w * w0.w);
+                    pk.z = pack2<T>(hi.x * w1.x, hi.y * w1.y);
+                    pk.w = pack2<T>(hi.z * w1.z, hi.w * w1.w);
                     reinterpret_cast<uint4*>(y + static_cast<long long>(m) * dim)[i] = pk;
                 }
             }
@@ -122,6 +118,7 @@ int launch_embed(const int* tok_ids, const void* emb, int dtype, int M, int dim,
     static bool attr = false;
     if (!attr) {
         cudaError_t ce = carveout_max(embed_kernel<bf16>);
+        if (ce == cudaSuccess) ce = carveout_max(embed_kernel<f16>);
         if (ce == cudaSuccess) ce = carveout_max(embed_kernel<float>);
         if (ce != cudaSuccess) return cuda_fail(ce, "cudaFuncSetAttribute(embed_kernel)");
         attr = true;
@@ -130,9 +127,12 @@ int launch_embed(const int* tok_ids, const void* emb, int dtype, int M, int dim,
     if (dtype == LLAMA_BF16)
         e = launch_k(embed_kernel<bf16>, dim3(M), dim3(128), 0, st, pdl, tok_ids, static_cast<const bf16*>(emb),
                      dim, V, x, status, ssq, static_cast<bf16*>(y), w_next);
+    else if (dtype == LLAMA_F16)
+        e = launch_k(embed_kernel<f16>, dim3(M), dim3(128), 0, st, pdl, tok_ids, static_cast<const f16*>(emb),
+                     dim, V, x, status, ssq, static_cast<f16*>(y), w_next);
     else
         e = launch_k(embed_kernel<float>, dim3(M), dim3(128), 0, st, pdl, tok_ids, static_cast<const float*>(emb),
-                     dim, V, x, status, static_cast<float*>(nullptr), static_cast<bf16*>(nullptr),
+                     dim, V, x, status, static_cast<float*>(nullptr), static_cast<float*>(nullptr),
                      static_cast<const float*>(nullptr));
     count_launch();
     if (e != cudaSuccess) return cuda_fail(e, "embed_kernel");
@@ -179,11 +179,9 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* x, const int*
         if (c < nv) {
             const float4 ww = w4[c];
             if constexpr (sizeof(TO) == 2) {
-                __nv_bfloat162 p0 = __floats2bfloat162_rn(v[i].x * inv * ww.x, v[i].y * inv * ww.y);
-                __nv_bfloat162 p1 = __floats2bfloat162_rn(v[i].z * inv * ww.z, v[i].w * inv * ww.w);
                 uint2 u;
-                u.x = *reinterpret_cast<uint32_t*>(&p0);
-                u.y = *reinterpret_cast<uint32_t*>(&p1);
+                u.x = pack2<TO>(v[i].x * inv * ww.x, v[i].y * inv * ww.y);
+                u.y = pack2<TO>(v[i].z * inv * ww.z, v[i].w * inv * ww.w);
                 reinterpret_cast<uint2*>(orow)[c] = u;
             } else {
                 reinterpret_cast<float4*>(orow)[c] =
@@ -217,6 +215,8 @@ int launch_rmsnorm(const float* x, const int* row_idx, const float* w, int M, in
     if (M <= 0) return LLAMA_OK;
     if (out_dtype == LLAMA_BF16)
         return rmsnorm_dispatch<bf16>(x, row_idx, w, M, dim, eps, static_cast<bf16*>(out), st, pdl);
+    if (out_dtype == LLAMA_F16)
+        return rmsnorm_dispatch<f16>(x, row_idx, w, M, dim, eps, static_cast<f16*>(out), st, pdl);
     return rmsnorm_dispatch<float>(x, row_idx, w, M, dim, eps, static_cast<float*>(out), st, pdl);
 }
 

@@ -1,4 +1,4 @@
-// Decode-shaped bf16 projections (few token rows) on tcgen05: a persistent,
+// Decode-shaped 16-bit (bf16 or fp16) projections (few token rows) on tcgen05: a persistent,
 // stream-K, weight-streaming kernel.
 //
 // acc[n, b] = sum_k W[n, k] * X[b, k] for b < M <= 64 token rows.  The weight
@@ -16,7 +16,8 @@
 //
 // Fused RMSNorm (Admin Guide §8.4, RMSNorm before wq/wk/wv, before w1/w3 and
 // before the output projection), see NormIO: a residual epilogue here also
-// writes the next projection's operand bf16(x * w_next) and per-tile sums of
+// writes the next projection's operand, x * w_next rounded to the model's 16-bit
+// type, and per-tile sums of
 // x^2; a consuming projection scales accumulator column b by r_b.
 // A deep ring (about 200 KB of weight tiles in flight per SM) keeps HBM
 // busy; the next projection's CTAs launch early (programmatic dependent
@@ -37,7 +38,7 @@ constexpr int kAccStride = 64;      // TMEM columns per accumulator buffer
 constexpr int kTmemCols = 128;      // two accumulator buffers
 }  // namespace
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, typename E>
 __global__ void __launch_bounds__(kThreads, 1)
 linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUtensorMap mapX,
                      int N, int M, int K, Epi ep, float* __restrict__ part, int* __restrict__ counters, NormIO nio) {
@@ -111,7 +112,7 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
         }
     } else if (warp == 1 && lane == 0) {
         // ---------------- MMA issuer
-        const uint32_t idesc = idesc_bf16_f32(128, BN);
+        const uint32_t idesc = idesc_16_f32<E>(128, BN);
         int u = u0;
         Seg sg;
         int i = 0, j = 0;
@@ -129,7 +130,7 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
                 const uint32_t b0 = a0 + kABytes;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    tc_mma_bf16(d, smem_desc_k_sw128(a0 + kk * 32), smem_desc_k_sw128(b0 + kk * 32), idesc,
+                    tc_mma_16(d, smem_desc_k_sw128(a0 + kk * 32), smem_desc_k_sw128(b0 + kk * 32), idesc,
                                 (k > sg.ks || kk > 0) ? 1u : 0u);
                 tc_commit(&empty[s]);
             }
@@ -150,7 +151,7 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
             rs[epi_tid] = rsqrtf(ss / static_cast<float>(K) + nio.eps);
         }
         named_sync(1, 128);
-        decode_epilogue_loop<BN>(tmem + lane_base, tfull, tempty, flag, part, counters, c, P, u0, u1, KT, N, M, ep,
+        decode_epilogue_loop<BN, E>(tmem + lane_base, tfull, tempty, flag, part, counters, c, P, u0, u1, KT, N, M, ep,
                                  nio, scale_in, rs, red, r, lane, q, epi_tid);
     }
 
@@ -163,12 +164,12 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
 // ---------------------------------------------------------------- host side
 static int g_sms = 0;
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, typename E>
 static int launch_decode(const CUtensorMap& w, const CUtensorMap& x, int N, int M, int K, const Epi& ep,
                          float* part, int* counters, int max_ctas, cudaStream_t st, bool pdl, const NormIO& nio) {
     constexpr int smem = 1024 + STAGES * (kABytes + BN * 128) + (2 * STAGES + 4) * 8 + 32 + 5 * 64 * 4;
     static_assert(smem <= 227 * 1024, "shared memory per CTA");
-    auto kern = linear_decode_kernel<BN, STAGES>;
+    auto kern = linear_decode_kernel<BN, STAGES, E>;
     static bool attr = false;
     if (!attr) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -187,8 +188,18 @@ static int launch_decode(const CUtensorMap& w, const CUtensorMap& x, int N, int 
     return LLAMA_OK;
 }
 
-int linear_bf16_decode(const TmaMaps* mapX, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
-                       size_t part_bytes, int* counters, cudaStream_t st, bool pdl, const NormIO* nio_in) {
+// Token-row count -> MMA width (BN) and ring depth.
+template <typename E>
+static int decode_by_rows(const TmaMaps* mapX, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
+                          int* counters, cudaStream_t st, bool pdl, const NormIO& nio) {
+    if (M <= 16) return launch_decode<16, 12, E>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio);
+    if (M <= 32) return launch_decode<32, 11, E>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio);
+    if (M <= 48) return launch_decode<48, 10, E>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio);
+    return launch_decode<64, 9, E>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio);
+}
+
+int linear16_decode(const TmaMaps* mapX, const TmaMaps* mapW, int M, int N, int K, int dtype, const Epi& ep, float* part,
+                    size_t part_bytes, int* counters, cudaStream_t st, bool pdl, const NormIO* nio_in) {
     if (M <= 0 || N <= 0) return LLAMA_OK;
     NormIO nio = {};
     if (nio_in) nio = *nio_in;
@@ -213,10 +224,10 @@ int linear_bf16_decode(const TmaMaps* mapX, const TmaMaps* mapW, int M, int N, i
         if (g_sms <= 0) g_sms = 148;
         if (g_sms > kMaxDecodeCtas) g_sms = kMaxDecodeCtas;
     }
-    if (M <= 16) return launch_decode<16, 12>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio);
-    if (M <= 32) return launch_decode<32, 11>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio);
-    if (M <= 48) return launch_decode<48, 10>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio);
-    return launch_decode<64, 9>(mapW->a128, mapX->b, N, M, K, ep, part, counters, g_sms, st, pdl, nio);
+    if (dtype == LLAMA_F16) return decode_by_rows<f16>(mapX, mapW, M, N, K, ep, part, counters, st, pdl, nio);
+    if (dtype == LLAMA_BF16) return decode_by_rows<bf16>(mapX, mapW, M, N, K, ep, part, counters, st, pdl, nio);
+    set_error("16-bit projection: dtype must be LLAMA_BF16 or LLAMA_F16");
+    return LLAMA_ERR_INVALID_ARG;
 }
 
 }  // namespace llb

@@ -1,4 +1,4 @@
-// bf16 projections on the 5th-generation tensor cores (tcgen05), fed by TMA,
+// 16-bit (bf16 or fp16) projections on the 5th-generation tensor cores (tcgen05), fed by TMA,
 // accumulating in TMEM, with the fused epilogues of the forward pass
 // (Admin Guide §8.4: wq/wk/wv + RoPE + KV-cache append, wo + residual,
 // w1/w3 + silu*mul, w2 + residual, output projection).
@@ -7,7 +7,7 @@
 // projections (<= 64 rows) run in gemm_decode.cu.
 //
 // D[i, j] = sum_k A[i, k] * B[j, k]; A = activations [tokens, K], B = weights
-// [N, K], both K-major bf16 read through 128-byte-swizzled TMA boxes of 64
+// [N, K], both K-major 16-bit read through 128-byte-swizzled TMA boxes of 64
 // K-elements.  D is cut into 128 x 256 tiles, ordered in groups of 16 tiles
 // along M (all N-tiles of one group before the next group), so that the
 // tiles in flight at any time share a few hundred KB of A and B in L2.
@@ -44,31 +44,28 @@ namespace {
 constexpr int kThreadsTc = 192;
 constexpr int kBN = 256;                     // tile width along N (weight rows)
 constexpr int kStagesTc = 4;
-constexpr int kA_BYTES = 128 * 128;          // 128 rows x 64 bf16
+constexpr int kA_BYTES = 128 * 128;          // 128 rows x 64 16-bit values
 constexpr int kB_BYTES = kBN * 128;
 constexpr int kStageBytes = kA_BYTES + kB_BYTES;
 constexpr int kPartFloats = 128 * kBN;       // one fp32 partial tile
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
-    __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<uint32_t*>(&p);
-}
-
-// Store 32 consecutive values as bf16 (64 bytes, 16-byte aligned destination).
-__device__ __forceinline__ void store32_bf16(bf16* dst, const float* v) {
+// Store 32 consecutive values in the 16-bit type E (64 bytes, 16-byte aligned destination).
+template <typename E>
+__device__ __forceinline__ void store32_16(E* dst, const float* v) {
     uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         uint4 u;
-        u.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
-        u.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
-        u.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
-        u.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+        u.x = pack2<E>(v[8 * q + 0], v[8 * q + 1]);
+        u.y = pack2<E>(v[8 * q + 2], v[8 * q + 3]);
+        u.z = pack2<E>(v[8 * q + 4], v[8 * q + 5]);
+        u.w = pack2<E>(v[8 * q + 6], v[8 * q + 7]);
         d[q] = u;
     }
 }
 
 // Epilogue of 32 consecutive output features n0..n0+31 of token row m.
+template <typename E>
 __device__ __forceinline__ void epi_chunk(const Epi& ep, int m, int n0, int rowsB, float (&v)[32]) {
     if (n0 >= rowsB) return;
     if (ep.mode == EPI_SWIGLU) {
@@ -76,32 +73,32 @@ __device__ __forceinline__ void epi_chunk(const Epi& ep, int m, int n0, int rows
         float g16[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t) g16[t] = silu_f(v[t]) * v[16 + t];
-        bf16* dst = static_cast<bf16*>(ep.g) + static_cast<long long>(m) * ep.H + (n0 / 32) * 16;
+        E* dst = static_cast<E*>(ep.g) + static_cast<long long>(m) * ep.H + (n0 / 32) * 16;
         uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
             uint4 u;
-            u.x = pack_bf16x2(g16[8 * q + 0], g16[8 * q + 1]);
-            u.y = pack_bf16x2(g16[8 * q + 2], g16[8 * q + 3]);
-            u.z = pack_bf16x2(g16[8 * q + 4], g16[8 * q + 5]);
-            u.w = pack_bf16x2(g16[8 * q + 6], g16[8 * q + 7]);
+            u.x = pack2<E>(g16[8 * q + 0], g16[8 * q + 1]);
+            u.y = pack2<E>(g16[8 * q + 2], g16[8 * q + 3]);
+            u.z = pack2<E>(g16[8 * q + 4], g16[8 * q + 5]);
+            u.w = pack2<E>(g16[8 * q + 6], g16[8 * q + 7]);
             d4[q] = u;
         }
     } else if (ep.mode == EPI_QKV) {
         const int pos = ep.tok_pos[m];
         if (pos < 0 || pos >= ep.max_seq) return;
-        bf16* dst;
+        E* dst;
         bool rot;
         int d0;
         if (n0 < ep.nq) {
             d0 = n0 % ep.hd;
             rot = true;
-            dst = static_cast<bf16*>(ep.q) + static_cast<long long>(m) * ep.nq + n0;
+            dst = static_cast<E*>(ep.q) + static_cast<long long>(m) * ep.nq + n0;
         } else {
             int cc = n0 - ep.nq;
-            bf16* cache = static_cast<bf16*>(ep.kc);
+            E* cache = static_cast<E*>(ep.kc);
             rot = cc < ep.nkvc;
-            if (!rot) { cc -= ep.nkvc; cache = static_cast<bf16*>(ep.vc); }
+            if (!rot) { cc -= ep.nkvc; cache = static_cast<E*>(ep.vc); }
             const int head = cc / ep.hd;
             d0 = cc % ep.hd;
             const int row = ep.tok_row ? ep.tok_row[m] : m;
@@ -112,7 +109,7 @@ __device__ __forceinline__ void epi_chunk(const Epi& ep, int m, int n0, int rows
 #pragma unroll
             for (int t = 0; t < 32; t += 2) rope_pair(ep.rope, ep.hd, pos, (d0 + t) >> 1, v[t], v[t + 1]);
         }
-        store32_bf16(dst, v);
+        store32_16<E>(dst, v);
     } else {
         float* o = ep.out + static_cast<long long>(m) * ep.ldo + n0;
         const int lim = min(32, rowsB - n0);
@@ -140,6 +137,7 @@ __device__ __forceinline__ void epi_chunk(const Epi& ep, int m, int n0, int rows
 
 }  // namespace
 
+template <typename E>
 __global__ void __launch_bounds__(kThreadsTc, 1)
 linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                   int rowsA, int rowsB, TcPlan plan, Epi ep, float* __restrict__ part, int* __restrict__ counters) {
@@ -190,7 +188,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
         }
     } else if (warp == 1 && lane == 0) {
         // ---------------- MMA issuer
-        const uint32_t idesc = idesc_bf16_f32(128, kBN);
+        const uint32_t idesc = idesc_16_f32<E>(128, kBN);
         WorkIt w = work_begin(plan, c, P);
         Item it;
         int i = 0, j = 0;
@@ -208,7 +206,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
                 const uint32_t b0 = a0 + kA_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    tc_mma_bf16(d, smem_desc_k_sw128(a0 + kk * 32), smem_desc_k_sw128(b0 + kk * 32), idesc,
+                    tc_mma_16(d, smem_desc_k_sw128(a0 + kk * 32), smem_desc_k_sw128(b0 + kk * 32), idesc,
                                 (k > it.ks || kk > 0) ? 1u : 0u);
                 tc_commit(&empty[s]);
             }
@@ -249,7 +247,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
                     float v[32];
                     tmem_ld_32x32b_x32(tb + cc * 32, v);
                     tc_wait_ld();
-                    if (row_ok) epi_chunk(ep, m, nbase + cc * 32, rowsB, v);
+                    if (row_ok) epi_chunk<E>(ep, m, nbase + cc * 32, rowsB, v);
                 }
                 tc_fence_before();
                 mbar_arrive(&tempty[acc]);
@@ -301,7 +299,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
                         for (int t = 0; t < 32; ++t) v[t] += f[t];
                     }
                 }
-                if (row_ok) epi_chunk(ep, m, nbase + cc * 32, rowsB, v);
+                if (row_ok) epi_chunk<E>(ep, m, nbase + cc * 32, rowsB, v);
             }
             tc_fence_before();
             mbar_arrive(&tempty[acc]);
@@ -318,7 +316,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
 
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
-int encode_kmajor_bf16(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
+int encode_kmajor_16(CUtensorMap* map, const void* base, int rows, int cols, int box_rows, int dtype) {
     if (!g_encode) {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -337,7 +335,8 @@ int encode_kmajor_bf16(CUtensorMap* map, const void* base, int rows, int cols, i
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
     cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+    const CUtensorMapDataType dt = dtype == LLAMA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUresult r = g_encode(map, dt, 2, const_cast<void*>(base), dims, strides,
                           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
@@ -350,14 +349,15 @@ int encode_kmajor_bf16(CUtensorMap* map, const void* base, int rows, int cols, i
 
 static int g_sms_tc = 0;
 
-int linear_bf16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
-                   int* counters, cudaStream_t st) {
+template <typename E>
+static int launch_tcp(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
+                      int* counters, cudaStream_t st) {
     if (M <= 0 || N <= 0) return LLAMA_OK;
     constexpr int smem = 1024 + kStagesTc * kStageBytes + (2 * kStagesTc + 4) * 8 + 16;
     static_assert(smem <= 227 * 1024, "shared memory per CTA");
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(linear_tcp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e = cudaFuncSetAttribute(linear_tcp_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(linear_tcp_kernel)");
         attr_set = true;
     }
@@ -377,16 +377,24 @@ int linear_bf16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K
     int grid = 0;
     plan_tc(static_cast<int>(T), plan.KT, g_sms_tc, part != nullptr && counters != nullptr, &plan, &grid);
     if (plan.sk > kMaxTiles) { set_error("internal: %d split tiles exceed the counters", plan.sk); return LLAMA_ERR_INVALID_ARG; }
-    linear_tcp_kernel<<<grid, kThreadsTc, smem, st>>>(mapA->a128, mapW->b, M, N, plan, ep, part, counters);
+    linear_tcp_kernel<E><<<grid, kThreadsTc, smem, st>>>(mapA->a128, mapW->b, M, N, plan, ep, part, counters);
     LLB_CHECK_LAUNCH("linear_tcp_kernel");
     return LLAMA_OK;
 }
 
-int linear_bf16(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
-                size_t part_bytes, int* counters, cudaStream_t st, bool pdl, const NormIO* nio) {
-    if (M <= 64) return linear_bf16_decode(mapA, mapW, M, N, K, ep, part, part_bytes, counters, st, pdl, nio);
+int linear16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, int dtype, const Epi& ep, float* part,
+                int* counters, cudaStream_t st) {
+    if (dtype == LLAMA_F16) return launch_tcp<f16>(mapA, mapW, M, N, K, ep, part, counters, st);
+    if (dtype == LLAMA_BF16) return launch_tcp<bf16>(mapA, mapW, M, N, K, ep, part, counters, st);
+    set_error("16-bit projection: dtype must be LLAMA_BF16 or LLAMA_F16");
+    return LLAMA_ERR_INVALID_ARG;
+}
+
+int linear16(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, int dtype, const Epi& ep, float* part,
+             size_t part_bytes, int* counters, cudaStream_t st, bool pdl, const NormIO* nio) {
+    if (M <= 64) return linear16_decode(mapA, mapW, M, N, K, dtype, ep, part, part_bytes, counters, st, pdl, nio);
     if (nio && (nio->ssq_in || nio->ssq_out)) { set_error("fused RMSNorm is a decode-shape feature"); return LLAMA_ERR_INVALID_ARG; }
-    return linear_bf16_tc(mapA, mapW, M, N, K, ep, part, counters, st);
+    return linear16_tc(mapA, mapW, M, N, K, dtype, ep, part, counters, st);
 }
 
 }  // namespace llb

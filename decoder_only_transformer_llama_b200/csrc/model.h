@@ -152,20 +152,20 @@ int launch_copy_interleave_w13(const void* src, void* w13, int H, int dim, int w
                                cudaStream_t st);
 
 // out = A W^T with epilogue `ep`.  A rows: M (tokens), W rows: N, K.
-// bf16 uses tcgen05 with the given maps (A-side/W-side), fp32 the SIMT kernel.
+// 16-bit dtypes use tcgen05 with the given maps (A-side/W-side), fp32 the SIMT kernel.
 int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, const void* W,
                const TmaMaps* mapW, int M, int N, int K, const Epi& ep, cudaStream_t st, bool pdl = false,
                const NormIO* nio = nullptr);
 int linear_f32(const float* A, const float* W, int M, int N, int K, const Epi& ep, cudaStream_t st);
 // Prefill-shaped projection; with part/counters (kGemmPartBytes, kMaxTiles
 // zeroed ints) the tail wave is split stream-K, without them whole tiles only.
-int linear_bf16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
-                   int* counters, cudaStream_t st);
-int linear_bf16_decode(const TmaMaps* mapX, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
-                       size_t part_bytes, int* counters, cudaStream_t st, bool pdl, const NormIO* nio = nullptr);
-// bf16 projection: M <= 64 token rows -> linear_bf16_decode, else linear_bf16_tc.
-int linear_bf16(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
-                size_t part_bytes, int* counters, cudaStream_t st, bool pdl = false, const NormIO* nio = nullptr);
+int linear16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, int dtype, const Epi& ep, float* part,
+                int* counters, cudaStream_t st);
+int linear16_decode(const TmaMaps* mapX, const TmaMaps* mapW, int M, int N, int K, int dtype, const Epi& ep, float* part,
+                    size_t part_bytes, int* counters, cudaStream_t st, bool pdl, const NormIO* nio = nullptr);
+// 16-bit projection: M <= 64 token rows -> linear16_decode, else linear16_tc.
+int linear16(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, int dtype, const Epi& ep, float* part,
+             size_t part_bytes, int* counters, cudaStream_t st, bool pdl = false, const NormIO* nio = nullptr);
 
 int launch_attention_prefill(const Model* m, int layer, const RowTable& rt, cudaStream_t st);
 int launch_attention_prefill_tc(const Model* m, int layer, const RowTable& rt, cudaStream_t st);
@@ -179,7 +179,9 @@ int launch_top_p(const float* logits, int B, int V, float temperature, float top
                  const float* uniforms, int32_t* out, int32_t* tokens_adv, int32_t* pos_adv,
                  cudaStream_t st, bool pdl = false);
 
-// TMA descriptor encoding (driver entry point resolved at run time).
-int encode_kmajor_bf16(CUtensorMap* map, const void* base, int rows, int cols, int box_rows);
+// TMA descriptor of a K-major 16-bit matrix (dtype LLAMA_BF16 or LLAMA_F16),
+// boxes of 64 columns x box_rows rows, 128-byte swizzle (driver entry point
+// resolved at run time).
+int encode_kmajor_16(CUtensorMap* map, const void* base, int rows, int cols, int box_rows, int dtype = LLAMA_BF16);
 
 }  // namespace llb

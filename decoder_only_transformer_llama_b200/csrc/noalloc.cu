@@ -86,15 +86,15 @@ extern "C" int llama_op_linear_noalloc(const void* A, const void* W, int M, int 
     cudaError_t e = cudaMemsetAsync(cnt, 0, kNoAllocCntBytes, st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(noalloc counters)");
     TmaMaps ma, mw;
-    int r2 = encode_kmajor_bf16(&ma.a128, A, M, K, 128);
-    if (r2 == LLAMA_OK) r2 = encode_kmajor_bf16(&ma.b, A, M, K, 16);
-    if (r2 == LLAMA_OK) r2 = encode_kmajor_bf16(&mw.a128, W, N, K, 128);
-    if (r2 == LLAMA_OK) r2 = encode_kmajor_bf16(&mw.b, W, N, K, 256);
+    int r2 = encode_kmajor_16(&ma.a128, A, M, K, 128);
+    if (r2 == LLAMA_OK) r2 = encode_kmajor_16(&ma.b, A, M, K, 16);
+    if (r2 == LLAMA_OK) r2 = encode_kmajor_16(&mw.a128, W, N, K, 128);
+    if (r2 == LLAMA_OK) r2 = encode_kmajor_16(&mw.b, W, N, K, 256);
     if (r2 != LLAMA_OK) return r2;
     Epi ep;
     memset(&ep, 0, sizeof(ep));
     ep.mode = EPI_STORE_F32;
     ep.out = out;
     ep.ldo = N;
-    return linear_bf16_decode(&ma, &mw, M, N, K, ep, part, kNoAllocPartBytes, cnt, st, false);
+    return linear16_decode(&ma, &mw, M, N, K, LLAMA_BF16, ep, part, kNoAllocPartBytes, cnt, st, false);
 }

@@ -29,7 +29,7 @@
  *     model's device status word instead; read it with llama_model_status.
  *   - Layouts: matrices are row-major [out_features, in_features] like
  *     nn.Linear (y = x W^T); RMSNorm weights are fp32; other weights are in
- *     the model dtype (fp32 or bf16).
+ *     the model dtype (fp32, bf16 or fp16).
  *   - Thread safety: calls on one model must be serialised by the caller
  *     (they share the model's workspace).
  */
@@ -61,6 +61,9 @@ extern "C" {
 /* ---- dtypes --------------------------------------------------------------- */
 #define LLAMA_F32   0   /* fp32 storage and fp32 arithmetic (no TF32)          */
 #define LLAMA_BF16  1   /* bf16 storage, fp32 accumulation                     */
+#define LLAMA_F16   2   /* fp16 storage (the reference's own dtype, Admin Guide
+                           §1.4 and §6.4), fp32 accumulation; the bf16
+                           kernels instantiated for fp16                    */
 
 /*
  * Structural configuration: the fields of ModelArgs (Admin Guide §3.3) plus

@@ -112,14 +112,15 @@ def test_token_outside_the_vocabulary_sets_token_range_status(llb):
     m.close()
 
 
-def test_prefix_reuse_across_prefill_calls(llb):
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_prefix_reuse_across_prefill_calls(llb, dtype):
     """A prefix prefilled once, then two different continuations prefilled at
     start_pos = len(prefix) one after the other (the second overwrites the
     first's cache entries): every position's logits equal the oracle's on
     prefix + continuation.  Continuation lengths put the projections on both
     kernels (<= 64 token rows: the weight-streaming kernel; more: the
     128 x 256-tile kernel) and the prefill attention on start_pos > 0."""
-    shape = SMALL.replace(max_seq_len=192)
+    shape = SMALL.replace(max_seq_len=192, dtype=dtype)
     w = make_weights(shape, 45)
     m = build_model(shape, w)
     w64 = to_numpy_f64_weights(w)

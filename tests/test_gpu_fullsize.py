@@ -58,10 +58,12 @@ def _run(llb, shape, B, T, lens, steps, rows, seed_idx, start_pos=0):
         check_greedy(seqs[b][L:], want[:steps])
 
 
-def test_7b_dims_prefill_4x512_then_decode(llb):
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_7b_dims_prefill_4x512_then_decode(llb, dtype):
     """7B layer dimensions, batch 4 x 512 prefill (the benchmark's launch
-    configuration), 3 greedy decode steps; oracle on rows 0 and 3."""
-    s = L7B.replace(n_layers=2)
+    configuration), 3 greedy decode steps; oracle on rows 0 and 3; bf16 and
+    the reference's own fp16."""
+    s = L7B.replace(n_layers=2, dtype=dtype)
     _run(llb, s, B=4, T=512, lens=[512] * 4, steps=3, rows=[0, 3], seed_idx=2)
 
 
@@ -75,8 +77,9 @@ def test_13b_dims_ragged_prefill_then_decode(llb):
     _run(llb, s, B=16, T=T, lens=lens, steps=2, rows=order[:2], seed_idx=3)
 
 
-def test_70b_gqa_dims_prefill_then_decode(llb):
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_70b_gqa_dims_prefill_then_decode(llb, dtype):
     """70B layer dimensions (64 query heads over 8 KV heads, hidden 28672),
-    batch 8 x 256 prefill, 2 decode steps; oracle on row 5."""
-    s = L70B_SLICE.replace(n_layers=2, max_tokens=8 * 256)
+    batch 8 x 256 prefill, 2 decode steps; oracle on row 5; bf16 and fp16."""
+    s = L70B_SLICE.replace(n_layers=2, max_tokens=8 * 256, dtype=dtype)
     _run(llb, s, B=8, T=256, lens=[256] * 8, steps=2, rows=[5], seed_idx=4)

@@ -251,13 +251,16 @@ SMALL_BF16 = ModelShape(dim=256, n_layers=2, n_heads=2, n_kv_heads=1, vocab_size
                         max_batch_size=3, dtype="bf16", hidden=768)
 
 
-def test_small_bf16_gqa_ragged_prefill_and_decode(llb):
-    """bf16 path (tcgen05 projections, head_dim 128, n_rep 2) with ragged
-    prompt lengths and per-row decode positions."""
-    w = make_weights(SMALL_BF16, 99)
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_small_bf16_gqa_ragged_prefill_and_decode(llb, dtype):
+    """16-bit path (tcgen05 projections, head_dim 128, n_rep 2) with ragged
+    prompt lengths and per-row decode positions, in bf16 and in the
+    reference's own fp16."""
+    shape = SMALL_BF16.replace(dtype=dtype)
+    w = make_weights(shape, 99)
     lens = [37, 64, 5]
-    seq, gl = _tiny_run(llb, SMALL_BF16, w, B=3, T=64, steps=12, lens=lens)
-    _oracle_check(SMALL_BF16, w, seq, gl, lens, BF16_TOL)
+    seq, gl = _tiny_run(llb, shape, w, B=3, T=64, steps=12, lens=lens)
+    _oracle_check(shape, w, seq, gl, lens, BF16_TOL)
 
 
 def test_small_bf16_decode_with_top_p_sampling(llb):
@@ -311,16 +314,16 @@ def test_small_bf16_decode_with_top_p_sampling(llb):
         assert rel_l2(got, want) <= BF16_TOL, (b, rel_l2(got, want))
 
 
-@pytest.mark.parametrize("B,L", [(1, 128), (8, 1024), (32, 4096)])
-def test_7b_layer_decode_against_oracle(llb, B, L):
+@pytest.mark.parametrize("B,L,dtype", [(1, 128, "bf16"), (8, 1024, "bf16"), (32, 4096, "bf16"), (8, 1024, "f16")])
+def test_7b_layer_decode_against_oracle(llb, B, L, dtype):
     """One 7B-shaped layer (bf16, fp32 norms), KV cache filled with N(0,1) for
     positions [0, L), one decode step at position L; oracle on sampled rows."""
-    s = L7B_LAYER
+    s = L7B_LAYER.replace(dtype=dtype)
     w = make_weights(s, weight_seed(1), device="cuda")
     m = build_model(s, w)
     kview, vview = m.kv_tensors(0)
-    fillk = make_normal((B, L, s.n_kv_heads, s.head_dim), 11, device="cuda")
-    fillv = make_normal((B, L, s.n_kv_heads, s.head_dim), 12, device="cuda")
+    fillk = make_normal((B, L, s.n_kv_heads, s.head_dim), 11, device="cuda", dtype=kview.dtype)
+    fillv = make_normal((B, L, s.n_kv_heads, s.head_dim), 12, device="cuda", dtype=kview.dtype)
     kview[:B, :L].copy_(fillk)
     vview[:B, :L].copy_(fillv)
     torch.cuda.synchronize()

@@ -14,7 +14,7 @@ real checkpoints are licence-gated (same guide, §7.1).
 Draw order (fixed, documented): tok_embeddings; then per layer
 attention_norm, wq, wk, wv, wo, ffn_norm, w1, w2, w3; then norm; output.
 Matrices are N(0, 0.02); RMSNorm weights are 1 + N(0, 0.02) stored fp32.
-bf16 models round each matrix to bf16 once, right after its draw.
+16-bit models (bf16, f16) round each matrix to that type once, right after its draw.
 """
 from __future__ import annotations
 
@@ -42,7 +42,7 @@ class ModelShape:
     max_seq_len: int = 2048
     max_batch_size: int = 32
     max_tokens: int = 0
-    dtype: str = "bf16"  # "f32" or "bf16"
+    dtype: str = "bf16"  # "f32", "bf16" or "f16"
     hidden: int = 0  # FFN width as the workload states it (checked against the oracle's rule)
 
     @property
@@ -120,7 +120,8 @@ def _draw(name: str, shape: tuple, gen: torch.Generator, device, dtype: str) -> 
     t = torch.randn(shape, generator=gen, device=device, dtype=torch.float32) * 0.02
     if name in NORM_WEIGHTS:
         return t + 1.0  # fp32 norm weights
-    return t.to(torch.bfloat16) if dtype == "bf16" else t
+    half = {"bf16": torch.bfloat16, "f16": torch.float16}.get(dtype)
+    return t.to(half) if half is not None else t
 
 
 def make_weights(s: ModelShape, seed: int, device="cpu", n_layers: Optional[int] = None) -> dict:
@@ -172,7 +173,7 @@ def make_normal(shape, seed: int, device="cpu", dtype=torch.bfloat16, std: float
 
 
 def to_numpy_f64_weights(w: dict) -> dict:
-    """Upcast a weight dict to float64 numpy arrays (exact for bf16 and fp32)."""
+    """Upcast a weight dict to float64 numpy arrays (exact for bf16, fp16 and fp32)."""
     out = {"tok_embeddings": w["tok_embeddings"].detach().cpu().double().numpy(),
            "norm": w["norm"].detach().cpu().double().numpy(),
            "output": w["output"].detach().cpu().double().numpy(),
