@@ -54,10 +54,10 @@ struct Epi {
     int* status;
 };
 
-// RMSNorm folded into the decode projections (16-bit decode chain), using
+// RMSNorm folded into the decode projections (bf16 decode chain), using
 // norm(x) W^T = r_b * ((x * w) W^T) with r_b = 1/sqrt(mean(x_b^2) + eps):
 //   producer side (residual epilogue of wo / w2, and the embedding): besides
-//     x it writes y_out[b, n] = x[b, n] * w_next[n] in the 16-bit type -- the operand of the
+//     x it writes y_out[b, n] = bf16(x[b, n] * w_next[n]) -- the operand of the
 //     next projection, w_next the weight of the norm in front of it -- and
 //     ssq_out[b * n_tiles + t] = sum of x^2 over the 128 features of tile t;
 //   consumer side (wq/wk/wv, w1/w3, output): multiplies accumulator column b
@@ -72,7 +72,7 @@ struct NormIO {
     const float* w_next;
 };
 
-struct TmaMaps {               // tensor maps of one K-major 16-bit matrix
+struct TmaMaps {               // tensor maps of one K-major bf16 matrix
     CUtensorMap a128;          // box 64 x 128 rows (the MMA's A operand)
     CUtensorMap b;             // box 64 x 256 rows (weights as B) or 64 x 16 (activations as B)
 };
@@ -142,7 +142,7 @@ int launch_token_map(const RowTable& rt, const int32_t* tokens, int* tok_ids, in
                      int* tok_pos, int* last_idx, cudaStream_t st);
 // `pdl`: launch as part of the decode chain (may start before its predecessor ends).
 // With `ssq`, also writes the sum of x^2 of every 128-feature block and
-// y = x * w_next in the 16-bit type (the fused RMSNorm's producer side, see NormIO).
+// y = bf16(x * w_next) (the fused RMSNorm's producer side, see NormIO).
 int launch_embed(const int* tok_ids, const void* emb, int dtype, int M, int dim, int V, float* x,
                  int* status, cudaStream_t st, bool pdl = false, float* ssq = nullptr, void* y = nullptr,
                  const float* w_next = nullptr);
