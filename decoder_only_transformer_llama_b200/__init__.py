@@ -276,9 +276,34 @@ def token_logprobs(logits, tokens, out, stream=None):
     return out
 
 
+_TORCH_DTYPES = {"torch.float32": LLAMA_F32, "torch.bfloat16": LLAMA_BF16, "torch.float16": LLAMA_F16}
+
+
+def _dtype_code(t, what: str) -> int:
+    code = _TORCH_DTYPES.get(str(t.dtype))
+    if code is None:
+        raise ValueError(f"{what} must be float32, bfloat16 or float16, not {t.dtype}")
+    return code
+
+
+def _need(cond: bool, msg: str):
+    if not cond:
+        raise ValueError(msg)
+
+
+def _check_linear_operands(A, W, out):
+    M, K = A.shape
+    _need(W.dim() == 2 and W.dtype == A.dtype and W.shape[1] == K, "W must be [N, K] of A's dtype")
+    _need(str(out.dtype) == "torch.float32" and tuple(out.shape) == (M, W.shape[0]), "out must be float32 [M, N]")
+    _need(A.is_contiguous() and W.is_contiguous() and out.is_contiguous(), "tensors must be contiguous")
+
+
 def op_rmsnorm(x, w, eps: float, out, stream=None):
     M, dim = x.shape
-    dt = {"torch.bfloat16": LLAMA_BF16, "torch.float16": LLAMA_F16}.get(out.dtype.__str__(), LLAMA_F32)
+    _need(str(x.dtype) == "torch.float32" and str(w.dtype) == "torch.float32", "x and w must be float32")
+    _need(tuple(out.shape) == (M, dim) and w.numel() == dim, "out must be [M, dim] and w [dim]")
+    _need(x.is_contiguous() and w.is_contiguous() and out.is_contiguous(), "tensors must be contiguous")
+    dt = _dtype_code(out, "out")
     _check(_lib.llama_op_rmsnorm(x.data_ptr(), w.data_ptr(), M, dim, float(eps), out.data_ptr(), dt,
                                  _stream(stream)))
     return out
@@ -301,27 +326,35 @@ def op_linear_noalloc(A, W, out, stream=None):
     the caller: for callers that cannot allocate device memory."""
     M, K = A.shape
     N = W.shape[0]
+    _check_linear_operands(A, W, out)
+    _need(_dtype_code(A, "A") == LLAMA_BF16, "op_linear_noalloc takes bfloat16 operands")
     _check(_lib.llama_op_linear_noalloc(A.data_ptr(), W.data_ptr(), M, N, K, out.data_ptr(), _stream(stream)))
     return out
 
 
 def op_linear_whole_tiles(A, W, out, stream=None):
-    """bf16 projection with M > 64 and no workspace: every tile runs whole
+    """16-bit projection with M > 64 and no workspace: every tile runs whole
     (no stream-K split of the last wave)."""
     M, K = A.shape
     N = W.shape[0]
     if M <= 64:
         raise ValueError("op_linear_whole_tiles takes M > 64 token rows")
-    _check(_lib.llama_op_linear(A.data_ptr(), W.data_ptr(), M, N, K, LLAMA_BF16, out.data_ptr(), None, 0,
+    _check_linear_operands(A, W, out)
+    dt = _dtype_code(A, "A")
+    _need(dt != LLAMA_F32, "op_linear_whole_tiles takes bfloat16 or float16 operands")
+    _check(_lib.llama_op_linear(A.data_ptr(), W.data_ptr(), M, N, K, dt, out.data_ptr(), None, 0,
                                 _stream(stream)))
     return out
 
 
 def op_linear(A, W, out, stream=None, workspace=None):
+    """out = A W^T: A [M, K] and W [N, K] of one type (float32, bfloat16 or
+    float16), out float32 [M, N]."""
     M, K = A.shape
     N = W.shape[0]
-    dt = LLAMA_BF16 if A.dtype.__str__() == "torch.bfloat16" else LLAMA_F32
-    ws = workspace if workspace is not None else (op_linear_workspace(A.device) if dt == LLAMA_BF16 else None)
+    dt = _dtype_code(A, "A")
+    _check_linear_operands(A, W, out)
+    ws = workspace if workspace is not None else (op_linear_workspace(A.device) if dt != LLAMA_F32 else None)
     _check(_lib.llama_op_linear(A.data_ptr(), W.data_ptr(), M, N, K, dt, out.data_ptr(), _ptr(ws),
                                 0 if ws is None else ws.numel(), _stream(stream)))
     return out

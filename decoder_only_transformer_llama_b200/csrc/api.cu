@@ -619,24 +619,24 @@ int llama_op_linear(const void* A, const void* W, int M, int N, int K, int dtype
     ep.ldo = N;
     if (dtype == LLAMA_F32)
         return linear_f32(static_cast<const float*>(A), static_cast<const float*>(W), M, N, K, ep, st);
-    if (dtype != LLAMA_BF16) { set_error("bad dtype"); return LLAMA_ERR_INVALID_ARG; }
-    if (K % 8) { set_error("bf16 linear needs K %% 8 == 0"); return LLAMA_ERR_INVALID_ARG; }
+    if (dtype != LLAMA_BF16 && dtype != LLAMA_F16) { set_error("bad dtype"); return LLAMA_ERR_INVALID_ARG; }
+    if (K % 8) { set_error("16-bit linear needs K %% 8 == 0"); return LLAMA_ERR_INVALID_ARG; }
     if ((N + 127) / 128 > kMaxTiles) { set_error("N too large"); return LLAMA_ERR_INVALID_ARG; }
     if ((M <= 64 || workspace) && (!workspace || workspace_bytes < llama_op_linear_workspace_bytes() ||
                                    (reinterpret_cast<uintptr_t>(workspace) & 255))) {
-        set_error("bf16 linear needs a 256-byte aligned workspace of llama_op_linear_workspace_bytes() "
+        set_error("16-bit linear needs a 256-byte aligned workspace of llama_op_linear_workspace_bytes() "
                   "(optional only for M > 64)");
         return LLAMA_ERR_INVALID_ARG;
     }
     if (M == 0) return LLAMA_OK;
     TmaMaps ma, mw;
-    LLB_TRY(encode_kmajor_16(&ma.a128, A, M, K, 128));
-    LLB_TRY(encode_kmajor_16(&ma.b, A, M, K, 16));
-    LLB_TRY(encode_kmajor_16(&mw.a128, W, N, K, 128));
-    LLB_TRY(encode_kmajor_16(&mw.b, W, N, K, 256));
+    LLB_TRY(encode_kmajor_16(&ma.a128, A, M, K, 128, dtype));
+    LLB_TRY(encode_kmajor_16(&ma.b, A, M, K, 16, dtype));
+    LLB_TRY(encode_kmajor_16(&mw.a128, W, N, K, 128, dtype));
+    LLB_TRY(encode_kmajor_16(&mw.b, W, N, K, 256, dtype));
     float* part = static_cast<float*>(workspace);
     int* cnt = workspace ? reinterpret_cast<int*>(static_cast<char*>(workspace) + kGemmPartBytes) : nullptr;
-    return linear16(&ma, &mw, M, N, K, LLAMA_BF16, ep, part, part ? kGemmPartBytes : 0, cnt, st);
+    return linear16(&ma, &mw, M, N, K, dtype, ep, part, part ? kGemmPartBytes : 0, cnt, st);
 }
 
 }  // extern "C"

@@ -21,24 +21,26 @@ extern "C" {
 
 /* RMSNorm of M rows: out[m,:] = x[m,:] / sqrt(mean(x[m,:]^2) + eps) * w
  * (Admin Guide §8.4, RMSNorm), fp32 arithmetic.
- *   x fp32 [M, dim]; w fp32 [dim]; out [M, dim] in out_dtype (LLAMA_F32 or
- *   LLAMA_BF16, rounded once).  dim % 4 == 0. */
+ *   x fp32 [M, dim]; w fp32 [dim]; out [M, dim] in out_dtype (LLAMA_F32,
+ *   LLAMA_BF16 or LLAMA_F16, rounded once).  dim % 4 == 0. */
 LLAMA_API int llama_op_rmsnorm(const float* x, const float* w, int M, int dim, float eps,
                      void* out, int out_dtype, void* stream);
 
 /* Dense projection out[m,n] = sum_k A[m,k] * W[n,k]  (nn.Linear, y = x W^T).
  *   A [M, K] and W [N, K] in `dtype` (LLAMA_F32: SIMT fp32 FMA, no TF32;
- *   LLAMA_BF16: tcgen05 tensor cores with fp32 accumulation in TMEM);
- *   out fp32 [M, N] (row-major, overwritten).  K % 8 == 0 for bf16.
- * The bf16 kernels are the ones the model path uses: for M <= 64 the
+ *   LLAMA_BF16 or LLAMA_F16: tcgen05 tensor cores, both operands of that
+ *   type, fp32 accumulation in TMEM); out fp32 [M, N] (row-major,
+ *   overwritten).  K % 8 == 0 for the 16-bit types; any other dtype code is
+ *   LLAMA_ERR_INVALID_ARG.
+ * The 16-bit kernels are the ones the model path uses: for M <= 64 the
  * persistent weight-streaming kernel (the weight is the 128-row MMA operand,
  * K split across CTAs), else the persistent 128 x 256-tile kernel.
  *   workspace  device scratch of llama_op_linear_workspace_bytes(), 256-byte
  *              aligned, zero-filled before its first use (the kernels leave
- *              their counters at zero again).  Required for bf16 with
- *              M <= 64.  Optional for M > 64: with it the last wave of tiles
- *              is split along K over all SMs (stream-K), with NULL every tile
- *              runs whole.  A non-NULL workspace that is too small or
+ *              their counters at zero again).  Required for the 16-bit
+ *              types with M <= 64.  Optional for M > 64: with it the last
+ *              wave of tiles is split along K over all SMs (stream-K), with
+ *              NULL every tile runs whole.  A non-NULL workspace that is too small or
  *              misaligned is rejected (LLAMA_ERR_INVALID_ARG).  Calls sharing
  *              a workspace must not overlap on the device. */
 LLAMA_API size_t llama_op_linear_workspace_bytes(void);

@@ -108,6 +108,40 @@ def test_calls_reject_null_model_and_bad_sizes():
     assert lib.llama_op_linear(0x1000, 0x1000, 1, 1, 7, 1, 0x1000, None, 0, None) == llb.LLAMA_ERR_INVALID_ARG  # K % 8
     # decode-shaped bf16 needs the scratch workspace
     assert lib.llama_op_linear(0x1000, 0x1000, 4, 128, 64, 1, 0x1000, None, 0, None) == llb.LLAMA_ERR_INVALID_ARG
+    # fp16 takes the same rules; an unknown dtype code is rejected
+    assert lib.llama_op_linear(0x1000, 0x1000, 1, 1, 7, llb.LLAMA_F16, 0x1000, None, 0, None) == llb.LLAMA_ERR_INVALID_ARG
+    assert lib.llama_op_linear(0x1000, 0x1000, 4, 128, 64, llb.LLAMA_F16, 0x1000, None, 0, None) == llb.LLAMA_ERR_INVALID_ARG
+    assert lib.llama_op_linear(0x1000, 0x1000, 4, 128, 64, 7, 0x1000, None, 0, None) == llb.LLAMA_ERR_INVALID_ARG
     assert lib.llama_op_linear_workspace_bytes() > 0
     assert lib.llama_op_rmsnorm(0x1000, 0x1000, 1, 6, 1e-5, 0x1000, 0, None) == llb.LLAMA_ERR_INVALID_ARG
     assert lib.llama_get_kv(None, 0, None, None, None) == llb.LLAMA_ERR_INVALID_ARG
+
+
+def test_op_bindings_reject_mismatched_tensors():
+    """The Python op wrappers check dtypes and shapes before the C call: a
+    float16 operand never reaches the fp32 kernel, and mixed operand types,
+    a non-fp32 output or an unsupported type raise ValueError."""
+    import torch
+    A16 = torch.zeros(4, 64, dtype=torch.float16)
+    W16 = torch.zeros(128, 64, dtype=torch.float16)
+    Wb = torch.zeros(128, 64, dtype=torch.bfloat16)
+    out = torch.zeros(4, 128)
+    with pytest.raises(ValueError):
+        llb.op_linear(A16, Wb, out)                                   # mixed 16-bit types
+    with pytest.raises(ValueError):
+        llb.op_linear(A16, W16, torch.zeros(4, 128, dtype=torch.float16))   # output not fp32
+    with pytest.raises(ValueError):
+        llb.op_linear(A16, W16, torch.zeros(4, 127))                  # output shape
+    with pytest.raises(ValueError):
+        llb.op_linear(A16.to(torch.float64), W16.to(torch.float64), out)
+    with pytest.raises(ValueError):
+        llb.op_linear(A16, W16.t().contiguous().t(), out)             # W not contiguous
+    with pytest.raises(ValueError):
+        llb.op_linear_noalloc(A16, W16, out)                          # bf16 only
+    with pytest.raises(ValueError):
+        llb.op_linear_whole_tiles(torch.zeros(80, 64), torch.zeros(128, 64), torch.zeros(80, 128))
+    x = torch.zeros(2, 64)
+    with pytest.raises(ValueError):
+        llb.op_rmsnorm(x, torch.zeros(64), 1e-5, torch.zeros(2, 64, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        llb.op_rmsnorm(x.to(torch.bfloat16), torch.zeros(64), 1e-5, torch.zeros(2, 64))

@@ -40,6 +40,11 @@ def test_rmsnorm_kernel(llb, M, dim):
     torch.cuda.synchronize()
     got = out16.cpu().double().numpy()
     assert np.all(np.abs(got - want) <= np.abs(want) * 2.0 ** -8 + 1e-6)
+    outh = torch.empty(M, dim, device="cuda", dtype=torch.float16)
+    llb.op_rmsnorm(x.cuda(), w.cuda(), 1e-5, outh)
+    torch.cuda.synchronize()
+    got = outh.cpu().double().numpy()
+    assert np.all(np.abs(got - want) <= np.abs(want) * 2.0 ** -11 + 1e-6)
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 384, 256), (70, 1000, 768), (130, 130, 64), (2, 2048, 96)])
@@ -58,12 +63,14 @@ def test_linear_f32_kernel(llb, M, N, K):
     (1, 256, 256), (7, 1000, 4096), (16, 4096, 256), (17, 384, 4160), (33, 512, 200), (64, 12288, 4096),
     (48, 640, 512),
     (65, 256, 256), (128, 1000, 4096), (300, 768, 1024), (2048, 512, 64)])
-def test_linear_bf16_tcgen05_kernel(llb, M, N, K):
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
+def test_linear_16bit_tcgen05_kernel(llb, M, N, K, dt):
     """tcgen05 GEMM in both orientations (M <= 64: weights as the 128-row
-    operand; else activations), with ragged M, N and K tails."""
+    operand; else activations), with ragged M, N and K tails, for both
+    16-bit operand types."""
     g = torch.Generator().manual_seed(7 * M + N + K)
-    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
-    W = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    A = torch.randn(M, K, generator=g).to(dt)
+    W = (torch.randn(N, K, generator=g) * 0.05).to(dt)
     out = torch.full((M, N), float("nan"), device="cuda")
     llb.op_linear(A.cuda(), W.cuda(), out)
     torch.cuda.synchronize()
