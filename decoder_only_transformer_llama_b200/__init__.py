@@ -153,6 +153,23 @@ def model_bytes(args: ModelArgs) -> dict:
     return {"weights": w.value, "kv": kv.value, "workspace": ws.value, "total": tot.value, "hidden": h.value}
 
 
+def _dev(t, dtype: str, numel: int, name: str, device=None):
+    """A tensor handed to a kernel: on a CUDA device (`device` if given),
+    of torch dtype `dtype` (e.g. "int32"), contiguous, with at least `numel`
+    elements.  Raises ValueError instead of passing a pointer a kernel would
+    read out of bounds or from host memory."""
+    if not getattr(t, "is_cuda", False):
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the model on {device}")
+    if str(t.dtype) != "torch." + dtype:
+        raise ValueError(f"{name} must be {dtype}, not {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() < numel:
+        raise ValueError(f"{name} has {t.numel()} elements, needs {numel}")
+
+
 class Model:
     """A model laid out in one torch-allocated device arena."""
 
@@ -179,8 +196,24 @@ class Model:
 
     def set_weight(self, layer: int, name: str, tensor, stream=None):
         t = tensor.contiguous()
+        _dev(t, self._weight_dtype(name), self._weight_numel(name), name, self.arena.device)
         _check(_lib.llama_set_weight(self.handle, layer, WEIGHT_IDS[name], t.data_ptr(), _stream(stream)))
         return t  # keep alive until the stream passes the copy
+
+    def _weight_dtype(self, name: str) -> str:
+        if name in ("norm", "attention_norm", "ffn_norm"):
+            return "float32"
+        return {LLAMA_BF16: "bfloat16", LLAMA_F16: "float16"}.get(self.args.dtype, "float32")
+
+    def _weight_numel(self, name: str) -> int:
+        a = self.args
+        hd = a.dim // a.n_heads
+        nkv = a.n_kv_heads or a.n_heads
+        H = self.sizes["hidden"]
+        return {"tok_embeddings": a.vocab_size * a.dim, "output": a.vocab_size * a.dim, "norm": a.dim,
+                "attention_norm": a.dim, "ffn_norm": a.dim, "wq": a.n_heads * hd * a.dim,
+                "wk": nkv * hd * a.dim, "wv": nkv * hd * a.dim, "wo": a.dim * a.n_heads * hd,
+                "w1": H * a.dim, "w2": a.dim * H, "w3": H * a.dim}[name]
 
     def load(self, weights: dict, stream=None):
         """Upload a weight dict in the workloads layout (torch tensors on the device)."""
@@ -223,9 +256,16 @@ class Model:
     def prefill(self, tokens, lens: Optional[Sequence[int]] = None, start_pos: int = 0, logits=None,
                 all_logits: bool = False, stream=None):
         B, T = tokens.shape
+        dev = self.arena.device
+        _dev(tokens, "int32", B * T, "tokens", dev)
         lens_arr = None
         if lens is not None:
+            if len(lens) != B:
+                raise ValueError(f"lens has {len(lens)} entries for {B} rows")
             lens_arr = (ctypes.c_int32 * B)(*[int(v) for v in lens])
+        if logits is not None:
+            rows = (sum(int(v) for v in lens) if lens is not None else B * T) if all_logits else B
+            _dev(logits, "float32", rows * self.args.vocab_size, "logits", dev)
         _check(_lib.llama_prefill(self.handle, tokens.data_ptr(), lens_arr, B, T, start_pos, _ptr(logits),
                                   1 if all_logits else 0, _stream(stream)))
         return logits
@@ -233,6 +273,15 @@ class Model:
     def decode_step(self, tokens, pos, temperature: Optional[float] = None, top_p: float = 0.9,
                     uniforms=None, next_tokens=None, logits=None, advance: bool = False, stream=None):
         B = tokens.shape[0]
+        dev = self.arena.device
+        _dev(tokens, "int32", B, "tokens", dev)
+        _dev(pos, "int32", B, "pos", dev)
+        if uniforms is not None:
+            _dev(uniforms, "float32", B, "uniforms", dev)
+        if next_tokens is not None:
+            _dev(next_tokens, "int32", B, "next_tokens", dev)
+        if logits is not None:
+            _dev(logits, "float32", B * self.args.vocab_size, "logits", dev)
         samp = None
         if temperature is not None:
             samp = Sampling(float(temperature), float(top_p))
@@ -264,6 +313,10 @@ class Model:
 
 def sample(logits, temperature: float, top_p: float, uniforms, out, stream=None):
     B, V = logits.shape
+    _dev(logits, "float32", B * V, "logits")
+    _dev(out, "int32", B, "out", logits.device)
+    if uniforms is not None:
+        _dev(uniforms, "float32", B, "uniforms", logits.device)
     _check(_lib.llama_sample(logits.data_ptr(), B, V, float(temperature), float(top_p), _ptr(uniforms),
                              out.data_ptr(), _stream(stream)))
     return out
@@ -272,6 +325,9 @@ def sample(logits, temperature: float, top_p: float, uniforms, out, stream=None)
 def token_logprobs(logits, tokens, out, stream=None):
     """out[i] = log_softmax(logits[i])[tokens[i]] (fp32 logits [N, V], int32 tokens [N])."""
     N, V = logits.shape
+    _dev(logits, "float32", N * V, "logits")
+    _dev(tokens, "int32", N, "tokens", logits.device)
+    _dev(out, "float32", N, "out", logits.device)
     _check(_lib.llama_token_logprobs(logits.data_ptr(), tokens.data_ptr(), N, V, out.data_ptr(), _stream(stream)))
     return out
 

@@ -145,3 +145,97 @@ def test_op_bindings_reject_mismatched_tensors():
         llb.op_rmsnorm(x, torch.zeros(64), 1e-5, torch.zeros(2, 64, dtype=torch.int32))
     with pytest.raises(ValueError):
         llb.op_rmsnorm(x.to(torch.bfloat16), torch.zeros(64), 1e-5, torch.zeros(2, 64))
+
+
+class _FakeCudaTensor:
+    """Stands in for a CUDA tensor on a machine without one: the binding's
+    checks read its device, dtype, contiguity and size; asking for its
+    address means a call got past them to the library."""
+    is_cuda = True
+
+    def __init__(self, shape, dtype, contiguous=True, device="cuda:0"):
+        import torch
+        self.shape = tuple(shape)
+        self.dtype = dtype
+        self.device = torch.device(device)
+        self._contiguous = contiguous
+
+    def is_contiguous(self):
+        return self._contiguous
+
+    def contiguous(self):
+        return self
+
+    def numel(self):
+        n = 1
+        for d in self.shape:
+            n *= d
+        return n
+
+    def data_ptr(self):
+        raise RuntimeError("reached the library")
+
+
+def _fake_model(dtype="bf16"):
+    import torch
+    m = object.__new__(llb.Model)
+    m.args = llb.make_args(256, 2, 8, 2, 512, max_seq_len=64, max_batch_size=4, dtype=dtype)
+    m.sizes = llb.model_bytes(m.args)
+    m.arena = _FakeCudaTensor((m.sizes["total"],), torch.uint8)
+    m.handle = None
+    return m
+
+
+def test_kernel_wrappers_refuse_host_mistyped_and_short_tensors():
+    """Every wrapper that hands a kernel a pointer checks the tensor first:
+    a host tensor, a wrong dtype, a non-contiguous view, a buffer shorter
+    than the call writes, or a tensor on another GPU raises ValueError; a
+    well-formed call passes the checks (and here reaches the stub)."""
+    import torch
+    F = _FakeCudaTensor
+    V = 512
+    with pytest.raises(ValueError):
+        llb.sample(torch.zeros(2, V), 0.0, 0.9, None, torch.zeros(2, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        llb.token_logprobs(torch.zeros(3, V), torch.zeros(3, dtype=torch.int32), torch.zeros(3))
+    with pytest.raises(ValueError):
+        llb.sample(F((2, V), torch.float32), 0.0, 0.9, None, F((1,), torch.int32))       # out too short
+    with pytest.raises(RuntimeError, match="reached the library"):
+        llb.sample(F((2, V), torch.float32), 0.7, 0.9, F((2,), torch.float32), F((2,), torch.int32))
+
+    m = _fake_model()
+    tok = F((2, 5), torch.int32)
+    with pytest.raises(ValueError):
+        m.prefill(F((2, 5), torch.int64))                                               # token dtype
+    with pytest.raises(ValueError):
+        m.prefill(tok, lens=[3])                                                         # one len per row
+    with pytest.raises(ValueError):
+        m.prefill(tok, logits=F((2, V - 1), torch.float32))                              # last-token logits
+    with pytest.raises(ValueError):
+        m.prefill(tok, lens=[5, 4], logits=F((8, V), torch.float32), all_logits=True)    # 9 rows needed
+    with pytest.raises(ValueError):
+        m.prefill(F((2, 5), torch.int32, device="cuda:1"))                               # other GPU
+    with pytest.raises(RuntimeError, match="reached the library"):
+        m.prefill(tok, lens=[5, 4], logits=F((9, V), torch.float32), all_logits=True)
+
+    t1, p1 = F((2,), torch.int32), F((2,), torch.int32)
+    with pytest.raises(ValueError):
+        m.decode_step(t1, F((2,), torch.int64))                                          # positions int32
+    with pytest.raises(ValueError):
+        m.decode_step(t1, p1, temperature=0.0, next_tokens=F((2,), torch.int32, contiguous=False))
+    with pytest.raises(ValueError):
+        m.decode_step(t1, p1, temperature=0.7, uniforms=F((2,), torch.float64), next_tokens=t1)
+    with pytest.raises(ValueError):
+        m.decode_step(t1, p1, logits=F((1, V), torch.float32))
+    with pytest.raises(RuntimeError, match="reached the library"):
+        m.decode_step(t1, p1, temperature=0.7, uniforms=F((2,), torch.float32), next_tokens=t1,
+                      logits=F((2, V), torch.float32))
+
+    with pytest.raises(ValueError):
+        m.set_weight(-1, "norm", F((256,), torch.bfloat16))                              # norms are fp32
+    with pytest.raises(ValueError):
+        m.set_weight(0, "wq", F((256, 255), torch.bfloat16))                             # short matrix
+    with pytest.raises(ValueError):
+        _fake_model("f16").set_weight(0, "wk", F((64, 256), torch.bfloat16))             # model is fp16
+    with pytest.raises(RuntimeError, match="reached the library"):
+        m.set_weight(0, "w2", F((256, m.sizes["hidden"]), torch.bfloat16))
