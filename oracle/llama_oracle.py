@@ -27,6 +27,11 @@ in the design notes):
     ascending; a token is kept iff the mass strictly before it is <= top_p;
     the draw is the inverse CDF of the renormalised kept mass at the given
     uniform u (the multinomial draw made deterministic).
+  * 16-bit storage (optional, `store=`): the reference holds its tensors in
+    fp16 (Admin Guide §1.4, §6.4; RMSNorm normalises in fp32 and casts back,
+    §8.4).  The oracle can round to bfloat16 or binary16 where a 16-bit run
+    stores activations, leaving every sum exact; this measures the error that
+    storage alone causes and is never the parity reference itself.
 
 Weights are passed as a mapping:
   w["tok_embeddings"] [V, dim], w["norm"] [dim], w["output"] [V, dim],
@@ -45,6 +50,31 @@ import numpy as np
 
 def _f64(a) -> np.ndarray:
     return np.asarray(a, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# 16-bit storage (an error model, used only when a caller asks for it)
+# ---------------------------------------------------------------------------
+
+def round_bf16(a) -> np.ndarray:
+    """Round to the nearest bfloat16 value, ties to even, returned as fp64.
+
+    bfloat16 is the upper half of an IEEE binary32 (sign, 8 exponent bits,
+    7 fraction bits).  The value is first rounded to binary32 (as an fp32
+    accumulator holds it), then the low 16 bits of that word are rounded off:
+    add 0x7FFF plus the lowest kept bit, and clear them.  Finite inputs only.
+    """
+    f = np.ascontiguousarray(a, dtype=np.float32)
+    u = f.view(np.uint32)
+    u = (u + (np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1)))) & np.uint32(0xFFFF0000)
+    return u.view(np.float32).astype(np.float64)
+
+
+def round_f16(a) -> np.ndarray:
+    """Round to the nearest IEEE binary16 value (the reference's own storage
+    type, Admin Guide §1.4 and §6.4), ties to even, returned as fp64; the
+    value passes through binary32 first, as above."""
+    return np.ascontiguousarray(a, dtype=np.float32).astype(np.float16).astype(np.float64)
 
 
 # ---------------------------------------------------------------------------
@@ -154,13 +184,14 @@ def causal_mask(seqlen: int, start_pos: int) -> np.ndarray:
     return m
 
 
-def attention(q, keys, values, start_pos: int, n_rep: int) -> np.ndarray:
+def attention(q, keys, values, start_pos: int, n_rep: int, store=None) -> np.ndarray:
     """softmax(Q K^T / sqrt(head_dim) + mask) V for each query head.
 
     q: [T, n_heads, hd] (already rotated); keys/values: [start_pos+T, n_kv_heads, hd]
     (the whole cache prefix, already holding this call's keys).  Query head h
     reads KV head h // n_rep (repeat_kv; source tour, "One model.py").
-    Admin Guide §8.4, Attention forward steps 5-7.
+    Admin Guide §8.4, Attention forward steps 5-7.  `store` (see
+    layer_forward) rounds the probabilities before they multiply V.
     """
     q, keys, values = _f64(q), _f64(keys), _f64(values)
     T, nh, hd = q.shape
@@ -169,7 +200,10 @@ def attention(q, keys, values, start_pos: int, n_rep: int) -> np.ndarray:
     for h in range(nh):
         g = h // n_rep
         scores = q[:, h, :] @ keys[:, g, :].T / math.sqrt(hd) + mask
-        out[:, h, :] = softmax(scores, axis=-1) @ values[:, g, :]
+        p = softmax(scores, axis=-1)
+        if store is not None:
+            p = store(p)
+        out[:, h, :] = p @ values[:, g, :]
     return out
 
 
@@ -179,10 +213,14 @@ def silu(z) -> np.ndarray:
     return z / (1.0 + np.exp(-z))
 
 
-def feed_forward(x, w1, w2, w3) -> np.ndarray:
-    """SwiGLU: w2(silu(w1 x) * w3 x)  (Admin Guide §8.4, FeedForward)."""
+def feed_forward(x, w1, w2, w3, store=None) -> np.ndarray:
+    """SwiGLU: w2(silu(w1 x) * w3 x)  (Admin Guide §8.4, FeedForward).
+    `store` (see layer_forward) rounds the gated product before w2."""
     x = _f64(x)
-    return (silu(x @ _f64(w1).T) * (x @ _f64(w3).T)) @ _f64(w2).T
+    g = silu(x @ _f64(w1).T) * (x @ _f64(w3).T)
+    if store is not None:
+        g = store(g)
+    return g @ _f64(w2).T
 
 
 # ---------------------------------------------------------------------------
@@ -223,53 +261,65 @@ def new_cache(args: Args) -> KVCache:
     return KVCache(args.n_layers, args.max_seq_len, args.n_kv_heads, args.head_dim)
 
 
-def layer_forward(args: Args, lw, x, cache: KVCache, layer: int, start_pos: int) -> np.ndarray:
+def layer_forward(args: Args, lw, x, cache: KVCache, layer: int, start_pos: int, store=None) -> np.ndarray:
     """One pre-norm TransformerBlock on the T new tokens of one row.
 
     h = x + attention(attention_norm(x)); out = h + feed_forward(ffn_norm(h))
     (Admin Guide §8.4, TransformerBlock).  The attention writes this call's
     keys and values into cache rows start_pos .. start_pos+T-1 and reads rows
     0 .. start_pos+T-1 (Admin Guide §8.4, Attention forward steps 1-8).
+
+    store: None for the exact fp64 definition.  Otherwise a rounding function
+    (round_bf16, round_f16) applied where a 16-bit run holds its activations
+    in the 16-bit type: the normalised inputs of the projections, q, k and v
+    after RoPE (so the cache holds 16-bit values), the attention
+    probabilities and output, and the SwiGLU product; the residual stream and
+    every sum stay exact.  It gives the error that 16-bit storage alone
+    causes, which the parity bounds at full model depth are derived from.
     """
     x = _f64(x)
     T = x.shape[0]
     nh, nkv, hd = args.n_heads, args.n_kv_heads, args.head_dim
+    keep = store if store is not None else (lambda a: a)
     pos = start_pos + np.arange(T)
-    y = rms_norm(x, lw["attention_norm"], args.norm_eps)
+    y = keep(rms_norm(x, lw["attention_norm"], args.norm_eps))
     q = (y @ _f64(lw["wq"]).T).reshape(T, nh, hd)
     k = (y @ _f64(lw["wk"]).T).reshape(T, nkv, hd)
-    v = (y @ _f64(lw["wv"]).T).reshape(T, nkv, hd)
-    q = apply_rope(q, pos, args.rope_theta)
-    k = apply_rope(k, pos, args.rope_theta)
+    v = keep((y @ _f64(lw["wv"]).T).reshape(T, nkv, hd))
+    q = keep(apply_rope(q, pos, args.rope_theta))
+    k = keep(apply_rope(k, pos, args.rope_theta))
     cache.k[layer][start_pos:start_pos + T] = k
     cache.v[layer][start_pos:start_pos + T] = v
     keys = cache.k[layer][:start_pos + T]
     values = cache.v[layer][:start_pos + T]
-    o = attention(q, keys, values, start_pos, args.n_rep).reshape(T, nh * hd)
+    o = keep(attention(q, keys, values, start_pos, args.n_rep, store).reshape(T, nh * hd))
     h = x + o @ _f64(lw["wo"]).T
-    f = rms_norm(h, lw["ffn_norm"], args.norm_eps)
-    return h + feed_forward(f, lw["w1"], lw["w2"], lw["w3"])
+    f = keep(rms_norm(h, lw["ffn_norm"], args.norm_eps))
+    return h + feed_forward(f, lw["w1"], lw["w2"], lw["w3"], store)
 
 
 def forward(args: Args, w, tokens: Sequence[int], start_pos: int, cache: KVCache,
-            n_layers: Optional[int] = None, logits_positions: Optional[Sequence[int]] = None
-            ) -> np.ndarray:
+            n_layers: Optional[int] = None, logits_positions: Optional[Sequence[int]] = None,
+            store=None) -> np.ndarray:
     """Transformer.forward(tokens, start_pos) for one batch row.
 
     Embedding lookup, the blocks, the final RMSNorm, the output projection;
     returns fp64 logits [T, V] for every new position (or only for the
     positions listed in `logits_positions`, indices into this call's tokens).
-    Admin Guide §8.4 ("The forward pass", steps 1-6).
+    Admin Guide §8.4 ("The forward pass", steps 1-6).  `store`: see
+    layer_forward (it also rounds the final normalised rows).
     """
     toks = np.asarray(tokens, dtype=np.int64)
     x = _f64(w["tok_embeddings"][toks])
     layers = w["layers"]
     L = args.n_layers if n_layers is None else n_layers
     for l in range(L):
-        x = layer_forward(args, layers[l], x, cache, l, start_pos)
+        x = layer_forward(args, layers[l], x, cache, l, start_pos, store)
     if logits_positions is not None:
         x = x[np.asarray(logits_positions, dtype=np.int64)]
     h = rms_norm(x, w["norm"], args.norm_eps)
+    if store is not None:
+        h = store(h)
     return h @ _f64(w["output"]).T
 
 

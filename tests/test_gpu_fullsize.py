@@ -1,9 +1,12 @@
 """Parity at the workloads' full layer dimensions (7B, 13B with ragged
 prompts, 70B GQA slice), with the model truncated to two layers so that the
-fp64 oracle can recompute sampled rows in seconds.  The GPU runs the same
+fp64 oracle can recompute sampled rows in seconds, and the full 32-layer 7B
+model on one sampled row.  The GPU runs the same
 launch configuration as the benchmark (batched prefill, then batched decode
 steps at per-row positions); the oracle recomputes one or two rows from
 scratch, teacher-forced on the GPU's greedy tokens."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -23,7 +26,7 @@ def llb(cuda_device):
     return m
 
 
-def _run(llb, shape, B, T, lens, steps, rows, seed_idx, start_pos=0):
+def _run(llb, shape, B, T, lens, steps, rows, seed_idx, start_pos=0, tol=BF16_TOL, gap=1e-2):
     s = shape
     w = make_weights(s, weight_seed(seed_idx), device="cuda")
     m = build_model(s, w)
@@ -54,8 +57,9 @@ def _run(llb, shape, B, T, lens, steps, rows, seed_idx, start_pos=0):
         positions = list(range(L - 1, L + steps))
         want = O.forward(args, lw, seqs[b], 0, O.new_cache(args), logits_positions=positions)
         err = rel_l2(np.stack(got[b]), want)
-        assert err <= BF16_TOL, (b, err)
-        check_greedy(seqs[b][L:], want[:steps])
+        print(f"{s.n_layers} layers, dim {s.dim}, {s.dtype}: row {b} rel-L2 {err:.3e} (bound {tol:.3e})")
+        assert err <= tol, (b, err)
+        check_greedy(seqs[b][L:], want[:steps], gap)
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f16"])
@@ -65,6 +69,37 @@ def test_7b_dims_prefill_4x512_then_decode(llb, dtype):
     the reference's own fp16."""
     s = L7B.replace(n_layers=2, dtype=dtype)
     _run(llb, s, B=4, T=512, lens=[512] * 4, steps=3, rows=[0, 3], seed_idx=2)
+
+
+def _storage_error_7b():
+    """Per-row figures of tests/golden/storage_error_7b.txt (written by
+    make_storage_error.py from the oracle alone)."""
+    rows = []
+    with open(os.path.join(os.path.dirname(__file__), "golden", "storage_error_7b.txt")) as f:
+        for line in f:
+            if line.startswith("row"):
+                kv = dict(item.split("=") for item in line.split(":", 1)[1].split())
+                rows.append({k: float(v) for k, v in kv.items()})
+    assert len(rows) == 4
+    return rows
+
+
+def test_7b_full_depth_benchmark_configuration(llb):
+    """The whole 32-layer 7B model in the benchmark's launch configuration
+    (4 x 512 prefill, then batched decode steps); the oracle recomputes row 2
+    (514 tokens through 32 layers, about a minute on the host).
+
+    Over 32 layers the rounding of bfloat16 activation storage compounds
+    past the 2e-2 that holds at two layers: the oracle with bf16 storage
+    (round_bf16 at its storage points) is 4.3e-2 to 4.6e-2 from the exact
+    oracle at this depth, on each of the batch's four rows.  The bounds are therefore that storage error's, from
+    tests/golden/storage_error_7b.txt: relative L2 within 1.5 x the largest
+    per-row figure, and greedy ids identical wherever the oracle's top-2 gap
+    exceeds 8 x the largest RMS element-wise difference."""
+    err = _storage_error_7b()
+    tol = 1.5 * max(r["rel_l2"] for r in err)
+    gap = 8.0 * max(r["rms_abs"] for r in err)
+    _run(llb, L7B, B=4, T=512, lens=[512] * 4, steps=2, rows=[2], seed_idx=5, tol=tol, gap=gap)
 
 
 def test_13b_dims_ragged_prefill_then_decode(llb):

@@ -458,3 +458,85 @@ def test_sample_margins_flags_boundary_draws_only():
     assert O.sample_margins(l2, 1.0, 1.0, 0.25) > 0.2
     # but a draw that lands on such a token is flagged
     assert O.sample_margins(l2, 1.0, 1.0, 0.9999999999999) < 1e-9
+
+
+# --------------------------------------------------------------------------- 16-bit storage error model
+
+def test_round_bf16_closed_forms():
+    """bfloat16 keeps 8 significant bits: 1 + 2^-7 is exact, 1 + 2^-8 lies
+    halfway between 1 and 1 + 2^-7 and goes to the even neighbour 1, and
+    1 + 3*2^-8 lies halfway between 1 + 2^-7 and 1 + 2^-6 and goes to the
+    even 1 + 2^-6.  Catches truncation instead of rounding, ties away from
+    zero, and a wrong count of kept bits."""
+    x = np.array([1.0, 1 + 2 ** -7, 1 + 2 ** -8, 1 + 3 * 2 ** -8, 1 + 2 ** -8 + 2 ** -20, 3 - 2 ** -9, 0.0])
+    want = np.array([1.0, 1 + 2 ** -7, 1.0, 1 + 2 ** -6, 1 + 2 ** -7, 3.0, 0.0])
+    np.testing.assert_array_equal(O.round_bf16(x), want)
+    np.testing.assert_array_equal(O.round_bf16(-x), -want)
+    np.testing.assert_array_equal(O.round_bf16(x * 2.0 ** 40), want * 2.0 ** 40)   # exponent untouched
+
+
+def test_round_bf16_bounds_and_idempotence():
+    """Half-ulp bound |r(x) - x| <= 2^-8 |x| for normal x, the low 16 bits of
+    every result's binary32 word are zero, and r(r(x)) = r(x)."""
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal(20000) * np.exp(rng.uniform(-20, 20, 20000))
+    r = O.round_bf16(x)
+    assert np.all(np.abs(r - x) <= 2.0 ** -8 * np.abs(x) * (1 + 1e-7))
+    assert np.all((r.astype(np.float32).view(np.uint32) & 0xFFFF) == 0)
+    np.testing.assert_array_equal(O.round_bf16(r), r)
+
+
+def test_round_f16_closed_forms():
+    """binary16 keeps 11 significant bits: ties at 1 + 2^-11 and 1 + 3*2^-11
+    go to the even neighbours 1 and 1 + 2^-9; 65504 is the largest finite."""
+    x = np.array([1.0, 1 + 2 ** -10, 1 + 2 ** -11, 1 + 3 * 2 ** -11, 65504.0, -0.5])
+    want = np.array([1.0, 1 + 2 ** -10, 1.0, 1 + 2 ** -9, 65504.0, -0.5])
+    np.testing.assert_array_equal(O.round_f16(x), want)
+
+
+def test_storage_hook_identity_is_the_exact_forward():
+    """With an identity `store` the forward is bit-identical to the plain
+    definition: the hook adds no arithmetic of its own."""
+    args = _tiny_args()
+    w = _rand_weights(args, seed=21)
+    toks = [3, 1, 4, 1, 5, 9, 2, 6]
+    a = O.forward(args, w, toks, 0, O.new_cache(args))
+    b = O.forward(args, w, toks, 0, O.new_cache(args), store=lambda v: np.array(v, dtype=np.float64))
+    np.testing.assert_array_equal(a, b)
+
+
+def test_storage_hook_rounds_the_cache_and_stays_close():
+    """With 16-bit storage the cache holds only 16-bit values, the logits
+    move from the exact ones by an amount of the format's precision, and
+    bfloat16 (8 significant bits) moves them further than binary16 (11):
+    catches a hook that never reaches the cache, or one that rounds nothing
+    or everything."""
+    args = _tiny_args(dim=64, n_heads=4, n_kv_heads=2, vocab=50)
+    w = _rand_weights(args, seed=22, scale=0.1)
+    toks = [7, 3, 22, 19, 0, 31, 8, 8, 2, 11, 25, 40]
+    exact = O.forward(args, w, toks, 0, O.new_cache(args))
+    errs = {}
+    for name, fn in (("bf16", O.round_bf16), ("f16", O.round_f16)):
+        cache = O.new_cache(args)
+        got = O.forward(args, w, toks, 0, cache, store=fn)
+        for l in range(args.n_layers):
+            for t in (cache.k[l][:len(toks)], cache.v[l][:len(toks)]):
+                np.testing.assert_array_equal(fn(t), t)
+        errs[name] = np.linalg.norm(got - exact) / np.linalg.norm(exact)
+    assert 0 < errs["f16"] < 2e-3 and 0 < errs["bf16"] < 2e-2
+    assert errs["bf16"] > 3 * errs["f16"]
+
+
+def test_storage_error_fixture_is_complete():
+    """tests/golden/storage_error_7b.txt (written by make_storage_error.py
+    from the oracle) holds one record per row of the 4-row batch, each a
+    bf16-sized error: above the two-layer figure and far below O(1)."""
+    rows = []
+    with open(os.path.join(GOLDEN, "storage_error_7b.txt")) as f:
+        for line in f:
+            if line.startswith("row"):
+                rows.append(dict(item.split("=") for item in line.split(":", 1)[1].split()))
+    assert len(rows) == 4
+    for r in rows:
+        assert 1e-2 < float(r["rel_l2"]) < 1e-1
+        assert 0 < float(r["rms_abs"]) < 0.1 * float(r["logits_rms"])
