@@ -32,6 +32,11 @@
  *     the model dtype (fp32, bf16 or fp16).
  *   - Thread safety: calls on one model must be serialised by the caller
  *     (they share the model's workspace).
+ *   - Devices: one CUDA device per process (one process per GPU).  The
+ *     first launch of each kernel sets its shared-memory attributes and
+ *     reads the SM count on the device current at that time, and later
+ *     launches reuse them; a second device in the same process is not
+ *     supported (its large-shared-memory launches fail with LLAMA_ERR_CUDA).
  */
 #ifndef LLAMA_B200_H
 #define LLAMA_B200_H
