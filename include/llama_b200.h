@@ -36,7 +36,8 @@
  *     first launch of each kernel sets its shared-memory attributes and
  *     reads the SM count on the device current at that time, and later
  *     launches reuse them; a second device in the same process is not
- *     supported (its large-shared-memory launches fail with LLAMA_ERR_CUDA).
+ *     supported (its large-shared-memory launches may fail with
+ *     LLAMA_ERR_CUDA).
  */
 #ifndef LLAMA_B200_H
 #define LLAMA_B200_H
