@@ -540,3 +540,24 @@ def test_storage_error_fixture_is_complete():
     for r in rows:
         assert 1e-2 < float(r["rel_l2"]) < 1e-1
         assert 0 < float(r["rms_abs"]) < 0.1 * float(r["logits_rms"])
+
+
+def test_storage_error_script_rows_on_a_tiny_model():
+    """make_storage_error.py's per-row routine (prefill, then one token per
+    step through the cache) on a tiny model: its exact logits equal one
+    full-sequence forward at the same positions, and its bf16-storage logits
+    differ from them by a bf16-sized amount."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("make_storage_error",
+                                                  os.path.join(GOLDEN, "make_storage_error.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    args = _tiny_args(dim=64, n_heads=4, n_kv_heads=2, vocab=50)
+    w = _rand_weights(args, seed=23, scale=0.1)
+    prompt, after = [4, 8, 15, 16, 23], [42, 7]
+    exact = mod.run_row(args, w, prompt, after, None)
+    full = O.forward(args, w, prompt + after, 0, O.new_cache(args), logits_positions=[4, 5, 6])
+    np.testing.assert_allclose(exact, full, rtol=1e-11, atol=1e-12)
+    rounded = mod.run_row(args, w, prompt, after, O.round_bf16)
+    rel = np.linalg.norm(rounded - exact) / np.linalg.norm(exact)
+    assert 1e-4 < rel < 2e-2
