@@ -207,6 +207,10 @@ static Epi base_epi(const Model* m) {
 
 static char* at(void* base, size_t off) { return static_cast<char*>(base) + off; }
 
+// Widest decode step (token rows) that runs the fused chain of
+// llama_decode_step: the weight-streaming projection's MMA N limit.
+constexpr int kFusedDecodeRows = 64;
+
 // One transformer block on M token rows held in m->x (Admin Guide §8.4,
 // TransformerBlock: h = x + attn(norm(x)); out = h + ffn(norm(h))).
 template <typename AttnFn>
@@ -464,7 +468,11 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B
     eo.mode = EPI_STORE_F32;
     eo.out = lg;
     eo.ldo = m->V;
-    if (m->dtype != LLAMA_F32) {
+    // The fused chain below needs the weight-streaming projection, whose MMA
+    // takes at most 64 token columns; wider 16-bit steps and fp32 models run
+    // one RMSNorm kernel per norm and the prefill projections instead.
+    const bool fused = m->dtype != LLAMA_F32 && B <= kFusedDecodeRows;
+    if (fused) {
         // The decode chain: five kernels per layer.  Every kernel may launch
         // before its predecessor ends (programmatic dependent launch) and waits
         // for it before reading its outputs.  RMSNorm runs inside the
@@ -516,7 +524,7 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B
         LLB_TRY(run_linear(m, m->dtype, m->ylast, &m->m_ylast, m->output, &m->m_output, B, m->V, m->dim, eo, st));
     }
     if (!sampling) return LLAMA_OK;
-    const bool pdl = m->dtype != LLAMA_F32;
+    const bool pdl = fused;
     const bool adv = (flags & LLAMA_DECODE_ADVANCE) != 0;
     int32_t* tok_adv = adv ? const_cast<int32_t*>(tokens) : nullptr;
     int32_t* pos_adv = adv ? pos : nullptr;

@@ -181,7 +181,11 @@ LLAMA_API int llama_prefill(llama_model* m, const int32_t* tokens, const int32_t
  *   flags       LLAMA_DECODE_ADVANCE: after sampling, write next_tokens and
  *               increment pos[b] on the device (for graph replay loops)
  * A row with pos[b] outside [0, max_seq_len) is skipped (its outputs are
- * unspecified) and the device status word records LLAMA_ERR_CAPACITY. */
+ * unspecified) and the device status word records LLAMA_ERR_CAPACITY.
+ * 16-bit models run steps of up to 64 rows as a fused chain (RMSNorm folded
+ * into the weight-streaming projections); wider steps (up to max_batch_size)
+ * run one RMSNorm kernel per norm and the prefill projections; both compute
+ * the same forward pass. */
 #define LLAMA_DECODE_ADVANCE 1
 LLAMA_API int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B,
                       const llama_sampling* sampling, const float* uniforms,

@@ -138,3 +138,40 @@ def test_prefix_reuse_across_prefill_calls(llb, dtype):
             want = _oracle_logits(shape, w64, seq)[P:]
             assert rel_l2(lg[b].cpu().numpy(), want) <= BF16_TOL, (T, b)
     m.close()
+
+
+def test_decode_wider_than_the_fused_chain(llb):
+    """A 16-bit decode step of more than 64 rows runs the un-fused sequence
+    (one RMSNorm kernel per norm, the 128 x 256-tile projections) instead of
+    the fused chain, whose weight-streaming projection takes at most 64 token
+    columns: 72 rows prefilled and decoded twice, sampled rows against the
+    oracle, greedy tokens written back on the device."""
+    shape = SMALL.replace(max_batch_size=72, max_seq_len=32)
+    w = make_weights(shape, 46)
+    m = build_model(shape, w)
+    B, T = 72, 6
+    toks = make_tokens(shape.vocab_size, (B, T), token_seed(16)).cuda()
+    logits = torch.empty(B, shape.vocab_size, device="cuda")
+    m.prefill(toks, logits=logits)
+    cur = torch.empty(B, dtype=torch.int32, device="cuda")
+    llb.sample(logits, 0.0, 0.9, None, cur)
+    pos = torch.full((B,), T, dtype=torch.int32, device="cuda")
+    seqs = [toks[b].cpu().tolist() for b in range(B)]
+    steps = []
+    for _ in range(2):
+        for b in range(B):
+            seqs[b].append(int(cur[b]))
+        lg = torch.empty(B, shape.vocab_size, device="cuda")
+        m.decode_step(cur, pos, temperature=0.0, next_tokens=cur, logits=lg, advance=True)
+        torch.cuda.synchronize()
+        steps.append(lg.cpu().numpy())
+    assert m.status() == 0
+    assert pos.cpu().tolist() == [T + 2] * B
+    w64 = to_numpy_f64_weights(w)
+    for b in (0, 40, 71):
+        want = _oracle_logits(shape, w64, seqs[b])[T:]
+        got = np.stack([steps[0][b], steps[1][b]])
+        assert rel_l2(got, want) <= BF16_TOL, b
+        if O.sample_margins(want[1], 0.0, 0.9, 0.0) > 1e-2:
+            assert int(cur[b]) == O.greedy(want[1]), b
+    m.close()
