@@ -39,7 +39,10 @@ EXPORTED = ("llama_model_bytes", "llama_model_create", "llama_set_weight", "llam
             "llama_prefill", "llama_decode_step", "llama_sample", "llama_model_status",
             "llama_model_destroy", "llama_last_error", "llama_launch_count",
             "llama_op_rmsnorm", "llama_op_linear", "llama_op_linear_workspace_bytes", "llama_op_linear_noalloc",
-            "llama_profile_start", "llama_profile_stop", "llama_token_logprobs")
+            "llama_profile_start", "llama_profile_stop", "llama_token_logprobs", "llama_timeline_start",
+            "llama_timeline_stop", "llama_debug_stall")
+LLAMA_STALL_NONE, LLAMA_STALL_PROJECTION, LLAMA_STALL_ATTENTION = 0, 1, 2
+TIMELINE_KINDS = {0: "embed", 1: "projection", 2: "attention", 3: "sample", 4: "rmsnorm"}
 
 
 class LlamaError(RuntimeError):
@@ -94,6 +97,10 @@ _sig("llama_op_linear", _i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp])
 _sig("llama_op_linear_workspace_bytes", _sz, [])
 _sig("llama_token_logprobs", _i, [_vp, _vp, _i, _i, _vp, _vp])
 _sig("llama_op_linear_noalloc", _i, [_vp, _vp, _i, _i, _i, _vp, _vp])
+_sig("llama_timeline_start", _i, [_vp, _vp])
+_sig("llama_timeline_stop", _i, [_vp, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_int32),
+                                 ctypes.POINTER(ctypes.c_int64), _i, ctypes.POINTER(ctypes.c_int)])
+_sig("llama_debug_stall", _i, [_vp, _i, _i, ctypes.c_int64])
 _sig("llama_profile_start", _i, [_vp, _i])
 _sig("llama_profile_stop", _i, [_vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int64),
                                 ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int32), _i,
@@ -304,6 +311,26 @@ class Model:
         n = ctypes.c_int()
         _check(_lib.llama_profile_stop(self.handle, ms, by, fl, rw, max_records, ctypes.byref(n)))
         return [(ms[i], by[i], fl[i], rw[i]) for i in range(n.value)]
+
+    def timeline_start(self, stream=None):
+        _check(_lib.llama_timeline_start(self.handle, _stream(stream)))
+
+    def timeline_stop(self, max_records: int = 8192):
+        """[(end_ns, kind name, algorithmic bytes)] of the decode launches that
+        took a timeline slot since timeline_start, in launch order."""
+        en = (ctypes.c_uint64 * max_records)()
+        kd = (ctypes.c_int32 * max_records)()
+        by = (ctypes.c_int64 * max_records)()
+        n = ctypes.c_int()
+        _check(_lib.llama_timeline_stop(self.handle, en, kd, by, max_records, ctypes.byref(n)))
+        return [(int(en[i]), TIMELINE_KINDS.get(kd[i], str(kd[i])), int(by[i])) for i in range(n.value)]
+
+    def debug_stall(self, which: str, unit: int = 0, wait_limit_ns: int = 1_000_000):
+        """Arm a one-shot stalled producer in the next `which` launch
+        ("projection", "attention" or "none"): tests of the device timeout."""
+        code = {"none": LLAMA_STALL_NONE, "projection": LLAMA_STALL_PROJECTION,
+                "attention": LLAMA_STALL_ATTENTION}[which]
+        _check(_lib.llama_debug_stall(self.handle, code, int(unit), int(wait_limit_ns)))
 
     def status(self) -> int:
         s = ctypes.c_int()

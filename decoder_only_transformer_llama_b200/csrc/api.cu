@@ -53,7 +53,7 @@ struct Layout {
     size_t off_kc, off_vc, kv_bytes;
     size_t off_x, off_y, off_q, off_attn, off_g, off_ylast, off_tok_ids, off_tok_row, off_tok_pos, off_last,
         off_logits, off_part_o, off_part_ml, off_attn_cnt, off_status, off_rope, off_gemm_part, off_gemm_cnt,
-        off_ssq, ws_end;
+        off_ssq, off_tl, off_best, off_step_cnt, ws_end;
 };
 
 static int make_layout(const llama_model_args* a, Layout* o) {
@@ -140,6 +140,9 @@ static int make_layout(const llama_model_args* a, Layout* o) {
     l.off_gemm_part = off; off = align256(off + (a->dtype != LLAMA_F32 ? kGemmPartBytes : 0));
     l.off_gemm_cnt = off; off = align256(off + kMaxTiles * sizeof(int));
     l.off_ssq = off; off = align256(off + static_cast<size_t>(l.Bmax) * (l.dim / 128 + 1) * 4);
+    l.off_tl = off; off = align256(off + static_cast<size_t>(kTimelineCap) * 8);
+    l.off_best = off; off = align256(off + static_cast<size_t>(l.Bmax) * 8);
+    l.off_step_cnt = off; off = align256(off + kStepCounters * sizeof(int));
     l.ws_end = off;
     return LLAMA_OK;
 }
@@ -150,15 +153,53 @@ static int make_maps(TmaMaps* t, const void* base, int rows, int cols, int b_box
     return LLAMA_OK;
 }
 
-static int64_t proj_bytes(int M, int N, int K, int mode) {
+// Algorithmic bytes of one projection: the weight once, the 16-bit input rows
+// once, and what its epilogue must move (fp32 store; fp32 residual read and
+// write; 16-bit q/k/v; the 16-bit SwiGLU product, half as wide as N; the
+// logits only when they are stored).
+static int64_t proj_bytes(int M, int N, int K, const Epi& ep) {
     const int64_t mn = static_cast<int64_t>(M) * N;
-    const int64_t out = mode == EPI_STORE_F32 ? 4 * mn : mode == EPI_RESID_F32 ? 8 * mn : mode == EPI_QKV ? 2 * mn : mn;
+    int64_t out = 0;
+    switch (ep.mode) {
+        case EPI_STORE_F32: out = 4 * mn; break;
+        case EPI_RESID_F32: out = 8 * mn; break;
+        case EPI_QKV: out = 2 * mn; break;
+        case EPI_SWIGLU: out = mn; break;
+        case EPI_LOGITS_ARGMAX: out = ep.out ? 4 * mn : 0; break;
+    }
     return 2LL * N * K + 2LL * M * K + out;
 }
 
+// The one-shot stall of llama_debug_stall, taken by the first launch of the
+// chosen kind: returns true and the stall's unit and wait limit, and clears it.
+static bool take_stall(Model* m, int kind, int* unit, long long* wait_ns) {
+    if (m->dbg_kind != kind) return false;
+    *unit = m->dbg_unit;
+    *wait_ns = m->dbg_wait_ns;
+    m->dbg_kind = 0;
+    return true;
+}
+
+unsigned long long* tl_next(Model* m, int kind, int64_t bytes) {
+    if (!m->tl_on || m->tl_n >= kTimelineCap) return nullptr;
+    m->tl_kind.push_back(kind);
+    m->tl_bytes.push_back(bytes);
+    return m->tl_end + m->tl_n++;
+}
+
 int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, const void* W,
-               const TmaMaps* mapW, int M, int N, int K, const Epi& ep, cudaStream_t st, bool pdl,
-               const NormIO* nio) {
+               const TmaMaps* mapW, int M, int N, int K, const Epi& ep_in, cudaStream_t st, bool pdl,
+               const NormIO* nio, bool stamp) {
+    Epi ep = ep_in;
+    if (stamp) ep.tl = tl_next(const_cast<Model*>(m), TL_PROJECTION, proj_bytes(M, N, K, ep));
+    if (dtype != LLAMA_F32 && M <= 64) {
+        int unit = 0;
+        long long wait_ns = 0;
+        if (take_stall(const_cast<Model*>(m), LLAMA_STALL_PROJECTION, &unit, &wait_ns)) {
+            ep.stall = unit + 1;
+            ep.wait_ns = wait_ns;
+        }
+    }
     Profile* pr = const_cast<Profile*>(&m->prof);
     const bool timed = pr->n < pr->capacity;
     if (timed) {
@@ -173,7 +214,7 @@ int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, co
     if (timed && rc == LLAMA_OK) {
         cudaError_t e = cudaEventRecord(pr->ev[2 * pr->n + 1], st);
         if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord(profile)");
-        pr->bytes[pr->n] = proj_bytes(M, N, K, ep.mode);
+        pr->bytes[pr->n] = proj_bytes(M, N, K, ep);
         pr->flops[pr->n] = 2LL * M * N * K;
         pr->rows[pr->n] = M;
         pr->n++;
@@ -215,10 +256,12 @@ constexpr int kFusedDecodeRows = 64;
 // TransformerBlock: h = x + attn(norm(x)); out = h + ffn(norm(h))).
 template <typename AttnFn>
 static int block_forward(Model* m, int l, int M, const int* tok_row, const int* tok_pos, AttnFn attn,
-                         cudaStream_t st, bool pdl) {
+                         cudaStream_t st, bool pdl, bool stamp = false) {
     LayerPtrs& Lp = m->layers[l];
     const size_t esz = m->esz;
-    LLB_TRY(launch_rmsnorm(m->x, nullptr, Lp.attn_norm, M, m->dim, m->a.norm_eps, m->y, m->dtype, st, pdl));
+    auto norm_tl = [&]() { return stamp ? tl_next(m, TL_RMSNORM, 0) : nullptr; };
+    LLB_TRY(launch_rmsnorm(m->x, nullptr, Lp.attn_norm, M, m->dim, m->a.norm_eps, m->y, m->dtype, st, pdl,
+                           norm_tl()));
     Epi ep = base_epi(m);
     ep.mode = EPI_QKV;
     ep.q = m->q;
@@ -226,19 +269,23 @@ static int block_forward(Model* m, int l, int M, const int* tok_row, const int* 
     ep.vc = static_cast<char*>(m->vc) + l * m->kv_layer_elems * esz;
     ep.tok_row = tok_row;
     ep.tok_pos = tok_pos;
-    LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.wqkv, &Lp.m_wqkv, M, m->nqkv, m->dim, ep, st, pdl));
+    LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.wqkv, &Lp.m_wqkv, M, m->nqkv, m->dim, ep, st, pdl, nullptr,
+                       stamp));
     LLB_TRY(attn());
     Epi er = base_epi(m);
     er.mode = EPI_RESID_F32;
     er.out = m->x;
     er.ldo = m->dim;
-    LLB_TRY(run_linear(m, m->dtype, m->attn, &m->m_attn, Lp.wo, &Lp.m_wo, M, m->dim, m->nq, er, st, pdl));
-    LLB_TRY(launch_rmsnorm(m->x, nullptr, Lp.ffn_norm, M, m->dim, m->a.norm_eps, m->y, m->dtype, st, pdl));
+    LLB_TRY(run_linear(m, m->dtype, m->attn, &m->m_attn, Lp.wo, &Lp.m_wo, M, m->dim, m->nq, er, st, pdl, nullptr,
+                       stamp));
+    LLB_TRY(launch_rmsnorm(m->x, nullptr, Lp.ffn_norm, M, m->dim, m->a.norm_eps, m->y, m->dtype, st, pdl,
+                           norm_tl()));
     Epi es = base_epi(m);
     es.mode = EPI_SWIGLU;
     es.g = m->g;
-    LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.w13, &Lp.m_w13, M, 2 * m->H, m->dim, es, st, pdl));
-    LLB_TRY(run_linear(m, m->dtype, m->g, &m->m_g, Lp.w2, &Lp.m_w2, M, m->dim, m->H, er, st, pdl));
+    LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.w13, &Lp.m_w13, M, 2 * m->H, m->dim, es, st, pdl, nullptr,
+                       stamp));
+    LLB_TRY(run_linear(m, m->dtype, m->g, &m->m_g, Lp.w2, &Lp.m_w2, M, m->dim, m->H, er, st, pdl, nullptr, stamp));
     return LLAMA_OK;
 }
 
@@ -322,6 +369,9 @@ int llama_model_create(const llama_model_args* args, void* dev_arena, size_t are
     m->gemm_part = reinterpret_cast<float*>(at(A, l.off_gemm_part));
     m->gemm_cnt = reinterpret_cast<int*>(at(A, l.off_gemm_cnt));
     m->ssq = reinterpret_cast<float*>(at(A, l.off_ssq));
+    m->tl_end = reinterpret_cast<unsigned long long*>(at(A, l.off_tl));
+    m->best = reinterpret_cast<unsigned long long*>(at(A, l.off_best));
+    m->step_cnt = reinterpret_cast<int*>(at(A, l.off_step_cnt));
     m->last_stream = static_cast<cudaStream_t>(stream);
 
     int rc = LLAMA_OK;
@@ -345,6 +395,8 @@ int llama_model_create(const llama_model_args* args, void* dev_arena, size_t are
         if (e == cudaSuccess) e = cudaMemsetAsync(m->status, 0, 16, st);
         if (e == cudaSuccess) e = cudaMemsetAsync(m->gemm_cnt, 0, kMaxTiles * sizeof(int), st);
         if (e == cudaSuccess) e = cudaMemsetAsync(m->attn_cnt, 0, static_cast<size_t>(l.Bmax) * l.nkv * 4, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(m->best, 0, static_cast<size_t>(l.Bmax) * 8, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(m->step_cnt, 0, kStepCounters * sizeof(int), st);
         if (e != cudaSuccess) rc = cuda_fail(e, "cudaMemsetAsync");
     }
     if (rc == LLAMA_OK) rc = launch_rope_table(m->rope, l.S, l.hd, args->rope_theta, st);
@@ -481,7 +533,7 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B
         const int nb = m->dim / 128;
         const float eps = m->a.norm_eps;
         LLB_TRY(launch_embed(tokens, m->tok_emb, m->dtype, B, m->dim, m->V, m->x, m->status, st, true, m->ssq, m->y,
-                             m->layers[0].attn_norm));
+                             m->layers[0].attn_norm, tl_next(m, TL_EMBED, 2LL * B * m->dim)));
         for (int l = 0; l < m->L; ++l) {
             LayerPtrs& Lp = m->layers[l];
             const float* next_norm = l + 1 < m->L ? m->layers[l + 1].attn_norm : m->norm;
@@ -493,44 +545,69 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B
             ep.tok_pos = pos;
             const NormIO n_in = {m->ssq, nb, eps, nullptr, nullptr, nullptr};
             LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.wqkv, &Lp.m_wqkv, B, m->nqkv, m->dim, ep, st, true,
-                               &n_in));
+                               &n_in, true));
             Epi er = base_epi(m);
             er.mode = EPI_RESID_F32;
             er.out = m->x;
             er.ldo = m->dim;
             const NormIO n_to_ffn = {nullptr, 0, 0.f, m->ssq, m->y, Lp.ffn_norm};
-            LLB_TRY(launch_attention_decode(m, l, pos, B, st, true));
+            int stall_unit = -1;
+            long long stall_wait = 0;
+            take_stall(m, LLAMA_STALL_ATTENTION, &stall_unit, &stall_wait);
+            LLB_TRY(launch_attention_decode(m, l, pos, B, st, true, tl_next(m, TL_ATTENTION, 0), stall_wait,
+                                            stall_unit));
             LLB_TRY(run_linear(m, m->dtype, m->attn, &m->m_attn, Lp.wo, &Lp.m_wo, B, m->dim, m->nq, er, st, true,
-                               &n_to_ffn));
+                               &n_to_ffn, true));
             Epi es = base_epi(m);
             es.mode = EPI_SWIGLU;
             es.g = m->g;
             LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.w13, &Lp.m_w13, B, 2 * m->H, m->dim, es, st, true,
-                               &n_in));
+                               &n_in, true));
             const NormIO n_to_next = {nullptr, 0, 0.f, m->ssq, m->y, next_norm};
             LLB_TRY(run_linear(m, m->dtype, m->g, &m->m_g, Lp.w2, &Lp.m_w2, B, m->dim, m->H, er, st, true,
-                               &n_to_next));
+                               &n_to_next, true));
         }
         const NormIO n_in = {m->ssq, nb, eps, nullptr, nullptr, nullptr};
-        LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, m->output, &m->m_output, B, m->V, m->dim, eo, st, true,
-                           &n_in));
-    } else {
-        LLB_TRY(launch_embed(tokens, m->tok_emb, m->dtype, B, m->dim, m->V, m->x, m->status, st));
-        for (int l = 0; l < m->L; ++l) {
-            auto attn = [&]() { return launch_attention_decode(m, l, pos, B, st); };
-            LLB_TRY(block_forward(m, l, B, nullptr, pos, attn, st, false));
+        const bool adv = (flags & LLAMA_DECODE_ADVANCE) != 0;
+        if (sampling && sampling->temperature == 0.f) {
+            // greedy: the output projection picks the next tokens itself
+            // (Admin Guide §8.5, argmax at temperature 0); logits are stored
+            // only when the caller asked for them
+            Epi eg = base_epi(m);
+            eg.mode = EPI_LOGITS_ARGMAX;
+            eg.out = logits;
+            eg.ldo = m->V;
+            eg.best = m->best;
+            eg.done = m->step_cnt;
+            eg.next = next_tokens;
+            eg.tok_adv = adv ? const_cast<int32_t*>(tokens) : nullptr;
+            eg.pos_adv = adv ? pos : nullptr;
+            return run_linear(m, m->dtype, m->y, &m->m_y, m->output, &m->m_output, B, m->V, m->dim, eg, st, true,
+                              &n_in, true);
         }
-        LLB_TRY(launch_rmsnorm(m->x, nullptr, m->norm, B, m->dim, m->a.norm_eps, m->ylast, m->dtype, st));
-        LLB_TRY(run_linear(m, m->dtype, m->ylast, &m->m_ylast, m->output, &m->m_output, B, m->V, m->dim, eo, st));
+        LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, m->output, &m->m_output, B, m->V, m->dim, eo, st, true,
+                           &n_in, true));
+    } else {
+        LLB_TRY(launch_embed(tokens, m->tok_emb, m->dtype, B, m->dim, m->V, m->x, m->status, st, false, nullptr,
+                             nullptr, nullptr, tl_next(m, TL_EMBED, 2LL * B * m->dim)));
+        for (int l = 0; l < m->L; ++l) {
+            auto attn = [&]() { return launch_attention_decode(m, l, pos, B, st, false, tl_next(m, TL_ATTENTION, 0)); };
+            LLB_TRY(block_forward(m, l, B, nullptr, pos, attn, st, false, true));
+        }
+        LLB_TRY(launch_rmsnorm(m->x, nullptr, m->norm, B, m->dim, m->a.norm_eps, m->ylast, m->dtype, st, false,
+                               tl_next(m, TL_RMSNORM, 0)));
+        LLB_TRY(run_linear(m, m->dtype, m->ylast, &m->m_ylast, m->output, &m->m_output, B, m->V, m->dim, eo, st,
+                           false, nullptr, true));
     }
     if (!sampling) return LLAMA_OK;
     const bool pdl = fused;
     const bool adv = (flags & LLAMA_DECODE_ADVANCE) != 0;
     int32_t* tok_adv = adv ? const_cast<int32_t*>(tokens) : nullptr;
     int32_t* pos_adv = adv ? pos : nullptr;
-    if (sampling->temperature == 0.f) return launch_argmax(lg, B, m->V, next_tokens, tok_adv, pos_adv, st, pdl);
+    unsigned long long* tls = tl_next(m, TL_SAMPLE, 4LL * B * m->V);
+    if (sampling->temperature == 0.f) return launch_argmax(lg, B, m->V, next_tokens, tok_adv, pos_adv, st, pdl, tls);
     return launch_top_p(lg, B, m->V, sampling->temperature, sampling->top_p, uniforms, next_tokens, tok_adv,
-                        pos_adv, st, pdl);
+                        pos_adv, st, pdl, tls);
 }
 
 int llama_sample(const float* logits, int B, int V, float temperature, float top_p, const float* uniforms,
@@ -557,6 +634,16 @@ int llama_model_status(llama_model* m, int* device_status) {
     cudaError_t e = cudaStreamSynchronize(m->last_stream);
     if (e == cudaSuccess) e = cudaMemcpy(device_status, m->status, sizeof(int), cudaMemcpyDeviceToHost);
     if (e == cudaSuccess) e = cudaMemset(m->status, 0, sizeof(int));
+    // A kernel that gave up on a wait left without adding to, or clearing,
+    // the arrival counters of its split tiles and split attention pairs; the
+    // next launches would pick the wrong last arrival.  Nothing is in flight
+    // here (the stream was synchronised), so start them all at zero again.
+    if (e == cudaSuccess && *device_status != 0) {
+        e = cudaMemset(m->gemm_cnt, 0, kMaxTiles * sizeof(int));
+        if (e == cudaSuccess) e = cudaMemset(m->attn_cnt, 0, static_cast<size_t>(m->Bmax) * m->nkv * sizeof(int));
+        if (e == cudaSuccess) e = cudaMemset(m->best, 0, static_cast<size_t>(m->Bmax) * 8);
+        if (e == cudaSuccess) e = cudaMemset(m->step_cnt, 0, kStepCounters * sizeof(int));
+    }
     if (e != cudaSuccess) return cuda_fail(e, "llama_model_status");
     return LLAMA_OK;
 }
@@ -564,6 +651,55 @@ int llama_model_status(llama_model* m, int* device_status) {
 int llama_model_destroy(llama_model* m) {
     if (m) profile_release(m->prof);
     delete m;
+    return LLAMA_OK;
+}
+
+int llama_debug_stall(llama_model* m, int which, int unit, int64_t wait_limit_ns) {
+    if (!m) { set_error("model is NULL"); return LLAMA_ERR_INVALID_ARG; }
+    if (which != LLAMA_STALL_NONE && which != LLAMA_STALL_PROJECTION && which != LLAMA_STALL_ATTENTION) {
+        set_error("which must be LLAMA_STALL_NONE, _PROJECTION or _ATTENTION");
+        return LLAMA_ERR_INVALID_ARG;
+    }
+    if (which != LLAMA_STALL_NONE && (unit < 0 || wait_limit_ns < 1000 || wait_limit_ns > 2000000000LL)) {
+        set_error("unit must be >= 0 and the wait limit between 1 us and 2 s");
+        return LLAMA_ERR_INVALID_ARG;
+    }
+    if (which != LLAMA_STALL_NONE && m->dtype == LLAMA_F32) {
+        set_error("the stall is a feature of the 16-bit decode kernels");
+        return LLAMA_ERR_INVALID_ARG;
+    }
+    m->dbg_kind = which;
+    m->dbg_unit = unit;
+    m->dbg_wait_ns = wait_limit_ns;
+    return LLAMA_OK;
+}
+
+int llama_timeline_start(llama_model* m, void* stream) {
+    if (!m) { set_error("model is NULL"); return LLAMA_ERR_INVALID_ARG; }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(m->tl_end, 0, static_cast<size_t>(kTimelineCap) * 8, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(timeline)");
+    m->last_stream = st;
+    m->tl_kind.clear();
+    m->tl_bytes.clear();
+    m->tl_n = 0;
+    m->tl_on = true;
+    return LLAMA_OK;
+}
+
+int llama_timeline_stop(llama_model* m, uint64_t* end_ns, int32_t* kind, int64_t* bytes, int max, int* n) {
+    if (!m || max < 0) { set_error("bad timeline arguments"); return LLAMA_ERR_INVALID_ARG; }
+    m->tl_on = false;
+    const int cnt = m->tl_n < max ? m->tl_n : max;
+    cudaError_t e = cudaStreamSynchronize(m->last_stream);
+    if (e == cudaSuccess && end_ns && cnt > 0)
+        e = cudaMemcpy(end_ns, m->tl_end, static_cast<size_t>(cnt) * 8, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "llama_timeline_stop");
+    for (int i = 0; i < cnt; ++i) {
+        if (kind) kind[i] = m->tl_kind[i];
+        if (bytes) bytes[i] = m->tl_bytes[i];
+    }
+    if (n) *n = cnt;
     return LLAMA_OK;
 }
 

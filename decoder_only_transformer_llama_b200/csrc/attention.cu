@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(128)
 attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
                    const int32_t* __restrict__ pos, int B, int nkv, int nq, int S, long long row_stride,
                    float* __restrict__ part_o, float* __restrict__ part_ml, int* __restrict__ counters,
-                   T* __restrict__ out, int* status) {
+                   T* __restrict__ out, int* status, unsigned long long* tl, long long wait_ns, int stall) {
     constexpr int EPL = HD / 32;   // head dims per lane
     constexpr int ROW = HD * static_cast<int>(sizeof(T));
     constexpr int CH_BYTES = kChunk * ROW;
@@ -202,7 +202,10 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
     }
     const long long W = static_cast<long long>(s_cum[B]) * nkv;
     const int P = static_cast<int>(W < gridDim.x ? W : gridDim.x), c = blockIdx.x;
-    if (c >= P) return;
+    if (c >= P) {
+        if (threadIdx.x == 0) tl_stamp(tl);
+        return;
+    }
     const long long u0 = run_begin64(c, W, P), u1 = run_begin64(c + 1, W, P);
     const int len = static_cast<int>(u1 - u0);
 
@@ -231,6 +234,8 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
     auto head_off = [&](const Cur& r) {
         return static_cast<long long>(r.b) * row_stride + static_cast<long long>(r.g) * S * HD;
     };
+    const uint64_t wlim = wait_ns > 0 ? static_cast<uint64_t>(wait_ns) : kWaitLimitNs;
+    const int stall_i = c == 0 ? stall : -1;     // tests of the timeout path only
     Cur icur = cur_at(u0);                       // issue cursor (thread 0)
     auto issue = [&](int i) {                    // i-th unit of this run into ring slot i % NSLOT
         const int ctx = s_pos[icur.b] + 1;
@@ -238,9 +243,11 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
         const int n = min(kChunk, ctx - j0);
         uint8_t* slot = dsm + (i % NSLOT) * 2 * CH_BYTES;
         const long long ho = head_off(icur);
-        mbar_arrive_expect_tx(&bar[i % NSLOT], 2u * n * ROW);
-        bulk_load(slot, kc + ho + static_cast<long long>(j0) * HD, n * ROW, &bar[i % NSLOT]);
-        bulk_load(slot + CH_BYTES, vc + ho + static_cast<long long>(j0) * HD, n * ROW, &bar[i % NSLOT]);
+        if (i != stall_i) {
+            mbar_arrive_expect_tx(&bar[i % NSLOT], 2u * n * ROW);
+            bulk_load(slot, kc + ho + static_cast<long long>(j0) * HD, n * ROW, &bar[i % NSLOT]);
+            bulk_load(slot + CH_BYTES, vc + ho + static_cast<long long>(j0) * HD, n * ROW, &bar[i % NSLOT]);
+        }
         advance(icur);
     };
     if (threadIdx.x == 0) {
@@ -267,10 +274,13 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
     start_pair();
     __syncthreads();   // barriers initialised
     bool ok = true;
+    int fail_i = 0;
     int seg_j0 = cur.j, seg_i0 = 0;
     for (int i = 0; i < len; ++i) {
-        ok = mbar_wait(&bar[i % NSLOT], (i / NSLOT) & 1);
-        if (!ok) break;
+        // every thread of the CTA takes the same branch, even if the wait ran
+        // out at slightly different times in different threads
+        ok = __syncthreads_and(mbar_wait(&bar[i % NSLOT], (i / NSLOT) & 1, wlim));
+        if (!ok) { fail_i = i; break; }
         const T* sK = reinterpret_cast<const T*>(dsm + (i % NSLOT) * 2 * CH_BYTES);
         const T* sV = reinterpret_cast<const T*>(dsm + (i % NSLOT) * 2 * CH_BYTES + CH_BYTES);
         const int ctx = s_pos[cur.b] + 1;
@@ -416,13 +426,22 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
             start_pair();
         }
     }
-    if (!ok && threadIdx.x == 0) report_status(status, LLAMA_ERR_DEVICE_TIMEOUT);
+    if (!ok && threadIdx.x == 0) {
+        report_status(status, LLAMA_ERR_DEVICE_TIMEOUT);
+        // units [fail_i, fail_i + NSLOT) were issued and not consumed: their
+        // copies land before the CTA exits (a skipped unit is not waited for)
+        for (int j = fail_i; j < len && j < fail_i + NSLOT; ++j)
+            if (j != stall_i) mbar_wait(&bar[j % NSLOT], (j / NSLOT) & 1, wlim);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) tl_stamp(tl);
 }
 
 static int g_attn_sms = 0;
 
 template <typename T, int HD, int NREP>
-static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl) {
+static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl,
+                     unsigned long long* tl, long long wait_ns, int stall) {
     const T* kc = static_cast<const T*>(m->kc) + layer * m->kv_layer_elems;
     const T* vc = static_cast<const T*>(m->vc) + layer * m->kv_layer_elems;
     auto kern = attn_decode_kernel<T, HD, NREP>;
@@ -450,39 +469,42 @@ static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaS
     P = std::max<long long>(P, 1);
     cudaError_t e = launch_k(kern, dim3(static_cast<unsigned>(P)), dim3(128), smem, st, pdl, static_cast<const T*>(m->q),
                              kc, vc, pos, B, m->nkv, m->nq, m->S, m->kv_row_elems, m->part_o, m->part_ml,
-                             m->attn_cnt, static_cast<T*>(m->attn), m->status);
+                             m->attn_cnt, static_cast<T*>(m->attn), m->status, tl, wait_ns, stall);
     count_launch();
     if (e != cudaSuccess) return cuda_fail(e, "attn_decode_kernel");
     return LLAMA_OK;
 }
 
 template <typename T, int HD>
-static int decode_rep(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl) {
+static int decode_rep(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl,
+                      unsigned long long* tl, long long wait_ns, int stall) {
     switch (m->n_rep) {
-        case 1: return decode_go<T, HD, 1>(m, layer, pos, B, st, pdl);
-        case 2: return decode_go<T, HD, 2>(m, layer, pos, B, st, pdl);
-        case 4: return decode_go<T, HD, 4>(m, layer, pos, B, st, pdl);
-        case 8: return decode_go<T, HD, 8>(m, layer, pos, B, st, pdl);
+        case 1: return decode_go<T, HD, 1>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+        case 2: return decode_go<T, HD, 2>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+        case 4: return decode_go<T, HD, 4>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+        case 8: return decode_go<T, HD, 8>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
     }
     set_error("n_heads / n_kv_heads = %d unsupported (1, 2, 4, 8)", m->n_rep);
     return LLAMA_ERR_INVALID_ARG;
 }
 
 template <typename T>
-static int decode_hd(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl) {
+static int decode_hd(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl,
+                     unsigned long long* tl, long long wait_ns, int stall) {
     switch (m->hd) {
-        case 32: return decode_rep<T, 32>(m, layer, pos, B, st, pdl);
-        case 64: return decode_rep<T, 64>(m, layer, pos, B, st, pdl);
-        case 128: return decode_rep<T, 128>(m, layer, pos, B, st, pdl);
+        case 32: return decode_rep<T, 32>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+        case 64: return decode_rep<T, 64>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+        case 128: return decode_rep<T, 128>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
     }
     set_error("head_dim %d unsupported", m->hd);
     return LLAMA_ERR_INVALID_ARG;
 }
 
-int launch_attention_decode(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl) {
-    if (m->dtype == LLAMA_BF16) return decode_hd<bf16>(m, layer, pos, B, st, pdl);
-    if (m->dtype == LLAMA_F16) return decode_hd<f16>(m, layer, pos, B, st, pdl);
-    return decode_hd<float>(m, layer, pos, B, st, pdl);
+int launch_attention_decode(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl,
+                            unsigned long long* tl, long long wait_ns, int stall) {
+    if (m->dtype == LLAMA_BF16) return decode_hd<bf16>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+    if (m->dtype == LLAMA_F16) return decode_hd<f16>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+    return decode_hd<float>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
 }
 
 // ---------------------------------------------------------------- prefill

@@ -33,6 +33,29 @@ __device__ __forceinline__ void report_status(int* status, int code) {
     if (status) atomicCAS(status, 0, code);
 }
 
+// ---------------------------------------------------------------- greedy pick
+// Order key of (logit, token id) for the greedy argmax: a larger key is a
+// larger logit, and among equal logits the lower id (its complement is
+// larger).  NaN gives 0, below every number, so it never wins.
+__device__ __forceinline__ unsigned long long argmax_key(float v, int id) {
+    if (v != v) return 0ull;
+    uint32_t u = __float_as_uint(v);
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return (static_cast<unsigned long long>(u) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(id));
+}
+// Token id of a key (0 for the empty key: every logit NaN gives token 0).
+__device__ __forceinline__ int argmax_key_id(unsigned long long k) {
+    return k ? static_cast<int>(~static_cast<uint32_t>(k & 0xffffffffull)) : 0;
+}
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
+        v = w > v ? w : v;
+    }
+    return v;
+}
+
 // ---------------------------------------------------------------- programmatic dependent launch
 // Kernels of the decode chain are launched so that they may start before
 // their predecessor has finished.  Each calls pdl_wait() before its first
@@ -95,6 +118,13 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // LLAMA_ERR_DEVICE_TIMEOUT; no kernel spins without a bound.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 
+// Timeline stamp (benchmarks): called by one thread of a CTA once the CTA's
+// work is done; the slot keeps the latest %globaltimer value over the
+// launch's CTAs, i.e. when the launch finished.
+__device__ __forceinline__ void tl_stamp(unsigned long long* tl) {
+    if (tl) atomicMax(tl, static_cast<unsigned long long>(globaltimer_ns()));
+}
+
 // ---------------------------------------------------------------- shared-memory addresses
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -120,13 +150,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
     return ok != 0;
 }
-// Bounded wait: returns false (and the caller must bail out) after kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Bounded wait: returns false (and the caller must bail out) after `limit_ns`.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
     }
 }
 

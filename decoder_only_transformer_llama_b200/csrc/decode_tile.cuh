@@ -119,6 +119,21 @@ __device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int la
             nio.ssq_out[epi_tid * n_tiles + t] = ((red[epi_tid] + red[64 + epi_tid]) + red[128 + epi_tid]) +
                                            red[192 + epi_tid];
         named_sync(2, 128);
+    } else if (ep.mode == EPI_LOGITS_ARGMAX) {
+        // logits (when kept) and this tile's share of each token column's
+        // greedy pick: the warp's largest key, folded into best[b]
+#pragma unroll
+        for (int b = 0; b < BN; ++b) {
+            if (b < nb) {   // uniform over the CTA
+                unsigned long long key = 0;
+                if (row_ok) {
+                    if (ep.out) ep.out[static_cast<long long>(b) * ep.ldo + n] = v[b];
+                    key = argmax_key(v[b], n);
+                }
+                key = warp_max_u64(key);
+                if (lane == 0 && key) atomicMax(&ep.best[b], key);
+            }
+        }
     } else if (row_ok) {
         if (ep.mode == EPI_RESID_F32) {
 #pragma unroll
@@ -151,7 +166,7 @@ __device__ __forceinline__ void decode_epilogue_loop(uint32_t tmem_lane, uint64_
                                                      float* part, int* counters, int c, int P, int u0, int u1,
                                                      int KT, int N, int M, const Epi& ep, const NormIO& nio,
                                                      bool scale_in, const float* rs, float* red, int r, int lane,
-                                                     int q, int epi_tid) {
+                                                     int q, int epi_tid, uint64_t wlim) {
     const int n_tiles = (N + 127) / 128;
     const int W = n_tiles * KT;
     int u = u0;
@@ -160,7 +175,7 @@ __device__ __forceinline__ void decode_epilogue_loop(uint32_t tmem_lane, uint64_
     const int nb = M < BN ? M : BN;
     while (next_seg(u, u1, KT, sg)) {
         const int acc = j & 1;
-        const bool ok_wait = mbar_wait(&tfull[acc], (j >> 1) & 1);
+        const bool ok_wait = mbar_wait(&tfull[acc], (j >> 1) & 1, wlim);
         tc_fence_after();
         float v[BN];
 #pragma unroll

@@ -56,7 +56,7 @@ int launch_token_map(const RowTable& rt, const int32_t* tokens, int* tok_ids, in
 // 16-bit type: the next projection's fused RMSNorm inputs.
 template <typename T>
 __global__ void embed_kernel(const int* tok, const T* emb, int dim, int V, float* x, int* status, float* ssq,
-                             T* y, const float* w_next) {
+                             T* y, const float* w_next, unsigned long long* tl) {
     pdl_trigger();
     pdl_wait();
     const int m = blockIdx.x;
@@ -67,6 +67,7 @@ __global__ void embed_kernel(const int* tok, const T* emb, int dim, int V, float
         for (int i = threadIdx.x; i < dim; i += blockDim.x) dst[i] = 0.f;
         if (ssq)
             for (int i = threadIdx.x; i < dim / 128; i += blockDim.x) ssq[static_cast<long long>(m) * (dim / 128) + i] = 0.f;
+        if (threadIdx.x == 0) tl_stamp(tl);
         return;
     }
     const T* src = emb + static_cast<long long>(id) * dim;
@@ -110,10 +111,12 @@ __global__ void embed_kernel(const int* tok, const T* emb, int dim, int V, float
         for (int i = threadIdx.x; i < dim / 4; i += blockDim.x)
             reinterpret_cast<float4*>(dst)[i] = s4[i];
     }
+    if (threadIdx.x == 0) tl_stamp(tl);
 }
 
 int launch_embed(const int* tok_ids, const void* emb, int dtype, int M, int dim, int V, float* x,
-                 int* status, cudaStream_t st, bool pdl, float* ssq, void* y, const float* w_next) {
+                 int* status, cudaStream_t st, bool pdl, float* ssq, void* y, const float* w_next,
+                 unsigned long long* tl) {
     if (M <= 0) return LLAMA_OK;
     static bool attr = false;
     if (!attr) {
@@ -126,14 +129,14 @@ int launch_embed(const int* tok_ids, const void* emb, int dtype, int M, int dim,
     cudaError_t e;
     if (dtype == LLAMA_BF16)
         e = launch_k(embed_kernel<bf16>, dim3(M), dim3(128), 0, st, pdl, tok_ids, static_cast<const bf16*>(emb),
-                     dim, V, x, status, ssq, static_cast<bf16*>(y), w_next);
+                     dim, V, x, status, ssq, static_cast<bf16*>(y), w_next, tl);
     else if (dtype == LLAMA_F16)
         e = launch_k(embed_kernel<f16>, dim3(M), dim3(128), 0, st, pdl, tok_ids, static_cast<const f16*>(emb),
-                     dim, V, x, status, ssq, static_cast<f16*>(y), w_next);
+                     dim, V, x, status, ssq, static_cast<f16*>(y), w_next, tl);
     else
         e = launch_k(embed_kernel<float>, dim3(M), dim3(128), 0, st, pdl, tok_ids, static_cast<const float*>(emb),
                      dim, V, x, status, static_cast<float*>(nullptr), static_cast<float*>(nullptr),
-                     static_cast<const float*>(nullptr));
+                     static_cast<const float*>(nullptr), tl);
     count_launch();
     if (e != cudaSuccess) return cuda_fail(e, "embed_kernel");
     return LLAMA_OK;
@@ -145,7 +148,8 @@ int launch_embed(const int* tok_ids, const void* emb, int dtype, int M, int dim,
 // One CTA per row; each thread keeps its float4 slices in registers.
 template <typename TO, int kVecPerThread>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* x, const int* row_idx,
-                                                      const float* w, int dim, float eps, TO* out) {
+                                                      const float* w, int dim, float eps, TO* out,
+                                                      unsigned long long* tl) {
     pdl_trigger();
     pdl_wait();
     const int m = blockIdx.x;
@@ -190,20 +194,21 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* x, const int*
             }
         }
     }
+    if (threadIdx.x == 0) tl_stamp(tl);
 }
 
 template <typename TO>
 static int rmsnorm_dispatch(const float* x, const int* row_idx, const float* w, int M, int dim,
-                            float eps, TO* out, cudaStream_t st, bool pdl) {
+                            float eps, TO* out, cudaStream_t st, bool pdl, unsigned long long* tl) {
     const int nv = dim / 4;
     const int threads = nv >= 256 ? 256 : ((nv + 31) / 32) * 32;
     const int per = (nv + threads - 1) / threads;
     cudaError_t e;
-    if (per <= 1)       e = launch_k(rmsnorm_kernel<TO, 1>, dim3(M), dim3(threads), 0, st, pdl, x, row_idx, w, dim, eps, out);
-    else if (per <= 2)  e = launch_k(rmsnorm_kernel<TO, 2>, dim3(M), dim3(threads), 0, st, pdl, x, row_idx, w, dim, eps, out);
-    else if (per <= 4)  e = launch_k(rmsnorm_kernel<TO, 4>, dim3(M), dim3(threads), 0, st, pdl, x, row_idx, w, dim, eps, out);
-    else if (per <= 8)  e = launch_k(rmsnorm_kernel<TO, 8>, dim3(M), dim3(threads), 0, st, pdl, x, row_idx, w, dim, eps, out);
-    else if (per <= 16) e = launch_k(rmsnorm_kernel<TO, 16>, dim3(M), dim3(threads), 0, st, pdl, x, row_idx, w, dim, eps, out);
+    if (per <= 1)       e = launch_k(rmsnorm_kernel<TO, 1>, dim3(M), dim3(threads), 0, st, pdl, x, row_idx, w, dim, eps, out, tl);
+    else if (per <= 2)  e = launch_k(rmsnorm_kernel<TO, 2>, dim3(M), dim3(threads), 0, st, pdl, x, row_idx, w, dim, eps, out, tl);
+    else if (per <= 4)  e = launch_k(rmsnorm_kernel<TO, 4>, dim3(M), dim3(threads), 0, st, pdl, x, row_idx, w, dim, eps, out, tl);
+    else if (per <= 8)  e = launch_k(rmsnorm_kernel<TO, 8>, dim3(M), dim3(threads), 0, st, pdl, x, row_idx, w, dim, eps, out, tl);
+    else if (per <= 16) e = launch_k(rmsnorm_kernel<TO, 16>, dim3(M), dim3(threads), 0, st, pdl, x, row_idx, w, dim, eps, out, tl);
     else { set_error("rmsnorm: dim %d too large", dim); return LLAMA_ERR_INVALID_ARG; }
     count_launch();
     if (e != cudaSuccess) return cuda_fail(e, "rmsnorm_kernel");
@@ -211,13 +216,13 @@ static int rmsnorm_dispatch(const float* x, const int* row_idx, const float* w, 
 }
 
 int launch_rmsnorm(const float* x, const int* row_idx, const float* w, int M, int dim, float eps,
-                   void* out, int out_dtype, cudaStream_t st, bool pdl) {
+                   void* out, int out_dtype, cudaStream_t st, bool pdl, unsigned long long* tl) {
     if (M <= 0) return LLAMA_OK;
     if (out_dtype == LLAMA_BF16)
-        return rmsnorm_dispatch<bf16>(x, row_idx, w, M, dim, eps, static_cast<bf16*>(out), st, pdl);
+        return rmsnorm_dispatch<bf16>(x, row_idx, w, M, dim, eps, static_cast<bf16*>(out), st, pdl, tl);
     if (out_dtype == LLAMA_F16)
-        return rmsnorm_dispatch<f16>(x, row_idx, w, M, dim, eps, static_cast<f16*>(out), st, pdl);
-    return rmsnorm_dispatch<float>(x, row_idx, w, M, dim, eps, static_cast<float*>(out), st, pdl);
+        return rmsnorm_dispatch<f16>(x, row_idx, w, M, dim, eps, static_cast<f16*>(out), st, pdl, tl);
+    return rmsnorm_dispatch<float>(x, row_idx, w, M, dim, eps, static_cast<float*>(out), st, pdl, tl);
 }
 
 // ---------------------------------------------------------------- w1/w3 interleave

@@ -50,11 +50,13 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
     uint64_t* empty = full + STAGES;
     uint64_t* tfull = empty + STAGES;    // [2]
     uint64_t* tempty = tfull + 2;        // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+    uint64_t* mdone = tempty + 2;        // the MMA issuer's last commit
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + 1);
     int* flag = reinterpret_cast<int*>(tmem_slot + 1);   // [0] abort, [1] fixup broadcast
     float* rs = reinterpret_cast<float*>(flag + 4);      // [64] RMSNorm factors of the token rows
     float* red = rs + 64;                                // [4][64] epilogue sums of squares
     const bool scale_in = nio.ssq_in != nullptr;
+    const uint64_t wlim = ep.wait_ns > 0 ? static_cast<uint64_t>(ep.wait_ns) : kWaitLimitNs;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = gridDim.x, c = blockIdx.x;
@@ -65,6 +67,7 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 128); }
+        mbar_init(mdone, 1);
         flag[0] = 0;
         fence_mbar_init();
         tma_prefetch_desc(&mapW);
@@ -77,6 +80,7 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
     const uint32_t tmem = *tmem_slot;
     pdl_trigger();
 
+    int issued = 0, stall = -1;   // producer: ring stages [0, issued) were issued, all but `stall`
     if (warp == 0 && lane == 0) {
         // ---------------- producer: one weight tile + the matching activation
         // tiles per ring slot, walking this CTA's units in order.  Weight
@@ -84,30 +88,40 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
         // has finished; activation tiles only after it has.
         const int nunits = u1 - u0;
         const int npre = nunits < STAGES ? nunits : STAGES;
+        stall = c == 0 ? ep.stall - 1 : -1;   // tests of the timeout path only
         int t0 = u0 / KT, k0 = u0 - t0 * KT;          // walk (tile, k) without divisions
         int tt = t0, kk = k0;
         for (int i = 0; i < npre; ++i) {
-            mbar_arrive_expect_tx(&full[i], STAGE);
-            tma_load_2d(smem + i * STAGE, &mapW, kk * 64, tt * 128, &full[i]);
+            if (i != stall) {
+                mbar_arrive_expect_tx(&full[i], STAGE);
+                tma_load_2d(smem + i * STAGE, &mapW, kk * 64, tt * 128, &full[i]);
+            }
             if (++kk == KT) { kk = 0; ++tt; }
         }
         pdl_wait();
         tt = t0;
         kk = k0;
         for (int i = 0; i < npre; ++i) {
+            if (i != stall) {
 #pragma unroll
-            for (int rr = 0; rr < BN / 16; ++rr)
-                tma_load_2d(smem + i * STAGE + kABytes + rr * 2048, &mapX, kk * 64, rr * 16, &full[i]);
+                for (int rr = 0; rr < BN / 16; ++rr)
+                    tma_load_2d(smem + i * STAGE + kABytes + rr * 2048, &mapX, kk * 64, rr * 16, &full[i]);
+            }
             if (++kk == KT) { kk = 0; ++tt; }
         }
+        issued = npre;
         for (int i = npre; i < nunits; ++i) {
             const int s = i % STAGES;
-            if (!mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1)) { atomicExch(&flag[0], 1); break; }
-            uint8_t* st = smem + s * STAGE;
-            mbar_arrive_expect_tx(&full[s], STAGE);
-            tma_load_2d(st, &mapW, kk * 64, tt * 128, &full[s]);
+            if (!mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, wlim)) { atomicExch(&flag[0], 1); break; }
+            if (i != stall) {
+                uint8_t* st = smem + s * STAGE;
+                mbar_arrive_expect_tx(&full[s], STAGE);
+                tma_load_2d(st, &mapW, kk * 64, tt * 128, &full[s]);
 #pragma unroll
-            for (int rr = 0; rr < BN / 16; ++rr) tma_load_2d(st + kABytes + rr * 2048, &mapX, kk * 64, rr * 16, &full[s]);
+                for (int rr = 0; rr < BN / 16; ++rr)
+                    tma_load_2d(st + kABytes + rr * 2048, &mapX, kk * 64, rr * 16, &full[s]);
+            }
+            issued = i + 1;
             if (++kk == KT) { kk = 0; ++tt; }
         }
     } else if (warp == 1 && lane == 0) {
@@ -119,12 +133,12 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
         bool abort = false;
         while (!abort && next_seg(u, u1, KT, sg)) {
             const int acc = j & 1;
-            if (!mbar_wait(&tempty[acc], ((j >> 1) & 1) ^ 1)) { atomicExch(&flag[0], 1); break; }
+            if (!mbar_wait(&tempty[acc], ((j >> 1) & 1) ^ 1, wlim)) { atomicExch(&flag[0], 1); break; }
             tc_fence_after();
             const uint32_t d = tmem + acc * kAccStride;
             for (int k = sg.ks; k < sg.ke; ++k, ++i) {
                 const int s = i % STAGES;
-                if (!mbar_wait(&full[s], (i / STAGES) & 1)) { atomicExch(&flag[0], 1); abort = true; break; }
+                if (!mbar_wait(&full[s], (i / STAGES) & 1, wlim)) { atomicExch(&flag[0], 1); abort = true; break; }
                 tc_fence_after();
                 const uint32_t a0 = smem_u32(smem + s * STAGE);
                 const uint32_t b0 = a0 + kABytes;
@@ -137,6 +151,10 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
             tc_commit(&tfull[acc]);
             ++j;
         }
+        // every MMA issued here has finished before TMEM is freed (on a normal
+        // run the epilogue has already waited for them)
+        tc_commit(mdone);
+        if (!mbar_wait(mdone, 0, wlim)) atomicExch(&flag[0], 1);
     } else if (warp >= 2) {
         // ---------------- epilogue (warp w reads TMEM lanes 32*(w%4) .. +31)
         pdl_wait();
@@ -152,12 +170,40 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
         }
         named_sync(1, 128);
         decode_epilogue_loop<BN, E>(tmem + lane_base, tfull, tempty, flag, part, counters, c, P, u0, u1, KT, N, M, ep,
-                                 nio, scale_in, rs, red, r, lane, q, epi_tid);
+                                 nio, scale_in, rs, red, r, lane, q, epi_tid, wlim);
+        if (ep.mode == EPI_LOGITS_ARGMAX) __threadfence();   // this CTA's keys before its finish count
     }
 
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+    if (warp == 0 && lane == 0 && *reinterpret_cast<volatile int*>(&flag[0]) != 0) {
+        // the CTA gave up: the copies it still has in flight land before it
+        // exits (the newest stage of each ring slot; a skipped one is not waited for)
+        for (int s = 0; s < STAGES; ++s) {
+            if (issued <= s) continue;
+            int j = s + ((issued - 1 - s) / STAGES) * STAGES;
+            if (j == stall) j -= STAGES;
+            if (j >= 0) mbar_wait(&full[s], (j / STAGES) & 1, wlim);
+        }
+    }
+    if (ep.mode == EPI_LOGITS_ARGMAX && ep.done && warp == 0) {
+        // greedy pick: the CTA that finishes last reads every row's key
+        int last = 0;
+        if (lane == 0) last = atomicAdd(ep.done, 1) == static_cast<int>(gridDim.x) - 1;
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+            __threadfence();
+            for (int b = lane; b < M; b += 32) {
+                const int id = argmax_key_id(atomicExch(&ep.best[b], 0ull));
+                if (ep.next) ep.next[b] = id;
+                if (ep.tok_adv) ep.tok_adv[b] = id;
+                if (ep.pos_adv) ep.pos_adv[b] += 1;
+            }
+            if (lane == 0) atomicExch(ep.done, 0);
+        }
+    }
+    if (threadIdx.x == 0) tl_stamp(ep.tl);
 }
 
 
@@ -167,7 +213,7 @@ static int g_sms = 0;
 template <int BN, int STAGES, typename E>
 static int launch_decode(const CUtensorMap& w, const CUtensorMap& x, int N, int M, int K, const Epi& ep,
                          float* part, int* counters, int max_ctas, cudaStream_t st, bool pdl, const NormIO& nio) {
-    constexpr int smem = 1024 + STAGES * (kABytes + BN * 128) + (2 * STAGES + 4) * 8 + 32 + 5 * 64 * 4;
+    constexpr int smem = 1024 + STAGES * (kABytes + BN * 128) + (2 * STAGES + 5) * 8 + 32 + 5 * 64 * 4;
     static_assert(smem <= 227 * 1024, "shared memory per CTA");
     auto kern = linear_decode_kernel<BN, STAGES, E>;
     static bool attr = false;

@@ -310,6 +310,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, 2 * kBN);
+    if (threadIdx.x == 0) tl_stamp(ep.tl);
 }
 
 // ---------------------------------------------------------------- host side

@@ -21,6 +21,8 @@ constexpr size_t kPrefillPartBytes = static_cast<size_t>(kMaxDecodeCtas) * 2 * 1
 constexpr size_t kGemmPartBytes = kPrefillPartBytes > kDecodePartBytes ? kPrefillPartBytes : kDecodePartBytes;
 constexpr int kMaxTiles = 4096;       // tile counters: N / 128 of the widest projection
 constexpr int kMaxAttnCtas = 1024;    // persistent CTAs of the decode attention kernel
+constexpr int kTimelineCap = 8192;    // launches one timeline can stamp
+constexpr int kStepCounters = 4;      // per-step finish counters
 
 // Token -> (batch row, position) map of one prefill call, passed by value.
 struct RowTable {
@@ -29,7 +31,7 @@ struct RowTable {
 };
 
 // Epilogue of a projection: what happens to acc[m, n] = sum_k A[m,k] W[n,k].
-enum EpiMode { EPI_STORE_F32 = 0, EPI_RESID_F32 = 1, EPI_QKV = 2, EPI_SWIGLU = 3 };
+enum EpiMode { EPI_STORE_F32 = 0, EPI_RESID_F32 = 1, EPI_QKV = 2, EPI_SWIGLU = 3, EPI_LOGITS_ARGMAX = 4 };
 
 struct Epi {
     int mode;
@@ -52,6 +54,25 @@ struct Epi {
     void* g;
     int H;
     int* status;
+    // Timeline slot of this launch (see Model::tl_end), or null.
+    unsigned long long* tl;
+    // LOGITS_ARGMAX (decode projection only): out[m*ldo + n] = acc if out is
+    // not null, and the greedy pick of every token row m: best[m] collects the
+    // largest key (ordered logit bits << 32 | ~n, so equal logits keep the
+    // lowest id); the CTA that finishes last (done counter) writes
+    // next[m] = its id, tok_adv[m] = id and ++pos_adv[m] where those are not
+    // null, and leaves best[] and the counter at zero again.
+    unsigned long long* best;
+    int* done;
+    int32_t* next;
+    int32_t* tok_adv;
+    int32_t* pos_adv;
+    // Decode projection only: every wait gives up after wait_ns (0 = the
+    // default limit); stall = u + 1 (tests of the timeout path) makes CTA 0
+    // issue neither the copies nor the barrier signal of ring stage u
+    // (0 = no stall, the value of a zero-initialised Epi).
+    long long wait_ns;
+    int stall;
 };
 
 // RMSNorm folded into the decode projections (bf16 decode chain), using
@@ -96,6 +117,9 @@ struct Profile {
     std::vector<int32_t> rows;       // token rows (M) per launch
 };
 
+// Kinds of launches a timeline records (the LLAMA_TL_* codes of llama_b200_ops.h).
+enum TlKind { TL_EMBED = 0, TL_PROJECTION = 1, TL_ATTENTION = 2, TL_SAMPLE = 3, TL_RMSNORM = 4 };
+
 struct Model {
     llama_model_args a;
     int dim, L, nh, nkv, hd, n_rep, H, V, S, Bmax, Mmax, dtype, esz;
@@ -130,11 +154,30 @@ struct Model {
     float* gemm_part;   // split-tile partials of the decode projection kernel
     int* gemm_cnt;      // per-tile arrival counters (zero between launches)
     float* ssq;         // [Bmax, dim/128] per-tile sums of x^2 for the fused RMSNorm
+    unsigned long long* best;   // [Bmax] greedy-pick keys of the fused output projection (zero between steps)
+    int* step_cnt;      // [kStepCounters] finish counters of the fused greedy pick (zero between steps)
     int* status;
     TmaMaps m_y, m_attn, m_g, m_ylast;   // activation maps (A box 128 rows, B box 16 rows)
     cudaStream_t last_stream;
     Profile prof;
+    // Timeline of decode launches: while tl_on, launch i of llama_decode_step
+    // is given slot tl_end + i, where its CTAs leave the %globaltimer value
+    // (ns) at which the last of them finished (atomicMax).
+    unsigned long long* tl_end;
+    // One-shot stall for tests of the device timeout (llama_debug_stall): the
+    // next launch of the chosen kernel gets it, then it is cleared.
+    int dbg_kind = 0;          // 0 none, LLAMA_STALL_PROJECTION or LLAMA_STALL_ATTENTION
+    int dbg_unit = -1;
+    long long dbg_wait_ns = 0;
+    bool tl_on = false;
+    int tl_n = 0;
+    std::vector<int> tl_kind;
+    std::vector<int64_t> tl_bytes;
 };
+
+// Next timeline slot of `m` for a launch of `kind` moving `bytes` algorithmic
+// bytes, or null when no timeline is recording (or it is full).
+unsigned long long* tl_next(Model* m, int kind, int64_t bytes);
 
 // ---------------------------------------------------------------- launchers (return LLAMA_* codes)
 int launch_rope_table(float2* rope, int S, int hd, float theta, cudaStream_t st);
@@ -145,17 +188,18 @@ int launch_token_map(const RowTable& rt, const int32_t* tokens, int* tok_ids, in
 // y = bf16(x * w_next) (the fused RMSNorm's producer side, see NormIO).
 int launch_embed(const int* tok_ids, const void* emb, int dtype, int M, int dim, int V, float* x,
                  int* status, cudaStream_t st, bool pdl = false, float* ssq = nullptr, void* y = nullptr,
-                 const float* w_next = nullptr);
+                 const float* w_next = nullptr, unsigned long long* tl = nullptr);
 int launch_rmsnorm(const float* x, const int* row_idx, const float* w, int M, int dim, float eps,
-                   void* out, int out_dtype, cudaStream_t st, bool pdl = false);
+                   void* out, int out_dtype, cudaStream_t st, bool pdl = false, unsigned long long* tl = nullptr);
 int launch_copy_interleave_w13(const void* src, void* w13, int H, int dim, int which, int esz,
                                cudaStream_t st);
 
 // out = A W^T with epilogue `ep`.  A rows: M (tokens), W rows: N, K.
 // 16-bit dtypes use tcgen05 with the given maps (A-side/W-side), fp32 the SIMT kernel.
+// With `stamp`, the launch takes the next timeline slot (see Model::tl_end).
 int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, const void* W,
                const TmaMaps* mapW, int M, int N, int K, const Epi& ep, cudaStream_t st, bool pdl = false,
-               const NormIO* nio = nullptr);
+               const NormIO* nio = nullptr, bool stamp = false);
 int linear_f32(const float* A, const float* W, int M, int N, int K, const Epi& ep, cudaStream_t st);
 // Prefill-shaped projection; with part/counters (kGemmPartBytes, kMaxTiles
 // zeroed ints) the tail wave is split stream-K, without them whole tiles only.
@@ -169,15 +213,18 @@ int linear16(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, int 
 
 int launch_attention_prefill(const Model* m, int layer, const RowTable& rt, cudaStream_t st);
 int launch_attention_prefill_tc(const Model* m, int layer, const RowTable& rt, cudaStream_t st);
+// wait_ns > 0 replaces the default wait limit; stall_unit >= 0: CTA 0 never
+// issues that unit's copies or their barrier signal (tests of the timeout).
 int launch_attention_decode(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st,
-                            bool pdl = false);
+                            bool pdl = false, unsigned long long* tl = nullptr, long long wait_ns = 0,
+                            int stall_unit = -1);
 
 int launch_argmax(const float* logits, int B, int V, int32_t* out, int32_t* tokens_adv,
-                  int32_t* pos_adv, cudaStream_t st, bool pdl = false);
+                  int32_t* pos_adv, cudaStream_t st, bool pdl = false, unsigned long long* tl = nullptr);
 int launch_logprobs(const float* logits, const int32_t* tokens, int N, int V, float* out, cudaStream_t st);
 int launch_top_p(const float* logits, int B, int V, float temperature, float top_p,
                  const float* uniforms, int32_t* out, int32_t* tokens_adv, int32_t* pos_adv,
-                 cudaStream_t st, bool pdl = false);
+                 cudaStream_t st, bool pdl = false, unsigned long long* tl = nullptr);
 
 // TMA descriptor of a K-major 16-bit matrix (dtype LLAMA_BF16 or LLAMA_F16),
 // boxes of 64 columns x box_rows rows, 128-byte swizzle (driver entry point

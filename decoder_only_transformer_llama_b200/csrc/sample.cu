@@ -35,7 +35,8 @@ __device__ __forceinline__ uint64_t sort_key(float l, int id) {
 
 // ---------------------------------------------------------------- argmax
 __global__ void __launch_bounds__(kSampleThreads)
-argmax_kernel(const float* __restrict__ logits, int V, int32_t* out, int32_t* tokens_adv, int32_t* pos_adv) {
+argmax_kernel(const float* __restrict__ logits, int V, int32_t* out, int32_t* tokens_adv, int32_t* pos_adv,
+              unsigned long long* tl) {
     pdl_trigger();
     pdl_wait();
     const int b = blockIdx.x;
@@ -71,6 +72,7 @@ argmax_kernel(const float* __restrict__ logits, int V, int32_t* out, int32_t* to
             out[b] = bi;
             if (tokens_adv) tokens_adv[b] = bi;
             if (pos_adv) pos_adv[b] += 1;
+            tl_stamp(tl);
         }
     }
 }
@@ -190,7 +192,8 @@ __device__ uint64_t radix_select(TopPShared& sh, const float* row, int V, double
 
 __global__ void __launch_bounds__(kSampleThreads)
 top_p_kernel(const float* __restrict__ logits, int V, float temperature, float top_p,
-             const float* __restrict__ uniforms, int32_t* out, int32_t* tokens_adv, int32_t* pos_adv) {
+             const float* __restrict__ uniforms, int32_t* out, int32_t* tokens_adv, int32_t* pos_adv,
+             unsigned long long* tl) {
     extern __shared__ uint8_t smem_raw[];
     TopPShared& sh = *reinterpret_cast<TopPShared*>(smem_raw);
     pdl_trigger();
@@ -244,6 +247,7 @@ top_p_kernel(const float* __restrict__ logits, int V, float temperature, float t
         out[b] = id;
         if (tokens_adv) tokens_adv[b] = id;
         if (pos_adv) pos_adv[b] += 1;
+        tl_stamp(tl);
     }
 }
 
@@ -286,7 +290,7 @@ int launch_logprobs(const float* logits, const int32_t* tokens, int N, int V, fl
 }
 
 int launch_argmax(const float* logits, int B, int V, int32_t* out, int32_t* tokens_adv, int32_t* pos_adv,
-                  cudaStream_t st, bool pdl) {
+                  cudaStream_t st, bool pdl, unsigned long long* tl) {
     static bool attr = false;
     if (!attr) {
         cudaError_t ce = carveout_max(argmax_kernel);
@@ -294,14 +298,15 @@ int launch_argmax(const float* logits, int B, int V, int32_t* out, int32_t* toke
         attr = true;
     }
     cudaError_t e = launch_k(argmax_kernel, dim3(B), dim3(kSampleThreads), 0, st, pdl, logits, V, out, tokens_adv,
-                             pos_adv);
+                             pos_adv, tl);
     count_launch();
     if (e != cudaSuccess) return cuda_fail(e, "argmax_kernel");
     return LLAMA_OK;
 }
 
 int launch_top_p(const float* logits, int B, int V, float temperature, float top_p, const float* uniforms,
-                 int32_t* out, int32_t* tokens_adv, int32_t* pos_adv, cudaStream_t st, bool pdl) {
+                 int32_t* out, int32_t* tokens_adv, int32_t* pos_adv, cudaStream_t st, bool pdl,
+                 unsigned long long* tl) {
     const int smem = static_cast<int>(sizeof(TopPShared));
     static bool attr = false;
     if (!attr) {
@@ -311,7 +316,7 @@ int launch_top_p(const float* logits, int B, int V, float temperature, float top
         attr = true;
     }
     cudaError_t e = launch_k(top_p_kernel, dim3(B), dim3(kSampleThreads), smem, st, pdl, logits, V, temperature,
-                             top_p, uniforms, out, tokens_adv, pos_adv);
+                             top_p, uniforms, out, tokens_adv, pos_adv, tl);
     count_launch();
     if (e != cudaSuccess) return cuda_fail(e, "top_p_kernel");
     return LLAMA_OK;

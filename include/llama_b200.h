@@ -215,7 +215,11 @@ LLAMA_API int llama_token_logprobs(const float* logits, const int32_t* tokens, i
                                    void* stream);
 
 /* Copies the device status word to *device_status (synchronous on the model's
- * last stream) and clears it.  0 = no device-side error since the last read. */
+ * last stream) and clears it.  0 = no device-side error since the last read.
+ * After a non-zero status it also resets the model's internal arrival
+ * counters (a kernel that gave up on a wait leaves them part-counted), so the
+ * next call computes correctly; read the status after any call whose result
+ * is in doubt. */
 LLAMA_API int llama_model_status(llama_model* m, int* device_status);
 
 /* Frees the host handle; the arena and everything in it stay with the caller. */

@@ -85,6 +85,52 @@ LLAMA_API int llama_profile_start(llama_model* m, int capacity);
 LLAMA_API int llama_profile_stop(llama_model* m, float* ms, int64_t* bytes, int64_t* flops, int32_t* rows, int max,
                                  int* n);
 
+/* Timeline of a model's decode steps (for benchmarks): where the time of a
+ * step goes when its kernels overlap (programmatic dependent launch, CUDA
+ * graph replay), which events between launches cannot show.
+ * llama_timeline_start: zeroes the timeline on `stream` and, from now on,
+ *   gives every kernel that llama_decode_step enqueues the next of up to 8192
+ *   slots (embedding, RMSNorm, projection, attention, sampling launches).  A
+ *   launch's CTAs leave in its slot the %globaltimer value (ns) at which the
+ *   last of them finished (an atomic maximum), so launch i ran, exclusive of
+ *   its predecessor, for end_ns[i] - end_ns[i-1].  A CUDA graph captured while
+ *   the timeline records keeps its slots: each replay stamps them again
+ *   (later replays leave later times).
+ * llama_timeline_stop: stops giving out slots, synchronises the model's last
+ *   stream and writes up to `max` records of the slots given out since the
+ *   last start (host arrays, any may be NULL); it may be called again, e.g.
+ *   after replaying a graph captured while recording, to read them anew:
+ *   end_ns[i], kind[i] (LLAMA_TL_*), bytes[i] = the launch's algorithmic
+ *   bytes where the host knows them (projections: every weight once, the
+ *   16-bit input rows, the epilogue's outputs; embedding rows; sampling: the
+ *   logits read), else 0; sets *n to the number of slots given out. */
+#define LLAMA_TL_EMBED       0
+#define LLAMA_TL_PROJECTION  1
+#define LLAMA_TL_ATTENTION   2
+#define LLAMA_TL_SAMPLE      3
+#define LLAMA_TL_RMSNORM     4
+LLAMA_API int llama_timeline_start(llama_model* m, void* stream);
+LLAMA_API int llama_timeline_stop(llama_model* m, uint64_t* end_ns, int32_t* kind, int64_t* bytes, int max, int* n);
+
+/* A stalled producer, for tests of the device-side timeout (failure
+ * detection without a GPU fault).  Every wait of a kernel on another agent is
+ * bounded; when one gives up, the kernel lets its own copies and tensor-core
+ * operations in flight finish, releases its tensor memory, records
+ * LLAMA_ERR_DEVICE_TIMEOUT in the model's device status word and returns.
+ * llama_debug_stall arms that path once: in the next launch of the chosen
+ * decode kernel by this model (16-bit models; the weight-streaming
+ * projection, or the decode attention), CTA 0 never issues the copies of
+ * pipeline stage `unit` of its run nor the barrier signal that would announce
+ * them, and every wait of that launch gives up after wait_limit_ns
+ * (1 us .. 2 s).  A unit past the end of CTA 0's run stalls nothing.  The
+ * outputs of that step are unspecified; llama_model_status then returns the
+ * timeout code and resets the model's internal counters, after which the next
+ * call computes correctly.  LLAMA_STALL_NONE disarms a stall not yet taken. */
+#define LLAMA_STALL_NONE        0
+#define LLAMA_STALL_PROJECTION  1
+#define LLAMA_STALL_ATTENTION   2
+LLAMA_API int llama_debug_stall(llama_model* m, int which, int unit, int64_t wait_limit_ns);
+
 #ifdef __cplusplus
 }
 #endif

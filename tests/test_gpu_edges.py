@@ -140,22 +140,27 @@ def test_prefix_reuse_across_prefill_calls(llb, dtype):
     m.close()
 
 
-def test_decode_wider_than_the_fused_chain(llb):
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_decode_wider_than_the_fused_chain(llb, dtype):
     """A 16-bit decode step of more than 64 rows runs the un-fused sequence
     (one RMSNorm kernel per norm, the 128 x 256-tile projections) instead of
     the fused chain, whose weight-streaming projection takes at most 64 token
-    columns: 72 rows prefilled and decoded twice, sampled rows against the
-    oracle, greedy tokens written back on the device."""
-    shape = SMALL.replace(max_batch_size=72, max_seq_len=32)
+    columns: 72 rows prefilled and decoded twice, in bf16 and fp16, sampled
+    rows against the oracle, greedy tokens written back on the device.  Row 13
+    asks for a position past the cache in both steps: the step reports
+    LLAMA_ERR_CAPACITY for it and the other rows stay exact."""
+    shape = SMALL.replace(max_batch_size=72, max_seq_len=32, dtype=dtype)
+    S = shape.max_seq_len
     w = make_weights(shape, 46)
     m = build_model(shape, w)
-    B, T = 72, 6
+    B, T, bad = 72, 6, 13
     toks = make_tokens(shape.vocab_size, (B, T), token_seed(16)).cuda()
     logits = torch.empty(B, shape.vocab_size, device="cuda")
     m.prefill(toks, logits=logits)
     cur = torch.empty(B, dtype=torch.int32, device="cuda")
     llb.sample(logits, 0.0, 0.9, None, cur)
     pos = torch.full((B,), T, dtype=torch.int32, device="cuda")
+    pos[bad] = S
     seqs = [toks[b].cpu().tolist() for b in range(B)]
     steps = []
     for _ in range(2):
@@ -165,8 +170,10 @@ def test_decode_wider_than_the_fused_chain(llb):
         m.decode_step(cur, pos, temperature=0.0, next_tokens=cur, logits=lg, advance=True)
         torch.cuda.synchronize()
         steps.append(lg.cpu().numpy())
-    assert m.status() == 0
-    assert pos.cpu().tolist() == [T + 2] * B
+    assert m.status() == llb.LLAMA_ERR_CAPACITY
+    want_pos = [T + 2] * B
+    want_pos[bad] = S + 2
+    assert pos.cpu().tolist() == want_pos
     w64 = to_numpy_f64_weights(w)
     for b in (0, 40, 71):
         want = _oracle_logits(shape, w64, seqs[b])[T:]

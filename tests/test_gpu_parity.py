@@ -321,10 +321,13 @@ def test_small_bf16_decode_with_top_p_sampling(llb):
         assert rel_l2(got, want) <= BF16_TOL, (b, rel_l2(got, want))
 
 
-@pytest.mark.parametrize("B,L,dtype", [(1, 128, "bf16"), (8, 1024, "bf16"), (32, 4096, "bf16"), (8, 1024, "f16")])
+@pytest.mark.parametrize("B,L,dtype", [(B, L, "bf16") for B in (1, 8, 32) for L in (128, 1024, 4096)] +
+                         [(8, 1024, "f16")])
 def test_7b_layer_decode_against_oracle(llb, B, L, dtype):
     """One 7B-shaped layer (bf16, fp32 norms), KV cache filled with N(0,1) for
-    positions [0, L), one decode step at position L; oracle on sampled rows."""
+    positions [0, L), one decode step at position L; oracle on sampled rows.
+    Every (batch, context) point of the decode microbenchmark grid, B in
+    {1, 8, 32} x L in {128, 1024, 4096}, plus an fp16 repeat."""
     s = L7B_LAYER.replace(dtype=dtype)
     w = make_weights(s, weight_seed(1), device="cuda")
     m = build_model(s, w)
