@@ -139,7 +139,7 @@ static int make_layout(const llama_model_args* a, Layout* o) {
     l.off_rope = off; off = align256(off + static_cast<size_t>(l.S) * (hd / 2) * 8);
     l.off_gemm_part = off; off = align256(off + (a->dtype != LLAMA_F32 ? kGemmPartBytes : 0));
     l.off_gemm_cnt = off; off = align256(off + kMaxTiles * sizeof(int));
-    l.off_ssq = off; off = align256(off + static_cast<size_t>(l.Bmax) * (l.dim / 128 + 1) * 4);
+    l.off_ssq = off; off = align256(off + static_cast<size_t>(M > Bn ? M : Bn) * (l.dim / 128 + 1) * 4);
     l.off_tl = off; off = align256(off + static_cast<size_t>(kTimelineCap) * 8);
     l.off_best = off; off = align256(off + static_cast<size_t>(l.Bmax) * 8);
     l.off_step_cnt = off; off = align256(off + kStepCounters * sizeof(int));
@@ -252,8 +252,49 @@ static char* at(void* base, size_t off) { return static_cast<char*>(base) + off;
 // llama_decode_step: the weight-streaming projection's MMA N limit.
 constexpr int kFusedDecodeRows = 64;
 
-// One transformer block on M token rows held in m->x (Admin Guide §8.4,
-// TransformerBlock: h = x + attn(norm(x)); out = h + ffn(norm(h))).
+// One transformer block of a 16-bit model on M token rows (Admin Guide §8.4,
+// TransformerBlock: h = x + attn(norm(x)); out = h + ffn(norm(h))), with both
+// RMSNorms folded into the projections: on entry m->y holds bf16(x * w_attn)
+// and m->ssq the per-128-feature sums of x^2 (left by the embedding or the
+// previous block); wq/wk/wv and w1/w3 scale their accumulator rows by 1/rms,
+// and the residual epilogues of wo and w2 leave the next norm's inputs
+// (w_ffn, then the next block's w_attn or the final norm's weight).  M <= 64
+// rows run the weight-streaming projections (pdl: launched early in the
+// decode chain), more rows the 128 x 256-tile ones.
+template <typename AttnFn>
+static int block_forward_fused(Model* m, int l, int M, const int* tok_row, const int* tok_pos, AttnFn attn,
+                               cudaStream_t st, bool pdl, bool stamp) {
+    LayerPtrs& Lp = m->layers[l];
+    const size_t esz = m->esz;
+    const float* next_norm = l + 1 < m->L ? m->layers[l + 1].attn_norm : m->norm;
+    const NormIO n_in = {m->ssq, m->dim / 128, m->a.norm_eps, nullptr, nullptr, nullptr};
+    const NormIO n_to_ffn = {nullptr, 0, 0.f, m->ssq, m->y, Lp.ffn_norm};
+    const NormIO n_to_next = {nullptr, 0, 0.f, m->ssq, m->y, next_norm};
+    Epi ep = base_epi(m);
+    ep.mode = EPI_QKV;
+    ep.q = m->q;
+    ep.kc = static_cast<char*>(m->kc) + l * m->kv_layer_elems * esz;
+    ep.vc = static_cast<char*>(m->vc) + l * m->kv_layer_elems * esz;
+    ep.tok_row = tok_row;
+    ep.tok_pos = tok_pos;
+    LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.wqkv, &Lp.m_wqkv, M, m->nqkv, m->dim, ep, st, pdl, &n_in,
+                       stamp));
+    LLB_TRY(attn());
+    Epi er = base_epi(m);
+    er.mode = EPI_RESID_F32;
+    er.out = m->x;
+    er.ldo = m->dim;
+    LLB_TRY(run_linear(m, m->dtype, m->attn, &m->m_attn, Lp.wo, &Lp.m_wo, M, m->dim, m->nq, er, st, pdl, &n_to_ffn,
+                       stamp));
+    Epi es = base_epi(m);
+    es.mode = EPI_SWIGLU;
+    es.g = m->g;
+    LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.w13, &Lp.m_w13, M, 2 * m->H, m->dim, es, st, pdl, &n_in,
+                       stamp));
+    return run_linear(m, m->dtype, m->g, &m->m_g, Lp.w2, &Lp.m_w2, M, m->dim, m->H, er, st, pdl, &n_to_next, stamp);
+}
+
+// One transformer block of an fp32 model: RMSNorm kernels, then the SIMT projections.
 template <typename AttnFn>
 static int block_forward(Model* m, int l, int M, const int* tok_row, const int* tok_pos, AttnFn attn,
                          cudaStream_t st, bool pdl, bool stamp = false) {
@@ -388,6 +429,13 @@ int llama_model_create(const llama_model_args* args, void* dev_arena, size_t are
         if (rc == LLAMA_OK) rc = make_maps(&m->m_attn, m->attn, l.Mrows, l.nq, 16, l.dtype);
         if (rc == LLAMA_OK) rc = make_maps(&m->m_g, m->g, l.Mrows, l.H, 16, l.dtype);
         if (rc == LLAMA_OK) rc = make_maps(&m->m_ylast, m->ylast, l.Brows, l.dim, 16, l.dtype);
+        const long long kv_rows = static_cast<long long>(l.L) * l.Bmax * l.nkv * l.S;
+        if (rc == LLAMA_OK && l.hd == 128 && kv_rows + 128 < (1LL << 31)) {
+            rc = encode_kmajor_16(&m->m_qtile, m->q, l.Mrows, l.nq, 128, l.dtype);
+            if (rc == LLAMA_OK) rc = encode_kmajor_16(&m->m_kcache, m->kc, static_cast<int>(kv_rows), l.hd, 128, l.dtype);
+            if (rc == LLAMA_OK) rc = encode_kmajor_16(&m->m_vcache, m->vc, static_cast<int>(kv_rows), l.hd, 128, l.dtype);
+            m->has_attn_maps = rc == LLAMA_OK;
+        }
     }
     cudaStream_t st = m->last_stream;
     if (rc == LLAMA_OK) {
@@ -485,10 +533,19 @@ int llama_prefill(llama_model* m, const int32_t* tokens, const int32_t* lens, in
     m->last_stream = st;
 
     LLB_TRY(launch_token_map(rt, tokens, m->tok_ids, m->tok_row, m->tok_pos, m->last_idx, st));
-    LLB_TRY(launch_embed(m->tok_ids, m->tok_emb, m->dtype, M, m->dim, m->V, m->x, m->status, st));
+    const bool fused = m->dtype != LLAMA_F32;
+    if (fused) {
+        LLB_TRY(launch_embed(m->tok_ids, m->tok_emb, m->dtype, M, m->dim, m->V, m->x, m->status, st, false, m->ssq,
+                             m->y, m->layers[0].attn_norm));
+    } else {
+        LLB_TRY(launch_embed(m->tok_ids, m->tok_emb, m->dtype, M, m->dim, m->V, m->x, m->status, st));
+    }
     for (int l = 0; l < m->L; ++l) {
         auto attn = [&]() { return launch_attention_prefill(m, l, rt, st); };
-        LLB_TRY(block_forward(m, l, M, m->tok_row, m->tok_pos, attn, st, false));
+        if (fused)
+            LLB_TRY(block_forward_fused(m, l, M, m->tok_row, m->tok_pos, attn, st, false, false));
+        else
+            LLB_TRY(block_forward(m, l, M, m->tok_row, m->tok_pos, attn, st, false));
     }
     if (!logits) return LLAMA_OK;
     Epi eo = base_epi(m);
@@ -498,6 +555,11 @@ int llama_prefill(llama_model* m, const int32_t* tokens, const int32_t* lens, in
     if (logits_mode == 0) {
         LLB_TRY(launch_rmsnorm(m->x, m->last_idx, m->norm, B, m->dim, m->a.norm_eps, m->ylast, m->dtype, st));
         return run_linear(m, m->dtype, m->ylast, &m->m_ylast, m->output, &m->m_output, B, m->V, m->dim, eo, st);
+    }
+    if (fused) {
+        // every position: y and the sums of squares already hold the final norm's inputs
+        const NormIO n_in = {m->ssq, m->dim / 128, m->a.norm_eps, nullptr, nullptr, nullptr};
+        return run_linear(m, m->dtype, m->y, &m->m_y, m->output, &m->m_output, M, m->V, m->dim, eo, st, false, &n_in);
     }
     LLB_TRY(launch_rmsnorm(m->x, nullptr, m->norm, M, m->dim, m->a.norm_eps, m->y, m->dtype, st));
     return run_linear(m, m->dtype, m->y, &m->m_y, m->output, &m->m_output, M, m->V, m->dim, eo, st);
@@ -520,56 +582,30 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B
     eo.mode = EPI_STORE_F32;
     eo.out = lg;
     eo.ldo = m->V;
-    // The fused chain below needs the weight-streaming projection, whose MMA
-    // takes at most 64 token columns; wider 16-bit steps and fp32 models run
-    // one RMSNorm kernel per norm and the prefill projections instead.
-    const bool fused = m->dtype != LLAMA_F32 && B <= kFusedDecodeRows;
-    if (fused) {
-        // The decode chain: five kernels per layer.  Every kernel may launch
-        // before its predecessor ends (programmatic dependent launch) and waits
-        // for it before reading its outputs.  RMSNorm runs inside the
-        // projections that consume it; the residual epilogues and the
-        // embedding leave per-block sums of squares for it in m->ssq.
-        const int nb = m->dim / 128;
-        const float eps = m->a.norm_eps;
-        LLB_TRY(launch_embed(tokens, m->tok_emb, m->dtype, B, m->dim, m->V, m->x, m->status, st, true, m->ssq, m->y,
+    // 16-bit models fold RMSNorm into the projections (block_forward_fused).
+    // Steps of up to 64 rows run the decode chain: the weight-streaming
+    // projections, every kernel launched early (programmatic dependent
+    // launch) and waiting for its predecessor before reading its outputs, and
+    // the greedy pick inside the vocabulary projection.  Wider steps run the
+    // 128 x 256-tile projections, launched one after another; fp32 models run
+    // RMSNorm kernels and the SIMT projections.
+    const bool chain = m->dtype != LLAMA_F32 && B <= kFusedDecodeRows;
+    if (m->dtype != LLAMA_F32) {
+        LLB_TRY(launch_embed(tokens, m->tok_emb, m->dtype, B, m->dim, m->V, m->x, m->status, st, chain, m->ssq, m->y,
                              m->layers[0].attn_norm, tl_next(m, TL_EMBED, 2LL * B * m->dim)));
         for (int l = 0; l < m->L; ++l) {
-            LayerPtrs& Lp = m->layers[l];
-            const float* next_norm = l + 1 < m->L ? m->layers[l + 1].attn_norm : m->norm;
-            Epi ep = base_epi(m);
-            ep.mode = EPI_QKV;
-            ep.q = m->q;
-            ep.kc = static_cast<char*>(m->kc) + l * m->kv_layer_elems * m->esz;
-            ep.vc = static_cast<char*>(m->vc) + l * m->kv_layer_elems * m->esz;
-            ep.tok_pos = pos;
-            const NormIO n_in = {m->ssq, nb, eps, nullptr, nullptr, nullptr};
-            LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.wqkv, &Lp.m_wqkv, B, m->nqkv, m->dim, ep, st, true,
-                               &n_in, true));
-            Epi er = base_epi(m);
-            er.mode = EPI_RESID_F32;
-            er.out = m->x;
-            er.ldo = m->dim;
-            const NormIO n_to_ffn = {nullptr, 0, 0.f, m->ssq, m->y, Lp.ffn_norm};
-            int stall_unit = -1;
-            long long stall_wait = 0;
-            take_stall(m, LLAMA_STALL_ATTENTION, &stall_unit, &stall_wait);
-            LLB_TRY(launch_attention_decode(m, l, pos, B, st, true, tl_next(m, TL_ATTENTION, 0), stall_wait,
-                                            stall_unit));
-            LLB_TRY(run_linear(m, m->dtype, m->attn, &m->m_attn, Lp.wo, &Lp.m_wo, B, m->dim, m->nq, er, st, true,
-                               &n_to_ffn, true));
-            Epi es = base_epi(m);
-            es.mode = EPI_SWIGLU;
-            es.g = m->g;
-            LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.w13, &Lp.m_w13, B, 2 * m->H, m->dim, es, st, true,
-                               &n_in, true));
-            const NormIO n_to_next = {nullptr, 0, 0.f, m->ssq, m->y, next_norm};
-            LLB_TRY(run_linear(m, m->dtype, m->g, &m->m_g, Lp.w2, &Lp.m_w2, B, m->dim, m->H, er, st, true,
-                               &n_to_next, true));
+            auto attn = [&]() {
+                int stall_unit = -1;
+                long long stall_wait = 0;
+                take_stall(m, LLAMA_STALL_ATTENTION, &stall_unit, &stall_wait);
+                return launch_attention_decode(m, l, pos, B, st, chain, tl_next(m, TL_ATTENTION, 0), stall_wait,
+                                               stall_unit);
+            };
+            LLB_TRY(block_forward_fused(m, l, B, nullptr, pos, attn, st, chain, true));
         }
-        const NormIO n_in = {m->ssq, nb, eps, nullptr, nullptr, nullptr};
+        const NormIO n_in = {m->ssq, m->dim / 128, m->a.norm_eps, nullptr, nullptr, nullptr};
         const bool adv = (flags & LLAMA_DECODE_ADVANCE) != 0;
-        if (sampling && sampling->temperature == 0.f) {
+        if (chain && sampling && sampling->temperature == 0.f) {
             // greedy: the output projection picks the next tokens itself
             // (Admin Guide §8.5, argmax at temperature 0); logits are stored
             // only when the caller asked for them
@@ -585,7 +621,7 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B
             return run_linear(m, m->dtype, m->y, &m->m_y, m->output, &m->m_output, B, m->V, m->dim, eg, st, true,
                               &n_in, true);
         }
-        LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, m->output, &m->m_output, B, m->V, m->dim, eo, st, true,
+        LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, m->output, &m->m_output, B, m->V, m->dim, eo, st, chain,
                            &n_in, true));
     } else {
         LLB_TRY(launch_embed(tokens, m->tok_emb, m->dtype, B, m->dim, m->V, m->x, m->status, st, false, nullptr,
@@ -600,7 +636,7 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B
                            false, nullptr, true));
     }
     if (!sampling) return LLAMA_OK;
-    const bool pdl = fused;
+    const bool pdl = chain;
     const bool adv = (flags & LLAMA_DECODE_ADVANCE) != 0;
     int32_t* tok_adv = adv ? const_cast<int32_t*>(tokens) : nullptr;
     int32_t* pos_adv = adv ? pos : nullptr;

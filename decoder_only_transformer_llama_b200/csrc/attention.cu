@@ -634,7 +634,9 @@ static int prefill_hd(const Model* m, int layer, const RowTable& rt, cudaStream_
 }
 
 int launch_attention_prefill(const Model* m, int layer, const RowTable& rt, cudaStream_t st) {
-    // 16-bit models run the tensor-core kernel; fp32 models the CUDA-core one (no TF32)
+    // 16-bit models run a tensor-core kernel (tcgen05 with TMEM accumulators
+    // for head_dim 128, mma.sync for 32 and 64); fp32 models the CUDA-core one (no TF32)
+    if (attention_prefill_tmem_ok(m)) return launch_attention_prefill_tmem(m, layer, rt, st);
     if (m->dtype != LLAMA_F32) return launch_attention_prefill_tc(m, layer, rt, st);
     return prefill_hd<float>(m, layer, rt, st);
 }

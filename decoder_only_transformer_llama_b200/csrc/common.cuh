@@ -276,6 +276,36 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, float* v) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 lanes x 32 consecutive fp32 columns from registers: thread i of the
+// warp writes lane (base+i).  Complete with tc_wait_st() before the columns
+// are read by an MMA.
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const float (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        :: "r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+           "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+           "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+           "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+           "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+           "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+           "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+           "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+           "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+           "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+           "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+__device__ __forceinline__ void tc_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// Generic-proxy writes to shared memory (st.shared) made visible to the
+// async proxy (the tensor core reading them as an MMA operand).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Shared-memory matrix descriptor for a K-major 16-bit tile stored as TMA
 // writes it with 128-byte swizzling: rows of 64 elements (128 B), groups of 8
 // rows 1024 B apart.  The tile base must be 1024-byte aligned.
@@ -286,6 +316,21 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr) {
     d |= static_cast<uint64_t>(1024 >> 4) << 32;                 // stride byte offset
     d |= static_cast<uint64_t>(1) << 46;                         // descriptor version (sm_100)
     d |= static_cast<uint64_t>(2) << 61;                         // SWIZZLE_128B
+    return d;
+}
+
+// Shared-memory matrix descriptor for an MN-major 16-bit operand stored as
+// TMA writes [K rows][64 MN-values] boxes with 128-byte swizzling: each K row
+// holds 64 consecutive MN values (128 B), 8 K rows form one 1024-byte atom
+// (the stride to the next 8 K rows, SBO), and the next 64 MN values start
+// `mn_atom_bytes` further on (LBO).  The base must be 1024-byte aligned.
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t mn_atom_bytes) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);           // start address
+    d |= static_cast<uint64_t>((mn_atom_bytes >> 4) & 0x3FFF) << 16;   // leading byte offset: next 64 MN values
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;                  // stride byte offset: next 8 K rows
+    d |= static_cast<uint64_t>(1) << 46;                          // descriptor version (sm_100)
+    d |= static_cast<uint64_t>(2) << 61;                          // SWIZZLE_128B
     return d;
 }
 
@@ -304,6 +349,10 @@ template <typename T> __host__ __device__ constexpr uint32_t idesc_16_f32(int M,
 template <> __host__ __device__ constexpr uint32_t idesc_16_f32<bf16>(int M, int N) { return idesc_bf16_f32(M, N); }
 template <> __host__ __device__ constexpr uint32_t idesc_16_f32<f16>(int M, int N) {
     return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+// The same with the B operand MN-major (bit 16: B transposed).
+template <typename T> __host__ __device__ constexpr uint32_t idesc_16_f32_bmn(int M, int N) {
+    return idesc_16_f32<T>(M, N) | (1u << 16);
 }
 
 #ifdef __CUDACC__

@@ -135,12 +135,68 @@ __device__ __forceinline__ void epi_chunk(const Epi& ep, int m, int n0, int rows
     }
 }
 
+// Residual epilogue of 32 consecutive features n0..n0+31 of token row m with
+// the next RMSNorm's producer side (NormIO): x += acc, y = x * w_next in the
+// 16-bit type; returns this chunk's sum of x^2.
+template <typename E>
+__device__ __forceinline__ float epi_chunk_resid_norm(const Epi& ep, const NormIO& nio, int m, int n0,
+                                                      const float (&v)[32]) {
+    float4* o4 = reinterpret_cast<float4*>(ep.out + static_cast<long long>(m) * ep.ldo + n0);
+    const float4* w4 = reinterpret_cast<const float4*>(nio.w_next + n0);
+    uint4* y4 = reinterpret_cast<uint4*>(static_cast<E*>(nio.y_out) + static_cast<long long>(m) * ep.ldo + n0);
+    float4 p[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) p[q] = o4[q];
+    float sq = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        p[q] = make_float4(p[q].x + v[4 * q], p[q].y + v[4 * q + 1], p[q].z + v[4 * q + 2], p[q].w + v[4 * q + 3]);
+        o4[q] = p[q];
+        sq += p[q].x * p[q].x + p[q].y * p[q].y + p[q].z * p[q].z + p[q].w * p[q].w;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float4 wa = w4[2 * q], wb = w4[2 * q + 1];
+        uint4 u;
+        u.x = pack2<E>(p[2 * q].x * wa.x, p[2 * q].y * wa.y);
+        u.y = pack2<E>(p[2 * q].z * wa.z, p[2 * q].w * wa.w);
+        u.z = pack2<E>(p[2 * q + 1].x * wb.x, p[2 * q + 1].y * wb.y);
+        u.w = pack2<E>(p[2 * q + 1].z * wb.z, p[2 * q + 1].w * wb.w);
+        y4[q] = u;
+    }
+    return sq;
+}
+
+// The whole epilogue of 32 features of row m: the consumer side of a fused
+// RMSNorm (scale by rs), then the producer side or the plain epilogue.
+// `sq` accumulates the sums of x^2, written per 128 features when the
+// chunk closes a 128-feature block (or the row's last block).
+template <typename E>
+__device__ __forceinline__ void epi_any(const Epi& ep, const NormIO& nio, int m, int n0, int rowsB, float rs,
+                                        float (&v)[32], float& sq) {
+    if (nio.ssq_in) {
+#pragma unroll
+        for (int t = 0; t < 32; ++t) v[t] *= rs;
+    }
+    if (!nio.ssq_out) {
+        epi_chunk<E>(ep, m, n0, rowsB, v);
+        return;
+    }
+    if (n0 >= rowsB) return;
+    sq += epi_chunk_resid_norm<E>(ep, nio, m, n0, v);
+    if (((n0 + 32) & 127) == 0 || n0 + 32 >= rowsB) {
+        nio.ssq_out[static_cast<long long>(m) * ((rowsB + 127) / 128) + n0 / 128] = sq;
+        sq = 0.f;
+    }
+}
+
 }  // namespace
 
 template <typename E>
 __global__ void __launch_bounds__(kThreadsTc, 1)
 linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                  int rowsA, int rowsB, TcPlan plan, Epi ep, float* __restrict__ part, int* __restrict__ counters) {
+                  int rowsA, int rowsB, TcPlan plan, Epi ep, float* __restrict__ part, int* __restrict__ counters,
+                  NormIO nio) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStagesTc * kStageBytes);
@@ -240,6 +296,13 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
             const bool row_ok = m < rowsA;
             const uint32_t tb = tmem + lane_base + acc * kBN;
             const int nbase = tn * kBN;
+            // fused RMSNorm, consumer side: 1/rms of row m from its sums of squares
+            float rs = 1.f, sq = 0.f;
+            if (nio.ssq_in && row_ok) {
+                float ss = 0.f;
+                for (int t2 = 0; t2 < nio.n_in; ++t2) ss += nio.ssq_in[static_cast<long long>(m) * nio.n_in + t2];
+                rs = rsqrtf(ss / static_cast<float>(KT * 64) + nio.eps);
+            }
             if (it.ks == 0 && it.ke == KT) {
                 // whole tile: TMEM -> epilogue, 32 features at a time
 #pragma unroll 1
@@ -247,7 +310,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
                     float v[32];
                     tmem_ld_32x32b_x32(tb + cc * 32, v);
                     tc_wait_ld();
-                    if (row_ok) epi_chunk<E>(ep, m, nbase + cc * 32, rowsB, v);
+                    if (row_ok) epi_any<E>(ep, nio, m, nbase + cc * 32, rowsB, rs, v, sq);
                 }
                 tc_fence_before();
                 mbar_arrive(&tempty[acc]);
@@ -299,7 +362,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
                         for (int t = 0; t < 32; ++t) v[t] += f[t];
                     }
                 }
-                if (row_ok) epi_chunk<E>(ep, m, nbase + cc * 32, rowsB, v);
+                if (row_ok) epi_any<E>(ep, nio, m, nbase + cc * 32, rowsB, rs, v, sq);
             }
             tc_fence_before();
             mbar_arrive(&tempty[acc]);
@@ -352,7 +415,7 @@ static int g_sms_tc = 0;
 
 template <typename E>
 static int launch_tcp(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
-                      int* counters, cudaStream_t st) {
+                      int* counters, cudaStream_t st, const NormIO& nio) {
     if (M <= 0 || N <= 0) return LLAMA_OK;
     constexpr int smem = 1024 + kStagesTc * kStageBytes + (2 * kStagesTc + 4) * 8 + 16;
     static_assert(smem <= 227 * 1024, "shared memory per CTA");
@@ -378,15 +441,22 @@ static int launch_tcp(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, in
     int grid = 0;
     plan_tc(static_cast<int>(T), plan.KT, g_sms_tc, part != nullptr && counters != nullptr, &plan, &grid);
     if (plan.sk > kMaxTiles) { set_error("internal: %d split tiles exceed the counters", plan.sk); return LLAMA_ERR_INVALID_ARG; }
-    linear_tcp_kernel<E><<<grid, kThreadsTc, smem, st>>>(mapA->a128, mapW->b, M, N, plan, ep, part, counters);
+    linear_tcp_kernel<E><<<grid, kThreadsTc, smem, st>>>(mapA->a128, mapW->b, M, N, plan, ep, part, counters, nio);
     LLB_CHECK_LAUNCH("linear_tcp_kernel");
     return LLAMA_OK;
 }
 
 int linear16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, int dtype, const Epi& ep, float* part,
-                int* counters, cudaStream_t st) {
-    if (dtype == LLAMA_F16) return launch_tcp<f16>(mapA, mapW, M, N, K, ep, part, counters, st);
-    if (dtype == LLAMA_BF16) return launch_tcp<bf16>(mapA, mapW, M, N, K, ep, part, counters, st);
+                int* counters, cudaStream_t st, const NormIO* nio_in) {
+    NormIO nio = {};
+    if (nio_in) nio = *nio_in;
+    if (nio.ssq_out && (N % 128 || !nio.y_out || !nio.w_next || ep.mode != EPI_RESID_F32 || ep.ldo != N)) {
+        set_error("fused RMSNorm producer needs a residual epilogue over whole rows, N %% 128 == 0, y_out and w_next");
+        return LLAMA_ERR_INVALID_ARG;
+    }
+    if (nio.ssq_in && K % 64) { set_error("fused RMSNorm consumer needs K %% 64 == 0"); return LLAMA_ERR_INVALID_ARG; }
+    if (dtype == LLAMA_F16) return launch_tcp<f16>(mapA, mapW, M, N, K, ep, part, counters, st, nio);
+    if (dtype == LLAMA_BF16) return launch_tcp<bf16>(mapA, mapW, M, N, K, ep, part, counters, st, nio);
     set_error("16-bit projection: dtype must be LLAMA_BF16 or LLAMA_F16");
     return LLAMA_ERR_INVALID_ARG;
 }
@@ -394,8 +464,7 @@ int linear16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, i
 int linear16(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, int dtype, const Epi& ep, float* part,
              size_t part_bytes, int* counters, cudaStream_t st, bool pdl, const NormIO* nio) {
     if (M <= 64) return linear16_decode(mapA, mapW, M, N, K, dtype, ep, part, part_bytes, counters, st, pdl, nio);
-    if (nio && (nio->ssq_in || nio->ssq_out)) { set_error("fused RMSNorm is a decode-shape feature"); return LLAMA_ERR_INVALID_ARG; }
-    return linear16_tc(mapA, mapW, M, N, K, dtype, ep, part, counters, st);
+    return linear16_tc(mapA, mapW, M, N, K, dtype, ep, part, counters, st, nio);
 }
 
 }  // namespace llb

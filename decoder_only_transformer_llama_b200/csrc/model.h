@@ -158,6 +158,11 @@ struct Model {
     int* step_cnt;      // [kStepCounters] finish counters of the fused greedy pick (zero between steps)
     int* status;
     TmaMaps m_y, m_attn, m_g, m_ylast;   // activation maps (A box 128 rows, B box 16 rows)
+    // Tensor-memory prefill attention (16-bit, head_dim 128): q as [rows][nq]
+    // and every layer's K and V caches as [L * Bmax * nkv * S][hd], boxes of
+    // 64 columns x 128 rows.
+    CUtensorMap m_qtile, m_kcache, m_vcache;
+    bool has_attn_maps = false;
     cudaStream_t last_stream;
     Profile prof;
     // Timeline of decode launches: while tl_on, launch i of llama_decode_step
@@ -204,7 +209,7 @@ int linear_f32(const float* A, const float* W, int M, int N, int K, const Epi& e
 // Prefill-shaped projection; with part/counters (kGemmPartBytes, kMaxTiles
 // zeroed ints) the tail wave is split stream-K, without them whole tiles only.
 int linear16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, int dtype, const Epi& ep, float* part,
-                int* counters, cudaStream_t st);
+                int* counters, cudaStream_t st, const NormIO* nio = nullptr);
 int linear16_decode(const TmaMaps* mapX, const TmaMaps* mapW, int M, int N, int K, int dtype, const Epi& ep, float* part,
                     size_t part_bytes, int* counters, cudaStream_t st, bool pdl, const NormIO* nio = nullptr);
 // 16-bit projection: M <= 64 token rows -> linear16_decode, else linear16_tc.
@@ -213,6 +218,8 @@ int linear16(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, int 
 
 int launch_attention_prefill(const Model* m, int layer, const RowTable& rt, cudaStream_t st);
 int launch_attention_prefill_tc(const Model* m, int layer, const RowTable& rt, cudaStream_t st);
+bool attention_prefill_tmem_ok(const Model* m);
+int launch_attention_prefill_tmem(const Model* m, int layer, const RowTable& rt, cudaStream_t st);
 // wait_ns > 0 replaces the default wait limit; stall_unit >= 0: CTA 0 never
 // issues that unit's copies or their barrier signal (tests of the timeout).
 int launch_attention_decode(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st,
