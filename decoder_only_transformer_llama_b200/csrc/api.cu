@@ -599,7 +599,8 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B
                 long long stall_wait = 0;
                 take_stall(m, LLAMA_STALL_ATTENTION, &stall_unit, &stall_wait);
                 return launch_attention_decode(m, l, pos, B, st, chain, tl_next(m, TL_ATTENTION, 0), stall_wait,
-                                               stall_unit);
+                                               stall_unit, m->layers[l].wo,
+                                               static_cast<long long>(m->dim) * m->nq * m->esz);
             };
             LLB_TRY(block_forward_fused(m, l, B, nullptr, pos, attn, st, chain, true));
         }

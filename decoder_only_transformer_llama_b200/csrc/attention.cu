@@ -82,8 +82,6 @@ template <> struct Vec<f16, 4> {
 // its run (slot 0 = the run's first segment, slot 1 = its last); each writes
 // its unnormalised (o, max, sum) and the CTA that arrives last at the pair's
 // counter merges them in CTA order (deterministic).  No CTA waits for another.
-constexpr int kPrefetchUnits = 4;   // cache blocks per CTA pulled into L2 ahead of the grid dependency
-
 __device__ __forceinline__ long long run_begin64(long long c, long long W, long long P) { return c * W / P; }
 __device__ __forceinline__ int owner64(long long u, long long W, long long P) {
     return static_cast<int>(((u + 1) * P - 1) / W);
@@ -94,7 +92,8 @@ __global__ void __launch_bounds__(128)
 attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
                    const int32_t* __restrict__ pos, int B, int nkv, int nq, int S, long long row_stride,
                    float* __restrict__ part_o, float* __restrict__ part_ml, int* __restrict__ counters,
-                   T* __restrict__ out, int* status, unsigned long long* tl, long long wait_ns, int stall) {
+                   T* __restrict__ out, int* status, unsigned long long* tl, long long wait_ns, int stall,
+                   const void* __restrict__ next_w, long long next_w_bytes) {
     constexpr int EPL = HD / 32;   // head dims per lane
     constexpr int ROW = HD * static_cast<int>(sizeof(T));
     constexpr int CH_BYTES = kChunk * ROW;
@@ -145,70 +144,6 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
         if (b0 + 2 <= B) s_cum[b0 + 2] = before + t;
         __syncthreads();
     };
-    // Before the previous kernel (which writes this step's K/V row and q) has
-    // finished: plan with the positions as they read now and pull the first
-    // kPrefetchUnits cache blocks of this CTA's run into L2 (a prefetch only:
-    // nothing read here is used, and L2 is coherent with the writes that
-    // follow; the cap keeps the total far below the L2 size, so long runs do
-    // not evict their own blocks before use).  After the grid dependency has
-    // resolved, the positions are read again and the plan is redone if any
-    // changed.
-    make_plan();
-    {
-        const long long W0 = static_cast<long long>(s_cum[B]) * nkv;
-        const int P0 = static_cast<int>(W0 < gridDim.x ? W0 : gridDim.x);
-        if (threadIdx.x == 0 && blockIdx.x < P0) {
-            const long long v0 = run_begin64(blockIdx.x, W0, P0), v1 = run_begin64(blockIdx.x + 1, W0, P0);
-            int lo = 0, hi = B - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (static_cast<long long>(s_cum[mid]) * nkv <= v0) lo = mid; else hi = mid - 1;
-            }
-            int b = lo;
-            long long rem = v0 - static_cast<long long>(s_cum[lo]) * nkv;
-            int g = static_cast<int>(rem / s_nch[b]);
-            int jj = static_cast<int>(rem - static_cast<long long>(g) * s_nch[b]);
-            const long long v1p = v1 < v0 + kPrefetchUnits ? v1 : v0 + kPrefetchUnits;
-            for (long long u = v0; u < v1p && b < B; ++u) {
-                const int ctx = s_pos[b] + 1;
-                const int j0 = jj * kChunk;
-                const int n = min(kChunk, ctx - j0);
-                if (n > 0) {
-                    const long long ho = static_cast<long long>(b) * row_stride + static_cast<long long>(g) * S * HD +
-                                         static_cast<long long>(j0) * HD;
-                    bulk_prefetch_l2(kc + ho, n * ROW);
-                    bulk_prefetch_l2(vc + ho, n * ROW);
-                }
-                if (++jj >= s_nch[b]) {
-                    jj = 0;
-                    if (++g >= nkv) { g = 0; do { ++b; } while (b < B && s_nch[b] == 0); }
-                }
-            }
-        }
-    }
-    pdl_wait();
-    {
-        bool changed = false;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int b = 2 * threadIdx.x + e;
-            if (b < B) {
-                const int p = __ldcg(pos + b);
-                changed |= p != my_pos[e];
-                if ((p < 0 || p >= S) && blockIdx.x == 0) report_status(status, LLAMA_ERR_CAPACITY);
-            }
-        }
-        if (__syncthreads_or(changed)) make_plan();
-    }
-    const long long W = static_cast<long long>(s_cum[B]) * nkv;
-    const int P = static_cast<int>(W < gridDim.x ? W : gridDim.x), c = blockIdx.x;
-    if (c >= P) {
-        if (threadIdx.x == 0) tl_stamp(tl);
-        return;
-    }
-    const long long u0 = run_begin64(c, W, P), u1 = run_begin64(c + 1, W, P);
-    const int len = static_cast<int>(u1 - u0);
-
     // cursor over (row, kv head, chunk) starting at unit u
     struct Cur { int b, g, j; };
     auto cur_at = [&](long long u) {
@@ -235,8 +170,8 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
         return static_cast<long long>(r.b) * row_stride + static_cast<long long>(r.g) * S * HD;
     };
     const uint64_t wlim = wait_ns > 0 ? static_cast<uint64_t>(wait_ns) : kWaitLimitNs;
-    const int stall_i = c == 0 ? stall : -1;     // tests of the timeout path only
-    Cur icur = cur_at(u0);                       // issue cursor (thread 0)
+    const int stall_i = blockIdx.x == 0 ? stall : -1;   // tests of the timeout path only
+    Cur icur = {0, 0, 0};                        // issue cursor (thread 0)
     auto issue = [&](int i) {                    // i-th unit of this run into ring slot i % NSLOT
         const int ctx = s_pos[icur.b] + 1;
         const int j0 = icur.j * kChunk;
@@ -250,10 +185,83 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
         }
         advance(icur);
     };
+
+    // The weights of the projection that follows (constant during decode):
+    // this CTA's share is pulled into L2 while the cache reads below leave
+    // HBM mostly idle.
+    if (threadIdx.x == 0 && next_w_bytes > 0) {
+        const long long per = ((next_w_bytes / gridDim.x) + 15) & ~15LL;
+        const long long b0 = per * blockIdx.x;
+        const long long b1 = b0 + per < next_w_bytes ? b0 + per : next_w_bytes;
+        for (long long o = b0; o < b1; o += 32768)
+            bulk_prefetch_l2(static_cast<const uint8_t*>(next_w) + o, static_cast<uint32_t>(b1 - o < 32768 ? b1 - o : 32768));
+    }
     if (threadIdx.x == 0) {
         for (int k = 0; k < NSLOT; ++k) mbar_init(&bar[k], 1);
         fence_mbar_init();
-        for (int k = 0; k < NSLOT && k < len; ++k) issue(k);
+    }
+    // Before the previous kernel (which writes this step's K/V row and q) has
+    // finished: plan with the positions as they read now, and start the
+    // copies of this CTA's first units whose keys all lie before their row's
+    // new position.  Those cache entries are final: positions that already
+    // read as this step's were advanced by a kernel that ran after every
+    // earlier kernel had completed (each kernel of the chain waits for its
+    // predecessor before it writes), and the copies of the units holding a
+    // new position start only after the grid dependency.  After it has
+    // resolved, the positions are read again; if any changed, the early
+    // copies are drained, the ring re-armed and the plan redone.
+    make_plan();
+    int n_early = 0;                             // thread 0: units issued before the dependency
+    {
+        const long long W0 = static_cast<long long>(s_cum[B]) * nkv;
+        const int P0 = static_cast<int>(W0 < gridDim.x ? W0 : gridDim.x);
+        if (threadIdx.x == 0 && blockIdx.x < P0) {
+            const long long v0 = run_begin64(blockIdx.x, W0, P0), v1 = run_begin64(blockIdx.x + 1, W0, P0);
+            icur = cur_at(v0);
+            while (n_early < NSLOT && v0 + n_early < v1) {
+                const int j0 = icur.j * kChunk;
+                if (j0 + kChunk > s_pos[icur.b]) break;   // holds the new position: wait for its writer
+                issue(n_early++);
+            }
+        }
+    }
+    pdl_wait();
+    {
+        bool changed = false;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int b = 2 * threadIdx.x + e;
+            if (b < B) {
+                const int p = __ldcg(pos + b);
+                changed |= p != my_pos[e];
+                if ((p < 0 || p >= S) && blockIdx.x == 0) report_status(status, LLAMA_ERR_CAPACITY);
+            }
+        }
+        if (__syncthreads_or(changed)) {
+            if (threadIdx.x == 0) {
+                for (int k = 0; k < n_early; ++k)
+                    if (k != stall_i) mbar_wait(&bar[k], 0, wlim);
+                for (int k = 0; k < NSLOT; ++k) {
+                    mbar_inval(&bar[k]);
+                    mbar_init(&bar[k], 1);
+                }
+                fence_mbar_init();
+                n_early = 0;
+            }
+            make_plan();
+        }
+    }
+    const long long W = static_cast<long long>(s_cum[B]) * nkv;
+    const int P = static_cast<int>(W < gridDim.x ? W : gridDim.x), c = blockIdx.x;
+    if (c >= P) {
+        if (threadIdx.x == 0) tl_stamp(tl);
+        return;
+    }
+    const long long u0 = run_begin64(c, W, P), u1 = run_begin64(c + 1, W, P);
+    const int len = static_cast<int>(u1 - u0);
+    if (threadIdx.x == 0) {
+        if (n_early == 0) icur = cur_at(u0);
+        for (int k = n_early; k < NSLOT && k < len; ++k) issue(k);
     }
     const float scale = rsqrtf(static_cast<float>(HD));
     Cur cur = cur_at(u0);
@@ -441,7 +449,7 @@ static int g_attn_sms = 0;
 
 template <typename T, int HD, int NREP>
 static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl,
-                     unsigned long long* tl, long long wait_ns, int stall) {
+                     unsigned long long* tl, long long wait_ns, int stall, const void* next_w, long long next_w_bytes) {
     const T* kc = static_cast<const T*>(m->kc) + layer * m->kv_layer_elems;
     const T* vc = static_cast<const T*>(m->vc) + layer * m->kv_layer_elems;
     auto kern = attn_decode_kernel<T, HD, NREP>;
@@ -469,7 +477,8 @@ static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaS
     P = std::max<long long>(P, 1);
     cudaError_t e = launch_k(kern, dim3(static_cast<unsigned>(P)), dim3(128), smem, st, pdl, static_cast<const T*>(m->q),
                              kc, vc, pos, B, m->nkv, m->nq, m->S, m->kv_row_elems, m->part_o, m->part_ml,
-                             m->attn_cnt, static_cast<T*>(m->attn), m->status, tl, wait_ns, stall);
+                             m->attn_cnt, static_cast<T*>(m->attn), m->status, tl, wait_ns, stall, next_w,
+                             next_w_bytes);
     count_launch();
     if (e != cudaSuccess) return cuda_fail(e, "attn_decode_kernel");
     return LLAMA_OK;
@@ -477,12 +486,12 @@ static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaS
 
 template <typename T, int HD>
 static int decode_rep(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl,
-                      unsigned long long* tl, long long wait_ns, int stall) {
+                      unsigned long long* tl, long long wait_ns, int stall, const void* nw, long long nwb) {
     switch (m->n_rep) {
-        case 1: return decode_go<T, HD, 1>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
-        case 2: return decode_go<T, HD, 2>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
-        case 4: return decode_go<T, HD, 4>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
-        case 8: return decode_go<T, HD, 8>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+        case 1: return decode_go<T, HD, 1>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, nw, nwb);
+        case 2: return decode_go<T, HD, 2>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, nw, nwb);
+        case 4: return decode_go<T, HD, 4>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, nw, nwb);
+        case 8: return decode_go<T, HD, 8>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, nw, nwb);
     }
     set_error("n_heads / n_kv_heads = %d unsupported (1, 2, 4, 8)", m->n_rep);
     return LLAMA_ERR_INVALID_ARG;
@@ -490,21 +499,23 @@ static int decode_rep(const Model* m, int layer, const int32_t* pos, int B, cuda
 
 template <typename T>
 static int decode_hd(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl,
-                     unsigned long long* tl, long long wait_ns, int stall) {
+                     unsigned long long* tl, long long wait_ns, int stall, const void* nw, long long nwb) {
     switch (m->hd) {
-        case 32: return decode_rep<T, 32>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
-        case 64: return decode_rep<T, 64>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
-        case 128: return decode_rep<T, 128>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+        case 32: return decode_rep<T, 32>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, nw, nwb);
+        case 64: return decode_rep<T, 64>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, nw, nwb);
+        case 128: return decode_rep<T, 128>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, nw, nwb);
     }
     set_error("head_dim %d unsupported", m->hd);
     return LLAMA_ERR_INVALID_ARG;
 }
 
 int launch_attention_decode(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl,
-                            unsigned long long* tl, long long wait_ns, int stall) {
-    if (m->dtype == LLAMA_BF16) return decode_hd<bf16>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
-    if (m->dtype == LLAMA_F16) return decode_hd<f16>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
-    return decode_hd<float>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+                            unsigned long long* tl, long long wait_ns, int stall, const void* next_w,
+                            long long next_w_bytes) {
+    if (next_w_bytes % 16 || (reinterpret_cast<uintptr_t>(next_w) & 15)) { next_w = nullptr; next_w_bytes = 0; }
+    if (m->dtype == LLAMA_BF16) return decode_hd<bf16>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, next_w, next_w_bytes);
+    if (m->dtype == LLAMA_F16) return decode_hd<f16>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, next_w, next_w_bytes);
+    return decode_hd<float>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, next_w, next_w_bytes);
 }
 
 // ---------------------------------------------------------------- prefill

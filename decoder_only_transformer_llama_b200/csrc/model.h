@@ -222,9 +222,11 @@ bool attention_prefill_tmem_ok(const Model* m);
 int launch_attention_prefill_tmem(const Model* m, int layer, const RowTable& rt, cudaStream_t st);
 // wait_ns > 0 replaces the default wait limit; stall_unit >= 0: CTA 0 never
 // issues that unit's copies or their barrier signal (tests of the timeout).
+// next_w / next_w_bytes: weights of the projection that follows, pulled into
+// L2 by the CTAs at their start (16-byte aligned; null = none).
 int launch_attention_decode(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st,
                             bool pdl = false, unsigned long long* tl = nullptr, long long wait_ns = 0,
-                            int stall_unit = -1);
+                            int stall_unit = -1, const void* next_w = nullptr, long long next_w_bytes = 0);
 
 int launch_argmax(const float* logits, int B, int V, int32_t* out, int32_t* tokens_adv,
                   int32_t* pos_adv, cudaStream_t st, bool pdl = false, unsigned long long* tl = nullptr);

@@ -25,14 +25,15 @@ def llb(cuda_device):
 
 
 def _run(llb, shape, B, T, lens, steps, rows, seed_idx, start_pos=0, tol=BF16_TOL, gap=1e-2,
-         storage_bound=False):
+         storage_bound=False, storage_gap=False):
     """Prefill B prompts (right-padded to T, real lengths `lens`), then `steps`
     greedy decode steps at per-row positions; the oracle recomputes `rows`
     teacher-forced on the GPU's tokens.  With `storage_bound`, the oracle runs
     each row a second time with bfloat16 storage (store=round_bf16) and the
     bounds become that storage error's on these very weights and tokens:
     rel-L2 <= 1.5 x rel-L2(rounded, exact), greedy ids equal where the top-2
-    gap exceeds 8 x the RMS of (rounded - exact)."""
+    gap exceeds 8 x the RMS of (rounded - exact).  With `storage_gap` only the
+    greedy gap is taken from it (the rel-L2 bound stays `tol`)."""
     s = shape
     w = make_weights(s, weight_seed(seed_idx), device="cuda")
     m = build_model(s, w)
@@ -63,11 +64,12 @@ def _run(llb, shape, B, T, lens, steps, rows, seed_idx, start_pos=0, tol=BF16_TO
         positions = list(range(L - 1, L + steps))
         want = O.forward(args, lw, seqs[b], 0, O.new_cache(args), logits_positions=positions)
         g = np.stack(got[b])
-        if storage_bound:
+        if storage_bound or storage_gap:
             rounded = O.forward(args, lw, seqs[b], 0, O.new_cache(args), logits_positions=positions,
                                 store=O.round_bf16)
             storage = rel_l2(rounded, want)
-            tol = 1.5 * storage
+            if storage_bound:
+                tol = 1.5 * storage
             gap = 8.0 * float(np.sqrt(np.mean((rounded - want) ** 2)))
             print(f"row {b}: bf16 storage error of the oracle {storage:.3e}; GPU to the bf16-storage oracle "
                   f"{rel_l2(g, rounded):.3e}")
@@ -105,12 +107,17 @@ def test_7b_full_depth_benchmark_configuration(llb):
 def test_13b_dims_ragged_prefill_then_decode(llb):
     """13B layer dimensions, 16 prompts of seeded lengths in [64, 1024]
     right-padded to a rectangle, then the workload's 128 greedy decode steps
-    at per-row positions; oracle on the shortest and the longest row."""
+    at per-row positions; oracle on the shortest and the longest row.  Logits
+    within rel-L2 2e-2 at every step.  Over 128 teacher-forced steps some
+    oracle top-2 gaps fall below what bf16 storage of the cache and
+    activations can resolve (RMS logit error ~1.6e-2 here, so gaps of a few
+    hundredths can flip), so greedy ids must agree where the gap exceeds
+    8 x the RMS of the oracle's own bf16-storage error on these rows."""
     s = L13B.replace(n_layers=2)
     lens = make_lengths(16, 64, 1024, token_seed(3))
     T = max(lens)
     order = sorted(range(16), key=lambda b: lens[b])
-    _run(llb, s, B=16, T=T, lens=lens, steps=128, rows=[order[0], order[-1]], seed_idx=3)
+    _run(llb, s, B=16, T=T, lens=lens, steps=128, rows=[order[0], order[-1]], seed_idx=3, storage_gap=True)
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f16"])
