@@ -40,7 +40,8 @@ EXPORTED = ("llama_model_bytes", "llama_model_create", "llama_set_weight", "llam
             "llama_model_destroy", "llama_last_error", "llama_launch_count",
             "llama_op_rmsnorm", "llama_op_linear", "llama_op_linear_workspace_bytes", "llama_op_linear_noalloc",
             "llama_profile_start", "llama_profile_stop", "llama_token_logprobs", "llama_timeline_start",
-            "llama_timeline_stop", "llama_debug_stall")
+            "llama_timeline_stop", "llama_debug_stall", "llama_model_bytes_tp", "llama_model_create_tp",
+            "llama_tp_prefill_all", "llama_tp_decode_step_all", "llama_tp_buffers", "llama_tp_bind")
 LLAMA_STALL_NONE, LLAMA_STALL_PROJECTION, LLAMA_STALL_ATTENTION = 0, 1, 2
 TIMELINE_KINDS = {0: "embed", 1: "projection", 2: "attention", 3: "sample", 4: "rmsnorm"}
 
@@ -101,6 +102,15 @@ _sig("llama_timeline_start", _i, [_vp, _vp])
 _sig("llama_timeline_stop", _i, [_vp, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_int32),
                                  ctypes.POINTER(ctypes.c_int64), _i, ctypes.POINTER(ctypes.c_int)])
 _sig("llama_debug_stall", _i, [_vp, _i, _i, ctypes.c_int64])
+_sig("llama_model_bytes_tp", _i, [ctypes.POINTER(ModelArgs), _i, _i, ctypes.POINTER(_sz), ctypes.POINTER(_sz),
+                                  ctypes.POINTER(_sz), ctypes.POINTER(_sz), ctypes.POINTER(ctypes.c_int32)])
+_sig("llama_model_create_tp", _i, [ctypes.POINTER(ModelArgs), _i, _i, _vp, _sz, _vp, ctypes.POINTER(_vp)])
+_sig("llama_tp_prefill_all", _i, [ctypes.POINTER(_vp), _i, _vp, ctypes.POINTER(ctypes.c_int32), _i, _i, _i, _vp, _i,
+                                  _vp])
+_sig("llama_tp_decode_step_all", _i, [ctypes.POINTER(_vp), _i, _vp, _vp, _i, ctypes.POINTER(Sampling), _vp, _vp, _vp,
+                                      _i, _vp])
+_sig("llama_tp_buffers", _i, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_vp)])
+_sig("llama_tp_bind", _i, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_vp)])
 _sig("llama_profile_start", _i, [_vp, _i])
 _sig("llama_profile_stop", _i, [_vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int64),
                                 ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int32), _i,
@@ -152,11 +162,13 @@ def args_from_shape(s) -> ModelArgs:
                      s.max_tokens, s.dtype)
 
 
-def model_bytes(args: ModelArgs) -> dict:
+def model_bytes(args: ModelArgs, tp_rank: int = 0, tp_size: int = 1) -> dict:
+    """Arena sizes of a model, or of shard tp_rank of a tensor-parallel group
+    of tp_size ranks ("hidden" is then the shard's FFN width)."""
     w, kv, ws, tot = _sz(), _sz(), _sz(), _sz()
     h = ctypes.c_int32()
-    _check(_lib.llama_model_bytes(ctypes.byref(args), ctypes.byref(w), ctypes.byref(kv), ctypes.byref(ws),
-                                  ctypes.byref(tot), ctypes.byref(h)))
+    _check(_lib.llama_model_bytes_tp(ctypes.byref(args), tp_rank, tp_size, ctypes.byref(w), ctypes.byref(kv),
+                                     ctypes.byref(ws), ctypes.byref(tot), ctypes.byref(h)))
     return {"weights": w.value, "kv": kv.value, "workspace": ws.value, "total": tot.value, "hidden": h.value}
 
 
@@ -180,14 +192,15 @@ def _dev(t, dtype: str, numel: int, name: str, device=None):
 class Model:
     """A model laid out in one torch-allocated device arena."""
 
-    def __init__(self, args: ModelArgs, device="cuda", stream=None):
+    def __init__(self, args: ModelArgs, device="cuda", stream=None, tp_rank: int = 0, tp_size: int = 1):
         import torch
         self.args = args
-        self.sizes = model_bytes(args)
+        self.tp_rank, self.tp_size = tp_rank, tp_size
+        self.sizes = model_bytes(args, tp_rank, tp_size)
         self.arena = torch.empty(self.sizes["total"], dtype=torch.uint8, device=device)
         h = _vp()
-        _check(_lib.llama_model_create(ctypes.byref(args), self.arena.data_ptr(), self.sizes["total"],
-                                       _stream(stream), ctypes.byref(h)))
+        _check(_lib.llama_model_create_tp(ctypes.byref(args), tp_rank, tp_size, self.arena.data_ptr(),
+                                          self.sizes["total"], _stream(stream), ctypes.byref(h)))
         self.handle = h
 
     def close(self):
@@ -214,12 +227,14 @@ class Model:
 
     def _weight_numel(self, name: str) -> int:
         a = self.args
+        t = getattr(self, "tp_size", 1)
         hd = a.dim // a.n_heads
-        nkv = a.n_kv_heads or a.n_heads
+        nh = a.n_heads // t
+        nkv = (a.n_kv_heads or a.n_heads) // t
         H = self.sizes["hidden"]
-        return {"tok_embeddings": a.vocab_size * a.dim, "output": a.vocab_size * a.dim, "norm": a.dim,
-                "attention_norm": a.dim, "ffn_norm": a.dim, "wq": a.n_heads * hd * a.dim,
-                "wk": nkv * hd * a.dim, "wv": nkv * hd * a.dim, "wo": a.dim * a.n_heads * hd,
+        return {"tok_embeddings": a.vocab_size * a.dim, "output": a.vocab_size // t * a.dim, "norm": a.dim,
+                "attention_norm": a.dim, "ffn_norm": a.dim, "wq": nh * hd * a.dim,
+                "wk": nkv * hd * a.dim, "wv": nkv * hd * a.dim, "wo": a.dim * nh * hd,
                 "w1": H * a.dim, "w2": a.dim * H, "w3": H * a.dim}[name]
 
     def load(self, weights: dict, stream=None):
@@ -336,6 +351,64 @@ class Model:
         s = ctypes.c_int()
         _check(_lib.llama_model_status(self.handle, ctypes.byref(s)))
         return s.value
+
+
+class TPGroup:
+    """Every rank of a tensor-parallel group on one GPU (llama_tp_*_all):
+    shards[r] holds rank r's slices of the weights (decoder_only_transformer_llama_b200.tp)."""
+
+    def __init__(self, args: ModelArgs, tp_size: int, device="cuda"):
+        self.args = args
+        self.tp_size = tp_size
+        self.shards = [Model(args, device=device, tp_rank=r, tp_size=tp_size) for r in range(tp_size)]
+        self.device = self.shards[0].arena.device
+        self._h = (_vp * tp_size)(*[s.handle for s in self.shards])
+
+    def load(self, weights: dict, shape):
+        """Upload a whole (unsharded) weight dict, cut per rank by tp.shard_weights."""
+        from . import tp as _tp
+        for r, s in enumerate(self.shards):
+            part = _tp.shard_weights(weights, _tp.plan_for(shape, r, self.tp_size))
+            s.load({"tok_embeddings": part["tok_embeddings"].contiguous(), "norm": part["norm"].contiguous(),
+                    "output": part["output"].contiguous(),
+                    "layers": [{k: v.contiguous() for k, v in layer.items()} for layer in part["layers"]]})
+
+    def prefill(self, tokens, lens=None, start_pos: int = 0, logits=None, all_logits: bool = False, stream=None):
+        B, T = tokens.shape
+        _dev(tokens, "int32", B * T, "tokens", self.device)
+        lens_arr = (ctypes.c_int32 * B)(*[int(v) for v in lens]) if lens is not None else None
+        if logits is not None:
+            rows = (sum(int(v) for v in lens) if lens is not None else B * T) if all_logits else B
+            _dev(logits, "float32", rows * self.args.vocab_size, "logits", self.device)
+        _check(_lib.llama_tp_prefill_all(self._h, self.tp_size, tokens.data_ptr(), lens_arr, B, T, start_pos,
+                                         _ptr(logits), 1 if all_logits else 0, _stream(stream)))
+        return logits
+
+    def decode_step(self, tokens, pos, temperature: Optional[float] = None, top_p: float = 0.9, uniforms=None,
+                    next_tokens=None, logits=None, advance: bool = False, stream=None):
+        B = tokens.shape[0]
+        _dev(tokens, "int32", B, "tokens", self.device)
+        _dev(pos, "int32", B, "pos", self.device)
+        if uniforms is not None:
+            _dev(uniforms, "float32", B, "uniforms", self.device)
+        if next_tokens is not None:
+            _dev(next_tokens, "int32", B, "next_tokens", self.device)
+        if logits is not None:
+            _dev(logits, "float32", B * self.args.vocab_size, "logits", self.device)
+        samp = Sampling(float(temperature), float(top_p)) if temperature is not None else None
+        _check(_lib.llama_tp_decode_step_all(self._h, self.tp_size, tokens.data_ptr(), pos.data_ptr(), B,
+                                             ctypes.byref(samp) if samp is not None else None, _ptr(uniforms),
+                                             _ptr(next_tokens), _ptr(logits),
+                                             LLAMA_DECODE_ADVANCE if advance else 0, _stream(stream)))
+        return next_tokens
+
+    def status(self) -> int:
+        codes = [s.status() for s in self.shards]
+        return next((c for c in codes if c), 0)
+
+    def close(self):
+        for s in self.shards:
+            s.close()
 
 
 def sample(logits, temperature: float, top_p: float, uniforms, out, stream=None):

@@ -46,18 +46,26 @@ static size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255);
 
 // Sizes and offsets of everything in the arena.
 struct Layout {
-    int dim, L, nh, nkv, hd, n_rep, H, V, S, Bmax, Mmax, Mrows, Brows, dtype, esz, nq, nkvc, nqkv, n_splits;
+    int dim, L, nh, nkv, hd, n_rep, H, V, Vl, S, Bmax, Mmax, Mrows, Brows, dtype, esz, nq, nkvc, nqkv, n_splits;
+    int tp_rank, tp_size;
     size_t off_tok_emb, off_norm, off_output, layer_bytes;
     size_t l_attn_norm, l_wqkv, l_wo, l_ffn_norm, l_w13, l_w2;
     size_t off_layers, weight_bytes;
     size_t off_kc, off_vc, kv_bytes;
     size_t off_x, off_y, off_q, off_attn, off_g, off_ylast, off_tok_ids, off_tok_row, off_tok_pos, off_last,
         off_logits, off_part_o, off_part_ml, off_attn_cnt, off_status, off_rope, off_gemm_part, off_gemm_cnt,
-        off_ssq, off_tl, off_best, off_step_cnt, ws_end;
+        off_ssq, off_tl, off_best, off_step_cnt, off_tp_part, off_tp_flag, ws_end;
 };
 
-static int make_layout(const llama_model_args* a, Layout* o) {
+// Sizes and offsets of one model, or of shard tp_rank of a tensor-parallel
+// group of tp_size: local query/KV heads, FFN hidden features and vocabulary
+// rows are 1/tp_size of the model's (the sharding of Admin Guide §1.3 / §4.2).
+static int make_layout(const llama_model_args* a, Layout* o, int tp_rank = 0, int tp_size = 1) {
     if (!a) { set_error("args is NULL"); return LLAMA_ERR_INVALID_ARG; }
+    if (tp_size < 1 || tp_size > kMaxTp || tp_rank < 0 || tp_rank >= tp_size) {
+        set_error("tensor-parallel rank %d of %d invalid (at most %d ranks)", tp_rank, tp_size, kMaxTp);
+        return LLAMA_ERR_INVALID_ARG;
+    }
     if (a->dim <= 0 || a->n_layers <= 0 || a->n_heads <= 0 || a->vocab_size <= 0 || a->multiple_of <= 0 ||
         a->max_seq_len <= 0 || a->max_batch_size <= 0 || a->n_kv_heads < 0 || a->max_tokens < 0) {
         set_error("non-positive size in llama_model_args");
@@ -77,11 +85,22 @@ static int make_layout(const llama_model_args* a, Layout* o) {
     if (hd != 32 && hd != 64 && hd != 128) { set_error("head_dim %d unsupported (32, 64, 128)", hd); return LLAMA_ERR_INVALID_ARG; }
     if (a->dim % 64) { set_error("dim must be a multiple of 64"); return LLAMA_ERR_INVALID_ARG; }
     if (a->max_batch_size > kMaxRows) { set_error("max_batch_size > %d", kMaxRows); return LLAMA_ERR_INVALID_ARG; }
-    const int H = hidden_dim(a->dim, a->multiple_of, a->ffn_dim_multiplier);
-    if (H % 64) { set_error("FFN hidden %d must be a multiple of 64", H); return LLAMA_ERR_INVALID_ARG; }
+    const int H_full = hidden_dim(a->dim, a->multiple_of, a->ffn_dim_multiplier);
+    if (H_full % 64) { set_error("FFN hidden %d must be a multiple of 64", H_full); return LLAMA_ERR_INVALID_ARG; }
+    if (tp_size > 1) {
+        if (a->dtype == LLAMA_F32) { set_error("tensor parallelism runs 16-bit models"); return LLAMA_ERR_INVALID_ARG; }
+        if (a->n_heads % tp_size || nkv % tp_size || H_full % tp_size || a->vocab_size % tp_size ||
+            (H_full / tp_size) % 64) {
+            set_error("n_heads, n_kv_heads, vocab_size and the FFN hidden width (in multiples of 64) must split "
+                      "evenly over %d ranks", tp_size);
+            return LLAMA_ERR_INVALID_ARG;
+        }
+    }
+    const int H = H_full / tp_size;
     {
-        const long long widest = std::max(std::max(static_cast<long long>(a->vocab_size), 2LL * H),
-                                          static_cast<long long>(a->dim) + 2LL * nkv * (a->dim / a->n_heads) + a->dim);
+        const long long nq_l = static_cast<long long>(a->n_heads / tp_size) * (a->dim / a->n_heads);
+        const long long widest = std::max(std::max(static_cast<long long>(a->vocab_size / tp_size), 2LL * H),
+                                          nq_l + 2LL * (nkv / tp_size) * (a->dim / a->n_heads));
         if ((widest + 127) / 128 > kMaxTiles) { set_error("a projection is wider than %d x 128 rows", kMaxTiles); return LLAMA_ERR_INVALID_ARG; }
     }
     if (a->dtype != LLAMA_F32 && (a->dim < 256 || a->vocab_size < 256 || a->dim % 128)) {
@@ -89,21 +108,22 @@ static int make_layout(const llama_model_args* a, Layout* o) {
         return LLAMA_ERR_INVALID_ARG;
     }
     Layout& l = *o;
-    l.dim = a->dim; l.L = a->n_layers; l.nh = a->n_heads; l.nkv = nkv; l.hd = hd; l.n_rep = n_rep; l.H = H;
-    l.V = a->vocab_size; l.S = a->max_seq_len; l.Bmax = a->max_batch_size; l.dtype = a->dtype;
+    l.dim = a->dim; l.L = a->n_layers; l.nh = a->n_heads / tp_size; l.nkv = nkv / tp_size; l.hd = hd; l.n_rep = n_rep;
+    l.H = H; l.V = a->vocab_size; l.Vl = a->vocab_size / tp_size; l.tp_rank = tp_rank; l.tp_size = tp_size;
+    l.S = a->max_seq_len; l.Bmax = a->max_batch_size; l.dtype = a->dtype;
     l.esz = a->dtype == LLAMA_F32 ? 4 : 2;
     const long long mt = a->max_tokens ? a->max_tokens : 1LL * a->max_batch_size * a->max_seq_len;
     if (mt > (1LL << 30)) { set_error("max_tokens too large"); return LLAMA_ERR_INVALID_ARG; }
     l.Mmax = static_cast<int>(mt > l.Bmax ? mt : l.Bmax);
     l.Mrows = l.Mmax < 128 ? 128 : l.Mmax;    // activation buffers hold whole 128-row tiles
     l.Brows = l.Bmax < 128 ? 128 : l.Bmax;
-    l.nq = l.nh * hd; l.nkvc = nkv * hd; l.nqkv = l.nq + 2 * l.nkvc;
+    l.nq = l.nh * hd; l.nkvc = l.nkv * hd; l.nqkv = l.nq + 2 * l.nkvc;
     l.n_splits = (l.S + kChunk - 1) / kChunk;
     const size_t e = l.esz, D = l.dim;
     size_t off = 0;
     l.off_tok_emb = off; off = align256(off + static_cast<size_t>(l.V) * D * e);
     l.off_norm = off; off = align256(off + D * 4);
-    l.off_output = off; off = align256(off + static_cast<size_t>(l.V) * D * e);
+    l.off_output = off; off = align256(off + static_cast<size_t>(l.Vl) * D * e);
     l.off_layers = off;
     size_t lo = 0;
     l.l_attn_norm = lo; lo = align256(lo + D * 4);
@@ -115,7 +135,7 @@ static int make_layout(const llama_model_args* a, Layout* o) {
     l.layer_bytes = lo;
     off += lo * l.L;
     l.weight_bytes = off;
-    const size_t kv_one = static_cast<size_t>(l.L) * l.Bmax * nkv * l.S * hd * e;
+    const size_t kv_one = static_cast<size_t>(l.L) * l.Bmax * l.nkv * l.S * hd * e;
     l.off_kc = off; off = align256(off + kv_one);
     l.off_vc = off; off = align256(off + kv_one);
     l.kv_bytes = off - l.weight_bytes;
@@ -134,7 +154,7 @@ static int make_layout(const llama_model_args* a, Layout* o) {
     const size_t slots = static_cast<size_t>(2) * kMaxAttnCtas * n_rep;   // decode attention partials
     l.off_part_o = off; off = align256(off + slots * hd * 4);
     l.off_part_ml = off; off = align256(off + slots * 2 * 4);
-    l.off_attn_cnt = off; off = align256(off + static_cast<size_t>(l.Bmax) * nkv * 4);
+    l.off_attn_cnt = off; off = align256(off + static_cast<size_t>(l.Bmax) * l.nkv * 4);
     l.off_status = off; off = align256(off + 16);
     l.off_rope = off; off = align256(off + static_cast<size_t>(l.S) * (hd / 2) * 8);
     l.off_gemm_part = off; off = align256(off + (a->dtype != LLAMA_F32 ? kGemmPartBytes : 0));
@@ -143,6 +163,8 @@ static int make_layout(const llama_model_args* a, Layout* o) {
     l.off_tl = off; off = align256(off + static_cast<size_t>(kTimelineCap) * 8);
     l.off_best = off; off = align256(off + static_cast<size_t>(l.Bmax) * 8);
     l.off_step_cnt = off; off = align256(off + kStepCounters * sizeof(int));
+    l.off_tp_part = off; off = align256(off + (tp_size > 1 ? 2 * M * D * 4 : 0));
+    l.off_tp_flag = off; off = align256(off + (kMaxTp + 2) * 8 + 16);
     l.ws_end = off;
     return LLAMA_OK;
 }
@@ -330,6 +352,196 @@ static int block_forward(Model* m, int l, int M, const int* tok_row, const int* 
     return LLAMA_OK;
 }
 
+// ---------------------------------------------------------------- tensor parallelism
+// The shards one call runs: every rank of a group on this GPU, or this rank
+// alone (its peers on other GPUs, reached through the bound buffers).
+struct Shards {
+    Model* m[kMaxTp];
+    int n;
+};
+
+static TpSync tp_sync_of(const Model* m) {
+    TpSync s = {};
+    s.wait = m->tp_wait ? 1 : 0;
+    s.rank = m->tp_rank;
+    s.size = m->tp_size;
+    s.my_flags = m->tp_flag;
+    for (int q = 0; q < m->tp_size; ++q) s.peer_flags[q] = m->peers.flag[q];
+    s.epoch = m->tp_epoch;
+    s.arrivals = m->tp_arrivals;
+    s.status = m->status;
+    return s;
+}
+
+// x += the partial sums of phase `parity` of every rank, then the next
+// RMSNorm's inputs, on every shard of `sh`.
+static int tp_reduce_all(const Shards& sh, int parity, int M, const float* const* w_next, cudaStream_t st) {
+    for (int i = 0; i < sh.n; ++i) {
+        const Model* m = sh.m[i];
+        const float* parts[kMaxTp];
+        for (int r = 0; r < m->tp_size; ++r) parts[r] = m->peers.part[r][parity];
+        LLB_TRY(launch_tp_reduce(m, parts, M, w_next[i], tp_sync_of(m), st));
+    }
+    return LLAMA_OK;
+}
+
+// One transformer block of a tensor-parallel group (Admin Guide §8.4
+// TransformerBlock, sharded as §1.3 / §4.2): each shard computes its query
+// and KV heads (wq/wk/wv, RoPE, cache append, attention) and its slice of
+// wo's input columns, leaving a partial residual update; the reduce adds the
+// ranks' updates to x and writes the FFN norm's inputs; each shard computes
+// its SwiGLU features (w1/w3) and its slice of w2's input columns; a second
+// reduce finishes the block.  M token rows; per-shard token maps.
+template <typename AttnFn>
+static int tp_block(const Shards& sh, int l, int M, bool prefill, const int32_t* pos, AttnFn attn, cudaStream_t st) {
+    for (int i = 0; i < sh.n; ++i) {
+        Model* m = sh.m[i];
+        LayerPtrs& Lp = m->layers[l];
+        const NormIO n_in = {m->ssq, m->dim / 128, m->a.norm_eps, nullptr, nullptr, nullptr};
+        Epi ep = base_epi(m);
+        ep.mode = EPI_QKV;
+        ep.q = m->q;
+        ep.kc = static_cast<char*>(m->kc) + l * m->kv_layer_elems * m->esz;
+        ep.vc = static_cast<char*>(m->vc) + l * m->kv_layer_elems * m->esz;
+        ep.tok_row = prefill ? m->tok_row : nullptr;
+        ep.tok_pos = prefill ? m->tok_pos : pos;
+        LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.wqkv, &Lp.m_wqkv, M, m->nqkv, m->dim, ep, st, false, &n_in));
+        LLB_TRY(attn(m));
+        Epi ew = base_epi(m);
+        ew.mode = EPI_STORE_F32;
+        ew.out = m->tp_part[0];
+        ew.ldo = m->dim;
+        LLB_TRY(run_linear(m, m->dtype, m->attn, &m->m_attn, Lp.wo, &Lp.m_wo, M, m->dim, m->nq, ew, st));
+    }
+    const float* ffn_norm[kMaxTp];
+    for (int i = 0; i < sh.n; ++i) ffn_norm[i] = sh.m[i]->layers[l].ffn_norm;
+    LLB_TRY(tp_reduce_all(sh, 0, M, ffn_norm, st));
+    for (int i = 0; i < sh.n; ++i) {
+        Model* m = sh.m[i];
+        LayerPtrs& Lp = m->layers[l];
+        const NormIO n_in = {m->ssq, m->dim / 128, m->a.norm_eps, nullptr, nullptr, nullptr};
+        Epi es = base_epi(m);
+        es.mode = EPI_SWIGLU;
+        es.g = m->g;
+        LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, Lp.w13, &Lp.m_w13, M, 2 * m->H, m->dim, es, st, false, &n_in));
+        Epi ew = base_epi(m);
+        ew.mode = EPI_STORE_F32;
+        ew.out = m->tp_part[1];
+        ew.ldo = m->dim;
+        LLB_TRY(run_linear(m, m->dtype, m->g, &m->m_g, Lp.w2, &Lp.m_w2, M, m->dim, m->H, ew, st));
+    }
+    const float* next_norm[kMaxTp];
+    for (int i = 0; i < sh.n; ++i)
+        next_norm[i] = l + 1 < sh.m[i]->L ? sh.m[i]->layers[l + 1].attn_norm : sh.m[i]->norm;
+    return tp_reduce_all(sh, 1, M, next_norm, st);
+}
+
+// The vocabulary projection of a group: shard r writes logits columns
+// [r * Vl, (r + 1) * Vl) of `out` ([rows, V]); with the shards on separate
+// GPUs each writes its own logits buffer, gathers the others' slices and
+// copies the rows to `out`.
+static int tp_logits(const Shards& sh, int rows, bool last_rows, float* out, cudaStream_t st) {
+    for (int i = 0; i < sh.n; ++i) {
+        Model* m = sh.m[i];
+        const bool remote = m->tp_wait;
+        float* dst = remote ? m->logits_ws : out;
+        Epi eo = base_epi(m);
+        eo.mode = EPI_STORE_F32;
+        eo.out = dst + static_cast<size_t>(m->tp_rank) * m->Vl;
+        eo.ldo = m->V;
+        if (last_rows) {
+            LLB_TRY(launch_rmsnorm(m->x, m->last_idx, m->norm, rows, m->dim, m->a.norm_eps, m->ylast, m->dtype, st));
+            LLB_TRY(run_linear(m, m->dtype, m->ylast, &m->m_ylast, m->output, &m->m_output, rows, m->Vl, m->dim, eo, st));
+        } else {
+            const NormIO n_in = {m->ssq, m->dim / 128, m->a.norm_eps, nullptr, nullptr, nullptr};
+            LLB_TRY(run_linear(m, m->dtype, m->y, &m->m_y, m->output, &m->m_output, rows, m->Vl, m->dim, eo, st, false,
+                               &n_in));
+        }
+        if (remote) {
+            LLB_TRY(launch_tp_gather_logits(m, m->logits_ws, rows, tp_sync_of(m), st));
+            if (out && out != m->logits_ws) {
+                cudaError_t e = cudaMemcpyAsync(out, m->logits_ws, static_cast<size_t>(rows) * m->V * 4,
+                                                cudaMemcpyDeviceToDevice, st);
+                if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(tp logits)");
+            }
+        }
+    }
+    return LLAMA_OK;
+}
+
+static int tp_prefill(const Shards& sh, const RowTable& rt, const int32_t* tokens, float* logits, int logits_mode,
+                      cudaStream_t st) {
+    const int M = rt.cu[rt.B];
+    for (int i = 0; i < sh.n; ++i) {
+        Model* m = sh.m[i];
+        LLB_TRY(launch_token_map(rt, tokens, m->tok_ids, m->tok_row, m->tok_pos, m->last_idx, st));
+        LLB_TRY(launch_embed(m->tok_ids, m->tok_emb, m->dtype, M, m->dim, m->V, m->x, m->status, st, false, m->ssq,
+                             m->y, m->layers[0].attn_norm));
+    }
+    for (int l = 0; l < sh.m[0]->L; ++l) {
+        auto attn = [&](Model* m) { return launch_attention_prefill(m, l, rt, st); };
+        LLB_TRY(tp_block(sh, l, M, true, nullptr, attn, st));
+    }
+    if (!logits) return LLAMA_OK;
+    return tp_logits(sh, logits_mode == 0 ? rt.B : M, logits_mode == 0, logits, st);
+}
+
+static int tp_decode(const Shards& sh, const int32_t* tokens, int32_t* pos, int B, const llama_sampling* sampling,
+                     const float* uniforms, int32_t* next_tokens, float* logits, int flags, cudaStream_t st) {
+    for (int i = 0; i < sh.n; ++i) {
+        Model* m = sh.m[i];
+        LLB_TRY(launch_embed(tokens, m->tok_emb, m->dtype, B, m->dim, m->V, m->x, m->status, st, false, m->ssq, m->y,
+                             m->layers[0].attn_norm));
+    }
+    for (int l = 0; l < sh.m[0]->L; ++l) {
+        auto attn = [&](Model* m) { return launch_attention_decode(m, l, pos, B, st); };
+        LLB_TRY(tp_block(sh, l, B, false, pos, attn, st));
+    }
+    Model* m0 = sh.m[0];
+    float* lg = logits ? logits : m0->logits_ws;
+    LLB_TRY(tp_logits(sh, B, false, lg, st));
+    if (!sampling) return LLAMA_OK;
+    const bool adv = (flags & LLAMA_DECODE_ADVANCE) != 0;
+    int32_t* tok_adv = adv ? const_cast<int32_t*>(tokens) : nullptr;
+    int32_t* pos_adv = adv ? pos : nullptr;
+    if (sampling->temperature == 0.f) return launch_argmax(lg, B, m0->V, next_tokens, tok_adv, pos_adv, st);
+    return launch_top_p(lg, B, m0->V, sampling->temperature, sampling->top_p, uniforms, next_tokens, tok_adv,
+                        pos_adv, st);
+}
+
+// The shards of a one-GPU group, checked: ranks 0 .. tp-1 in order, one
+// configuration; their buffers are bound to each other (no handshake).
+static int group_of(llama_model_args* ref, Model* const* shards, int tp, Shards* out) {
+    if (!shards || tp < 1 || tp > kMaxTp) { set_error("shards must hold 1..%d models", kMaxTp); return LLAMA_ERR_INVALID_ARG; }
+    out->n = tp;
+    for (int r = 0; r < tp; ++r) {
+        Model* m = shards[r];
+        if (!m) { set_error("shard %d is NULL", r); return LLAMA_ERR_INVALID_ARG; }
+        if (m->tp_size != tp || m->tp_rank != r) {
+            set_error("shard %d is rank %d of %d, expected rank %d of %d", r, m->tp_rank, m->tp_size, r, tp);
+            return LLAMA_ERR_INVALID_ARG;
+        }
+        if (memcmp(&m->a, &shards[0]->a, sizeof(llama_model_args)) != 0) {
+            set_error("shard %d was created with other model arguments", r);
+            return LLAMA_ERR_INVALID_ARG;
+        }
+        out->m[r] = m;
+    }
+    for (int r = 0; r < tp; ++r) {
+        Model* m = shards[r];
+        for (int q = 0; q < tp; ++q) {
+            m->peers.part[q][0] = shards[q]->tp_part[0];
+            m->peers.part[q][1] = shards[q]->tp_part[1];
+            m->peers.flag[q] = shards[q]->tp_flag;
+            m->peers.logits[q] = shards[q]->logits_ws;
+        }
+        m->tp_bound = true;
+        m->tp_wait = false;
+    }
+    if (ref) *ref = shards[0]->a;
+    return LLAMA_OK;
+}
+
 }  // namespace llb
 
 using namespace llb;
@@ -343,8 +555,13 @@ uint64_t llama_launch_count(void) { return g_launches.load(std::memory_order_rel
 
 int llama_model_bytes(const llama_model_args* args, size_t* weight_bytes, size_t* kv_bytes,
                       size_t* workspace_bytes, size_t* total_bytes, int32_t* hidden) {
+    return llama_model_bytes_tp(args, 0, 1, weight_bytes, kv_bytes, workspace_bytes, total_bytes, hidden);
+}
+
+int llama_model_bytes_tp(const llama_model_args* args, int tp_rank, int tp_size, size_t* weight_bytes,
+                         size_t* kv_bytes, size_t* workspace_bytes, size_t* total_bytes, int32_t* hidden) {
     Layout l;
-    LLB_TRY(make_layout(args, &l));
+    LLB_TRY(make_layout(args, &l, tp_rank, tp_size));
     if (weight_bytes) *weight_bytes = l.weight_bytes;
     if (kv_bytes) *kv_bytes = l.kv_bytes;
     if (workspace_bytes) *workspace_bytes = l.ws_end - l.weight_bytes - l.kv_bytes;
@@ -355,10 +572,15 @@ int llama_model_bytes(const llama_model_args* args, size_t* weight_bytes, size_t
 
 int llama_model_create(const llama_model_args* args, void* dev_arena, size_t arena_bytes, void* stream,
                        llama_model** out) {
+    return llama_model_create_tp(args, 0, 1, dev_arena, arena_bytes, stream, out);
+}
+
+int llama_model_create_tp(const llama_model_args* args, int tp_rank, int tp_size, void* dev_arena,
+                          size_t arena_bytes, void* stream, llama_model** out) {
     if (!out) { set_error("out is NULL"); return LLAMA_ERR_INVALID_ARG; }
     *out = nullptr;
     Layout l;
-    LLB_TRY(make_layout(args, &l));
+    LLB_TRY(make_layout(args, &l, tp_rank, tp_size));
     if (!dev_arena) { set_error("arena is NULL"); return LLAMA_ERR_INVALID_ARG; }
     if (reinterpret_cast<uintptr_t>(dev_arena) & 255) { set_error("arena must be 256-byte aligned"); return LLAMA_ERR_INVALID_ARG; }
     if (arena_bytes < l.ws_end) {
@@ -370,6 +592,7 @@ int llama_model_create(const llama_model_args* args, void* dev_arena, size_t are
     m->a = *args;
     m->dim = l.dim; m->L = l.L; m->nh = l.nh; m->nkv = l.nkv; m->hd = l.hd; m->n_rep = l.n_rep; m->H = l.H;
     m->V = l.V; m->S = l.S; m->Bmax = l.Bmax; m->Mmax = l.Mmax; m->dtype = l.dtype; m->esz = l.esz;
+    m->Vl = l.Vl; m->tp_rank = l.tp_rank; m->tp_size = l.tp_size;
     m->nq = l.nq; m->nkvc = l.nkvc; m->nqkv = l.nqkv; m->n_splits = l.n_splits;
     void* A = dev_arena;
     m->tok_emb = at(A, l.off_tok_emb);
@@ -413,6 +636,13 @@ int llama_model_create(const llama_model_args* args, void* dev_arena, size_t are
     m->tl_end = reinterpret_cast<unsigned long long*>(at(A, l.off_tl));
     m->best = reinterpret_cast<unsigned long long*>(at(A, l.off_best));
     m->step_cnt = reinterpret_cast<int*>(at(A, l.off_step_cnt));
+    if (l.tp_size > 1) {
+        m->tp_part[0] = reinterpret_cast<float*>(at(A, l.off_tp_part));
+        m->tp_part[1] = m->tp_part[0] + static_cast<size_t>(l.Mrows) * l.dim;
+    }
+    m->tp_flag = reinterpret_cast<unsigned long long*>(at(A, l.off_tp_flag));
+    m->tp_epoch = m->tp_flag + kMaxTp;
+    m->tp_arrivals = reinterpret_cast<int*>(m->tp_epoch + 1);
     m->last_stream = static_cast<cudaStream_t>(stream);
 
     int rc = LLAMA_OK;
@@ -424,7 +654,7 @@ int llama_model_create(const llama_model_args* args, void* dev_arena, size_t are
             if (rc == LLAMA_OK) rc = make_maps(&p.m_w13, p.w13, 2 * l.H, l.dim, 256, l.dtype);
             if (rc == LLAMA_OK) rc = make_maps(&p.m_w2, p.w2, l.dim, l.H, 256, l.dtype);
         }
-        if (rc == LLAMA_OK) rc = make_maps(&m->m_output, m->output, l.V, l.dim, 256, l.dtype);
+        if (rc == LLAMA_OK) rc = make_maps(&m->m_output, m->output, l.Vl, l.dim, 256, l.dtype);
         if (rc == LLAMA_OK) rc = make_maps(&m->m_y, m->y, l.Mrows, l.dim, 16, l.dtype);
         if (rc == LLAMA_OK) rc = make_maps(&m->m_attn, m->attn, l.Mrows, l.nq, 16, l.dtype);
         if (rc == LLAMA_OK) rc = make_maps(&m->m_g, m->g, l.Mrows, l.H, 16, l.dtype);
@@ -445,6 +675,7 @@ int llama_model_create(const llama_model_args* args, void* dev_arena, size_t are
         if (e == cudaSuccess) e = cudaMemsetAsync(m->attn_cnt, 0, static_cast<size_t>(l.Bmax) * l.nkv * 4, st);
         if (e == cudaSuccess) e = cudaMemsetAsync(m->best, 0, static_cast<size_t>(l.Bmax) * 8, st);
         if (e == cudaSuccess) e = cudaMemsetAsync(m->step_cnt, 0, kStepCounters * sizeof(int), st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(m->tp_flag, 0, (kMaxTp + 2) * 8 + 16, st);
         if (e != cudaSuccess) rc = cuda_fail(e, "cudaMemsetAsync");
     }
     if (rc == LLAMA_OK) rc = launch_rope_table(m->rope, l.S, l.hd, args->rope_theta, st);
@@ -473,7 +704,7 @@ int llama_set_weight(llama_model* m, int layer, int which, const void* src, void
     switch (which) {
         case LLAMA_W_TOK_EMBEDDINGS: dst = m->tok_emb; bytes = static_cast<size_t>(m->V) * D * e; break;
         case LLAMA_W_NORM: dst = m->norm; bytes = D * 4; break;
-        case LLAMA_W_OUTPUT: dst = m->output; bytes = static_cast<size_t>(m->V) * D * e; break;
+        case LLAMA_W_OUTPUT: dst = m->output; bytes = static_cast<size_t>(m->Vl) * D * e; break;
         case LLAMA_W_ATTENTION_NORM: dst = p->attn_norm; bytes = D * 4; break;
         case LLAMA_W_WQ: dst = p->wqkv; bytes = static_cast<size_t>(m->nq) * D * e; break;
         case LLAMA_W_WK: dst = static_cast<char*>(p->wqkv) + static_cast<size_t>(m->nq) * D * e;
@@ -508,8 +739,110 @@ int llama_get_kv(llama_model* m, int layer, void** k, void** v, int64_t strides[
     return LLAMA_OK;
 }
 
+}  // extern "C"
+
+namespace llb {
+// Argument checks of a prefill call and its row table (host lens).
+static int prefill_rows(const Model* m, const int32_t* tokens, const int32_t* lens, int B, int T, int start_pos,
+                        const float* logits, int logits_mode, RowTable* rt_out) {
+    if (!m || !tokens) { set_error("model or tokens is NULL"); return LLAMA_ERR_INVALID_ARG; }
+    if (B <= 0 || T <= 0 || start_pos < 0) { set_error("B and T must be positive, start_pos >= 0"); return LLAMA_ERR_INVALID_ARG; }
+    if (logits_mode != 0 && logits_mode != 1) { set_error("logits_mode must be 0 or 1"); return LLAMA_ERR_INVALID_ARG; }
+    if (logits_mode == 1 && !logits) { set_error("logits_mode 1 needs a logits buffer"); return LLAMA_ERR_INVALID_ARG; }
+    if (logits_mode == 1 && m->tp_size > 1 && m->tp_wait) {
+        set_error("a tensor-parallel rank on its own GPU returns last-token logits only (logits_mode 0)");
+        return LLAMA_ERR_INVALID_ARG;
+    }
+    if (B > m->Bmax) { set_error("B=%d > max_batch_size=%d", B, m->Bmax); return LLAMA_ERR_CAPACITY; }
+    if (static_cast<long long>(start_pos) + T > m->S) {
+        set_error("start_pos + T = %lld > max_seq_len=%d", static_cast<long long>(start_pos) + T, m->S);
+        return LLAMA_ERR_CAPACITY;
+    }
+    RowTable& rt = *rt_out;
+    rt.B = B; rt.T = T; rt.start_pos = start_pos;
+    rt.cu[0] = 0;
+    for (int b = 0; b < B; ++b) {
+        const int len = lens ? lens[b] : T;
+        if (len < 1 || len > T) { set_error("lens[%d]=%d outside [1, T=%d]", b, len, T); return LLAMA_ERR_INVALID_ARG; }
+        rt.cu[b + 1] = rt.cu[b] + len;
+    }
+    if (rt.cu[B] > m->Mmax) { set_error("sum(lens)=%d > max_tokens=%d", rt.cu[B], m->Mmax); return LLAMA_ERR_CAPACITY; }
+    return LLAMA_OK;
+}
+
+static int decode_args(const Model* m, const int32_t* tokens, const int32_t* pos, int B, const llama_sampling* sampling,
+                       const float* uniforms, const int32_t* next_tokens, int flags) {
+    if (!m || !tokens || !pos) { set_error("model, tokens or pos is NULL"); return LLAMA_ERR_INVALID_ARG; }
+    if (B <= 0) { set_error("B must be positive"); return LLAMA_ERR_INVALID_ARG; }
+    if (B > m->Bmax) { set_error("B=%d > max_batch_size=%d", B, m->Bmax); return LLAMA_ERR_CAPACITY; }
+    if (sampling && !next_tokens) { set_error("sampling needs next_tokens"); return LLAMA_ERR_INVALID_ARG; }
+    if (sampling && sampling->temperature < 0.f) { set_error("temperature must be >= 0"); return LLAMA_ERR_INVALID_ARG; }
+    if (sampling && sampling->temperature > 0.f && !uniforms) { set_error("top-p sampling needs uniforms"); return LLAMA_ERR_INVALID_ARG; }
+    if ((flags & LLAMA_DECODE_ADVANCE) && !sampling) { set_error("LLAMA_DECODE_ADVANCE needs sampling"); return LLAMA_ERR_INVALID_ARG; }
+    return LLAMA_OK;
+}
+}  // namespace llb
+
+extern "C" {
+
+int llama_tp_prefill_all(llama_model* const* shards, int tp, const int32_t* tokens, const int32_t* lens, int B, int T,
+                         int start_pos, float* logits, int logits_mode, void* stream) {
+    Shards sh;
+    LLB_TRY(group_of(nullptr, reinterpret_cast<Model* const*>(shards), tp, &sh));
+    RowTable rt;
+    LLB_TRY(prefill_rows(sh.m[0], tokens, lens, B, T, start_pos, logits, logits_mode, &rt));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    for (int i = 0; i < sh.n; ++i) sh.m[i]->last_stream = st;
+    return tp_prefill(sh, rt, tokens, logits, logits_mode, st);
+}
+
+int llama_tp_decode_step_all(llama_model* const* shards, int tp, const int32_t* tokens, int32_t* pos, int B,
+                             const llama_sampling* sampling, const float* uniforms, int32_t* next_tokens,
+                             float* logits, int flags, void* stream) {
+    Shards sh;
+    LLB_TRY(group_of(nullptr, reinterpret_cast<Model* const*>(shards), tp, &sh));
+    LLB_TRY(decode_args(sh.m[0], tokens, pos, B, sampling, uniforms, next_tokens, flags));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    for (int i = 0; i < sh.n; ++i) sh.m[i]->last_stream = st;
+    return tp_decode(sh, tokens, pos, B, sampling, uniforms, next_tokens, logits, flags, st);
+}
+
+int llama_tp_buffers(llama_model* m, float** part0, float** part1, unsigned long long** flags, float** logits) {
+    if (!m) { set_error("model is NULL"); return LLAMA_ERR_INVALID_ARG; }
+    if (part0) *part0 = m->tp_part[0];
+    if (part1) *part1 = m->tp_part[1];
+    if (flags) *flags = m->tp_flag;
+    if (logits) *logits = m->logits_ws;
+    return LLAMA_OK;
+}
+
+int llama_tp_bind(llama_model* m, float* const* part0, float* const* part1, unsigned long long* const* flags,
+                  float* const* logits) {
+    if (!m || !part0 || !part1 || !flags || !logits) { set_error("model or buffer table is NULL"); return LLAMA_ERR_INVALID_ARG; }
+    if (m->tp_size < 2) { set_error("llama_tp_bind needs a shard of a group of 2 or more ranks"); return LLAMA_ERR_INVALID_ARG; }
+    for (int q = 0; q < m->tp_size; ++q) {
+        if (!part0[q] || !part1[q] || !flags[q] || !logits[q]) { set_error("rank %d's buffers are NULL", q); return LLAMA_ERR_INVALID_ARG; }
+        m->peers.part[q][0] = part0[q];
+        m->peers.part[q][1] = part1[q];
+        m->peers.flag[q] = flags[q];
+        m->peers.logits[q] = logits[q];
+    }
+    m->tp_bound = true;
+    m->tp_wait = true;
+    return LLAMA_OK;
+}
+
 int llama_prefill(llama_model* m, const int32_t* tokens, const int32_t* lens, int B, int T, int start_pos,
                   float* logits, int logits_mode, void* stream) {
+    if (m && m->tp_size > 1) {
+        if (!m->tp_bound) { set_error("a tensor-parallel shard needs llama_tp_bind (or llama_tp_prefill_all)"); return LLAMA_ERR_INVALID_ARG; }
+        RowTable rt;
+        LLB_TRY(prefill_rows(m, tokens, lens, B, T, start_pos, logits, logits_mode, &rt));
+        cudaStream_t st = static_cast<cudaStream_t>(stream);
+        m->last_stream = st;
+        Shards sh = {{m}, 1};
+        return tp_prefill(sh, rt, tokens, logits, logits_mode, st);
+    }
     if (!m || !tokens) { set_error("model or tokens is NULL"); return LLAMA_ERR_INVALID_ARG; }
     if (B <= 0 || T <= 0 || start_pos < 0) { set_error("B and T must be positive, start_pos >= 0"); return LLAMA_ERR_INVALID_ARG; }
     if (logits_mode != 0 && logits_mode != 1) { set_error("logits_mode must be 0 or 1"); return LLAMA_ERR_INVALID_ARG; }
@@ -567,6 +900,14 @@ int llama_prefill(llama_model* m, const int32_t* tokens, const int32_t* lens, in
 
 int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B, const llama_sampling* sampling,
                       const float* uniforms, int32_t* next_tokens, float* logits, int flags, void* stream) {
+    if (m && m->tp_size > 1) {
+        if (!m->tp_bound) { set_error("a tensor-parallel shard needs llama_tp_bind (or llama_tp_decode_step_all)"); return LLAMA_ERR_INVALID_ARG; }
+        LLB_TRY(decode_args(m, tokens, pos, B, sampling, uniforms, next_tokens, flags));
+        cudaStream_t st = static_cast<cudaStream_t>(stream);
+        m->last_stream = st;
+        Shards sh = {{m}, 1};
+        return tp_decode(sh, tokens, pos, B, sampling, uniforms, next_tokens, logits, flags, st);
+    }
     if (!m || !tokens || !pos) { set_error("model, tokens or pos is NULL"); return LLAMA_ERR_INVALID_ARG; }
     if (B <= 0) { set_error("B must be positive"); return LLAMA_ERR_INVALID_ARG; }
     if (B > m->Bmax) { set_error("B=%d > max_batch_size=%d", B, m->Bmax); return LLAMA_ERR_CAPACITY; }
@@ -599,8 +940,7 @@ int llama_decode_step(llama_model* m, const int32_t* tokens, int32_t* pos, int B
                 long long stall_wait = 0;
                 take_stall(m, LLAMA_STALL_ATTENTION, &stall_unit, &stall_wait);
                 return launch_attention_decode(m, l, pos, B, st, chain, tl_next(m, TL_ATTENTION, 0), stall_wait,
-                                               stall_unit, m->layers[l].wo,
-                                               static_cast<long long>(m->dim) * m->nq * m->esz);
+                                               stall_unit);
             };
             LLB_TRY(block_forward_fused(m, l, B, nullptr, pos, attn, st, chain, true));
         }

@@ -78,10 +78,13 @@ template <> struct Vec<f16, 4> {
 // per warp and merged across the 4 warps at the end of a segment.
 //
 // A segment that covers its whole pair writes the output row directly.  A pair
-// split between CTAs has at most one partial segment per CTA at each end of
-// its run (slot 0 = the run's first segment, slot 1 = its last); each writes
-// its unnormalised (o, max, sum) and the CTA that arrives last at the pair's
-// counter merges them in CTA order (deterministic).  No CTA waits for another.
+// split between CTAs is finished by its first contributor, whose segment is
+// the last of its run; every other contributor's segment is the first of its
+// run: it writes its unnormalised (o, max, sum) and counts it at the pair's
+// counter early in its run, and the finisher, at the end of its run, waits
+// (bounded) for that count, then merges its own state with the published
+// ones in CTA order (deterministic).  Only a finisher waits, and only for
+// other CTAs' first segments, which never wait.
 __device__ __forceinline__ long long run_begin64(long long c, long long W, long long P) { return c * W / P; }
 __device__ __forceinline__ int owner64(long long u, long long W, long long P) {
     return static_cast<int>(((u + 1) * P - 1) / W);
@@ -92,8 +95,7 @@ __global__ void __launch_bounds__(128)
 attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
                    const int32_t* __restrict__ pos, int B, int nkv, int nq, int S, long long row_stride,
                    float* __restrict__ part_o, float* __restrict__ part_ml, int* __restrict__ counters,
-                   T* __restrict__ out, int* status, unsigned long long* tl, long long wait_ns, int stall,
-                   const void* __restrict__ next_w, long long next_w_bytes) {
+                   T* __restrict__ out, int* status, unsigned long long* tl, long long wait_ns, int stall) {
     constexpr int EPL = HD / 32;   // head dims per lane
     constexpr int ROW = HD * static_cast<int>(sizeof(T));
     constexpr int CH_BYTES = kChunk * ROW;
@@ -186,16 +188,6 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
         advance(icur);
     };
 
-    // The weights of the projection that follows (constant during decode):
-    // this CTA's share is pulled into L2 while the cache reads below leave
-    // HBM mostly idle.
-    if (threadIdx.x == 0 && next_w_bytes > 0) {
-        const long long per = ((next_w_bytes / gridDim.x) + 15) & ~15LL;
-        const long long b0 = per * blockIdx.x;
-        const long long b1 = b0 + per < next_w_bytes ? b0 + per : next_w_bytes;
-        for (long long o = b0; o < b1; o += 32768)
-            bulk_prefetch_l2(static_cast<const uint8_t*>(next_w) + o, static_cast<uint32_t>(b1 - o < 32768 ? b1 - o : 32768));
-    }
     if (threadIdx.x == 0) {
         for (int k = 0; k < NSLOT; ++k) mbar_init(&bar[k], 1);
         fence_mbar_init();
@@ -373,6 +365,33 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
         __syncthreads();
         const long long pair_u0 = static_cast<long long>(s_cum[cur.b]) * nkv + static_cast<long long>(cur.g) * nch;
         const int slot_id = c * 2 + (seg_i0 == 0 ? 0 : 1);
+        // A pair split between runs is finished by its first contributor cf:
+        // that segment is the last of cf's run (its run ends inside the pair),
+        // while every other contributor's run starts inside the pair, so its
+        // segment is the first of its run and is published early.
+        const int cf = whole ? c : owner64(pair_u0, W, P), cl = whole ? c : owner64(pair_u0 + nch - 1, W, P);
+        const bool finisher = !whole && c == cf;
+        const int cnt_idx = cur.b * nkv + cur.g;
+        if (finisher) {
+            if (threadIdx.x == 0) {
+                const int need = cl - cf;
+                const volatile int* cnt = counters + cnt_idx;
+                bool okc = *cnt >= need;
+                if (!okc) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (!(okc = *cnt >= need) && globaltimer_ns() - t0 <= wlim) {
+                    }
+                }
+                s_last = okc ? 1 : 0;
+            }
+            __syncthreads();
+            if (!s_last) {       // units up to i were consumed; i + 1 .. i + NSLOT may be in flight
+                ok = false;
+                fail_i = i + 1;
+                break;
+            }
+            __threadfence();
+        }
         for (int idx = threadIdx.x; idx < NREP * HD; idx += blockDim.x) {
             const int r = idx / HD, d = idx % HD;
             float M = -INFINITY;
@@ -388,44 +407,39 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
             const int h = cur.g * NREP + r;
             if (whole) {
                 out[static_cast<long long>(cur.b) * nq + h * HD + d] = from_f32<T>(acc / L);
-            } else {
+            } else if (!finisher) {
                 part_o[(static_cast<long long>(slot_id) * NREP + r) * HD + d] = acc;
                 if (d == 0) {
                     part_ml[(static_cast<long long>(slot_id) * NREP + r) * 2] = M;
                     part_ml[(static_cast<long long>(slot_id) * NREP + r) * 2 + 1] = L;
                 }
+            } else {
+                // merge this CTA's (M, L, acc) with the published ones, in CTA order
+                float Mt = M;
+                for (int cc = cf + 1; cc <= cl; ++cc) {
+                    const int sid = cc * 2 + (run_begin64(cc, W, P) >= pair_u0 ? 0 : 1);
+                    Mt = fmaxf(Mt, __ldcg(part_ml + (static_cast<long long>(sid) * NREP + r) * 2));
+                }
+                const float f0 = (M == -INFINITY) ? 0.f : __expf(M - Mt);
+                float Lt = 0.f, at = 0.f;
+                Lt += L * f0;
+                at += acc * f0;
+                for (int cc = cf + 1; cc <= cl; ++cc) {
+                    const int sid = cc * 2 + (run_begin64(cc, W, P) >= pair_u0 ? 0 : 1);
+                    const float mm = __ldcg(part_ml + (static_cast<long long>(sid) * NREP + r) * 2);
+                    const float f = (mm == -INFINITY) ? 0.f : __expf(mm - Mt);
+                    Lt += __ldcg(part_ml + (static_cast<long long>(sid) * NREP + r) * 2 + 1) * f;
+                    at += __ldcg(part_o + (static_cast<long long>(sid) * NREP + r) * HD + d) * f;
+                }
+                out[static_cast<long long>(cur.b) * nq + h * HD + d] = from_f32<T>(at / Lt);
             }
         }
-        if (!whole) {
-            const int cf = owner64(pair_u0, W, P), cl = owner64(pair_u0 + nch - 1, W, P);
-            const int cnt_idx = cur.b * nkv + cur.g;
+        if (!whole && !finisher) {
             __threadfence();
             __syncthreads();
-            if (threadIdx.x == 0) s_last = atomicAdd(&counters[cnt_idx], 1) == cl - cf;
-            __syncthreads();
-            if (s_last) {
-                __threadfence();
-                for (int idx = threadIdx.x; idx < NREP * HD; idx += blockDim.x) {
-                    const int r = idx / HD, d = idx % HD;
-                    const int h = cur.g * NREP + r;
-                    float M = -INFINITY;
-                    for (int cc = cf; cc <= cl; ++cc) {
-                        const int sid = cc * 2 + (run_begin64(cc, W, P) >= pair_u0 ? 0 : 1);
-                        M = fmaxf(M, part_ml[(static_cast<long long>(sid) * NREP + r) * 2]);
-                    }
-                    float L = 0.f, acc = 0.f;
-                    for (int cc = cf; cc <= cl; ++cc) {
-                        const int sid = cc * 2 + (run_begin64(cc, W, P) >= pair_u0 ? 0 : 1);
-                        const float mm = part_ml[(static_cast<long long>(sid) * NREP + r) * 2];
-                        const float f = (mm == -INFINITY) ? 0.f : __expf(mm - M);
-                        L += part_ml[(static_cast<long long>(sid) * NREP + r) * 2 + 1] * f;
-                        acc += part_o[(static_cast<long long>(sid) * NREP + r) * HD + d] * f;
-                    }
-                    out[static_cast<long long>(cur.b) * nq + h * HD + d] = from_f32<T>(acc / L);
-                }
-                if (threadIdx.x == 0) counters[cnt_idx] = 0;
-            }
+            if (threadIdx.x == 0) atomicAdd(&counters[cnt_idx], 1);
         }
+        if (finisher && threadIdx.x == 0) counters[cnt_idx] = 0;
         __syncthreads();   // s_m / s_o / s_last reused by the next segment
         if (i + 1 < len) {
             advance(cur);
@@ -449,7 +463,7 @@ static int g_attn_sms = 0;
 
 template <typename T, int HD, int NREP>
 static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl,
-                     unsigned long long* tl, long long wait_ns, int stall, const void* next_w, long long next_w_bytes) {
+                     unsigned long long* tl, long long wait_ns, int stall) {
     const T* kc = static_cast<const T*>(m->kc) + layer * m->kv_layer_elems;
     const T* vc = static_cast<const T*>(m->vc) + layer * m->kv_layer_elems;
     auto kern = attn_decode_kernel<T, HD, NREP>;
@@ -477,8 +491,7 @@ static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaS
     P = std::max<long long>(P, 1);
     cudaError_t e = launch_k(kern, dim3(static_cast<unsigned>(P)), dim3(128), smem, st, pdl, static_cast<const T*>(m->q),
                              kc, vc, pos, B, m->nkv, m->nq, m->S, m->kv_row_elems, m->part_o, m->part_ml,
-                             m->attn_cnt, static_cast<T*>(m->attn), m->status, tl, wait_ns, stall, next_w,
-                             next_w_bytes);
+                             m->attn_cnt, static_cast<T*>(m->attn), m->status, tl, wait_ns, stall);
     count_launch();
     if (e != cudaSuccess) return cuda_fail(e, "attn_decode_kernel");
     return LLAMA_OK;
@@ -486,12 +499,12 @@ static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaS
 
 template <typename T, int HD>
 static int decode_rep(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl,
-                      unsigned long long* tl, long long wait_ns, int stall, const void* nw, long long nwb) {
+                      unsigned long long* tl, long long wait_ns, int stall) {
     switch (m->n_rep) {
-        case 1: return decode_go<T, HD, 1>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, nw, nwb);
-        case 2: return decode_go<T, HD, 2>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, nw, nwb);
-        case 4: return decode_go<T, HD, 4>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, nw, nwb);
-        case 8: return decode_go<T, HD, 8>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, nw, nwb);
+        case 1: return decode_go<T, HD, 1>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+        case 2: return decode_go<T, HD, 2>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+        case 4: return decode_go<T, HD, 4>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+        case 8: return decode_go<T, HD, 8>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
     }
     set_error("n_heads / n_kv_heads = %d unsupported (1, 2, 4, 8)", m->n_rep);
     return LLAMA_ERR_INVALID_ARG;
@@ -499,23 +512,21 @@ static int decode_rep(const Model* m, int layer, const int32_t* pos, int B, cuda
 
 template <typename T>
 static int decode_hd(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl,
-                     unsigned long long* tl, long long wait_ns, int stall, const void* nw, long long nwb) {
+                     unsigned long long* tl, long long wait_ns, int stall) {
     switch (m->hd) {
-        case 32: return decode_rep<T, 32>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, nw, nwb);
-        case 64: return decode_rep<T, 64>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, nw, nwb);
-        case 128: return decode_rep<T, 128>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, nw, nwb);
+        case 32: return decode_rep<T, 32>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+        case 64: return decode_rep<T, 64>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+        case 128: return decode_rep<T, 128>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
     }
     set_error("head_dim %d unsupported", m->hd);
     return LLAMA_ERR_INVALID_ARG;
 }
 
 int launch_attention_decode(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl,
-                            unsigned long long* tl, long long wait_ns, int stall, const void* next_w,
-                            long long next_w_bytes) {
-    if (next_w_bytes % 16 || (reinterpret_cast<uintptr_t>(next_w) & 15)) { next_w = nullptr; next_w_bytes = 0; }
-    if (m->dtype == LLAMA_BF16) return decode_hd<bf16>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, next_w, next_w_bytes);
-    if (m->dtype == LLAMA_F16) return decode_hd<f16>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, next_w, next_w_bytes);
-    return decode_hd<float>(m, layer, pos, B, st, pdl, tl, wait_ns, stall, next_w, next_w_bytes);
+                            unsigned long long* tl, long long wait_ns, int stall) {
+    if (m->dtype == LLAMA_BF16) return decode_hd<bf16>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+    if (m->dtype == LLAMA_F16) return decode_hd<f16>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+    return decode_hd<float>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
 }
 
 // ---------------------------------------------------------------- prefill

@@ -15,6 +15,18 @@ struct Seg {
     int tile, ks, ke;
 };
 
+// A tile whose k-range is split between the runs of CTAs cf .. cl (cf < cl) is
+// finished by cf, the CTA holding its first unit: cf's run ends inside the
+// tile (a run that held the whole tile would not split it), so that segment
+// is the LAST of cf's run, while every other contributor's run starts inside
+// the tile, so its segment is the FIRST of its run.  Each CTA therefore
+// publishes at most one partial (its first segment, when it does not start at
+// a tile boundary), early in its run, and the finisher, at the end of its
+// own run, only has to collect them: it never publishes or counts itself.
+__host__ __device__ __forceinline__ int split_finisher(int tile, int KT, int W, int P) {
+    return owner(tile * KT, W, P);
+}
+
 // Next segment (one tile's k-range) of a run of units; false past the end.
 __host__ __device__ __forceinline__ bool next_seg(int& u, int u1, int KT, Seg& s) {
     if (u >= u1) return false;
@@ -157,10 +169,13 @@ __device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int la
 // The epilogue warps' loop over the segments of one CTA's stream-K run of a
 // decode projection: wait for each segment's accumulator (TMEM buffer j % 2,
 // 64 columns apart; tmem_lane = TMEM base + this warp's lane quarter), read
-// it, hand the buffer back to the MMA warp, then either finish the tile or
-// publish this CTA's partial; the CTA that arrives last at a split tile's
-// counter adds the partials in CTA order and finishes it.  Runs are
-// run_begin(c, W, P) .. run_begin(c + 1, W, P) over W = n_tiles * KT units.
+// it, hand the buffer back to the MMA warp, then finish the tile, or publish
+// this CTA's partial of a split tile it does not finish (and count it), or --
+// as the split tile's finisher (split_finisher) -- wait until every other
+// contributor has counted its partial, add them after its own in CTA order
+// (deterministic) and finish the tile.  Runs are run_begin(c, W, P) ..
+// run_begin(c + 1, W, P) over W = n_tiles * KT units; partials are one
+// 128 x BN fp32 block per CTA.
 template <int BN, typename T>
 __device__ __forceinline__ void decode_epilogue_loop(uint32_t tmem_lane, uint64_t* tfull, uint64_t* tempty, int* flag,
                                                      float* part, int* counters, int c, int P, int u0, int u1,
@@ -191,36 +206,55 @@ __device__ __forceinline__ void decode_epilogue_loop(uint32_t tmem_lane, uint64_
         }
         const int t = sg.tile;
         const int tb = t * KT;
-        const int cf = owner(tb, W, P), cl = owner(tb + KT - 1, W, P);
-        if (cl > cf) {
-            // split tile: publish this CTA's partial, the last arrival reduces
-            const int slot = (tb + sg.ks == u0) ? 0 : 1;   // the run's first segment, or its last
-            float* my = part + ((static_cast<long long>(c) * 2 + slot) * 128 + r) * BN;
+        const int cf = split_finisher(t, KT, W, P), cl = owner(tb + KT - 1, W, P);
+        if (cl > cf && c != cf) {
+            // a split tile this CTA does not finish (its run's first segment):
+            // publish the partial and count it
+            float* my = part + (static_cast<long long>(c) * 128 + r) * BN;
 #pragma unroll
             for (int b = 0; b < BN; b += 4)
                 *reinterpret_cast<float4*>(my + b) = make_float4(v[b], v[b + 1], v[b + 2], v[b + 3]);
             __threadfence();
             named_sync(1, 128);
-            if (epi_tid == 0) flag[1] = atomicAdd(&counters[t], 1);
+            if (epi_tid == 0) atomicAdd(&counters[t], 1);
+            continue;
+        }
+        if (cl > cf) {
+            // the finisher (its run's last segment): the other cl - cf
+            // contributors published theirs early in their runs
+            if (epi_tid == 0) {
+                const int need = cl - cf;
+                const volatile int* cnt = counters + t;
+                bool okc = *cnt >= need;
+                if (!okc) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (!(okc = *cnt >= need) && globaltimer_ns() - t0 <= wlim) {
+                    }
+                }
+                flag[1] = okc ? 1 : 0;
+            }
             named_sync(1, 128);
-            const int arrived = flag[1];
-            if (arrived != cl - cf) continue;      // not the last contributor
+            if (!flag[1]) {
+                if (epi_tid == 0) {
+                    report_status(ep.status, LLAMA_ERR_DEVICE_TIMEOUT);
+                    atomicExch(&flag[0], 1);
+                }
+                break;
+            }
             __threadfence();
-#pragma unroll
-            for (int b = 0; b < BN; ++b) v[b] = 0.f;
-            // partials in CTA order, CB contributors per batch of independent loads
+            // partials after this CTA's own, in CTA order, CB contributors per
+            // batch of independent loads
             constexpr int CB = BN <= 16 ? 4 : (BN <= 32 ? 2 : 1);
-            for (int cb = cf; cb <= cl; cb += CB) {
+            for (int cb = cf + 1; cb <= cl; cb += CB) {
                 float4 f[CB][BN / 4];
 #pragma unroll
                 for (int e = 0; e < CB; ++e) {
                     const int cc = cb + e;
                     if (cc <= cl) {
-                        const int sl = run_begin(cc, W, P) >= tb ? 0 : 1;   // slot 0: first segment, 1: last
                         const float4* pp = reinterpret_cast<const float4*>(
-                            part + ((static_cast<long long>(cc) * 2 + sl) * 128 + r) * BN);
+                            part + (static_cast<long long>(cc) * 128 + r) * BN);
 #pragma unroll
-                        for (int qq = 0; qq < BN / 4; ++qq) f[e][qq] = pp[qq];
+                        for (int qq = 0; qq < BN / 4; ++qq) f[e][qq] = __ldcg(pp + qq);
                     }
                 }
 #pragma unroll

@@ -23,6 +23,27 @@ constexpr int kMaxTiles = 4096;       // tile counters: N / 128 of the widest pr
 constexpr int kMaxAttnCtas = 1024;    // persistent CTAs of the decode attention kernel
 constexpr int kTimelineCap = 8192;    // launches one timeline can stamp
 constexpr int kStepCounters = 4;      // per-step finish counters
+constexpr int kMaxTp = 8;             // tensor-parallel ranks of one model
+
+// Tensor parallelism: the buffers of every rank of a group, as device
+// addresses this GPU can read (its own, or peers' through NVLink / P2P).
+struct TpPeers {
+    float* part[kMaxTp][2];               // fp32 partial residual updates (wo / w2), by phase parity
+    unsigned long long* flag[kMaxTp];     // flag words: flag[q][r] = last phase rank r announced to rank q
+    float* logits[kMaxTp];                // each rank's logits buffer [Bmax][V]
+};
+
+// Cross-rank handshake of one reduce or gather launch (multi-GPU groups only).
+struct TpSync {
+    int wait;                             // 0: every rank's data is ready by stream order (one GPU)
+    int rank, size;
+    unsigned long long* my_flags;         // [kMaxTp] this rank's flag words
+    unsigned long long* peer_flags[kMaxTp];
+    unsigned long long* epoch;            // this rank's count of completed handshakes
+    int* arrivals;                        // CTAs of the launch that passed the handshake
+    int* status;
+    long long wait_ns;
+};
 
 // Token -> (batch row, position) map of one prefill call, passed by value.
 struct RowTable {
@@ -171,6 +192,16 @@ struct Model {
     unsigned long long* tl_end;
     // One-shot stall for tests of the device timeout (llama_debug_stall): the
     // next launch of the chosen kernel gets it, then it is cleared.
+    // tensor parallelism: this shard's rank and group size, its vocabulary
+    // slice, its double-buffered partial sums, flag words and handshake
+    // counters, and every rank's buffers once bound
+    int tp_rank = 0, tp_size = 1, Vl = 0;
+    float* tp_part[2] = {nullptr, nullptr};
+    unsigned long long* tp_flag = nullptr;     // [kMaxTp]
+    unsigned long long* tp_epoch = nullptr;
+    int* tp_arrivals = nullptr;
+    TpPeers peers = {};
+    bool tp_bound = false, tp_wait = false;
     int dbg_kind = 0;          // 0 none, LLAMA_STALL_PROJECTION or LLAMA_STALL_ATTENTION
     int dbg_unit = -1;
     long long dbg_wait_ns = 0;
@@ -222,11 +253,9 @@ bool attention_prefill_tmem_ok(const Model* m);
 int launch_attention_prefill_tmem(const Model* m, int layer, const RowTable& rt, cudaStream_t st);
 // wait_ns > 0 replaces the default wait limit; stall_unit >= 0: CTA 0 never
 // issues that unit's copies or their barrier signal (tests of the timeout).
-// next_w / next_w_bytes: weights of the projection that follows, pulled into
-// L2 by the CTAs at their start (16-byte aligned; null = none).
 int launch_attention_decode(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st,
                             bool pdl = false, unsigned long long* tl = nullptr, long long wait_ns = 0,
-                            int stall_unit = -1, const void* next_w = nullptr, long long next_w_bytes = 0);
+                            int stall_unit = -1);
 
 int launch_argmax(const float* logits, int B, int V, int32_t* out, int32_t* tokens_adv,
                   int32_t* pos_adv, cudaStream_t st, bool pdl = false, unsigned long long* tl = nullptr);
@@ -234,6 +263,14 @@ int launch_logprobs(const float* logits, const int32_t* tokens, int N, int V, fl
 int launch_top_p(const float* logits, int B, int V, float temperature, float top_p,
                  const float* uniforms, int32_t* out, int32_t* tokens_adv, int32_t* pos_adv,
                  cudaStream_t st, bool pdl = false, unsigned long long* tl = nullptr);
+
+// Tensor parallelism: x[m, :] += sum over ranks r (in rank order) of
+// part_r[m, :] for M rows, then the next RMSNorm's producer side (y =
+// x * w_next in the model's 16-bit type, per-128-feature sums of x^2).
+int launch_tp_reduce(const Model* m, const float* const* parts, int M, const float* w_next, const TpSync& sync,
+                     cudaStream_t st);
+// Copies every other rank's [rows, Vl] logits slice into this rank's [rows, V] buffer.
+int launch_tp_gather_logits(const Model* m, float* logits, int rows, const TpSync& sync, cudaStream_t st);
 
 // TMA descriptor of a K-major 16-bit matrix (dtype LLAMA_BF16 or LLAMA_F16),
 // boxes of 64 columns x box_rows rows, 128-byte swizzle (driver entry point

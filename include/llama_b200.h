@@ -222,6 +222,54 @@ LLAMA_API int llama_token_logprobs(const float* logits, const int32_t* tokens, i
  * is in doubt. */
 LLAMA_API int llama_model_status(llama_model* m, int* device_status);
 
+/* ---- tensor parallelism --------------------------------------------------
+ * The reference's model-parallel layout (Admin Guide §1.3 NOTE on fairscale,
+ * §4.2 "Single-host, multi-GPU", §6.1 "Hot path"; source tour, "One model.py"):
+ * rank r of tp_size ranks holds query heads [r*nh/tp, (r+1)*nh/tp) with their
+ * KV heads [r*nkv/tp, (r+1)*nkv/tp) (rows of wq, wk, wv; columns of wo), FFN
+ * features [r*H/tp, (r+1)*H/tp) (rows of w1, w3; columns of w2), vocabulary
+ * rows [r*V/tp, (r+1)*V/tp) of the output projection, and whole copies of the
+ * token embedding and the three RMSNorm weights.  wo and w2 leave partial
+ * residual updates; each rank adds every rank's update, in rank order, to its
+ * own copy of the residual stream (two reductions per layer), so the copies
+ * stay identical; the logits slices are gathered.  16-bit models only;
+ * n_heads, n_kv_heads, vocab_size and the FFN width (in multiples of 64) must
+ * split evenly.  Weights are uploaded with llama_set_weight in their shard
+ * shapes ([nh/tp*hd, dim] for wq, [dim, nh/tp*hd] for wo, [V/tp, dim] for
+ * output, ...).
+ *
+ * llama_model_bytes_tp / llama_model_create_tp: as llama_model_bytes /
+ *   llama_model_create for shard tp_rank of tp_size (1 <= tp_size <= 8).
+ * llama_tp_prefill_all / llama_tp_decode_step_all: one GPU runs every rank
+ *   (shards[r] = rank r, all on this device): the calls of llama_prefill /
+ *   llama_decode_step for the whole group, phase by phase on `stream`, each
+ *   rank reading the others' partial sums directly; `logits` ([rows, V], or
+ *   NULL) receives every rank's slice.  Used to check the sharded forward
+ *   pass against the unsharded one.
+ * llama_tp_buffers / llama_tp_bind: ranks on separate GPUs (one process per
+ *   GPU).  Each rank publishes its two partial-sum buffers, its flag words and
+ *   its logits buffer (device addresses; share them through CUDA IPC), and
+ *   binds the table of every rank's buffers, mapped into its own address
+ *   space (indexed by rank, its own included).  After that, llama_prefill
+ *   (logits_mode 0) and llama_decode_step on each rank's shard run the
+ *   group's forward pass: every reduction first announces its phase in every
+ *   peer's flag words and waits (bounded, LLAMA_ERR_DEVICE_TIMEOUT) until all
+ *   ranks announced it, then reads the peers' partial sums over NVLink (plain
+ *   peer loads).  Every rank must make the same sequence of calls. */
+LLAMA_API int llama_model_bytes_tp(const llama_model_args* args, int tp_rank, int tp_size, size_t* weight_bytes,
+                                   size_t* kv_bytes, size_t* workspace_bytes, size_t* total_bytes, int32_t* hidden);
+LLAMA_API int llama_model_create_tp(const llama_model_args* args, int tp_rank, int tp_size, void* dev_arena,
+                                    size_t arena_bytes, void* stream, llama_model** out);
+LLAMA_API int llama_tp_prefill_all(llama_model* const* shards, int tp, const int32_t* tokens, const int32_t* lens,
+                                   int B, int T, int start_pos, float* logits, int logits_mode, void* stream);
+LLAMA_API int llama_tp_decode_step_all(llama_model* const* shards, int tp, const int32_t* tokens, int32_t* pos, int B,
+                                       const llama_sampling* sampling, const float* uniforms, int32_t* next_tokens,
+                                       float* logits, int flags, void* stream);
+LLAMA_API int llama_tp_buffers(llama_model* m, float** part0, float** part1, unsigned long long** flags,
+                               float** logits);
+LLAMA_API int llama_tp_bind(llama_model* m, float* const* part0, float* const* part1,
+                            unsigned long long* const* flags, float* const* logits);
+
 /* Frees the host handle; the arena and everything in it stay with the caller. */
 LLAMA_API int llama_model_destroy(llama_model* m);
 

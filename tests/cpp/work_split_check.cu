@@ -106,12 +106,18 @@ static void check_prefill(int TM, int TN, int KT, int P, bool can_split) {
     }
 }
 
+// Decode projection: the split tile's finisher is split_finisher() (its first
+// contributor); its segment must be the LAST of its run (so it is processed
+// after the CTA's other work) and every other contributor's segment the FIRST
+// of its run, so each CTA publishes at most one partial, and the finisher
+// collects exactly the other contributors' partials.
 static void check_decode(int T, int KT, int sms) {
     const int W = T * KT;
     const int P = W < sms ? W : sms;   // the decode launcher's grid
     std::vector<int> cover(static_cast<size_t>(W), 0);
-    std::map<int, std::vector<Piece>> pieces;
-    std::set<std::pair<int, int>> slots;
+    std::map<int, std::vector<int>> published;   // tile -> CTAs that published a partial of it
+    std::map<int, int> finished;                 // tile -> finishing CTA
+    std::vector<int> n_pub(static_cast<size_t>(P), 0);
     for (int c = 0; c < P; ++c) {
         const int u0 = run_begin(c, W, P), u1 = run_begin(c + 1, W, P);
         CHECK(u1 > u0, "decode cta %d has an empty run (W=%d P=%d)", c, W, P);
@@ -120,19 +126,36 @@ static void check_decode(int T, int KT, int sms) {
         while (next_seg(u, u1, KT, sg)) {
             for (int k = sg.ks; k < sg.ke; ++k) ++cover[static_cast<size_t>(sg.tile) * KT + k];
             const int tb = sg.tile * KT;
-            const int cf = owner(tb, W, P), cl = owner(tb + KT - 1, W, P);
+            const int cf = split_finisher(sg.tile, KT, W, P), cl = owner(tb + KT - 1, W, P);
             if (cl == cf) {
                 CHECK(sg.ks == 0 && sg.ke == KT, "decode tile %d owned by one cta but cut", sg.tile);
                 continue;
             }
-            const int slot = (tb + sg.ks == u0) ? 0 : 1;
-            CHECK(slots.insert({c, slot}).second, "decode cta %d writes slot %d twice", c, slot);
-            pieces[sg.tile].push_back({c, slot, sg.ks, sg.ke});
+            if (c == cf) {
+                CHECK(tb + sg.ke == u1, "decode tile %d: finisher cta %d's segment is not its run's last", sg.tile, c);
+                CHECK(sg.ks == 0, "decode tile %d: finisher cta %d does not hold the first unit", sg.tile, c);
+                CHECK(finished.insert({sg.tile, c}).second, "decode tile %d finished twice", sg.tile);
+            } else {
+                CHECK(tb + sg.ks == u0, "decode tile %d: cta %d's published segment is not its run's first", sg.tile, c);
+                published[sg.tile].push_back(c);
+                CHECK(++n_pub[static_cast<size_t>(c)] == 1, "decode cta %d publishes two partials", c);
+            }
         }
     }
     for (size_t i = 0; i < cover.size(); ++i)
         CHECK(cover[i] == 1, "decode unit %zu processed %d times (T=%d KT=%d)", i, cover[i], T, KT);
-    check_split_tiles(pieces, KT, W, P, 0, "decode");
+    for (const auto& kv : published) {
+        const int t = kv.first, tb = t * KT;
+        const int cf = owner(tb, W, P), cl = owner(tb + KT - 1, W, P);
+        CHECK(finished.count(t) == 1 && finished[t] == cf, "decode tile %d has no finisher", t);
+        CHECK(static_cast<int>(kv.second.size()) == cl - cf, "decode tile %d: %zu partials, the finisher waits for %d",
+              t, kv.second.size(), cl - cf);
+        for (size_t i = 0; i < kv.second.size(); ++i)
+            CHECK(kv.second[i] == cf + 1 + static_cast<int>(i), "decode tile %d: partial of cta %d out of order", t,
+                  kv.second[i]);
+    }
+    for (const auto& kv : finished)
+        CHECK(published.count(kv.first) == 1, "decode tile %d finished with no partials to collect", kv.first);
 }
 
 int main() {
