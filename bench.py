@@ -644,6 +644,8 @@ def run_workload(a):
     name = a.workload
     wl = WORKLOADS[name]
     s = wl["shape"]
+    if a.layers:
+        s = s.replace(n_layers=a.layers)   # a shallower copy of the shape (profiling one kernel on a small case)
     stream = torch.cuda.current_stream()
     w = make_weights(s, weight_seed(wl["index"]), device=dev)
     model = llb.Model(llb.args_from_shape(s), device=dev)
@@ -674,7 +676,8 @@ def run_workload(a):
                 once, _ = _timed(g.replay, 20, stream)
                 ms, clk = _timed(g.replay, max(100, a.iters, _reps_for(once)), stream, clocks=True)
                 byts = decode_step_bytes(s, B, L + 1)
-                out.append({"workload": name, "batch": B, "context": L + 1, "us_per_step": round(ms * 1e3, 2),
+                out.append({"workload": name, "n_layers": s.n_layers, "batch": B, "context": L + 1,
+                            "us_per_step": round(ms * 1e3, 2),
                             "tok_s": round(B / (ms / 1e3), 1), "GB_s": round(byts / ms / 1e6, 1),
                             "hbm_frac": round(byts / ms / 1e6 / hbm, 4), "peak_source": peak_src,
                             "clocks": clk})
@@ -736,7 +739,8 @@ def run_workload(a):
         n_tok = sum(lens)
         mean_ctx = sum(lens) / B + steps / 2
         byts = decode_step_bytes(s, B, int(mean_ctx), logits=False) if s.dtype != "f32" else None
-        out.append({"workload": name, "batch": B, "prompt_tokens": n_tok, "prefill_ms": round(pre_ms, 3),
+        out.append({"workload": name, "n_layers": s.n_layers, "batch": B, "prompt_tokens": n_tok,
+                    "prefill_ms": round(pre_ms, 3),
                     "prefill_tok_s": round(n_tok / (pre_ms / 1e3), 1), "decode_steps": steps,
                     "decode_ms_per_step": round(dec_ms, 4), "decode_tok_s": round(B / (dec_ms / 1e3), 1),
                     "decode_hbm_frac": round(byts / dec_ms / 1e6 / hbm, 4) if byts else None,
@@ -744,6 +748,54 @@ def run_workload(a):
         del g
     for line in out:
         print(json.dumps(line), flush=True)
+
+
+def run_profile_steps(a):
+    """A short, fixed launch sequence for ncu captures: the 7B shape (--layers
+    to shorten it), one 4 x 512 prefill, then --profile-steps greedy decode
+    steps launched directly (no graph).  With --profile-prefill-kernels the
+    prefill projections are also timed one by one (events; the prefill runs
+    no programmatic dependent launch) and printed as one JSON line."""
+    import decoder_only_transformer_llama_b200 as llb
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    s = L7B.replace(n_layers=a.layers) if a.layers else L7B
+    w = make_weights(s, weight_seed(WL["index"]), device=dev)
+    model = llb.Model(llb.args_from_shape(s), device=dev)
+    model.load(w)
+    del w
+    torch.cuda.empty_cache()
+    B, T = WL["batch"], WL["prompt_len"]
+    prompt = make_tokens(s.vocab_size, (B, T), token_seed(WL["index"])).to(dev)
+    logits = torch.empty(B, s.vocab_size, device=dev)
+    tok = torch.empty(B, dtype=torch.int32, device=dev)
+    pos = torch.full((B,), T, dtype=torch.int32, device=dev)
+    if a.profile_prefill_kernels:
+        model.prefill(prompt, logits=logits)
+        torch.cuda.synchronize()
+        model.profile_start(8 * s.n_layers + 8)
+    model.prefill(prompt, logits=logits)
+    if a.profile_prefill_kernels:
+        recs = model.profile_stop(8 * s.n_layers + 8)
+        names = ["wq/wk/wv", "wo", "w1/w3", "w2"]
+        per = {}
+        for i, r in enumerate(recs):
+            if r[3] <= 64:
+                continue
+            k = names[i % 4] if i < 4 * s.n_layers else "output"
+            per.setdefault(k, [0.0, 0])
+            per[k][0] += r[0]
+            per[k][1] += r[2]
+        print(json.dumps({"prefill_projection_ms": {k: round(v[0], 3) for k, v in per.items()},
+                          "prefill_projection_tflops": {k: round(v[1] / (v[0] / 1e3) / 1e12, 1)
+                                                        for k, v in per.items() if v[0] > 0}}), flush=True)
+    llb.sample(logits, 0.0, 0.9, None, tok)
+    for _ in range(a.profile_steps):
+        model.decode_step(tok, pos, temperature=0.0, next_tokens=tok, advance=True)
+    torch.cuda.synchronize()
+    assert model.status() == 0
+    print(json.dumps({"profile_steps": a.profile_steps, "n_layers": s.n_layers,
+                      "launches": llb.launch_count()}), flush=True)
 
 
 # ----------------------------------------------------------------------------- main
@@ -762,9 +814,19 @@ def main():
     ap.add_argument("--workload", default="7b", choices=list(WORKLOADS),
                     help="7b is the headline line; the others print throughput lines of their own")
     ap.add_argument("--decode-steps", type=int, default=0, help="decode steps of the 70b_slice workload")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="--workload / --profile-steps: run the shape with this many layers (small cases for kernel profiles)")
+    ap.add_argument("--profile-steps", type=int, default=0,
+                    help="ncu helper: 7B prefill 4x512 + this many directly launched decode steps, then exit")
+    ap.add_argument("--profile-prefill-kernels", action="store_true",
+                    help="with --profile-steps: time the prefill projections one by one and print them")
     a = ap.parse_args()
     if a.op_linear:
         run_op_linear(a)
+        return
+    if a.profile_steps or a.profile_prefill_kernels:
+        a.profile_steps = max(a.profile_steps, 1)
+        run_profile_steps(a)
         return
     if a.workload != "7b":
         run_workload(a)

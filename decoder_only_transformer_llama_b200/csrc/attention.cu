@@ -85,6 +85,15 @@ template <> struct Vec<f16, 4> {
 // (bounded) for that count, then merges its own state with the published
 // ones in CTA order (deterministic).  Only a finisher waits, and only for
 // other CTAs' first segments, which never wait.
+// Fewest cache units (64-key blocks) a CTA's run holds when there are fewer
+// than that many per CTA of the grid: short runs split every pair across many
+// CTAs, and each split adds a merge to the pair's finisher.
+constexpr int kMinUnitsPerCta = 1;
+__device__ __forceinline__ int attn_ctas(long long W, int grid) {
+    const long long p = (W + kMinUnitsPerCta - 1) / kMinUnitsPerCta;
+    return static_cast<int>(p < grid ? p : grid);
+}
+
 __device__ __forceinline__ long long run_begin64(long long c, long long W, long long P) { return c * W / P; }
 __device__ __forceinline__ int owner64(long long u, long long W, long long P) {
     return static_cast<int>(((u + 1) * P - 1) / W);
@@ -206,7 +215,7 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
     int n_early = 0;                             // thread 0: units issued before the dependency
     {
         const long long W0 = static_cast<long long>(s_cum[B]) * nkv;
-        const int P0 = static_cast<int>(W0 < gridDim.x ? W0 : gridDim.x);
+        const int P0 = attn_ctas(W0, gridDim.x);
         if (threadIdx.x == 0 && blockIdx.x < P0) {
             const long long v0 = run_begin64(blockIdx.x, W0, P0), v1 = run_begin64(blockIdx.x + 1, W0, P0);
             icur = cur_at(v0);
@@ -244,7 +253,7 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
         }
     }
     const long long W = static_cast<long long>(s_cum[B]) * nkv;
-    const int P = static_cast<int>(W < gridDim.x ? W : gridDim.x), c = blockIdx.x;
+    const int P = attn_ctas(W, gridDim.x), c = blockIdx.x;
     if (c >= P) {
         if (threadIdx.x == 0) tl_stamp(tl);
         return;

@@ -37,14 +37,50 @@ __host__ __device__ __forceinline__ bool next_seg(int& u, int u1, int KT, Seg& s
     return true;
 }
 
+// The inputs of a tile's epilogue that do not depend on its accumulator,
+// loaded while its MMAs still run: the RoPE factors of each token column
+// (QKV: from the row's position), or the old residual values and the next
+// norm's weight (residual modes).
+template <int BN>
+struct EpiPre {
+    float2 cs[BN];
+    float xo[BN];
+    float wn;
+};
+
+template <int BN>
+__device__ __forceinline__ void prefetch_tile(EpiPre<BN>& pre, int t, int r, int nb, int N, const Epi& ep,
+                                              const NormIO& nio, const int (&posv)[BN]) {
+    const int n = t * 128 + r;
+    const bool row_ok = n < N;
+    if (ep.mode == EPI_QKV) {
+        const bool is_q = n < ep.nq;
+        const int cc = n - ep.nq;
+        const bool rot = is_q || cc < ep.nkvc;
+        const int d = is_q ? n % ep.hd : cc % ep.hd;
+#pragma unroll
+        for (int b = 0; b < BN; ++b) {
+            const bool okp = row_ok && rot && posv[b] >= 0 && posv[b] < ep.max_seq;
+            pre.cs[b] = okp ? ep.rope[static_cast<long long>(posv[b]) * (ep.hd / 2) + (d >> 1)] : make_float2(1.f, 0.f);
+        }
+    } else if (ep.mode == EPI_RESID_F32) {
+        pre.wn = (row_ok && nio.ssq_out) ? nio.w_next[n] : 0.f;
+#pragma unroll
+        for (int b = 0; b < BN; ++b)
+            pre.xo[b] = (row_ok && b < nb) ? ep.out[static_cast<long long>(b) * ep.ldo + n] : 0.f;
+    }
+}
+
 // Epilogue of one finished 128-row weight tile t: v[b] = acc[row r of the
 // tile, token column b] for the nb real token columns.  All 128 epilogue
 // threads of the CTA call it together (the residual + sum-of-squares mode
-// synchronises them on named barrier 2).
+// synchronises them on named barrier 2).  `pre` (or null: loaded here) holds
+// the inputs prefetch_tile loaded; `posv` the token columns' positions.
 template <int BN, typename T>
 __device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int lane, int q, int epi_tid, int nb,
                                             int N, int n_tiles, const Epi& ep, const NormIO& nio, bool scale_in,
-                                            const float* rs, float* red) {
+                                            const float* rs, float* red, const EpiPre<BN>* pre = nullptr,
+                                            const int* posv_in = nullptr) {
     if (scale_in) {
 #pragma unroll
         for (int b = 0; b < BN; ++b) v[b] *= (b < nb) ? rs[b] : 0.f;
@@ -78,13 +114,21 @@ __device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int la
         for (int b0 = 0; b0 < BN; b0 += 16) {
             int posv[16];
             float2 cs[16];
+            if (pre) {
 #pragma unroll
-            for (int u = 0; u < 16; ++u) posv[u] = (b0 + u < nb) ? ep.tok_pos[b0 + u] : -1;
+                for (int u = 0; u < 16; ++u) {
+                    posv[u] = posv_in[b0 + u];
+                    cs[u] = pre->cs[b0 + u];
+                }
+            } else {
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const bool okp = row_ok && posv[u] >= 0 && posv[u] < ep.max_seq && (is_q || is_k);
-                cs[u] = okp ? ep.rope[static_cast<long long>(posv[u]) * (ep.hd / 2) + (d >> 1)]
-                            : make_float2(1.f, 0.f);
+                for (int u = 0; u < 16; ++u) posv[u] = (b0 + u < nb) ? ep.tok_pos[b0 + u] : -1;
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const bool okp = row_ok && posv[u] >= 0 && posv[u] < ep.max_seq && (is_q || is_k);
+                    cs[u] = okp ? ep.rope[static_cast<long long>(posv[u]) * (ep.hd / 2) + (d >> 1)]
+                                : make_float2(1.f, 0.f);
+                }
             }
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
@@ -107,14 +151,15 @@ __device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int la
     } else if (ep.mode == EPI_RESID_F32 && nio.ssq_out) {
         // residual add, plus this tile's share of sum(x^2) for the next RMSNorm;
         // the old x values of a 16-column group are loaded together
-        const float wn = row_ok ? nio.w_next[n] : 0.f;
+        const float wn = pre ? pre->wn : (row_ok ? nio.w_next[n] : 0.f);
         float xo[16];
 #pragma unroll
         for (int b = 0; b < BN; ++b) {
             if ((b & 15) == 0) {
 #pragma unroll
                 for (int u = 0; u < 16; ++u)
-                    xo[u] = (row_ok && b + u < nb) ? ep.out[static_cast<long long>(b + u) * ep.ldo + n] : 0.f;
+                    xo[u] = pre ? pre->xo[b + u]
+                                : ((row_ok && b + u < nb) ? ep.out[static_cast<long long>(b + u) * ep.ldo + n] : 0.f);
             }
             float sq = 0.f;
             if (row_ok && b < nb) {
@@ -153,7 +198,8 @@ __device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int la
                 float xo[16];
 #pragma unroll
                 for (int u = 0; u < 16; ++u)
-                    xo[u] = (b0 + u < nb) ? ep.out[static_cast<long long>(b0 + u) * ep.ldo + n] : 0.f;
+                    xo[u] = pre ? pre->xo[b0 + u]
+                                : ((b0 + u < nb) ? ep.out[static_cast<long long>(b0 + u) * ep.ldo + n] : 0.f);
 #pragma unroll
                 for (int u = 0; u < 16; ++u)
                     if (b0 + u < nb) ep.out[static_cast<long long>(b0 + u) * ep.ldo + n] = xo[u] + v[b0 + u];
@@ -188,8 +234,18 @@ __device__ __forceinline__ void decode_epilogue_loop(uint32_t tmem_lane, uint64_
     Seg sg;
     int j = 0;
     const int nb = M < BN ? M : BN;
+    // narrow steps load each finished tile's epilogue inputs while its MMAs run
+    constexpr bool kPre = BN <= 32;
+    int posv[BN];
+#pragma unroll
+    for (int b = 0; b < BN; ++b) posv[b] = (kPre && ep.mode == EPI_QKV && b < nb) ? ep.tok_pos[b] : -1;
     while (next_seg(u, u1, KT, sg)) {
         const int acc = j & 1;
+        const int t = sg.tile;
+        const int tb = t * KT;
+        const int cf = split_finisher(t, KT, W, P), cl = owner(tb + KT - 1, W, P);
+        EpiPre<BN> pre;
+        if (kPre && !(cl > cf && c != cf)) prefetch_tile<BN>(pre, t, r, nb, N, ep, nio, posv);
         const bool ok_wait = mbar_wait(&tfull[acc], (j >> 1) & 1, wlim);
         tc_fence_after();
         float v[BN];
@@ -204,9 +260,6 @@ __device__ __forceinline__ void decode_epilogue_loop(uint32_t tmem_lane, uint64_
             if (epi_tid == 0) report_status(ep.status, LLAMA_ERR_DEVICE_TIMEOUT);
             break;
         }
-        const int t = sg.tile;
-        const int tb = t * KT;
-        const int cf = split_finisher(t, KT, W, P), cl = owner(tb + KT - 1, W, P);
         if (cl > cf && c != cf) {
             // a split tile this CTA does not finish (its run's first segment):
             // publish the partial and count it
@@ -272,7 +325,8 @@ __device__ __forceinline__ void decode_epilogue_loop(uint32_t tmem_lane, uint64_
             }
             if (epi_tid == 0) counters[t] = 0;
         }
-        finish_tile<BN, T>(v, t, r, lane, q, epi_tid, nb, N, n_tiles, ep, nio, scale_in, rs, red);
+        finish_tile<BN, T>(v, t, r, lane, q, epi_tid, nb, N, n_tiles, ep, nio, scale_in, rs, red, kPre ? &pre : nullptr,
+                           posv);
     }
 }
 
