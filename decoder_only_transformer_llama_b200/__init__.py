@@ -340,6 +340,19 @@ class Model:
         _check(_lib.llama_timeline_stop(self.handle, en, kd, by, max_records, ctypes.byref(n)))
         return [(int(en[i]), TIMELINE_KINDS.get(kd[i], str(kd[i])), int(by[i])) for i in range(n.value)]
 
+    def tp_buffers(self):
+        """(partial sums phase 0, phase 1, flag words, logits) device addresses of a shard."""
+        p0, p1, fl, lg = _vp(), _vp(), _vp(), _vp()
+        _check(_lib.llama_tp_buffers(self.handle, ctypes.byref(p0), ctypes.byref(p1), ctypes.byref(fl),
+                                     ctypes.byref(lg)))
+        return p0.value, p1.value, fl.value, lg.value
+
+    def tp_bind(self, part0, part1, flags, logits):
+        """Bind every rank's buffers (lists indexed by rank, addresses mapped into this process)."""
+        n = self.tp_size
+        arr = [(_vp * n)(*[int(v) for v in t]) for t in (part0, part1, flags, logits)]
+        _check(_lib.llama_tp_bind(self.handle, *arr))
+
     def debug_stall(self, which: str, unit: int = 0, wait_limit_ns: int = 1_000_000):
         """Arm a one-shot stalled producer in the next `which` launch
         ("projection", "attention" or "none"): tests of the device timeout."""
@@ -351,6 +364,65 @@ class Model:
         s = ctypes.c_int()
         _check(_lib.llama_model_status(self.handle, ctypes.byref(s)))
         return s.value
+
+
+def tp_bind_distributed(model: "Model", group=None, ipc=None):
+    """Ranks of a tensor-parallel group on separate GPUs (one process per GPU,
+    torch.distributed initialised, one rank per shard): shares this shard's
+    buffers with the other ranks through a CUDA IPC handle of the allocation
+    that holds its arena, maps theirs, and binds every rank's buffers
+    (llama_tp_bind).  Call it on every rank, after creating the shard.
+    `ipc` replaces the CUDA IPC calls (tests of the exchange on CPU): an
+    object with base_of(ptr) -> (allocation base, handle bytes) and
+    open(handle bytes) -> mapped base."""
+    import torch.distributed as dist
+    if ipc is None:
+        ipc = _CudaIpc()
+    bufs = model.tp_buffers()
+    base, handle = ipc.base_of(bufs[0])
+    mine = {"rank": model.tp_rank, "handle": handle, "offsets": [b - base for b in bufs]}
+    world = dist.get_world_size(group)
+    if world != model.tp_size:
+        raise ValueError(f"process group of {world} ranks for a shard of a {model.tp_size}-rank group")
+    everyone = [None] * world
+    dist.all_gather_object(everyone, mine, group=group)
+    tables = [[0] * model.tp_size for _ in range(4)]
+    model._tp_mapped = []
+    for entry in everyone:
+        r = entry["rank"]
+        mapped = base if r == model.tp_rank else ipc.open(entry["handle"])
+        if r != model.tp_rank:
+            model._tp_mapped.append(mapped)
+        for i in range(4):
+            tables[i][r] = mapped + entry["offsets"][i]
+    model.tp_bind(*tables)
+    return tables
+
+
+class _CudaIpc:
+    """CUDA IPC through cuda-python: the allocation base of a device pointer,
+    its IPC handle, and the mapping of a peer's handle."""
+
+    def __init__(self):
+        from cuda.bindings import driver, runtime
+        self._drv, self._rt = driver, runtime
+
+    def base_of(self, ptr: int):
+        err, base, _size = self._drv.cuMemGetAddressRange(ptr)
+        if int(err) != 0:
+            raise RuntimeError(f"cuMemGetAddressRange failed ({err})")
+        err, h = self._rt.cudaIpcGetMemHandle(int(base))
+        if int(err) != 0:
+            raise RuntimeError(f"cudaIpcGetMemHandle failed ({err})")
+        return int(base), bytes(h.reserved)
+
+    def open(self, handle: bytes) -> int:
+        h = self._rt.cudaIpcMemHandle_t()
+        h.reserved = handle
+        err, ptr = self._rt.cudaIpcOpenMemHandle(h, self._rt.cudaIpcMemLazyEnablePeerAccess)
+        if int(err) != 0:
+            raise RuntimeError(f"cudaIpcOpenMemHandle failed ({err})")
+        return int(ptr)
 
 
 class TPGroup:

@@ -125,3 +125,70 @@ def test_plan_keeps_query_groups_with_their_kv_head():
             assert covered == list(range(n))
     with pytest.raises(ValueError):
         TP.shard_plan(64, 8, 128, 28672, 32000, 0, 16)   # 8 KV heads cannot split 16 ways
+
+
+class _FakeShard:
+    """Stands in for a shard on its own GPU: fixed buffer addresses inside a
+    per-rank arena, and a record of what was bound."""
+
+    def __init__(self, rank, tp):
+        self.tp_rank, self.tp_size = rank, tp
+        self.base = 0x10000000 * (rank + 1)
+        self.bound = None
+
+    def tp_buffers(self):
+        b = self.base
+        return b + 0x100 + self.tp_rank, b + 0x2000, b + 0x3000 + 8 * self.tp_rank, b + 0x4000
+
+    def tp_bind(self, *tables):
+        self.bound = [list(t) for t in tables]
+
+
+class _FakeIpc:
+    def __init__(self, shard):
+        self.shard = shard
+
+    def base_of(self, ptr):
+        return self.shard.base, b"handle-of-rank-%d" % self.shard.tp_rank
+
+    def open(self, handle):
+        r = int(handle.decode().rsplit("-", 1)[1])
+        return 0x90000000 + 0x1000000 * r      # where this process maps rank r's arena
+
+
+def _bind_rank(rank, world, port, q):
+    try:
+        os.environ["MASTER_ADDR"] = "127.0.0.1"
+        os.environ["MASTER_PORT"] = str(port)
+        dist.init_process_group("gloo", rank=rank, world_size=world)
+        import decoder_only_transformer_llama_b200 as llb
+        shard = _FakeShard(rank, world)
+        llb.tp_bind_distributed(shard, ipc=_FakeIpc(shard))
+        dist.barrier()
+        dist.destroy_process_group()
+        q.put((rank, shard.bound, None))
+    except Exception as e:  # pragma: no cover - reported to the parent
+        q.put((rank, None, repr(e)))
+
+
+def test_distributed_binding_maps_every_ranks_buffers():
+    """Ranks on separate GPUs exchange their buffers' offsets and IPC handles;
+    each binds, for every rank, that rank's mapped arena plus its offsets (its
+    own arena for itself)."""
+    world = 3
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_bind_rank, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=300) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+    for rank, bound, exc in res:
+        assert exc is None, (rank, exc)
+        for r in range(world):
+            owner = _FakeShard(r, world)
+            mapped = owner.base if r == rank else 0x90000000 + 0x1000000 * r
+            want = [mapped + (b - owner.base) for b in owner.tp_buffers()]
+            assert [bound[i][r] for i in range(4)] == want, (rank, r)
