@@ -88,7 +88,7 @@ template <> struct Vec<f16, 4> {
 // Fewest cache units (64-key blocks) a CTA's run holds when there are fewer
 // than that many per CTA of the grid: short runs split every pair across many
 // CTAs, and each split adds a merge to the pair's finisher.
-constexpr int kMinUnitsPerCta = 1;
+constexpr int kMinUnitsPerCta = 2;
 __device__ __forceinline__ int attn_ctas(long long W, int grid) {
     const long long p = (W + kMinUnitsPerCta - 1) / kMinUnitsPerCta;
     return static_cast<int>(p < grid ? p : grid);
@@ -183,6 +183,7 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
     const uint64_t wlim = wait_ns > 0 ? static_cast<uint64_t>(wait_ns) : kWaitLimitNs;
     const int stall_i = blockIdx.x == 0 ? stall : -1;   // tests of the timeout path only
     Cur icur = {0, 0, 0};                        // issue cursor (thread 0)
+    const uint64_t pol_kv = l2_policy_evict_first();   // read once per step
     auto issue = [&](int i) {                    // i-th unit of this run into ring slot i % NSLOT
         const int ctx = s_pos[icur.b] + 1;
         const int j0 = icur.j * kChunk;
@@ -191,8 +192,9 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
         const long long ho = head_off(icur);
         if (i != stall_i) {
             mbar_arrive_expect_tx(&bar[i % NSLOT], 2u * n * ROW);
-            bulk_load(slot, kc + ho + static_cast<long long>(j0) * HD, n * ROW, &bar[i % NSLOT]);
-            bulk_load(slot + CH_BYTES, vc + ho + static_cast<long long>(j0) * HD, n * ROW, &bar[i % NSLOT]);
+            bulk_load_hint(slot, kc + ho + static_cast<long long>(j0) * HD, n * ROW, &bar[i % NSLOT], pol_kv);
+            bulk_load_hint(slot + CH_BYTES, vc + ho + static_cast<long long>(j0) * HD, n * ROW, &bar[i % NSLOT],
+                           pol_kv);
         }
         advance(icur);
     };

@@ -92,6 +92,7 @@ __device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int la
         // w1 rows, lanes 16-31 the matching w3 rows
 #pragma unroll
         for (int b = 0; b < BN; ++b) {
+            if (b >= nb) break;   // uniform over the CTA
             const float up = __shfl_xor_sync(0xffffffffu, v[b], 16);
             if (lane < 16 && row_ok && b < nb) {
                 const int h = (n >> 5) * 16 + (n & 15);
@@ -133,6 +134,7 @@ __device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int la
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
                 const int b = b0 + u;
+                if (b >= nb) break;   // uniform over the CTA
                 const float partner = __shfl_xor_sync(0xffffffffu, v[b], 1);
                 const int pos = posv[u];
                 if (!row_ok || b >= nb || pos < 0 || pos >= ep.max_seq) continue;
@@ -155,6 +157,7 @@ __device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int la
         float xo[16];
 #pragma unroll
         for (int b = 0; b < BN; ++b) {
+            if (b >= nb) break;   // uniform over the CTA
             if ((b & 15) == 0) {
 #pragma unroll
                 for (int u = 0; u < 16; ++u)
@@ -266,7 +269,7 @@ __device__ __forceinline__ void decode_epilogue_loop(uint32_t tmem_lane, uint64_
             float* my = part + (static_cast<long long>(c) * 128 + r) * BN;
 #pragma unroll
             for (int b = 0; b < BN; b += 4)
-                *reinterpret_cast<float4*>(my + b) = make_float4(v[b], v[b + 1], v[b + 2], v[b + 3]);
+                if (b < nb) *reinterpret_cast<float4*>(my + b) = make_float4(v[b], v[b + 1], v[b + 2], v[b + 3]);
             __threadfence();
             named_sync(1, 128);
             if (epi_tid == 0) atomicAdd(&counters[t], 1);
@@ -295,10 +298,30 @@ __device__ __forceinline__ void decode_epilogue_loop(uint32_t tmem_lane, uint64_
                 break;
             }
             __threadfence();
-            // partials after this CTA's own, in CTA order, CB contributors per
-            // batch of independent loads
+            // partials after this CTA's own, in CTA order.  Up to 4 token
+            // columns: one float4 per contributor, 8 contributors per batch of
+            // independent loads (each batch is an L2 round trip under full
+            // HBM load); wider: CB contributors' whole rows per batch.
             constexpr int CB = BN <= 16 ? 4 : (BN <= 32 ? 2 : 1);
-            for (int cb = cf + 1; cb <= cl; cb += CB) {
+            if (nb <= 4) {
+                for (int cb = cf + 1; cb <= cl; cb += 8) {
+                    float4 f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        if (cb + e <= cl)
+                            f[e] = __ldcg(reinterpret_cast<const float4*>(part + (static_cast<long long>(cb + e) * 128 + r) * BN));
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        if (cb + e <= cl) {
+                            v[0] += f[e].x;
+                            v[1] += f[e].y;
+                            v[2] += f[e].z;
+                            v[3] += f[e].w;
+                        }
+                    }
+                }
+            }
+            for (int cb = cf + 1; nb > 4 && cb <= cl; cb += CB) {
                 float4 f[CB][BN / 4];
 #pragma unroll
                 for (int e = 0; e < CB; ++e) {

@@ -89,12 +89,13 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
         const int nunits = u1 - u0;
         const int npre = nunits < STAGES ? nunits : STAGES;
         stall = c == 0 ? ep.stall - 1 : -1;   // tests of the timeout path only
+        const uint64_t pol_w = l2_policy_evict_first();   // weights are read once per step
         int t0 = u0 / KT, k0 = u0 - t0 * KT;          // walk (tile, k) without divisions
         int tt = t0, kk = k0;
         for (int i = 0; i < npre; ++i) {
             if (i != stall) {
                 mbar_arrive_expect_tx(&full[i], STAGE);
-                tma_load_2d(smem + i * STAGE, &mapW, kk * 64, tt * 128, &full[i]);
+                tma_load_2d_hint(smem + i * STAGE, &mapW, kk * 64, tt * 128, &full[i], pol_w);
             }
             if (++kk == KT) { kk = 0; ++tt; }
         }
@@ -116,7 +117,7 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
             if (i != stall) {
                 uint8_t* st = smem + s * STAGE;
                 mbar_arrive_expect_tx(&full[s], STAGE);
-                tma_load_2d(st, &mapW, kk * 64, tt * 128, &full[s]);
+                tma_load_2d_hint(st, &mapW, kk * 64, tt * 128, &full[s], pol_w);
 #pragma unroll
                 for (int rr = 0; rr < BN / 16; ++rr)
                     tma_load_2d(st + kABytes + rr * 2048, &mapX, kk * 64, rr * 16, &full[s]);

@@ -430,7 +430,7 @@ static int launch_tcp(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, in
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&g_sms_tc, cudaDevAttrMultiProcessorCount, dev);
         if (g_sms_tc <= 0) g_sms_tc = 148;
-        if (g_sms_tc > kMaxDecodeCtas) g_sms_tc = kMaxDecodeCtas;
+        if (g_sms_tc > kMaxPrefillCtas) g_sms_tc = kMaxPrefillCtas;
     }
     TcPlan plan;
     plan.TM = (M + 127) / 128;

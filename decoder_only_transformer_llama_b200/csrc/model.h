@@ -13,11 +13,12 @@ namespace llb {
 
 constexpr int kMaxRows = 256;         // max_batch_size limit (by-value row tables)
 constexpr int kChunk = 64;            // keys per chunk in decode attention
-constexpr int kMaxDecodeCtas = 256;   // persistent CTAs of the decode projection kernel
+constexpr int kMaxDecodeCtas = 512;   // persistent CTAs of the decode projection kernel (two per SM)
+constexpr int kMaxPrefillCtas = 256;  // persistent CTAs of the prefill projection kernel (one per SM)
 // fp32 partials of split tiles, two per persistent CTA: 128 x 64 blocks in the
 // decode projection, 128 x 256 tiles in the prefill projection
 constexpr size_t kDecodePartBytes = static_cast<size_t>(kMaxDecodeCtas) * 2 * 128 * 64 * 4;
-constexpr size_t kPrefillPartBytes = static_cast<size_t>(kMaxDecodeCtas) * 2 * 128 * 256 * 4;
+constexpr size_t kPrefillPartBytes = static_cast<size_t>(kMaxPrefillCtas) * 2 * 128 * 256 * 4;
 constexpr size_t kGemmPartBytes = kPrefillPartBytes > kDecodePartBytes ? kPrefillPartBytes : kDecodePartBytes;
 constexpr int kMaxTiles = 4096;       // tile counters: N / 128 of the widest projection
 constexpr int kMaxAttnCtas = 1024;    // persistent CTAs of the decode attention kernel
