@@ -425,22 +425,52 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
                     part_ml[(static_cast<long long>(slot_id) * NREP + r) * 2 + 1] = L;
                 }
             } else {
-                // merge this CTA's (M, L, acc) with the published ones, in CTA order
-                float Mt = M;
-                for (int cc = cf + 1; cc <= cl; ++cc) {
-                    const int sid = cc * 2 + (run_begin64(cc, W, P) >= pair_u0 ? 0 : 1);
-                    Mt = fmaxf(Mt, __ldcg(part_ml + (static_cast<long long>(sid) * NREP + r) * 2));
-                }
-                const float f0 = (M == -INFINITY) ? 0.f : __expf(M - Mt);
-                float Lt = 0.f, at = 0.f;
-                Lt += L * f0;
-                at += acc * f0;
-                for (int cc = cf + 1; cc <= cl; ++cc) {
-                    const int sid = cc * 2 + (run_begin64(cc, W, P) >= pair_u0 ? 0 : 1);
-                    const float mm = __ldcg(part_ml + (static_cast<long long>(sid) * NREP + r) * 2);
-                    const float f = (mm == -INFINITY) ? 0.f : __expf(mm - Mt);
-                    Lt += __ldcg(part_ml + (static_cast<long long>(sid) * NREP + r) * 2 + 1) * f;
-                    at += __ldcg(part_o + (static_cast<long long>(sid) * NREP + r) * HD + d) * f;
+                // merge this CTA's (M, L, acc) with the published ones, in CTA
+                // order.  Every other contributor published its first segment
+                // (slot 0).  Up to kMergeBatch contributors' values are loaded
+                // together (one L2 round trip under full HBM load), more in a
+                // pass for the maxima and one per contributor after it.
+                constexpr int kMergeBatch = 8;
+                const int ncon = cl - cf;
+                float Mt = M, Lt = 0.f, at = 0.f;
+                if (ncon <= kMergeBatch) {
+                    float mm[kMergeBatch], ll[kMergeBatch], oo[kMergeBatch];
+#pragma unroll
+                    for (int e = 0; e < kMergeBatch; ++e) {
+                        if (e < ncon) {
+                            const long long base = static_cast<long long>((cf + 1 + e) * 2) * NREP + r;
+                            mm[e] = __ldcg(part_ml + base * 2);
+                            ll[e] = __ldcg(part_ml + base * 2 + 1);
+                            oo[e] = __ldcg(part_o + base * HD + d);
+                        }
+                    }
+#pragma unroll
+                    for (int e = 0; e < kMergeBatch; ++e)
+                        if (e < ncon) Mt = fmaxf(Mt, mm[e]);
+                    const float f0 = (M == -INFINITY) ? 0.f : __expf(M - Mt);
+                    Lt += L * f0;
+                    at += acc * f0;
+#pragma unroll
+                    for (int e = 0; e < kMergeBatch; ++e) {
+                        if (e < ncon) {
+                            const float f = (mm[e] == -INFINITY) ? 0.f : __expf(mm[e] - Mt);
+                            Lt += ll[e] * f;
+                            at += oo[e] * f;
+                        }
+                    }
+                } else {
+                    for (int cc = cf + 1; cc <= cl; ++cc)
+                        Mt = fmaxf(Mt, __ldcg(part_ml + (static_cast<long long>(cc * 2) * NREP + r) * 2));
+                    const float f0 = (M == -INFINITY) ? 0.f : __expf(M - Mt);
+                    Lt += L * f0;
+                    at += acc * f0;
+                    for (int cc = cf + 1; cc <= cl; ++cc) {
+                        const long long base = static_cast<long long>(cc * 2) * NREP + r;
+                        const float mm = __ldcg(part_ml + base * 2);
+                        const float f = (mm == -INFINITY) ? 0.f : __expf(mm - Mt);
+                        Lt += __ldcg(part_ml + base * 2 + 1) * f;
+                        at += __ldcg(part_o + base * HD + d) * f;
+                    }
                 }
                 out[static_cast<long long>(cur.b) * nq + h * HD + d] = from_f32<T>(at / Lt);
             }
