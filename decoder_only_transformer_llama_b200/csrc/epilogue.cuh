@@ -53,4 +53,21 @@ __device__ __forceinline__ void epi_qkv_pair(const Epi& ep, int m, int n, float 
     dst[1] = from_f32<T>(v1);
 }
 
+// Sum of x^2 of one token row from its n per-128-feature partial sums (fused
+// RMSNorm, consumer side), added in order; the loads are issued eight at a
+// time so that they are in flight together.
+__device__ __forceinline__ float row_ssq(const float* p, int n) {
+    float ss = 0.f;
+    int t = 0;
+    for (; t + 8 <= n; t += 8) {
+        float a[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) a[u] = p[t + u];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) ss += a[u];
+    }
+    for (; t < n; ++t) ss += p[t];
+    return ss;
+}
+
 }  // namespace llb

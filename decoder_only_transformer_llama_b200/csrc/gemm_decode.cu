@@ -166,7 +166,7 @@ linear_decode_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_cons
         if (scale_in && epi_tid < M) {
             // RMSNorm factor of token row epi_tid (fused RMSNorm, consumer side)
             float ss = 0.f;
-            for (int t2 = 0; t2 < nio.n_in; ++t2) ss += nio.ssq_in[epi_tid * nio.n_in + t2];
+            ss = row_ssq(nio.ssq_in + epi_tid * nio.n_in, nio.n_in);
             rs[epi_tid] = rsqrtf(ss / static_cast<float>(K) + nio.eps);
         }
         named_sync(1, 128);

@@ -300,7 +300,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
             float rs = 1.f, sq = 0.f;
             if (nio.ssq_in && row_ok) {
                 float ss = 0.f;
-                for (int t2 = 0; t2 < nio.n_in; ++t2) ss += nio.ssq_in[static_cast<long long>(m) * nio.n_in + t2];
+                ss = row_ssq(nio.ssq_in + static_cast<long long>(m) * nio.n_in, nio.n_in);
                 rs = rsqrtf(ss / static_cast<float>(KT * 64) + nio.eps);
             }
             if (it.ks == 0 && it.ke == KT) {
@@ -376,6 +376,264 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
     if (threadIdx.x == 0) tl_stamp(ep.tl);
 }
 
+// ---------------------------------------------------------------- CTA-pair kernel
+// The same projection with 256 x 256 tiles on a pair of SMs (a cluster of two
+// CTAs, cta_group::2).  CTA rank r of a pair holds token rows r*128..+127 of
+// the tile (the A half) and weight rows r*128..+127 (the B half); the rank-0
+// CTA issues M=256, N=256 MMAs that read both CTAs' halves from their shared
+// memory, and each CTA's tensor memory receives its 128 token rows over all
+// 256 features, so each CTA runs the same epilogue as the one-SM kernel on
+// its half.  Per 64-deep k-block an SM receives 32 KB of operands instead of
+// 48 KB for the same MMA work, and a 6-stage ring covers 6 k-blocks of
+// latency instead of 4.
+//
+// Handshakes (every wait bounded):
+//   full[s]    rank 0: both CTAs' TMA copies of stage s landed (each CTA's
+//              copies complete on rank 0's barrier; rank 0 expects both)
+//   empty[s]   each CTA: the MMAs reading stage s are done (rank 0 commits to
+//              its own and to the peer's barrier)
+//   tfull[a]   each CTA: accumulator a is complete (both commits likewise)
+//   tempty[a]  rank 0: both CTAs' epilogues drained accumulator a (count 2)
+// A CTA that gives up cannot wait on rank 0's barrier for its own copies, so
+// on that path rank 1 lets kDrainNs pass before it leaves (a copy lands within
+// microseconds) and rank 0 waits for the stages it expected.
+// A split tile is reduced per half: counters[2 * tile + r], partials of CTA
+// (2 * pair + r).  No TMA multicast.
+constexpr int kPairTile = 256;
+constexpr int kStagesPair = 6;
+constexpr int kPairHalfBytes = 128 * 128;            // 128 rows x 64 16-bit values
+constexpr int kPairStageBytes = 2 * kPairHalfBytes;  // A half + B half
+constexpr uint64_t kDrainNs = 100000;                // rank 1's wait for its copies on the give-up path
+
+template <typename E>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsTc, 1)
+linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                       int rowsA, int rowsB, TcPlan plan, Epi ep, float* __restrict__ part,
+                       int* __restrict__ counters, NormIO nio) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStagesPair * kPairStageBytes);
+    uint64_t* empty = full + kStagesPair;
+    uint64_t* tfull = empty + kStagesPair;   // [2]
+    uint64_t* tempty = tfull + 2;            // [2]
+    uint64_t* mdone = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + 1);
+    int* flag = reinterpret_cast<int*>(tmem_slot + 1);   // [0] abort, [1] arrival broadcast
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const uint32_t peer = rank ^ 1u;
+    const int P = gridDim.x >> 1, c = blockIdx.x >> 1;   // pairs
+    const int KT = plan.KT;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStagesPair; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 2); }
+        mbar_init(mdone, 1);
+        flag[0] = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&mapA);
+        tma_prefetch_desc(&mapB);
+    }
+    if (warp == 1) { tmem_alloc_pair(tmem_slot, 2 * kPairTile); tmem_relinquish_pair(); }
+    tc_fence_before();
+    cluster_sync();   // both CTAs' barriers initialised before any remote arrive
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    int issued = 0;   // producer: stages [0, issued) were issued
+    if (warp == 0 && lane == 0) {
+        // ---------------- TMA producer (both CTAs): this CTA's A and B halves
+        WorkIt w = work_begin(plan, c, P);
+        Item it;
+        int i = 0;
+        bool abort = false;
+        while (!abort && work_next(w, plan, P, it)) {
+            int tm, tn;
+            tile_coords(it.tile, plan, tm, tn);
+            for (int k = it.ks; k < it.ke; ++k, ++i) {
+                const int s = i % kStagesPair;
+                if (!mbar_wait(&empty[s], ((i / kStagesPair) & 1) ^ 1)) { atomicExch(&flag[0], 1); abort = true; break; }
+                if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * kPairStageBytes);
+                uint8_t* st = smem + s * kPairStageBytes;
+                const uint32_t fb = cluster_addr(&full[s], 0);
+                tma_load_2d_pair(st, &mapA, k * 64, tm * kPairTile + static_cast<int>(rank) * 128, fb);
+                tma_load_2d_pair(st + kPairHalfBytes, &mapB, k * 64, tn * kPairTile + static_cast<int>(rank) * 128,
+                                 fb);
+                issued = i + 1;
+            }
+        }
+    } else if (warp == 1 && lane == 0 && rank == 0) {
+        // ---------------- MMA issuer (rank 0)
+        const uint32_t idesc = idesc_16_f32<E>(kPairTile, kPairTile);
+        WorkIt w = work_begin(plan, c, P);
+        Item it;
+        int i = 0, j = 0;
+        bool abort = false;
+        while (!abort && work_next(w, plan, P, it)) {
+            const int acc = j & 1;
+            if (!mbar_wait_cluster(&tempty[acc], ((j >> 1) & 1) ^ 1)) { atomicExch(&flag[0], 1); break; }
+            tc_fence_after();
+            const uint32_t d = tmem + acc * kPairTile;
+            for (int k = it.ks; k < it.ke; ++k, ++i) {
+                const int s = i % kStagesPair;
+                const uint32_t par = (i / kStagesPair) & 1;
+                if (!mbar_wait(&full[s], par)) {
+                    atomicExch(&flag[0], 1);
+                    abort = true;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(smem + s * kPairStageBytes);
+                const uint32_t b0 = a0 + kPairHalfBytes;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc_mma_16_pair(d, smem_desc_k_sw128(a0 + kk * 32), smem_desc_k_sw128(b0 + kk * 32), idesc,
+                                   (k > it.ks || kk > 0) ? 1u : 0u);
+                tc_commit_pair(smem_u32(&empty[s]));
+                tc_commit_pair(cluster_addr(&empty[s], peer));
+            }
+            tc_commit_pair(smem_u32(&tfull[acc]));
+            tc_commit_pair(cluster_addr(&tfull[acc], peer));
+            ++j;
+        }
+        // every pair MMA issued here has finished before either CTA frees its
+        // tensor memory or shared memory
+        tc_commit_pair(smem_u32(mdone));
+        if (!mbar_wait(mdone, 0)) atomicExch(&flag[0], 1);
+    } else if (warp >= 2) {
+        // ---------------- epilogue (both CTAs): thread = token row of this CTA's half
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        const int epi_tid = threadIdx.x - 64;
+        const int Wsk = plan.sk * KT;
+        const int Psk = plan.psk;
+        const int u0 = c < Psk ? run_begin(c, Wsk, Psk) : 0;
+        const uint32_t tempty_rank0 = cluster_addr(tempty, 0);   // tempty[0] of rank 0; [1] is 8 bytes on
+        WorkIt w = work_begin(plan, c, P);
+        Item it;
+        int j = 0;
+        // hand accumulator `a` back to rank 0's MMA issuer: one arrive per CTA
+        auto release = [&](int a) {
+            tc_fence_before();
+            named_sync(1, 128);
+            if (epi_tid == 0) mbar_arrive_cluster(tempty_rank0 + 8u * static_cast<uint32_t>(a));
+        };
+        while (work_next(w, plan, P, it)) {
+            const int acc = j & 1;
+            const bool ok_wait = mbar_wait(&tfull[acc], (j >> 1) & 1);
+            tc_fence_after();
+            if (named_any(1, 128, !ok_wait || *reinterpret_cast<volatile int*>(&flag[0]) != 0)) {
+                if (epi_tid == 0) report_status(ep.status, LLAMA_ERR_DEVICE_TIMEOUT);
+                break;
+            }
+            ++j;
+            int tm, tn;
+            tile_coords(it.tile, plan, tm, tn);
+            const int m = tm * kPairTile + static_cast<int>(rank) * 128 + r;
+            const bool row_ok = m < rowsA;
+            const uint32_t tb = tmem + lane_base + acc * kPairTile;
+            const int nbase = tn * kPairTile;
+            float rs = 1.f, sq = 0.f;
+            if (nio.ssq_in && row_ok) {
+                float ss = 0.f;
+                ss = row_ssq(nio.ssq_in + static_cast<long long>(m) * nio.n_in, nio.n_in);
+                rs = rsqrtf(ss / static_cast<float>(KT * 64) + nio.eps);
+            }
+            if (it.ks == 0 && it.ke == KT) {
+#pragma unroll 1
+                for (int cc = 0; cc < kPairTile / 32; ++cc) {
+                    float v[32];
+                    tmem_ld_32x32b_x32(tb + cc * 32, v);
+                    tc_wait_ld();
+                    if (row_ok) epi_any<E>(ep, nio, m, nbase + cc * 32, rowsB, rs, v, sq);
+                }
+                release(acc);
+                continue;
+            }
+            // split tile: this CTA's half of it, reduced among the same halves
+            // of the tile's other pairs (last arrival finishes, in pair order)
+            const int tl = it.tile - plan.dp;
+            const int ub = tl * KT;
+            const int cf = owner(ub, Wsk, Psk), cl = owner(ub + KT - 1, Wsk, Psk);
+            const int slot = (ub + it.ks == u0) ? 0 : 1;
+            const int cnt_idx = 2 * tl + static_cast<int>(rank);
+            float* my = part + (static_cast<long long>(2 * c + static_cast<int>(rank)) * 2 + slot) * kPartFloats + r;
+#pragma unroll 1
+            for (int cc = 0; cc < kPairTile / 32; ++cc) {
+                float v[32];
+                tmem_ld_32x32b_x32(tb + cc * 32, v);
+                tc_wait_ld();
+#pragma unroll
+                for (int t = 0; t < 32; ++t) my[(cc * 32 + t) * 128] = v[t];
+            }
+            __threadfence();
+            named_sync(1, 128);
+            if (epi_tid == 0) flag[1] = atomicAdd(&counters[cnt_idx], 1);
+            named_sync(1, 128);
+            if (flag[1] != cl - cf) {
+                release(acc);
+                continue;
+            }
+            __threadfence();
+#pragma unroll 1
+            for (int cc = 0; cc < kPairTile / 32; ++cc) {
+                float own[32], v[32];
+                tmem_ld_32x32b_x32(tb + cc * 32, own);
+                tc_wait_ld();
+#pragma unroll
+                for (int t = 0; t < 32; ++t) v[t] = 0.f;
+                for (int cb = cf; cb <= cl; ++cb) {
+                    if (cb == c) {
+#pragma unroll
+                        for (int t = 0; t < 32; ++t) v[t] += own[t];
+                    } else {
+                        const int sl = run_begin(cb, Wsk, Psk) >= ub ? 0 : 1;
+                        const float* pp =
+                            part + (static_cast<long long>(2 * cb + static_cast<int>(rank)) * 2 + sl) * kPartFloats + r;
+                        float f[32];
+#pragma unroll
+                        for (int t = 0; t < 32; ++t) f[t] = pp[(cc * 32 + t) * 128];
+#pragma unroll
+                        for (int t = 0; t < 32; ++t) v[t] += f[t];
+                    }
+                }
+                if (row_ok) epi_any<E>(ep, nio, m, nbase + cc * 32, rowsB, rs, v, sq);
+            }
+            release(acc);
+            if (epi_tid == 0) counters[cnt_idx] = 0;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0 && lane == 0 && *reinterpret_cast<volatile int*>(&flag[0]) != 0) {
+        // the CTA gave up: its copies still in flight land before it exits
+        if (rank == 0) {
+            // the newest stage of each ring slot (a stage the peer never
+            // issued does not complete: that wait gives up after kDrainNs)
+            for (int s = 0; s < kStagesPair; ++s) {
+                if (issued <= s) continue;
+                const int jn = s + ((issued - 1 - s) / kStagesPair) * kStagesPair;
+                mbar_wait(&full[s], (jn / kStagesPair) & 1, kDrainNs);
+            }
+        } else {
+            const uint64_t t0 = globaltimer_ns();
+            while (globaltimer_ns() - t0 < kDrainNs) {
+            }
+        }
+    }
+    // neither CTA leaves while the other may still signal its barriers or
+    // (rank 0's MMAs, waited for above) read its shared memory
+    cluster_sync();
+    if (warp == 1) tmem_dealloc_pair(tmem, 2 * kPairTile);
+    if (threadIdx.x == 0) tl_stamp(ep.tl);
+}
+
 // ---------------------------------------------------------------- host side
 
 static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -446,6 +704,53 @@ static int launch_tcp(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, in
     return LLAMA_OK;
 }
 
+// When a projection runs on CTA pairs: at least 256 token rows (fewer would
+// leave most of a 256-row pair tile empty) and a weight matrix larger than
+// 4096 x 4096.  Measured on the 7B prefill (4 x 512 tokens, interleaved runs,
+// medians): pairs take w1/w3 (22016 x 4096) from 9.8 to 9.3 ms and w2
+// (4096 x 11008) from 6.1 to 5.7 ms per prefill, wq/wk/wv (12288 x 4096) is
+// even, and wo (4096 x 4096) goes from 3.4 to 3.9 ms, so it keeps one SM per
+// tile.
+constexpr int kPairMinRows = 256;
+constexpr long long kPairMinWeights = 4096LL * 4096;
+
+template <typename E>
+static int launch_tcp_pair(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
+                           int* counters, cudaStream_t st, const NormIO& nio) {
+    constexpr int smem = 1024 + kStagesPair * kPairStageBytes + (2 * kStagesPair + 5) * 8 + 16;
+    static_assert(smem <= 227 * 1024, "shared memory per CTA");
+    auto kern = linear_tcp_pair_kernel<E>;
+    static int pairs = 0;   // clusters of two that are resident at once
+    if (pairs == 0) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(linear_tcp_pair_kernel)");
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(kMaxPrefillCtas);
+        cfg.blockDim = dim3(kThreadsTc);
+        cfg.dynamicSmemBytes = smem;
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters(linear_tcp_pair_kernel)");
+        if (n < 1) { set_error("linear_tcp_pair_kernel: no CTA pair fits on this GPU"); return LLAMA_ERR_CUDA; }
+        pairs = n < kMaxPrefillCtas / 2 ? n : kMaxPrefillCtas / 2;
+    }
+    TcPlan plan;
+    plan.TM = (M + kPairTile - 1) / kPairTile;
+    plan.TN = (N + kPairTile - 1) / kPairTile;
+    plan.KT = (K + 63) / 64;
+    const long long T = static_cast<long long>(plan.TM) * plan.TN;
+    if (T >= (1LL << 30)) { set_error("prefill projection too large (%lld tiles)", T); return LLAMA_ERR_INVALID_ARG; }
+    int grid = 0;
+    plan_tc(static_cast<int>(T), plan.KT, pairs, part != nullptr && counters != nullptr, &plan, &grid);
+    if (2 * plan.sk > kMaxTiles) {
+        set_error("internal: %d split tile halves exceed the counters", 2 * plan.sk);
+        return LLAMA_ERR_INVALID_ARG;
+    }
+    kern<<<2 * grid, kThreadsTc, smem, st>>>(mapA->a128, mapW->a128, M, N, plan, ep, part, counters, nio);
+    LLB_CHECK_LAUNCH("linear_tcp_pair_kernel");
+    return LLAMA_OK;
+}
+
 int linear16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, int dtype, const Epi& ep, float* part,
                 int* counters, cudaStream_t st, const NormIO* nio_in) {
     NormIO nio = {};
@@ -455,6 +760,11 @@ int linear16_tc(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, i
         return LLAMA_ERR_INVALID_ARG;
     }
     if (nio.ssq_in && K % 64) { set_error("fused RMSNorm consumer needs K %% 64 == 0"); return LLAMA_ERR_INVALID_ARG; }
+    if (M <= 0 || N <= 0) return LLAMA_OK;
+    if (M >= kPairMinRows && static_cast<long long>(N) * K > kPairMinWeights) {
+        if (dtype == LLAMA_F16) return launch_tcp_pair<f16>(mapA, mapW, M, N, K, ep, part, counters, st, nio);
+        if (dtype == LLAMA_BF16) return launch_tcp_pair<bf16>(mapA, mapW, M, N, K, ep, part, counters, st, nio);
+    }
     if (dtype == LLAMA_F16) return launch_tcp<f16>(mapA, mapW, M, N, K, ep, part, counters, st, nio);
     if (dtype == LLAMA_BF16) return launch_tcp<bf16>(mapA, mapW, M, N, K, ep, part, counters, st, nio);
     set_error("16-bit projection: dtype must be LLAMA_BF16 or LLAMA_F16");

@@ -62,12 +62,14 @@ def test_linear_f32_kernel(llb, M, N, K):
 @pytest.mark.parametrize("M,N,K", [
     (1, 256, 256), (7, 1000, 4096), (16, 4096, 256), (17, 384, 4160), (33, 512, 200), (64, 12288, 4096),
     (48, 640, 512),
-    (65, 256, 256), (128, 1000, 4096), (300, 768, 1024), (2048, 512, 64)])
+    (65, 256, 256), (128, 1000, 4096), (300, 768, 1024), (2048, 512, 64),
+    (300, 4224, 4096)])
 @pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
 def test_linear_16bit_tcgen05_kernel(llb, M, N, K, dt):
     """tcgen05 GEMM in both orientations (M <= 64: weights as the 128-row
-    operand; else activations), with ragged M, N and K tails, for both
-    16-bit operand types."""
+    operand; else activations, on one SM per tile or, for at least 256 rows
+    and more than 4096 x 4096 weights, on CTA pairs), with ragged M, N and K
+    tails, for both 16-bit operand types."""
     g = torch.Generator().manual_seed(7 * M + N + K)
     A = torch.randn(M, K, generator=g).to(dt)
     W = (torch.randn(N, K, generator=g) * 0.05).to(dt)
@@ -88,6 +90,11 @@ def test_linear_16bit_tcgen05_kernel(llb, M, N, K, dt):
     (2048, 4864, 512),     # 304 tiles: one wave of whole tiles, then a stream-K run
     (256, 35584, 256),     # 278 tiles: last wave 88 % full, whole tiles only
     (1000, 1000, 4160),    # ragged M, N and K, 32 tiles split up to 4 ways
+    # CTA pairs (256 x 256 tiles, 74 pairs on a 148-SM B200)
+    (512, 18944, 1024),    # 148 pair tiles: two full waves, whole tiles only
+    (2048, 5120, 4096),    # 160 pair tiles: two waves, then 12 tiles stream-K over 48 runs
+    (1000, 4160, 4160),    # ragged M, N and K, 68 pair tiles all split (the last half-tile partly past M)
+    (384, 16384, 1088),    # the second pair tile's upper half lies wholly past M
 ])
 def test_linear_bf16_prefill_work_split(llb, M, N, K):
     """The persistent prefill projection under each of its work splits, with
