@@ -9,7 +9,10 @@
 // two tokens that matter (the last kept one and the drawn one) without a
 // sort, by a most-significant-digit radix select over a 64-bit order key
 //     key = ordered_bits(logit) << 32 | ~id      (descending key = sampling order)
-// using histograms of probability mass.  Masses are e_i = exp((l_i - l_max)/T)
+// using histograms of probability mass: the first-digit histogram of the whole
+// row (which also gives the total mass) serves both selects, and once a chosen
+// digit prefix holds at most kListCap keys they are copied into shared memory
+// and the remaining passes read only them.  Masses are e_i = exp((l_i - l_max)/T)
 // evaluated in fp64 and held as 64-bit fixed point (2^-46 resolution), so
 // every prefix sum is an exact integer and the result does not depend on the
 // summation order.
@@ -78,15 +81,24 @@ argmax_kernel(const float* __restrict__ logits, int V, int32_t* out, int32_t* to
 }
 
 // ---------------------------------------------------------------- top-p
+// Candidates of the radix select kept in shared memory once the chosen digit
+// prefix holds few enough keys: later passes read them instead of the row.
+constexpr int kListCap = 4096;
+
 struct TopPShared {
     unsigned long long hist_mass[kWarps][256];
     unsigned int hist_cnt[kWarps][256];
     unsigned long long tot_mass[256];
     unsigned int tot_cnt[256];
+    unsigned long long p1_mass[256];     // first-digit histogram of the whole row (both selects start from it)
+    unsigned int p1_cnt[256];
+    unsigned long long list_key[kListCap];
+    unsigned long long list_mass[kListCap];
     unsigned long long red_u64[kWarps];
     float red_f[kWarps];
     unsigned long long sel_prefix, sel_before;
-    unsigned long long result_key[2], result_before[2];
+    unsigned int sel_cnt;
+    int list_n;
     float lmax;
 };
 
@@ -95,96 +107,178 @@ __device__ __forceinline__ unsigned long long fixed_mass(float l, double lmax, d
     return static_cast<unsigned long long>(e * kFixScale + 0.5);
 }
 
-// First key in descending order whose inclusive prefix mass exceeds `target`
-// (or the smallest key if none does).  Returns the key; *before_out = mass of
-// all keys strictly before it.
-__device__ uint64_t radix_select(TopPShared& sh, const float* row, int V, double lmax, double inv_t,
-                                 unsigned long long target, unsigned long long* before_out) {
+// Per-warp histograms of digit (key >> shift) & 255 over the keys that match
+// `prefix` under `mask`, from the row (masses computed here) or from the
+// candidate list; then the per-digit totals in sh.tot_*.  A thread's
+// consecutive keys mostly share a digit: they are summed in registers, one
+// pair of shared-memory atomics per change of digit.
+__device__ void digit_histogram(TopPShared& sh, const float* row, int V, bool from_list, double lmax, double inv_t,
+                                uint64_t prefix, uint64_t mask, int shift) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint64_t prefix = 0, mask = 0;
-    unsigned long long before = 0;
-    for (int pass = 0; pass < 8; ++pass) {
-        const int shift = 56 - 8 * pass;
-        for (int i = lane; i < 256; i += 32) {
-            sh.hist_mass[warp][i] = 0ull;
-            sh.hist_cnt[warp][i] = 0u;
+    for (int i = lane; i < 256; i += 32) {
+        sh.hist_mass[warp][i] = 0ull;
+        sh.hist_cnt[warp][i] = 0u;
+    }
+    __syncthreads();
+    int cur = -1;
+    unsigned long long cur_mass = 0;
+    unsigned int cur_cnt = 0;
+    auto add = [&](uint64_t key, unsigned long long m) {
+        const int bin = static_cast<int>((key >> shift) & 255u);
+        if (bin != cur) {
+            if (cur >= 0) {
+                atomicAdd(&sh.hist_mass[warp][cur], cur_mass);
+                atomicAdd(&sh.hist_cnt[warp][cur], cur_cnt);
+            }
+            cur = bin;
+            cur_mass = 0;
+            cur_cnt = 0;
         }
-        __syncthreads();
+        cur_mass += m;
+        ++cur_cnt;
+    };
+    if (from_list) {
+        for (int j = threadIdx.x; j < sh.list_n; j += blockDim.x) {
+            const uint64_t key = sh.list_key[j];
+            if ((key & mask) == prefix) add(key, sh.list_mass[j]);
+        }
+    } else {
         for (int i = threadIdx.x; i < V; i += blockDim.x) {
             const float l = row[i];
             const uint64_t key = sort_key(l, i);
-            if ((key & mask) == prefix) {
-                const int bin = static_cast<int>((key >> shift) & 255u);
-                atomicAdd(&sh.hist_mass[warp][bin], fixed_mass(l, lmax, inv_t));
-                atomicAdd(&sh.hist_cnt[warp][bin], 1u);
-            }
+            if ((key & mask) == prefix) add(key, fixed_mass(l, lmax, inv_t));
         }
-        __syncthreads();
-        if (threadIdx.x < 256) {
-            unsigned long long m = 0;
-            unsigned int c = 0;
-            for (int w = 0; w < kWarps; ++w) {
-                m += sh.hist_mass[w][threadIdx.x];
-                c += sh.hist_cnt[w][threadIdx.x];
-            }
-            sh.tot_mass[threadIdx.x] = m;
-            sh.tot_cnt[threadIdx.x] = c;
+    }
+    if (cur >= 0) {
+        atomicAdd(&sh.hist_mass[warp][cur], cur_mass);
+        atomicAdd(&sh.hist_cnt[warp][cur], cur_cnt);
+    }
+    __syncthreads();
+    if (threadIdx.x < 256) {
+        unsigned long long m = 0;
+        unsigned int c = 0;
+        for (int w = 0; w < kWarps; ++w) {
+            m += sh.hist_mass[w][threadIdx.x];
+            c += sh.hist_cnt[w][threadIdx.x];
         }
-        __syncthreads();
-        if (warp == 0) {
-            // lane L scans bins 255-8L .. 248-8L (descending)
-            unsigned long long part = 0;
-            for (int k = 0; k < 8; ++k) part += sh.tot_mass[255 - 8 * lane - k];
-            // exclusive scan from lane 0 (highest bins) upwards
-            unsigned long long incl = part;
+        sh.tot_mass[threadIdx.x] = m;
+        sh.tot_cnt[threadIdx.x] = c;
+    }
+    __syncthreads();
+}
+
+// Warp 0: in descending digit order over the totals `tm` / `tc` (256 bins),
+// the first digit whose inclusive prefix mass, after `before`, exceeds
+// `target` (or the last non-empty digit if none does).  Writes the extended
+// prefix, the mass before the chosen digit and its key count to sh.sel_*.
+__device__ void choose_digit(TopPShared& sh, const unsigned long long* tm, const unsigned int* tc, uint64_t prefix,
+                             int shift, unsigned long long before, unsigned long long target) {
+    const int lane = threadIdx.x & 31;
+    unsigned long long part = 0;
+    for (int k = 0; k < 8; ++k) part += tm[255 - 8 * lane - k];   // lane L: digits 255-8L .. 248-8L
+    unsigned long long incl = part;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const unsigned long long t = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += t;
-            }
-            const unsigned long long excl = incl - part;
-            const bool cross = before + incl > target;
-            const unsigned int ballot = __ballot_sync(0xffffffffu, cross);
-            int chosen = -1;
-            unsigned long long chosen_before = 0;
-            if (ballot) {
-                const int L = __ffs(ballot) - 1;
-                if (lane == L) {
-                    unsigned long long cum = before + excl;
-                    for (int k = 0; k < 8; ++k) {
-                        const int bin = 255 - 8 * lane - k;
-                        if (sh.tot_cnt[bin] == 0) continue;
-                        if (cum + sh.tot_mass[bin] > target) { chosen = bin; chosen_before = cum; break; }
-                        cum += sh.tot_mass[bin];
-                    }
-                }
-                chosen = __shfl_sync(0xffffffffu, chosen, L);
-                chosen_before = __shfl_sync(0xffffffffu, chosen_before, L);
-            }
-            if (chosen < 0) {
-                // no bin crosses: take the lowest non-empty bin (the last key in order)
-                if (lane == 0) {
-                    unsigned long long cum = before;
-                    for (int bin = 255; bin >= 0; --bin) {
-                        if (sh.tot_cnt[bin] == 0) continue;
-                        chosen = bin;
-                        chosen_before = cum;
-                        cum += sh.tot_mass[bin];
-                    }
-                }
-                chosen = __shfl_sync(0xffffffffu, chosen, 0);
-                chosen_before = __shfl_sync(0xffffffffu, chosen_before, 0);
-            }
-            if (lane == 0) {
-                sh.sel_prefix = prefix | (static_cast<uint64_t>(chosen) << shift);
-                sh.sel_before = chosen_before;
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    const unsigned long long excl = incl - part;
+    const bool cross = before + incl > target;
+    const unsigned int ballot = __ballot_sync(0xffffffffu, cross);
+    int chosen = -1;
+    unsigned long long chosen_before = 0;
+    if (ballot) {
+        const int L = __ffs(ballot) - 1;
+        if (lane == L) {
+            unsigned long long cum = before + excl;
+            for (int k = 0; k < 8; ++k) {
+                const int bin = 255 - 8 * lane - k;
+                if (tc[bin] == 0) continue;
+                if (cum + tm[bin] > target) { chosen = bin; chosen_before = cum; break; }
+                cum += tm[bin];
             }
         }
+        chosen = __shfl_sync(0xffffffffu, chosen, L);
+        chosen_before = __shfl_sync(0xffffffffu, chosen_before, L);
+    }
+    if (chosen < 0) {
+        // no digit crosses: the lowest non-empty digit (the last key in order)
+        if (lane == 0) {
+            unsigned long long cum = before;
+            for (int bin = 255; bin >= 0; --bin) {
+                if (tc[bin] == 0) continue;
+                chosen = bin;
+                chosen_before = cum;
+                cum += tm[bin];
+            }
+        }
+        chosen = __shfl_sync(0xffffffffu, chosen, 0);
+        chosen_before = __shfl_sync(0xffffffffu, chosen_before, 0);
+    }
+    if (lane == 0) {
+        sh.sel_prefix = prefix | (static_cast<uint64_t>(chosen) << shift);
+        sh.sel_before = chosen_before;
+        sh.sel_cnt = tc[chosen];
+    }
+}
+
+// The candidates matching `prefix` under `mask` copied from the row into the
+// shared list (the caller knows there are at most kListCap of them).
+__device__ void compact(TopPShared& sh, const float* row, int V, double lmax, double inv_t, uint64_t prefix,
+                        uint64_t mask) {
+    if (threadIdx.x == 0) sh.list_n = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < V; i += blockDim.x) {
+        const float l = row[i];
+        const uint64_t key = sort_key(l, i);
+        if ((key & mask) == prefix) {
+            const int j = atomicAdd(&sh.list_n, 1);
+            sh.list_key[j] = key;
+            sh.list_mass[j] = fixed_mass(l, lmax, inv_t);
+        }
+    }
+    __syncthreads();
+}
+
+// First key in descending order whose inclusive prefix mass exceeds `target`
+// (or the smallest key if none does), starting from the first-digit histogram
+// of the whole row (sh.p1_*).  `*list_prefix` names the first-digit prefix
+// the shared list holds (or ~0 for none); the list is rebuilt when this select
+// chooses another first digit with at most kListCap keys.  Returns the key;
+// *before_out = the mass of all keys strictly before it.
+__device__ uint64_t radix_select(TopPShared& sh, const float* row, int V, double lmax, double inv_t,
+                                 unsigned long long target, uint64_t* list_prefix, unsigned long long* before_out) {
+    const int warp = threadIdx.x >> 5;
+    if (warp == 0) choose_digit(sh, sh.p1_mass, sh.p1_cnt, 0, 56, 0, target);
+    __syncthreads();
+    uint64_t prefix = sh.sel_prefix, mask = static_cast<uint64_t>(255) << 56;
+    unsigned long long before = sh.sel_before;
+    bool use_list = false;
+    if (prefix == *list_prefix) {
+        use_list = true;
+    } else if (sh.sel_cnt <= static_cast<unsigned int>(kListCap)) {
+        compact(sh, row, V, lmax, inv_t, prefix, mask);
+        *list_prefix = prefix;
+        use_list = true;
+    }
+    __syncthreads();
+    for (int pass = 1; pass < 8; ++pass) {
+        const int shift = 56 - 8 * pass;
+        digit_histogram(sh, row, V, use_list, lmax, inv_t, prefix, mask, shift);
+        if (warp == 0) choose_digit(sh, sh.tot_mass, sh.tot_cnt, prefix, shift, before, target);
         __syncthreads();
         prefix = sh.sel_prefix;
         before = sh.sel_before;
         mask |= static_cast<uint64_t>(255) << shift;
+        const bool fits = sh.sel_cnt <= static_cast<unsigned int>(kListCap);
         __syncthreads();
+        if (!use_list && fits && pass < 7) {
+            // few enough keys under the longer prefix: the remaining passes
+            // read them from the list (which then serves no other prefix)
+            compact(sh, row, V, lmax, inv_t, prefix, mask);
+            *list_prefix = ~0ull;
+            use_list = true;
+        }
     }
     *before_out = before;
     return prefix;
@@ -217,21 +311,23 @@ top_p_kernel(const float* __restrict__ logits, int V, float temperature, float t
     const double lmax = static_cast<double>(sh.lmax);
     const double inv_t = 1.0 / static_cast<double>(temperature);
 
-    // total mass
-    unsigned long long tot = 0;
-    for (int i = threadIdx.x; i < V; i += blockDim.x) tot += fixed_mass(row[i], lmax, inv_t);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-    if (lane == 0) sh.red_u64[warp] = tot;
-    __syncthreads();
+    // first-digit histogram of the whole row; its digits add up to the row's
+    // total mass S (exact integers, so in any order)
+    digit_histogram(sh, row, V, false, lmax, inv_t, 0, 0, 56);
     unsigned long long S = 0;
-    for (int w = 0; w < kWarps; ++w) S += sh.red_u64[w];
+    for (int i = 0; i < 256; ++i) S += sh.tot_mass[i];
+    if (threadIdx.x < 256) {
+        sh.p1_mass[threadIdx.x] = sh.tot_mass[threadIdx.x];
+        sh.p1_cnt[threadIdx.x] = sh.tot_cnt[threadIdx.x];
+    }
+    __syncthreads();
 
     // nucleus edge: first key whose inclusive mass exceeds top_p * S
+    uint64_t list_prefix = ~0ull;
     const double tp = static_cast<double>(top_p) * static_cast<double>(S);
     const unsigned long long t1 = tp >= 18446744073709549568.0 ? ~0ull : static_cast<unsigned long long>(tp);
     unsigned long long before_edge;
-    const uint64_t edge = radix_select(sh, row, V, lmax, inv_t, t1, &before_edge);
+    const uint64_t edge = radix_select(sh, row, V, lmax, inv_t, t1, &list_prefix, &before_edge);
     const int edge_id = static_cast<int>(~static_cast<uint32_t>(edge & 0xffffffffu));
     const unsigned long long Z = before_edge + fixed_mass(row[edge_id], lmax, inv_t);
 
@@ -240,7 +336,7 @@ top_p_kernel(const float* __restrict__ logits, int V, float temperature, float t
     u = fmin(fmax(u, 0.0), 1.0);
     const unsigned long long t2 = static_cast<unsigned long long>(u * static_cast<double>(Z));
     unsigned long long before_draw;
-    const uint64_t drawn = radix_select(sh, row, V, lmax, inv_t, t2, &before_draw);
+    const uint64_t drawn = radix_select(sh, row, V, lmax, inv_t, t2, &list_prefix, &before_draw);
     const uint64_t pick = drawn < edge ? edge : drawn;   // never past the nucleus edge
     if (threadIdx.x == 0) {
         const int id = static_cast<int>(~static_cast<uint32_t>(pick & 0xffffffffu));
