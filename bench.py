@@ -340,6 +340,16 @@ def run_ours(a, rank, world, local_rank):
     tl_step_ns, tl_kind_ns, tl_kind_bytes = timeline_breakdown(tl_recs, n_step)
     assert model.status() == 0
 
+    # ---------------- SM clocks while prefills run back to back (outside the timed region): the
+    # tensor-core-bound prefill runs under the 1 kW power cap, unlike the HBM-bound decode
+    pre_clocks = ClockSampler(local_rank, os.path.join(tempfile.gettempdir(), f"llama_b200_clocks_pre_rank{rank}.csv"))
+    pre_clocks.start()
+    t_pc = time.time()
+    while time.time() - t_pc < 0.8:
+        start_request()
+        torch.cuda.synchronize()
+    pre_clk = pre_clocks.stop()
+
     # ---------------- serialised per-launch timing (outside the timed region): events around every
     # projection of one prefill and of 16 decode steps launched directly (programmatic dependent
     # launch off while timed, so each launch runs alone)
@@ -459,9 +469,13 @@ def run_ours(a, rank, world, local_rank):
                                         "dependent launch): ramp and tail of every launch included"},
         "decode_step_breakdown_us": {k: round(v / 1e3, 2) for k, v in sorted(tl_kind_ns.items())},
         "decode_step_timeline_us": round(tl_step_ns / 1e3, 2),
-        "roofline_prefill": {"bound": "tensor", "kernel": "linear_tcp_kernel (prefill projections: wq/wk/wv, wo, w1/w3, w2; persistent, 128x256 tiles)",
+        "roofline_prefill": {"bound": "tensor", "kernel": "linear_tcp_pair_kernel / linear_tcp_kernel (prefill projections: wq/wk/wv, w1/w3, w2 on CTA pairs with 256x256 tiles, wo on single SMs with 128x256 tiles; persistent)",
                              "achieved": round(pre_tfs, 1), "peak": tc_burst, "unit": "TFLOP/s",
                              "frac": round(pre_tfs / tc_burst, 4), "peak_source": f"{peak_src} bf16_tflops (burst)",
+                             "sustained_peak": tc_sust, "frac_sustained": round(pre_tfs / tc_sust, 4),
+                             "clocks": pre_clk,
+                             "clocks_what": "SM clocks sampled while prefills run back to back: the power cap holds "
+                                            "them below the maximum, which is what the sustained peak describes",
                              "traffic": _traffic("linear_tcp_kernel"), "launches": len(pre),
                              "what": "2*M*N*K of one prefill's projection launches / their event-timed durations "
                                      "(prefill launches run one after another in the product path too)",

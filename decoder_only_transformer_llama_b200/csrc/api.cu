@@ -214,7 +214,7 @@ int run_linear(const Model* m, int dtype, const void* A, const TmaMaps* mapA, co
                const NormIO* nio, bool stamp) {
     Epi ep = ep_in;
     if (stamp) ep.tl = tl_next(const_cast<Model*>(m), TL_PROJECTION, proj_bytes(M, N, K, ep));
-    if (dtype != LLAMA_F32 && M <= 64) {
+    if (dtype != LLAMA_F32) {
         int unit = 0;
         long long wait_ns = 0;
         if (take_stall(const_cast<Model*>(m), LLAMA_STALL_PROJECTION, &unit, &wait_ns)) {

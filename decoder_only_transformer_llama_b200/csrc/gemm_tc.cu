@@ -203,16 +203,19 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
     uint64_t* empty = full + kStagesTc;
     uint64_t* tfull = empty + kStagesTc;   // [2]
     uint64_t* tempty = tfull + 2;          // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+    uint64_t* mdone = tempty + 2;          // the MMA issuer's last commit
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + 1);
     int* flag = reinterpret_cast<int*>(tmem_slot + 1);   // [0] abort, [1] arrival broadcast
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = gridDim.x, c = blockIdx.x;
     const int KT = plan.KT;
+    const uint64_t wlim = ep.wait_ns > 0 ? static_cast<uint64_t>(ep.wait_ns) : kWaitLimitNs;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStagesTc; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 128); }
+        mbar_init(mdone, 1);
         flag[0] = 0;
         fence_mbar_init();
         tma_prefetch_desc(&mapA);
@@ -224,8 +227,10 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    int issued = 0, stall = -1;   // producer: stages [0, issued) were issued, all but `stall`
     if (warp == 0 && lane == 0) {
         // ---------------- TMA producer
+        stall = c == 0 ? ep.stall - 1 : -1;   // tests of the timeout path only
         WorkIt w = work_begin(plan, c, P);
         Item it;
         int i = 0;
@@ -235,11 +240,14 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
             tile_coords(it.tile, plan, tm, tn);
             for (int k = it.ks; k < it.ke; ++k, ++i) {
                 const int s = i % kStagesTc;
-                if (!mbar_wait(&empty[s], ((i / kStagesTc) & 1) ^ 1)) { atomicExch(&flag[0], 1); abort = true; break; }
-                mbar_arrive_expect_tx(&full[s], kStageBytes);
-                uint8_t* st = smem + s * kStageBytes;
-                tma_load_2d(st, &mapA, k * 64, tm * 128, &full[s]);
-                tma_load_2d(st + kA_BYTES, &mapB, k * 64, tn * kBN, &full[s]);
+                if (!mbar_wait(&empty[s], ((i / kStagesTc) & 1) ^ 1, wlim)) { atomicExch(&flag[0], 1); abort = true; break; }
+                if (i != stall) {
+                    mbar_arrive_expect_tx(&full[s], kStageBytes);
+                    uint8_t* st = smem + s * kStageBytes;
+                    tma_load_2d(st, &mapA, k * 64, tm * 128, &full[s]);
+                    tma_load_2d(st + kA_BYTES, &mapB, k * 64, tn * kBN, &full[s]);
+                }
+                issued = i + 1;
             }
         }
     } else if (warp == 1 && lane == 0) {
@@ -251,12 +259,12 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
         bool abort = false;
         while (!abort && work_next(w, plan, P, it)) {
             const int acc = j & 1;
-            if (!mbar_wait(&tempty[acc], ((j >> 1) & 1) ^ 1)) { atomicExch(&flag[0], 1); break; }
+            if (!mbar_wait(&tempty[acc], ((j >> 1) & 1) ^ 1, wlim)) { atomicExch(&flag[0], 1); break; }
             tc_fence_after();
             const uint32_t d = tmem + acc * kBN;
             for (int k = it.ks; k < it.ke; ++k, ++i) {
                 const int s = i % kStagesTc;
-                if (!mbar_wait(&full[s], (i / kStagesTc) & 1)) { atomicExch(&flag[0], 1); abort = true; break; }
+                if (!mbar_wait(&full[s], (i / kStagesTc) & 1, wlim)) { atomicExch(&flag[0], 1); abort = true; break; }
                 tc_fence_after();
                 const uint32_t a0 = smem_u32(smem + s * kStageBytes);
                 const uint32_t b0 = a0 + kA_BYTES;
@@ -269,6 +277,9 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
             tc_commit(&tfull[acc]);
             ++j;
         }
+        // every MMA issued here has finished before TMEM is freed
+        tc_commit(mdone);
+        if (!mbar_wait(mdone, 0, wlim)) atomicExch(&flag[0], 1);
     } else if (warp >= 2) {
         // ---------------- epilogue: thread = token row of the tile, TMEM columns = features
         const int q = warp & 3;
@@ -283,7 +294,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
         int j = 0;
         while (work_next(w, plan, P, it)) {
             const int acc = j & 1;
-            const bool ok_wait = mbar_wait(&tfull[acc], (j >> 1) & 1);
+            const bool ok_wait = mbar_wait(&tfull[acc], (j >> 1) & 1, wlim);
             tc_fence_after();
             if (named_any(1, 128, !ok_wait || *reinterpret_cast<volatile int*>(&flag[0]) != 0)) {
                 if (epi_tid == 0) report_status(ep.status, LLAMA_ERR_DEVICE_TIMEOUT);
@@ -372,6 +383,16 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
 
     tc_fence_before();
     __syncthreads();
+    if (warp == 0 && lane == 0 && *reinterpret_cast<volatile int*>(&flag[0]) != 0) {
+        // the CTA gave up: the copies it still has in flight land before it
+        // exits (the newest stage of each ring slot; a skipped one is not waited for)
+        for (int s = 0; s < kStagesTc; ++s) {
+            if (issued <= s) continue;
+            int jn = s + ((issued - 1 - s) / kStagesTc) * kStagesTc;
+            if (jn == stall) jn -= kStagesTc;
+            if (jn >= 0) mbar_wait(&full[s], (jn / kStagesTc) & 1, wlim);
+        }
+    }
     if (warp == 1) tmem_dealloc(tmem, 2 * kBN);
     if (threadIdx.x == 0) tl_stamp(ep.tl);
 }
@@ -425,6 +446,7 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
     const uint32_t peer = rank ^ 1u;
     const int P = gridDim.x >> 1, c = blockIdx.x >> 1;   // pairs
     const int KT = plan.KT;
+    const uint64_t wlim = ep.wait_ns > 0 ? static_cast<uint64_t>(ep.wait_ns) : kWaitLimitNs;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStagesPair; ++s) {
@@ -444,9 +466,10 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    int issued = 0;   // producer: stages [0, issued) were issued
+    int issued = 0, stall = -1;   // producer: stages [0, issued) were issued, all but `stall`
     if (warp == 0 && lane == 0) {
         // ---------------- TMA producer (both CTAs): this CTA's A and B halves
+        stall = blockIdx.x == 0 ? ep.stall - 1 : -1;   // tests of the timeout path only (rank 0 of pair 0)
         WorkIt w = work_begin(plan, c, P);
         Item it;
         int i = 0;
@@ -456,13 +479,15 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
             tile_coords(it.tile, plan, tm, tn);
             for (int k = it.ks; k < it.ke; ++k, ++i) {
                 const int s = i % kStagesPair;
-                if (!mbar_wait(&empty[s], ((i / kStagesPair) & 1) ^ 1)) { atomicExch(&flag[0], 1); abort = true; break; }
-                if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * kPairStageBytes);
-                uint8_t* st = smem + s * kPairStageBytes;
-                const uint32_t fb = cluster_addr(&full[s], 0);
-                tma_load_2d_pair(st, &mapA, k * 64, tm * kPairTile + static_cast<int>(rank) * 128, fb);
-                tma_load_2d_pair(st + kPairHalfBytes, &mapB, k * 64, tn * kPairTile + static_cast<int>(rank) * 128,
-                                 fb);
+                if (!mbar_wait(&empty[s], ((i / kStagesPair) & 1) ^ 1, wlim)) { atomicExch(&flag[0], 1); abort = true; break; }
+                if (i != stall) {
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * kPairStageBytes);
+                    uint8_t* st = smem + s * kPairStageBytes;
+                    const uint32_t fb = cluster_addr(&full[s], 0);
+                    tma_load_2d_pair(st, &mapA, k * 64, tm * kPairTile + static_cast<int>(rank) * 128, fb);
+                    tma_load_2d_pair(st + kPairHalfBytes, &mapB, k * 64,
+                                     tn * kPairTile + static_cast<int>(rank) * 128, fb);
+                }
                 issued = i + 1;
             }
         }
@@ -475,13 +500,13 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
         bool abort = false;
         while (!abort && work_next(w, plan, P, it)) {
             const int acc = j & 1;
-            if (!mbar_wait_cluster(&tempty[acc], ((j >> 1) & 1) ^ 1)) { atomicExch(&flag[0], 1); break; }
+            if (!mbar_wait_cluster(&tempty[acc], ((j >> 1) & 1) ^ 1, wlim)) { atomicExch(&flag[0], 1); break; }
             tc_fence_after();
             const uint32_t d = tmem + acc * kPairTile;
             for (int k = it.ks; k < it.ke; ++k, ++i) {
                 const int s = i % kStagesPair;
                 const uint32_t par = (i / kStagesPair) & 1;
-                if (!mbar_wait(&full[s], par)) {
+                if (!mbar_wait(&full[s], par, wlim)) {
                     atomicExch(&flag[0], 1);
                     abort = true;
                     break;
@@ -503,7 +528,7 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
         // every pair MMA issued here has finished before either CTA frees its
         // tensor memory or shared memory
         tc_commit_pair(smem_u32(mdone));
-        if (!mbar_wait(mdone, 0)) atomicExch(&flag[0], 1);
+        if (!mbar_wait(mdone, 0, wlim)) atomicExch(&flag[0], 1);
     } else if (warp >= 2) {
         // ---------------- epilogue (both CTAs): thread = token row of this CTA's half
         const int q = warp & 3;
@@ -525,7 +550,7 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
         };
         while (work_next(w, plan, P, it)) {
             const int acc = j & 1;
-            const bool ok_wait = mbar_wait(&tfull[acc], (j >> 1) & 1);
+            const bool ok_wait = mbar_wait(&tfull[acc], (j >> 1) & 1, wlim);
             tc_fence_after();
             if (named_any(1, 128, !ok_wait || *reinterpret_cast<volatile int*>(&flag[0]) != 0)) {
                 if (epi_tid == 0) report_status(ep.status, LLAMA_ERR_DEVICE_TIMEOUT);
@@ -618,8 +643,9 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
             // issued does not complete: that wait gives up after kDrainNs)
             for (int s = 0; s < kStagesPair; ++s) {
                 if (issued <= s) continue;
-                const int jn = s + ((issued - 1 - s) / kStagesPair) * kStagesPair;
-                mbar_wait(&full[s], (jn / kStagesPair) & 1, kDrainNs);
+                int jn = s + ((issued - 1 - s) / kStagesPair) * kStagesPair;
+                if (jn == stall) jn -= kStagesPair;
+                if (jn >= 0) mbar_wait(&full[s], (jn / kStagesPair) & 1, kDrainNs);
             }
         } else {
             const uint64_t t0 = globaltimer_ns();
@@ -675,7 +701,7 @@ template <typename E>
 static int launch_tcp(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
                       int* counters, cudaStream_t st, const NormIO& nio) {
     if (M <= 0 || N <= 0) return LLAMA_OK;
-    constexpr int smem = 1024 + kStagesTc * kStageBytes + (2 * kStagesTc + 4) * 8 + 16;
+    constexpr int smem = 1024 + kStagesTc * kStageBytes + (2 * kStagesTc + 5) * 8 + 16;
     static_assert(smem <= 227 * 1024, "shared memory per CTA");
     static bool attr_set = false;
     if (!attr_set) {

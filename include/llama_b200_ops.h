@@ -118,10 +118,11 @@ LLAMA_API int llama_timeline_stop(llama_model* m, uint64_t* end_ns, int32_t* kin
  * operations in flight finish, releases its tensor memory, records
  * LLAMA_ERR_DEVICE_TIMEOUT in the model's device status word and returns.
  * llama_debug_stall arms that path once: in the next launch of the chosen
- * decode kernel by this model (16-bit models; the weight-streaming
- * projection, or the decode attention), CTA 0 never issues the copies of
- * pipeline stage `unit` of its run nor the barrier signal that would announce
- * them, and every wait of that launch gives up after wait_limit_ns
+ * kernel by this model (16-bit models; LLAMA_STALL_PROJECTION: the next
+ * projection, decode-shaped or prefill-shaped, on single SMs or CTA pairs;
+ * LLAMA_STALL_ATTENTION: the next decode attention), CTA 0 never issues the
+ * copies of pipeline stage `unit` of its run nor the barrier signal that
+ * would announce them, and every wait of that launch gives up after wait_limit_ns
  * (1 us .. 2 s).  A unit past the end of CTA 0's run stalls nothing.  The
  * outputs of that step are unspecified; llama_model_status then returns the
  * timeout code and resets the model's internal counters, after which the next

@@ -1,7 +1,8 @@
 """The device-side timeout path, exercised without a GPU fault.
 
 Every wait of a kernel on another agent (the TMA/MMA rings of the decode
-projection, the bulk-copy ring of the decode attention) is bounded.  A test
+and prefill projections, single-SM and CTA-pair, the bulk-copy ring of the
+decode attention) is bounded.  A test
 arms a one-shot stalled producer (llama_debug_stall): in the next launch of
 the chosen kernel, CTA 0 never issues the copies of one pipeline stage nor the
 barrier signal that would announce them, and that launch's waits give up after
@@ -77,4 +78,39 @@ def test_stall_arguments_are_checked(llb):
     m.debug_stall("projection", unit=0)
     m.debug_stall("none")                         # disarmed before any launch took it
     assert m.status() == 0
+    m.close()
+
+
+# wq/wk/wv of this shape (6144 x 4096 weights) runs on CTA pairs: 300 tokens
+# make 2 x 24 pair tiles, all split along K over the 74 pairs (41 or 42
+# stages each); the SHAPE above runs its wq/wk/wv (4096 x 2048) on single SMs
+# (4800 tokens: 38 x 16 tiles, 4 waves and a stream-K tail).
+PAIR_SHAPE = ModelShape(dim=4096, n_layers=1, n_heads=32, n_kv_heads=8, vocab_size=512, max_seq_len=320,
+                        max_batch_size=1, dtype="bf16", hidden=11008)
+
+
+@pytest.mark.parametrize("shape,B,T,unit", [(SHAPE, 8, 600, 0), (SHAPE, 8, 600, 2), (PAIR_SHAPE, 1, 300, 0),
+                                            (PAIR_SHAPE, 1, 300, 3)])
+def test_stalled_prefill_projection_times_out_and_the_next_prefill_is_exact(llb, shape, B, T, unit):
+    """The same for the prefill projections: the stall takes the first 16-bit
+    projection launch, which is the prefill's wq/wk/wv."""
+    s = shape
+    w = make_weights(s, 73)
+    m = build_model(s, w)
+    toks = make_tokens(s.vocab_size, (B, T), token_seed(23)).cuda()
+    m.debug_stall("projection", unit=unit, wait_limit_ns=1_000_000)
+    bad = torch.empty(B, s.vocab_size, device="cuda")
+    m.prefill(toks, logits=bad)
+    torch.cuda.synchronize()
+    assert m.status() == llb.LLAMA_ERR_DEVICE_TIMEOUT
+
+    good = torch.empty(B, s.vocab_size, device="cuda")
+    m.prefill(toks, logits=good)
+    torch.cuda.synchronize()
+    assert m.status() == 0
+    w64 = to_numpy_f64_weights(w)
+    args = oracle_args(s)
+    for b in (0, B - 1):
+        want = O.forward(args, w64, toks[b].cpu().tolist(), 0, O.new_cache(args))[-1]
+        assert rel_l2(good[b].cpu().numpy(), want) <= BF16_TOL, (unit, b)
     m.close()
