@@ -476,7 +476,7 @@ def run_ours(a, rank, world, local_rank):
                              "clocks": pre_clk,
                              "clocks_what": "SM clocks sampled while prefills run back to back: the power cap holds "
                                             "them below the maximum, which is what the sustained peak describes",
-                             "traffic": _traffic("linear_tcp_kernel"), "launches": len(pre),
+                             "traffic": _traffic("prefill_projections"), "launches": len(pre),
                              "what": "2*M*N*K of one prefill's projection launches / their event-timed durations "
                                      "(prefill launches run one after another in the product path too)",
                              "traffic_what": "DRAM bytes per launch, mean over the 128 projection launches of one "
