@@ -301,8 +301,7 @@ __device__ __forceinline__ void decode_epilogue_loop(uint32_t tmem_lane, uint64_
             // partials after this CTA's own, in CTA order.  Up to 4 token
             // columns: one float4 per contributor, 8 contributors per batch of
             // independent loads (each batch is an L2 round trip under full
-            // HBM load); wider: CB contributors' whole rows per batch.
-            constexpr int CB = BN <= 16 ? 4 : (BN <= 32 ? 2 : 1);
+            // HBM load); wider: see below.
             if (nb <= 4) {
                 for (int cb = cf + 1; cb <= cl; cb += 8) {
                     float4 f[8];
@@ -321,28 +320,41 @@ __device__ __forceinline__ void decode_epilogue_loop(uint32_t tmem_lane, uint64_
                     }
                 }
             }
-            for (int cb = cf + 1; nb > 4 && cb <= cl; cb += CB) {
-                float4 f[CB][BN / 4];
+            if (nb > 4) {
+                // the real columns of one contributor's row per load group;
+                // up to 32 columns, the next contributor's loads are issued
+                // before this one's are added (two groups in flight)
+                auto load = [&](float4 (&f)[BN / 4], int cc) {
+                    const float4* pp = reinterpret_cast<const float4*>(part + (static_cast<long long>(cc) * 128 + r) * BN);
 #pragma unroll
-                for (int e = 0; e < CB; ++e) {
-                    const int cc = cb + e;
-                    if (cc <= cl) {
-                        const float4* pp = reinterpret_cast<const float4*>(
-                            part + (static_cast<long long>(cc) * 128 + r) * BN);
+                    for (int qq = 0; qq < BN / 4; ++qq)
+                        if (4 * qq < nb) f[qq] = __ldcg(pp + qq);
+                };
+                auto add = [&](const float4 (&f)[BN / 4]) {
 #pragma unroll
-                        for (int qq = 0; qq < BN / 4; ++qq) f[e][qq] = __ldcg(pp + qq);
-                    }
-                }
-#pragma unroll
-                for (int e = 0; e < CB; ++e) {
-                    if (cb + e <= cl) {
-#pragma unroll
-                        for (int qq = 0; qq < BN / 4; ++qq) {
-                            v[4 * qq] += f[e][qq].x;
-                            v[4 * qq + 1] += f[e][qq].y;
-                            v[4 * qq + 2] += f[e][qq].z;
-                            v[4 * qq + 3] += f[e][qq].w;
+                    for (int qq = 0; qq < BN / 4; ++qq) {
+                        if (4 * qq < nb) {
+                            v[4 * qq] += f[qq].x;
+                            v[4 * qq + 1] += f[qq].y;
+                            v[4 * qq + 2] += f[qq].z;
+                            v[4 * qq + 3] += f[qq].w;
                         }
+                    }
+                };
+                if constexpr (BN <= 32) {
+                    float4 fa[BN / 4], fb[BN / 4];
+                    load(fa, cf + 1);
+                    for (int cb = cf + 1; cb <= cl; cb += 2) {
+                        if (cb + 1 <= cl) load(fb, cb + 1);
+                        add(fa);
+                        if (cb + 2 <= cl) load(fa, cb + 2);
+                        if (cb + 1 <= cl) add(fb);
+                    }
+                } else {
+                    for (int cb = cf + 1; cb <= cl; ++cb) {
+                        float4 f[BN / 4];
+                        load(f, cb);
+                        add(f);
                     }
                 }
             }

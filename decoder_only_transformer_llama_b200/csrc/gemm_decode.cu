@@ -36,6 +36,8 @@ namespace {
 constexpr int kThreads = 192;
 constexpr int kAccStride = 64;      // TMEM columns per accumulator buffer
 constexpr int kTmemCols = 128;      // two accumulator buffers
+constexpr int kMinUnitsPerCta = 4;   // 64 KB of weights
+constexpr int kMaxSplit = 8;         // CTAs sharing one weight tile, at most
 }  // namespace
 
 template <int BN, int STAGES, typename E>
@@ -227,8 +229,14 @@ static int launch_decode(const CUtensorMap& w, const CUtensorMap& x, int N, int 
     }
     const long long units = static_cast<long long>((N + 127) / 128) * ((K + 63) / 64);
     if (units > (1 << 22)) { set_error("decode projection too large (%lld work units)", units); return LLAMA_ERR_INVALID_ARG; }
+    // at least kMinUnitsPerCta units per CTA and at most kMaxSplit CTAs per
+    // weight tile: a small projection spread over every SM would split each
+    // tile among dozens of CTAs, and its finisher would add as many partials
     int P = max_ctas;
-    if (units < P) P = static_cast<int>(units);
+    const long long p_units = (units + kMinUnitsPerCta - 1) / kMinUnitsPerCta;
+    const long long p_tiles = static_cast<long long>(kMaxSplit) * ((N + 127) / 128);
+    if (p_units < P) P = static_cast<int>(p_units);
+    if (p_tiles < P) P = static_cast<int>(p_tiles);
     cudaError_t e = launch_k(kern, dim3(P), dim3(kThreads), smem, st, pdl, w, x, N, M, K, ep, part, counters, nio);
     count_launch();
     if (e != cudaSuccess) return cuda_fail(e, "linear_decode_kernel");
