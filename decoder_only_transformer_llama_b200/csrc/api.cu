@@ -665,6 +665,9 @@ int llama_model_create_tp(const llama_model_args* args, int tp_rank, int tp_size
             if (rc == LLAMA_OK) rc = encode_kmajor_16(&m->m_kcache, m->kc, static_cast<int>(kv_rows), l.hd, 128, l.dtype);
             if (rc == LLAMA_OK) rc = encode_kmajor_16(&m->m_vcache, m->vc, static_cast<int>(kv_rows), l.hd, 128, l.dtype);
             m->has_attn_maps = rc == LLAMA_OK;
+            if (rc == LLAMA_OK) rc = encode_kmajor_16(&m->m_kdec, m->kc, static_cast<int>(kv_rows), l.hd, 64, l.dtype);
+            if (rc == LLAMA_OK) rc = encode_kmajor_16(&m->m_vdec, m->vc, static_cast<int>(kv_rows), l.hd, 64, l.dtype);
+            m->has_dec_maps = rc == LLAMA_OK;
         }
     }
     cudaStream_t st = m->last_stream;

@@ -11,6 +11,7 @@
 // softmax over 64-key tiles staged in shared memory (fp32 CUDA-core
 // arithmetic).  16-bit models use the tensor-core kernel of attention_prefill_tc.cu.
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "model.h"
@@ -99,17 +100,117 @@ __device__ __forceinline__ int owner64(long long u, long long W, long long P) {
     return static_cast<int>(((u + 1) * P - 1) / W);
 }
 
-template <typename T, int HD, int NREP>
+// ---------------------------------------------------------------- decode units on the tensor cores
+// (mma.sync m16n8k16, bf16 or fp16 in, fp32 accumulate: a decode unit is a
+// 16-row problem, too small for tcgen05's 128-row tiles)
+namespace {
+__device__ __forceinline__ void dec_ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void dec_ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                              uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+// c += A B with A rows 8..15 zero (a1 = a3 = 0).
+template <typename T>
+__device__ __forceinline__ void dec_mma(float (&c)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+    if constexpr (std::is_same<T, bf16>::value) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+    } else {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+    }
+}
+// Shared-memory address of key `key`, dims d..d+7 of a 64-key block stored as
+// two 128-byte-swizzled TMA boxes (dims 0-63, then 64-127; 8 KB each).
+__device__ __forceinline__ uint32_t dec_swz(uint32_t base, int key, int d) {
+    return base + static_cast<uint32_t>((d >> 6) * 8192 + key * 128 + ((((d & 63) >> 3) ^ (key & 7)) << 4));
+}
+}  // namespace
+
+// Ring slots (64-key K+V units) per decode-attention CTA (six for one CTA per
+// SM measured the same as three on the 70B-shaped slice).
+constexpr int kDecodeSlots = 3;
+
+// One 64-key unit for warp `warp` (keys 16*warp .. 16*warp+15 of it, n valid):
+// S = Q K^T for the group's query heads, online softmax per head (m, l), and
+// O += P V, all as m16n8k16 fragments; lane (g = lane/4, t = lane%4) holds
+// head g's scores of keys 8nt + 2t, +1 and O columns 8nd + 2t, +1.
+template <typename T, int NREP>
+__device__ __forceinline__ void tc_unit(const T* sK, const T* sV, int warp, int lane, int n, float scale,
+                                        const uint32_t (&qa)[8][2], float& m_run, float& l_run,
+                                        float (&oacc)[16][4]) {
+    const int mi = lane >> 3, rr = lane & 7, t = lane & 3;
+    const uint32_t kb = smem_u32(sK), vb = smem_u32(sV);
+    float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+        // matrices: keys 0-7 / dims 0-7, keys 0-7 / dims 8-15, keys 8-15 / dims 0-7, keys 8-15 / dims 8-15
+        uint32_t b00, b01, b10, b11;
+        dec_ldsm_x4(dec_swz(kb, 16 * warp + ((mi >> 1) << 3) + rr, 16 * ks + ((mi & 1) << 3)), b00, b01, b10, b11);
+        dec_mma<T>(sc[0], qa[ks][0], qa[ks][1], b00, b01);
+        dec_mma<T>(sc[1], qa[ks][0], qa[ks][1], b10, b11);
+    }
+    float s4[4] = {sc[0][0] * scale, sc[0][1] * scale, sc[1][0] * scale, sc[1][1] * scale};
+    const int k0 = 16 * warp + 2 * t;
+    if (k0 >= n) s4[0] = -INFINITY;
+    if (k0 + 1 >= n) s4[1] = -INFINITY;
+    if (k0 + 8 >= n) s4[2] = -INFINITY;
+    if (k0 + 9 >= n) s4[3] = -INFINITY;
+    float mx = fmaxf(fmaxf(s4[0], s4[1]), fmaxf(s4[2], s4[3]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float mnew = fmaxf(m_run, mx);          // finite: key 16*warp is valid
+    const float corr = __expf(m_run - mnew);      // 0 while m_run is -inf
+    float p[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) p[e] = __expf(s4[e] - mnew);
+    float rs = (p[0] + p[1]) + (p[2] + p[3]);
+    rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+    rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+    l_run = l_run * corr + rs;
+    m_run = mnew;
+    const uint32_t pa0 = pack2<T>(p[0], p[1]), pa2 = pack2<T>(p[2], p[3]);
+#pragma unroll
+    for (int nd = 0; nd < 16; ++nd) {
+        oacc[nd][0] *= corr;
+        oacc[nd][1] *= corr;
+    }
+#pragma unroll
+    for (int np = 0; np < 8; ++np) {
+        // transposed: keys 0-7 / dims 16np.., keys 8-15 / dims 16np.., keys 0-7 / dims 16np+8.., keys 8-15 / dims 16np+8..
+        uint32_t v00, v01, v10, v11;
+        dec_ldsm_x4_t(dec_swz(vb, 16 * warp + ((mi & 1) << 3) + rr, 16 * np + ((mi >> 1) << 3)), v00, v01, v10, v11);
+        dec_mma<T>(oacc[2 * np], pa0, pa2, v00, v01);
+        dec_mma<T>(oacc[2 * np + 1], pa0, pa2, v10, v11);
+    }
+}
+
+template <typename T, int HD, int NREP, bool TC>
 __global__ void __launch_bounds__(128)
 attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* __restrict__ vc,
-                   const int32_t* __restrict__ pos, int B, int nkv, int nq, int S, long long row_stride,
-                   float* __restrict__ part_o, float* __restrict__ part_ml, int* __restrict__ counters,
-                   T* __restrict__ out, int* status, unsigned long long* tl, long long wait_ns, int stall) {
+                   const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+                   long long row_base, const int32_t* __restrict__ pos, int B, int nkv, int nq, int S,
+                   long long row_stride, float* __restrict__ part_o, float* __restrict__ part_ml,
+                   int* __restrict__ counters, T* __restrict__ out, int* status, unsigned long long* tl,
+                   long long wait_ns, int stall) {
     constexpr int EPL = HD / 32;   // head dims per lane
     constexpr int ROW = HD * static_cast<int>(sizeof(T));
     constexpr int CH_BYTES = kChunk * ROW;
-    constexpr int NSLOT = 3;
-    extern __shared__ __align__(128) uint8_t dsm[];
+    constexpr int NSLOT = kDecodeSlots;
+    static_assert(!TC || (HD == 128 && sizeof(T) == 2), "tensor-core units: 16-bit cache, head_dim 128");
+    extern __shared__ __align__(128) uint8_t dsm_raw[];
+    // ring slots 1024-byte aligned (128-byte swizzled TMA boxes on the tensor-core path)
+    uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t bar[NSLOT];
     __shared__ float s_m[4][NREP], s_l[4][NREP];
     __shared__ float s_o[4][NREP][HD];
@@ -191,10 +292,21 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
         uint8_t* slot = dsm + (i % NSLOT) * 2 * CH_BYTES;
         const long long ho = head_off(icur);
         if (i != stall_i) {
-            mbar_arrive_expect_tx(&bar[i % NSLOT], 2u * n * ROW);
-            bulk_load_hint(slot, kc + ho + static_cast<long long>(j0) * HD, n * ROW, &bar[i % NSLOT], pol_kv);
-            bulk_load_hint(slot + CH_BYTES, vc + ho + static_cast<long long>(j0) * HD, n * ROW, &bar[i % NSLOT],
-                           pol_kv);
+            if constexpr (TC) {
+                // four 64-key x 64-dim boxes (K and V, dims 0-63 and 64-127), whole
+                // boxes even past the valid keys (masked in the scores)
+                const int row = static_cast<int>(row_base + (static_cast<long long>(icur.b) * nkv + icur.g) * S + j0);
+                mbar_arrive_expect_tx(&bar[i % NSLOT], 2u * CH_BYTES);
+                tma_load_2d_hint(slot, &mapK, 0, row, &bar[i % NSLOT], pol_kv);
+                tma_load_2d_hint(slot + CH_BYTES / 2, &mapK, 64, row, &bar[i % NSLOT], pol_kv);
+                tma_load_2d_hint(slot + CH_BYTES, &mapV, 0, row, &bar[i % NSLOT], pol_kv);
+                tma_load_2d_hint(slot + CH_BYTES + CH_BYTES / 2, &mapV, 64, row, &bar[i % NSLOT], pol_kv);
+            } else {
+                mbar_arrive_expect_tx(&bar[i % NSLOT], 2u * n * ROW);
+                bulk_load_hint(slot, kc + ho + static_cast<long long>(j0) * HD, n * ROW, &bar[i % NSLOT], pol_kv);
+                bulk_load_hint(slot + CH_BYTES, vc + ho + static_cast<long long>(j0) * HD, n * ROW, &bar[i % NSLOT],
+                               pol_kv);
+            }
         }
         advance(icur);
     };
@@ -270,7 +382,28 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
     Cur cur = cur_at(u0);
     float qv[NREP][EPL];
     float mx[NREP], sl[NREP], o[NREP][EPL];
+    // tensor-core path (TC): per warp, rows g = lane / 4 of the m16n8k16
+    // fragments are the group's query heads (rows >= NREP stay zero)
+    const int tg = lane >> 2, tt = lane & 3;
+    uint32_t qa[TC ? 8 : 1][2];          // Q A-fragments per 16-dim step: dims 2tt.., 2tt+8..
+    float m_run = -INFINITY, l_run = 0.f;
+    float oacc[TC ? 16 : 1][4];          // O rows tg (and tg+8, unused), dims 8nd + 2tt, +1
     auto start_pair = [&]() {
+        if constexpr (TC) {
+            const T* qrow = q + static_cast<long long>(cur.b) * nq + (cur.g * NREP + tg) * HD;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                qa[ks][0] = tg < NREP ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tt) : 0u;
+                qa[ks][1] = tg < NREP ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tt + 8) : 0u;
+            }
+            m_run = -INFINITY;
+            l_run = 0.f;
+#pragma unroll
+            for (int nd = 0; nd < 16; ++nd)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) oacc[nd][e] = 0.f;
+            return;
+        }
 #pragma unroll
         for (int r = 0; r < NREP; ++r) {
             Vec<T, EPL>::load(q + static_cast<long long>(cur.b) * nq + (cur.g * NREP + r) * HD + lane * EPL, qv[r]);
@@ -296,6 +429,9 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
         const T* sV = reinterpret_cast<const T*>(dsm + (i % NSLOT) * 2 * CH_BYTES + CH_BYTES);
         const int ctx = s_pos[cur.b] + 1;
         const int n = min(kChunk, ctx - cur.j * kChunk);
+        if constexpr (TC) {
+            if (16 * warp < n) tc_unit<T, NREP>(sK, sV, warp, lane, n, scale, qa, m_run, l_run, oacc);
+        } else {
 #pragma unroll 1
         for (int jb = warp * 16; jb < min(n, warp * 16 + 16); jb += 8) {
             // eight keys: this lane's partial dot products ...
@@ -358,6 +494,7 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
                 }
             }
         }
+        }
         __syncthreads();                               // ring slot i % NSLOT is free again
         if (threadIdx.x == 0 && i + NSLOT < len) issue(i + NSLOT);
         const int nch = s_nch[cur.b];
@@ -365,14 +502,25 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
 
         // ---- end of a segment: merge the 4 warps, then write the row or a partial
         const bool whole = seg_j0 == 0 && cur.j + 1 == nch;
-        if (lane == 0) {
+        if constexpr (TC) {
+            if (tg < NREP) {
+                if (tt == 0) { s_m[warp][tg] = m_run; s_l[warp][tg] = l_run; }
 #pragma unroll
-            for (int r = 0; r < NREP; ++r) { s_m[warp][r] = mx[r]; s_l[warp][r] = sl[r]; }
+                for (int nd = 0; nd < 16; ++nd) {
+                    s_o[warp][tg][8 * nd + 2 * tt] = oacc[nd][0];
+                    s_o[warp][tg][8 * nd + 2 * tt + 1] = oacc[nd][1];
+                }
+            }
+        } else {
+            if (lane == 0) {
+#pragma unroll
+                for (int r = 0; r < NREP; ++r) { s_m[warp][r] = mx[r]; s_l[warp][r] = sl[r]; }
+            }
+#pragma unroll
+            for (int r = 0; r < NREP; ++r)
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) s_o[warp][r][lane * EPL + e] = o[r][e];
         }
-#pragma unroll
-        for (int r = 0; r < NREP; ++r)
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) s_o[warp][r][lane * EPL + e] = o[r][e];
         __syncthreads();
         const long long pair_u0 = static_cast<long long>(s_cum[cur.b]) * nkv + static_cast<long long>(cur.g) * nch;
         const int slot_id = c * 2 + (seg_i0 == 0 ? 0 : 1);
@@ -502,13 +650,16 @@ attn_decode_kernel(const T* __restrict__ q, const T* __restrict__ kc, const T* _
 
 static int g_attn_sms = 0;
 
-template <typename T, int HD, int NREP>
+template <typename T, int HD, int NREP, bool TC>
 static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl,
                      unsigned long long* tl, long long wait_ns, int stall) {
     const T* kc = static_cast<const T*>(m->kc) + layer * m->kv_layer_elems;
     const T* vc = static_cast<const T*>(m->vc) + layer * m->kv_layer_elems;
-    auto kern = attn_decode_kernel<T, HD, NREP>;
-    const int smem = 3 * 2 * kChunk * HD * static_cast<int>(sizeof(T));   // three K+V chunks
+    auto kern = attn_decode_kernel<T, HD, NREP, TC>;
+    // the ring's K+V chunks, 1024-byte aligned
+    const int smem = kDecodeSlots * 2 * kChunk * HD * static_cast<int>(sizeof(T)) + 1024;
+    // first cache row of this layer in the [L * Bmax * nkv * S][hd] tensor maps
+    const long long row_base = static_cast<long long>(layer) * m->Bmax * m->nkv * m->S;
     static int per_sm = 0;
     if (per_sm == 0) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -531,8 +682,9 @@ static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaS
     P = std::min<long long>(P, static_cast<long long>(B) * m->nkv * m->n_splits);
     P = std::max<long long>(P, 1);
     cudaError_t e = launch_k(kern, dim3(static_cast<unsigned>(P)), dim3(128), smem, st, pdl, static_cast<const T*>(m->q),
-                             kc, vc, pos, B, m->nkv, m->nq, m->S, m->kv_row_elems, m->part_o, m->part_ml,
-                             m->attn_cnt, static_cast<T*>(m->attn), m->status, tl, wait_ns, stall);
+                             kc, vc, m->m_kdec, m->m_vdec, row_base, pos, B, m->nkv, m->nq, m->S, m->kv_row_elems,
+                             m->part_o, m->part_ml, m->attn_cnt, static_cast<T*>(m->attn), m->status, tl, wait_ns,
+                             stall);
     count_launch();
     if (e != cudaSuccess) return cuda_fail(e, "attn_decode_kernel");
     return LLAMA_OK;
@@ -541,11 +693,21 @@ static int decode_go(const Model* m, int layer, const int32_t* pos, int B, cudaS
 template <typename T, int HD>
 static int decode_rep(const Model* m, int layer, const int32_t* pos, int B, cudaStream_t st, bool pdl,
                       unsigned long long* tl, long long wait_ns, int stall) {
+    // 16-bit caches with head_dim 128 and their tensor maps: units on the tensor cores
+    constexpr bool kTcOk = HD == 128 && sizeof(T) == 2;
+    if (kTcOk && m->has_dec_maps) {
+        switch (m->n_rep) {
+            case 1: return decode_go<T, HD, 1, kTcOk>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+            case 2: return decode_go<T, HD, 2, kTcOk>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+            case 4: return decode_go<T, HD, 4, kTcOk>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+            case 8: return decode_go<T, HD, 8, kTcOk>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+        }
+    }
     switch (m->n_rep) {
-        case 1: return decode_go<T, HD, 1>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
-        case 2: return decode_go<T, HD, 2>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
-        case 4: return decode_go<T, HD, 4>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
-        case 8: return decode_go<T, HD, 8>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+        case 1: return decode_go<T, HD, 1, false>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+        case 2: return decode_go<T, HD, 2, false>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+        case 4: return decode_go<T, HD, 4, false>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
+        case 8: return decode_go<T, HD, 8, false>(m, layer, pos, B, st, pdl, tl, wait_ns, stall);
     }
     set_error("n_heads / n_kv_heads = %d unsupported (1, 2, 4, 8)", m->n_rep);
     return LLAMA_ERR_INVALID_ARG;

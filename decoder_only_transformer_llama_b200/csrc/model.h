@@ -185,6 +185,9 @@ struct Model {
     // 64 columns x 128 rows.
     CUtensorMap m_qtile, m_kcache, m_vcache;
     bool has_attn_maps = false;
+    // the same caches in 64-key x 64-dim boxes (decode attention on the tensor cores)
+    CUtensorMap m_kdec, m_vdec;
+    bool has_dec_maps = false;
     cudaStream_t last_stream;
     Profile prof;
     // Timeline of decode launches: while tl_on, launch i of llama_decode_step
