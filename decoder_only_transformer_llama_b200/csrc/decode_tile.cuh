@@ -154,7 +154,7 @@ __device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int la
         // residual add, plus this tile's share of sum(x^2) for the next RMSNorm;
         // the old x values of a 16-column group are loaded together
         const float wn = pre ? pre->wn : (row_ok ? nio.w_next[n] : 0.f);
-        float xo[16];
+        float xo[16];   // v[b] becomes x^2 of column b below
 #pragma unroll
         for (int b = 0; b < BN; ++b) {
             if (b >= nb) break;   // uniform over the CTA
@@ -165,14 +165,33 @@ __device__ __forceinline__ void finish_tile(float (&v)[BN], int t, int r, int la
                                 : ((row_ok && b + u < nb) ? ep.out[static_cast<long long>(b + u) * ep.ldo + n] : 0.f);
             }
             float sq = 0.f;
-            if (row_ok && b < nb) {
+            if (row_ok) {
                 const float nv = xo[b & 15] + v[b];
                 ep.out[static_cast<long long>(b) * ep.ldo + n] = nv;
                 static_cast<T*>(nio.y_out)[static_cast<long long>(b) * ep.ldo + n] = from_f32<T>(nv * wn);
                 sq = nv * nv;
             }
-            sq = warp_sum(sq);
-            if (lane == 0) red[q * 64 + b] = sq;
+            v[b] = sq;
+        }
+        // the warp's column sums of x^2, 32 columns at a time, by a
+        // transposing butterfly: after it lane l holds column c0 + l's sum
+#pragma unroll
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+            if (c0 >= nb) break;   // uniform over the CTA
+            float a[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) a[i] = (c0 + i < BN && c0 + i < nb) ? v[c0 + i] : 0.f;
+#pragma unroll
+            for (int step = 16, h = 16; step >= 1; step >>= 1, h >>= 1) {
+                const bool upper = (lane & step) != 0;
+#pragma unroll
+                for (int i = 0; i < h; ++i) {
+                    const float send = upper ? a[i] : a[i + h];
+                    const float keep = upper ? a[i + h] : a[i];
+                    a[i] = keep + __shfl_xor_sync(0xffffffffu, send, step);
+                }
+            }
+            if (c0 + lane < nb) red[q * 64 + c0 + lane] = a[0];
         }
         named_sync(2, 128);
         if (epi_tid < nb)
