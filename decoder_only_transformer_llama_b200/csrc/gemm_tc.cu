@@ -22,12 +22,14 @@
 // counter: it adds the fp32 partials in CTA order (deterministic) and applies
 // the epilogue; no CTA ever waits for another.
 //
-// Warp roles (192 threads):
+// Warp roles (320 threads):
 //   warp 0 lane 0  TMA producer (4-deep ring of 128x64 A + 256x64 B tiles)
 //   warp 1 lane 0  MMA issuer (tcgen05.mma kind::f16, M=128, N=256, K=16)
 //   warp 1         TMEM owner: two 256-column accumulators, so the MMAs of
 //                  one item run while the epilogue drains the previous one
-//   warps 2-5      epilogue: warp w reads TMEM lanes 32*(w%4)..+31 = token rows
+//   warps 2-9      epilogue: warp w reads TMEM lanes 32*(w%4)..+31 = token rows,
+//                  warps 2-5 the tile's first 128 columns, warps 6-9 the other
+//                  128 (twice the epilogue's loads and stores in flight)
 // Every wait is bounded; no TMA multicast.
 #include "common.cuh"
 #include "epilogue.cuh"
@@ -41,7 +43,8 @@ namespace llb {
 
 namespace {
 
-constexpr int kThreadsTc = 192;
+constexpr int kEpiThreads = 256;             // eight epilogue warps: two per TMEM lane quarter
+constexpr int kThreadsTc = 64 + kEpiThreads;
 constexpr int kBN = 256;                     // tile width along N (weight rows)
 constexpr int kStagesTc = 4;
 constexpr int kA_BYTES = 128 * 128;          // 128 rows x 64 16-bit values
@@ -214,7 +217,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStagesTc; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-        for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 128); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], kEpiThreads); }
         mbar_init(mdone, 1);
         flag[0] = 0;
         fence_mbar_init();
@@ -286,6 +289,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
         const int r = q * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const int epi_tid = threadIdx.x - 64;
+        const int c_lo = ((warp - 2) >> 2) * 4;   // warps 2-5: 32-column chunks 0-3, warps 6-9: chunks 4-7
         const int Wsk = plan.sk * KT;
         const int Psk = plan.psk;
         const int u0 = c < Psk ? run_begin(c, Wsk, Psk) : 0;
@@ -296,7 +300,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
             const int acc = j & 1;
             const bool ok_wait = mbar_wait(&tfull[acc], (j >> 1) & 1, wlim);
             tc_fence_after();
-            if (named_any(1, 128, !ok_wait || *reinterpret_cast<volatile int*>(&flag[0]) != 0)) {
+            if (named_any(1, kEpiThreads, !ok_wait || *reinterpret_cast<volatile int*>(&flag[0]) != 0)) {
                 if (epi_tid == 0) report_status(ep.status, LLAMA_ERR_DEVICE_TIMEOUT);
                 break;
             }
@@ -317,7 +321,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
             if (it.ks == 0 && it.ke == KT) {
                 // whole tile: TMEM -> epilogue, 32 features at a time
 #pragma unroll 1
-                for (int cc = 0; cc < kBN / 32; ++cc) {
+                for (int cc = c_lo; cc < c_lo + 4; ++cc) {
                     float v[32];
                     tmem_ld_32x32b_x32(tb + cc * 32, v);
                     tc_wait_ld();
@@ -334,7 +338,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
             const int slot = (ub + it.ks == u0) ? 0 : 1;   // the run's first segment, or its last
             float* my = part + (static_cast<long long>(c) * 2 + slot) * kPartFloats + r;
 #pragma unroll 1
-            for (int cc = 0; cc < kBN / 32; ++cc) {
+            for (int cc = c_lo; cc < c_lo + 4; ++cc) {
                 float v[32];
                 tmem_ld_32x32b_x32(tb + cc * 32, v);
                 tc_wait_ld();
@@ -342,9 +346,9 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
                 for (int t = 0; t < 32; ++t) my[(cc * 32 + t) * 128] = v[t];
             }
             __threadfence();
-            named_sync(1, 128);
+            named_sync(1, kEpiThreads);
             if (epi_tid == 0) flag[1] = atomicAdd(&counters[tl], 1);
-            named_sync(1, 128);
+            named_sync(1, kEpiThreads);
             if (flag[1] != cl - cf) {   // not the last contributor
                 tc_fence_before();
                 mbar_arrive(&tempty[acc]);
@@ -353,7 +357,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
             __threadfence();
             // last contributor: sum the partials in CTA order, then the epilogue
 #pragma unroll 1
-            for (int cc = 0; cc < kBN / 32; ++cc) {
+            for (int cc = c_lo; cc < c_lo + 4; ++cc) {
                 float own[32], v[32];
                 tmem_ld_32x32b_x32(tb + cc * 32, own);
                 tc_wait_ld();
@@ -535,6 +539,7 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
         const int r = q * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const int epi_tid = threadIdx.x - 64;
+        const int c_lo = ((warp - 2) >> 2) * 4;   // warps 2-5: 32-column chunks 0-3, warps 6-9: chunks 4-7
         const int Wsk = plan.sk * KT;
         const int Psk = plan.psk;
         const int u0 = c < Psk ? run_begin(c, Wsk, Psk) : 0;
@@ -545,14 +550,14 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
         // hand accumulator `a` back to rank 0's MMA issuer: one arrive per CTA
         auto release = [&](int a) {
             tc_fence_before();
-            named_sync(1, 128);
+            named_sync(1, kEpiThreads);
             if (epi_tid == 0) mbar_arrive_cluster(tempty_rank0 + 8u * static_cast<uint32_t>(a));
         };
         while (work_next(w, plan, P, it)) {
             const int acc = j & 1;
             const bool ok_wait = mbar_wait(&tfull[acc], (j >> 1) & 1, wlim);
             tc_fence_after();
-            if (named_any(1, 128, !ok_wait || *reinterpret_cast<volatile int*>(&flag[0]) != 0)) {
+            if (named_any(1, kEpiThreads, !ok_wait || *reinterpret_cast<volatile int*>(&flag[0]) != 0)) {
                 if (epi_tid == 0) report_status(ep.status, LLAMA_ERR_DEVICE_TIMEOUT);
                 break;
             }
@@ -571,7 +576,7 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
             }
             if (it.ks == 0 && it.ke == KT) {
 #pragma unroll 1
-                for (int cc = 0; cc < kPairTile / 32; ++cc) {
+                for (int cc = c_lo; cc < c_lo + 4; ++cc) {
                     float v[32];
                     tmem_ld_32x32b_x32(tb + cc * 32, v);
                     tc_wait_ld();
@@ -589,7 +594,7 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
             const int cnt_idx = 2 * tl + static_cast<int>(rank);
             float* my = part + (static_cast<long long>(2 * c + static_cast<int>(rank)) * 2 + slot) * kPartFloats + r;
 #pragma unroll 1
-            for (int cc = 0; cc < kPairTile / 32; ++cc) {
+            for (int cc = c_lo; cc < c_lo + 4; ++cc) {
                 float v[32];
                 tmem_ld_32x32b_x32(tb + cc * 32, v);
                 tc_wait_ld();
@@ -597,16 +602,16 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
                 for (int t = 0; t < 32; ++t) my[(cc * 32 + t) * 128] = v[t];
             }
             __threadfence();
-            named_sync(1, 128);
+            named_sync(1, kEpiThreads);
             if (epi_tid == 0) flag[1] = atomicAdd(&counters[cnt_idx], 1);
-            named_sync(1, 128);
+            named_sync(1, kEpiThreads);
             if (flag[1] != cl - cf) {
                 release(acc);
                 continue;
             }
             __threadfence();
 #pragma unroll 1
-            for (int cc = 0; cc < kPairTile / 32; ++cc) {
+            for (int cc = c_lo; cc < c_lo + 4; ++cc) {
                 float own[32], v[32];
                 tmem_ld_32x32b_x32(tb + cc * 32, own);
                 tc_wait_ld();
