@@ -704,10 +704,35 @@ def run_workload(a):
                 ms, clk = _timed(g.replay, max(100, a.iters, _reps_for(once)), stream, clocks=True)
                 ms /= LAYER_CHAIN
                 byts = decode_step_bytes(s, B, L + 1)
+                # the layer's own share of a step (the microbench has no
+                # embedding and no head): exclusive device time of its five
+                # launches in the second of two graph-replayed steps, from the
+                # library's timeline, against the layer's bytes alone
+                model.timeline_start()
+                g_tl = capture_graph(lambda: (step(), step()), dev, stream)
+                model.timeline_stop()
+                for _ in range(8):
+                    g_tl.replay()
+                del g_tl
+                recs = model.timeline_stop()
+                n_step = len(recs) // 2
+                ends = [r[0] for r in recs]
+                second = range(n_step, 2 * n_step)
+                head = max(i for i in second if recs[i][1] == "projection")
+                layer_ns = sum(ends[i] - ends[i - 1] for i in second
+                               if recs[i][1] in ("projection", "attention") and i != head)
+                layer_bytes = (byts - 2 * s.vocab_size * s.dim - 4 * s.dim - 2 * B * s.dim
+                               - 4 * B * s.vocab_size)
                 out.append({"workload": name, "n_layers": s.n_layers, "head_rows": s.vocab_size, "batch": B,
                             "context": L + 1, "steps_per_graph": LAYER_CHAIN, "us_per_step": round(ms * 1e3, 2),
                             "tok_s": round(B / (ms / 1e3), 1), "GB_s": round(byts / ms / 1e6, 1),
                             "hbm_frac": round(byts / ms / 1e6 / hbm, 4), "peak_source": peak_src,
+                            "layer_us": round(layer_ns / 1e3, 2),
+                            "layer_tok_s": round(B / (layer_ns / 1e9), 1),
+                            "layer_hbm_frac": round(layer_bytes / layer_ns / hbm, 4),
+                            "layer_what": "the layer's five launches (wq/wk/wv, attention, wo, w1/w3, w2) of a "
+                                          "graph-replayed step, exclusive %globaltimer time each, without the "
+                                          "embedding and the 256-row stand-in head a library step also runs",
                             "clocks": clk})
                 del g
     else:
