@@ -51,33 +51,38 @@ constexpr int kA_BYTES = 128 * 128;          // 128 rows x 64 16-bit values
 constexpr int kB_BYTES = kBN * 128;
 constexpr int kStageBytes = kA_BYTES + kB_BYTES;
 constexpr int kPartFloats = 128 * kBN;       // one fp32 partial tile
+constexpr int kStgBytes = (kEpiThreads / 32) * 32 * 32 * 4;   // epilogue staging: 32 x 32 fp32 per warp
 
-// Store 32 consecutive values in the 16-bit type E (64 bytes, 16-byte aligned destination).
+// Epilogue of one 32 x 32 block of a tile: token rows m0..m0+31 (one warp's
+// TMEM lane quarter; lane = row as tcgen05.ld delivers it) x output features
+// n0..n0+31, after the consumer side of a fused RMSNorm (scale by the row's
+// 1/rms).  The 16-bit outputs (q/k/v with RoPE, silu(w1 x) * w3 x) are
+// written straight from the lane's row: 64 or 32 contiguous bytes each.  The
+// fp32 outputs (residual add, stores) go through the warp's 4 KB of shared
+// memory so that every global access is row-contiguous: phase 1 writes the
+// lane's row as float4s whose slot is XOR-swizzled by the row (conflict-free
+// both ways), phase 2 has lane = (row rr of a group of 4, float4 column f):
+// 4 rows x 128 bytes per warp access instead of 32 rows x 16 bytes.  `sq`
+// accumulates the lane's row's sum of x^2 for the next RMSNorm; it is written
+// when the chunk closes a 128-feature block.
 template <typename E>
-__device__ __forceinline__ void store32_16(E* dst, const float* v) {
-    uint4* d = reinterpret_cast<uint4*>(dst);
+__device__ __forceinline__ void epi_block(const Epi& ep, const NormIO& nio, int m0, int n0, int rowsA, int rowsB,
+                                          float rs, float (&v)[32], float4* stg, int lane, float& sq) {
+    if (n0 >= rowsB) return;   // the same for the whole warp
+    if (nio.ssq_in) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint4 u;
-        u.x = pack2<E>(v[8 * q + 0], v[8 * q + 1]);
-        u.y = pack2<E>(v[8 * q + 2], v[8 * q + 3]);
-        u.z = pack2<E>(v[8 * q + 4], v[8 * q + 5]);
-        u.w = pack2<E>(v[8 * q + 6], v[8 * q + 7]);
-        d[q] = u;
+        for (int t = 0; t < 32; ++t) v[t] *= rs;
     }
-}
-
-// Epilogue of 32 consecutive output features n0..n0+31 of token row m.
-template <typename E>
-__device__ __forceinline__ void epi_chunk(const Epi& ep, int m, int n0, int rowsB, float (&v)[32]) {
-    if (n0 >= rowsB) return;
+    const int sw = lane & 7;
+    const int mrow = m0 + lane;
     if (ep.mode == EPI_SWIGLU) {
-        // each 32-column chunk holds 16 w1 outputs then the same 16 w3 outputs
+        // lane = token row: each 32-column chunk holds 16 w1 outputs, then the
+        // same 16 w3 outputs; 32 bytes of g per row
+        if (mrow >= rowsA) return;
         float g16[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t) g16[t] = silu_f(v[t]) * v[16 + t];
-        E* dst = static_cast<E*>(ep.g) + static_cast<long long>(m) * ep.H + (n0 / 32) * 16;
-        uint4* d4 = reinterpret_cast<uint4*>(dst);
+        uint4* d4 = reinterpret_cast<uint4*>(static_cast<E*>(ep.g) + static_cast<long long>(mrow) * ep.H + (n0 / 32) * 16);
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
             uint4 u;
@@ -87,110 +92,136 @@ __device__ __forceinline__ void epi_chunk(const Epi& ep, int m, int n0, int rows
             u.w = pack2<E>(g16[8 * q + 6], g16[8 * q + 7]);
             d4[q] = u;
         }
-    } else if (ep.mode == EPI_QKV) {
-        const int pos = ep.tok_pos[m];
+        return;
+    }
+    if (ep.mode == EPI_QKV) {
+        // lane = token row: RoPE on q and k, 64 bytes to q or to the cache
+        // (the chunk lies inside one head of q, k or v: hd is a multiple of 32)
+        if (mrow >= rowsA) return;
+        const int pos = ep.tok_pos[mrow];
         if (pos < 0 || pos >= ep.max_seq) return;
         E* dst;
-        bool rot;
+        bool rot = true;
         int d0;
         if (n0 < ep.nq) {
             d0 = n0 % ep.hd;
-            rot = true;
-            dst = static_cast<E*>(ep.q) + static_cast<long long>(m) * ep.nq + n0;
+            dst = static_cast<E*>(ep.q) + static_cast<long long>(mrow) * ep.nq + n0;
         } else {
             int cc = n0 - ep.nq;
             E* cache = static_cast<E*>(ep.kc);
-            rot = cc < ep.nkvc;
-            if (!rot) { cc -= ep.nkvc; cache = static_cast<E*>(ep.vc); }
+            if (cc >= ep.nkvc) {
+                cc -= ep.nkvc;
+                cache = static_cast<E*>(ep.vc);
+                rot = false;
+            }
             const int head = cc / ep.hd;
             d0 = cc % ep.hd;
-            const int row = ep.tok_row ? ep.tok_row[m] : m;
+            const int row = ep.tok_row ? ep.tok_row[mrow] : mrow;
             dst = cache + static_cast<long long>(row) * ep.kv_row_stride +
                   (static_cast<long long>(head) * ep.max_seq + pos) * ep.hd + d0;
         }
         if (rot) {
+            // (cos, sin) of rotation pairs d0/2 .. d0/2 + 15, two per float4
+            const float4* cs4 = reinterpret_cast<const float4*>(ep.rope + static_cast<long long>(pos) * (ep.hd / 2) + (d0 >> 1));
 #pragma unroll
-            for (int t = 0; t < 32; t += 2) rope_pair(ep.rope, ep.hd, pos, (d0 + t) >> 1, v[t], v[t + 1]);
-        }
-        store32_16<E>(dst, v);
-    } else {
-        float* o = ep.out + static_cast<long long>(m) * ep.ldo + n0;
-        const int lim = min(32, rowsB - n0);
-        if (lim == 32 && (ep.ldo % 4) == 0) {
-            float4* o4 = reinterpret_cast<float4*>(o);
-            if (ep.mode == EPI_RESID_F32) {
-                float4 p[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) p[q] = o4[q];
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    o4[q] = make_float4(p[q].x + v[4 * q], p[q].y + v[4 * q + 1], p[q].z + v[4 * q + 2],
-                                        p[q].w + v[4 * q + 3]);
-            } else {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) o4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            for (int t = 0; t < 32; t += 4) {
+                const float4 cs = cs4[t >> 2];
+                const float a0 = v[t] * cs.x - v[t + 1] * cs.y, b0 = v[t] * cs.y + v[t + 1] * cs.x;
+                const float a1 = v[t + 2] * cs.z - v[t + 3] * cs.w, b1 = v[t + 2] * cs.w + v[t + 3] * cs.z;
+                v[t] = a0;
+                v[t + 1] = b0;
+                v[t + 2] = a1;
+                v[t + 3] = b1;
             }
-        } else {
-#pragma unroll
-            for (int t = 0; t < 32; ++t)
-                if (t < lim) o[t] = (ep.mode == EPI_RESID_F32) ? o[t] + v[t] : v[t];
         }
-    }
-}
-
-// Residual epilogue of 32 consecutive features n0..n0+31 of token row m with
-// the next RMSNorm's producer side (NormIO): x += acc, y = x * w_next in the
-// 16-bit type; returns this chunk's sum of x^2.
-template <typename E>
-__device__ __forceinline__ float epi_chunk_resid_norm(const Epi& ep, const NormIO& nio, int m, int n0,
-                                                      const float (&v)[32]) {
-    float4* o4 = reinterpret_cast<float4*>(ep.out + static_cast<long long>(m) * ep.ldo + n0);
-    const float4* w4 = reinterpret_cast<const float4*>(nio.w_next + n0);
-    uint4* y4 = reinterpret_cast<uint4*>(static_cast<E*>(nio.y_out) + static_cast<long long>(m) * ep.ldo + n0);
-    float4 p[8];
+        uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) p[q] = o4[q];
-    float sq = 0.f;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        p[q] = make_float4(p[q].x + v[4 * q], p[q].y + v[4 * q + 1], p[q].z + v[4 * q + 2], p[q].w + v[4 * q + 3]);
-        o4[q] = p[q];
-        sq += p[q].x * p[q].x + p[q].y * p[q].y + p[q].z * p[q].z + p[q].w * p[q].w;
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float4 wa = w4[2 * q], wb = w4[2 * q + 1];
-        uint4 u;
-        u.x = pack2<E>(p[2 * q].x * wa.x, p[2 * q].y * wa.y);
-        u.y = pack2<E>(p[2 * q].z * wa.z, p[2 * q].w * wa.w);
-        u.z = pack2<E>(p[2 * q + 1].x * wb.x, p[2 * q + 1].y * wb.y);
-        u.w = pack2<E>(p[2 * q + 1].z * wb.z, p[2 * q + 1].w * wb.w);
-        y4[q] = u;
-    }
-    return sq;
-}
-
-// The whole epilogue of 32 features of row m: the consumer side of a fused
-// RMSNorm (scale by rs), then the producer side or the plain epilogue.
-// `sq` accumulates the sums of x^2, written per 128 features when the
-// chunk closes a 128-feature block (or the row's last block).
-template <typename E>
-__device__ __forceinline__ void epi_any(const Epi& ep, const NormIO& nio, int m, int n0, int rowsB, float rs,
-                                        float (&v)[32], float& sq) {
-    if (nio.ssq_in) {
-#pragma unroll
-        for (int t = 0; t < 32; ++t) v[t] *= rs;
-    }
-    if (!nio.ssq_out) {
-        epi_chunk<E>(ep, m, n0, rowsB, v);
+        for (int q = 0; q < 4; ++q) {
+            uint4 u;
+            u.x = pack2<E>(v[8 * q + 0], v[8 * q + 1]);
+            u.y = pack2<E>(v[8 * q + 2], v[8 * q + 3]);
+            u.z = pack2<E>(v[8 * q + 4], v[8 * q + 5]);
+            u.w = pack2<E>(v[8 * q + 6], v[8 * q + 7]);
+            d4[q] = u;
+        }
         return;
     }
-    if (n0 >= rowsB) return;
-    sq += epi_chunk_resid_norm<E>(ep, nio, m, n0, v);
-    if (((n0 + 32) & 127) == 0 || n0 + 32 >= rowsB) {
-        nio.ssq_out[static_cast<long long>(m) * ((rowsB + 127) / 128) + n0 / 128] = sq;
-        sq = 0.f;
+    // fp32 outputs: staged
+#pragma unroll
+    for (int qq = 0; qq < 8; ++qq)
+        stg[lane * 8 + (qq ^ sw)] = make_float4(v[4 * qq], v[4 * qq + 1], v[4 * qq + 2], v[4 * qq + 3]);
+    __syncwarp();
+    const int f = lane & 7;
+    const int n = n0 + 4 * f;
+    if (nio.ssq_out) {
+        // x += acc; y = x * w_next in E (rowsB % 128 == 0, ldo == rowsB); x
+        // back into the staging slots, then lane = row again for its sum of x^2
+        const float4 w = *reinterpret_cast<const float4*>(nio.w_next + n);
+        float4 p[8];
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+            const int m = m0 + it * 4 + (lane >> 3);
+            p[it] = m < rowsA ? *reinterpret_cast<const float4*>(ep.out + static_cast<long long>(m) * ep.ldo + n)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+            const int rr = it * 4 + (lane >> 3);
+            const int m = m0 + rr;
+            float4& slot = stg[rr * 8 + (f ^ (rr & 7))];
+            const float4 x = slot;
+            const float4 o = make_float4(p[it].x + x.x, p[it].y + x.y, p[it].z + x.z, p[it].w + x.w);
+            slot = o;
+            if (m < rowsA) {
+                *reinterpret_cast<float4*>(ep.out + static_cast<long long>(m) * ep.ldo + n) = o;
+                uint2 u;
+                u.x = pack2<E>(o.x * w.x, o.y * w.y);
+                u.y = pack2<E>(o.z * w.z, o.w * w.w);
+                *reinterpret_cast<uint2*>(static_cast<E*>(nio.y_out) + static_cast<long long>(m) * ep.ldo + n) = u;
+            }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int qq = 0; qq < 8; ++qq) {
+            const float4 o = stg[lane * 8 + (qq ^ sw)];
+            sq += o.x * o.x + o.y * o.y + o.z * o.z + o.w * o.w;
+        }
+        if (((n0 + 32) & 127) == 0 || n0 + 32 >= rowsB) {
+            const int m = m0 + lane;
+            if (m < rowsA) nio.ssq_out[static_cast<long long>(m) * ((rowsB + 127) / 128) + n0 / 128] = sq;
+            sq = 0.f;
+        }
+    } else {
+        // fp32 store, or residual add (x += acc)
+        const bool resid = ep.mode == EPI_RESID_F32;
+        const bool vec = n + 4 <= rowsB && (ep.ldo % 4) == 0;
+        float4 p[8];
+        if (resid) {
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+                const int m = m0 + it * 4 + (lane >> 3);
+                p[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (m < rowsA && vec) p[it] = *reinterpret_cast<const float4*>(ep.out + static_cast<long long>(m) * ep.ldo + n);
+            }
+        }
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+            const int rr = it * 4 + (lane >> 3);
+            const int m = m0 + rr;
+            float4 x = stg[rr * 8 + (f ^ (rr & 7))];
+            float* o = ep.out + static_cast<long long>(m) * ep.ldo + n;
+            if (m < rowsA && vec) {
+                if (resid) x = make_float4(p[it].x + x.x, p[it].y + x.y, p[it].z + x.z, p[it].w + x.w);
+                *reinterpret_cast<float4*>(o) = x;
+            } else if (m < rowsA) {
+                if (n < rowsB) o[0] = resid ? o[0] + x.x : x.x;
+                if (n + 1 < rowsB) o[1] = resid ? o[1] + x.y : x.y;
+                if (n + 2 < rowsB) o[2] = resid ? o[2] + x.z : x.z;
+                if (n + 3 < rowsB) o[3] = resid ? o[3] + x.w : x.w;
+            }
+        }
     }
+    __syncwarp();
 }
 
 }  // namespace
@@ -202,7 +233,8 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
                   NormIO nio) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStagesTc * kStageBytes);
+    float4* stg_all = reinterpret_cast<float4*>(smem + kStagesTc * kStageBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStagesTc * kStageBytes + kStgBytes);
     uint64_t* empty = full + kStagesTc;
     uint64_t* tfull = empty + kStagesTc;   // [2]
     uint64_t* tempty = tfull + 2;          // [2]
@@ -289,6 +321,7 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
         const int r = q * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const int epi_tid = threadIdx.x - 64;
+        float4* stg = stg_all + (warp - 2) * 256;   // this warp's 32 x 32 fp32 staging block
         const int c_lo = ((warp - 2) >> 2) * 4;   // warps 2-5: 32-column chunks 0-3, warps 6-9: chunks 4-7
         const int Wsk = plan.sk * KT;
         const int Psk = plan.psk;
@@ -318,70 +351,68 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
                 ss = row_ssq(nio.ssq_in + static_cast<long long>(m) * nio.n_in, nio.n_in);
                 rs = rsqrtf(ss / static_cast<float>(KT * 64) + nio.eps);
             }
-            if (it.ks == 0 && it.ke == KT) {
-                // whole tile: TMEM -> epilogue, 32 features at a time
+            // a split tile: publish this CTA's partial (feature-major, coalesced
+            // over rows); only the last contributor to arrive goes on
+            const bool whole = it.ks == 0 && it.ke == KT;
+            const int tl = it.tile - plan.dp;
+            const int ub = tl * KT;
+            const int cf = whole ? c : owner(ub, Wsk, Psk), cl = whole ? c : owner(ub + KT - 1, Wsk, Psk);
+            if (!whole) {
+                const int slot = (ub + it.ks == u0) ? 0 : 1;   // the run's first segment, or its last
+                float* my = part + (static_cast<long long>(c) * 2 + slot) * kPartFloats + r;
 #pragma unroll 1
                 for (int cc = c_lo; cc < c_lo + 4; ++cc) {
                     float v[32];
                     tmem_ld_32x32b_x32(tb + cc * 32, v);
                     tc_wait_ld();
-                    if (row_ok) epi_any<E>(ep, nio, m, nbase + cc * 32, rowsB, rs, v, sq);
+#pragma unroll
+                    for (int t = 0; t < 32; ++t) my[(cc * 32 + t) * 128] = v[t];
                 }
-                tc_fence_before();
-                mbar_arrive(&tempty[acc]);
-                continue;
+                __threadfence();
+                named_sync(1, kEpiThreads);
+                if (epi_tid == 0) flag[1] = atomicAdd(&counters[tl], 1);
+                named_sync(1, kEpiThreads);
+                if (flag[1] != cl - cf) {   // not the last contributor
+                    tc_fence_before();
+                    mbar_arrive(&tempty[acc]);
+                    continue;
+                }
+                __threadfence();
             }
-            // split tile: publish this CTA's partial (feature-major, coalesced over rows)
-            const int tl = it.tile - plan.dp;
-            const int ub = tl * KT;
-            const int cf = owner(ub, Wsk, Psk), cl = owner(ub + KT - 1, Wsk, Psk);
-            const int slot = (ub + it.ks == u0) ? 0 : 1;   // the run's first segment, or its last
-            float* my = part + (static_cast<long long>(c) * 2 + slot) * kPartFloats + r;
+            // TMEM (summed with the other contributors' partials in CTA order)
+            // -> epilogue, 32 features at a time
 #pragma unroll 1
             for (int cc = c_lo; cc < c_lo + 4; ++cc) {
                 float v[32];
                 tmem_ld_32x32b_x32(tb + cc * 32, v);
                 tc_wait_ld();
+                if (!whole) {
+                    float own[32];
 #pragma unroll
-                for (int t = 0; t < 32; ++t) my[(cc * 32 + t) * 128] = v[t];
-            }
-            __threadfence();
-            named_sync(1, kEpiThreads);
-            if (epi_tid == 0) flag[1] = atomicAdd(&counters[tl], 1);
-            named_sync(1, kEpiThreads);
-            if (flag[1] != cl - cf) {   // not the last contributor
-                tc_fence_before();
-                mbar_arrive(&tempty[acc]);
-                continue;
-            }
-            __threadfence();
-            // last contributor: sum the partials in CTA order, then the epilogue
-#pragma unroll 1
-            for (int cc = c_lo; cc < c_lo + 4; ++cc) {
-                float own[32], v[32];
-                tmem_ld_32x32b_x32(tb + cc * 32, own);
-                tc_wait_ld();
+                    for (int t = 0; t < 32; ++t) {
+                        own[t] = v[t];
+                        v[t] = 0.f;
+                    }
+                    for (int cb = cf; cb <= cl; ++cb) {
+                        if (cb == c) {
 #pragma unroll
-                for (int t = 0; t < 32; ++t) v[t] = 0.f;
-                for (int cb = cf; cb <= cl; ++cb) {
-                    if (cb == c) {
+                            for (int t = 0; t < 32; ++t) v[t] += own[t];
+                        } else {
+                            const int sl = run_begin(cb, Wsk, Psk) >= ub ? 0 : 1;
+                            const float* pp = part + (static_cast<long long>(cb) * 2 + sl) * kPartFloats + r;
+                            float f[32];
 #pragma unroll
-                        for (int t = 0; t < 32; ++t) v[t] += own[t];
-                    } else {
-                        const int sl = run_begin(cb, Wsk, Psk) >= ub ? 0 : 1;
-                        const float* pp = part + (static_cast<long long>(cb) * 2 + sl) * kPartFloats + r;
-                        float f[32];
+                            for (int t = 0; t < 32; ++t) f[t] = pp[(cc * 32 + t) * 128];
 #pragma unroll
-                        for (int t = 0; t < 32; ++t) f[t] = pp[(cc * 32 + t) * 128];
-#pragma unroll
-                        for (int t = 0; t < 32; ++t) v[t] += f[t];
+                            for (int t = 0; t < 32; ++t) v[t] += f[t];
+                        }
                     }
                 }
-                if (row_ok) epi_any<E>(ep, nio, m, nbase + cc * 32, rowsB, rs, v, sq);
+                epi_block<E>(ep, nio, m - lane, nbase + cc * 32, rowsA, rowsB, rs, v, stg, lane, sq);
             }
             tc_fence_before();
             mbar_arrive(&tempty[acc]);
-            if (epi_tid == 0) counters[tl] = 0;
+            if (!whole && epi_tid == 0) counters[tl] = 0;
         }
     }
 
@@ -437,7 +468,8 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
                        int* __restrict__ counters, NormIO nio) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStagesPair * kPairStageBytes);
+    float4* stg_all = reinterpret_cast<float4*>(smem + kStagesPair * kPairStageBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStagesPair * kPairStageBytes + kStgBytes);
     uint64_t* empty = full + kStagesPair;
     uint64_t* tfull = empty + kStagesPair;   // [2]
     uint64_t* tempty = tfull + 2;            // [2]
@@ -539,6 +571,7 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
         const int r = q * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         const int epi_tid = threadIdx.x - 64;
+        float4* stg = stg_all + (warp - 2) * 256;   // this warp's 32 x 32 fp32 staging block
         const int c_lo = ((warp - 2) >> 2) * 4;   // warps 2-5: 32-column chunks 0-3, warps 6-9: chunks 4-7
         const int Wsk = plan.sk * KT;
         const int Psk = plan.psk;
@@ -574,68 +607,67 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
                 ss = row_ssq(nio.ssq_in + static_cast<long long>(m) * nio.n_in, nio.n_in);
                 rs = rsqrtf(ss / static_cast<float>(KT * 64) + nio.eps);
             }
-            if (it.ks == 0 && it.ke == KT) {
+            // a split tile: this CTA's half of it, reduced among the same halves
+            // of the tile's other pairs (last arrival finishes, in pair order)
+            const bool whole = it.ks == 0 && it.ke == KT;
+            const int tl = it.tile - plan.dp;
+            const int ub = tl * KT;
+            const int cf = whole ? c : owner(ub, Wsk, Psk), cl = whole ? c : owner(ub + KT - 1, Wsk, Psk);
+            const int cnt_idx = 2 * tl + static_cast<int>(rank);
+            if (!whole) {
+                const int slot = (ub + it.ks == u0) ? 0 : 1;
+                float* my =
+                    part + (static_cast<long long>(2 * c + static_cast<int>(rank)) * 2 + slot) * kPartFloats + r;
 #pragma unroll 1
                 for (int cc = c_lo; cc < c_lo + 4; ++cc) {
                     float v[32];
                     tmem_ld_32x32b_x32(tb + cc * 32, v);
                     tc_wait_ld();
-                    if (row_ok) epi_any<E>(ep, nio, m, nbase + cc * 32, rowsB, rs, v, sq);
+#pragma unroll
+                    for (int t = 0; t < 32; ++t) my[(cc * 32 + t) * 128] = v[t];
                 }
-                release(acc);
-                continue;
+                __threadfence();
+                named_sync(1, kEpiThreads);
+                if (epi_tid == 0) flag[1] = atomicAdd(&counters[cnt_idx], 1);
+                named_sync(1, kEpiThreads);
+                if (flag[1] != cl - cf) {
+                    release(acc);
+                    continue;
+                }
+                __threadfence();
             }
-            // split tile: this CTA's half of it, reduced among the same halves
-            // of the tile's other pairs (last arrival finishes, in pair order)
-            const int tl = it.tile - plan.dp;
-            const int ub = tl * KT;
-            const int cf = owner(ub, Wsk, Psk), cl = owner(ub + KT - 1, Wsk, Psk);
-            const int slot = (ub + it.ks == u0) ? 0 : 1;
-            const int cnt_idx = 2 * tl + static_cast<int>(rank);
-            float* my = part + (static_cast<long long>(2 * c + static_cast<int>(rank)) * 2 + slot) * kPartFloats + r;
 #pragma unroll 1
             for (int cc = c_lo; cc < c_lo + 4; ++cc) {
                 float v[32];
                 tmem_ld_32x32b_x32(tb + cc * 32, v);
                 tc_wait_ld();
+                if (!whole) {
+                    float own[32];
 #pragma unroll
-                for (int t = 0; t < 32; ++t) my[(cc * 32 + t) * 128] = v[t];
-            }
-            __threadfence();
-            named_sync(1, kEpiThreads);
-            if (epi_tid == 0) flag[1] = atomicAdd(&counters[cnt_idx], 1);
-            named_sync(1, kEpiThreads);
-            if (flag[1] != cl - cf) {
-                release(acc);
-                continue;
-            }
-            __threadfence();
-#pragma unroll 1
-            for (int cc = c_lo; cc < c_lo + 4; ++cc) {
-                float own[32], v[32];
-                tmem_ld_32x32b_x32(tb + cc * 32, own);
-                tc_wait_ld();
+                    for (int t = 0; t < 32; ++t) {
+                        own[t] = v[t];
+                        v[t] = 0.f;
+                    }
+                    for (int cb = cf; cb <= cl; ++cb) {
+                        if (cb == c) {
 #pragma unroll
-                for (int t = 0; t < 32; ++t) v[t] = 0.f;
-                for (int cb = cf; cb <= cl; ++cb) {
-                    if (cb == c) {
+                            for (int t = 0; t < 32; ++t) v[t] += own[t];
+                        } else {
+                            const int sl = run_begin(cb, Wsk, Psk) >= ub ? 0 : 1;
+                            const float* pp = part +
+                                (static_cast<long long>(2 * cb + static_cast<int>(rank)) * 2 + sl) * kPartFloats + r;
+                            float f[32];
 #pragma unroll
-                        for (int t = 0; t < 32; ++t) v[t] += own[t];
-                    } else {
-                        const int sl = run_begin(cb, Wsk, Psk) >= ub ? 0 : 1;
-                        const float* pp =
-                            part + (static_cast<long long>(2 * cb + static_cast<int>(rank)) * 2 + sl) * kPartFloats + r;
-                        float f[32];
+                            for (int t = 0; t < 32; ++t) f[t] = pp[(cc * 32 + t) * 128];
 #pragma unroll
-                        for (int t = 0; t < 32; ++t) f[t] = pp[(cc * 32 + t) * 128];
-#pragma unroll
-                        for (int t = 0; t < 32; ++t) v[t] += f[t];
+                            for (int t = 0; t < 32; ++t) v[t] += f[t];
+                        }
                     }
                 }
-                if (row_ok) epi_any<E>(ep, nio, m, nbase + cc * 32, rowsB, rs, v, sq);
+                epi_block<E>(ep, nio, m - lane, nbase + cc * 32, rowsA, rowsB, rs, v, stg, lane, sq);
             }
             release(acc);
-            if (epi_tid == 0) counters[cnt_idx] = 0;
+            if (!whole && epi_tid == 0) counters[cnt_idx] = 0;
         }
     }
 
@@ -706,7 +738,7 @@ template <typename E>
 static int launch_tcp(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
                       int* counters, cudaStream_t st, const NormIO& nio) {
     if (M <= 0 || N <= 0) return LLAMA_OK;
-    constexpr int smem = 1024 + kStagesTc * kStageBytes + (2 * kStagesTc + 5) * 8 + 16;
+    constexpr int smem = 1024 + kStagesTc * kStageBytes + kStgBytes + (2 * kStagesTc + 5) * 8 + 16;
     static_assert(smem <= 227 * 1024, "shared memory per CTA");
     static bool attr_set = false;
     if (!attr_set) {
@@ -748,7 +780,7 @@ constexpr long long kPairMinWeights = 4096LL * 4096;
 template <typename E>
 static int launch_tcp_pair(const TmaMaps* mapA, const TmaMaps* mapW, int M, int N, int K, const Epi& ep, float* part,
                            int* counters, cudaStream_t st, const NormIO& nio) {
-    constexpr int smem = 1024 + kStagesPair * kPairStageBytes + (2 * kStagesPair + 5) * 8 + 16;
+    constexpr int smem = 1024 + kStagesPair * kPairStageBytes + kStgBytes + (2 * kStagesPair + 5) * 8 + 16;
     static_assert(smem <= 227 * 1024, "shared memory per CTA");
     auto kern = linear_tcp_pair_kernel<E>;
     static int pairs = 0;   // clusters of two that are resident at once
