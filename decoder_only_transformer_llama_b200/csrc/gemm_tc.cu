@@ -17,10 +17,12 @@
 // item: the CTAs of a wave walk K in step, so the A and B tiles in flight at
 // any moment share a few MB of L2.  The `sk` tiles of a partial last wave form
 // one flat run of sk * K/64 k-tile units cut into psk equal contiguous runs
-// (stream-K, at most 4 runs per tile), so the SMs end together.  A tile split
-// between CTAs is finished by the contributor that arrives last at the tile's
-// counter: it adds the fp32 partials in CTA order (deterministic) and applies
-// the epilogue; no CTA ever waits for another.
+// (stream-K, at most 4 runs per tile), so the SMs end together; each CTA
+// takes its stream-K run before its whole tiles.  A tile split between CTAs
+// is finished by the contributor that arrives last at the tile's counter: it
+// adds the fp32 partials in CTA order (deterministic) and applies the
+// epilogue while its MMAs go on with the whole tiles; no CTA ever waits for
+// another.
 //
 // Warp roles (320 threads):
 //   warp 0 lane 0  TMA producer (4-deep ring of 128x64 A + 256x64 B tiles)

@@ -12,8 +12,10 @@ namespace llb {
 
 constexpr int kGroupM = 16;   // M-tiles per rasterisation group
 
-// Work list of one CTA: whole tiles c, c+P, ... below dp, then (c < psk) its
-// stream-K run over the last sk tiles.
+// Work list of one CTA: (c < psk) its stream-K run over the last sk tiles
+// first, then whole tiles c, c+P, ... below dp.  Split tiles come first so
+// that their fixups (partials published, the last arrival adding them up)
+// overlap the MMAs of the CTA's whole tiles instead of ending the launch.
 struct TcPlan {
     int TM, TN, KT;
     int dp, sk, psk;
@@ -35,6 +37,14 @@ __host__ __device__ __forceinline__ WorkIt work_begin(const TcPlan& p, int c, in
 }
 
 __host__ __device__ __forceinline__ bool work_next(WorkIt& w, const TcPlan& p, int P, Item& it) {
+    if (w.u < w.u1) {
+        const int tl = w.u / p.KT;
+        it.tile = p.dp + tl;
+        it.ks = w.u - tl * p.KT;
+        it.ke = p.KT < it.ks + (w.u1 - w.u) ? p.KT : it.ks + (w.u1 - w.u);
+        w.u += it.ke - it.ks;
+        return true;
+    }
     if (w.next_dp < p.dp) {
         it.tile = w.next_dp;
         it.ks = 0;
@@ -42,13 +52,7 @@ __host__ __device__ __forceinline__ bool work_next(WorkIt& w, const TcPlan& p, i
         w.next_dp += P;
         return true;
     }
-    if (w.u >= w.u1) return false;
-    const int tl = w.u / p.KT;
-    it.tile = p.dp + tl;
-    it.ks = w.u - tl * p.KT;
-    it.ke = p.KT < it.ks + (w.u1 - w.u) ? p.KT : it.ks + (w.u1 - w.u);
-    w.u += it.ke - it.ks;
-    return true;
+    return false;
 }
 
 // Tile t -> (M-tile, N-tile): groups of kGroupM M-tiles, N-major inside a group.
