@@ -55,6 +55,22 @@ constexpr int kStageBytes = kA_BYTES + kB_BYTES;
 constexpr int kPartFloats = 128 * kBN;       // one fp32 partial tile
 constexpr int kStgBytes = (kEpiThreads / 32) * 32 * 32 * 4;   // epilogue staging: 32 x 32 fp32 per warp
 
+// A tile's epilogue inputs that do not depend on its accumulator, taken
+// while its MMAs run: 1/rms of token row m (the consumer side of a fused
+// RMSNorm over K features, from the row's per-128-feature sums of squares)
+// and, for a residual epilogue, the 128 residual features n0.. of row m that
+// this warp will add into, pulled into L2.
+__device__ __forceinline__ void epi_tile_inputs(const Epi& ep, const NormIO& nio, int m, bool row_ok, int n0, int rowsB,
+                                                int K, float& rs) {
+    if (!row_ok) return;
+    if (nio.ssq_in) rs = rsqrtf(row_ssq(nio.ssq_in + static_cast<long long>(m) * nio.n_in, nio.n_in) /
+                                    static_cast<float>(K) + nio.eps);
+    if (ep.mode == EPI_RESID_F32 && n0 < rowsB && (ep.ldo % 4) == 0) {
+        const int nf = rowsB - n0 < 128 ? rowsB - n0 : 128;
+        bulk_prefetch_l2(ep.out + static_cast<long long>(m) * ep.ldo + n0, static_cast<uint32_t>((nf * 4 + 15) & ~15));
+    }
+}
+
 // Epilogue of one 32 x 32 block of a tile: token rows m0..m0+31 (one warp's
 // TMEM lane quarter; lane = row as tcgen05.ld delivers it) x output features
 // n0..n0+31, after the consumer side of a fused RMSNorm (scale by the row's
@@ -333,6 +349,14 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
         int j = 0;
         while (work_next(w, plan, P, it)) {
             const int acc = j & 1;
+            int tm, tn;
+            tile_coords(it.tile, plan, tm, tn);
+            const int m = tm * 128 + r;
+            const bool row_ok = m < rowsA;
+            const uint32_t tb = tmem + lane_base + acc * kBN;
+            const int nbase = tn * kBN;
+            float rs = 1.f, sq = 0.f;
+            epi_tile_inputs(ep, nio, m, row_ok, nbase + c_lo * 32, rowsB, KT * 64, rs);
             const bool ok_wait = mbar_wait(&tfull[acc], (j >> 1) & 1, wlim);
             tc_fence_after();
             if (named_any(1, kEpiThreads, !ok_wait || *reinterpret_cast<volatile int*>(&flag[0]) != 0)) {
@@ -340,19 +364,6 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
                 break;
             }
             ++j;
-            int tm, tn;
-            tile_coords(it.tile, plan, tm, tn);
-            const int m = tm * 128 + r;
-            const bool row_ok = m < rowsA;
-            const uint32_t tb = tmem + lane_base + acc * kBN;
-            const int nbase = tn * kBN;
-            // fused RMSNorm, consumer side: 1/rms of row m from its sums of squares
-            float rs = 1.f, sq = 0.f;
-            if (nio.ssq_in && row_ok) {
-                float ss = 0.f;
-                ss = row_ssq(nio.ssq_in + static_cast<long long>(m) * nio.n_in, nio.n_in);
-                rs = rsqrtf(ss / static_cast<float>(KT * 64) + nio.eps);
-            }
             // a split tile: publish this CTA's partial (feature-major, coalesced
             // over rows); only the last contributor to arrive goes on
             const bool whole = it.ks == 0 && it.ke == KT;
@@ -590,13 +601,6 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
         };
         while (work_next(w, plan, P, it)) {
             const int acc = j & 1;
-            const bool ok_wait = mbar_wait(&tfull[acc], (j >> 1) & 1, wlim);
-            tc_fence_after();
-            if (named_any(1, kEpiThreads, !ok_wait || *reinterpret_cast<volatile int*>(&flag[0]) != 0)) {
-                if (epi_tid == 0) report_status(ep.status, LLAMA_ERR_DEVICE_TIMEOUT);
-                break;
-            }
-            ++j;
             int tm, tn;
             tile_coords(it.tile, plan, tm, tn);
             const int m = tm * kPairTile + static_cast<int>(rank) * 128 + r;
@@ -604,11 +608,14 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
             const uint32_t tb = tmem + lane_base + acc * kPairTile;
             const int nbase = tn * kPairTile;
             float rs = 1.f, sq = 0.f;
-            if (nio.ssq_in && row_ok) {
-                float ss = 0.f;
-                ss = row_ssq(nio.ssq_in + static_cast<long long>(m) * nio.n_in, nio.n_in);
-                rs = rsqrtf(ss / static_cast<float>(KT * 64) + nio.eps);
+            epi_tile_inputs(ep, nio, m, row_ok, nbase + c_lo * 32, rowsB, KT * 64, rs);
+            const bool ok_wait = mbar_wait(&tfull[acc], (j >> 1) & 1, wlim);
+            tc_fence_after();
+            if (named_any(1, kEpiThreads, !ok_wait || *reinterpret_cast<volatile int*>(&flag[0]) != 0)) {
+                if (epi_tid == 0) report_status(ep.status, LLAMA_ERR_DEVICE_TIMEOUT);
+                break;
             }
+            ++j;
             // a split tile: this CTA's half of it, reduced among the same halves
             // of the tile's other pairs (last arrival finishes, in pair order)
             const bool whole = it.ks == 0 && it.ke == KT;
