@@ -99,7 +99,7 @@ __device__ __forceinline__ void epi_block(const Epi& ep, const NormIO& nio, int 
         if (mrow >= rowsA) return;
         float g16[16];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) g16[t] = silu_f(v[t]) * v[16 + t];
+        for (int t = 0; t < 16; ++t) g16[t] = __fdividef(v[t], 1.f + __expf(-v[t])) * v[16 + t];
         uint4* d4 = reinterpret_cast<uint4*>(static_cast<E*>(ep.g) + static_cast<long long>(mrow) * ep.H + (n0 / 32) * 16);
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
