@@ -171,7 +171,8 @@ __device__ void digit_histogram(TopPShared& sh, const float* row, int V, bool fr
 // the first digit whose inclusive prefix mass, after `before`, exceeds
 // `target` (or the last non-empty digit if none does).  Writes the extended
 // prefix, the mass before the chosen digit and its key count to sh.sel_*.
-__device__ void choose_digit(TopPShared& sh, const unsigned long long* tm, const unsigned int* tc, uint64_t prefix,
+template <typename SH>
+__device__ void choose_digit(SH& sh, const unsigned long long* tm, const unsigned int* tc, uint64_t prefix,
                              int shift, unsigned long long before, unsigned long long target) {
     const int lane = threadIdx.x & 31;
     unsigned long long part = 0;
@@ -347,6 +348,242 @@ top_p_kernel(const float* __restrict__ logits, int V, float temperature, float t
     }
 }
 
+// ---------------------------------------------------------------- top-p on a cluster per row
+// The selection of top_p_kernel (same keys, masses, targets and digit rule,
+// so the same picks) with each row spread over a cluster of kTpRanks CTAs.
+// CTA r owns the contiguous slice [r*S, min(V, (r+1)*S)), S = ceil(V /
+// kTpRanks), and keeps its slice's ordered logit bits and fixed-point masses
+// in shared memory, so each fp64 exponential is taken once.  Every digit
+// histogram is built per CTA and summed over the cluster through distributed
+// shared memory; the CTAs then take identical decisions from identical
+// integer totals.  Once a digit prefix holds a single key, the CTA that owns
+// it publishes the key and the select ends.  Exchanges alternate between two
+// buffers, so one cluster barrier per exchange orders every write before the
+// reads of the same round and after the reads of two rounds before.
+constexpr int kTpRanks = 8;
+constexpr int kTpThreads = 512;
+constexpr int kTpWarps = kTpThreads / 32;
+constexpr int kTpSub = 4;   // shared-memory sub-histograms (warp w adds into sub[w % kTpSub])
+
+struct TpHist {
+    unsigned long long mass[256];
+    unsigned int cnt[256];
+};
+struct TpClShared {
+    TpHist xh[2];                   // this CTA's digit histogram, read by the cluster
+    TpHist sub[kTpSub];
+    TpHist tot;                     // cluster totals of the current digit
+    TpHist p1;                      // cluster totals of the first digit (both selects start from it)
+    unsigned long long xkey[2];     // a key this CTA publishes (0: none; no key is 0)
+    unsigned long long sel_prefix, sel_before;
+    unsigned int sel_cnt;
+    float xmax;                     // this CTA's slice maximum, read by the cluster
+    float red_f[kTpWarps];
+};
+// Behind the struct: uint32_t ob[S] (ordered logit bits), then, 8-byte
+// aligned, unsigned long long mass[S].
+constexpr size_t kTpFixedBytes = (sizeof(TpClShared) + 15) & ~size_t(15);
+
+__device__ __forceinline__ unsigned long long ld_cluster_u64(uint32_t a) {
+    unsigned long long v;
+    asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ unsigned int ld_cluster_u32(uint32_t a) {
+    unsigned int v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t a) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+    return v;
+}
+
+// This CTA's histogram of digit (key >> shift) & 255 over its slice's keys
+// that match `prefix` under `mask`, into sh.xh[k].
+__device__ void tp_local_hist(TpClShared& sh, const uint32_t* ob, const unsigned long long* mass, int n, int lo,
+                              uint64_t prefix, uint64_t mask, int shift, int k) {
+    for (int i = threadIdx.x; i < kTpSub * 256; i += blockDim.x) {
+        sh.sub[i >> 8].mass[i & 255] = 0ull;
+        sh.sub[i >> 8].cnt[i & 255] = 0u;
+    }
+    __syncthreads();
+    TpHist& h = sh.sub[(threadIdx.x >> 5) % kTpSub];
+    for (int j = threadIdx.x; j < n; j += blockDim.x) {
+        const uint64_t key = (static_cast<uint64_t>(ob[j]) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(lo + j));
+        if ((key & mask) == prefix) {
+            const int bin = static_cast<int>((key >> shift) & 255u);
+            atomicAdd(&h.mass[bin], mass[j]);
+            atomicAdd(&h.cnt[bin], 1u);
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) {
+        unsigned long long m = 0;
+        unsigned int c = 0;
+#pragma unroll
+        for (int q = 0; q < kTpSub; ++q) {
+            m += sh.sub[q].mass[i];
+            c += sh.sub[q].cnt[i];
+        }
+        sh.xh[k].mass[i] = m;
+        sh.xh[k].cnt[i] = c;
+    }
+}
+
+// sh.tot = the sum over the cluster's CTAs of their sh.xh[k].
+__device__ void tp_reduce(TpClShared& sh, int k) {
+    cluster_sync();
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) {
+        unsigned long long m = 0;
+        unsigned int c = 0;
+#pragma unroll
+        for (uint32_t r = 0; r < kTpRanks; ++r) {
+            m += ld_cluster_u64(cluster_addr(&sh.xh[k].mass[i], r));
+            c += ld_cluster_u32(cluster_addr(&sh.xh[k].cnt[i], r));
+        }
+        sh.tot.mass[i] = m;
+        sh.tot.cnt[i] = c;
+    }
+    __syncthreads();
+}
+
+// First key in descending order whose inclusive prefix mass exceeds
+// `target` (or the smallest key if none does), from the first-digit totals
+// sh.p1; *before_out = the mass of the keys strictly before it.  `k` is the
+// exchange buffer of the next round (advanced here).
+__device__ uint64_t tp_select(TpClShared& sh, const uint32_t* ob, const unsigned long long* mass, int n, int lo,
+                              unsigned long long target, int& k, unsigned long long* before_out) {
+    const int warp = threadIdx.x >> 5;
+    if (warp == 0) choose_digit(sh, sh.p1.mass, sh.p1.cnt, 0, 56, 0, target);
+    __syncthreads();
+    uint64_t prefix = sh.sel_prefix, mask = static_cast<uint64_t>(255) << 56;
+    unsigned long long before = sh.sel_before;
+    unsigned int cnt = sh.sel_cnt;
+    __syncthreads();
+    for (int pass = 1; pass < 8 && cnt > 1; ++pass) {
+        const int shift = 56 - 8 * pass;
+        tp_local_hist(sh, ob, mass, n, lo, prefix, mask, shift, k);
+        tp_reduce(sh, k);
+        k ^= 1;
+        if (warp == 0) choose_digit(sh, sh.tot.mass, sh.tot.cnt, prefix, shift, before, target);
+        __syncthreads();
+        prefix = sh.sel_prefix;
+        before = sh.sel_before;
+        cnt = sh.sel_cnt;
+        mask |= static_cast<uint64_t>(255) << shift;
+        __syncthreads();
+    }
+    if (mask != ~0ull) {
+        // one key under `prefix`: the CTA that owns it publishes it
+        if (threadIdx.x == 0) sh.xkey[k] = 0ull;
+        __syncthreads();
+        for (int j = threadIdx.x; j < n; j += blockDim.x) {
+            const uint64_t key =
+                (static_cast<uint64_t>(ob[j]) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(lo + j));
+            if ((key & mask) == prefix) sh.xkey[k] = key;
+        }
+        cluster_sync();
+        uint64_t key = 0;
+#pragma unroll
+        for (uint32_t r = 0; r < kTpRanks; ++r) key |= ld_cluster_u64(cluster_addr(&sh.xkey[k], r));
+        k ^= 1;
+        prefix = key;
+    }
+    *before_out = before;
+    return prefix;
+}
+
+__global__ void __cluster_dims__(kTpRanks, 1, 1) __launch_bounds__(kTpThreads, 1)
+top_p_cluster_kernel(const float* __restrict__ logits, int V, float temperature, float top_p,
+                     const float* __restrict__ uniforms, int32_t* out, int32_t* tokens_adv, int32_t* pos_adv,
+                     unsigned long long* tl) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    TpClShared& sh = *reinterpret_cast<TpClShared*>(smem_raw);
+    pdl_trigger();
+    pdl_wait();
+    const int rank = static_cast<int>(cluster_rank());
+    const int b = blockIdx.x / kTpRanks;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float* row = logits + static_cast<long long>(b) * V;
+    const int S = (V + kTpRanks - 1) / kTpRanks;
+    const int lo = rank * S;
+    const int n = V - lo < S ? (V - lo > 0 ? V - lo : 0) : S;
+    uint32_t* ob = reinterpret_cast<uint32_t*>(smem_raw + kTpFixedBytes);
+    unsigned long long* mass =
+        reinterpret_cast<unsigned long long*>(smem_raw + kTpFixedBytes + ((static_cast<size_t>(S) * 4 + 7) & ~size_t(7)));
+
+    // row maximum: slice maxima, then the cluster's
+    float mx = -INFINITY;
+    for (int j = threadIdx.x; j < n; j += blockDim.x) mx = fmaxf(mx, row[lo + j]);
+    mx = warp_max(mx);
+    if (lane == 0) sh.red_f[warp] = mx;
+    __syncthreads();
+    if (warp == 0) {
+        float t = lane < kTpWarps ? sh.red_f[lane] : -INFINITY;
+        t = warp_max(t);
+        if (lane == 0) sh.xmax = t;
+    }
+    cluster_sync();
+    float lm = -INFINITY;
+#pragma unroll
+    for (uint32_t r = 0; r < kTpRanks; ++r) lm = fmaxf(lm, ld_cluster_f32(cluster_addr(&sh.xmax, r)));
+    const double lmax = static_cast<double>(lm);
+    const double inv_t = 1.0 / static_cast<double>(temperature);
+
+    // the slice's keys and masses, once; the first-digit histogram over the cluster
+    for (int j = threadIdx.x; j < n; j += blockDim.x) {
+        const float l = row[lo + j];
+        ob[j] = ordered_bits(l);
+        mass[j] = fixed_mass(l, lmax, inv_t);
+    }
+    __syncthreads();
+    int k = 0;
+    tp_local_hist(sh, ob, mass, n, lo, 0, 0, 56, k);
+    tp_reduce(sh, k);
+    k ^= 1;
+    unsigned long long S_mass = 0;
+    for (int i = 0; i < 256; ++i) S_mass += sh.tot.mass[i];
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) {
+        sh.p1.mass[i] = sh.tot.mass[i];
+        sh.p1.cnt[i] = sh.tot.cnt[i];
+    }
+    __syncthreads();
+
+    // nucleus edge: first key whose inclusive mass exceeds top_p * S
+    const double tp = static_cast<double>(top_p) * static_cast<double>(S_mass);
+    const unsigned long long t1 = tp >= 18446744073709549568.0 ? ~0ull : static_cast<unsigned long long>(tp);
+    unsigned long long before_edge;
+    const uint64_t edge = tp_select(sh, ob, mass, n, lo, t1, k, &before_edge);
+    const int edge_id = static_cast<int>(~static_cast<uint32_t>(edge & 0xffffffffu));
+    const unsigned long long Z = before_edge + fixed_mass(row[edge_id], lmax, inv_t);
+
+    // draw: first kept key whose inclusive mass exceeds u * Z
+    double u = static_cast<double>(uniforms[b]);
+    u = fmin(fmax(u, 0.0), 1.0);
+    const unsigned long long t2 = static_cast<unsigned long long>(u * static_cast<double>(Z));
+    unsigned long long before_draw;
+    const uint64_t drawn = tp_select(sh, ob, mass, n, lo, t2, k, &before_draw);
+    const uint64_t pick = drawn < edge ? edge : drawn;   // never past the nucleus edge
+    if (rank == 0 && threadIdx.x == 0) {
+        const int id = static_cast<int>(~static_cast<uint32_t>(pick & 0xffffffffu));
+        out[b] = id;
+        if (tokens_adv) tokens_adv[b] = id;
+        if (pos_adv) pos_adv[b] += 1;
+        tl_stamp(tl);
+    }
+    cluster_sync();   // no CTA leaves while the cluster may still read its shared memory
+}
+
+// Vocabularies whose slices fit (V up to about 137k) take the cluster kernel.
+constexpr size_t kTpClusterMaxSmem = 227 * 1024;
+// Bytes of dynamic shared memory the cluster kernel needs for a vocabulary of V.
+static size_t top_p_cluster_smem(int V) {
+    const size_t S = static_cast<size_t>((V + kTpRanks - 1) / kTpRanks);
+    return kTpFixedBytes + ((S * 4 + 7) & ~size_t(7)) + S * 8;
+}
+
 // ---------------------------------------------------------------- token log-probabilities
 // out[i] = log softmax(logits[i, :])[tok[i]] = l[tok] - (m + log sum_j exp(l_j - m)),
 // m = max_j l_j, the sum in fp64 (the log-probabilities that generate returns,
@@ -403,6 +640,22 @@ int launch_argmax(const float* logits, int B, int V, int32_t* out, int32_t* toke
 int launch_top_p(const float* logits, int B, int V, float temperature, float top_p, const float* uniforms,
                  int32_t* out, int32_t* tokens_adv, int32_t* pos_adv, cudaStream_t st, bool pdl,
                  unsigned long long* tl) {
+    const size_t csmem = top_p_cluster_smem(V);
+    if (csmem <= kTpClusterMaxSmem) {
+        static bool cattr = false;
+        if (!cattr) {
+            cudaError_t e = cudaFuncSetAttribute(top_p_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(kTpClusterMaxSmem));
+            if (e == cudaSuccess) e = carveout_max(top_p_cluster_kernel);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(top_p_cluster_kernel)");
+            cattr = true;
+        }
+        cudaError_t e = launch_k(top_p_cluster_kernel, dim3(B * kTpRanks), dim3(kTpThreads), csmem, st, pdl, logits, V,
+                                 temperature, top_p, uniforms, out, tokens_adv, pos_adv, tl);
+        count_launch();
+        if (e != cudaSuccess) return cuda_fail(e, "top_p_cluster_kernel");
+        return LLAMA_OK;
+    }
     const int smem = static_cast<int>(sizeof(TopPShared));
     static bool attr = false;
     if (!attr) {
