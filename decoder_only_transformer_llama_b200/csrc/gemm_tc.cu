@@ -357,12 +357,13 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
             const int nbase = tn * kBN;
             float rs = 1.f, sq = 0.f;
             epi_tile_inputs(ep, nio, m, row_ok, nbase + c_lo * 32, rowsB, KT * 64, rs);
-            const bool ok_wait = mbar_wait(&tfull[acc], (j >> 1) & 1, wlim);
-            tc_fence_after();
+            // one thread waits for the accumulator; the named barrier releases the others
+            const bool ok_wait = epi_tid != 0 || mbar_wait(&tfull[acc], (j >> 1) & 1, wlim);
             if (named_any(1, kEpiThreads, !ok_wait || *reinterpret_cast<volatile int*>(&flag[0]) != 0)) {
                 if (epi_tid == 0) report_status(ep.status, LLAMA_ERR_DEVICE_TIMEOUT);
                 break;
             }
+            tc_fence_after();
             ++j;
             // a split tile: publish this CTA's partial (feature-major, coalesced
             // over rows); only the last contributor to arrive goes on
@@ -609,12 +610,13 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
             const int nbase = tn * kPairTile;
             float rs = 1.f, sq = 0.f;
             epi_tile_inputs(ep, nio, m, row_ok, nbase + c_lo * 32, rowsB, KT * 64, rs);
-            const bool ok_wait = mbar_wait(&tfull[acc], (j >> 1) & 1, wlim);
-            tc_fence_after();
+            // one thread waits for the accumulator; the named barrier releases the others
+            const bool ok_wait = epi_tid != 0 || mbar_wait(&tfull[acc], (j >> 1) & 1, wlim);
             if (named_any(1, kEpiThreads, !ok_wait || *reinterpret_cast<volatile int*>(&flag[0]) != 0)) {
                 if (epi_tid == 0) report_status(ep.status, LLAMA_ERR_DEVICE_TIMEOUT);
                 break;
             }
+            tc_fence_after();
             ++j;
             // a split tile: this CTA's half of it, reduced among the same halves
             // of the tile's other pairs (last arrival finishes, in pair order)
