@@ -184,6 +184,30 @@ def test_top_p_sampler_matches_oracle(llb, V, T, p, scale):
     assert ambiguous == 0
 
 
+@pytest.mark.parametrize("V", [1000, 32000])
+def test_top_p_sampler_with_tied_logits(llb, V):
+    """Logits on a 0.25 grid (thousands of exact ties, which the select
+    resolves on the id digits of its key, across the slices of the CTAs that
+    share a row), a row of equal logits and a row with -inf entries: indices
+    identical to the oracle's (ties: lowest id first)."""
+    B, draws = 6, 12
+    g = torch.Generator().manual_seed(77 + V)
+    base = torch.round(torch.randn(B, V, generator=g) * 4.0) / 4.0
+    base[1, :] = 0.0
+    base[2, ::3] = float("-inf")
+    lg = base.repeat_interleave(draws, 0).contiguous()
+    u = make_uniforms((B * draws,), 4100 + V)
+    T, p = 0.7, 0.9003
+    out = torch.empty(B * draws, dtype=torch.int32, device="cuda")
+    llb.sample(lg.cuda(), T, p, u.cuda(), out)
+    torch.cuda.synchronize()
+    got = out.cpu().tolist()
+    for i in range(B * draws):
+        row = lg[i].numpy()
+        assert O.sample_margins(row, T, p, float(u[i])) >= 1e-9, i
+        assert got[i] == O.sample_top_p(row, T, p, float(u[i])), i
+
+
 # ----------------------------------------------------------------------------- whole model
 
 def _tiny_run(llb, shape, weights, B, T, steps, lens=None):
