@@ -617,6 +617,33 @@ def run_op_linear(a):
                       "peak_source": peak_src}), flush=True)
 
 
+def run_op_sample(a):
+    """Times top-p sampling (llama_sample, temperature 0.6, top-p 0.9) of B
+    rows of V seeded N(0, 2.5) logits with seeded uniforms, back to back.
+    Prints a JSON line with the time per call and the logit bytes it reads."""
+    import decoder_only_transformer_llama_b200 as llb
+    B, V = (int(v) for v in a.op_sample.split(","))
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    g = torch.Generator(device=dev).manual_seed(B)
+    logits = torch.randn(B, V, generator=g, device=dev) * 2.5
+    uni = torch.rand(B, generator=g, device=dev)
+    out = torch.empty(B, dtype=torch.int32, device=dev)
+    for _ in range(3):
+        llb.sample(logits, 0.6, 0.9, uni, out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.iters):
+        llb.sample(logits, 0.6, 0.9, uni, out)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / a.iters
+    print(json.dumps({"op": "sample_top_p", "B": B, "V": V, "temperature": 0.6, "top_p": 0.9,
+                      "us": round(ms * 1e3, 2), "logit_bytes": 4 * B * V,
+                      "picks": out[:8].tolist()}), flush=True)
+
+
 # ----------------------------------------------------------------------------- other workloads
 
 def _timed(fn, iters, stream, clocks=False):
@@ -862,6 +889,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op-linear", default=None, metavar="M,N,K",
                     help="time one bf16 projection instead of the model (kernel microbenchmark)")
+    ap.add_argument("--op-sample", default=None, metavar="B,V",
+                    help="time top-p sampling of B rows of V logits (llama_sample) and exit")
     ap.add_argument("--iters", type=int, default=50)
     ap.add_argument("--no-graph", action="store_true", help="launch decode steps directly instead of a CUDA graph")
     ap.add_argument("--workload", default="7b", choices=list(WORKLOADS),
@@ -876,6 +905,9 @@ def main():
     a = ap.parse_args()
     if a.op_linear:
         run_op_linear(a)
+        return
+    if a.op_sample:
+        run_op_sample(a)
         return
     if a.profile_steps or a.profile_prefill_kernels:
         a.profile_steps = max(a.profile_steps, 1)
