@@ -31,8 +31,10 @@
 //                  one item run while the epilogue drains the previous one
 //   warps 2-9      epilogue: warp w reads TMEM lanes 32*(w%4)..+31 = token rows,
 //                  warps 2-5 the tile's first 128 columns, warps 6-9 the other
-//                  128 (twice the epilogue's loads and stores in flight)
-// Every wait is bounded; no TMA multicast.
+//                  128 (twice the epilogue's loads and stores in flight); each
+//                  warp owns 4 KB of shared memory for staging fp32 outputs
+// Shared memory: the operand ring, then the epilogue staging (8 x 4 KB),
+// then the barriers.  Every wait is bounded; no TMA multicast.
 #include "common.cuh"
 #include "epilogue.cuh"
 #include "model.h"
