@@ -395,40 +395,41 @@ linear_tcp_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constan
                 }
                 __threadfence();
             }
-            // TMEM (summed with the other contributors' partials in CTA order)
+            if (!whole) {
+                // the last contributor: its accumulator is in its published
+                // partial as well, so the MMAs get it back now
+                tc_fence_before();
+                mbar_arrive(&tempty[acc]);
+            }
+            // TMEM, or the contributors' partials summed in CTA order
             // -> epilogue, 32 features at a time
 #pragma unroll 1
             for (int cc = c_lo; cc < c_lo + 4; ++cc) {
                 float v[32];
-                tmem_ld_32x32b_x32(tb + cc * 32, v);
-                tc_wait_ld();
-                if (!whole) {
-                    float own[32];
+                if (whole) {
+                    tmem_ld_32x32b_x32(tb + cc * 32, v);
+                    tc_wait_ld();
+                } else {
 #pragma unroll
-                    for (int t = 0; t < 32; ++t) {
-                        own[t] = v[t];
-                        v[t] = 0.f;
-                    }
+                    for (int t = 0; t < 32; ++t) v[t] = 0.f;
                     for (int cb = cf; cb <= cl; ++cb) {
-                        if (cb == c) {
+                        const int sl = run_begin(cb, Wsk, Psk) >= ub ? 0 : 1;
+                        const float* pp = part + (static_cast<long long>(cb) * 2 + sl) * kPartFloats + r;
+                        float f[32];
 #pragma unroll
-                            for (int t = 0; t < 32; ++t) v[t] += own[t];
-                        } else {
-                            const int sl = run_begin(cb, Wsk, Psk) >= ub ? 0 : 1;
-                            const float* pp = part + (static_cast<long long>(cb) * 2 + sl) * kPartFloats + r;
-                            float f[32];
+                        for (int t = 0; t < 32; ++t) f[t] = pp[(cc * 32 + t) * 128];
 #pragma unroll
-                            for (int t = 0; t < 32; ++t) f[t] = pp[(cc * 32 + t) * 128];
-#pragma unroll
-                            for (int t = 0; t < 32; ++t) v[t] += f[t];
-                        }
+                        for (int t = 0; t < 32; ++t) v[t] += f[t];
                     }
                 }
                 epi_block<E>(ep, nio, m - lane, nbase + cc * 32, rowsA, rowsB, rs, v, stg, lane, sq);
             }
-            tc_fence_before();
-            mbar_arrive(&tempty[acc]);
-            if (!whole && epi_tid == 0) counters[tl] = 0;
+            if (whole) {
+                tc_fence_before();
+                mbar_arrive(&tempty[acc]);
+            } else if (epi_tid == 0) {
+                counters[tl] = 0;
+            }
         }
     }
 
@@ -649,38 +650,31 @@ linear_tcp_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_co
                 }
                 __threadfence();
             }
+            if (!whole) release(acc);   // the last contributor's accumulator is in its partial too
 #pragma unroll 1
             for (int cc = c_lo; cc < c_lo + 4; ++cc) {
                 float v[32];
-                tmem_ld_32x32b_x32(tb + cc * 32, v);
-                tc_wait_ld();
-                if (!whole) {
-                    float own[32];
+                if (whole) {
+                    tmem_ld_32x32b_x32(tb + cc * 32, v);
+                    tc_wait_ld();
+                } else {
 #pragma unroll
-                    for (int t = 0; t < 32; ++t) {
-                        own[t] = v[t];
-                        v[t] = 0.f;
-                    }
+                    for (int t = 0; t < 32; ++t) v[t] = 0.f;
                     for (int cb = cf; cb <= cl; ++cb) {
-                        if (cb == c) {
+                        const int sl = run_begin(cb, Wsk, Psk) >= ub ? 0 : 1;
+                        const float* pp = part +
+                            (static_cast<long long>(2 * cb + static_cast<int>(rank)) * 2 + sl) * kPartFloats + r;
+                        float f[32];
 #pragma unroll
-                            for (int t = 0; t < 32; ++t) v[t] += own[t];
-                        } else {
-                            const int sl = run_begin(cb, Wsk, Psk) >= ub ? 0 : 1;
-                            const float* pp = part +
-                                (static_cast<long long>(2 * cb + static_cast<int>(rank)) * 2 + sl) * kPartFloats + r;
-                            float f[32];
+                        for (int t = 0; t < 32; ++t) f[t] = pp[(cc * 32 + t) * 128];
 #pragma unroll
-                            for (int t = 0; t < 32; ++t) f[t] = pp[(cc * 32 + t) * 128];
-#pragma unroll
-                            for (int t = 0; t < 32; ++t) v[t] += f[t];
-                        }
+                        for (int t = 0; t < 32; ++t) v[t] += f[t];
                     }
                 }
                 epi_block<E>(ep, nio, m - lane, nbase + cc * 32, rowsA, rowsB, rs, v, stg, lane, sq);
             }
-            release(acc);
-            if (!whole && epi_tid == 0) counters[cnt_idx] = 0;
+            if (whole) release(acc);
+            else if (epi_tid == 0) counters[cnt_idx] = 0;
         }
     }
 
