@@ -422,6 +422,17 @@ def run_ours(a, rank, world, local_rank):
     pre_flops = sum(r[2] for r in pre)
     pre_ms_k = sum(r[0] for r in pre)
     pre_tfs = pre_flops / (pre_ms_k / 1e3) / 1e12 if pre_ms_k else 0.0
+    # per projection kind (the layer's launch order: wq/wk/wv, wo, w1/w3, w2): mean
+    # microseconds per launch and TFLOP/s
+    pre_kinds = {}
+    for i, r in enumerate(pre[:4 * s.n_layers]):
+        k = ("wq/wk/wv", "wo", "w1/w3", "w2")[i % 4]
+        acc = pre_kinds.setdefault(k, [0.0, 0, 0])
+        acc[0] += r[0]
+        acc[1] += r[2]
+        acc[2] += 1
+    pre_kind_line = {k: {"us_per_launch": round(v[0] * 1e3 / v[2], 1),
+                         "TFLOP_s": round(v[1] / (v[0] / 1e3) / 1e12, 1)} for k, v in pre_kinds.items() if v[0] > 0}
 
     # in-graph: the projections' algorithmic bytes over their exclusive time in the replayed step
     proj_ns = tl_kind_ns.get("projection", 0)
@@ -477,6 +488,7 @@ def run_ours(a, rank, world, local_rank):
                              "clocks_what": "SM clocks sampled while prefills run back to back: the power cap holds "
                                             "them below the maximum, which is what the sustained peak describes",
                              "traffic": _traffic("prefill_projections"), "launches": len(pre),
+                             "per_kind": pre_kind_line,
                              "what": "2*M*N*K of one prefill's projection launches / their event-timed durations "
                                      "(prefill launches run one after another in the product path too)",
                              "traffic_what": "DRAM bytes per launch, mean over the 128 projection launches of one "
