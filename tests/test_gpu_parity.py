@@ -63,14 +63,14 @@ def test_linear_f32_kernel(llb, M, N, K):
     (1, 256, 256), (7, 1000, 4096), (16, 4096, 256), (17, 384, 4160), (33, 512, 200), (64, 12288, 4096),
     (48, 640, 512),
     (65, 256, 256), (128, 1000, 4096), (300, 768, 1024), (2048, 512, 64),
-    (300, 4224, 4096), (7, 1003, 512), (130, 1003, 512)])
+    (300, 4224, 4096), (7, 1003, 512), (130, 1003, 512), (300, 5003, 4096)])
 @pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
 def test_linear_16bit_tcgen05_kernel(llb, M, N, K, dt):
     """tcgen05 GEMM in both orientations (M <= 64: weights as the 128-row
     operand; else activations, on one SM per tile or, for at least 256 rows
     and more than 4096 x 4096 weights, on CTA pairs), with ragged M, N and K
-    tails (N = 1003: fp32 rows that are not 16-byte aligned, stored element
-    by element), for both 16-bit operand types."""
+    tails (N = 1003 and 5003: fp32 rows that are not 16-byte aligned, stored
+    element by element), for both 16-bit operand types."""
     g = torch.Generator().manual_seed(7 * M + N + K)
     A = torch.randn(M, K, generator=g).to(dt)
     W = (torch.randn(N, K, generator=g) * 0.05).to(dt)
